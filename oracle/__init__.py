@@ -1,0 +1,18 @@
+"""fp64 CPU oracle for exact attention (forward and backward).
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, ``__graft_entry__.smoke()``
+and the CPU-baseline leg of ``bench.py``; never by the product package.
+
+Parity status of each function (what pins it; see ``tests/test_oracle.py``):
+* attention_forward       pinned: the pages' worked examples, closed forms,
+                          brute-force blockwise recurrence, invariances.
+* attention_backward      pinned: central finite differences, sum invariants,
+                          closed form for uniform keys.
+* attention_forward_rows  pinned: equals attention_forward on every row.
+* attention_fwd_bwd_rows  pinned: equals the full forward/backward restricted
+                          to the rows.
+* online_blockwise_forward, online_softmax_stats, merge_softmax_stats
+                          pinned: the pages' printed numbers.
+"""
+from .attention import *  # noqa: F401,F403
+from .attention import __all__  # noqa: F401

@@ -1,0 +1,352 @@
+"""Plain fp64 CPU attention: the oracle that the CUDA path is checked against.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path may import this module:
+only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` use it.  It shares no code with the CUDA library and imports
+nothing from the ``exact_io_aware_90_b200`` package.
+
+Everything here is deliberately slow and literal.  The method it checks
+reaches the exact attention result, only reordered (FlashAttention 详解（零基础入门）,
+§5.2 WARNING box: the rescaling is exact; FlashAttention 与算子融合, "online
+softmax" paragraph: mathematically equivalent to the one-shot softmax;
+FlashAttention 短片讲解稿, segment "适用范围与关键结论": same definition, not
+bit-identical).  So the oracle is that definition written out in float64,
+materialising the score matrix S and the probability matrix P for every
+(sequence, head):
+
+* scores   S = Q Kᵀ · scale                  (详解 §2.3, S = QKᵀ/√d)
+* mask     S_ij = −∞ for key j > query i      (Flash Attention 优化, nanoGPT
+                                               manual fallback: lower-triangular
+                                               mask filled with −inf)
+* softmax  P_ij = exp(S_ij − m_i) / Σ_k exp(S_ik − m_i), m_i = max_k S_ik
+                                               (详解 §2.4, the safe form)
+* output   O = P V                            (详解 §2.5)
+* row log-sum-exp LSE_i = m_i + ln Σ_k exp(S_ik − m_i): the "few row
+  statistics" the forward keeps for the backward (短片讲解稿, segment
+  "第三招 · 反向重计算").
+
+The backward is not printed on the pages; they only say that it recomputes P
+from the inputs, the output and the row statistics (短片讲解稿 "第三招";
+the foundit article: "反向传播也会重新计算部分中间值").  The oracle takes the
+plainest reading, the chain rule applied to the four steps above:
+dV = Pᵀ dO, dP = dO Vᵀ, D_i = Σ_j P_ij dP_ij, dS = P ∘ (dP − D), dQ = scale·dS K,
+dK = scale·dSᵀ Q.
+
+``online_blockwise_forward`` follows the tiled algorithm of 详解 §6.2 in the
+pages' own order and notation (Q blocks outside, K/V blocks inside, running
+m and ℓ, the normalised O update of §5.4).  It exists to pin the one-shot
+definition against the pages' worked examples; the GPU is never compared
+with it.
+
+Tensor layout everywhere: [T, H, d] row-major (token, head, feature), T the
+total token count; ``cu_seqlens`` (int, length B+1, starting at 0,
+non-decreasing) packs B sequences of different lengths one after another
+(FlashAttention 与算子融合, 工程实践 "变长序列 … varlen 接口（packing）").
+Without ``cu_seqlens`` the T = B·N tokens form B sequences of N tokens.
+"""
+
+from __future__ import annotations
+
+import math
+from typing import Iterable, List, Optional, Sequence, Tuple
+
+import numpy as np
+
+__all__ = [
+    "sequence_segments",
+    "attention_forward",
+    "attention_backward",
+    "attention_forward_rows",
+    "attention_fwd_bwd_rows",
+    "online_blockwise_forward",
+    "online_softmax_stats",
+    "merge_softmax_stats",
+    "attention_flops",
+]
+
+
+def _f64(x) -> np.ndarray:
+    """Widen any array-like (numpy, or a CPU torch tensor) to float64 numpy."""
+    if hasattr(x, "detach"):  # a torch tensor: widen through float32 (exact for 16-bit inputs)
+        x = x.detach().cpu().float().numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def sequence_segments(T: int, B: int, N: int, cu_seqlens=None) -> List[Tuple[int, int]]:
+    """(start token, length) of every sequence in the packed [T, H, d] layout."""
+    if cu_seqlens is None:
+        if T != B * N:
+            raise ValueError(f"dense layout needs T == B*N, got T={T}, B={B}, N={N}")
+        return [(b * N, N) for b in range(B)]
+    cu = [int(c) for c in np.asarray(cu_seqlens).reshape(-1)]
+    if len(cu) != B + 1 or cu[0] != 0:
+        raise ValueError("cu_seqlens must have B+1 entries starting at 0")
+    segs = []
+    for b in range(B):
+        if cu[b + 1] < cu[b]:
+            raise ValueError("cu_seqlens must be non-decreasing")
+        segs.append((cu[b], cu[b + 1] - cu[b]))
+    if cu[B] > T:
+        raise ValueError("cu_seqlens[B] exceeds the token count")
+    return segs
+
+
+def _scores(Q: np.ndarray, K: np.ndarray, scale: float, causal: bool) -> np.ndarray:
+    """S = Q Kᵀ · scale with the causal mask applied (key j visible iff j <= i)."""
+    S = (Q @ K.T) * scale
+    if causal:
+        L = S.shape[0]
+        S[np.triu_indices(L, k=1)] = -np.inf
+    return S
+
+
+def _softmax_rows(S: np.ndarray):
+    """Safe softmax along rows: returns P, the row max m and the row sum ℓ of exp(S - m)."""
+    m = S.max(axis=1)
+    E = np.exp(S - m[:, None])
+    ell = E.sum(axis=1)
+    P = E / ell[:, None]
+    return P, m, ell
+
+
+def attention_forward(q, k, v, scale: float, causal: bool = False, cu_seqlens=None,
+                      B: Optional[int] = None, N: Optional[int] = None):
+    """Exact attention forward in fp64.
+
+    q, k, v: [T, H, d].  Returns (O [T, H, d] float64, LSE [T, H] float64).
+    LSE is the natural-log log-sum-exp of the scaled, masked scores of each row.
+    Tokens not covered by any sequence keep O = 0 and LSE = -inf.
+    """
+    Q, K, V = _f64(q), _f64(k), _f64(v)
+    T, H, d = Q.shape
+    if B is None:
+        B = 1 if cu_seqlens is None else len(np.asarray(cu_seqlens)) - 1
+    if N is None:
+        N = T // B if cu_seqlens is None else 0
+    O = np.zeros((T, H, d), dtype=np.float64)
+    LSE = np.full((T, H), -np.inf, dtype=np.float64)
+    for start, L in sequence_segments(T, B, N, cu_seqlens):
+        if L == 0:
+            continue
+        sl = slice(start, start + L)
+        for h in range(H):
+            S = _scores(Q[sl, h], K[sl, h], scale, causal)
+            P, m, ell = _softmax_rows(S)
+            O[sl, h] = P @ V[sl, h]
+            LSE[sl, h] = m + np.log(ell)
+    return O, LSE
+
+
+def attention_backward(q, k, v, do, scale: float, causal: bool = False, cu_seqlens=None,
+                       B: Optional[int] = None, N: Optional[int] = None):
+    """Gradients of L = <O, dO> with respect to q, k, v, in fp64.
+
+    P is recomputed from the inputs (the plain definition, no tiling).
+    Returns (dQ, dK, dV), each [T, H, d] float64.
+    """
+    Q, K, V, dO = _f64(q), _f64(k), _f64(v), _f64(do)
+    T, H, d = Q.shape
+    if B is None:
+        B = 1 if cu_seqlens is None else len(np.asarray(cu_seqlens)) - 1
+    if N is None:
+        N = T // B if cu_seqlens is None else 0
+    dQ = np.zeros_like(Q)
+    dK = np.zeros_like(K)
+    dV = np.zeros_like(V)
+    for start, L in sequence_segments(T, B, N, cu_seqlens):
+        if L == 0:
+            continue
+        sl = slice(start, start + L)
+        for h in range(H):
+            S = _scores(Q[sl, h], K[sl, h], scale, causal)
+            P, _, _ = _softmax_rows(S)
+            g = dO[sl, h]
+            dV[sl, h] = P.T @ g
+            dP = g @ V[sl, h].T
+            D = (P * dP).sum(axis=1)
+            dS = P * (dP - D[:, None])  # masked entries have P = 0, so dS = 0 there
+            dQ[sl, h] = scale * (dS @ K[sl, h])
+            dK[sl, h] = scale * (dS.T @ Q[sl, h])
+    return dQ, dK, dV
+
+
+def attention_forward_rows(q, k, v, rows: Sequence[int], scale: float, causal: bool = False,
+                           cu_seqlens=None, B: Optional[int] = None, N: Optional[int] = None):
+    """O and LSE for a chosen set of query tokens only (all heads), in fp64.
+
+    Each requested row is computed from its own sequence's keys, so the full
+    [L, L] score matrix is never formed: this is how long sequences are
+    checked on sampled rows.  Returns (O [len(rows), H, d], LSE [len(rows), H]).
+    """
+    T, H, d = q.shape
+    if B is None:
+        B = 1 if cu_seqlens is None else len(np.asarray(cu_seqlens)) - 1
+    if N is None:
+        N = T // B if cu_seqlens is None else 0
+    segs = sequence_segments(T, B, N, cu_seqlens)
+    starts = np.array([s for s, _ in segs])
+    rows = [int(r) for r in rows]
+    O = np.zeros((len(rows), H, d), dtype=np.float64)
+    LSE = np.full((len(rows), H), -np.inf, dtype=np.float64)
+    for n, t in enumerate(rows):
+        b = int(np.searchsorted(starts, t, side="right")) - 1
+        start, L = segs[b]
+        if not (start <= t < start + L):
+            continue
+        i = t - start
+        hi = start + (i + 1 if causal else L)
+        Qr = _f64(q[t])                 # [H, d]
+        Kr = _f64(k[start:hi])          # [j, H, d]
+        Vr = _f64(v[start:hi])
+        for h in range(H):
+            s = (Kr[:, h] @ Qr[h]) * scale
+            m = s.max()
+            e = np.exp(s - m)
+            ell = e.sum()
+            O[n, h] = (e / ell) @ Vr[:, h]
+            LSE[n, h] = m + math.log(ell)
+    return O, LSE
+
+
+def attention_fwd_bwd_rows(q, k, v, do, row_lo: int, row_hi: int, scale: float, causal: bool,
+                           head: int = 0):
+    """Forward and backward restricted to query rows [row_lo, row_hi) of one dense sequence.
+
+    q, k, v, do: [L, H, d] for one sequence.  Returns (O, LSE, dQ) for the
+    chosen rows and the partial (dK, dV) that those rows contribute to every
+    key, all float64.  Used as a bounded CPU workload sample; it is the same
+    arithmetic as ``attention_forward`` / ``attention_backward`` restricted to
+    a block of rows.
+    """
+    Q = _f64(q[row_lo:row_hi, head])
+    K = _f64(k[:, head])
+    V = _f64(v[:, head])
+    g = _f64(do[row_lo:row_hi, head])
+    S = (Q @ K.T) * scale
+    if causal:
+        i = np.arange(row_lo, row_hi)[:, None]
+        j = np.arange(K.shape[0])[None, :]
+        S[j > i] = -np.inf
+    P, m, ell = _softmax_rows(S)
+    O = P @ V
+    LSE = m + np.log(ell)
+    dV = P.T @ g
+    dP = g @ V.T
+    D = (P * dP).sum(axis=1)
+    dS = P * (dP - D[:, None])
+    dQ = scale * (dS @ K)
+    dK = scale * (dS.T @ Q)
+    return O, LSE, dQ, dK, dV
+
+
+def online_blockwise_forward(q, k, v, scale: float, causal: bool = False, bq: int = 64,
+                             bk: int = 64, trace: Optional[list] = None):
+    """The tiled forward of FlashAttention 详解 §6.2, taken step by step (one sequence).
+
+    q: [N, H, d] or [N, d] (one head); k, v: the same with their own row count
+    (equal to N when causal).  Block sizes need not divide the row counts;
+    the last block is shorter (the pages use N // B blocks and are silent on
+    remainders).  Q blocks are the outer loop, K/V blocks the inner loop; the
+    running max m, the running sum ℓ and the output block are updated with the
+    normalised rule of §5.4 / the §6.2 update line:
+        m_new = max(m, rowmax(S_ij));  P_ij = exp(S_ij − m_new)
+        ℓ_new = ℓ·exp(m − m_new) + rowsum(P_ij)
+        O = O·(ℓ/ℓ_new)·exp(m − m_new) + P_ij V_j / ℓ_new
+    A row that has seen only masked keys so far has m = −∞ and ℓ = 0; for it
+    the correction factor is taken as 0 and O stays 0 (the pages are silent on
+    this case; it needs a block whose keys are all hidden from the row).
+
+    If ``trace`` is a list, (i, j, m_new, ℓ_new, numerator = O·ℓ_new) is
+    appended after every inner step, so the pages' running numerator and
+    denominator can be checked.  Returns (O, LSE) with the input's head shape.
+    """
+    Q, K, V = _f64(q), _f64(k), _f64(v)
+    squeeze = Q.ndim == 2
+    if squeeze:
+        Q, K, V = Q[:, None, :], K[:, None, :], V[:, None, :]
+    N, H, d = Q.shape
+    Nk = K.shape[0]
+    if causal and Nk != N:
+        raise ValueError("the causal mask needs as many keys as queries")
+    O = np.zeros((N, H, d))
+    LSE = np.zeros((N, H))
+    for h in range(H):
+        for i0 in range(0, N, bq):
+            i1 = min(i0 + bq, N)
+            Qi = Q[i0:i1, h]
+            Oi = np.zeros((i1 - i0, d))
+            mi = np.full(i1 - i0, -np.inf)
+            li = np.zeros(i1 - i0)
+            for j0 in range(0, Nk, bk):
+                j1 = min(j0 + bk, Nk)
+                Kj, Vj = K[j0:j1, h], V[j0:j1, h]
+                Sij = (Qi @ Kj.T) * scale
+                if causal:
+                    qi = np.arange(i0, i1)[:, None]
+                    kj = np.arange(j0, j1)[None, :]
+                    Sij = np.where(kj > qi, -np.inf, Sij)
+                mij = Sij.max(axis=1)
+                m_new = np.maximum(mi, mij)
+                live = np.isfinite(m_new)
+                shift = np.where(live, m_new, 0.0)
+                Pij = np.where(live[:, None], np.exp(Sij - shift[:, None]), 0.0)
+                corr = np.where(np.isfinite(mi), np.exp(mi - shift), 0.0)
+                l_new = li * corr + Pij.sum(axis=1)
+                safe_l = np.where(l_new > 0, l_new, 1.0)
+                Oi = np.where(
+                    (l_new > 0)[:, None],
+                    Oi * (li / safe_l * corr)[:, None] + (Pij @ Vj) / safe_l[:, None],
+                    0.0,
+                )
+                mi, li = m_new, l_new
+                if trace is not None:
+                    trace.append((i0 // bq, j0 // bk, mi.copy(), li.copy(), Oi * li[:, None]))
+            O[i0:i1, h] = Oi
+            LSE[i0:i1, h] = mi + np.log(li)
+    if squeeze:
+        return O[:, 0, :], LSE[:, 0]
+    return O, LSE
+
+
+def online_softmax_stats(x: Iterable[float], blocks: Sequence[int]):
+    """Running (m, ℓ) of one row of scores fed in blocks of the given sizes.
+
+    This is the two-statistic recurrence of 详解 §5.2:
+        m⁽ᵗ⁾ = max(m⁽ᵗ⁻¹⁾, max_j x_j⁽ᵗ⁾)
+        ℓ⁽ᵗ⁾ = ℓ⁽ᵗ⁻¹⁾·exp(m⁽ᵗ⁻¹⁾ − m⁽ᵗ⁾) + Σ_j exp(x_j⁽ᵗ⁾ − m⁽ᵗ⁾)
+    Returns the list of (m, ℓ) after each block.
+    """
+    x = [float(t) for t in x]
+    if sum(blocks) != len(x):
+        raise ValueError("block sizes must add up to the row length")
+    m, ell, out, pos = -math.inf, 0.0, [], 0
+    for b in blocks:
+        blk = x[pos:pos + b]
+        pos += b
+        m_new = max([m] + blk)
+        ell = (ell * math.exp(m - m_new) if ell > 0 else 0.0) + sum(math.exp(t - m_new) for t in blk)
+        m = m_new
+        out.append((m, ell))
+    return out
+
+
+def merge_softmax_stats(m_a: float, l_a: float, m_b: float, l_b: float):
+    """Merge two partial (max, sum) pairs: the form given by FlashAttention 与算子融合
+    (online softmax paragraph): m = max(m_a, m_b), ℓ = ℓ_a·e^{m_a−m} + ℓ_b·e^{m_b−m}."""
+    m = max(m_a, m_b)
+    ell = 0.0
+    if l_a > 0:
+        ell += l_a * math.exp(m_a - m)
+    if l_b > 0:
+        ell += l_b * math.exp(m_b - m)
+    return m, ell
+
+
+def attention_flops(seqlens: Sequence[int], H: int, d: int, causal: bool, backward: bool = False) -> float:
+    """Attention FLOPs by the convention of FlashAttention 与算子融合 (4·B·h·s²·d for
+    the forward), summed over sequences, halved when causal; the backward counts
+    2.5× the forward."""
+    f = sum(4.0 * H * float(L) * float(L) * d for L in seqlens)
+    if causal:
+        f *= 0.5
+    return f * 2.5 if backward else f

@@ -1,0 +1,459 @@
+"""Pins for the fp64 oracle: what the pages and the mathematics fix, not the oracle itself.
+
+Each test checks the oracle against something other than its own formula:
+the worked examples printed on the pages (``tests/golden/``), closed forms,
+invariants that a wrong term, sign, index or operand order would break,
+brute force (the tiled recurrence of the pages on tiny inputs) and central
+finite differences for the backward.  ``test_pins_catch_planted_mistakes``
+plants plausible mistakes in a copy of the oracle and checks that the pins
+reject every one of them.
+"""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import attention as A
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _load(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _hand_qkv(d=4):
+    """The narration's example: scale·q·k_j = ln c_j, V_j = value_j (feature 0)."""
+    ex = _load("hand_example.json")
+    scale = 0.5
+    q = np.zeros((4, 1, d))
+    k = np.zeros((4, 1, d))
+    v = np.zeros((4, 1, d))
+    q[:, 0, 0] = 1.0 / scale
+    k[:, 0, 0] = np.log(ex["exp_scores"])
+    v[:, 0, 0] = ex["v"]
+    return ex, q, k, v, scale
+
+
+def _rand(rng, T, H, d):
+    return rng.standard_normal((T, H, d)), rng.standard_normal((T, H, d)), rng.standard_normal((T, H, d))
+
+
+# ----------------------------------------------------------------------------- worked examples
+
+
+def test_hand_example_one_shot():
+    ex, q, k, v, scale = _hand_qkv()
+    O, LSE = oracle.attention_forward(q, k, v, scale, causal=False)
+    assert np.all(np.abs(O[:, 0, 0] - ex["full"]["result"]) < 1e-12)
+    # LSE = ln(sum of exponentiated scores) = ln(weight total)
+    assert np.all(np.abs(np.exp(LSE[:, 0]) - ex["full"]["weight_total"]) < 1e-12)
+    # weighted sum = result x weight total
+    assert abs(O[0, 0, 0] * np.exp(LSE[0, 0]) - ex["full"]["weighted_sum"]) < 1e-10
+    assert np.all(O[:, 0, 1:] == 0.0)
+
+
+def test_hand_example_two_blocks_trace():
+    ex, q, k, v, scale = _hand_qkv()
+    trace = []
+    O, _ = oracle.online_blockwise_forward(q[:1, 0], k[:, 0], v[:, 0], scale, bq=1, bk=2, trace=trace)
+    assert len(trace) == 2
+    _, _, m1, l1, num1 = trace[0]
+    _, _, m2, l2, num2 = trace[1]
+    b1, b2 = ex["after_block_1"], ex["after_block_2"]
+    assert abs(math.exp(m1[0]) - b1["max_exp_score"]) < 1e-12
+    assert abs(l1[0] - b1["denominator"]) < 1e-12
+    assert abs(num1[0, 0] - b1["numerator"]) < 1e-12
+    assert abs(math.exp(m1[0] - m2[0]) - ex["rescale_factor_at_block_2"]) < 1e-12
+    assert abs(l2[0] - b2["denominator"]) < 1e-12
+    assert abs(num2[0, 0] - b2["numerator"]) < 1e-12
+    assert abs(O[0, 0] - b2["result"]) < 1e-12
+    # the block-2 weights: new denominator minus the rescaled old one, and each weight
+    new_part = l2[0] - b1["denominator"] * ex["rescale_factor_at_block_2"]
+    assert abs(new_part - sum(ex["block_2_weights"])) < 1e-12
+
+
+def test_hand_example_causal_prefixes():
+    """Causal version of the same row set: row i averages the first i+1 values."""
+    ex, q, k, v, scale = _hand_qkv()
+    O, LSE = oracle.attention_forward(q, k, v, scale, causal=True)
+    c = np.array(ex["exp_scores"], float)
+    vals = np.array(ex["v"], float)
+    for i in range(4):
+        want = (c[: i + 1] * vals[: i + 1]).sum() / c[: i + 1].sum()
+        assert abs(O[i, 0, 0] - want) < 1e-12
+        assert abs(LSE[i, 0] - math.log(c[: i + 1].sum())) < 1e-12
+    assert abs(O[1, 0, 0] - 50.0 / 3.0) < 1e-12 and abs(O[2, 0, 0] - 170.0 / 7.0) < 1e-12
+
+
+def test_online_softmax_numeric_example():
+    ex = _load("online_softmax_example.json")
+    stats = oracle.online_softmax_stats(ex["x"], ex["blocks"])
+    (m1, l1), (m2, l2) = stats
+    assert m1 == ex["block_1"]["m"] and m2 == ex["block_2"]["m"]
+    # printed to 4 decimals, with the page summing already-rounded parts
+    assert abs(l1 - ex["block_1"]["l"]) < 1e-4
+    assert abs(l2 - ex["block_2"]["l"]) < 2e-4
+    assert abs(l1 * math.exp(m1 - m2) - ex["block_2"]["rescaled_old_l"]) < 2e-4
+    # the merge form (two partial pairs) gives the same statistics
+    mm, lm = oracle.merge_softmax_stats(m1, l1, 4.0, ex["block_2"]["new_block_contribution"])
+    assert mm == 4.0 and abs(lm - ex["block_2"]["l"]) < 2e-4
+    # one-shot softmax through the attention oracle: q·k_j = x_j, V = identity rows
+    x = np.array(ex["x"], float)
+    q = np.zeros((1, 1, 4)); q[0, 0, 0] = 1.0
+    k = np.zeros((4, 1, 4)); k[:, 0, 0] = x
+    v = np.eye(4)[:, None, :]
+    # one query attending to four keys: put the query last in a causal-free 4-token call
+    Q = np.zeros((4, 1, 4)); Q[:] = q
+    O, LSE = oracle.attention_forward(Q, k, v, 1.0)
+    assert np.allclose(O[0, 0], ex["one_shot"]["softmax"], atol=5e-4)
+    assert abs(math.exp(LSE[0, 0] - ex["one_shot"]["max"]) - ex["one_shot"]["sum"]) < 5e-4
+    assert np.allclose(np.exp(x - x.max()), ex["one_shot"]["exp"], atol=5e-5)
+
+
+# ----------------------------------------------------------------------------- closed forms and invariants
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_rows_of_p_sum_to_one(causal):
+    rng = np.random.default_rng(1)
+    q, k, v = _rand(rng, 37, 3, 8)
+    v[:] = 1.0  # O = P·1 = row sums of P
+    O, _ = oracle.attention_forward(q, k, v, 0.7, causal=causal)
+    assert np.max(np.abs(O - 1.0)) < 1e-12
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_shift_invariance(causal):
+    """Adding u to every key adds scale·q_i·u to row i of S: P and O unchanged, LSE shifted."""
+    rng = np.random.default_rng(2)
+    q, k, v = _rand(rng, 29, 2, 16)
+    u = rng.standard_normal(16) * 3.0
+    scale = 0.25
+    O1, L1 = oracle.attention_forward(q, k, v, scale, causal=causal)
+    O2, L2 = oracle.attention_forward(q, k + u, v, scale, causal=causal)
+    assert np.max(np.abs(O1 - O2)) < 1e-11
+    assert np.max(np.abs((L2 - L1) - scale * np.einsum("thd,d->th", q, u))) < 1e-10
+
+
+def test_large_scores_do_not_overflow():
+    """The row max is subtracted before exponentiating (safe softmax)."""
+    rng = np.random.default_rng(3)
+    q, k, v = _rand(rng, 16, 1, 4)
+    O1, L1 = oracle.attention_forward(q, k, v, 1.0)
+    big = np.zeros(4); big[0] = 1.0
+    # add 1000 to every score of every row through a key shift along q's direction
+    q2 = np.concatenate([q, np.ones((16, 1, 1))], axis=2)
+    k2 = np.concatenate([k, np.full((16, 1, 1), 1000.0)], axis=2)
+    v2 = np.concatenate([v, np.zeros((16, 1, 1))], axis=2)
+    O2, L2 = oracle.attention_forward(q2, k2, v2, 1.0)
+    assert np.all(np.isfinite(O2)) and np.max(np.abs(O2[..., :4] - O1)) < 1e-10
+    assert np.max(np.abs(L2 - (L1 + 1000.0))) < 1e-9
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_uniform_keys_give_mean_of_values(causal):
+    rng = np.random.default_rng(4)
+    L, d = 11, 6
+    q = rng.standard_normal((L, 1, d))
+    k = np.tile(rng.standard_normal((1, 1, d)), (L, 1, 1))
+    v = rng.standard_normal((L, 1, d))
+    scale = 0.3
+    O, LSE = oracle.attention_forward(q, k, v, scale, causal=causal)
+    for i in range(L):
+        n = i + 1 if causal else L
+        assert np.max(np.abs(O[i, 0] - v[:n, 0].mean(axis=0))) < 1e-12
+        s = scale * float(q[i, 0] @ k[0, 0])
+        assert abs(LSE[i, 0] - (s + math.log(n))) < 1e-12
+
+
+def test_single_token_returns_its_value():
+    rng = np.random.default_rng(5)
+    q, k, v = _rand(rng, 1, 3, 5)
+    O, LSE = oracle.attention_forward(q, k, v, 0.4, causal=True)
+    assert np.max(np.abs(O - v)) < 1e-15
+    assert np.max(np.abs(LSE - 0.4 * np.einsum("thd,thd->th", q, k))) < 1e-14
+
+
+def test_causal_row_ignores_future_keys():
+    """Changing keys/values after position i leaves causal row i unchanged."""
+    rng = np.random.default_rng(6)
+    q, k, v = _rand(rng, 20, 2, 4)
+    O1, L1 = oracle.attention_forward(q, k, v, 0.5, causal=True)
+    k2, v2 = k.copy(), v.copy()
+    k2[12:] = rng.standard_normal(k2[12:].shape) * 10
+    v2[12:] = rng.standard_normal(v2[12:].shape) * 10
+    O2, L2 = oracle.attention_forward(q, k2, v2, 0.5, causal=True)
+    assert np.array_equal(O1[:12], O2[:12]) and np.array_equal(L1[:12], L2[:12])
+    assert np.max(np.abs(O1[12:] - O2[12:])) > 1e-3
+
+
+def test_key_permutation_invariance_non_causal():
+    rng = np.random.default_rng(7)
+    q, k, v = _rand(rng, 17, 2, 8)
+    perm = rng.permutation(17)
+    O1, L1 = oracle.attention_forward(q, k, v, 0.35)
+    O2, L2 = oracle.attention_forward(q, k[perm], v[perm], 0.35)
+    assert np.max(np.abs(O1 - O2)) < 1e-12 and np.max(np.abs(L1 - L2)) < 1e-12
+
+
+def test_brute_force_scalar_loop_tiny():
+    """Direct scalar loops (no matrix products) on a 3-token, 2-feature case."""
+    rng = np.random.default_rng(8)
+    q, k, v = _rand(rng, 3, 1, 2)
+    scale = 0.9
+    for causal in (False, True):
+        O, LSE = oracle.attention_forward(q, k, v, scale, causal=causal)
+        for i in range(3):
+            js = range(i + 1) if causal else range(3)
+            s = {j: scale * (q[i, 0, 0] * k[j, 0, 0] + q[i, 0, 1] * k[j, 0, 1]) for j in js}
+            z = sum(math.exp(x) for x in s.values())
+            for c in range(2):
+                want = sum(math.exp(s[j]) * v[j, 0, c] for j in js) / z
+                assert abs(O[i, 0, c] - want) < 1e-12
+            assert abs(LSE[i, 0] - math.log(z)) < 1e-12
+
+
+# ----------------------------------------------------------------------------- tiled recurrence
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("bq,bk", [(1, 1), (64, 64), (3, 5), (7, 2), (16, 13), (50, 50)])
+def test_blockwise_recurrence_equals_one_shot(causal, bq, bk):
+    rng = np.random.default_rng(100 + bq * 7 + bk)
+    q, k, v = _rand(rng, 50, 2, 8)
+    scale = 1.0 / math.sqrt(8)
+    O1, L1 = oracle.attention_forward(q, k, v, scale, causal=causal)
+    O2, L2 = oracle.online_blockwise_forward(q, k, v, scale, causal=causal, bq=bq, bk=bk)
+    assert np.max(np.abs(O1 - O2)) < 1e-12
+    assert np.max(np.abs(L1 - L2)) < 1e-12
+
+
+def test_online_stats_random_splits_match_one_shot():
+    rng = np.random.default_rng(9)
+    for _ in range(50):
+        n = int(rng.integers(1, 40))
+        x = rng.standard_normal(n) * 5
+        cuts = sorted(set(int(c) for c in rng.integers(1, n + 1, size=int(rng.integers(0, 5)))) | {n})
+        blocks = [b - a for a, b in zip([0] + cuts[:-1], cuts)]
+        m, l = oracle.online_softmax_stats(x, blocks)[-1]
+        assert m == x.max()
+        assert abs(l - np.exp(x - x.max()).sum()) < 1e-12
+
+
+# ----------------------------------------------------------------------------- varlen and row sampling
+
+
+def test_varlen_equals_separate_sequences():
+    rng = np.random.default_rng(10)
+    lens = [5, 1, 9, 0, 4]
+    cu = np.cumsum([0] + lens)
+    T = int(cu[-1])
+    q, k, v = _rand(rng, T, 2, 4)
+    do = rng.standard_normal((T, 2, 4))
+    for causal in (False, True):
+        O, L = oracle.attention_forward(q, k, v, 0.6, causal, cu_seqlens=cu)
+        dq, dk, dv = oracle.attention_backward(q, k, v, do, 0.6, causal, cu_seqlens=cu)
+        for b, n in enumerate(lens):
+            if n == 0:
+                continue
+            sl = slice(cu[b], cu[b + 1])
+            Ob, Lb = oracle.attention_forward(q[sl], k[sl], v[sl], 0.6, causal)
+            g = oracle.attention_backward(q[sl], k[sl], v[sl], do[sl], 0.6, causal)
+            assert np.array_equal(O[sl], Ob) and np.array_equal(L[sl], Lb)
+            for a, bb in zip((dq, dk, dv), g):
+                assert np.array_equal(a[sl], bb)
+
+
+def test_rows_sampler_matches_full():
+    rng = np.random.default_rng(11)
+    lens = [7, 12, 3]
+    cu = np.cumsum([0] + lens)
+    q, k, v = _rand(rng, int(cu[-1]), 3, 4)
+    rows = list(range(int(cu[-1])))
+    for causal in (False, True):
+        O, L = oracle.attention_forward(q, k, v, 0.5, causal, cu_seqlens=cu)
+        Or, Lr = oracle.attention_forward_rows(q, k, v, rows, 0.5, causal, cu_seqlens=cu)
+        assert np.max(np.abs(O - Or)) < 1e-12 and np.max(np.abs(L - Lr)) < 1e-12
+
+
+def test_row_block_fwd_bwd_sums_to_full():
+    rng = np.random.default_rng(12)
+    L, H, d = 24, 2, 4
+    q, k, v = _rand(rng, L, H, d)
+    do = rng.standard_normal((L, H, d))
+    for causal in (False, True):
+        O, LSE = oracle.attention_forward(q, k, v, 0.5, causal)
+        dq, dk, dv = oracle.attention_backward(q, k, v, do, 0.5, causal)
+        for h in range(H):
+            dk_sum = np.zeros((L, d)); dv_sum = np.zeros((L, d))
+            for lo in range(0, L, 10):
+                hi = min(lo + 10, L)
+                o, lse, dqr, dkr, dvr = oracle.attention_fwd_bwd_rows(q, k, v, do, lo, hi, 0.5, causal, head=h)
+                assert np.max(np.abs(o - O[lo:hi, h])) < 1e-12
+                assert np.max(np.abs(lse - LSE[lo:hi, h])) < 1e-12
+                assert np.max(np.abs(dqr - dq[lo:hi, h])) < 1e-12
+                dk_sum += dkr; dv_sum += dvr
+            assert np.max(np.abs(dk_sum - dk[:, h])) < 1e-12
+            assert np.max(np.abs(dv_sum - dv[:, h])) < 1e-12
+
+
+# ----------------------------------------------------------------------------- backward
+
+
+def _fd_check(q, k, v, do, scale, causal, cu=None, h=1e-6):
+    dq, dk, dv = oracle.attention_backward(q, k, v, do, scale, causal, cu_seqlens=cu)
+
+    def f(qq, kk, vv):
+        O, _ = oracle.attention_forward(qq, kk, vv, scale, causal, cu_seqlens=cu)
+        return float((O * do).sum())
+
+    worst = 0.0
+    for which, grad in ((0, dq), (1, dk), (2, dv)):
+        it = np.nditer(grad, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            args_p = [q.copy(), k.copy(), v.copy()]
+            args_m = [q.copy(), k.copy(), v.copy()]
+            args_p[which][idx] += h
+            args_m[which][idx] -= h
+            fd = (f(*args_p) - f(*args_m)) / (2 * h)
+            worst = max(worst, abs(fd - grad[idx]) / max(1.0, abs(grad[idx])))
+    return worst
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_finite_differences(causal):
+    rng = np.random.default_rng(13)
+    q, k, v = _rand(rng, 6, 2, 3)
+    do = rng.standard_normal((6, 2, 3))
+    assert _fd_check(q, k, v, do, 0.8, causal) < 1e-6
+
+
+def test_backward_finite_differences_varlen():
+    rng = np.random.default_rng(14)
+    cu = np.array([0, 3, 4, 8])
+    q, k, v = _rand(rng, 8, 1, 2)
+    do = rng.standard_normal((8, 1, 2))
+    assert _fd_check(q, k, v, do, 1.1, True, cu=cu) < 1e-6
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_sum_invariants(causal):
+    """Σ_j dK_j = 0 (softmax is shift invariant in the keys) and Σ_j dV_j = Σ_i dO_i."""
+    rng = np.random.default_rng(15)
+    q, k, v = _rand(rng, 33, 3, 8)
+    do = rng.standard_normal((33, 3, 8))
+    dq, dk, dv = oracle.attention_backward(q, k, v, do, 0.4, causal)
+    assert np.max(np.abs(dk.sum(axis=0))) < 1e-10
+    assert np.max(np.abs(dv.sum(axis=0) - do.sum(axis=0))) < 1e-10
+
+
+def test_backward_uniform_keys_closed_form():
+    """With all keys equal P is uniform and dV_j = (1/L)·Σ_i dO_i (non-causal)."""
+    rng = np.random.default_rng(16)
+    L, d = 9, 4
+    q = rng.standard_normal((L, 1, d))
+    k = np.tile(rng.standard_normal((1, 1, d)), (L, 1, 1))
+    v = rng.standard_normal((L, 1, d))
+    do = rng.standard_normal((L, 1, d))
+    dq, dk, dv = oracle.attention_backward(q, k, v, do, 0.5, False)
+    for j in range(L):
+        assert np.max(np.abs(dv[j, 0] - do[:, 0].mean(axis=0))) < 1e-12
+    # dQ_i = scale · Σ_j P_ij (dP_ij − D_i) k_j = scale · k · Σ_j P_ij (dP_ij − D_i) = 0
+    assert np.max(np.abs(dq)) < 1e-12
+
+
+def test_flop_convention():
+    # 4·B·h·s²·d for B=4, h=16, s=8192, d=128, halved when causal
+    assert oracle.attention_flops([8192] * 4, 16, 128, causal=False) == 4 * 4 * 16 * 8192 ** 2 * 128
+    assert oracle.attention_flops([8192] * 4, 16, 128, causal=True) == 2 * 4 * 16 * 8192 ** 2 * 128
+    assert oracle.attention_flops([10], 1, 2, causal=False, backward=True) == 2.5 * 4 * 100 * 2
+
+
+# ----------------------------------------------------------------------------- planted mistakes
+
+
+def _pins_pass():
+    """A compact battery of the pins above; returns False as soon as one fails."""
+    checks = [
+        test_hand_example_one_shot, test_hand_example_causal_prefixes,
+        lambda: test_rows_of_p_sum_to_one(True), lambda: test_shift_invariance(True),
+        test_large_scores_do_not_overflow, lambda: test_uniform_keys_give_mean_of_values(True),
+        test_brute_force_scalar_loop_tiny, test_causal_row_ignores_future_keys,
+        lambda: test_backward_finite_differences(True), lambda: test_backward_sum_invariants(True),
+        test_backward_uniform_keys_closed_form,
+    ]
+    for c in checks:
+        try:
+            with np.errstate(all="ignore"):
+                c()
+        except (AssertionError, FloatingPointError, ValueError, IndexError):
+            return False
+    return True
+
+
+def test_pins_catch_planted_mistakes(monkeypatch):
+    assert _pins_pass()
+    orig_scores, orig_softmax = A._scores, A._softmax_rows
+
+    def no_scale(Q, K, scale, causal):
+        return orig_scores(Q, K, 1.0, causal)
+
+    def transposed(Q, K, scale, causal):
+        S = (K @ Q.T) * scale if Q.shape[0] == K.shape[0] else (Q @ K.T) * scale
+        if causal:
+            S[np.triu_indices(S.shape[0], k=1)] = -np.inf
+        return S
+
+    def upper_mask(Q, K, scale, causal):
+        S = (Q @ K.T) * scale
+        if causal:
+            S[np.tril_indices(S.shape[0], k=-1)] = -np.inf
+        return S
+
+    def mask_off_by_one(Q, K, scale, causal):
+        S = (Q @ K.T) * scale
+        if causal:
+            S[np.triu_indices(S.shape[0], k=2)] = -np.inf
+        return S
+
+    def no_max_shift(S):
+        E = np.exp(S)
+        ell = E.sum(axis=1)
+        return E / ell[:, None], np.zeros(S.shape[0]), ell
+
+    def wrong_sign(S):
+        m = S.max(axis=1)
+        E = np.exp(m[:, None] - S)
+        ell = E.sum(axis=1)
+        return E / ell[:, None], m, ell
+
+    def dropped_norm(S):
+        m = S.max(axis=1)
+        E = np.exp(S - m[:, None])
+        return E, m, E.sum(axis=1)
+
+    for name, patch in [("_scores", no_scale), ("_scores", transposed), ("_scores", upper_mask),
+                        ("_scores", mask_off_by_one), ("_softmax_rows", no_max_shift),
+                        ("_softmax_rows", wrong_sign), ("_softmax_rows", dropped_norm)]:
+        with monkeypatch.context() as mp:
+            mp.setattr(A, name, patch)
+            assert not _pins_pass(), f"planted mistake {patch.__name__} was not caught"
+
+    # a mistake in the backward only: D computed without P, dK missing its scale
+    orig_bwd = A.attention_backward
+
+    def bwd_no_dk_scale(q, k, v, do, scale, causal=False, cu_seqlens=None, B=None, N=None):
+        dq, dk, dv = orig_bwd(q, k, v, do, scale, causal, cu_seqlens, B, N)
+        return dq, dk / scale, dv
+
+    with monkeypatch.context() as mp:
+        mp.setattr(A, "attention_backward", bwd_no_dk_scale)
+        mp.setattr(oracle, "attention_backward", bwd_no_dk_scale)
+        assert not _pins_pass()

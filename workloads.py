@@ -1,0 +1,146 @@
+"""Seeded synthetic inputs for the attention workloads.
+
+Shared by the tests, ``bench.py`` and ``__graft_entry__``.  This module holds
+none of the attention arithmetic: it only draws i.i.d. N(0, 1) numbers from a
+seeded CPU generator, rounds them to the storage dtype, draws sequence lengths
+and builds the ``cu_seqlens`` prefix array.  Both the CUDA path and the fp64
+oracle consume exactly the tensors made here (the oracle widens the rounded
+values to float64).
+
+Layout: q, k, v, dO are [T, H, d] row-major; ``cu_seqlens`` is int32 [B+1]
+or None (then T = B·N).  The workloads are the five measured shapes:
+
+==================  =========================================================
+name                shape
+==================  =========================================================
+tiny_d64            B=1, H=1, N=256, d=64, bf16, non-causal, forward only
+mha_n4k_d64         B=8, H=16, N=4096, d=64, fp16, non-causal, fwd+bwd
+causal_n8k_d128     B=4, H=16, N=8192, d=128, bf16, causal, fwd+bwd
+varlen_causal_d128  32 sequences, lengths uniform in [128, 4096], H=32,
+                    d=128, bf16, causal, fwd+bwd
+long_n128k_d128     B=1, H=8, N=131072, d=128, bf16, causal, forward only
+==================  =========================================================
+"""
+
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+from typing import List, Optional
+
+import numpy as np
+import torch
+
+WORKLOADS = {
+    "tiny_d64": dict(B=1, H=1, N=256, d=64, dtype="bf16", causal=False, backward=False, seed=1001),
+    "mha_n4k_d64": dict(B=8, H=16, N=4096, d=64, dtype="fp16", causal=False, backward=True, seed=1002),
+    "causal_n8k_d128": dict(B=4, H=16, N=8192, d=128, dtype="bf16", causal=True, backward=True, seed=1003),
+    "varlen_causal_d128": dict(nseq=32, lmin=128, lmax=4096, H=32, d=128, dtype="bf16", causal=True,
+                               backward=True, seed=1004),
+    "long_n128k_d128": dict(B=1, H=8, N=131072, d=128, dtype="bf16", causal=True, backward=False, seed=1005),
+}
+
+TORCH_DTYPES = {"bf16": torch.bfloat16, "fp16": torch.float16}
+
+
+@dataclass
+class AttnInputs:
+    q: torch.Tensor
+    k: torch.Tensor
+    v: torch.Tensor
+    do: Optional[torch.Tensor]
+    cu_seqlens: Optional[torch.Tensor]  # int32 [B+1] or None
+    seqlens: List[int]
+    B: int
+    H: int
+    N: int            # maximum sequence length
+    d: int
+    scale: float
+    causal: bool
+    dtype: str
+    name: str = ""
+    extra: dict = field(default_factory=dict)
+
+    @property
+    def T(self) -> int:
+        return int(self.q.shape[0])
+
+    def to(self, device) -> "AttnInputs":
+        mv = lambda t: None if t is None else t.to(device)
+        return AttnInputs(mv(self.q), mv(self.k), mv(self.v), mv(self.do), mv(self.cu_seqlens),
+                          list(self.seqlens), self.B, self.H, self.N, self.d, self.scale, self.causal,
+                          self.dtype, self.name, dict(self.extra))
+
+
+def _randn(g: torch.Generator, shape, dtype: str) -> torch.Tensor:
+    return torch.randn(*shape, generator=g, dtype=torch.float32).to(TORCH_DTYPES[dtype])
+
+
+def varlen_lengths(nseq: int, lmin: int, lmax: int, seed: int) -> List[int]:
+    """Sequence lengths drawn uniformly from the integers [lmin, lmax]."""
+    rng = np.random.default_rng(seed)
+    return [int(x) for x in rng.integers(lmin, lmax + 1, size=nseq)]
+
+
+def cu_from_lengths(lengths: List[int]) -> torch.Tensor:
+    cu = [0]
+    for L in lengths:
+        cu.append(cu[-1] + int(L))
+    return torch.tensor(cu, dtype=torch.int32)
+
+
+def random_inputs(H: int, d: int, dtype: str, seed: int, *, B: int = 1, N: int = 0,
+                  seqlens: Optional[List[int]] = None, causal: bool = False,
+                  backward: bool = True, scale: Optional[float] = None, name: str = "") -> AttnInputs:
+    """i.i.d. N(0,1) q, k, v (and dO) for a dense [B·N] or a packed (``seqlens``) batch."""
+    if seqlens is not None:
+        cu = cu_from_lengths(seqlens)
+        T, B, N = int(cu[-1]), len(seqlens), max(seqlens) if seqlens else 0
+    else:
+        cu, T, seqlens = None, B * N, [N] * B
+    g = torch.Generator().manual_seed(seed)
+    q = _randn(g, (T, H, d), dtype)
+    k = _randn(g, (T, H, d), dtype)
+    v = _randn(g, (T, H, d), dtype)
+    do = None
+    if backward:
+        g2 = torch.Generator().manual_seed(seed + 1)
+        do = _randn(g2, (T, H, d), dtype)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    return AttnInputs(q, k, v, do, cu, list(seqlens), B, H, N, d, float(scale), bool(causal), dtype, name)
+
+
+def make_workload(name: str, backward: Optional[bool] = None) -> AttnInputs:
+    """Inputs of one of the named workloads (on the CPU)."""
+    w = dict(WORKLOADS[name])
+    bwd = w["backward"] if backward is None else backward
+    if "nseq" in w:
+        lens = varlen_lengths(w["nseq"], w["lmin"], w["lmax"], w["seed"])
+        return random_inputs(w["H"], w["d"], w["dtype"], w["seed"], seqlens=lens, causal=w["causal"],
+                             backward=bwd, name=name)
+    return random_inputs(w["H"], w["d"], w["dtype"], w["seed"], B=w["B"], N=w["N"], causal=w["causal"],
+                         backward=bwd, name=name)
+
+
+def hand_example_inputs(dtype: str = "fp16", d: int = 64) -> AttnInputs:
+    """The narration's worked example as an attention call (B=1, H=1, N=4).
+
+    Every query row is (1/scale)·e₀, so scale·q·k_j equals the first feature of
+    k_j; key j carries ln c_j in that feature with c = [1, 2, 4, 3], and value
+    j carries [10, 20, 30, 40][j] in its first feature.  All other features are
+    zero.  The exact non-causal answer in feature 0 is 29 for every row.
+    """
+    scale = 1.0 / math.sqrt(d)
+    c = [1.0, 2.0, 4.0, 3.0]
+    vals = [10.0, 20.0, 30.0, 40.0]
+    q = torch.zeros(4, 1, d, dtype=torch.float64)
+    k = torch.zeros(4, 1, d, dtype=torch.float64)
+    v = torch.zeros(4, 1, d, dtype=torch.float64)
+    q[:, 0, 0] = 1.0 / scale
+    for j in range(4):
+        k[j, 0, 0] = math.log(c[j])
+        v[j, 0, 0] = vals[j]
+    tdt = TORCH_DTYPES[dtype]
+    return AttnInputs(q.to(tdt), k.to(tdt), v.to(tdt), None, None, [4], 1, 1, 4, d, scale, False, dtype,
+                      "hand_example")
