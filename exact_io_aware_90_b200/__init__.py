@@ -1,0 +1,212 @@
+"""B200-native exact attention (forward and recomputing backward) for sm_100a.
+
+This package is a thin Python binding over ``libfa_b200.so`` — the C ABI
+declared in ``include/fa.h``.  Every step of the computation runs in the
+library's CUDA kernels; Python only marshals arguments (device pointers, sizes,
+the current CUDA stream) and, in the convenience wrappers, allocates output
+tensors with PyTorch.  There is no fallback: if the library is missing or no
+GPU is present the calls raise.
+
+Raw ABI (same names and argument order as ``include/fa.h``; pointers are ints):
+    fa_fwd, fa_bwd, fa_bwd_preprocess, fa_bwd_main, fa_bwd_postprocess,
+    fa_bwd_workspace_bytes, fa_check_device_status, fa_set_watchdog_ns,
+    fa_watchdog_selftest, fa_status_string, fa_version
+Torch wrappers:
+    attention_forward(q, k, v, ...)          -> (o, lse)
+    attention_backward(q, k, v, o, lse, do, ...) -> (dq, dk, dv)
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+__all__ = [
+    "FAError", "LIB_PATH", "lib", "FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA",
+    "FA_ERR_TIMEOUT", "FA_BF16", "FA_FP16",
+    "fa_fwd", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_postprocess", "fa_bwd_workspace_bytes",
+    "fa_check_device_status", "fa_set_watchdog_ns", "fa_watchdog_selftest", "fa_status_string", "fa_version",
+    "attention_forward", "attention_backward", "dtype_code",
+]
+
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = 0, 1, 2, 3, 4
+FA_BF16, FA_FP16 = 0, 1
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa_b200.so")
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {fa_status_string(status)} ({status})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m exact_io_aware_90_b200.build` "
+            "(nvcc, sm_100a). There is no fallback implementation.")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, F, S, U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_uint64
+    sig = {
+        "fa_fwd": (I, [P, P, P, P, P, I, I, I, I, F, I, P, I, I, P]),
+        "fa_bwd_workspace_bytes": (S, [I, I, I]),
+        "fa_bwd": (I, [P, P, P, P, P, P, P, P, P, I, I, I, I, F, I, P, I, I, P, S, P]),
+        "fa_bwd_preprocess": (I, [P, P, I, I, I, I, P, I, I, P, S, P]),
+        "fa_bwd_main": (I, [P, P, P, P, P, P, P, I, I, I, I, F, I, P, I, I, P, S, P]),
+        "fa_bwd_postprocess": (I, [P, I, I, I, I, F, P, I, I, P, S, P]),
+        "fa_check_device_status": (I, [P]),
+        "fa_set_watchdog_ns": (None, [U64]),
+        "fa_watchdog_selftest": (I, [U64, P]),
+        "fa_status_string": (ctypes.c_char_p, [I]),
+        "fa_version": (ctypes.c_char_p, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    return L
+
+
+lib = _load()
+
+
+# ----------------------------------------------------------------------------- raw ABI (ints for pointers)
+
+def fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, cu_seqlens, total_tokens, dtype, stream) -> int:
+    return lib.fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, cu_seqlens, total_tokens, dtype, stream)
+
+
+def fa_bwd_workspace_bytes(total_tokens, H, d) -> int:
+    return lib.fa_bwd_workspace_bytes(total_tokens, H, d)
+
+
+def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, cu_seqlens, total_tokens, dtype,
+           workspace, workspace_bytes, stream) -> int:
+    return lib.fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, cu_seqlens, total_tokens, dtype,
+                      workspace, workspace_bytes, stream)
+
+
+def fa_bwd_preprocess(o, dO, B, H, N, d, cu_seqlens, total_tokens, dtype, workspace, workspace_bytes, stream) -> int:
+    return lib.fa_bwd_preprocess(o, dO, B, H, N, d, cu_seqlens, total_tokens, dtype, workspace, workspace_bytes,
+                                 stream)
+
+
+def fa_bwd_main(q, k, v, lse, dO, dk, dv, B, H, N, d, scale, causal, cu_seqlens, total_tokens, dtype, workspace,
+                workspace_bytes, stream) -> int:
+    return lib.fa_bwd_main(q, k, v, lse, dO, dk, dv, B, H, N, d, scale, causal, cu_seqlens, total_tokens, dtype,
+                           workspace, workspace_bytes, stream)
+
+
+def fa_bwd_postprocess(dq, B, H, N, d, scale, cu_seqlens, total_tokens, dtype, workspace, workspace_bytes,
+                       stream) -> int:
+    return lib.fa_bwd_postprocess(dq, B, H, N, d, scale, cu_seqlens, total_tokens, dtype, workspace,
+                                  workspace_bytes, stream)
+
+
+def fa_check_device_status(stream) -> int:
+    return lib.fa_check_device_status(stream)
+
+
+def fa_set_watchdog_ns(ns: int) -> None:
+    lib.fa_set_watchdog_ns(int(ns))
+
+
+def fa_watchdog_selftest(timeout_ns: int, stream) -> int:
+    return lib.fa_watchdog_selftest(int(timeout_ns), stream)
+
+
+def fa_status_string(status: int) -> str:
+    return lib.fa_status_string(int(status)).decode()
+
+
+def fa_version() -> str:
+    return lib.fa_version().decode()
+
+
+# ----------------------------------------------------------------------------- torch wrappers
+
+def dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return FA_BF16
+    if t.dtype == torch.float16:
+        return FA_FP16
+    raise TypeError(f"unsupported dtype {t.dtype}: q/k/v must be bfloat16 or float16")
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _shape(q, cu_seqlens, max_seqlen, batch):
+    T, H, d = q.shape
+    if cu_seqlens is None:
+        B = 1 if batch is None else int(batch)
+        if T % B:
+            raise ValueError("token count must be a multiple of the batch size")
+        N = T // B
+    else:
+        B = int(cu_seqlens.numel()) - 1
+        if max_seqlen is None:
+            raise ValueError("max_seqlen is required with cu_seqlens")
+        N = int(max_seqlen)
+    return B, H, N, d, T
+
+
+def _check(t, name, q):
+    if not t.is_cuda or not t.is_contiguous() or t.dtype != q.dtype or t.shape != q.shape:
+        raise ValueError(f"{name} must be a contiguous CUDA tensor like q")
+
+
+def attention_forward(q, k, v, causal: bool = False, scale: Optional[float] = None, cu_seqlens=None,
+                      max_seqlen: Optional[int] = None, batch: Optional[int] = None, out=None, lse=None,
+                      stream=None) -> Tuple["torch.Tensor", "torch.Tensor"]:
+    """O and LSE for q, k, v of shape [T, H, d] (see ``include/fa.h``)."""
+    import torch
+    for t, n in ((k, "k"), (v, "v")):
+        _check(t, n, q)
+    _check(q, "q", q)
+    B, H, N, d, T = _shape(q, cu_seqlens, max_seqlen, batch)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((T, H), dtype=torch.float32, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    st = lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, d, float(scale), int(bool(causal)),
+                    _ptr(cu_seqlens), T, dtype_code(q), stream)
+    if st != FA_OK:
+        raise FAError(st, "fa_fwd")
+    return out, lse
+
+
+def attention_backward(q, k, v, o, lse, do, causal: bool = False, scale: Optional[float] = None, cu_seqlens=None,
+                       max_seqlen: Optional[int] = None, batch: Optional[int] = None, dq=None, dk=None, dv=None,
+                       workspace=None, stream=None):
+    """dq, dk, dv for the forward that produced (o, lse)."""
+    import torch
+    for t, n in ((k, "k"), (v, "v"), (o, "o"), (do, "do")):
+        _check(t, n, q)
+    _check(q, "q", q)
+    B, H, N, d, T = _shape(q, cu_seqlens, max_seqlen, batch)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    need = lib.fa_bwd_workspace_bytes(T, H, d)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    st = lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv), B, H, N,
+                    d, float(scale), int(bool(causal)), _ptr(cu_seqlens), T, dtype_code(q), _ptr(workspace),
+                    workspace.numel() * workspace.element_size(), stream)
+    if st != FA_OK:
+        raise FAError(st, "fa_bwd")
+    return dq, dk, dv

@@ -1,0 +1,665 @@
+// fa_bwd.cu — attention backward for sm_100a.
+//
+// The forward keeps only O and the row log-sum-exp; the backward recomputes
+// the probabilities tile by tile from Q, K and the LSE ("FlashAttention
+// 短片讲解稿", segment "第三招 · 反向重计算").  The gradient equations are the
+// chain rule of the forward definition:
+//   P = exp(scale·QKᵀ − LSE),  dV = Pᵀ dO,  dP = dO Vᵀ,  D_i = Σ_c dO_ic O_ic,
+//   dS = P ∘ (dP − D),  dQ = scale·dS K,  dK = scale·dSᵀ Q.
+//
+// Three kernels on one stream:
+//   fa_bwd_pre_kernel   D (fp32 [T, H]) and a zeroed fp32 dQ accumulator
+//   fa_bwd_main_kernel  one CTA per (sequence, head, 128-key tile j):
+//                       K_j, V_j stay in shared memory; Q_i, dO_i stream in.
+//                       Per Q tile (BQ rows: 64 at d = 128, 128 at d = 64):
+//                         Sᵀ  = K_j Q_iᵀ        (tensor memory, fp32)
+//                         dPᵀ = V_j dO_iᵀ
+//                         Pᵀ  = 2^(c·Sᵀ − LSE_i·log2 e), masked   (warps 0-3)
+//                         dV += Pᵀ dO_i         (Pᵀ read from tensor memory)
+//                         dSᵀ = Pᵀ ∘ (dPᵀ − D_i)                  (warps 0-3)
+//                         dK += dSᵀ Q_i         (dSᵀ read from tensor memory)
+//                         dQ_i partial = dS K_j (dSᵀ staged in shared memory)
+//                       and warps 4-7 add the dQ partial into the fp32
+//                       accumulator with vector reductions.  dK (× scale)
+//                       and dV are written once at the end.
+//   fa_bwd_post_kernel  dq = scale · accumulator, rounded to the dtype
+// All five MMAs are M = 128 (full tensor-core rate): at d = 128 the dQ
+// product is formed transposed, dQᵀ = K_jᵀ dSᵀ (M = d), at d = 64 directly
+// (M = BQ = 128).
+#include "fa_internal.h"
+#include "sm100.cuh"
+
+namespace fa {
+
+// ============================================================================ preprocess / postprocess
+
+// One thread per 8 features of one (token, head) row.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const uint4* __restrict__ o, const uint4* __restrict__ dO,
+                                                         float* __restrict__ delta, float4* __restrict__ dq_acc,
+                                                         long long rows) {
+  constexpr int TPR = D / 8;  // threads per row
+  const long long n = rows * TPR;
+  const int lane = threadIdx.x & 31;
+  const long long warp0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
+  // whole warps step together so the row reduction below always has 32 lanes
+  for (long long base = warp0 * 32; base < n; base += nwarps * 32) {
+    const long long idx = base + lane;
+    const bool live = idx < n;
+    float acc = 0.f;
+    if (live) {
+      const uint4 a = __ldg(o + idx);
+      const uint4 g = __ldg(dO + idx);
+      const uint32_t av[4] = {a.x, a.y, a.z, a.w};
+      const uint32_t gv[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float2 fa, fg;
+        if constexpr (BF16) {
+          fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&av[i]));
+          fg = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gv[i]));
+        } else {
+          fa = __half22float2(*reinterpret_cast<const __half2*>(&av[i]));
+          fg = __half22float2(*reinterpret_cast<const __half2*>(&gv[i]));
+        }
+        acc = fmaf(fa.x, fg.x, acc);
+        acc = fmaf(fa.y, fg.y, acc);
+      }
+    }
+    // reduce over the TPR consecutive lanes of this row (TPR divides 32, rows start at multiples of TPR)
+#pragma unroll
+    for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (live) {
+      if ((lane % TPR) == 0) delta[idx / TPR] = acc;
+      const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+      dq_acc[2 * idx] = z;
+      dq_acc[2 * idx + 1] = z;
+    }
+  }
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(256) fa_bwd_post_kernel(const float4* __restrict__ dq_acc, uint2* __restrict__ dq,
+                                                          long long n4, float scale, const int32_t* cu_seqlens,
+                                                          int B, long long row_elems4) {
+  long long limit = n4;
+  if (cu_seqlens != nullptr) limit = min(n4, (long long)__ldg(cu_seqlens + B) * row_elems4);
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < limit; i += (long long)gridDim.x * blockDim.x) {
+    const float4 a = dq_acc[i];
+    uint2 out;
+    out.x = pack2<BF16>(a.x * scale, a.y * scale);
+    out.y = pack2<BF16>(a.z * scale, a.w * scale);
+    dq[i] = out;
+  }
+}
+
+// ============================================================================ main kernel
+
+struct BwdParams {
+  const float* lse;
+  const float* delta;
+  float* dq_acc;
+  void* dk;
+  void* dv;
+  const int32_t* cu_seqlens;
+  int B, H, N, T;
+  int causal;
+  int num_kblocks;  // ceil(N / 128)
+  int heads_group;
+  float scale;
+  float scale_log2;
+  uint64_t timeout_ns;
+};
+
+constexpr int kBwdThreads = 320;
+constexpr int kBK = 128;  // keys per CTA
+
+template <int D>
+struct BwdCfg {
+  static constexpr int BQ = (D == 128) ? 64 : 128;  // query rows per inner step
+  static constexpr int NCH = D / 64;
+  static constexpr uint32_t KV_TILE = kBK * D * 2;
+  static constexpr uint32_t Q_TILE = BQ * D * 2;
+  static constexpr uint32_t DS_TILE = kBK * BQ * 2;
+  static constexpr int STAGES = 2;
+  // tensor memory columns
+  static constexpr uint32_t T_ST = 0;          // Sᵀ  [128 keys × BQ]
+  static constexpr uint32_t T_DPT = BQ;        // dPᵀ [128 keys × BQ]
+  static constexpr uint32_t T_DQ = 2 * BQ;     // dQᵀ [d × 64] or dQ [128 × 64]: 64 columns
+  static constexpr uint32_t T_DK = (D == 128) ? 256 : 320;
+  static constexpr uint32_t T_DV = T_DK + D;
+  // barriers
+  static constexpr int B_KV = 0;
+  static constexpr int B_QFULL = 1;
+  static constexpr int B_QEMPTY = B_QFULL + STAGES;
+  static constexpr int B_ROWFULL = B_QEMPTY + STAGES;  // LSE / D of the Q tile in shared memory
+  static constexpr int B_SFULL = B_ROWFULL + STAGES;
+  static constexpr int B_DPFULL = B_SFULL + 1;
+  static constexpr int B_PREADY = B_DPFULL + 1;
+  static constexpr int B_DSREADY = B_PREADY + 1;
+  static constexpr int B_DQFULL = B_DSREADY + 1;
+  static constexpr int B_DQFREE = B_DQFULL + 1;
+  static constexpr int B_DKV = B_DQFREE + 1;
+  static constexpr int B_DRAIN = B_DKV + 1;
+  static constexpr int NBARS = B_DRAIN + 1;
+  // shared memory
+  static constexpr uint32_t OFF_K = 0;
+  static constexpr uint32_t OFF_V = KV_TILE;
+  static constexpr uint32_t OFF_Q = 2 * KV_TILE;
+  static constexpr uint32_t OFF_DO = OFF_Q + STAGES * Q_TILE;
+  static constexpr uint32_t OFF_DS = OFF_DO + STAGES * Q_TILE;
+  static constexpr uint32_t OFF_ROW = OFF_DS + DS_TILE;  // per stage: lse·log2(e)[BQ], D[BQ] (fp32)
+  static constexpr uint32_t OFF_BAR = OFF_ROW + STAGES * 2 * BQ * 4;
+  static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
+  static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;
+};
+
+__device__ __forceinline__ void drain_wait_b(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > limit_ns) {
+      record_status(4);
+      return;
+    }
+  }
+}
+
+__device__ __forceinline__ bool warp_wait_b(uint32_t bar, uint32_t parity, const Watchdog& wd) {
+  const bool ok = mbar_wait(bar, parity, wd);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ void red_add_f32(float* p, float v) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+}
+
+__device__ __forceinline__ void red_add_v4_f32(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                       const BwdParams p) {
+  using C = BwdCfg<D>;
+  constexpr int BQ = C::BQ;
+  // Sᵀ = K Qᵀ and dPᵀ = V dOᵀ: M = 128 keys, N = BQ, both operands K-major
+  constexpr uint32_t IDESC_ST = idesc_f16(BF16, kBK, BQ, false, false);
+  // dV += Pᵀ dO and dK += dSᵀ Q: A from tensor memory, B (dO / Q) MN-major, N = d
+  constexpr uint32_t IDESC_DKV = idesc_f16(BF16, kBK, D, false, true);
+  // d = 128: dQᵀ = Kᵀ dSᵀ, M = d, N = 64, A = K MN-major, B = dSᵀ MN-major
+  // d = 64 : dQ  = dS K,   M = 128, N = 64, A = dS MN-major, B = K MN-major
+  constexpr uint32_t IDESC_DQ = idesc_f16(BF16, 128, 64, true, true);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t s_base = smem_u32(smem);
+  const uint32_t sK = s_base + C::OFF_K;
+  const uint32_t sV = s_base + C::OFF_V;
+  const uint32_t sQ = s_base + C::OFF_Q;
+  const uint32_t sDO = s_base + C::OFF_DO;
+  const uint32_t sDS = s_base + C::OFF_DS;
+  float* row_buf = reinterpret_cast<float*>(smem + C::OFF_ROW);
+  const uint32_t bar0 = s_base + C::OFF_BAR;
+  auto bar = [&](int i) -> uint32_t { return bar0 + 8u * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  int* abort_flag = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work unit: heads in groups, heaviest key tiles (the first ones when causal) first
+  const int BH = p.B * p.H;
+  const int nkb = p.num_kblocks;
+  const int G = p.heads_group;
+  const int unit = blockIdx.x;
+  const int group = unit / (G * nkb);
+  const int g_heads = min(G, BH - group * G);
+  const int r = unit - group * G * nkb;
+  const int kb = r / g_heads;
+  const int bh = group * G + r % g_heads;
+  const int b = bh / p.H;
+  const int h = bh - b * p.H;
+
+  int tok0, L;
+  if (p.cu_seqlens != nullptr) {
+    tok0 = __ldg(p.cu_seqlens + b);
+    const int end = __ldg(p.cu_seqlens + b + 1);
+    L = end - tok0;
+    if (tok0 < 0 || L < 0 || end > p.T || L > p.N) {
+      if (threadIdx.x == 0) record_status(1);
+      return;
+    }
+  } else {
+    tok0 = b * p.N;
+    L = p.N;
+  }
+  const int k0 = kb * kBK;
+  if (k0 >= L) return;
+  const int nq_all = (L + BQ - 1) / BQ;
+  const int i_begin = p.causal ? k0 / BQ : 0;
+  const int n_it = nq_all - i_begin;  // ≥ 1
+
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 0) {
+    mbar_init(bar(C::B_KV), 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(bar(C::B_QFULL + s), 1);
+      mbar_init(bar(C::B_QEMPTY + s), 1);
+      mbar_init(bar(C::B_ROWFULL + s), 32);
+    }
+    mbar_init(bar(C::B_SFULL), 1);
+    mbar_init(bar(C::B_DPFULL), 1);
+    mbar_init(bar(C::B_PREADY), 128);
+    mbar_init(bar(C::B_DSREADY), 128);
+    mbar_init(bar(C::B_DQFULL), 1);
+    mbar_init(bar(C::B_DQFREE), 128);
+    mbar_init(bar(C::B_DKV), 1);
+    mbar_init(bar(C::B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8 && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    prefetch_tmap(&tm_do);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Watchdog wd{abort_flag, p.timeout_ns};
+
+  if (warp == 8) {
+    // ================================================================ TMA producer (+ row terms)
+    const uint64_t pol_kv = l2_policy_evict_first();
+    const uint64_t pol_q = l2_policy_evict_last();
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar(C::B_KV), 2 * C::KV_TILE);
+      for (int c = 0; c < C::NCH; ++c) {
+        tma_load_3d(sK + c * (kBK * 128), &tm_k, bar(C::B_KV), c * 64, h, tok0 + k0, pol_kv);
+        tma_load_3d(sV + c * (kBK * 128), &tm_v, bar(C::B_KV), c * 64, h, tok0 + k0, pol_kv);
+      }
+    }
+    int issued = 0;
+    const float LOG2E = 1.4426950408889634f;
+    for (int it = 0; it < n_it; ++it) {
+      const int s = it % C::STAGES;
+      if (it >= C::STAGES && !warp_wait_b(bar(C::B_QEMPTY + s), ((it / C::STAGES) - 1) & 1, wd)) break;
+      const int i0 = (i_begin + it) * BQ;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar(C::B_QFULL + s), 2 * C::Q_TILE);
+        for (int c = 0; c < C::NCH; ++c) {
+          tma_load_3d(sQ + s * C::Q_TILE + c * (BQ * 128), &tm_q, bar(C::B_QFULL + s), c * 64, h, tok0 + i0, pol_q);
+          tma_load_3d(sDO + s * C::Q_TILE + c * (BQ * 128), &tm_do, bar(C::B_QFULL + s), c * 64, h, tok0 + i0, pol_q);
+        }
+      }
+      // LSE (pre-multiplied by log2 e) and D of the tile's query rows; rows past the sequence get 0
+      float* lse_s = row_buf + s * 2 * BQ;
+      float* del_s = lse_s + BQ;
+      for (int q = lane; q < BQ; q += 32) {
+        const int qrow = i0 + q;
+        const bool v = qrow < L;
+        lse_s[q] = v ? __ldg(p.lse + (size_t)(tok0 + qrow) * p.H + h) * LOG2E : 0.f;
+        del_s[q] = v ? __ldg(p.delta + (size_t)(tok0 + qrow) * p.H + h) : 0.f;
+      }
+      mbar_arrive(bar(C::B_ROWFULL + s));  // release: the stores above are visible to waiters
+      issued = it + 1;
+    }
+    if (lane == 0) {
+      drain_wait_b(bar(C::B_KV), 0, p.timeout_ns);
+      for (int it = max(0, issued - C::STAGES); it < issued; ++it)
+        drain_wait_b(bar(C::B_QFULL + it % C::STAGES), (it / C::STAGES) & 1, p.timeout_ns);
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      const uint32_t tST = tmem + C::T_ST, tDPT = tmem + C::T_DPT, tDQ = tmem + C::T_DQ;
+      const uint32_t tDK = tmem + C::T_DK, tDV = tmem + C::T_DV;
+      bool ok = mbar_wait(bar(C::B_KV), 0, wd);
+      for (int it = 0; ok && it < n_it; ++it) {
+        const int s = it % C::STAGES;
+        if (!mbar_wait(bar(C::B_QFULL + s), (it / C::STAGES) & 1, wd)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t q_t = sQ + s * C::Q_TILE, do_t = sDO + s * C::Q_TILE;
+        // Sᵀ = K Qᵀ, dPᵀ = V dOᵀ (K-major operands; K dim = d)
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off_k = (kk >> 2) * (kBK * 128) + (kk & 3) * 32;
+          const uint32_t off_q = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
+          mma_ss(tST, sdesc_sw128(sK + off_k, 16, 1024), sdesc_sw128(q_t + off_q, 16, 1024), IDESC_ST, kk > 0);
+        }
+        tc_commit(bar(C::B_SFULL));
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off_k = (kk >> 2) * (kBK * 128) + (kk & 3) * 32;
+          const uint32_t off_q = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
+          mma_ss(tDPT, sdesc_sw128(sV + off_k, 16, 1024), sdesc_sw128(do_t + off_q, 16, 1024), IDESC_ST, kk > 0);
+        }
+        tc_commit(bar(C::B_DPFULL));
+        // dV += Pᵀ dO   (Pᵀ packed in the Sᵀ columns; dO MN-major, K dim = BQ queries)
+        if (!mbar_wait(bar(C::B_PREADY), it & 1, wd)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BQ / 16; ++kk)
+          mma_ts(tDV, tST + kk * 8, sdesc_sw128(do_t + kk * 16 * 128, BQ * 128, 1024), IDESC_DKV,
+                 (it > 0 || kk > 0) ? 1u : 0u);
+        // dK += dSᵀ Q
+        if (!mbar_wait(bar(C::B_DSREADY), it & 1, wd)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BQ / 16; ++kk)
+          mma_ts(tDK, tDPT + kk * 8, sdesc_sw128(q_t + kk * 16 * 128, BQ * 128, 1024), IDESC_DKV,
+                 (it > 0 || kk > 0) ? 1u : 0u);
+        // dQ partial (K dim = 128 keys); the dQ columns must have been read out
+        if (it > 0 && !mbar_wait(bar(C::B_DQFREE), (it - 1) & 1, wd)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+          if constexpr (D == 128) {
+            // A = Kᵀ (MN-major: 64-feature chunks 16 KB apart), B = dSᵀ [keys][64 q] (MN-major)
+            mma_ss(tDQ, sdesc_sw128(sK + kk * 16 * 128, kBK * 128, 1024), sdesc_sw128(sDS + kk * 16 * 128, 16, 1024),
+                   IDESC_DQ, kk > 0);
+          } else {
+            // A = dS (MN-major over queries: 64-query chunks 16 KB apart), B = K (MN-major, one chunk)
+            mma_ss(tDQ, sdesc_sw128(sDS + kk * 16 * 128, kBK * 128, 1024), sdesc_sw128(sK + kk * 16 * 128, 16, 1024),
+                   IDESC_DQ, kk > 0);
+          }
+        }
+        tc_commit(bar(C::B_DQFULL));
+        tc_commit(bar(C::B_QEMPTY + s));
+      }
+      tc_commit(bar(C::B_DKV));
+      tc_commit(bar(C::B_DRAIN));
+      drain_wait_b(bar(C::B_DRAIN), 0, p.timeout_ns);
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ================================================================ Pᵀ / dSᵀ warpgroup (thread = key row)
+    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+    const uint32_t tST = tmem + lane_off + C::T_ST;
+    const uint32_t tDPT = tmem + lane_off + C::T_DPT;
+    const uint32_t tDV = tmem + lane_off + C::T_DV;
+    const int kr = 32 * warp + lane;  // key row within the tile
+    const int key = k0 + kr;          // position in the sequence
+    const float c = p.scale_log2;
+    bool ok = true;
+    for (int it = 0; it < n_it; ++it) {
+      const int i0 = (i_begin + it) * BQ;
+      const int s = it % C::STAGES;
+      if (!warp_wait_b(bar(C::B_ROWFULL + s), (it / C::STAGES) & 1, wd)) { ok = false; break; }
+      const float* lse_s = row_buf + s * 2 * BQ;
+      const float* del_s = lse_s + BQ;
+      // visible queries for this key: q >= key (causal) and q < L; key < L
+      int q_lo = p.causal ? key - i0 : 0;  // first visible column
+      int q_hi = L - i0;                   // one past the last visible column
+      if (key >= L) q_hi = -1;
+      if (!warp_wait_b(bar(C::B_SFULL), it & 1, wd)) { ok = false; break; }
+      tc_fence_after();
+      float pt[BQ];
+      {
+        uint32_t sr[BQ];
+#pragma unroll
+        for (int q = 0; q < BQ / 32; ++q) tmem_ld32(tST + 32u * q, reinterpret_cast<uint32_t(&)[32]>(sr[32 * q]));
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < BQ; ++i) {
+          const float e = ex2(fmaf(__uint_as_float(sr[i]), c, -lse_s[i]));
+          pt[i] = (i >= q_lo && i < q_hi) ? e : 0.f;
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < BQ / 64; ++q) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) pk[i] = pack2<BF16>(pt[64 * q + 2 * i], pt[64 * q + 2 * i + 1]);
+        tmem_st32(tST + 32u * q, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(C::B_PREADY));
+      if (!warp_wait_b(bar(C::B_DPFULL), it & 1, wd)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t dsk[BQ / 2];
+      {
+        uint32_t dr[BQ];
+#pragma unroll
+        for (int q = 0; q < BQ / 32; ++q) tmem_ld32(tDPT + 32u * q, reinterpret_cast<uint32_t(&)[32]>(dr[32 * q]));
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < BQ / 2; ++i) {
+          const float d0 = pt[2 * i] * (__uint_as_float(dr[2 * i]) - del_s[2 * i]);
+          const float d1 = pt[2 * i + 1] * (__uint_as_float(dr[2 * i + 1]) - del_s[2 * i + 1]);
+          dsk[i] = pack2<BF16>(d0, d1);
+        }
+      }
+      // dSᵀ into tensor memory (A of the dK product) ...
+#pragma unroll
+      for (int q = 0; q < BQ / 64; ++q) tmem_st32(tDPT + 32u * q, reinterpret_cast<uint32_t(&)[32]>(dsk[32 * q]));
+      // ... and into shared memory, 128-byte swizzled rows = keys (operand of the dQ product);
+      // the previous dQ product must have finished reading the buffer
+      if (it > 0 && !warp_wait_b(bar(C::B_DQFULL), (it - 1) & 1, wd)) { ok = false; break; }
+      {
+        uint8_t* ds_row = smem + C::OFF_DS + kr * 128;
+#pragma unroll
+        for (int q = 0; q < BQ / 64; ++q) {
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            const int sw = ch ^ (kr & 7);
+            uint4 v4 = make_uint4(dsk[32 * q + 4 * ch], dsk[32 * q + 4 * ch + 1], dsk[32 * q + 4 * ch + 2],
+                                  dsk[32 * q + 4 * ch + 3]);
+            *reinterpret_cast<uint4*>(ds_row + q * (kBK * 128) + sw * 16) = v4;
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(C::B_DSREADY));
+    }
+    // ---- epilogue: dV rows of this tile
+    if (ok && warp_wait_b(bar(C::B_DKV), 0, wd)) {
+      tc_fence_after();
+      const bool valid = key < L;
+      uint8_t* dst = reinterpret_cast<uint8_t*>(p.dv) + (((size_t)(tok0 + (valid ? key : 0)) * p.H + h) * D) * 2;
+#pragma unroll
+      for (int q = 0; q < D / 32; ++q) {
+        uint32_t r32[32];
+        tmem_ld32(tDV + 32u * q, r32);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[i] = pack2<BF16>(__uint_as_float(r32[2 * i]), __uint_as_float(r32[2 * i + 1]));
+        if (valid) {
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            st_global_v4(dst + q * 64 + v4 * 16, pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ================================================================ dQ warpgroup (warps 4-7)
+    const int quarter = warp & 3;
+    const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
+    const uint32_t tDQ = tmem + lane_off + C::T_DQ;
+    const uint32_t tDK = tmem + lane_off + C::T_DK;
+    const int lrow = 32 * quarter + lane;  // tensor-memory lane of this thread
+    bool ok = true;
+    for (int it = 0; it < n_it; ++it) {
+      const int i0 = (i_begin + it) * BQ;
+      if (!warp_wait_b(bar(C::B_DQFULL), it & 1, wd)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t qr[64];
+      tmem_ld32(tDQ, reinterpret_cast<uint32_t(&)[32]>(qr[0]));
+      tmem_ld32(tDQ + 32u, reinterpret_cast<uint32_t(&)[32]>(qr[32]));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar(C::B_DQFREE));
+      if constexpr (D == 128) {
+        // lane = feature, columns = 64 queries: each warp instruction covers 32 consecutive features
+        float* base = p.dq_acc + ((size_t)(tok0 + i0) * p.H + h) * D + lrow;
+        const int nq = min(64, L - i0);
+#pragma unroll 8
+        for (int q = 0; q < 64; ++q)
+          if (q < nq) red_add_f32(base + (size_t)q * p.H * D, __uint_as_float(qr[q]));
+      } else {
+        // lane = query row, columns = 64 features
+        const int qrow = i0 + lrow;
+        if (qrow < L) {
+          float* base = p.dq_acc + ((size_t)(tok0 + qrow) * p.H + h) * D;
+#pragma unroll
+          for (int f = 0; f < 64; f += 4)
+            red_add_v4_f32(base + f, __uint_as_float(qr[f]), __uint_as_float(qr[f + 1]), __uint_as_float(qr[f + 2]),
+                           __uint_as_float(qr[f + 3]));
+        }
+      }
+    }
+    // ---- epilogue: dK rows (× scale)
+    if (ok && warp_wait_b(bar(C::B_DKV), 0, wd)) {
+      tc_fence_after();
+      const int key = k0 + lrow;
+      const bool valid = key < L;
+      uint8_t* dst = reinterpret_cast<uint8_t*>(p.dk) + (((size_t)(tok0 + (valid ? key : 0)) * p.H + h) * D) * 2;
+#pragma unroll
+      for (int q = 0; q < D / 32; ++q) {
+        uint32_t r32[32];
+        tmem_ld32(tDK + 32u * q, r32);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pk[i] = pack2<BF16>(__uint_as_float(r32[2 * i]) * p.scale, __uint_as_float(r32[2 * i + 1]) * p.scale);
+        if (valid) {
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            st_global_v4(dst + q * 64 + v4 * 16, pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+        }
+      }
+    }
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ============================================================================ launchers
+
+static int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int D, bool BF16>
+static cudaError_t launch_pre_t(const Problem& pb, const BwdArgs& a, cudaStream_t stream) {
+  const long long rows = (long long)pb.T * pb.H;
+  const long long threads = rows * (D / 8);
+  long long blocks = (threads + 255) / 256;
+  const long long cap = (long long)num_sms() * 8;
+  if (blocks > cap) blocks = cap;
+  fa_bwd_pre_kernel<D, BF16><<<(unsigned)blocks, 256, 0, stream>>>(
+      reinterpret_cast<const uint4*>(a.o), reinterpret_cast<const uint4*>(a.dO), a.delta,
+      reinterpret_cast<float4*>(a.dq_acc), rows);
+  return cudaPeekAtLastError();
+}
+
+cudaError_t launch_bwd_pre(const Problem& pb, const BwdArgs& a, cudaStream_t stream) {
+  if (pb.d == 128) return pb.bf16 ? launch_pre_t<128, true>(pb, a, stream) : launch_pre_t<128, false>(pb, a, stream);
+  return pb.bf16 ? launch_pre_t<64, true>(pb, a, stream) : launch_pre_t<64, false>(pb, a, stream);
+}
+
+cudaError_t launch_bwd_post(const Problem& pb, const BwdArgs& a, cudaStream_t stream) {
+  const long long n4 = (long long)pb.T * pb.H * pb.d / 4;
+  long long blocks = (n4 + 255) / 256;
+  const long long cap = (long long)num_sms() * 8;
+  if (blocks > cap) blocks = cap;
+  const long long row4 = (long long)pb.H * pb.d / 4;
+  if (pb.bf16)
+    fa_bwd_post_kernel<true><<<(unsigned)blocks, 256, 0, stream>>>(reinterpret_cast<const float4*>(a.dq_acc),
+                                                                   reinterpret_cast<uint2*>(a.dq), n4, pb.scale,
+                                                                   pb.cu_seqlens, pb.B, row4);
+  else
+    fa_bwd_post_kernel<false><<<(unsigned)blocks, 256, 0, stream>>>(reinterpret_cast<const float4*>(a.dq_acc),
+                                                                    reinterpret_cast<uint2*>(a.dq), n4, pb.scale,
+                                                                    pb.cu_seqlens, pb.B, row4);
+  return cudaPeekAtLastError();
+}
+
+template <int D, bool BF16>
+static cudaError_t launch_main_t(const Problem& pb, const BwdArgs& a, cudaStream_t stream) {
+  using C = BwdCfg<D>;
+  static bool configured = false;
+  auto kern = fa_bwd_main_kernel<D, BF16>;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  BwdParams p;
+  p.lse = a.lse;
+  p.delta = a.delta;
+  p.dq_acc = a.dq_acc;
+  p.dk = a.dk;
+  p.dv = a.dv;
+  p.cu_seqlens = pb.cu_seqlens;
+  p.B = pb.B;
+  p.H = pb.H;
+  p.N = pb.N;
+  p.T = pb.T;
+  p.causal = pb.causal;
+  p.num_kblocks = (pb.N + kBK - 1) / kBK;
+  p.heads_group = 8;
+  p.scale = pb.scale;
+  p.scale_log2 = pb.scale * 1.4426950408889634f;
+  p.timeout_ns = pb.timeout_ns;
+  const long long units = (long long)pb.B * pb.H * p.num_kblocks;
+  kern<<<dim3((unsigned)units), dim3(kBwdThreads), C::SMEM_BYTES, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, p);
+  return cudaPeekAtLastError();
+}
+
+cudaError_t launch_bwd_main(const Problem& pb, const BwdArgs& a, cudaStream_t stream) {
+  if (pb.d == 128) return pb.bf16 ? launch_main_t<128, true>(pb, a, stream) : launch_main_t<128, false>(pb, a, stream);
+  return pb.bf16 ? launch_main_t<64, true>(pb, a, stream) : launch_main_t<64, false>(pb, a, stream);
+}
+
+// ============================================================================ watchdog self-test
+
+__global__ void fa_watchdog_selftest_kernel(uint64_t timeout_ns) {
+  __shared__ __align__(8) uint64_t never;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&never), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const Watchdog wd{&abort_flag, timeout_ns};
+  // nothing arrives on `never`: the wait must give up and record FA_ERR_TIMEOUT
+  mbar_wait(smem_u32(&never), 0, wd);
+  __syncthreads();
+}
+
+cudaError_t launch_watchdog_selftest(uint64_t timeout_ns, cudaStream_t stream) {
+  fa_watchdog_selftest_kernel<<<1, 64, 0, stream>>>(timeout_ns);
+  return cudaPeekAtLastError();
+}
+
+}  // namespace fa

@@ -1,0 +1,430 @@
+// fa_fwd.cu — attention forward for sm_100a.
+//
+// Computes O = softmax(Q Kᵀ·scale [+ causal mask]) V and the row log-sum-exp
+// tile by tile with an online softmax ("FlashAttention 详解（零基础入门）" §5.2,
+// §5.4, §6.2): the [128 × 128] score tile S lives only in tensor memory, P is
+// written back over it in the input dtype and fed to the P·V MMA from there,
+// so neither S nor P ever reaches device memory.
+//
+// CTA = one work unit = (sequence, head, 256 query rows) split into two
+// 128-row Q tiles that take turns on the tensor core:
+//   warps 0-3  softmax of Q tile 0 (one thread per row; TMEM lanes 0-127)
+//   warps 4-7  softmax of Q tile 1
+//   warp  8    TMA producer: Q0/Q1 once, then the K/V ring
+//   warp  9    tensor-memory allocator and single-thread tcgen05 MMA issuer
+// Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+d),
+// O1 [256+d, 256+2d).  MMA issue order per KV tile j:
+//   P·V(0,j)  S(0,j+1)  P·V(1,j)  S(1,j+1)
+// so while one warpgroup exponentiates, the tensor core works for the other.
+// tcgen05 MMAs from one thread execute in issue order, so S(t,j+1) may
+// overwrite the columns holding P(t,j) once P·V(t,j) has been issued.
+//
+// Online softmax in base 2 with c = scale·log2(e): m is kept in the scaled
+// domain and P = 2^(c·s − m).  The running max is only raised when the tile
+// max exceeds it by more than 8 (a factor 256): O and ℓ are then both
+// expressed against the same, slightly stale reference, which leaves
+// O = Σ P V / Σ P unchanged (the rescaling argument of §5.2 run in reverse),
+// keeps every P ≤ 256, and makes the O rescale in tensor memory rare.
+#include "fa_internal.h"
+#include "sm100.cuh"
+
+namespace fa {
+
+struct FwdParams {
+  void* o;
+  float* lse;
+  const int32_t* cu_seqlens;
+  int B, H, N, T;
+  int causal;
+  int num_qblocks;   // ceil(N / 256)
+  int heads_group;   // heads per L2 group in the unit order
+  float scale_log2;  // scale · log2(e)
+  uint64_t timeout_ns;
+};
+
+constexpr int kFwdThreads = 320;
+constexpr int kBM = 128;  // query rows per tile
+constexpr int kBN = 128;  // keys per tile
+constexpr float kRescaleThreshold = 8.0f;
+
+template <int D>
+struct FwdCfg {
+  static constexpr int NCH = D / 64;                   // 128-byte feature chunks per row
+  static constexpr uint32_t TILE = kBM * D * 2;        // bytes of a 128-row tile
+  static constexpr int STAGES = (D == 128) ? 2 : 4;    // K/V ring depth
+  // barrier indices
+  static constexpr int B_Q = 0;
+  static constexpr int B_KFULL = 1;
+  static constexpr int B_VFULL = B_KFULL + STAGES;
+  static constexpr int B_KVEMPTY = B_VFULL + STAGES;
+  static constexpr int B_SFULL = B_KVEMPTY + STAGES;
+  static constexpr int B_PFULL = B_SFULL + 2;
+  static constexpr int B_PVDONE = B_PFULL + 2;
+  static constexpr int B_DRAIN = B_PVDONE + 2;
+  static constexpr int NBARS = B_DRAIN + 1;
+  static constexpr uint32_t OFF_Q = 0;
+  static constexpr uint32_t OFF_K = 2 * TILE;
+  static constexpr uint32_t OFF_V = OFF_K + STAGES * TILE;
+  static constexpr uint32_t OFF_BAR = OFF_V + STAGES * TILE;
+  static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
+  static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
+};
+
+// Bounded wait that ignores the abort flag: used on the way out, for work
+// that completes on its own (outstanding TMA loads and MMAs).
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > limit_ns) {
+      record_status(4);
+      return;
+    }
+  }
+}
+
+// Warp-uniform bounded wait: every lane waits, and the warp proceeds only if
+// all lanes succeeded (keeps the .sync.aligned tensor-memory instructions that
+// follow convergent even when one lane's wait gives up).
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const Watchdog& wd) {
+  const bool ok = mbar_wait(bar, parity, wd);
+  return __all_sync(0xffffffffu, ok);
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using C = FwdCfg<D>;
+  constexpr uint32_t IDESC_S = idesc_f16(BF16, kBM, kBN, false, false);  // S = Q·Kᵀ, both K-major
+  constexpr uint32_t IDESC_O = idesc_f16(BF16, kBM, D, false, true);     // O += P·V, V MN-major
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t s_base = smem_u32(smem);
+  const uint32_t sQ = s_base + C::OFF_Q;
+  const uint32_t sK = s_base + C::OFF_K;
+  const uint32_t sV = s_base + C::OFF_V;
+  const uint32_t bar0 = s_base + C::OFF_BAR;
+  auto bar = [&](int i) -> uint32_t { return bar0 + 8u * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  int* abort_flag = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- decode the work unit: heads in groups (K/V of a group stay in L2),
+  //      heaviest query blocks first inside a group (causal load balance)
+  const int BH = p.B * p.H;
+  const int nqb = p.num_qblocks;
+  const int G = p.heads_group;
+  const int unit = blockIdx.x;
+  const int group = unit / (G * nqb);
+  const int g_heads = min(G, BH - group * G);
+  const int r = unit - group * G * nqb;
+  const int qb = nqb - 1 - r / g_heads;
+  const int bh = group * G + r % g_heads;
+  const int b = bh / p.H;
+  const int h = bh - b * p.H;
+
+  int tok0, L;
+  if (p.cu_seqlens != nullptr) {
+    tok0 = __ldg(p.cu_seqlens + b);
+    const int end = __ldg(p.cu_seqlens + b + 1);
+    L = end - tok0;
+    if (tok0 < 0 || L < 0 || end > p.T || L > p.N) {
+      if (threadIdx.x == 0) record_status(1);
+      return;
+    }
+  } else {
+    tok0 = b * p.N;
+    L = p.N;
+  }
+  const int q0 = qb * 2 * kBM;
+  if (q0 >= L) return;  // uniform over the CTA: nothing allocated yet
+  const int nkv_all = (L + kBN - 1) / kBN;
+  int nkv[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int first_row = q0 + t * kBM;
+    if (first_row >= L) nkv[t] = 0;
+    else nkv[t] = p.causal ? min(nkv_all, (first_row + kBM - 1) / kBN + 1) : nkv_all;
+  }
+  const int n_iter = max(nkv[0], nkv[1]);
+
+  // ---- set-up: barriers, tensor memory
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 0) {
+    mbar_init(bar(C::B_Q), 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(bar(C::B_KFULL + s), 1);
+      mbar_init(bar(C::B_VFULL + s), 1);
+      mbar_init(bar(C::B_KVEMPTY + s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(C::B_SFULL + t), 1);
+      mbar_init(bar(C::B_PFULL + t), kBM);
+      mbar_init(bar(C::B_PVDONE + t), 1);
+    }
+    mbar_init(bar(C::B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8 && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Watchdog wd{abort_flag, p.timeout_ns};
+
+  if (warp == 8) {
+    // ================================================================ TMA producer
+    if (lane == 0) {
+      const uint64_t pol_q = l2_policy_evict_first();
+      const uint64_t pol_kv = l2_policy_evict_last();
+      const int nq = nkv[1] > 0 ? 2 : 1;
+      mbar_arrive_expect_tx(bar(C::B_Q), nq * C::TILE);
+      for (int t = 0; t < nq; ++t)
+        for (int c = 0; c < C::NCH; ++c)
+          tma_load_3d(sQ + t * C::TILE + c * (kBM * 128), &tm_q, bar(C::B_Q), c * 64, h,
+                      tok0 + q0 + t * kBM, pol_q);
+      int issued = 0;
+      for (int j = 0; j < n_iter; ++j) {
+        const int s = j % C::STAGES;
+        if (j >= C::STAGES && !mbar_wait(bar(C::B_KVEMPTY + s), ((j / C::STAGES) - 1) & 1, wd)) break;
+        mbar_arrive_expect_tx(bar(C::B_KFULL + s), C::TILE);
+        for (int c = 0; c < C::NCH; ++c)
+          tma_load_3d(sK + s * C::TILE + c * (kBN * 128), &tm_k, bar(C::B_KFULL + s), c * 64, h,
+                      tok0 + j * kBN, pol_kv);
+        mbar_arrive_expect_tx(bar(C::B_VFULL + s), C::TILE);
+        for (int c = 0; c < C::NCH; ++c)
+          tma_load_3d(sV + s * C::TILE + c * (kBN * 128), &tm_v, bar(C::B_VFULL + s), c * 64, h,
+                      tok0 + j * kBN, pol_kv);
+        issued = j + 1;
+      }
+      // Let every load this thread issued land before the CTA can exit.
+      drain_wait(bar(C::B_Q), 0, p.timeout_ns);
+      for (int j = max(0, issued - C::STAGES); j < issued; ++j) {
+        const int s = j % C::STAGES;
+        drain_wait(bar(C::B_KFULL + s), (j / C::STAGES) & 1, p.timeout_ns);
+        drain_wait(bar(C::B_VFULL + s), (j / C::STAGES) & 1, p.timeout_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
+      const uint32_t tO[2] = {tmem + 256u, tmem + 256u + (uint32_t)D};
+      auto issue_s = [&](int t, int s) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
+          const uint64_t ad = sdesc_sw128(sQ + t * C::TILE + off, 16, 1024);
+          const uint64_t bd = sdesc_sw128(sK + s * C::TILE + off, 16, 1024);
+          mma_ss(tS[t], ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, int s, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          const uint64_t bd = sdesc_sw128(sV + s * C::TILE + kk * 16 * 128, kBN * 128, 1024);
+          mma_ts(tO[t], tS[t] + kk * 8, bd, IDESC_O, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(bar(C::B_Q), 0, wd) && mbar_wait(bar(C::B_KFULL + 0), 0, wd);
+      if (ok) {
+        tc_fence_after();
+        for (int t = 0; t < 2; ++t)
+          if (nkv[t] > 0) {
+            issue_s(t, 0);
+            tc_commit(bar(C::B_SFULL + t));
+          }
+      }
+      for (int j = 0; ok && j < n_iter; ++j) {
+        const int s = j % C::STAGES;
+        const uint32_t ph = (j / C::STAGES) & 1;
+        bool v_ready = false;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (j >= nkv[t]) continue;
+          if (!mbar_wait(bar(C::B_PFULL + t), j & 1, wd)) { ok = false; break; }
+          if (!v_ready) {
+            if (!mbar_wait(bar(C::B_VFULL + s), ph, wd)) { ok = false; break; }
+            v_ready = true;
+          }
+          tc_fence_after();
+          issue_pv(t, s, j > 0);
+          tc_commit(bar(C::B_PVDONE + t));
+          if (j + 1 < nkv[t]) {
+            const int s1 = (j + 1) % C::STAGES;
+            if (!mbar_wait(bar(C::B_KFULL + s1), ((j + 1) / C::STAGES) & 1, wd)) { ok = false; break; }
+            tc_fence_after();
+            issue_s(t, s1);
+            tc_commit(bar(C::B_SFULL + t));
+          }
+        }
+        tc_commit(bar(C::B_KVEMPTY + s));
+      }
+      // every MMA issued so far must finish before tensor memory is released
+      tc_commit(bar(C::B_DRAIN));
+      drain_wait(bar(C::B_DRAIN), 0, p.timeout_ns);
+    }
+    __syncwarp();
+  } else {
+    // ================================================================ softmax warpgroups
+    const int t = warp >> 2;
+    const int quarter = warp & 3;
+    if (nkv[t] > 0) {
+      const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
+      const uint32_t tS = tmem + lane_off + 128u * t;
+      const uint32_t tO = tmem + lane_off + 256u + (uint32_t)(D * t);
+      const int row = q0 + t * kBM + 32 * quarter + lane;  // position in the sequence
+      const int key_limit = p.causal ? min(L, row + 1) : L;
+      const float c = p.scale_log2;
+      float m_ref = -INFINITY;  // running (possibly stale) max, scaled domain
+      float ell = 0.f;
+      bool ok = true;
+      for (int j = 0; j < nkv[t]; ++j) {
+        if (!warp_wait(bar(C::B_SFULL + t), j & 1, wd)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t sr[kBN];
+#pragma unroll
+        for (int q = 0; q < kBN / 32; ++q) tmem_ld32(tS + 32u * q, reinterpret_cast<uint32_t(&)[32]>(sr[32 * q]));
+        tmem_wait_ld();
+        float sv[kBN];
+#pragma unroll
+        for (int i = 0; i < kBN; ++i) sv[i] = __uint_as_float(sr[i]);
+        const int lim = key_limit - j * kBN;  // keys [lim, 128) of this tile are hidden from this row
+        if (lim < kBN) {
+#pragma unroll
+          for (int i = 0; i < kBN; ++i) sv[i] = (i < lim) ? sv[i] : -INFINITY;
+        }
+        float mx0 = sv[0], mx1 = sv[1];
+#pragma unroll
+        for (int i = 2; i < kBN; i += 2) {
+          mx0 = fmaxf(mx0, sv[i]);
+          mx1 = fmaxf(mx1, sv[i + 1]);
+        }
+        const float m_tile = fmaxf(mx0, mx1) * c;
+        // raise the reference max only when the tile max exceeds it by more than the threshold
+        const float m_new = (m_tile > m_ref + kRescaleThreshold) ? m_tile : m_ref;
+        const float alpha = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - m_new);
+        const bool rescale_o = (j > 0) && (m_new != m_ref);
+        if (__any_sync(0xffffffffu, rescale_o)) {
+          // O(t) must hold P·V(t, j-1) before it is rescaled
+          if (!warp_wait(bar(C::B_PVDONE + t), (j - 1) & 1, wd)) { ok = false; break; }
+          tc_fence_after();
+          const float f = rescale_o ? alpha : 1.f;
+#pragma unroll
+          for (int q = 0; q < D / 32; ++q) {
+            uint32_t r32[32];
+            tmem_ld32(tO + 32u * q, r32);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r32[i] = __float_as_uint(__uint_as_float(r32[i]) * f);
+            tmem_st32(tO + 32u * q, r32);
+          }
+        }
+        ell *= alpha;
+        m_ref = m_new;
+        // a row that has seen no visible key yet keeps m = -inf; its P is 0 either way
+        const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
+        float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float p0 = ex2(fmaf(sv[64 * q + 2 * i], c, neg_m));
+            const float p1 = ex2(fmaf(sv[64 * q + 2 * i + 1], c, neg_m));
+            rs0 += p0;
+            rs1 += p1;
+            pk[i] = pack2<BF16>(p0, p1);
+          }
+          tmem_st32(tS + 32u * q, pk);
+        }
+        ell += rs0 + rs1;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(C::B_PFULL + t));
+      }
+      // ---- epilogue: O / ℓ -> dtype, LSE
+      if (ok && warp_wait(bar(C::B_PVDONE + t), (nkv[t] - 1) & 1, wd)) {
+        tc_fence_after();
+        const bool valid = row < L;
+        const float inv = (ell > 0.f) ? 1.f / ell : 0.f;
+        const size_t obase = ((size_t)(tok0 + (valid ? row : 0)) * p.H + h) * D;
+        uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) + obase * 2;
+#pragma unroll
+        for (int q = 0; q < D / 32; ++q) {
+          uint32_t r32[32];
+          tmem_ld32(tO + 32u * q, r32);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack2<BF16>(__uint_as_float(r32[2 * i]) * inv, __uint_as_float(r32[2 * i + 1]) * inv);
+          if (valid) {
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              st_global_v4(orow + q * 64 + v4 * 16, pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+          }
+        }
+        if (valid) {
+          const float lse = (ell > 0.f && m_ref != -INFINITY) ? (m_ref + __log2f(ell)) * 0.69314718055994531f : -INFINITY;
+          p.lse[(size_t)(tok0 + row) * p.H + h] = lse;
+        }
+      }
+    }
+    __syncwarp();
+  }
+
+  // ---- tear-down
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D, bool BF16>
+static cudaError_t launch_fwd_t(const Problem& pb, const FwdArgs& a, cudaStream_t stream) {
+  using C = FwdCfg<D>;
+  static bool configured = false;  // per instantiation
+  auto kern = fa_fwd_kernel<D, BF16>;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  FwdParams p;
+  p.o = a.o;
+  p.lse = a.lse;
+  p.cu_seqlens = pb.cu_seqlens;
+  p.B = pb.B;
+  p.H = pb.H;
+  p.N = pb.N;
+  p.T = pb.T;
+  p.causal = pb.causal;
+  p.num_qblocks = (pb.N + 2 * kBM - 1) / (2 * kBM);
+  p.heads_group = 8;
+  p.scale_log2 = pb.scale * 1.4426950408889634f;
+  p.timeout_ns = pb.timeout_ns;
+  const long long units = (long long)pb.B * pb.H * p.num_qblocks;
+  kern<<<dim3((unsigned)units), dim3(kFwdThreads), C::SMEM_BYTES, stream>>>(a.tm_q, a.tm_k, a.tm_v, p);
+  return cudaPeekAtLastError();
+}
+
+cudaError_t launch_fwd(const Problem& pb, const FwdArgs& a, cudaStream_t stream) {
+  if (pb.d == 128) return pb.bf16 ? launch_fwd_t<128, true>(pb, a, stream) : launch_fwd_t<128, false>(pb, a, stream);
+  return pb.bf16 ? launch_fwd_t<64, true>(pb, a, stream) : launch_fwd_t<64, false>(pb, a, stream);
+}
+
+}  // namespace fa

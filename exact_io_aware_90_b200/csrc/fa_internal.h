@@ -1,0 +1,52 @@
+// fa_internal.h — declarations shared by the host-side entry points and the
+// kernel launchers of libfa_b200.so (not part of the public ABI).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace fa {
+
+// Work of one attention call, resolved on the host.
+struct Problem {
+  int B, H, N, d, T;
+  float scale;
+  int causal;
+  const int32_t* cu_seqlens;  // device pointer or nullptr
+  bool bf16;
+  uint64_t timeout_ns;
+};
+
+struct FwdArgs {
+  CUtensorMap tm_q, tm_k, tm_v;
+  void* o;
+  float* lse;
+};
+
+struct BwdArgs {
+  CUtensorMap tm_q, tm_k, tm_v, tm_do;
+  const void* q;
+  const void* k;
+  const float* lse;
+  const void* o;
+  const void* dO;
+  void* dq;
+  void* dk;
+  void* dv;
+  float* dq_acc;  // [T, H, d] fp32
+  float* delta;   // [T, H] fp32
+};
+
+// Encodes a [T, H, d] 16-bit tensor as a 3-D TMA map with 128-byte swizzle
+// and a box of 64 features × 1 head × `rows` tokens.  Returns false on failure.
+bool encode_tmap(CUtensorMap* map, const void* base, int T, int H, int d, bool bf16, int rows);
+
+cudaError_t launch_fwd(const Problem& pb, const FwdArgs& a, cudaStream_t stream);
+cudaError_t launch_bwd_pre(const Problem& pb, const BwdArgs& a, cudaStream_t stream);
+cudaError_t launch_bwd_main(const Problem& pb, const BwdArgs& a, cudaStream_t stream);
+cudaError_t launch_bwd_post(const Problem& pb, const BwdArgs& a, cudaStream_t stream);
+cudaError_t launch_watchdog_selftest(uint64_t timeout_ns, cudaStream_t stream);
+
+}  // namespace fa

@@ -1,0 +1,177 @@
+/*
+ * fa.h — C ABI of the B200 (sm_100a) exact attention library (libfa_b200.so).
+ *
+ * The library computes exact scaled-dot-product attention
+ *     O = softmax(Q Kᵀ · scale [+ causal mask]) V
+ * tile by tile with an online softmax, so the N×N score and probability
+ * matrices never reach device memory, and the training backward that
+ * recomputes the probabilities per tile from Q, K, V, O and the saved row
+ * log-sum-exp.
+ *
+ * Where each operation is defined (page title and section):
+ *   scores S = QKᵀ/√d ............ "FlashAttention 详解（零基础入门）" §2.3
+ *   safe softmax, row max ........ same page, §2.4
+ *   O = PV ....................... same page, §2.5
+ *   tiling, running m and ℓ ...... same page, §5.2, §5.4 and the §6.2 pseudocode
+ *   causal mask (key j ≤ query i)  "Flash Attention 优化", nanoGPT manual fallback
+ *   varlen packing ............... "FlashAttention 与算子融合", 工程实践 (varlen / packing)
+ *   backward recomputation ....... "FlashAttention 短片讲解稿", segment "第三招 · 反向重计算"
+ *   FLOP convention 4·B·h·s²·d ... "FlashAttention 与算子融合", 标准 Attention 浪费在哪
+ *
+ * Common conventions for every entry point
+ * ----------------------------------------
+ * Layout.  q, k, v, o, dO, dq, dk, dv are row-major [T, H, d] arrays (token,
+ *   head, feature) with d contiguous, a token stride of H·d elements, all in
+ *   one 16-bit dtype (FA_BF16 or FA_FP16).  lse is fp32 [T, H].  Self-attention
+ *   only: queries and keys come from the same T tokens.
+ * Sequences.  cu_seqlens == NULL: the T = B·N tokens form B sequences of N
+ *   tokens (total_tokens must equal B·N).  cu_seqlens != NULL: a DEVICE int32
+ *   array of B+1 non-decreasing prefix offsets with cu_seqlens[0] = 0 and
+ *   cu_seqlens[B] ≤ total_tokens; N is then an upper bound on every sequence
+ *   length (it sizes the launch grid).  A sequence of length 0 produces no rows.
+ *   Offsets are not read on the host; a kernel that finds them inconsistent
+ *   (decreasing, above total_tokens, a length above N) skips its work and
+ *   records FA_ERR_INVALID_ARG in the device status word.
+ * Causal.  causal = 1 hides key j from query i when j > i, with positions
+ *   counted from the start of each sequence.
+ * Numerics.  Products accumulate in fp32 on the tensor cores; the softmax runs
+ *   in fp32 with base-2 exponentials (scale·log2(e) folded in, an exact
+ *   reformulation); P is rounded to the input dtype before P·V; outputs are
+ *   rounded to nearest-even.  Results equal the mathematical definition up to
+ *   rounding, not bit for bit.
+ * lse.  Natural-log log-sum-exp of the scaled, masked scores of each row.
+ * Pointers.  Device pointers, 16-byte aligned, owned by the caller.  The
+ *   library never allocates, frees or synchronises (except
+ *   fa_check_device_status, which synchronises the given stream).
+ * Streams.  Every launch goes on `stream` (a cudaStream_t; 0 = legacy default).
+ * Sizes.  d ∈ {64, 128}; B, H, N ≥ 1; total_tokens ≥ 1; H·d·2 bytes and T·H·d
+ *   elements must fit the tensor-map limits (checked: FA_ERR_UNSUPPORTED).
+ * Errors.  Argument errors are returned synchronously before anything is
+ *   launched.  Launch failures map to FA_ERR_CUDA.  Every wait inside the
+ *   kernels is bounded by a watchdog; when one expires the kernel records
+ *   FA_ERR_TIMEOUT in the device status word and returns, leaving the context
+ *   usable.  Read that word with fa_check_device_status.
+ */
+#ifndef FA_B200_H
+#define FA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1,
+  FA_ERR_UNSUPPORTED = 2,
+  FA_ERR_CUDA = 3,
+  FA_ERR_TIMEOUT = 4
+} fa_status;
+
+typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype;
+
+/* Opaque stream handle: pass a cudaStream_t. */
+typedef void* fa_stream_t;
+
+/*
+ * Forward pass ("FlashAttention 详解" §6.2; the tiled loop with running m, ℓ).
+ *   q, k, v      in   [T, H, d] dtype
+ *   o            out  [T, H, d] dtype   O = softmax(QKᵀ·scale + mask) V
+ *   lse          out  [T, H] fp32       row log-sum-exp (natural log)
+ *   B, H, N, d   batch (number of sequences), heads, sequence length (max
+ *                length when cu_seqlens != NULL), head dimension (64 or 128)
+ *   scale        finite, > 0 (usually 1/√d)
+ *   causal       0 or 1
+ *   cu_seqlens   NULL or device int32 [B+1]
+ *   total_tokens T, the number of token rows in every [T, …] array
+ *   dtype        FA_BF16 or FA_FP16
+ * Rows of o/lse that belong to no sequence are left untouched.
+ * Returns FA_OK or an error code; see the conventions above.
+ */
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+           int B, int H, int N, int d, float scale, int causal,
+           const int32_t* cu_seqlens, int total_tokens, int dtype, fa_stream_t stream);
+
+/*
+ * Bytes of device workspace fa_bwd needs: an fp32 dQ accumulator [T, H, d]
+ * and the fp32 row terms D_i = Σ_c dO_ic·O_ic [T, H], each 256-byte aligned.
+ * Returns 0 for invalid sizes.
+ */
+size_t fa_bwd_workspace_bytes(int total_tokens, int H, int d);
+
+/*
+ * Backward pass: gradients of ⟨O, dO⟩ with respect to q, k, v, recomputing P
+ * tile by tile from q, k and lse ("FlashAttention 短片讲解稿", segment
+ * "第三招 · 反向重计算").  The gradient equations are the chain rule of the
+ * forward definition: dV = Pᵀ dO, dP = dO Vᵀ, D_i = Σ_c dO_ic O_ic,
+ * dS = P ∘ (dP − D), dQ = scale·dS K, dK = scale·dSᵀ Q.
+ *   q, k, v, o   in   [T, H, d] dtype (o from fa_fwd with the same arguments)
+ *   lse          in   [T, H] fp32 (from fa_fwd)
+ *   dO           in   [T, H, d] dtype
+ *   dq, dk, dv   out  [T, H, d] dtype; rows that belong to no sequence are left
+ *                untouched
+ *   workspace    device buffer of at least fa_bwd_workspace_bytes(T, H, d)
+ *                bytes, 256-byte aligned, owned by the caller; its contents on
+ *                entry do not matter and on return are unspecified
+ * Other arguments as for fa_fwd.  Launches three kernels on `stream`:
+ * fa_bwd_preprocess, fa_bwd_main and fa_bwd_postprocess, in that order.
+ */
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dO, void* dq, void* dk, void* dv,
+           int B, int H, int N, int d, float scale, int causal,
+           const int32_t* cu_seqlens, int total_tokens, int dtype,
+           void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/*
+ * The three stages of fa_bwd, callable one at a time (same arguments and
+ * rules as fa_bwd; each returns after launching its kernel).  Calling
+ * preprocess, main and postprocess in order on one stream is fa_bwd.
+ *   preprocess  D_i = Σ_c dO_ic·O_ic (fp32) and a zeroed fp32 dQ accumulator
+ *   main        per key tile: recompute Sᵀ and Pᵀ, accumulate dV, dK in tensor
+ *               memory and write them; add dQ partial sums into the accumulator
+ *   postprocess dq = scale · accumulator, rounded to the dtype
+ */
+int fa_bwd_preprocess(const void* o, const void* dO, int B, int H, int N, int d,
+                      const int32_t* cu_seqlens, int total_tokens, int dtype,
+                      void* workspace, size_t workspace_bytes, fa_stream_t stream);
+int fa_bwd_main(const void* q, const void* k, const void* v, const float* lse,
+                const void* dO, void* dk, void* dv,
+                int B, int H, int N, int d, float scale, int causal,
+                const int32_t* cu_seqlens, int total_tokens, int dtype,
+                void* workspace, size_t workspace_bytes, fa_stream_t stream);
+int fa_bwd_postprocess(void* dq, int B, int H, int N, int d, float scale,
+                       const int32_t* cu_seqlens, int total_tokens, int dtype,
+                       void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/*
+ * Synchronises `stream`, returns the device status word (FA_OK, or the first
+ * FA_ERR_TIMEOUT / FA_ERR_INVALID_ARG a kernel recorded since the last call)
+ * and clears it.  Returns FA_ERR_CUDA if the synchronisation itself failed.
+ */
+int fa_check_device_status(fa_stream_t stream);
+
+/* Sets the watchdog limit of every later launch, in nanoseconds of device
+ * time one wait may take (default 4e9).  Values below 1e6 are raised to 1e6. */
+void fa_set_watchdog_ns(uint64_t ns);
+
+/*
+ * Self-test of the watchdog: launches one block that waits on a barrier no
+ * thread ever completes, under a limit of `timeout_ns`.  The wait gives up,
+ * the kernel records FA_ERR_TIMEOUT and returns.  Returns the status read
+ * back by fa_check_device_status (FA_ERR_TIMEOUT when the watchdog works).
+ */
+int fa_watchdog_selftest(uint64_t timeout_ns, fa_stream_t stream);
+
+/* Human-readable name of a status code (static string). */
+const char* fa_status_string(int status);
+
+/* Library version string (static). */
+const char* fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H */

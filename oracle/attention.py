@@ -176,7 +176,9 @@ def attention_forward_rows(q, k, v, rows: Sequence[int], scale: float, causal: b
 
     Each requested row is computed from its own sequence's keys, so the full
     [L, L] score matrix is never formed: this is how long sequences are
-    checked on sampled rows.  Returns (O [len(rows), H, d], LSE [len(rows), H]).
+    checked on sampled rows.  Per (sequence, head) the sampled rows form a
+    small [rows, L] score block with the same steps as ``attention_forward``.
+    Returns (O [len(rows), H, d], LSE [len(rows), H]).
     """
     T, H, d = q.shape
     if B is None:
@@ -188,23 +190,27 @@ def attention_forward_rows(q, k, v, rows: Sequence[int], scale: float, causal: b
     rows = [int(r) for r in rows]
     O = np.zeros((len(rows), H, d), dtype=np.float64)
     LSE = np.full((len(rows), H), -np.inf, dtype=np.float64)
+    by_seq = {}
     for n, t in enumerate(rows):
         b = int(np.searchsorted(starts, t, side="right")) - 1
         start, L = segs[b]
-        if not (start <= t < start + L):
-            continue
-        i = t - start
-        hi = start + (i + 1 if causal else L)
-        Qr = _f64(q[t])                 # [H, d]
-        Kr = _f64(k[start:hi])          # [j, H, d]
-        Vr = _f64(v[start:hi])
+        if start <= t < start + L:
+            by_seq.setdefault(b, []).append((n, t - start))
+    for b, items in by_seq.items():
+        start, L = segs[b]
+        idx = np.array([n for n, _ in items])
+        pos = np.array([i for _, i in items])
+        hi = start + (int(pos.max()) + 1 if causal else L)  # keys any sampled row can see
         for h in range(H):
-            s = (Kr[:, h] @ Qr[h]) * scale
-            m = s.max()
-            e = np.exp(s - m)
-            ell = e.sum()
-            O[n, h] = (e / ell) @ Vr[:, h]
-            LSE[n, h] = m + math.log(ell)
+            Qr = _f64(q[start + pos, h] if not hasattr(q, "detach") else q[(start + pos).tolist(), h])
+            Kh = _f64(k[start:hi, h])
+            Vh = _f64(v[start:hi, h])
+            S = (Qr @ Kh.T) * scale
+            if causal:
+                S[np.arange(Kh.shape[0])[None, :] > pos[:, None]] = -np.inf
+            P, m, ell = _softmax_rows(S)
+            O[idx, h] = P @ Vh
+            LSE[idx, h] = m + np.log(ell)
     return O, LSE
 
 

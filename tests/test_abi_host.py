@@ -1,0 +1,115 @@
+"""Host-side checks of the C ABI: no GPU needed, no kernel launched.
+
+The library must load, export every function ``include/fa.h`` declares, and
+reject invalid arguments synchronously (before any CUDA call), so these run on
+a machine without a GPU.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(fa_[a-z0-9_]+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def fa():
+    from _lib import load_fa
+    return load_fa()
+
+
+def test_header_declares_the_entry_points():
+    names = _declared_functions()
+    for n in ["fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_bwd_preprocess", "fa_bwd_main",
+              "fa_bwd_postprocess", "fa_check_device_status", "fa_status_string", "fa_set_watchdog_ns",
+              "fa_watchdog_selftest", "fa_version"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(fa):
+    lib = ctypes.CDLL(fa.LIB_PATH)
+    for n in _declared_functions():
+        assert hasattr(lib, n), f"{n} declared in fa.h but not exported"
+
+
+def test_status_strings(fa):
+    assert fa.fa_status_string(0) == "FA_OK"
+    assert fa.fa_status_string(4) == "FA_ERR_TIMEOUT"
+    assert fa.fa_status_string(99) == "FA_UNKNOWN_STATUS"
+    assert "sm_100a" in fa.fa_version()
+
+
+def test_workspace_bytes(fa):
+    # fp32 dQ accumulator [T,H,d] + fp32 D [T,H], each rounded up to 256 bytes
+    def up(x):
+        return (x + 255) // 256 * 256
+    assert fa.fa_bwd_workspace_bytes(32768 * 1, 16, 128) == up(32768 * 16 * 128 * 4) + up(32768 * 16 * 4)
+    assert fa.fa_bwd_workspace_bytes(3, 1, 64) == up(3 * 64 * 4) + up(3 * 4)
+    assert fa.fa_bwd_workspace_bytes(0, 16, 128) == 0
+    assert fa.fa_bwd_workspace_bytes(16, 16, 96) == 0
+
+
+GOOD = dict(B=2, H=4, N=256, d=64, scale=0.125, causal=0, cu=None, T=512, dtype=0)
+P16 = 1 << 20  # a fake, 16-byte aligned "device" address: never dereferenced (validation fails first)
+
+
+def _fwd(fa, **kw):
+    a = dict(GOOD)
+    a.update(kw)
+    ptrs = a.pop("ptrs", [P16] * 5)
+    return fa.fa_fwd(*ptrs, a["B"], a["H"], a["N"], a["d"], a["scale"], a["causal"], a["cu"], a["T"], a["dtype"], None)
+
+
+@pytest.mark.parametrize("bad", [
+    dict(d=96), dict(d=0), dict(B=0), dict(H=0), dict(N=0), dict(T=0), dict(T=511),
+    dict(scale=float("nan")), dict(scale=float("inf")), dict(scale=0.0), dict(scale=-1.0),
+    dict(causal=2), dict(causal=-1), dict(dtype=2),
+    dict(ptrs=[0, P16, P16, P16, P16]), dict(ptrs=[P16, P16, P16, P16, 0]),
+    dict(ptrs=[P16 + 8, P16, P16, P16, P16]), dict(ptrs=[P16, P16, P16 + 2, P16, P16]),
+    dict(ptrs=[P16, P16, P16, P16, P16 + 2]), dict(cu=P16 + 2),
+])
+def test_forward_rejects_invalid_arguments(fa, bad):
+    assert _fwd(fa, **bad) == fa.FA_ERR_INVALID_ARG
+
+
+def test_backward_rejects_invalid_arguments(fa):
+    ws = fa.fa_bwd_workspace_bytes(512, 4, 64)
+    args = [P16] * 9 + [2, 4, 256, 64, 0.125, 0, None, 512, 0, P16, ws, None]
+    assert fa.fa_bwd(*args[:19], ws - 1, None) == fa.FA_ERR_INVALID_ARG          # workspace too small
+    bad_ws = list(args)
+    bad_ws[18] = P16 + 16                                                        # workspace not 256-byte aligned
+    assert fa.fa_bwd(*bad_ws) == fa.FA_ERR_INVALID_ARG
+    bad_d = list(args)
+    bad_d[12] = 80
+    assert fa.fa_bwd(*bad_d) == fa.FA_ERR_INVALID_ARG
+    null_dq = list(args)
+    null_dq[6] = 0
+    assert fa.fa_bwd(*null_dq) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_bwd_preprocess(P16, P16, 2, 4, 256, 64, None, 512, 0, P16, ws - 256, None) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_bwd_postprocess(P16, 2, 4, 256, 64, float("nan"), None, 512, 0, P16, ws, None) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_bwd_main(P16, P16, P16, P16, P16, P16, P16, 2, 4, 256, 64, 0.125, 3, None, 512, 0, P16, ws,
+                          None) == fa.FA_ERR_INVALID_ARG
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    """The binding has no fallback: without the shared library the import raises."""
+    import importlib.util
+    import shutil
+    pkg = os.path.join(ROOT, "exact_io_aware_90_b200")
+    dst = tmp_path / "exact_io_aware_90_b200"
+    os.makedirs(dst)
+    shutil.copy(os.path.join(pkg, "__init__.py"), dst / "__init__.py")  # no .so beside it
+    spec = importlib.util.spec_from_file_location("fa_copy_without_lib", dst / "__init__.py")
+    mod = importlib.util.module_from_spec(spec)
+    with pytest.raises(ImportError, match="missing"):
+        spec.loader.exec_module(mod)

@@ -1,0 +1,176 @@
+"""GPU parity of the forward kernel against the fp64 oracle (through the C ABI).
+
+Small shapes are compared element by element on every row; the full-size
+workloads are run in the launch configuration the benchmark times and checked
+on seeded samples of rows (all heads) that the oracle computes one by one.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from _gpu import LSE_TOL, O_TOL, covered_rows, f64, gpu_forward, max_abs, oracle_forward
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fa():
+    from _lib import load_fa
+    m = load_fa()
+    if not torch.cuda.is_available():
+        pytest.fail("a CUDA device is required for the gpu-marked tests")
+    m.fa_set_watchdog_ns(2_000_000_000)
+    return m
+
+
+def _check_fwd(fa, inp, o_tol=O_TOL, lse_tol=LSE_TOL):
+    o, lse = gpu_forward(fa, inp)
+    O_ref, L_ref = oracle_forward(inp)
+    rows = covered_rows(inp)
+    eo = max_abs(f64(o)[rows], O_ref[rows])
+    el = max_abs(f64(lse)[rows], L_ref[rows])
+    assert np.all(np.isfinite(f64(o)[rows])) and np.all(np.isfinite(f64(lse)[rows]))
+    assert eo <= o_tol, f"max|O-O_ref| = {eo}"
+    assert el <= lse_tol, f"max|LSE-LSE_ref| = {el}"
+    return eo, el
+
+
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+def test_hand_example(fa, dtype):
+    """The narration's example: weights [1,2,4,3] on values [10,20,30,40] give 29."""
+    inp = workloads.hand_example_inputs(dtype)
+    o, lse = gpu_forward(fa, inp)
+    O_ref, L_ref = oracle_forward(inp)  # on the rounded inputs
+    assert max_abs(f64(o), O_ref) <= O_TOL
+    assert max_abs(f64(lse), L_ref) <= LSE_TOL
+    # against the exact value: within the input rounding of ln c_j (fp16: 2^-11 relative) and one output ulp
+    tol = 0.03 if dtype == "fp16" else 0.25
+    assert np.all(np.abs(f64(o)[:, 0, 0] - 29.0) <= tol)
+    assert np.all(np.abs(f64(lse)[:, 0] - math.log(10.0)) <= 5e-3)
+
+
+def test_hand_example_causal(fa):
+    inp = workloads.hand_example_inputs("fp16")
+    inp.causal = True
+    o, lse = gpu_forward(fa, inp)
+    want = [10.0, 50.0 / 3.0, 170.0 / 7.0, 29.0]
+    assert np.all(np.abs(f64(o)[:, 0, 0] - want) <= 0.03)
+    O_ref, L_ref = oracle_forward(inp)
+    assert max_abs(f64(o), O_ref) <= O_TOL and max_abs(f64(lse), L_ref) <= LSE_TOL
+
+
+@pytest.mark.parametrize("N", [1, 3, 63, 64, 127, 128, 129, 255, 256, 257, 1000])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+def test_small_shapes(fa, N, d, causal, dtype):
+    inp = workloads.random_inputs(3, d, dtype, seed=7 * N + d + int(causal), B=2, N=N, causal=causal,
+                                  backward=False)
+    _check_fwd(fa, inp)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_ragged(fa, d, causal):
+    lens = [1, 127, 128, 129, 0, 300, 4096, 5]
+    inp = workloads.random_inputs(2, d, "bf16", seed=11 + d, seqlens=lens, causal=causal, backward=False)
+    _check_fwd(fa, inp)
+
+
+def test_varlen_leaves_uncovered_rows_untouched(fa):
+    """Rows past cu_seqlens[B] belong to no sequence: O and LSE there keep their contents."""
+    lens = [100, 37]
+    inp = workloads.random_inputs(2, 64, "bf16", seed=5, seqlens=lens, causal=True, backward=False)
+    pad = 50
+    dev = torch.device("cuda")
+    q = torch.cat([inp.q, torch.zeros(pad, 2, 64, dtype=inp.q.dtype)]).to(dev)
+    k = torch.cat([inp.k, torch.zeros(pad, 2, 64, dtype=inp.q.dtype)]).to(dev)
+    v = torch.cat([inp.v, torch.zeros(pad, 2, 64, dtype=inp.q.dtype)]).to(dev)
+    o = torch.full_like(q, 7.0)
+    lse = torch.full((q.shape[0], 2), 3.0, device=dev)
+    fa.attention_forward(q, k, v, causal=True, scale=inp.scale, cu_seqlens=inp.cu_seqlens.to(dev), max_seqlen=100,
+                         out=o, lse=lse)
+    assert fa.fa_check_device_status(torch.cuda.current_stream().cuda_stream) == fa.FA_OK
+    T = inp.T
+    assert torch.all(o[T:] == 7.0) and torch.all(lse[T:] == 3.0)
+    O_ref, L_ref = oracle_forward(inp)
+    assert max_abs(f64(o[:T]), O_ref) <= O_TOL and max_abs(f64(lse[:T]), L_ref) <= LSE_TOL
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_key_shift_invariance(fa, causal):
+    """Adding u to every key row leaves O unchanged and shifts LSE_i by scale·q_i·u."""
+    inp = workloads.random_inputs(2, 128, "bf16", seed=21, B=1, N=700, causal=causal, backward=False)
+    o1, l1 = gpu_forward(fa, inp)
+    u = torch.zeros(128)
+    u[::7] = 0.75  # exactly representable; k + u stays exact in bf16 for most entries, the oracle decides anyway
+    inp2 = workloads.AttnInputs(inp.q, (inp.k.float() + u).to(inp.k.dtype), inp.v, None, None, inp.seqlens, inp.B,
+                                inp.H, inp.N, inp.d, inp.scale, causal, inp.dtype)
+    o2, l2 = gpu_forward(fa, inp2)
+    O2_ref, L2_ref = oracle_forward(inp2)
+    assert max_abs(f64(o2), O2_ref) <= O_TOL and max_abs(f64(l2), L2_ref) <= LSE_TOL
+    assert max_abs(f64(o1), f64(o2)) <= 2 * O_TOL
+
+
+def test_large_scores_are_stable(fa):
+    """Scores of several hundred: the running max keeps every exponent finite."""
+    inp = workloads.random_inputs(1, 64, "bf16", seed=3, B=1, N=384, causal=False, backward=False)
+    inp.q = (inp.q.float() * 30).to(torch.bfloat16)
+    _check_fwd(fa, inp)
+
+
+def test_guard_bytes_untouched(fa):
+    """Outputs written only inside their bounds: canary regions around O and LSE survive."""
+    inp = workloads.random_inputs(2, 128, "bf16", seed=9, B=1, N=333, causal=True, backward=False)
+    dev = torch.device("cuda")
+    T, H, d = inp.q.shape
+    guard = 4096
+    obuf = torch.full((guard + T * H * d + guard,), -3.0, dtype=torch.bfloat16, device=dev)
+    lbuf = torch.full((guard + T * H + guard,), -5.0, dtype=torch.float32, device=dev)
+    o = obuf[guard:guard + T * H * d].view(T, H, d)
+    lse = lbuf[guard:guard + T * H].view(T, H)
+    gpu_forward(fa, inp, out=o, lse=lse)
+    assert torch.all(obuf[:guard] == -3.0) and torch.all(obuf[guard + T * H * d:] == -3.0)
+    assert torch.all(lbuf[:guard] == -5.0) and torch.all(lbuf[guard + T * H:] == -5.0)
+
+
+def test_workload_tiny(fa):
+    inp = workloads.make_workload("tiny_d64")
+    _check_fwd(fa, inp)
+
+
+def _sampled_rows(inp, n, seed):
+    rows = covered_rows(inp)
+    rng = np.random.default_rng(seed)
+    pick = rng.choice(rows, size=min(n, rows.size), replace=False)
+    # always include the first and last row of the first and last sequence
+    extra = [rows[0], rows[-1]]
+    return np.unique(np.concatenate([pick, extra]))
+
+
+@pytest.mark.parametrize("name", ["mha_n4k_d64", "causal_n8k_d128", "varlen_causal_d128", "long_n128k_d128"])
+def test_workload_forward_sampled_rows(fa, name):
+    inp = workloads.make_workload(name, backward=False)
+    o, lse = gpu_forward(fa, inp)
+    rows = _sampled_rows(inp, 256, seed=hash(name) % 1000)
+    cu = None if inp.cu_seqlens is None else inp.cu_seqlens.numpy()
+    O_ref, L_ref = oracle.attention_forward_rows(inp.q, inp.k, inp.v, rows, inp.scale, inp.causal, cu_seqlens=cu,
+                                                 B=inp.B, N=inp.N if cu is None else None)
+    oc, lc = f64(o[torch.as_tensor(rows)]), f64(lse[torch.as_tensor(rows)])
+    assert max_abs(oc, O_ref) <= O_TOL, max_abs(oc, O_ref)
+    assert max_abs(lc, L_ref) <= LSE_TOL, max_abs(lc, L_ref)
+    # every covered row is finite
+    allrows = covered_rows(inp)
+    assert torch.isfinite(lse[torch.as_tensor(allrows)]).all()
+
+
+def test_watchdog_gives_up_and_context_survives(fa):
+    stream = torch.cuda.current_stream().cuda_stream
+    assert fa.fa_watchdog_selftest(20_000_000, stream) == fa.FA_ERR_TIMEOUT
+    assert fa.fa_check_device_status(stream) == fa.FA_OK  # cleared
+    _check_fwd(fa, workloads.random_inputs(1, 64, "bf16", seed=1, B=1, N=129, backward=False))
