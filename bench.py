@@ -1,0 +1,489 @@
+"""Benchmark: exact attention forward + backward on B200, attention TFLOP/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+the forward (O, LSE) followed by the backward (D and the zeroed dQ
+accumulator, the main dK/dV/dQ kernel, the dQ conversion), all through the C
+ABI of libfa_b200.so on the caller's CUDA stream.  FLOPs follow the pages'
+convention: forward 4·B·H·N²·d (halved when causal), backward 2.5× forward.
+
+Timing: W warm-up steps, then K timed steps.  Before every step a 256 MiB
+buffer is written to flush the 126 MB L2; each step is bracketed by CUDA
+events on the stream the kernels run on (and each kernel by its own events,
+for the per-kernel roofline).  Under torchrun every rank runs its own copy
+of the workload (independent heads and sequences: weak scaling, no data-path
+collective); the time is the max over ranks.
+
+``--impl reference`` times the fp64 CPU oracle instead (rank 0 only), on a
+bounded sample of the same workload: the pages describe the method but ship
+no code, so the oracle is the reference arm.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention TFLOP/s (fwd, fwd+bwd) on 1 B200 and % of dense bf16 tensor peak"
+DEFAULT_WORKLOAD = "causal_n8k_d128"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    return dict(FALLBACK_PEAKS)
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "exact_io_aware_90_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on this kernel source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel, {}).get(workload)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """Samples the SM clock and the clock-event (throttle) reasons through NVML every
+    ~10 ms while the timed region runs (read-only; no setting is changed)."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, torch_device):
+        self.dev = torch_device
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self.handle = None
+
+    def _handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            import torch
+            p = torch.cuda.get_device_properties(self.dev)
+            bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+            return pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(self.dev.index or 0)
+
+    def start(self):
+        try:
+            import pynvml
+            self.nvml = pynvml
+            self.handle = self._handle()
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM))
+        except Exception:
+            self.handle = None
+            return
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+
+    def _run(self):
+        n = self.nvml
+        while not self._stop.is_set():
+            try:
+                clk = n.nvmlDeviceGetClockInfo(self.handle, n.NVML_CLOCK_SM)
+                rs = n.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                self.samples.append((float(clk), int(rs)))
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def stop(self):
+        if self.handle is None:
+            return None
+        self._stop.set()
+        self.thread.join(timeout=2)
+        if not self.samples:
+            return None
+        reasons = set()
+        for _, rs in self.samples:
+            for bit, name in self.REASONS.items():
+                if rs & bit:
+                    reasons.add(name)
+        return {"sm_mhz": float(np.median([c for c, _ in self.samples])), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(self.samples), "source": "NVML, 10 ms polling"}
+
+
+# ----------------------------------------------------------------------------- distributed plumbing
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        backend = "gloo" if args.impl == "reference" else "nccl"
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=300))
+        pg = dist
+    return world, rank, local, pg
+
+
+def max_over_ranks(x, pg, device=None):
+    if pg is None:
+        return x
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+
+def run_gpu(args, world, rank, local, pg):
+    import torch
+
+    import workloads
+    import exact_io_aware_90_b200 as fa
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    wname = args.workload
+    spec = workloads.WORKLOADS[wname]
+    inp_h = workloads.make_workload(wname, backward=spec["backward"])
+    # weak scaling: each rank gets its own seeded copy of the workload
+    if rank > 0:
+        inp_h = workloads.random_inputs(inp_h.H, inp_h.d, inp_h.dtype, spec["seed"] + 1000 * rank, B=inp_h.B,
+                                        N=inp_h.N, seqlens=inp_h.seqlens if inp_h.cu_seqlens is not None else None,
+                                        causal=inp_h.causal, backward=spec["backward"])
+    backward = spec["backward"]
+    B, H, N, d, T = inp_h.B, inp_h.H, inp_h.N, inp_h.d, inp_h.T
+    dt = fa.dtype_code(inp_h.q)
+    scale, causal = inp_h.scale, int(inp_h.causal)
+    flops_fwd = 4.0 * H * d * sum(float(L) * L for L in inp_h.seqlens) * (0.5 if causal else 1.0)
+    flops_bwd = 2.5 * flops_fwd if backward else 0.0
+
+    # device buffers
+    q, k, v = inp_h.q.to(dev), inp_h.k.to(dev), inp_h.v.to(dev)
+    do = inp_h.do.to(dev) if backward else None
+    cu = inp_h.cu_seqlens.to(dev) if inp_h.cu_seqlens is not None else None
+    cu_p = cu.data_ptr() if cu is not None else None
+    o = torch.empty_like(q)
+    lse = torch.empty((T, H), dtype=torch.float32, device=dev)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3)) if backward else (None, None, None)
+    ws_bytes = fa.fa_bwd_workspace_bytes(T, H, d)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if backward else None
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def check(st, where):
+        if st != fa.FA_OK:
+            raise fa.FAError(st, where)
+
+    def fwd():
+        check(fa.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, N, d, scale,
+                        causal, cu_p, T, dt, sp), "fa_fwd")
+
+    def bwd_pre():
+        check(fa.fa_bwd_preprocess(o.data_ptr(), do.data_ptr(), B, H, N, d, cu_p, T, dt, ws.data_ptr(), ws_bytes, sp),
+              "fa_bwd_preprocess")
+
+    def bwd_main():
+        check(fa.fa_bwd_main(q.data_ptr(), k.data_ptr(), v.data_ptr(), lse.data_ptr(), do.data_ptr(), dk.data_ptr(),
+                             dv.data_ptr(), B, H, N, d, scale, causal, cu_p, T, dt, ws.data_ptr(), ws_bytes, sp),
+              "fa_bwd_main")
+
+    def bwd_post():
+        check(fa.fa_bwd_postprocess(dq.data_ptr(), B, H, N, d, scale, cu_p, T, dt, ws.data_ptr(), ws_bytes, sp),
+              "fa_bwd_postprocess")
+
+    stages = [("fa_fwd_kernel", fwd)]
+    if backward:
+        stages += [("fa_bwd_pre_kernel", bwd_pre), ("fa_bwd_main_kernel", bwd_main),
+                   ("fa_bwd_post_kernel", bwd_post)]
+    flops_of = {"fa_fwd_kernel": flops_fwd, "fa_bwd_main_kernel": flops_bwd}
+
+    def one_step(record):
+        flush.fill_(1)  # outside the timed events
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
+        evs[0].record(stream)
+        for i, (_, fn) in enumerate(stages):
+            fn()
+            evs[i + 1].record(stream)
+        if record is not None:
+            record.append(evs)
+
+    for _ in range(args.warmup):
+        one_step(None)
+    torch.cuda.synchronize(dev)
+    st = fa.fa_check_device_status(sp)
+    if st != fa.FA_OK:
+        raise fa.FAError(st, "warm-up")
+
+    clocks = ClockSampler(dev)
+    if pg is not None:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    recs = []
+    for _ in range(args.steps):
+        one_step(recs)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    if pg is not None:
+        pg.barrier()
+    st = fa.fa_check_device_status(sp)
+    if st != fa.FA_OK:
+        raise fa.FAError(st, "timed steps")
+    step_ms = [r[0].elapsed_time(r[-1]) for r in recs]
+    per_kernel = {name: float(np.mean([r[i].elapsed_time(r[i + 1]) for r in recs]))
+                  for i, (name, _) in enumerate(stages)}
+    total_ms = max_over_ranks(float(np.sum(step_ms)), pg, dev)
+    ms_per_step = total_ms / args.steps
+    flops_step = flops_fwd + flops_bwd
+    value = world * flops_step / (ms_per_step * 1e-3) / 1e12
+
+    # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
+    pin = lambda t: None if t is None else t.pin_memory()
+    hq, hk, hv, hdo = pin(inp_h.q), pin(inp_h.k), pin(inp_h.v), pin(inp_h.do)
+    ho = torch.empty_like(hq).pin_memory()
+    hl = torch.empty((T, H), dtype=torch.float32).pin_memory()
+    hdq, hdk, hdv = ((torch.empty_like(hq).pin_memory() for _ in range(3)) if backward else (None, None, None))
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo) if t is not None)
+    d2h = sum(t.numel() * t.element_size() for t in (ho, hl, hdq, hdk, hdv) if t is not None)
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        if backward:
+            do.copy_(hdo, non_blocking=True)
+        fa.attention_forward(q, k, v, causal=bool(causal), scale=scale, cu_seqlens=cu,
+                             max_seqlen=N if cu is not None else None, batch=B, out=o, lse=lse, stream=sp)
+        if backward:
+            fa.attention_backward(q, k, v, o, lse, do, causal=bool(causal), scale=scale, cu_seqlens=cu,
+                                  max_seqlen=N if cu is not None else None, batch=B, dq=dq, dk=dk, dv=dv,
+                                  workspace=ws, stream=sp)
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+        if backward:
+            hdq.copy_(dq, non_blocking=True)
+            hdk.copy_(dk, non_blocking=True)
+            hdv.copy_(dv, non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, 5))
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(a.elapsed_time(b) / e2e_steps, pg, dev)
+    st = fa.fa_check_device_status(sp)
+    if st != fa.FA_OK:
+        raise fa.FAError(st, "e2e steps")
+
+    # ---- roofline of the dominant kernel
+    peaks = load_peaks()
+    dom = max(per_kernel, key=per_kernel.get)
+    dom_ms = per_kernel[dom]
+    if dom in flops_of:
+        achieved = flops_of[dom] / (dom_ms * 1e-3) / 1e12
+        roof = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 1), "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
+                "frac_of_sustained": round(achieved / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]), 4),
+                "peak_source": peaks["source"] + " (burst bf16; kernels timed one launch at a time)",
+                "traffic": load_traffic(dom, wname), "launch_ms": round(dom_ms, 4)}
+    else:
+        roof = {"kernel": dom, "bound": "hbm", "achieved": None, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": None, "traffic": load_traffic(dom, wname)}
+    kernels = {}
+    for name, ms in per_kernel.items():
+        e = {"ms": round(ms, 4)}
+        if name in flops_of:
+            e["tflops"] = round(flops_of[name] / (ms * 1e-3) / 1e12, 1)
+            e["frac_of_peak"] = round(e["tflops"] / peaks["bf16_tflops"], 4)
+        kernels[name] = e
+
+    out = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": inp_h.dtype,
+        "data": "synthetic: i.i.d. N(0,1) q, k, v, dO from a seeded CPU generator, rounded to the dtype",
+        "config": {"workload": wname, "B": B, "H": H, "N": N, "d": d, "causal": bool(causal),
+                   "varlen": inp_h.cu_seqlens is not None, "tokens": T, "step": "fwd+bwd" if backward else "fwd",
+                   "flops_per_step": flops_step, "l2": "flushed before every step (256 MiB write, outside the events)",
+                   "parallelism": f"replicas x{world} (independent workloads per GPU)"},
+        "fwd_tflops": round(flops_fwd / (per_kernel["fa_fwd_kernel"] * 1e-3) / 1e12, 1),
+        "fwd_frac_of_peak": round(flops_fwd / (per_kernel["fa_fwd_kernel"] * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
+        "pct_of_peak": round(100.0 * value / world / peaks["bf16_tflops"], 2),
+        "kernels": kernels,
+        "roofline": roof,
+        "e2e": {"value": round(world * flops_step / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": len(stages) * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(inp_h, budget_s=args.cpu_budget)
+    return out
+
+
+# ----------------------------------------------------------------------------- CPU oracle (baseline / reference arm)
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(n[0])
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_sample(inp, rows, head=0):
+    """fp64 oracle forward+backward on one head of the first sequence, query rows [L-rows, L).
+
+    Returns (seconds, flops credited by the same convention as the GPU arm)."""
+    import oracle
+    L = inp.seqlens[0]
+    lo = max(0, L - rows)
+    sl = slice(0, L)
+    t0 = time.perf_counter()
+    oracle.attention_fwd_bwd_rows(inp.q[sl], inp.k[sl], inp.v[sl],
+                                  inp.do[sl] if inp.do is not None else inp.q[sl], lo, L, inp.scale, inp.causal,
+                                  head=head)
+    dt = time.perf_counter() - t0
+    # visible (query, key) pairs of the sampled rows, times 4·d, times 3.5 for fwd+bwd
+    pairs = sum((i + 1) if inp.causal else L for i in range(lo, L))
+    f = 4.0 * inp.d * pairs * (3.5 if inp.do is not None else 1.0)
+    return dt, f
+
+
+def cpu_baseline(inp, budget_s=15.0):
+    """Whole heads of sequence 0 through the oracle until about `budget_s` seconds of CPU work."""
+    L = inp.seqlens[0]
+    tot_t, tot_f, heads = 0.0, 0.0, 0
+    for h in range(inp.H):
+        dt, f = oracle_sample(inp, L, head=h)
+        tot_t += dt
+        tot_f += f
+        heads += 1
+        if tot_t >= budget_s:
+            break
+    return {"value": round(tot_f / tot_t / 1e12, 6), "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"fp64 NumPy oracle, {'fwd+bwd' if inp.do is not None else 'fwd'} of {heads} whole head(s) of "
+                      f"sequence 0 ({L} query rows x all visible keys each), {tot_t:.2f} s"}
+
+
+def run_reference(args, rank):
+    import workloads
+    spec = workloads.WORKLOADS[args.workload]
+    inp = workloads.make_workload(args.workload, backward=spec["backward"])
+    L = inp.seqlens[0]
+    # size each step so the whole run stays within ~3 minutes
+    dt0, _ = oracle_sample(inp, 128)
+    per_step = 180.0 / max(1, args.steps + args.warmup)
+    rows = 128
+    while rows < L and dt0 * (2 * rows / 128) < per_step:
+        rows *= 2
+    rows = min(rows, L)
+    for _ in range(args.warmup):
+        oracle_sample(inp, rows)
+    times, flops = [], 0.0
+    for _ in range(args.steps):
+        dt, f = oracle_sample(inp, rows)
+        times.append(dt)
+        flops = f
+    ms = 1e3 * float(np.mean(times))
+    value = flops / (ms * 1e-3) / 1e12
+    sample = (f"fp64 NumPy oracle {'fwd+bwd' if inp.do is not None else 'fwd'} of query rows [{L - rows}, {L}) of "
+              f"one head of sequence 0 per step")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "B": inp.B, "H": inp.H, "N": inp.N, "d": inp.d,
+                   "causal": inp.causal, "sample_rows": rows},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
+    args.steps = max(1, args.steps)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, rank)), flush=True)
+        return 0
+    world, rank, local, pg = dist_setup(args)
+    try:
+        out = run_gpu(args, world, rank, local, pg)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if pg is not None:
+            pg.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -231,11 +231,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           mma_ss(tS[t], ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
         }
       };
-      auto issue_pv = [&](int t, int s, bool acc) {
+      auto issue_pv = [&](int t, int s, bool acc, uint32_t p_col) {
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
           const uint64_t bd = sdesc_sw128(sV + s * C::TILE + kk * 16 * 128, kBN * 128, 1024);
-          mma_ts(tO[t], tS[t] + kk * 8, bd, IDESC_O, (acc || kk > 0) ? 1u : 0u);
+          mma_ts(tO[t], tS[t] + p_col + kk * 8, bd, IDESC_O, (acc || kk > 0) ? 1u : 0u);
         }
       };
       bool ok = mbar_wait(bar(C::B_Q), 0, wd) && mbar_wait(bar(C::B_KFULL + 0), 0, wd);
@@ -259,7 +259,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             v_ready = true;
           }
           tc_fence_after();
-          issue_pv(t, s, j > 0);
+          issue_pv(t, s, j > 0, 0u);
+          if (nkv[t] == 1) issue_pv(t, s, true, 64u);  // lo part of a split P
           tc_commit(bar(C::B_PVDONE + t));
           if (j + 1 < nkv[t]) {
             const int s1 = (j + 1) % C::STAGES;
@@ -287,6 +288,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const int row = q0 + t * kBM + 32 * quarter + lane;  // position in the sequence
       const int key_limit = p.causal ? min(L, row + 1) : L;
       const float c = p.scale_log2;
+      // A tile whose rows see a single KV tile (the first 128 rows of a causal
+      // sequence, or a sequence of at most 128 tokens) averages few values, so
+      // the rounding of P to 16 bits would show in O: there P is carried as
+      // hi + lo parts and multiplied by V twice.
+      const bool split_p = (nkv[t] == 1);
       float m_ref = -INFINITY;  // running (possibly stale) max, scaled domain
       float ell = 0.f;
       bool ok = true;
@@ -336,18 +342,38 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // a row that has seen no visible key yet keeps m = -inf; its P is 0 either way
         const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
         float rs0 = 0.f, rs1 = 0.f;
+        if (!split_p) {
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          uint32_t pk[32];
+          for (int q = 0; q < 2; ++q) {
+            uint32_t pk[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float p0 = ex2(fmaf(sv[64 * q + 2 * i], c, neg_m));
-            const float p1 = ex2(fmaf(sv[64 * q + 2 * i + 1], c, neg_m));
-            rs0 += p0;
-            rs1 += p1;
-            pk[i] = pack2<BF16>(p0, p1);
+            for (int i = 0; i < 32; ++i) {
+              const float p0 = ex2(fmaf(sv[64 * q + 2 * i], c, neg_m));
+              const float p1 = ex2(fmaf(sv[64 * q + 2 * i + 1], c, neg_m));
+              rs0 += p0;
+              rs1 += p1;
+              pk[i] = pack2<BF16>(p0, p1);
+            }
+            tmem_st32(tS + 32u * q, pk);
           }
-          tmem_st32(tS + 32u * q, pk);
+        } else {
+          // P = hi + lo, both in the input dtype: hi in columns [0, 64), lo in [64, 128)
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            uint32_t hi[32], lo[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float p0 = ex2(fmaf(sv[64 * q + 2 * i], c, neg_m));
+              const float p1 = ex2(fmaf(sv[64 * q + 2 * i + 1], c, neg_m));
+              rs0 += p0;
+              rs1 += p1;
+              hi[i] = pack2<BF16>(p0, p1);
+              const float2 h = unpack2<BF16>(hi[i]);
+              lo[i] = pack2<BF16>(p0 - h.x, p1 - h.y);
+            }
+            tmem_st32(tS + 32u * q, hi);
+            tmem_st32(tS + 64u + 32u * q, lo);
+          }
         }
         ell += rs0 + rs1;
         tmem_wait_st();

@@ -46,7 +46,11 @@ def test_hand_example(fa, dtype):
     inp = workloads.hand_example_inputs(dtype)
     o, lse = gpu_forward(fa, inp)
     O_ref, L_ref = oracle_forward(inp)  # on the rounded inputs
-    assert max_abs(f64(o), O_ref) <= O_TOL
+    # O = 29 is beyond what a 16-bit output can hold to 1e-2 in bf16: its spacing at 29 is 0.125, so the
+    # bound there is half a bf16 spacing (the output's own rounding) plus the 1e-2 allowance.  In fp16
+    # (spacing 1/64) the plain 1e-2 bound applies.
+    o_tol = O_TOL if dtype == "fp16" else 0.0625 + O_TOL
+    assert max_abs(f64(o), O_ref) <= o_tol
     assert max_abs(f64(lse), L_ref) <= LSE_TOL
     # against the exact value: within the input rounding of ln c_j (fp16: 2^-11 relative) and one output ulp
     tol = 0.03 if dtype == "fp16" else 0.25
@@ -157,7 +161,7 @@ def _sampled_rows(inp, n, seed):
 def test_workload_forward_sampled_rows(fa, name):
     inp = workloads.make_workload(name, backward=False)
     o, lse = gpu_forward(fa, inp)
-    rows = _sampled_rows(inp, 256, seed=hash(name) % 1000)
+    rows = _sampled_rows(inp, 256, seed=sum(name.encode()))
     cu = None if inp.cu_seqlens is None else inp.cu_seqlens.numpy()
     O_ref, L_ref = oracle.attention_forward_rows(inp.q, inp.k, inp.v, rows, inp.scale, inp.causal, cu_seqlens=cu,
                                                  B=inp.B, N=inp.N if cu is None else None)
