@@ -9,7 +9,7 @@ GPU is present the calls raise.
 
 Raw ABI (same names and argument order as ``include/fa.h``; pointers are ints):
     fa_fwd, fa_bwd, fa_bwd_preprocess, fa_bwd_main, fa_bwd_postprocess,
-    fa_bwd_workspace_bytes, fa_check_device_status, fa_set_watchdog_ns,
+    fa_bwd_workspace_bytes, fa_bwd_noalloc, fa_check_device_status, fa_set_watchdog_ns,
     fa_watchdog_selftest, fa_status_string, fa_version
 Torch wrappers:
     attention_forward(q, k, v, ...)          -> (o, lse)
@@ -27,12 +27,13 @@ __all__ = [
     "FAError", "LIB_PATH", "lib", "FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA",
     "FA_ERR_TIMEOUT", "FA_BF16", "FA_FP16",
     "fa_fwd", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_postprocess", "fa_bwd_workspace_bytes",
-    "fa_check_device_status", "fa_set_watchdog_ns", "fa_watchdog_selftest", "fa_status_string", "fa_version",
+    "fa_bwd_noalloc", "FA_NOALLOC_SCRATCH_BYTES", "fa_check_device_status", "fa_set_watchdog_ns", "fa_watchdog_selftest", "fa_status_string", "fa_version",
     "attention_forward", "attention_backward", "dtype_code",
 ]
 
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = 0, 1, 2, 3, 4
 FA_BF16, FA_FP16 = 0, 1
+FA_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024  # include/fa.h
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa_b200.so")
 
@@ -57,6 +58,7 @@ def _load() -> ctypes.CDLL:
         "fa_bwd_preprocess": (I, [P, P, I, I, I, I, P, I, I, P, S, P]),
         "fa_bwd_main": (I, [P, P, P, P, P, P, P, I, I, I, I, F, I, P, I, I, P, S, P]),
         "fa_bwd_postprocess": (I, [P, I, I, I, I, F, P, I, I, P, S, P]),
+        "fa_bwd_noalloc": (I, [P, P, P, P, P, P, P, P, P, I, I, I, I, F, I, P, I, I, P]),
         "fa_check_device_status": (I, [P]),
         "fa_set_watchdog_ns": (None, [U64]),
         "fa_watchdog_selftest": (I, [U64, P]),
@@ -104,6 +106,15 @@ def fa_bwd_postprocess(dq, B, H, N, d, scale, cu_seqlens, total_tokens, dtype, w
                        stream) -> int:
     return lib.fa_bwd_postprocess(dq, B, H, N, d, scale, cu_seqlens, total_tokens, dtype, workspace,
                                   workspace_bytes, stream)
+
+
+def fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, cu_seqlens, total_tokens, dtype,
+                   stream) -> int:
+    """fa_bwd with its workspace in the library's static device scratch, for callers that cannot
+    allocate device memory; limited to problems needing at most FA_NOALLOC_SCRATCH_BYTES of
+    scratch (see include/fa.h)."""
+    return lib.fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, cu_seqlens, total_tokens,
+                              dtype, stream)
 
 
 def fa_check_device_status(stream) -> int:

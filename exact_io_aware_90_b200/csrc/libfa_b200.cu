@@ -3,3 +3,4 @@
 #include "fa_api.cu"
 #include "fa_fwd.cu"
 #include "fa_bwd.cu"
+#include "fa_noalloc.cu"

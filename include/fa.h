@@ -146,6 +146,37 @@ int fa_bwd_postprocess(void* dq, int B, int H, int N, int d, float scale,
                        void* workspace, size_t workspace_bytes, fa_stream_t stream);
 
 /*
+ * Size in bytes of the library's static device scratch used by fa_bwd_noalloc
+ * (32 MiB, held by every GPU that loads the library until the process exits).
+ */
+#define FA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+/*
+ * fa_bwd without a caller-provided workspace.  The method's pages have no
+ * counterpart: this exists for callers that cannot allocate device memory —
+ * a plugin whose host engine owns all of the GPU's memory and passes it only
+ * input and output buffers, or code that must not call cudaMalloc (it can
+ * synchronise the device and can fail under a fixed memory budget).
+ * Arguments and results as for fa_bwd, minus workspace and workspace_bytes;
+ * the dQ accumulator and D live in a static device array of
+ * FA_NOALLOC_SCRATCH_BYTES inside the library.  Nothing is allocated or freed.
+ *   - Returns FA_ERR_UNSUPPORTED, launching nothing, when the problem needs more
+ *     scratch than that: fa_bwd_workspace_bytes(total_tokens, H, d) must not
+ *     exceed FA_NOALLOC_SCRATCH_BYTES (about 63k token-heads at d = 128,
+ *     126k at d = 64).
+ *   - All calls on a device share the one array, which keeps the last call's
+ *     contents (the first kernel of every call zeroes what must start at zero).
+ *     Calls whose kernels overlap on the GPU — e.g. on two streams with no
+ *     ordering between them — race on the array and give wrong results.
+ *   - The first call on a device looks up the array's device address with that
+ *     device current; make that first call before any stream capture.
+ */
+int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                   const void* dO, void* dq, void* dk, void* dv,
+                   int B, int H, int N, int d, float scale, int causal,
+                   const int32_t* cu_seqlens, int total_tokens, int dtype, fa_stream_t stream);
+
+/*
  * Synchronises `stream`, returns the device status word (FA_OK, or the first
  * FA_ERR_TIMEOUT / FA_ERR_INVALID_ARG a kernel recorded since the last call)
  * and clears it.  Returns FA_ERR_CUDA if the synchronisation itself failed.
