@@ -122,10 +122,25 @@ def test_key_shift_invariance(fa, causal):
 
 
 def test_large_scores_are_stable(fa):
-    """Scores of several hundred: the running max keeps every exponent finite."""
+    """Scores of several hundred: the running max keeps every exponent finite.
+
+    With q scaled by 30 the softmax is dominated by a few keys per row, so this
+    input is outside the i.i.d. N(0,1) workloads the 1e-2 bound is stated for.
+    The bound here follows from the arithmetic: each weight of P is rounded to
+    bf16 (relative 2^-9) before P·V, which moves O by at most
+    2^-9 · Σ_j w_j |V_j − O| ≤ 2^-8 · max|V|, and the output itself is rounded
+    to bf16 (half a spacing at |O|)."""
     inp = workloads.random_inputs(1, 64, "bf16", seed=3, B=1, N=384, causal=False, backward=False)
     inp.q = (inp.q.float() * 30).to(torch.bfloat16)
-    _check_fwd(fa, inp)
+    o, lse = gpu_forward(fa, inp)
+    O_ref, L_ref = oracle_forward(inp)
+    go = f64(o)
+    assert np.all(np.isfinite(go)) and np.all(np.isfinite(f64(lse)))
+    vmax = float(np.abs(f64(inp.v)).max())
+    half_spacing = np.exp2(np.floor(np.log2(np.maximum(np.abs(O_ref), 1e-30))) - 8)
+    bound = 2.0 ** -8 * vmax + half_spacing + 1e-4
+    assert np.all(np.abs(go - O_ref) <= bound), float(np.max(np.abs(go - O_ref) - bound))
+    assert max_abs(f64(lse), L_ref) <= LSE_TOL
 
 
 def test_guard_bytes_untouched(fa):
