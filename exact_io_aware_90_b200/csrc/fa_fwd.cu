@@ -12,6 +12,11 @@
 //   warps 4-7  softmax of Q tile 1
 //   warp  8    TMA producer: Q0/Q1 once, then the K/V ring
 //   warp  9    tensor-memory allocator and single-thread tcgen05 MMA issuer
+//   warps 10-11 idle (they complete the third warpgroup, whose registers
+//              setmaxnreg hands to the softmax warpgroups: 224 / 224 / 56)
+// The exponentials of an unmasked tile are split between the MUFU (ex2) and
+// the FMA pipe (a polynomial, last kPolyCols columns): one ex2 per score
+// would keep the MUFU exactly as busy as the tensor core at d = 128.
 // Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+d),
 // O1 [256+d, 256+2d).  MMA issue order per KV tile j:
 //   P·V(0,j)  S(0,j+1)  P·V(1,j)  S(1,j+1)
@@ -42,7 +47,8 @@ struct FwdParams {
   uint64_t timeout_ns;
 };
 
-constexpr int kFwdThreads = 320;
+constexpr int kFwdThreads = 384;  // 3 warpgroups
+constexpr int kPolyCols = 32;     // columns [128 - kPolyCols, 128) of an unmasked tile use the FMA-pipe exp2
 constexpr int kBM = 128;  // query rows per tile
 constexpr int kBN = 128;  // keys per tile
 constexpr float kRescaleThreshold = 8.0f;
@@ -183,102 +189,105 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const Watchdog wd{abort_flag, p.timeout_ns};
 
-  if (warp == 8) {
-    // ================================================================ TMA producer
-    if (lane == 0) {
-      const uint64_t pol_q = l2_policy_evict_first();
-      const uint64_t pol_kv = l2_policy_evict_last();
-      const int nq = nkv[1] > 0 ? 2 : 1;
-      mbar_arrive_expect_tx(bar(C::B_Q), nq * C::TILE);
-      for (int t = 0; t < nq; ++t)
-        for (int c = 0; c < C::NCH; ++c)
-          tma_load_3d(sQ + t * C::TILE + c * (kBM * 128), &tm_q, bar(C::B_Q), c * 64, h,
-                      tok0 + q0 + t * kBM, pol_q);
-      int issued = 0;
-      for (int j = 0; j < n_iter; ++j) {
-        const int s = j % C::STAGES;
-        if (j >= C::STAGES && !mbar_wait(bar(C::B_KVEMPTY + s), ((j / C::STAGES) - 1) & 1, wd)) break;
-        mbar_arrive_expect_tx(bar(C::B_KFULL + s), C::TILE);
-        for (int c = 0; c < C::NCH; ++c)
-          tma_load_3d(sK + s * C::TILE + c * (kBN * 128), &tm_k, bar(C::B_KFULL + s), c * 64, h,
-                      tok0 + j * kBN, pol_kv);
-        mbar_arrive_expect_tx(bar(C::B_VFULL + s), C::TILE);
-        for (int c = 0; c < C::NCH; ++c)
-          tma_load_3d(sV + s * C::TILE + c * (kBN * 128), &tm_v, bar(C::B_VFULL + s), c * 64, h,
-                      tok0 + j * kBN, pol_kv);
-        issued = j + 1;
-      }
-      // Let every load this thread issued land before the CTA can exit.
-      drain_wait(bar(C::B_Q), 0, p.timeout_ns);
-      for (int j = max(0, issued - C::STAGES); j < issued; ++j) {
-        const int s = j % C::STAGES;
-        drain_wait(bar(C::B_KFULL + s), (j / C::STAGES) & 1, p.timeout_ns);
-        drain_wait(bar(C::B_VFULL + s), (j / C::STAGES) & 1, p.timeout_ns);
-      }
-    }
-    __syncwarp();
-  } else if (warp == 9) {
-    // ================================================================ MMA issuer
-    if (lane == 0) {
-      const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
-      const uint32_t tO[2] = {tmem + 256u, tmem + 256u + (uint32_t)D};
-      auto issue_s = [&](int t, int s) {
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
-          const uint64_t ad = sdesc_sw128(sQ + t * C::TILE + off, 16, 1024);
-          const uint64_t bd = sdesc_sw128(sK + s * C::TILE + off, 16, 1024);
-          mma_ss(tS[t], ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+  if (warp >= 8) {
+    regs_dec<56>();
+    if (warp == 8) {
+      // ================================================================ TMA producer
+      if (lane == 0) {
+        const uint64_t pol_q = l2_policy_evict_first();
+        const uint64_t pol_kv = l2_policy_evict_last();
+        const int nq = nkv[1] > 0 ? 2 : 1;
+        mbar_arrive_expect_tx(bar(C::B_Q), nq * C::TILE);
+        for (int t = 0; t < nq; ++t)
+          for (int c = 0; c < C::NCH; ++c)
+            tma_load_3d(sQ + t * C::TILE + c * (kBM * 128), &tm_q, bar(C::B_Q), c * 64, h,
+                        tok0 + q0 + t * kBM, pol_q);
+        int issued = 0;
+        for (int j = 0; j < n_iter; ++j) {
+          const int s = j % C::STAGES;
+          if (j >= C::STAGES && !mbar_wait(bar(C::B_KVEMPTY + s), ((j / C::STAGES) - 1) & 1, wd)) break;
+          mbar_arrive_expect_tx(bar(C::B_KFULL + s), C::TILE);
+          for (int c = 0; c < C::NCH; ++c)
+            tma_load_3d(sK + s * C::TILE + c * (kBN * 128), &tm_k, bar(C::B_KFULL + s), c * 64, h,
+                        tok0 + j * kBN, pol_kv);
+          mbar_arrive_expect_tx(bar(C::B_VFULL + s), C::TILE);
+          for (int c = 0; c < C::NCH; ++c)
+            tma_load_3d(sV + s * C::TILE + c * (kBN * 128), &tm_v, bar(C::B_VFULL + s), c * 64, h,
+                        tok0 + j * kBN, pol_kv);
+          issued = j + 1;
         }
-      };
-      auto issue_pv = [&](int t, int s, bool acc, uint32_t p_col) {
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t bd = sdesc_sw128(sV + s * C::TILE + kk * 16 * 128, kBN * 128, 1024);
-          mma_ts(tO[t], tS[t] + p_col + kk * 8, bd, IDESC_O, (acc || kk > 0) ? 1u : 0u);
+        // Let every load this thread issued land before the CTA can exit.
+        drain_wait(bar(C::B_Q), 0, p.timeout_ns);
+        for (int j = max(0, issued - C::STAGES); j < issued; ++j) {
+          const int s = j % C::STAGES;
+          drain_wait(bar(C::B_KFULL + s), (j / C::STAGES) & 1, p.timeout_ns);
+          drain_wait(bar(C::B_VFULL + s), (j / C::STAGES) & 1, p.timeout_ns);
         }
-      };
-      bool ok = mbar_wait(bar(C::B_Q), 0, wd) && mbar_wait(bar(C::B_KFULL + 0), 0, wd);
-      if (ok) {
-        tc_fence_after();
-        for (int t = 0; t < 2; ++t)
-          if (nkv[t] > 0) {
-            issue_s(t, 0);
-            tc_commit(bar(C::B_SFULL + t));
-          }
       }
-      for (int j = 0; ok && j < n_iter; ++j) {
-        const int s = j % C::STAGES;
-        const uint32_t ph = (j / C::STAGES) & 1;
-        bool v_ready = false;
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (j >= nkv[t]) continue;
-          if (!mbar_wait(bar(C::B_PFULL + t), j & 1, wd)) { ok = false; break; }
-          if (!v_ready) {
-            if (!mbar_wait(bar(C::B_VFULL + s), ph, wd)) { ok = false; break; }
-            v_ready = true;
+      } else if (warp == 9) {
+      // ================================================================ MMA issuer
+      if (lane == 0) {
+        const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
+        const uint32_t tO[2] = {tmem + 256u, tmem + 256u + (uint32_t)D};
+        auto issue_s = [&](int t, int s) {
+  #pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
+            const uint64_t ad = sdesc_sw128(sQ + t * C::TILE + off, 16, 1024);
+            const uint64_t bd = sdesc_sw128(sK + s * C::TILE + off, 16, 1024);
+            mma_ss(tS[t], ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
           }
+        };
+        auto issue_pv = [&](int t, int s, bool acc, uint32_t p_col) {
+  #pragma unroll
+          for (int kk = 0; kk < kBN / 16; ++kk) {
+            const uint64_t bd = sdesc_sw128(sV + s * C::TILE + kk * 16 * 128, kBN * 128, 1024);
+            mma_ts(tO[t], tS[t] + p_col + kk * 8, bd, IDESC_O, (acc || kk > 0) ? 1u : 0u);
+          }
+        };
+        bool ok = mbar_wait(bar(C::B_Q), 0, wd) && mbar_wait(bar(C::B_KFULL + 0), 0, wd);
+        if (ok) {
           tc_fence_after();
-          issue_pv(t, s, j > 0, 0u);
-          if (nkv[t] == 1) issue_pv(t, s, true, 64u);  // lo part of a split P
-          tc_commit(bar(C::B_PVDONE + t));
-          if (j + 1 < nkv[t]) {
-            const int s1 = (j + 1) % C::STAGES;
-            if (!mbar_wait(bar(C::B_KFULL + s1), ((j + 1) / C::STAGES) & 1, wd)) { ok = false; break; }
-            tc_fence_after();
-            issue_s(t, s1);
-            tc_commit(bar(C::B_SFULL + t));
-          }
+          for (int t = 0; t < 2; ++t)
+            if (nkv[t] > 0) {
+              issue_s(t, 0);
+              tc_commit(bar(C::B_SFULL + t));
+            }
         }
-        tc_commit(bar(C::B_KVEMPTY + s));
+        for (int j = 0; ok && j < n_iter; ++j) {
+          const int s = j % C::STAGES;
+          const uint32_t ph = (j / C::STAGES) & 1;
+          bool v_ready = false;
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (j >= nkv[t]) continue;
+            if (!mbar_wait(bar(C::B_PFULL + t), j & 1, wd)) { ok = false; break; }
+            if (!v_ready) {
+              if (!mbar_wait(bar(C::B_VFULL + s), ph, wd)) { ok = false; break; }
+              v_ready = true;
+            }
+            tc_fence_after();
+            issue_pv(t, s, j > 0, 0u);
+            if (nkv[t] == 1) issue_pv(t, s, true, 64u);  // lo part of a split P
+            tc_commit(bar(C::B_PVDONE + t));
+            if (j + 1 < nkv[t]) {
+              const int s1 = (j + 1) % C::STAGES;
+              if (!mbar_wait(bar(C::B_KFULL + s1), ((j + 1) / C::STAGES) & 1, wd)) { ok = false; break; }
+              tc_fence_after();
+              issue_s(t, s1);
+              tc_commit(bar(C::B_SFULL + t));
+            }
+          }
+          tc_commit(bar(C::B_KVEMPTY + s));
+        }
+        // every MMA issued so far must finish before tensor memory is released
+        tc_commit(bar(C::B_DRAIN));
+        drain_wait(bar(C::B_DRAIN), 0, p.timeout_ns);
       }
-      // every MMA issued so far must finish before tensor memory is released
-      tc_commit(bar(C::B_DRAIN));
-      drain_wait(bar(C::B_DRAIN), 0, p.timeout_ns);
     }
     __syncwarp();
   } else {
     // ================================================================ softmax warpgroups
+    regs_inc<224>();
     const int t = warp >> 2;
     const int quarter = warp & 3;
     if (nkv[t] > 0) {
@@ -307,17 +316,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
         for (int i = 0; i < kBN; ++i) sv[i] = __uint_as_float(sr[i]);
         const int lim = key_limit - j * kBN;  // keys [lim, 128) of this tile are hidden from this row
-        if (lim < kBN) {
+        const bool need_mask = __any_sync(0xffffffffu, lim < kBN);  // warp-uniform
+        if (need_mask) {
 #pragma unroll
           for (int i = 0; i < kBN; ++i) sv[i] = (i < lim) ? sv[i] : -INFINITY;
         }
-        float mx0 = sv[0], mx1 = sv[1];
+        float mx0 = sv[0], mx1 = sv[1], mx2 = sv[2], mx3 = sv[3];
 #pragma unroll
-        for (int i = 2; i < kBN; i += 2) {
-          mx0 = fmaxf(mx0, sv[i]);
-          mx1 = fmaxf(mx1, sv[i + 1]);
+        for (int i = 4; i < kBN; i += 8) {
+          mx0 = max3f(mx0, sv[i], sv[i + 1]);
+          mx1 = max3f(mx1, sv[i + 2], sv[i + 3]);
+          mx2 = max3f(mx2, sv[i + 4], sv[i + 5]);
+          mx3 = max3f(mx3, sv[i + 6], sv[i + 7]);
         }
-        const float m_tile = fmaxf(mx0, mx1) * c;
+        const float m_tile = max3f(mx0, mx1, fmaxf(mx2, mx3)) * c;
         // raise the reference max only when the tile max exceeds it by more than the threshold
         const float m_new = (m_tile > m_ref + kRescaleThreshold) ? m_tile : m_ref;
         const float alpha = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - m_new);
@@ -341,40 +353,62 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         m_ref = m_new;
         // a row that has seen no visible key yet keeps m = -inf; its P is 0 either way
         const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
-        float rs0 = 0.f, rs1 = 0.f;
-        if (!split_p) {
+        const float2 c2 = make_float2(c, c), nm2 = make_float2(neg_m, neg_m);
+        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        if (!need_mask && !split_p) {
+          // fast path: ex2 on the MUFU for the first columns, the polynomial on the FMA pipe for the rest
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
             uint32_t pk[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-              const float p0 = ex2(fmaf(sv[64 * q + 2 * i], c, neg_m));
-              const float p1 = ex2(fmaf(sv[64 * q + 2 * i + 1], c, neg_m));
-              rs0 += p0;
-              rs1 += p1;
-              pk[i] = pack2<BF16>(p0, p1);
+              const int idx = 64 * q + 2 * i;
+              const float2 x = __ffma2_rn(make_float2(sv[idx], sv[idx + 1]), c2, nm2);
+              float2 e;
+              if (idx >= kBN - kPolyCols) e = exp2_poly2(x);
+              else e = make_float2(ex2(x.x), ex2(x.y));
+              acc[i & 3] = __fadd2_rn(acc[i & 3], e);
+              pk[i] = pack2<BF16>(e.x, e.y);
+            }
+            tmem_st32(tS + 32u * q, pk);
+          }
+        } else if (!split_p) {
+          // masked tile: every exponential on the MUFU (ex2(-inf) = 0 exactly)
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            uint32_t pk[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int idx = 64 * q + 2 * i;
+              const float2 x = __ffma2_rn(make_float2(sv[idx], sv[idx + 1]), c2, nm2);
+              const float2 e = make_float2(ex2(x.x), ex2(x.y));
+              acc[i & 3] = __fadd2_rn(acc[i & 3], e);
+              pk[i] = pack2<BF16>(e.x, e.y);
             }
             tmem_st32(tS + 32u * q, pk);
           }
         } else {
           // P = hi + lo, both in the input dtype: hi in columns [0, 64), lo in [64, 128)
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            uint32_t hi[32], lo[32];
+          for (int q = 0; q < 4; ++q) {
+            uint32_t hi[16], lo[16];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float p0 = ex2(fmaf(sv[64 * q + 2 * i], c, neg_m));
-              const float p1 = ex2(fmaf(sv[64 * q + 2 * i + 1], c, neg_m));
-              rs0 += p0;
-              rs1 += p1;
-              hi[i] = pack2<BF16>(p0, p1);
-              const float2 h = unpack2<BF16>(hi[i]);
-              lo[i] = pack2<BF16>(p0 - h.x, p1 - h.y);
+            for (int i = 0; i < 16; ++i) {
+              const int idx = 32 * q + 2 * i;
+              const float2 x = __ffma2_rn(make_float2(sv[idx], sv[idx + 1]), c2, nm2);
+              const float2 e = make_float2(ex2(x.x), ex2(x.y));
+              acc[i & 3] = __fadd2_rn(acc[i & 3], e);
+              hi[i] = pack2<BF16>(e.x, e.y);
+              const float2 hf = unpack2<BF16>(hi[i]);
+              lo[i] = pack2<BF16>(e.x - hf.x, e.y - hf.y);
             }
-            tmem_st32(tS + 32u * q, hi);
-            tmem_st32(tS + 64u + 32u * q, lo);
+            tmem_st16(tS + 16u * q, hi);
+            tmem_st16(tS + 64u + 16u * q, lo);
           }
         }
+        const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
+        const float2 a = __fadd2_rn(a01, a23);
+        const float rs0 = a.x, rs1 = a.y;
         ell += rs0 + rs1;
         tmem_wait_st();
         tc_fence_before();

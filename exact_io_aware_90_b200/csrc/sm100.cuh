@@ -260,7 +260,45 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       : "memory");
 }
 
+// ---------------------------------------------------------------- register reconfiguration
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---------------------------------------------------------------- small math
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x on the FMA pipe, two lanes at a time, for x <= 8 (values below -126
+// are clamped; they come out below 2^-126, i.e. negligible next to the row's
+// largest weight, which is >= 2^-8).  x = j + f with j = round(x) taken from
+// the low bits of x + 1.5·2^23, f in [-1/2, 1/2]; 2^f by a degree-3
+// polynomial fitted here by a relative-error minimax (Remez) fit — maximum
+// relative error 7.5e-5, below the 2^-9 rounding P then gets in bf16 — and j
+// added straight into the exponent field.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  const float2 kMagic = make_float2(12582912.f, 12582912.f);
+  const float2 kNegMagic = make_float2(-12582912.f, -12582912.f);
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = __fadd2_rn(x, kMagic);
+  const float2 j = __fadd2_rn(t, kNegMagic);
+  const float2 f = __fadd2_rn(x, make_float2(-j.x, -j.y));
+  float2 p = __ffma2_rn(f, make_float2(0.0551716685f, 0.0551716685f), make_float2(0.2426111251f, 0.2426111251f));
+  p = __ffma2_rn(p, f, make_float2(0.6932609677f, 0.6932609677f));
+  p = __ffma2_rn(p, f, make_float2(0.9999280572f, 0.9999280572f));
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
