@@ -10,13 +10,13 @@
 // 128-row Q tiles that take turns on the tensor core:
 //   warps 0-3  softmax of Q tile 0 (one thread per row; TMEM lanes 0-127)
 //   warps 4-7  softmax of Q tile 1
-//   warp  8    TMA producer: Q0/Q1 once, then the K/V ring
-//   warp  9    tensor-memory allocator and single-thread tcgen05 MMA issuer
+//   warp  8    TMA producer: Q0/Q1 once, then the K and V rings
+//   warp  9    tensor-memory allocator and MMA issuer (one elected lane)
 //   warps 10-11 idle (they complete the third warpgroup, whose registers
-//              setmaxnreg hands to the softmax warpgroups: 224 / 224 / 56)
-// The exponentials of an unmasked tile are split between the MUFU (ex2) and
-// the FMA pipe (a polynomial, last kPolyCols columns): one ex2 per score
-// would keep the MUFU exactly as busy as the tensor core at d = 128.
+//              setmaxnreg hands to the softmax warpgroups: 208 / 208 / 88)
+// K_j and V_j have separate empty barriers: K_j's stage is handed back to
+// the producer as soon as both S(·, j) products are done, so the next K tile
+// streams in while P·V(·, j) still reads V_j.
 // Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+d),
 // O1 [256+d, 256+2d).  MMA issue order per KV tile j:
 //   P·V(0,j)  S(0,j+1)  P·V(1,j)  S(1,j+1)
@@ -48,7 +48,6 @@ struct FwdParams {
 };
 
 constexpr int kFwdThreads = 384;  // 3 warpgroups
-constexpr int kPolyCols = 32;     // columns [128 - kPolyCols, 128) of an unmasked tile use the FMA-pipe exp2
 constexpr int kBM = 128;  // query rows per tile
 constexpr int kBN = 128;  // keys per tile
 constexpr float kRescaleThreshold = 8.0f;
@@ -57,23 +56,26 @@ template <int D>
 struct FwdCfg {
   static constexpr int NCH = D / 64;                   // 128-byte feature chunks per row
   static constexpr uint32_t TILE = kBM * D * 2;        // bytes of a 128-row tile
-  static constexpr int STAGES = (D == 128) ? 2 : 4;    // K/V ring depth
+  static constexpr int KSTAGES = (D == 128) ? 3 : 5;   // K ring depth
+  static constexpr int VSTAGES = (D == 128) ? 2 : 4;   // V ring depth
   // barrier indices
   static constexpr int B_Q = 0;
   static constexpr int B_KFULL = 1;
-  static constexpr int B_VFULL = B_KFULL + STAGES;
-  static constexpr int B_KVEMPTY = B_VFULL + STAGES;
-  static constexpr int B_SFULL = B_KVEMPTY + STAGES;
+  static constexpr int B_KEMPTY = B_KFULL + KSTAGES;
+  static constexpr int B_VFULL = B_KEMPTY + KSTAGES;
+  static constexpr int B_VEMPTY = B_VFULL + VSTAGES;
+  static constexpr int B_SFULL = B_VEMPTY + VSTAGES;
   static constexpr int B_PFULL = B_SFULL + 2;
   static constexpr int B_PVDONE = B_PFULL + 2;
   static constexpr int B_DRAIN = B_PVDONE + 2;
   static constexpr int NBARS = B_DRAIN + 1;
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_K = 2 * TILE;
-  static constexpr uint32_t OFF_V = OFF_K + STAGES * TILE;
-  static constexpr uint32_t OFF_BAR = OFF_V + STAGES * TILE;
+  static constexpr uint32_t OFF_V = OFF_K + KSTAGES * TILE;
+  static constexpr uint32_t OFF_BAR = OFF_V + VSTAGES * TILE;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
   static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
 // Bounded wait that ignores the abort flag: used on the way out, for work
@@ -94,6 +96,27 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const Watchdog& wd) {
   const bool ok = mbar_wait(bar, parity, wd);
   return __all_sync(0xffffffffu, ok);
+}
+
+// S = Q·Kᵀ for one 128 × 128 tile: D/16 MMAs of K = 16 along the head dimension.
+// Q and K are K-major with 128-byte rows; a 16-element step is +32 bytes inside a
+// swizzle atom, a 64-element step the next 16 KB atom column.
+template <int D, uint32_t IDESC>
+__device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint64_t dq, uint64_t dk) {
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = ((kk >> 2) * (kBM * 128) + (kk & 3) * 32) >> 4;
+    mma_ss(s_tmem, dq + off, dk + off, IDESC, kk > 0 ? 1u : 0u);
+  }
+}
+
+// O (+)= P·V for one tile: 8 MMAs of K = 16 keys; P is read from tensor memory
+// (8 columns of packed 16-bit values per step), V is MN-major (+2 KB per 16 keys).
+template <uint32_t IDESC>
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint64_t dv, uint32_t acc) {
+#pragma unroll
+  for (int kk = 0; kk < kBN / 16; ++kk)
+    mma_ts(o_tmem, p_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), IDESC, kk > 0 ? 1u : acc);
 }
 
 template <int D, bool BF16>
@@ -164,10 +187,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   }
   if (threadIdx.x == 0) {
     mbar_init(bar(C::B_Q), 1);
-    for (int s = 0; s < C::STAGES; ++s) {
+    for (int s = 0; s < C::KSTAGES; ++s) {
       mbar_init(bar(C::B_KFULL + s), 1);
+      mbar_init(bar(C::B_KEMPTY + s), 1);
+    }
+    for (int s = 0; s < C::VSTAGES; ++s) {
       mbar_init(bar(C::B_VFULL + s), 1);
-      mbar_init(bar(C::B_KVEMPTY + s), 1);
+      mbar_init(bar(C::B_VEMPTY + s), 1);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar(C::B_SFULL + t), 1);
@@ -190,122 +216,153 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const Watchdog wd{abort_flag, p.timeout_ns};
 
   if (warp >= 8) {
-    regs_dec<56>();
+    regs_dec<88>();
+    // The producer and MMA warps run their loops with all 32 lanes (warp-uniform state the
+    // compiler can keep in uniform registers); one elected lane issues each TMA copy, MMA and
+    // commit.  elect.sync picks the lowest active lane, so every MMA and every commit that
+    // tracks it come from the same thread.
     if (warp == 8) {
       // ================================================================ TMA producer
-      if (lane == 0) {
-        const uint64_t pol_q = l2_policy_evict_first();
-        const uint64_t pol_kv = l2_policy_evict_last();
-        const int nq = nkv[1] > 0 ? 2 : 1;
+      const uint64_t pol_q = l2_policy_evict_first();
+      const uint64_t pol_kv = l2_policy_evict_last();
+      const int nq = nkv[1] > 0 ? 2 : 1;
+      if (elect_one()) {
         mbar_arrive_expect_tx(bar(C::B_Q), nq * C::TILE);
         for (int t = 0; t < nq; ++t)
           for (int c = 0; c < C::NCH; ++c)
-            tma_load_3d(sQ + t * C::TILE + c * (kBM * 128), &tm_q, bar(C::B_Q), c * 64, h,
-                        tok0 + q0 + t * kBM, pol_q);
-        int issued = 0;
-        for (int j = 0; j < n_iter; ++j) {
-          const int s = j % C::STAGES;
-          if (j >= C::STAGES && !mbar_wait(bar(C::B_KVEMPTY + s), ((j / C::STAGES) - 1) & 1, wd)) break;
-          mbar_arrive_expect_tx(bar(C::B_KFULL + s), C::TILE);
-          for (int c = 0; c < C::NCH; ++c)
-            tma_load_3d(sK + s * C::TILE + c * (kBN * 128), &tm_k, bar(C::B_KFULL + s), c * 64, h,
-                        tok0 + j * kBN, pol_kv);
-          mbar_arrive_expect_tx(bar(C::B_VFULL + s), C::TILE);
-          for (int c = 0; c < C::NCH; ++c)
-            tma_load_3d(sV + s * C::TILE + c * (kBN * 128), &tm_v, bar(C::B_VFULL + s), c * 64, h,
-                        tok0 + j * kBN, pol_kv);
-          issued = j + 1;
-        }
-        // Let every load this thread issued land before the CTA can exit.
-        drain_wait(bar(C::B_Q), 0, p.timeout_ns);
-        for (int j = max(0, issued - C::STAGES); j < issued; ++j) {
-          const int s = j % C::STAGES;
-          drain_wait(bar(C::B_KFULL + s), (j / C::STAGES) & 1, p.timeout_ns);
-          drain_wait(bar(C::B_VFULL + s), (j / C::STAGES) & 1, p.timeout_ns);
-        }
+            tma_load_3d(sQ + t * C::TILE + c * (kBM * 128), &tm_q, bar(C::B_Q), c * 64, h, tok0 + q0 + t * kBM,
+                        pol_q);
       }
-      } else if (warp == 9) {
+      __syncwarp();
+      int issued = 0;
+      for (int j = 0; j < n_iter; ++j) {
+        const int sk = j % C::KSTAGES, sv = j % C::VSTAGES;
+        if (j >= C::KSTAGES && !warp_wait(bar(C::B_KEMPTY + sk), ((j / C::KSTAGES) - 1) & 1, wd)) break;
+        if (elect_one()) {
+          mbar_arrive_expect_tx(bar(C::B_KFULL + sk), C::TILE);
+          for (int c = 0; c < C::NCH; ++c)
+            tma_load_3d(sK + sk * C::TILE + c * (kBN * 128), &tm_k, bar(C::B_KFULL + sk), c * 64, h, tok0 + j * kBN,
+                        pol_kv);
+        }
+        __syncwarp();
+        if (j >= C::VSTAGES && !warp_wait(bar(C::B_VEMPTY + sv), ((j / C::VSTAGES) - 1) & 1, wd)) {
+          issued = -(j + 1);  // K_j issued, V_j not
+          break;
+        }
+        if (elect_one()) {
+          mbar_arrive_expect_tx(bar(C::B_VFULL + sv), C::TILE);
+          for (int c = 0; c < C::NCH; ++c)
+            tma_load_3d(sV + sv * C::TILE + c * (kBN * 128), &tm_v, bar(C::B_VFULL + sv), c * 64, h, tok0 + j * kBN,
+                        pol_kv);
+        }
+        __syncwarp();
+        issued = j + 1;
+      }
+      // Let every load this warp issued land before the CTA can exit.
+      if (elect_one()) {
+        const int k_issued = issued >= 0 ? issued : -issued;
+        const int v_issued = issued >= 0 ? issued : -issued - 1;
+        drain_wait(bar(C::B_Q), 0, p.timeout_ns);
+        for (int j = max(0, k_issued - C::KSTAGES); j < k_issued; ++j)
+          drain_wait(bar(C::B_KFULL + j % C::KSTAGES), (j / C::KSTAGES) & 1, p.timeout_ns);
+        for (int j = max(0, v_issued - C::VSTAGES); j < v_issued; ++j)
+          drain_wait(bar(C::B_VFULL + j % C::VSTAGES), (j / C::VSTAGES) & 1, p.timeout_ns);
+      }
+      __syncwarp();
+    } else if (warp == 9) {
       // ================================================================ MMA issuer
-      if (lane == 0) {
-        const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
-        const uint32_t tO[2] = {tmem + 256u, tmem + 256u + (uint32_t)D};
-        auto issue_s = [&](int t, int s) {
-  #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * (kBM * 128) + (kk & 3) * 32;
-            const uint64_t ad = sdesc_sw128(sQ + t * C::TILE + off, 16, 1024);
-            const uint64_t bd = sdesc_sw128(sK + s * C::TILE + off, 16, 1024);
-            mma_ss(tS[t], ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+      // Descriptors are computed once; per instruction only a constant start-address offset
+      // (in 16-byte units, no carry out of the 14-bit field: shared addresses stay below 228 KB).
+      const uint64_t dq_base = sdesc_sw128(sQ, 16, 1024);
+      const uint64_t dk_base = sdesc_sw128(sK, 16, 1024);
+      const uint64_t dv_base = sdesc_sw128(sV, kBN * 128, 1024);
+      bool ok = warp_wait(bar(C::B_Q), 0, wd) && warp_wait(bar(C::B_KFULL + 0), 0, wd);
+      if (ok) {
+        tc_fence_after();
+        if (elect_one()) {
+          if (nkv[0] > 0) {
+            issue_qk<D, IDESC_S>(tmem + 0u, dq_base, dk_base);
+            tc_commit(bar(C::B_SFULL + 0));
           }
-        };
-        auto issue_pv = [&](int t, int s, bool acc, uint32_t p_col) {
-  #pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk) {
-            const uint64_t bd = sdesc_sw128(sV + s * C::TILE + kk * 16 * 128, kBN * 128, 1024);
-            mma_ts(tO[t], tS[t] + p_col + kk * 8, bd, IDESC_O, (acc || kk > 0) ? 1u : 0u);
+          if (nkv[1] > 0) {
+            issue_qk<D, IDESC_S>(tmem + 128u, dq_base + (C::TILE >> 4), dk_base);
+            tc_commit(bar(C::B_SFULL + 1));
           }
-        };
-        bool ok = mbar_wait(bar(C::B_Q), 0, wd) && mbar_wait(bar(C::B_KFULL + 0), 0, wd);
-        if (ok) {
+          tc_commit(bar(C::B_KEMPTY + 0));  // K_0 is read by no later MMA
+        }
+        __syncwarp();
+      }
+      for (int j = 0; ok && j < n_iter; ++j) {
+        const int s = j % C::VSTAGES;                  // V_j
+        const uint32_t ph = (j / C::VSTAGES) & 1;
+        const uint64_t dv_s = dv_base + ((s * C::TILE) >> 4);
+        const int s1 = (j + 1) % C::KSTAGES;           // K_{j+1}
+        const uint64_t dk_s1 = dk_base + ((s1 * C::TILE) >> 4);
+        bool v_ready = false;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (j >= nkv[t]) continue;
+          const uint32_t s_tmem = tmem + 128u * t;
+          const uint32_t o_tmem = tmem + 256u + (uint32_t)D * t;
+          if (!warp_wait(bar(C::B_PFULL + t), j & 1, wd)) { ok = false; break; }
+          if (!v_ready) {
+            if (!warp_wait(bar(C::B_VFULL + s), ph, wd)) { ok = false; break; }
+            v_ready = true;
+          }
           tc_fence_after();
-          for (int t = 0; t < 2; ++t)
-            if (nkv[t] > 0) {
-              issue_s(t, 0);
-              tc_commit(bar(C::B_SFULL + t));
-            }
-        }
-        for (int j = 0; ok && j < n_iter; ++j) {
-          const int s = j % C::STAGES;
-          const uint32_t ph = (j / C::STAGES) & 1;
-          bool v_ready = false;
-          for (int t = 0; t < 2 && ok; ++t) {
-            if (j >= nkv[t]) continue;
-            if (!mbar_wait(bar(C::B_PFULL + t), j & 1, wd)) { ok = false; break; }
-            if (!v_ready) {
-              if (!mbar_wait(bar(C::B_VFULL + s), ph, wd)) { ok = false; break; }
-              v_ready = true;
-            }
-            tc_fence_after();
-            issue_pv(t, s, j > 0, 0u);
-            if (nkv[t] == 1) issue_pv(t, s, true, 64u);  // lo part of a split P
+          if (elect_one()) {
+            issue_pv<IDESC_O>(o_tmem, s_tmem, dv_s, j > 0 ? 1u : 0u);
+            if (nkv[t] == 1) issue_pv<IDESC_O>(o_tmem, s_tmem + 64u, dv_s, 1u);  // lo part of a split P
             tc_commit(bar(C::B_PVDONE + t));
-            if (j + 1 < nkv[t]) {
-              const int s1 = (j + 1) % C::STAGES;
-              if (!mbar_wait(bar(C::B_KFULL + s1), ((j + 1) / C::STAGES) & 1, wd)) { ok = false; break; }
-              tc_fence_after();
-              issue_s(t, s1);
+          }
+          __syncwarp();
+          if (j + 1 < nkv[t]) {
+            if (!warp_wait(bar(C::B_KFULL + s1), ((j + 1) / C::KSTAGES) & 1, wd)) { ok = false; break; }
+            tc_fence_after();
+            if (elect_one()) {
+              issue_qk<D, IDESC_S>(s_tmem, dq_base + ((t * C::TILE) >> 4), dk_s1);
               tc_commit(bar(C::B_SFULL + t));
             }
+            __syncwarp();
           }
-          tc_commit(bar(C::B_KVEMPTY + s));
         }
-        // every MMA issued so far must finish before tensor memory is released
+        if (elect_one()) {
+          tc_commit(bar(C::B_VEMPTY + s));                     // V_j: both P·V(·, j) issued
+          if (j + 1 < n_iter) tc_commit(bar(C::B_KEMPTY + s1));  // K_{j+1}: both S(·, j+1) issued
+        }
+        __syncwarp();
+      }
+      // every MMA issued so far must finish before tensor memory is released
+      if (elect_one()) {
         tc_commit(bar(C::B_DRAIN));
         drain_wait(bar(C::B_DRAIN), 0, p.timeout_ns);
       }
+      __syncwarp();
     }
     __syncwarp();
   } else {
     // ================================================================ softmax warpgroups
-    regs_inc<224>();
+    regs_inc<208>();
     const int t = warp >> 2;
     const int quarter = warp & 3;
-    if (nkv[t] > 0) {
+    const int my_nkv = (t == 0) ? nkv[0] : nkv[1];
+    if (my_nkv > 0) {
       const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
       const uint32_t tS = tmem + lane_off + 128u * t;
       const uint32_t tO = tmem + lane_off + 256u + (uint32_t)(D * t);
       const int row = q0 + t * kBM + 32 * quarter + lane;  // position in the sequence
       const int key_limit = p.causal ? min(L, row + 1) : L;
       const float c = p.scale_log2;
+      const float2 c2 = make_float2(c, c);
       // A tile whose rows see a single KV tile (the first 128 rows of a causal
       // sequence, or a sequence of at most 128 tokens) averages few values, so
       // the rounding of P to 16 bits would show in O: there P is carried as
       // hi + lo parts and multiplied by V twice.
-      const bool split_p = (nkv[t] == 1);
+      const bool split_p = (my_nkv == 1);
       float m_ref = -INFINITY;  // running (possibly stale) max, scaled domain
       float ell = 0.f;
       bool ok = true;
-      for (int j = 0; j < nkv[t]; ++j) {
+      for (int j = 0; j < my_nkv; ++j) {
         if (!warp_wait(bar(C::B_SFULL + t), j & 1, wd)) { ok = false; break; }
         tc_fence_after();
         uint32_t sr[kBN];
@@ -321,59 +378,28 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
           for (int i = 0; i < kBN; ++i) sv[i] = (i < lim) ? sv[i] : -INFINITY;
         }
-        float mx0 = sv[0], mx1 = sv[1], mx2 = sv[2], mx3 = sv[3];
+        // row max: 8 independent chains of 3-input max, then a short tree
+        float mx[8];
 #pragma unroll
-        for (int i = 4; i < kBN; i += 8) {
-          mx0 = max3f(mx0, sv[i], sv[i + 1]);
-          mx1 = max3f(mx1, sv[i + 2], sv[i + 3]);
-          mx2 = max3f(mx2, sv[i + 4], sv[i + 5]);
-          mx3 = max3f(mx3, sv[i + 6], sv[i + 7]);
+        for (int k = 0; k < 8; ++k) mx[k] = fmaxf(sv[k], sv[k + 8]);
+#pragma unroll
+        for (int i = 16; i < kBN; i += 16) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mx[k] = max3f(mx[k], sv[i + k], sv[i + k + 8]);
         }
-        const float m_tile = max3f(mx0, mx1, fmaxf(mx2, mx3)) * c;
+        const float m_tile = max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * c;
         // raise the reference max only when the tile max exceeds it by more than the threshold
         const float m_new = (m_tile > m_ref + kRescaleThreshold) ? m_tile : m_ref;
         const float alpha = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - m_new);
         const bool rescale_o = (j > 0) && (m_new != m_ref);
-        if (__any_sync(0xffffffffu, rescale_o)) {
-          // O(t) must hold P·V(t, j-1) before it is rescaled
-          if (!warp_wait(bar(C::B_PVDONE + t), (j - 1) & 1, wd)) { ok = false; break; }
-          tc_fence_after();
-          const float f = rescale_o ? alpha : 1.f;
-#pragma unroll
-          for (int q = 0; q < D / 32; ++q) {
-            uint32_t r32[32];
-            tmem_ld32(tO + 32u * q, r32);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) r32[i] = __float_as_uint(__uint_as_float(r32[i]) * f);
-            tmem_st32(tO + 32u * q, r32);
-          }
-        }
         ell *= alpha;
         m_ref = m_new;
         // a row that has seen no visible key yet keeps m = -inf; its P is 0 either way
         const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
-        const float2 c2 = make_float2(c, c), nm2 = make_float2(neg_m, neg_m);
+        const float2 nm2 = make_float2(neg_m, neg_m);
         float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        if (!need_mask && !split_p) {
-          // fast path: ex2 on the MUFU for the first columns, the polynomial on the FMA pipe for the rest
-#pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            uint32_t pk[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int idx = 64 * q + 2 * i;
-              const float2 x = __ffma2_rn(make_float2(sv[idx], sv[idx + 1]), c2, nm2);
-              float2 e;
-              if (idx >= kBN - kPolyCols) e = exp2_poly2(x);
-              else e = make_float2(ex2(x.x), ex2(x.y));
-              acc[i & 3] = __fadd2_rn(acc[i & 3], e);
-              pk[i] = pack2<BF16>(e.x, e.y);
-            }
-            tmem_st32(tS + 32u * q, pk);
-          }
-        } else if (!split_p) {
-          // masked tile: every exponential on the MUFU (ex2(-inf) = 0 exactly)
+        if (!split_p) {
+          // P = 2^(c·s − m) on the MUFU (ex2(−inf) = 0 exactly), packed to 16 bits, written over S
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
             uint32_t pk[32];
@@ -406,16 +432,30 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             tmem_st16(tS + 64u + 16u * q, lo);
           }
         }
-        const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
-        const float2 a = __fadd2_rn(a01, a23);
-        const float rs0 = a.x, rs1 = a.y;
-        ell += rs0 + rs1;
+        const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+        ell += a.x + a.y;
+        if (__any_sync(0xffffffffu, rescale_o)) {
+          // The reference max rose (rare past the first tile): O(t) must hold P·V(t, j-1) before it
+          // is rescaled, and the rescale must land before P·V(t, j) is issued.
+          if (!warp_wait(bar(C::B_PVDONE + t), (j - 1) & 1, wd)) { ok = false; break; }
+          tc_fence_after();
+          const float f = rescale_o ? alpha : 1.f;
+#pragma unroll
+          for (int q = 0; q < D / 32; ++q) {
+            uint32_t r32[32];
+            tmem_ld32(tO + 32u * q, r32);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r32[i] = __float_as_uint(__uint_as_float(r32[i]) * f);
+            tmem_st32(tO + 32u * q, r32);
+          }
+        }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(C::B_PFULL + t));
       }
       // ---- epilogue: O / ℓ -> dtype, LSE
-      if (ok && warp_wait(bar(C::B_PVDONE + t), (nkv[t] - 1) & 1, wd)) {
+      if (ok && warp_wait(bar(C::B_PVDONE + t), (my_nkv - 1) & 1, wd)) {
         tc_fence_after();
         const bool valid = row < L;
         const float inv = (ell > 0.f) ? 1.f / ell : 0.f;
@@ -437,7 +477,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           }
         }
         if (valid) {
-          const float lse = (ell > 0.f && m_ref != -INFINITY) ? (m_ref + __log2f(ell)) * 0.69314718055994531f : -INFINITY;
+          const float lse = (ell > 0.f && m_ref != -INFINITY) ? (m_ref + __log2f(ell)) * 0.69314718055994531f
+                                                             : -INFINITY;
           p.lse[(size_t)(tok0 + row) * p.H + h] = lse;
         }
       }
