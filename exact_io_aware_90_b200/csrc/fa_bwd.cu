@@ -112,7 +112,7 @@ struct BwdParams {
   uint64_t timeout_ns;
 };
 
-constexpr int kBwdThreads = 320;
+constexpr int kBwdThreads = 384;  // 3 warpgroups
 constexpr int kBK = 128;  // keys per CTA
 
 template <int D>
@@ -153,6 +153,11 @@ struct BwdCfg {
   static constexpr uint32_t OFF_BAR = OFF_ROW + STAGES * 2 * BQ * 4;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
   static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;
+  // registers per thread after setmaxnreg (block of 384 launched at 168: 3 × 168 = 504 per lane triple)
+  static constexpr uint32_t REGS_CMP = 256;  // Pᵀ / dSᵀ warpgroup
+  static constexpr uint32_t REGS_DQ = 128;   // dQ warpgroup
+  static constexpr uint32_t REGS_IO = 120;   // producer / MMA warpgroup
+  static_assert(REGS_CMP + REGS_DQ + REGS_IO <= 504, "register budget");
 };
 
 __device__ __forceinline__ void drain_wait_b(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
@@ -176,6 +181,36 @@ __device__ __forceinline__ void red_add_f32(float* p, float v) {
 
 __device__ __forceinline__ void red_add_v4_f32(float* p, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
+
+// Products of one Q tile, issued by one elected lane.  Descriptor arguments
+// are pre-built bases; per 16-element K step only a constant start-address
+// offset (16-byte units) is added.
+// Sᵀ = K Qᵀ and dPᵀ = V dOᵀ: A = K or V (K-major, 128 rows), B = Q or dO
+// (K-major, BQ rows); K dim = d.
+template <int D, int BQ, uint32_t IDESC>
+__device__ __forceinline__ void bwd_issue_kt(uint32_t d_tmem, uint64_t da, uint64_t db) {
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t oa = ((kk >> 2) * (kBK * 128) + (kk & 3) * 32) >> 4;
+    const uint32_t ob = ((kk >> 2) * (BQ * 128) + (kk & 3) * 32) >> 4;
+    mma_ss(d_tmem, da + oa, db + ob, IDESC, kk > 0 ? 1u : 0u);
+  }
+}
+
+// dV += Pᵀ dO or dK += dSᵀ Q: A from tensor memory (8 packed columns per step),
+// B = dO or Q MN-major (+2 KB per 16 query rows); K dim = BQ.
+template <int BQ, uint32_t IDESC>
+__device__ __forceinline__ void bwd_issue_acc(uint32_t d_tmem, uint32_t a_tmem, uint64_t db, uint32_t acc) {
+#pragma unroll
+  for (int kk = 0; kk < BQ / 16; ++kk) mma_ts(d_tmem, a_tmem + kk * 8, db + ((kk * 2048) >> 4), IDESC, kk > 0 ? 1u : acc);
+}
+
+// dQ partial: K dim = the 128 keys, both operands MN-major (+2 KB per 16 keys).
+template <uint32_t IDESC>
+__device__ __forceinline__ void bwd_issue_dq(uint32_t d_tmem, uint64_t da, uint64_t db) {
+#pragma unroll
+  for (int kk = 0; kk < kBK / 16; ++kk) mma_ss(d_tmem, da + ((kk * 2048) >> 4), db + ((kk * 2048) >> 4), IDESC, kk > 0 ? 1u : 0u);
 }
 
 template <int D, bool BF16>
@@ -276,113 +311,129 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const Watchdog wd{abort_flag, p.timeout_ns};
 
-  if (warp == 8) {
-    // ================================================================ TMA producer (+ row terms)
-    const uint64_t pol_kv = l2_policy_evict_first();
-    const uint64_t pol_q = l2_policy_evict_last();
-    if (lane == 0) {
-      mbar_arrive_expect_tx(bar(C::B_KV), 2 * C::KV_TILE);
-      for (int c = 0; c < C::NCH; ++c) {
-        tma_load_3d(sK + c * (kBK * 128), &tm_k, bar(C::B_KV), c * 64, h, tok0 + k0, pol_kv);
-        tma_load_3d(sV + c * (kBK * 128), &tm_v, bar(C::B_KV), c * 64, h, tok0 + k0, pol_kv);
-      }
-    }
-    int issued = 0;
-    const float LOG2E = 1.4426950408889634f;
-    for (int it = 0; it < n_it; ++it) {
-      const int s = it % C::STAGES;
-      if (it >= C::STAGES && !warp_wait_b(bar(C::B_QEMPTY + s), ((it / C::STAGES) - 1) & 1, wd)) break;
-      const int i0 = (i_begin + it) * BQ;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(bar(C::B_QFULL + s), 2 * C::Q_TILE);
+  if (warp >= 8) {
+    regs_dec<C::REGS_IO>();
+    // The producer and MMA warps run their loops with all 32 lanes (warp-uniform state);
+    // one elected lane (always the lowest) issues each copy, MMA and commit.
+    if (warp == 8) {
+      // ================================================================ TMA producer (+ row terms)
+      const uint64_t pol_kv = l2_policy_evict_first();
+      const uint64_t pol_q = l2_policy_evict_last();
+      if (elect_one()) {
+        mbar_arrive_expect_tx(bar(C::B_KV), 2 * C::KV_TILE);
         for (int c = 0; c < C::NCH; ++c) {
-          tma_load_3d(sQ + s * C::Q_TILE + c * (BQ * 128), &tm_q, bar(C::B_QFULL + s), c * 64, h, tok0 + i0, pol_q);
-          tma_load_3d(sDO + s * C::Q_TILE + c * (BQ * 128), &tm_do, bar(C::B_QFULL + s), c * 64, h, tok0 + i0, pol_q);
+          tma_load_3d(sK + c * (kBK * 128), &tm_k, bar(C::B_KV), c * 64, h, tok0 + k0, pol_kv);
+          tma_load_3d(sV + c * (kBK * 128), &tm_v, bar(C::B_KV), c * 64, h, tok0 + k0, pol_kv);
         }
       }
-      // LSE (pre-multiplied by log2 e) and D of the tile's query rows; rows past the sequence get 0
-      float* lse_s = row_buf + s * 2 * BQ;
-      float* del_s = lse_s + BQ;
-      for (int q = lane; q < BQ; q += 32) {
-        const int qrow = i0 + q;
-        const bool v = qrow < L;
-        lse_s[q] = v ? __ldg(p.lse + (size_t)(tok0 + qrow) * p.H + h) * LOG2E : 0.f;
-        del_s[q] = v ? __ldg(p.delta + (size_t)(tok0 + qrow) * p.H + h) : 0.f;
-      }
-      mbar_arrive(bar(C::B_ROWFULL + s));  // release: the stores above are visible to waiters
-      issued = it + 1;
-    }
-    if (lane == 0) {
-      drain_wait_b(bar(C::B_KV), 0, p.timeout_ns);
-      for (int it = max(0, issued - C::STAGES); it < issued; ++it)
-        drain_wait_b(bar(C::B_QFULL + it % C::STAGES), (it / C::STAGES) & 1, p.timeout_ns);
-    }
-    __syncwarp();
-  } else if (warp == 9) {
-    // ================================================================ MMA issuer
-    if (lane == 0) {
-      const uint32_t tST = tmem + C::T_ST, tDPT = tmem + C::T_DPT, tDQ = tmem + C::T_DQ;
-      const uint32_t tDK = tmem + C::T_DK, tDV = tmem + C::T_DV;
-      bool ok = mbar_wait(bar(C::B_KV), 0, wd);
-      for (int it = 0; ok && it < n_it; ++it) {
+      __syncwarp();
+      int issued = 0;
+      const float LOG2E = 1.4426950408889634f;
+      for (int it = 0; it < n_it; ++it) {
         const int s = it % C::STAGES;
-        if (!mbar_wait(bar(C::B_QFULL + s), (it / C::STAGES) & 1, wd)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t q_t = sQ + s * C::Q_TILE, do_t = sDO + s * C::Q_TILE;
-        // Sᵀ = K Qᵀ, dPᵀ = V dOᵀ (K-major operands; K dim = d)
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off_k = (kk >> 2) * (kBK * 128) + (kk & 3) * 32;
-          const uint32_t off_q = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
-          mma_ss(tST, sdesc_sw128(sK + off_k, 16, 1024), sdesc_sw128(q_t + off_q, 16, 1024), IDESC_ST, kk > 0);
-        }
-        tc_commit(bar(C::B_SFULL));
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off_k = (kk >> 2) * (kBK * 128) + (kk & 3) * 32;
-          const uint32_t off_q = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
-          mma_ss(tDPT, sdesc_sw128(sV + off_k, 16, 1024), sdesc_sw128(do_t + off_q, 16, 1024), IDESC_ST, kk > 0);
-        }
-        tc_commit(bar(C::B_DPFULL));
-        // dV += Pᵀ dO   (Pᵀ packed in the Sᵀ columns; dO MN-major, K dim = BQ queries)
-        if (!mbar_wait(bar(C::B_PREADY), it & 1, wd)) { ok = false; break; }
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < BQ / 16; ++kk)
-          mma_ts(tDV, tST + kk * 8, sdesc_sw128(do_t + kk * 16 * 128, BQ * 128, 1024), IDESC_DKV,
-                 (it > 0 || kk > 0) ? 1u : 0u);
-        // dK += dSᵀ Q
-        if (!mbar_wait(bar(C::B_DSREADY), it & 1, wd)) { ok = false; break; }
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < BQ / 16; ++kk)
-          mma_ts(tDK, tDPT + kk * 8, sdesc_sw128(q_t + kk * 16 * 128, BQ * 128, 1024), IDESC_DKV,
-                 (it > 0 || kk > 0) ? 1u : 0u);
-        // dQ partial (K dim = 128 keys); the dQ columns must have been read out
-        if (it > 0 && !mbar_wait(bar(C::B_DQFREE), (it - 1) & 1, wd)) { ok = false; break; }
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk) {
-          if constexpr (D == 128) {
-            // A = Kᵀ (MN-major: 64-feature chunks 16 KB apart), B = dSᵀ [keys][64 q] (MN-major)
-            mma_ss(tDQ, sdesc_sw128(sK + kk * 16 * 128, kBK * 128, 1024), sdesc_sw128(sDS + kk * 16 * 128, 16, 1024),
-                   IDESC_DQ, kk > 0);
-          } else {
-            // A = dS (MN-major over queries: 64-query chunks 16 KB apart), B = K (MN-major, one chunk)
-            mma_ss(tDQ, sdesc_sw128(sDS + kk * 16 * 128, kBK * 128, 1024), sdesc_sw128(sK + kk * 16 * 128, 16, 1024),
-                   IDESC_DQ, kk > 0);
+        if (it >= C::STAGES && !warp_wait_b(bar(C::B_QEMPTY + s), ((it / C::STAGES) - 1) & 1, wd)) break;
+        const int i0 = (i_begin + it) * BQ;
+        if (elect_one()) {
+          mbar_arrive_expect_tx(bar(C::B_QFULL + s), 2 * C::Q_TILE);
+          for (int c = 0; c < C::NCH; ++c) {
+            tma_load_3d(sQ + s * C::Q_TILE + c * (BQ * 128), &tm_q, bar(C::B_QFULL + s), c * 64, h, tok0 + i0, pol_q);
+            tma_load_3d(sDO + s * C::Q_TILE + c * (BQ * 128), &tm_do, bar(C::B_QFULL + s), c * 64, h, tok0 + i0,
+                        pol_q);
           }
         }
-        tc_commit(bar(C::B_DQFULL));
-        tc_commit(bar(C::B_QEMPTY + s));
+        __syncwarp();
+        // LSE (pre-multiplied by log2 e) and D of the tile's query rows; rows past the sequence get 0
+        float* lse_s = row_buf + s * 2 * BQ;
+        float* del_s = lse_s + BQ;
+        for (int q = lane; q < BQ; q += 32) {
+          const int qrow = i0 + q;
+          const bool v = qrow < L;
+          lse_s[q] = v ? __ldg(p.lse + (size_t)(tok0 + qrow) * p.H + h) * LOG2E : 0.f;
+          del_s[q] = v ? __ldg(p.delta + (size_t)(tok0 + qrow) * p.H + h) : 0.f;
+        }
+        mbar_arrive(bar(C::B_ROWFULL + s));  // release: the stores above are visible to waiters
+        issued = it + 1;
       }
-      tc_commit(bar(C::B_DKV));
-      tc_commit(bar(C::B_DRAIN));
-      drain_wait_b(bar(C::B_DRAIN), 0, p.timeout_ns);
+      if (elect_one()) {
+        drain_wait_b(bar(C::B_KV), 0, p.timeout_ns);
+        for (int it = max(0, issued - C::STAGES); it < issued; ++it)
+          drain_wait_b(bar(C::B_QFULL + it % C::STAGES), (it / C::STAGES) & 1, p.timeout_ns);
+      }
+      __syncwarp();
+    } else if (warp == 9) {
+      // ================================================================ MMA issuer
+      // Per Q tile i:  dV += Pᵀ_i dO_i,  Sᵀ_{i+1} = K Qᵀ_{i+1},  dK += dSᵀ_i Q_i,  dQ_i,
+      // dPᵀ_{i+1} = V dOᵀ_{i+1}.  Sᵀ_{i+1} overwrites the columns of Pᵀ_i only after
+      // dV_i (issued before it, and tcgen05 MMAs of one thread run in order) has read
+      // them; dPᵀ_{i+1} likewise follows dK_i, which reads dSᵀ_i from those columns.
+      const uint32_t tST = tmem + C::T_ST, tDPT = tmem + C::T_DPT, tDQ = tmem + C::T_DQ;
+      const uint32_t tDK = tmem + C::T_DK, tDV = tmem + C::T_DV;
+      const uint64_t dK_kmaj = sdesc_sw128(sK, 16, 1024), dV_kmaj = sdesc_sw128(sV, 16, 1024);
+      const uint64_t dQ_kmaj = sdesc_sw128(sQ, 16, 1024), dDO_kmaj = sdesc_sw128(sDO, 16, 1024);
+      const uint64_t dQ_mn = sdesc_sw128(sQ, BQ * 128, 1024), dDO_mn = sdesc_sw128(sDO, BQ * 128, 1024);
+      // dQ operands (see IDESC_DQ)
+      const uint64_t dqa = (D == 128) ? sdesc_sw128(sK, kBK * 128, 1024) : sdesc_sw128(sDS, kBK * 128, 1024);
+      const uint64_t dqb = (D == 128) ? sdesc_sw128(sDS, 16, 1024) : sdesc_sw128(sK, 16, 1024);
+      constexpr uint32_t QT16 = C::Q_TILE >> 4;  // stage stride of Q / dO in descriptor units
+      bool ok = warp_wait_b(bar(C::B_KV), 0, wd) && warp_wait_b(bar(C::B_QFULL + 0), 0, wd);
+      if (ok) {
+        tc_fence_after();
+        if (elect_one()) {
+          bwd_issue_kt<D, BQ, IDESC_ST>(tST, dK_kmaj, dQ_kmaj);
+          tc_commit(bar(C::B_SFULL));
+          bwd_issue_kt<D, BQ, IDESC_ST>(tDPT, dV_kmaj, dDO_kmaj);
+          tc_commit(bar(C::B_DPFULL));
+        }
+        __syncwarp();
+      }
+      for (int it = 0; ok && it < n_it; ++it) {
+        const int s = it % C::STAGES;
+        const int s1 = (it + 1) % C::STAGES;
+        const bool more = it + 1 < n_it;
+        // dV += Pᵀ dO
+        if (!warp_wait_b(bar(C::B_PREADY), it & 1, wd)) { ok = false; break; }
+        tc_fence_after();
+        if (elect_one()) bwd_issue_acc<BQ, IDESC_DKV>(tDV, tST, dDO_mn + s * QT16, it > 0 ? 1u : 0u);
+        __syncwarp();
+        // Sᵀ of the next Q tile, computed while the dS of this one is formed
+        if (more) {
+          if (!warp_wait_b(bar(C::B_QFULL + s1), ((it + 1) / C::STAGES) & 1, wd)) { ok = false; break; }
+          tc_fence_after();
+          if (elect_one()) {
+            bwd_issue_kt<D, BQ, IDESC_ST>(tST, dK_kmaj, dQ_kmaj + s1 * QT16);
+            tc_commit(bar(C::B_SFULL));
+          }
+          __syncwarp();
+        }
+        // dK += dSᵀ Q
+        if (!warp_wait_b(bar(C::B_DSREADY), it & 1, wd)) { ok = false; break; }
+        tc_fence_after();
+        if (elect_one()) bwd_issue_acc<BQ, IDESC_DKV>(tDK, tDPT, dQ_mn + s * QT16, it > 0 ? 1u : 0u);
+        __syncwarp();
+        // dQ partial, once the dQ warpgroup has read the previous one out
+        if (it > 0 && !warp_wait_b(bar(C::B_DQFREE), (it - 1) & 1, wd)) { ok = false; break; }
+        tc_fence_after();
+        if (elect_one()) {
+          bwd_issue_dq<IDESC_DQ>(tDQ, dqa, dqb);
+          tc_commit(bar(C::B_DQFULL));
+          tc_commit(bar(C::B_QEMPTY + s));  // Q_i, dO_i and their row terms are no longer read
+          if (more) {
+            bwd_issue_kt<D, BQ, IDESC_ST>(tDPT, dV_kmaj, dDO_kmaj + s1 * QT16);
+            tc_commit(bar(C::B_DPFULL));
+          }
+        }
+        __syncwarp();
+      }
+      if (elect_one()) {
+        tc_commit(bar(C::B_DKV));
+        tc_commit(bar(C::B_DRAIN));
+        drain_wait_b(bar(C::B_DRAIN), 0, p.timeout_ns);
+      }
+      __syncwarp();
     }
-    __syncwarp();
   } else if (warp < 4) {
     // ================================================================ Pᵀ / dSᵀ warpgroup (thread = key row)
+    regs_inc<C::REGS_CMP>();
     const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
     const uint32_t tST = tmem + lane_off + C::T_ST;
     const uint32_t tDPT = tmem + lane_off + C::T_DPT;
@@ -398,9 +449,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const float* lse_s = row_buf + s * 2 * BQ;
       const float* del_s = lse_s + BQ;
       // visible queries for this key: q >= key (causal) and q < L; key < L
-      int q_lo = p.causal ? key - i0 : 0;  // first visible column
-      int q_hi = L - i0;                   // one past the last visible column
-      if (key >= L) q_hi = -1;
+      const int q_lo = p.causal ? key - i0 : 0;  // first visible column
+      const int q_hi = (key < L) ? L - i0 : -1;  // one past the last visible column
       if (!warp_wait_b(bar(C::B_SFULL), it & 1, wd)) { ok = false; break; }
       tc_fence_after();
       float pt[BQ];
@@ -427,36 +477,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_arrive(bar(C::B_PREADY));
       if (!warp_wait_b(bar(C::B_DPFULL), it & 1, wd)) { ok = false; break; }
       tc_fence_after();
-      uint32_t dsk[BQ / 2];
-      {
-        uint32_t dr[BQ];
+      // the previous dQ product must have finished reading the shared-memory dSᵀ buffer
+      if (it > 0 && !warp_wait_b(bar(C::B_DQFULL), (it - 1) & 1, wd)) { ok = false; break; }
+      // dSᵀ = Pᵀ ∘ (dPᵀ − D), 32 query columns at a time: into tensor memory over dPᵀ (A of the dK
+      // product) and into shared memory as 128-byte swizzled rows = keys (operand of the dQ product)
+      uint8_t* ds_row = smem + C::OFF_DS + kr * 128;
 #pragma unroll
-        for (int q = 0; q < BQ / 32; ++q) tmem_ld32(tDPT + 32u * q, reinterpret_cast<uint32_t(&)[32]>(dr[32 * q]));
+      for (int q = 0; q < BQ / 32; ++q) {
+        uint32_t dr[32];
+        tmem_ld32(tDPT + 32u * q, dr);
         tmem_wait_ld();
+        uint32_t dsk[16];
 #pragma unroll
-        for (int i = 0; i < BQ / 2; ++i) {
-          const float d0 = pt[2 * i] * (__uint_as_float(dr[2 * i]) - del_s[2 * i]);
-          const float d1 = pt[2 * i + 1] * (__uint_as_float(dr[2 * i + 1]) - del_s[2 * i + 1]);
+        for (int i = 0; i < 16; ++i) {
+          const int col = 32 * q + 2 * i;
+          const float d0 = pt[col] * (__uint_as_float(dr[2 * i]) - del_s[col]);
+          const float d1 = pt[col + 1] * (__uint_as_float(dr[2 * i + 1]) - del_s[col + 1]);
           dsk[i] = pack2<BF16>(d0, d1);
         }
-      }
-      // dSᵀ into tensor memory (A of the dK product) ...
+        tmem_st16(tDPT + 16u * q, dsk);
+        // 32 query columns = 64 bytes = 4 of the row's eight 16-byte chunks (64-query chunk q / 2)
 #pragma unroll
-      for (int q = 0; q < BQ / 64; ++q) tmem_st32(tDPT + 32u * q, reinterpret_cast<uint32_t(&)[32]>(dsk[32 * q]));
-      // ... and into shared memory, 128-byte swizzled rows = keys (operand of the dQ product);
-      // the previous dQ product must have finished reading the buffer
-      if (it > 0 && !warp_wait_b(bar(C::B_DQFULL), (it - 1) & 1, wd)) { ok = false; break; }
-      {
-        uint8_t* ds_row = smem + C::OFF_DS + kr * 128;
-#pragma unroll
-        for (int q = 0; q < BQ / 64; ++q) {
-#pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
-            const int sw = ch ^ (kr & 7);
-            uint4 v4 = make_uint4(dsk[32 * q + 4 * ch], dsk[32 * q + 4 * ch + 1], dsk[32 * q + 4 * ch + 2],
-                                  dsk[32 * q + 4 * ch + 3]);
-            *reinterpret_cast<uint4*>(ds_row + q * (kBK * 128) + sw * 16) = v4;
-          }
+        for (int ch = 0; ch < 4; ++ch) {
+          const int chunk = (q & 1) * 4 + ch;
+          const int sw = chunk ^ (kr & 7);
+          *reinterpret_cast<uint4*>(ds_row + (q >> 1) * (kBK * 128) + sw * 16) =
+              make_uint4(dsk[4 * ch], dsk[4 * ch + 1], dsk[4 * ch + 2], dsk[4 * ch + 3]);
         }
       }
       fence_proxy_async_smem();
@@ -487,6 +533,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncwarp();
   } else {
     // ================================================================ dQ warpgroup (warps 4-7)
+    regs_dec<C::REGS_DQ>();
     const int quarter = warp & 3;
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
     const uint32_t tDQ = tmem + lane_off + C::T_DQ;
@@ -507,9 +554,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // lane = feature, columns = 64 queries: each warp instruction covers 32 consecutive features
         float* base = p.dq_acc + ((size_t)(tok0 + i0) * p.H + h) * D + lrow;
         const int nq = min(64, L - i0);
-#pragma unroll 8
+        const size_t stride = (size_t)p.H * D;
+#pragma unroll
         for (int q = 0; q < 64; ++q)
-          if (q < nq) red_add_f32(base + (size_t)q * p.H * D, __uint_as_float(qr[q]));
+          if (q < nq) red_add_f32(base + q * stride, __uint_as_float(qr[q]));
       } else {
         // lane = query row, columns = 64 features
         const int qrow = i0 + lrow;
