@@ -129,6 +129,11 @@ struct BwdCfg {
   static constexpr uint32_t T_DQ = 2 * BQ;     // dQᵀ [d × 64] or dQ [128 × 64]: 64 columns
   static constexpr uint32_t T_DK = (D == 128) ? 256 : 320;
   static constexpr uint32_t T_DV = T_DK + D;
+  // dSᵀ as packed 16-bit (BQ/2 columns), A of the dK product: two buffers at d = 128 in the free
+  // columns [192, 256), one at d = 64 in [448, 512)
+  static constexpr int NDS = (D == 128) ? 2 : 1;
+  static constexpr uint32_t T_DS = (D == 128) ? 192 : 448;
+  static constexpr uint32_t T_DS_STRIDE = BQ / 2;
   // barriers
   static constexpr int B_KV = 0;
   static constexpr int B_QFULL = 1;
@@ -136,11 +141,13 @@ struct BwdCfg {
   static constexpr int B_ROWFULL = B_QEMPTY + STAGES;  // LSE / D of the Q tile in shared memory
   static constexpr int B_SFULL = B_ROWFULL + STAGES;
   static constexpr int B_DPFULL = B_SFULL + 1;
-  static constexpr int B_PREADY = B_DPFULL + 1;
+  static constexpr int B_DPFREE = B_DPFULL + 1;   // the compute warpgroup has read dPᵀ out
+  static constexpr int B_PREADY = B_DPFREE + 1;
   static constexpr int B_DSREADY = B_PREADY + 1;
   static constexpr int B_DQFULL = B_DSREADY + 1;
   static constexpr int B_DQFREE = B_DQFULL + 1;
-  static constexpr int B_DKV = B_DQFREE + 1;
+  static constexpr int B_DSFREE = B_DQFREE + 1;   // [NDS]: dK and dQ have read dSᵀ buffer b
+  static constexpr int B_DKV = B_DSFREE + NDS;
   static constexpr int B_DRAIN = B_DKV + 1;
   static constexpr int NBARS = B_DRAIN + 1;
   // shared memory
@@ -149,7 +156,7 @@ struct BwdCfg {
   static constexpr uint32_t OFF_Q = 2 * KV_TILE;
   static constexpr uint32_t OFF_DO = OFF_Q + STAGES * Q_TILE;
   static constexpr uint32_t OFF_DS = OFF_DO + STAGES * Q_TILE;
-  static constexpr uint32_t OFF_ROW = OFF_DS + DS_TILE;  // per stage: lse·log2(e)[BQ], D[BQ] (fp32)
+  static constexpr uint32_t OFF_ROW = OFF_DS + NDS * DS_TILE;  // per stage: −lse·log2(e)[BQ], −D[BQ] (fp32)
   static constexpr uint32_t OFF_BAR = OFF_ROW + STAGES * 2 * BQ * 4;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
   static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;
@@ -290,10 +297,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     mbar_init(bar(C::B_SFULL), 1);
     mbar_init(bar(C::B_DPFULL), 1);
+    mbar_init(bar(C::B_DPFREE), 128);
     mbar_init(bar(C::B_PREADY), 128);
     mbar_init(bar(C::B_DSREADY), 128);
     mbar_init(bar(C::B_DQFULL), 1);
     mbar_init(bar(C::B_DQFREE), 128);
+    for (int b = 0; b < C::NDS; ++b) mbar_init(bar(C::B_DSFREE + b), 1);
     mbar_init(bar(C::B_DKV), 1);
     mbar_init(bar(C::B_DRAIN), 1);
     *abort_flag = 0;
@@ -342,14 +351,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
         }
         __syncwarp();
-        // LSE (pre-multiplied by log2 e) and D of the tile's query rows; rows past the sequence get 0
+        // −LSE·log2 e and −D of the tile's query rows; rows past the sequence get 0
         float* lse_s = row_buf + s * 2 * BQ;
         float* del_s = lse_s + BQ;
         for (int q = lane; q < BQ; q += 32) {
           const int qrow = i0 + q;
           const bool v = qrow < L;
-          lse_s[q] = v ? __ldg(p.lse + (size_t)(tok0 + qrow) * p.H + h) * LOG2E : 0.f;
-          del_s[q] = v ? __ldg(p.delta + (size_t)(tok0 + qrow) * p.H + h) : 0.f;
+          lse_s[q] = v ? -__ldg(p.lse + (size_t)(tok0 + qrow) * p.H + h) * LOG2E : 0.f;
+          del_s[q] = v ? -__ldg(p.delta + (size_t)(tok0 + qrow) * p.H + h) : 0.f;
         }
         mbar_arrive(bar(C::B_ROWFULL + s));  // release: the stores above are visible to waiters
         issued = it + 1;
@@ -362,18 +371,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       __syncwarp();
     } else if (warp == 9) {
       // ================================================================ MMA issuer
-      // Per Q tile i:  dV += Pᵀ_i dO_i,  Sᵀ_{i+1} = K Qᵀ_{i+1},  dK += dSᵀ_i Q_i,  dQ_i,
-      // dPᵀ_{i+1} = V dOᵀ_{i+1}.  Sᵀ_{i+1} overwrites the columns of Pᵀ_i only after
-      // dV_i (issued before it, and tcgen05 MMAs of one thread run in order) has read
-      // them; dPᵀ_{i+1} likewise follows dK_i, which reads dSᵀ_i from those columns.
+      // Per Q tile i:  dV += Pᵀ_i dO_i,  Sᵀ_{i+1} = K Qᵀ_{i+1},  dPᵀ_{i+1} = V dOᵀ_{i+1},
+      // dK += dSᵀ_i Q_i,  dQ_i (at d = 64, with one dSᵀ buffer, dPᵀ_{i+1} comes last).  Sᵀ_{i+1} overwrites the columns of Pᵀ_i only after dV_i
+      // (issued before it; tcgen05 MMAs of one thread run in order) has read them, and
+      // dPᵀ_{i+1} overwrites dPᵀ_i once the compute warpgroup has read it out (dPᵀ free).
+      // dSᵀ_i has columns of its own, so dPᵀ_{i+1} need not wait for dK_i.
       const uint32_t tST = tmem + C::T_ST, tDPT = tmem + C::T_DPT, tDQ = tmem + C::T_DQ;
-      const uint32_t tDK = tmem + C::T_DK, tDV = tmem + C::T_DV;
+      const uint32_t tDK = tmem + C::T_DK, tDV = tmem + C::T_DV, tDS = tmem + C::T_DS;
       const uint64_t dK_kmaj = sdesc_sw128(sK, 16, 1024), dV_kmaj = sdesc_sw128(sV, 16, 1024);
       const uint64_t dQ_kmaj = sdesc_sw128(sQ, 16, 1024), dDO_kmaj = sdesc_sw128(sDO, 16, 1024);
       const uint64_t dQ_mn = sdesc_sw128(sQ, BQ * 128, 1024), dDO_mn = sdesc_sw128(sDO, BQ * 128, 1024);
       // dQ operands (see IDESC_DQ)
       const uint64_t dqa = (D == 128) ? sdesc_sw128(sK, kBK * 128, 1024) : sdesc_sw128(sDS, kBK * 128, 1024);
       const uint64_t dqb = (D == 128) ? sdesc_sw128(sDS, 16, 1024) : sdesc_sw128(sK, 16, 1024);
+      constexpr uint32_t DS16 = C::DS_TILE >> 4;  // dSᵀ buffer stride in descriptor units
       constexpr uint32_t QT16 = C::Q_TILE >> 4;  // stage stride of Q / dO in descriptor units
       bool ok = warp_wait_b(bar(C::B_KV), 0, wd) && warp_wait_b(bar(C::B_QFULL + 0), 0, wd);
       if (ok) {
@@ -395,8 +406,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after();
         if (elect_one()) bwd_issue_acc<BQ, IDESC_DKV>(tDV, tST, dDO_mn + s * QT16, it > 0 ? 1u : 0u);
         __syncwarp();
-        // Sᵀ of the next Q tile, computed while the dS of this one is formed
         if (more) {
+          // Sᵀ and dPᵀ of the next Q tile, computed while dS of this one is formed
           if (!warp_wait_b(bar(C::B_QFULL + s1), ((it + 1) / C::STAGES) & 1, wd)) { ok = false; break; }
           tc_fence_after();
           if (elect_one()) {
@@ -404,25 +415,47 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tc_commit(bar(C::B_SFULL));
           }
           __syncwarp();
+          if constexpr (C::NDS == 2) {
+            // with two dSᵀ buffers the next dPᵀ goes ahead of dK_i / dQ_i
+            if (!warp_wait_b(bar(C::B_DPFREE), it & 1, wd)) { ok = false; break; }
+            tc_fence_after();
+            if (elect_one()) {
+              bwd_issue_kt<D, BQ, IDESC_ST>(tDPT, dV_kmaj, dDO_kmaj + s1 * QT16);
+              tc_commit(bar(C::B_DPFULL));
+            }
+            __syncwarp();
+          }
         }
         // dK += dSᵀ Q
         if (!warp_wait_b(bar(C::B_DSREADY), it & 1, wd)) { ok = false; break; }
         tc_fence_after();
-        if (elect_one()) bwd_issue_acc<BQ, IDESC_DKV>(tDK, tDPT, dQ_mn + s * QT16, it > 0 ? 1u : 0u);
+        const int db = it % C::NDS;  // dSᵀ buffer of this Q tile
+        if (elect_one())
+          bwd_issue_acc<BQ, IDESC_DKV>(tDK, tDS + db * C::T_DS_STRIDE, dQ_mn + s * QT16, it > 0 ? 1u : 0u);
         __syncwarp();
         // dQ partial, once the dQ warpgroup has read the previous one out
         if (it > 0 && !warp_wait_b(bar(C::B_DQFREE), (it - 1) & 1, wd)) { ok = false; break; }
         tc_fence_after();
         if (elect_one()) {
-          bwd_issue_dq<IDESC_DQ>(tDQ, dqa, dqb);
+          if constexpr (D == 128) bwd_issue_dq<IDESC_DQ>(tDQ, dqa, dqb + db * DS16);
+          else bwd_issue_dq<IDESC_DQ>(tDQ, dqa + db * DS16, dqb);
           tc_commit(bar(C::B_DQFULL));
-          tc_commit(bar(C::B_QEMPTY + s));  // Q_i, dO_i and their row terms are no longer read
-          if (more) {
-            bwd_issue_kt<D, BQ, IDESC_ST>(tDPT, dV_kmaj, dDO_kmaj + s1 * QT16);
-            tc_commit(bar(C::B_DPFULL));
-          }
+          tc_commit(bar(C::B_DSFREE + db));  // dK_i and dQ_i have read dSᵀ buffer db
+          tc_commit(bar(C::B_QEMPTY + s));   // Q_i, dO_i and their row terms are no longer read
         }
         __syncwarp();
+        if constexpr (C::NDS == 1) {
+          // one dSᵀ buffer: the next dPᵀ follows dK_i / dQ_i, which the next dSᵀ write waits for anyway
+          if (more) {
+            if (!warp_wait_b(bar(C::B_DPFREE), it & 1, wd)) { ok = false; break; }
+            tc_fence_after();
+            if (elect_one()) {
+              bwd_issue_kt<D, BQ, IDESC_ST>(tDPT, dV_kmaj, dDO_kmaj + s1 * QT16);
+              tc_commit(bar(C::B_DPFULL));
+            }
+            __syncwarp();
+          }
+        }
       }
       if (elect_one()) {
         tc_commit(bar(C::B_DKV));
@@ -437,6 +470,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
     const uint32_t tST = tmem + lane_off + C::T_ST;
     const uint32_t tDPT = tmem + lane_off + C::T_DPT;
+    const uint32_t tDS = tmem + lane_off + C::T_DS;
     const uint32_t tDV = tmem + lane_off + C::T_DV;
     const int kr = 32 * warp + lane;  // key row within the tile
     const int key = k0 + kr;          // position in the sequence
@@ -451,8 +485,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // visible queries for this key: q >= key (causal) and q < L; key < L
       const int q_lo = p.causal ? key - i0 : 0;  // first visible column
       const int q_hi = (key < L) ? L - i0 : -1;  // one past the last visible column
+      const bool full = __all_sync(0xffffffffu, q_lo <= 0 && q_hi >= BQ);  // no masking in this tile
       if (!warp_wait_b(bar(C::B_SFULL), it & 1, wd)) { ok = false; break; }
       tc_fence_after();
+      const float2 c2 = make_float2(c, c);
       float pt[BQ];
       {
         uint32_t sr[BQ];
@@ -460,9 +496,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int q = 0; q < BQ / 32; ++q) tmem_ld32(tST + 32u * q, reinterpret_cast<uint32_t(&)[32]>(sr[32 * q]));
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < BQ; ++i) {
-          const float e = ex2(fmaf(__uint_as_float(sr[i]), c, -lse_s[i]));
-          pt[i] = (i >= q_lo && i < q_hi) ? e : 0.f;
+        for (int i = 0; i < BQ; i += 2) {
+          const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), c2,
+                                      make_float2(lse_s[i], lse_s[i + 1]));
+          pt[i] = ex2(x.x);
+          pt[i + 1] = ex2(x.y);
+        }
+        if (!full) {
+#pragma unroll
+          for (int i = 0; i < BQ; ++i) pt[i] = (i >= q_lo && i < q_hi) ? pt[i] : 0.f;
         }
       }
 #pragma unroll
@@ -477,25 +519,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_arrive(bar(C::B_PREADY));
       if (!warp_wait_b(bar(C::B_DPFULL), it & 1, wd)) { ok = false; break; }
       tc_fence_after();
-      // the previous dQ product must have finished reading the shared-memory dSᵀ buffer
-      if (it > 0 && !warp_wait_b(bar(C::B_DQFULL), (it - 1) & 1, wd)) { ok = false; break; }
-      // dSᵀ = Pᵀ ∘ (dPᵀ − D), 32 query columns at a time: into tensor memory over dPᵀ (A of the dK
-      // product) and into shared memory as 128-byte swizzled rows = keys (operand of the dQ product)
-      uint8_t* ds_row = smem + C::OFF_DS + kr * 128;
+      // dSᵀ buffer db: dK and dQ of the Q tile that used it before must have read it
+      const int db = it % C::NDS;
+      if (it >= C::NDS && !warp_wait_b(bar(C::B_DSFREE + db), ((it / C::NDS) - 1) & 1, wd)) { ok = false; break; }
+      // dSᵀ = Pᵀ ∘ (dPᵀ − D), 32 query columns at a time: into its tensor-memory columns (A of the
+      // dK product) and into shared memory as 128-byte swizzled rows = keys (operand of the dQ product)
+      uint8_t* ds_row = smem + C::OFF_DS + db * C::DS_TILE + kr * 128;
+      const uint32_t tDSb = tDS + db * C::T_DS_STRIDE;
 #pragma unroll
       for (int q = 0; q < BQ / 32; ++q) {
         uint32_t dr[32];
         tmem_ld32(tDPT + 32u * q, dr);
         tmem_wait_ld();
+        if (q == BQ / 32 - 1) {
+          // dPᵀ fully read out: the next dPᵀ may overwrite it
+          tc_fence_before();
+          mbar_arrive(bar(C::B_DPFREE));
+        }
         uint32_t dsk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int col = 32 * q + 2 * i;
-          const float d0 = pt[col] * (__uint_as_float(dr[2 * i]) - del_s[col]);
-          const float d1 = pt[col + 1] * (__uint_as_float(dr[2 * i + 1]) - del_s[col + 1]);
-          dsk[i] = pack2<BF16>(d0, d1);
+          const float2 dd = __fadd2_rn(make_float2(__uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1])),
+                                       make_float2(del_s[col], del_s[col + 1]));
+          const float2 ds = __fmul2_rn(make_float2(pt[col], pt[col + 1]), dd);
+          dsk[i] = pack2<BF16>(ds.x, ds.y);
         }
-        tmem_st16(tDPT + 16u * q, dsk);
+        tmem_st16(tDSb + 16u * q, dsk);
         // 32 query columns = 64 bytes = 4 of the row's eight 16-byte chunks (64-query chunk q / 2)
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {

@@ -51,6 +51,12 @@ constexpr int kFwdThreads = 384;  // 3 warpgroups
 constexpr int kBM = 128;  // query rows per tile
 constexpr int kBN = 128;  // keys per tile
 constexpr float kRescaleThreshold = 8.0f;
+// Column pairs i (of 64 per row) with bit (i % 8) set take the FMA-pipe exp2 in unmasked tiles.  At
+// d = 128 the tensor core needs as long per tile as the MUFU, and the polynomial costs about as much
+// per element as ex2, so it stays off; at d = 64 the MMAs take half as long and the exponentials bound
+// the tile, so part of them moves to the FMA pipe.
+template <int D> struct PolyMask { static constexpr uint32_t value = 0x00u; };
+template <> struct PolyMask<64> { static constexpr uint32_t value = 0x22u; };
 
 template <int D>
 struct FwdCfg {
@@ -398,7 +404,24 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
         const float2 nm2 = make_float2(neg_m, neg_m);
         float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        if (!split_p) {
+        if (!split_p && !need_mask && PolyMask<D>::value != 0u) {
+          // unmasked tile: part of the exponentials on the FMA pipe, interleaved with the MUFU ones
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            uint32_t pk[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int idx = 64 * q + 2 * i;
+              const float2 x = __ffma2_rn(make_float2(sv[idx], sv[idx + 1]), c2, nm2);
+              float2 e;
+              if ((PolyMask<D>::value >> (i & 7)) & 1u) e = exp2_poly2(x);
+              else e = make_float2(ex2(x.x), ex2(x.y));
+              acc[i & 3] = __fadd2_rn(acc[i & 3], e);
+              pk[i] = pack2<BF16>(e.x, e.y);
+            }
+            tmem_st32(tS + 32u * q, pk);
+          }
+        } else if (!split_p) {
           // P = 2^(c·s − m) on the MUFU (ex2(−inf) = 0 exactly), packed to 16 bits, written over S
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
