@@ -6,14 +6,20 @@
 // written back over it in the input dtype and fed to the P·V MMA from there,
 // so neither S nor P ever reaches device memory.
 //
-// CTA = one work unit = (sequence, head, 256 query rows) split into two
-// 128-row Q tiles that take turns on the tensor core:
+// Work unit = (sequence, head, 256 query rows), split into two 128-row Q
+// tiles that take turns on the tensor core.  The kernel is persistent: the
+// grid has one CTA per unit, but a running CTA keeps its tensor memory,
+// barriers and pipelines and takes further units from the hardware scheduler
+// (cluster launch control: it cancels the launch of a CTA that has not started
+// yet and does that CTA's unit), so on a busy GPU ~one CTA per SM does all the
+// work, and the next unit's first score tiles are computed while the current
+// unit's last P·V and O epilogue run.
 //   warps 0-3  softmax of Q tile 0 (one thread per row; TMEM lanes 0-127)
 //   warps 4-7  softmax of Q tile 1
-//   warp  8    TMA producer: Q0/Q1 once, then the K and V rings
+//   warp  8    scheduler and TMA producer: Q0/Q1 per unit, the K and V rings
 //   warp  9    tensor-memory allocator and MMA issuer (one elected lane)
 //   warps 10-11 idle (they complete the third warpgroup, whose registers
-//              setmaxnreg hands to the softmax warpgroups: 208 / 208 / 88)
+//              setmaxnreg hands to the softmax warpgroups: 200 / 200 / 104)
 // K_j and V_j have separate empty barriers: K_j's stage is handed back to
 // the producer as soon as both S(·, j) products are done, so the next K tile
 // streams in while P·V(·, j) still reads V_j.
@@ -22,7 +28,8 @@
 //   P·V(0,j)  S(0,j+1)  P·V(1,j)  S(1,j+1)
 // so while one warpgroup exponentiates, the tensor core works for the other.
 // tcgen05 MMAs from one thread execute in issue order, so S(t,j+1) may
-// overwrite the columns holding P(t,j) once P·V(t,j) has been issued.
+// overwrite the columns holding P(t,j) once P·V(t,j) has been issued; the
+// same holds for S(t,0) of the next unit after the last P·V(t,·) of this one.
 //
 // Online softmax in base 2 with c = scale·log2(e): m is kept in the scaled
 // domain and P = 2^(c·s − m).  The running max is only raised when the tile
@@ -65,21 +72,26 @@ struct FwdCfg {
   static constexpr int KSTAGES = (D == 128) ? 3 : 5;   // K ring depth
   static constexpr int VSTAGES = (D == 128) ? 2 : 4;   // V ring depth
   // barrier indices
-  static constexpr int B_Q = 0;
-  static constexpr int B_KFULL = 1;
+  static constexpr int B_QFULL = 0;                   // [2] Q tile t loaded
+  static constexpr int B_QEMPTY = B_QFULL + 2;        // [2] last S of Q tile t in its unit done
+  static constexpr int B_KFULL = B_QEMPTY + 2;
   static constexpr int B_KEMPTY = B_KFULL + KSTAGES;
   static constexpr int B_VFULL = B_KEMPTY + KSTAGES;
   static constexpr int B_VEMPTY = B_VFULL + VSTAGES;
   static constexpr int B_SFULL = B_VEMPTY + VSTAGES;
   static constexpr int B_PFULL = B_SFULL + 2;
   static constexpr int B_PVDONE = B_PFULL + 2;
-  static constexpr int B_DRAIN = B_PVDONE + 2;
+  static constexpr int B_UFULL = B_PVDONE + 2;        // [2] work-unit ring slot written
+  static constexpr int B_UEMPTY = B_UFULL + 2;        // [2] slot read by the MMA warp and the 8 softmax warps
+  static constexpr int B_CLC = B_UEMPTY + 2;          // scheduler response landed
+  static constexpr int B_DRAIN = B_CLC + 1;
   static constexpr int NBARS = B_DRAIN + 1;
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_K = 2 * TILE;
   static constexpr uint32_t OFF_V = OFF_K + KSTAGES * TILE;
-  static constexpr uint32_t OFF_BAR = OFF_V + VSTAGES * TILE;
-  static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
+  static constexpr uint32_t OFF_CLC = OFF_V + VSTAGES * TILE;  // 16-byte scheduler response
+  static constexpr uint32_t OFF_BAR = OFF_CLC + 16;
+  static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;     // TMEM base, abort flag, unit ring [2]
   static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
@@ -107,8 +119,18 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const W
 // S = Q·Kᵀ for one 128 × 128 tile: D/16 MMAs of K = 16 along the head dimension.
 // Q and K are K-major with 128-byte rows; a 16-element step is +32 bytes inside a
 // swizzle atom, a 64-element step the next 16 KB atom column.
+// Returns x unchanged but opaque to the compiler, so descriptors derived from it
+// are formed at the issue site instead of being kept live across the MMA loop
+// (the MMA warp runs with 104 registers).
+__device__ __forceinline__ uint64_t opaque64(uint64_t x) {
+  asm volatile("mov.b64 %0, %0;" : "+l"(x));
+  return x;
+}
+
 template <int D, uint32_t IDESC>
 __device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint64_t dq, uint64_t dk) {
+  dq = opaque64(dq);
+  dk = opaque64(dk);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
     const uint32_t off = ((kk >> 2) * (kBM * 128) + (kk & 3) * 32) >> 4;
@@ -120,9 +142,64 @@ __device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint64_t dq, uint64_t 
 // (8 columns of packed 16-bit values per step), V is MN-major (+2 KB per 16 keys).
 template <uint32_t IDESC>
 __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint64_t dv, uint32_t acc) {
+  dv = opaque64(dv);
 #pragma unroll
   for (int kk = 0; kk < kBN / 16; ++kk)
     mma_ts(o_tmem, p_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), IDESC, kk > 0 ? 1u : acc);
+}
+
+// A decoded work unit: query rows [q0, q0 + 256) of the sequence whose tokens
+// are [tok0, tok0 + L), head h; nkv[t] KV tiles for Q tile t (0 when the tile
+// lies past the end of the sequence), n_iter = max(nkv[0], nkv[1]).
+struct FwdUnit {
+  int tok0, L, q0, h;
+  int nkv[2];
+  int n_iter;
+};
+
+// Unit order: heads in groups (K/V of a group stay in L2), heaviest query
+// blocks first inside a group (causal load balance).  Returns false for a unit
+// with no query row inside its sequence; invalid sequence bounds are recorded
+// as FA_ERR_INVALID_ARG and the unit is skipped.
+__device__ __forceinline__ bool decode_unit(const FwdParams& p, int unit, FwdUnit& u) {
+  const int BH = p.B * p.H;
+  const int nqb = p.num_qblocks;
+  const int G = p.heads_group;
+  const int group = unit / (G * nqb);
+  const int g_heads = min(G, BH - group * G);
+  const int r = unit - group * G * nqb;
+  const int qb = nqb - 1 - r / g_heads;
+  const int bh = group * G + r % g_heads;
+  const int b = bh / p.H;
+  u.h = bh - b * p.H;
+  if (p.cu_seqlens != nullptr) {
+    u.tok0 = __ldg(p.cu_seqlens + b);
+    const int end = __ldg(p.cu_seqlens + b + 1);
+    u.L = end - u.tok0;
+    if (u.tok0 < 0 || u.L < 0 || end > p.T || u.L > p.N) {
+      record_status(1);
+      return false;
+    }
+  } else {
+    u.tok0 = b * p.N;
+    u.L = p.N;
+  }
+  u.q0 = qb * 2 * kBM;
+  if (u.q0 >= u.L) return false;
+  const int nkv_all = (u.L + kBN - 1) / kBN;
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int first_row = u.q0 + t * kBM;
+    if (first_row >= u.L) u.nkv[t] = 0;
+    else u.nkv[t] = p.causal ? min(nkv_all, (first_row + kBM - 1) / kBN + 1) : nkv_all;
+  }
+  u.n_iter = max(u.nkv[0], u.nkv[1]);
+  return true;
+}
+
+// Warp-uniform non-blocking probe of one barrier phase.
+__device__ __forceinline__ bool warp_test(uint32_t bar, uint32_t parity) {
+  return __all_sync(0xffffffffu, mbar_test_wait(bar, parity));
 }
 
 template <int D, bool BF16>
@@ -139,60 +216,31 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const uint32_t sQ = s_base + C::OFF_Q;
   const uint32_t sK = s_base + C::OFF_K;
   const uint32_t sV = s_base + C::OFF_V;
+  const uint32_t clc_resp = s_base + C::OFF_CLC;
   const uint32_t bar0 = s_base + C::OFF_BAR;
   auto bar = [&](int i) -> uint32_t { return bar0 + 8u * i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   int* abort_flag = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
+  volatile int* unit_ring = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- decode the work unit: heads in groups (K/V of a group stay in L2),
-  //      heaviest query blocks first inside a group (causal load balance)
-  const int BH = p.B * p.H;
-  const int nqb = p.num_qblocks;
-  const int G = p.heads_group;
-  const int unit = blockIdx.x;
-  const int group = unit / (G * nqb);
-  const int g_heads = min(G, BH - group * G);
-  const int r = unit - group * G * nqb;
-  const int qb = nqb - 1 - r / g_heads;
-  const int bh = group * G + r % g_heads;
-  const int b = bh / p.H;
-  const int h = bh - b * p.H;
-
-  int tok0, L;
-  if (p.cu_seqlens != nullptr) {
-    tok0 = __ldg(p.cu_seqlens + b);
-    const int end = __ldg(p.cu_seqlens + b + 1);
-    L = end - tok0;
-    if (tok0 < 0 || L < 0 || end > p.T || L > p.N) {
-      if (threadIdx.x == 0) record_status(1);
-      return;
-    }
-  } else {
-    tok0 = b * p.N;
-    L = p.N;
-  }
-  const int q0 = qb * 2 * kBM;
-  if (q0 >= L) return;  // uniform over the CTA: nothing allocated yet
-  const int nkv_all = (L + kBN - 1) / kBN;
-  int nkv[2];
-#pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    const int first_row = q0 + t * kBM;
-    if (first_row >= L) nkv[t] = 0;
-    else nkv[t] = p.causal ? min(nkv_all, (first_row + kBM - 1) / kBN + 1) : nkv_all;
-  }
-  const int n_iter = max(nkv[0], nkv[1]);
-
-  // ---- set-up: barriers, tensor memory
+  // ---- set-up, once per CTA: the CTA then runs work units until none is left
   if (warp == 9) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
   if (threadIdx.x == 0) {
-    mbar_init(bar(C::B_Q), 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(C::B_QFULL + t), 1);
+      mbar_init(bar(C::B_QEMPTY + t), 1);
+      mbar_init(bar(C::B_SFULL + t), 1);
+      mbar_init(bar(C::B_PFULL + t), kBM);
+      mbar_init(bar(C::B_PVDONE + t), 1);
+      mbar_init(bar(C::B_UFULL + t), 1);
+      mbar_init(bar(C::B_UEMPTY + t), 9);
+    }
     for (int s = 0; s < C::KSTAGES; ++s) {
       mbar_init(bar(C::B_KFULL + s), 1);
       mbar_init(bar(C::B_KEMPTY + s), 1);
@@ -201,11 +249,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(bar(C::B_VFULL + s), 1);
       mbar_init(bar(C::B_VEMPTY + s), 1);
     }
-    for (int t = 0; t < 2; ++t) {
-      mbar_init(bar(C::B_SFULL + t), 1);
-      mbar_init(bar(C::B_PFULL + t), kBM);
-      mbar_init(bar(C::B_PVDONE + t), 1);
-    }
+    mbar_init(bar(C::B_CLC), 1);
     mbar_init(bar(C::B_DRAIN), 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -222,57 +266,125 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const Watchdog wd{abort_flag, p.timeout_ns};
 
   if (warp >= 8) {
-    regs_dec<88>();
+    regs_dec<104>();
     // The producer and MMA warps run their loops with all 32 lanes (warp-uniform state the
     // compiler can keep in uniform registers); one elected lane issues each TMA copy, MMA and
     // commit.  elect.sync picks the lowest active lane, so every MMA and every commit that
     // tracks it come from the same thread.
     if (warp == 8) {
-      // ================================================================ TMA producer
+      // ================================================================ scheduler and TMA producer
+      // Units come from the hardware scheduler: this CTA's own index first, then, one at a time,
+      // the index of a CTA of the grid that has not started yet, whose launch is cancelled.  Each
+      // unit is published to the other roles through a two-slot ring.  Loads follow the order in
+      // which the MMA warp consumes them across a unit boundary: Q0, K0, Q1, V0, K1, V1, ...
       const uint64_t pol_q = l2_policy_evict_first();
       const uint64_t pol_kv = l2_policy_evict_last();
-      const int nq = nkv[1] > 0 ? 2 : 1;
-      if (elect_one()) {
-        mbar_arrive_expect_tx(bar(C::B_Q), nq * C::TILE);
-        for (int t = 0; t < nq; ++t)
-          for (int c = 0; c < C::NCH; ++c)
-            tma_load_3d(sQ + t * C::TILE + c * (kBM * 128), &tm_q, bar(C::B_Q), c * 64, h, tok0 + q0 + t * kBM,
-                        pol_q);
-      }
-      __syncwarp();
-      int issued = 0;
-      for (int j = 0; j < n_iter; ++j) {
-        const int sk = j % C::KSTAGES, sv = j % C::VSTAGES;
-        if (j >= C::KSTAGES && !warp_wait(bar(C::B_KEMPTY + sk), ((j / C::KSTAGES) - 1) & 1, wd)) break;
+      uint32_t kc = 0, vc = 0;      // K / V tiles loaded so far (ring positions)
+      uint32_t qn[2] = {0u, 0u};    // loads of Q tile t
+      uint32_t un = 0;              // units published
+      uint32_t c_issued = 0, c_done = 0;  // cancellation requests / responses
+      bool can_steal = true, ok = true;
+      auto steal = [&]() -> int {
+        if (!can_steal) return -1;
         if (elect_one()) {
-          mbar_arrive_expect_tx(bar(C::B_KFULL + sk), C::TILE);
-          for (int c = 0; c < C::NCH; ++c)
-            tma_load_3d(sK + sk * C::TILE + c * (kBN * 128), &tm_k, bar(C::B_KFULL + sk), c * 64, h, tok0 + j * kBN,
-                        pol_kv);
+          mbar_arrive_expect_tx(bar(C::B_CLC), 16);
+          clc_try_cancel(clc_resp, bar(C::B_CLC));
         }
         __syncwarp();
-        if (j >= C::VSTAGES && !warp_wait(bar(C::B_VEMPTY + sv), ((j / C::VSTAGES) - 1) & 1, wd)) {
-          issued = -(j + 1);  // K_j issued, V_j not
-          break;
+        ++c_issued;
+        if (!warp_wait(bar(C::B_CLC), c_done & 1, wd)) {
+          ok = false;
+          return -1;
         }
+        ++c_done;
+        int x = -1;
+        const bool got = clc_query(clc_resp, x);
+        fence_proxy_async_smem();  // the read above before the next response overwrites it
+        __syncwarp();
+        if (!got) {
+          can_steal = false;  // no CTA left; no further request may be made
+          return -1;
+        }
+        return x;
+      };
+      auto publish = [&](int unit) -> bool {
+        const int s = un & 1;
+        if (un >= 2 && !warp_wait(bar(C::B_UEMPTY + s), ((un >> 1) - 1) & 1, wd)) return false;
         if (elect_one()) {
-          mbar_arrive_expect_tx(bar(C::B_VFULL + sv), C::TILE);
-          for (int c = 0; c < C::NCH; ++c)
-            tma_load_3d(sV + sv * C::TILE + c * (kBN * 128), &tm_v, bar(C::B_VFULL + sv), c * 64, h, tok0 + j * kBN,
-                        pol_kv);
+          unit_ring[s] = unit;
+          mbar_arrive(bar(C::B_UFULL + s));  // release: the store is visible once the phase flips
         }
         __syncwarp();
-        issued = j + 1;
+        ++un;
+        return true;
+      };
+      auto load_q = [&](const FwdUnit& u, int t) -> bool {
+        if (qn[t] > 0 && !warp_wait(bar(C::B_QEMPTY + t), (qn[t] - 1) & 1, wd)) return false;
+        if (elect_one()) {
+          mbar_arrive_expect_tx(bar(C::B_QFULL + t), C::TILE);
+          for (int c = 0; c < C::NCH; ++c)
+            tma_load_3d(sQ + t * C::TILE + c * (kBM * 128), &tm_q, bar(C::B_QFULL + t), c * 64, u.h,
+                        u.tok0 + u.q0 + t * kBM, pol_q);
+        }
+        __syncwarp();
+        ++qn[t];
+        return true;
+      };
+      auto load_k = [&](const FwdUnit& u, int j) -> bool {
+        const uint32_t s = kc % C::KSTAGES;
+        if (kc >= (uint32_t)C::KSTAGES && !warp_wait(bar(C::B_KEMPTY + s), ((kc / C::KSTAGES) - 1) & 1, wd))
+          return false;
+        if (elect_one()) {
+          mbar_arrive_expect_tx(bar(C::B_KFULL + s), C::TILE);
+          for (int c = 0; c < C::NCH; ++c)
+            tma_load_3d(sK + s * C::TILE + c * (kBN * 128), &tm_k, bar(C::B_KFULL + s), c * 64, u.h,
+                        u.tok0 + j * kBN, pol_kv);
+        }
+        __syncwarp();
+        ++kc;
+        return true;
+      };
+      auto load_v = [&](const FwdUnit& u, int j) -> bool {
+        const uint32_t s = vc % C::VSTAGES;
+        if (vc >= (uint32_t)C::VSTAGES && !warp_wait(bar(C::B_VEMPTY + s), ((vc / C::VSTAGES) - 1) & 1, wd))
+          return false;
+        if (elect_one()) {
+          mbar_arrive_expect_tx(bar(C::B_VFULL + s), C::TILE);
+          for (int c = 0; c < C::NCH; ++c)
+            tma_load_3d(sV + s * C::TILE + c * (kBN * 128), &tm_v, bar(C::B_VFULL + s), c * 64, u.h,
+                        u.tok0 + j * kBN, pol_kv);
+        }
+        __syncwarp();
+        ++vc;
+        return true;
+      };
+      int unit = blockIdx.x;
+      while (ok) {
+        FwdUnit U;
+        bool have = decode_unit(p, unit, U);
+        while (!have) {  // a unit past the end of its sequence: take the next one
+          unit = steal();
+          if (unit < 0) break;
+          have = decode_unit(p, unit, U);
+        }
+        if (!have) break;
+        ok = publish(unit) && load_q(U, 0) && load_k(U, 0) && (U.nkv[1] == 0 || load_q(U, 1)) && load_v(U, 0);
+        for (int j = 1; ok && j < U.n_iter; ++j) ok = load_k(U, j) && load_v(U, j);
+        if (!ok) break;
+        unit = steal();
+        if (unit < 0) break;
       }
-      // Let every load this warp issued land before the CTA can exit.
+      if (ok) publish(-1);  // no unit left
+      // Let every load and scheduler response this warp asked for land before the CTA can exit.
       if (elect_one()) {
-        const int k_issued = issued >= 0 ? issued : -issued;
-        const int v_issued = issued >= 0 ? issued : -issued - 1;
-        drain_wait(bar(C::B_Q), 0, p.timeout_ns);
-        for (int j = max(0, k_issued - C::KSTAGES); j < k_issued; ++j)
-          drain_wait(bar(C::B_KFULL + j % C::KSTAGES), (j / C::KSTAGES) & 1, p.timeout_ns);
-        for (int j = max(0, v_issued - C::VSTAGES); j < v_issued; ++j)
-          drain_wait(bar(C::B_VFULL + j % C::VSTAGES), (j / C::VSTAGES) & 1, p.timeout_ns);
+        if (c_issued > c_done) drain_wait(bar(C::B_CLC), c_done & 1, p.timeout_ns);
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+          if (qn[t] > 0) drain_wait(bar(C::B_QFULL + t), (qn[t] - 1) & 1, p.timeout_ns);
+        for (uint32_t i = kc > (uint32_t)C::KSTAGES ? kc - C::KSTAGES : 0u; i < kc; ++i)
+          drain_wait(bar(C::B_KFULL + i % C::KSTAGES), (i / C::KSTAGES) & 1, p.timeout_ns);
+        for (uint32_t i = vc > (uint32_t)C::VSTAGES ? vc - C::VSTAGES : 0u; i < vc; ++i)
+          drain_wait(bar(C::B_VFULL + i % C::VSTAGES), (i / C::VSTAGES) & 1, p.timeout_ns);
       }
       __syncwarp();
     } else if (warp == 9) {
@@ -282,61 +394,130 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const uint64_t dq_base = sdesc_sw128(sQ, 16, 1024);
       const uint64_t dk_base = sdesc_sw128(sK, 16, 1024);
       const uint64_t dv_base = sdesc_sw128(sV, kBN * 128, 1024);
-      bool ok = warp_wait(bar(C::B_Q), 0, wd) && warp_wait(bar(C::B_KFULL + 0), 0, wd);
-      if (ok) {
+      uint32_t kc = 0, vc = 0;    // ring positions of the current unit's first K / V tile
+      uint32_t qn[2] = {0u, 0u};  // Q tile t loads consumed
+      uint32_t pn[2] = {0u, 0u};  // P tiles of Q tile t consumed (all units)
+      uint32_t un = 0;            // units read
+      bool ok = true;
+      auto read_unit = [&](int& unit) -> bool {
+        const int s = un & 1;
+        if (!warp_wait(bar(C::B_UFULL + s), (un >> 1) & 1, wd)) return false;
+        unit = unit_ring[s];
+        __syncwarp();
+        if (elect_one()) mbar_arrive(bar(C::B_UEMPTY + s));
+        __syncwarp();
+        ++un;
+        return true;
+      };
+      auto k_wait = [&](uint32_t kpos) -> bool {
+        return warp_wait(bar(C::B_KFULL + kpos % C::KSTAGES), (kpos / C::KSTAGES) & 1, wd);
+      };
+      // S(t, 0) of unit u with its K tile at ring position kpos
+      auto first_s = [&](const FwdUnit& u, int t, uint32_t kpos) -> bool {
+        if (!warp_wait(bar(C::B_QFULL + t), qn[t] & 1, wd)) return false;
+        ++qn[t];
         tc_fence_after();
         if (elect_one()) {
-          if (nkv[0] > 0) {
-            issue_qk<D, IDESC_S>(tmem + 0u, dq_base, dk_base);
-            tc_commit(bar(C::B_SFULL + 0));
-          }
-          if (nkv[1] > 0) {
-            issue_qk<D, IDESC_S>(tmem + 128u, dq_base + (C::TILE >> 4), dk_base);
-            tc_commit(bar(C::B_SFULL + 1));
-          }
-          tc_commit(bar(C::B_KEMPTY + 0));  // K_0 is read by no later MMA
+          issue_qk<D, IDESC_S>(tmem + 128u * t, dq_base + ((t * C::TILE) >> 4),
+                               dk_base + (((kpos % C::KSTAGES) * C::TILE) >> 4));
+          tc_commit(bar(C::B_SFULL + t));
+          if (u.nkv[t] == 1) tc_commit(bar(C::B_QEMPTY + t));  // Q tile t is read by no later MMA of u
         }
+        __syncwarp();
+        return true;
+      };
+      int cur = -1;
+      FwdUnit U;
+      ok = read_unit(cur);
+      if (ok && cur >= 0) {
+        decode_unit(p, cur, U);
+        ok = k_wait(0) && first_s(U, 0, 0) && (U.nkv[1] == 0 || first_s(U, 1, 0));
+        if (ok && elect_one()) tc_commit(bar(C::B_KEMPTY + 0));  // K_0: both S(·, 0) issued
         __syncwarp();
       }
-      for (int j = 0; ok && j < n_iter; ++j) {
-        const int s = j % C::VSTAGES;                  // V_j
-        const uint32_t ph = (j / C::VSTAGES) & 1;
-        const uint64_t dv_s = dv_base + ((s * C::TILE) >> 4);
-        const int s1 = (j + 1) % C::KSTAGES;           // K_{j+1}
-        const uint64_t dk_s1 = dk_base + ((s1 * C::TILE) >> 4);
-        bool v_ready = false;
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          if (j >= nkv[t]) continue;
-          const uint32_t s_tmem = tmem + 128u * t;
-          const uint32_t o_tmem = tmem + 256u + (uint32_t)D * t;
-          if (!warp_wait(bar(C::B_PFULL + t), j & 1, wd)) { ok = false; break; }
-          if (!v_ready) {
-            if (!warp_wait(bar(C::B_VFULL + s), ph, wd)) { ok = false; break; }
-            v_ready = true;
+      while (ok && cur >= 0) {
+        // The next unit's S(t, 0) go to the tensor core as soon as Q tile t has issued its last
+        // P·V of this unit (MMAs of one thread run in issue order, so S(t, 0) cannot overwrite
+        // P(t, last) before that P·V has read it).  Until the unit's last step only non-blocking
+        // probes are used: the producer may still be waiting for this warp to free a ring stage.
+        int nxt = -1;
+        bool nxt_read = false, nx_s0 = false, nx_s1 = false;
+        FwdUnit N;
+        const uint32_t kn = kc + U.n_iter;  // ring position of the next unit's K_0
+        auto prefetch_next = [&](bool done1, bool force) -> bool {
+          if (!nxt_read) {
+            if (!force && !warp_test(bar(C::B_UFULL + (un & 1)), (un >> 1) & 1)) return true;
+            if (!read_unit(nxt)) return false;
+            nxt_read = true;
+            if (nxt >= 0) decode_unit(p, nxt, N);
           }
-          tc_fence_after();
-          if (elect_one()) {
-            issue_pv<IDESC_O>(o_tmem, s_tmem, dv_s, j > 0 ? 1u : 0u);
-            if (nkv[t] == 1) issue_pv<IDESC_O>(o_tmem, s_tmem + 64u, dv_s, 1u);  // lo part of a split P
-            tc_commit(bar(C::B_PVDONE + t));
+          if (nxt < 0) return true;
+          if (!nx_s0) {
+            if (!force && !(warp_test(bar(C::B_QFULL + 0), qn[0] & 1) &&
+                            warp_test(bar(C::B_KFULL + kn % C::KSTAGES), (kn / C::KSTAGES) & 1)))
+              return true;
+            if (!k_wait(kn) || !first_s(N, 0, kn)) return false;
+            nx_s0 = true;
           }
-          __syncwarp();
-          if (j + 1 < nkv[t]) {
-            if (!warp_wait(bar(C::B_KFULL + s1), ((j + 1) / C::KSTAGES) & 1, wd)) { ok = false; break; }
-            tc_fence_after();
-            if (elect_one()) {
-              issue_qk<D, IDESC_S>(s_tmem, dq_base + ((t * C::TILE) >> 4), dk_s1);
-              tc_commit(bar(C::B_SFULL + t));
+          if (!nx_s1 && (N.nkv[1] == 0 || done1)) {
+            if (N.nkv[1] > 0) {
+              if (!force && !warp_test(bar(C::B_QFULL + 1), qn[1] & 1)) return true;
+              if (!first_s(N, 1, kn)) return false;
             }
+            nx_s1 = true;
+            if (elect_one()) tc_commit(bar(C::B_KEMPTY + kn % C::KSTAGES));  // both S(·, 0) of the next unit issued
             __syncwarp();
           }
+          return true;
+        };
+        for (int j = 0; ok && j < U.n_iter; ++j) {
+          const uint32_t vpos = vc + j;
+          const uint64_t dv_s = dv_base + (((vpos % C::VSTAGES) * C::TILE) >> 4);
+          const uint32_t kpos1 = kc + j + 1;  // K_{j+1}
+          const uint64_t dk_s1 = dk_base + (((kpos1 % C::KSTAGES) * C::TILE) >> 4);
+          bool v_ready = false;
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            if (j >= U.nkv[t]) continue;
+            const uint32_t s_tmem = tmem + 128u * t;
+            const uint32_t o_tmem = tmem + 256u + (uint32_t)D * t;
+            if (!warp_wait(bar(C::B_PFULL + t), pn[t] & 1, wd)) { ok = false; break; }
+            ++pn[t];
+            if (!v_ready) {
+              if (!warp_wait(bar(C::B_VFULL + vpos % C::VSTAGES), (vpos / C::VSTAGES) & 1, wd)) { ok = false; break; }
+              v_ready = true;
+            }
+            tc_fence_after();
+            if (elect_one()) {
+              issue_pv<IDESC_O>(o_tmem, s_tmem, dv_s, j > 0 ? 1u : 0u);
+              if (U.nkv[t] == 1) issue_pv<IDESC_O>(o_tmem, s_tmem + 64u, dv_s, 1u);  // lo part of a split P
+              tc_commit(bar(C::B_PVDONE + t));
+            }
+            __syncwarp();
+            if (j + 1 < U.nkv[t]) {
+              if (!k_wait(kpos1)) { ok = false; break; }
+              tc_fence_after();
+              if (elect_one()) {
+                issue_qk<D, IDESC_S>(s_tmem, dq_base + ((t * C::TILE) >> 4), dk_s1);
+                tc_commit(bar(C::B_SFULL + t));
+                if (j + 2 == U.nkv[t]) tc_commit(bar(C::B_QEMPTY + t));  // last S of Q tile t in this unit
+              }
+              __syncwarp();
+            }
+          }
+          if (!ok) break;
+          if (elect_one()) {
+            tc_commit(bar(C::B_VEMPTY + vpos % C::VSTAGES));                // V_j: both P·V(·, j) issued
+            if (j + 1 < U.n_iter) tc_commit(bar(C::B_KEMPTY + kpos1 % C::KSTAGES));  // K_{j+1}: both S(·, j+1)
+          }
+          __syncwarp();
+          if (j + 1 >= U.nkv[0] && j + 1 < U.n_iter && !prefetch_next(j + 1 >= U.nkv[1], false)) ok = false;
         }
-        if (elect_one()) {
-          tc_commit(bar(C::B_VEMPTY + s));                     // V_j: both P·V(·, j) issued
-          if (j + 1 < n_iter) tc_commit(bar(C::B_KEMPTY + s1));  // K_{j+1}: both S(·, j+1) issued
-        }
-        __syncwarp();
+        if (!ok || !prefetch_next(true, true)) break;
+        kc += U.n_iter;
+        vc += U.n_iter;
+        cur = nxt;
+        U = N;
       }
       // every MMA issued so far must finish before tensor memory is released
       if (elect_one()) {
@@ -348,18 +529,31 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     __syncwarp();
   } else {
     // ================================================================ softmax warpgroups
-    regs_inc<208>();
+    regs_inc<200>();
     const int t = warp >> 2;
     const int quarter = warp & 3;
-    const int my_nkv = (t == 0) ? nkv[0] : nkv[1];
-    if (my_nkv > 0) {
-      const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
-      const uint32_t tS = tmem + lane_off + 128u * t;
-      const uint32_t tO = tmem + lane_off + 256u + (uint32_t)(D * t);
-      const int row = q0 + t * kBM + 32 * quarter + lane;  // position in the sequence
-      const int key_limit = p.causal ? min(L, row + 1) : L;
-      const float c = p.scale_log2;
-      const float2 c2 = make_float2(c, c);
+    const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
+    const uint32_t tS = tmem + lane_off + 128u * t;
+    const uint32_t tO = tmem + lane_off + 256u + (uint32_t)(D * t);
+    const float c = p.scale_log2;
+    const float2 c2 = make_float2(c, c);
+    uint32_t un = 0;  // units read
+    uint32_t sn = 0;  // S tiles of Q tile t consumed (all units)
+    bool ok = true;
+    while (ok) {
+      const int us = un & 1;
+      if (!warp_wait(bar(C::B_UFULL + us), (un >> 1) & 1, wd)) break;
+      const int unit = unit_ring[us];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::B_UEMPTY + us));
+      ++un;
+      if (unit < 0) break;
+      FwdUnit U;
+      decode_unit(p, unit, U);
+      const int my_nkv = U.nkv[t];
+      if (my_nkv == 0) continue;
+      const int row = U.q0 + t * kBM + 32 * quarter + lane;  // position in the sequence
+      const int key_limit = p.causal ? min(U.L, row + 1) : U.L;
       // A tile whose rows see a single KV tile (the first 128 rows of a causal
       // sequence, or a sequence of at most 128 tokens) averages few values, so
       // the rounding of P to 16 bits would show in O: there P is carried as
@@ -367,9 +561,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const bool split_p = (my_nkv == 1);
       float m_ref = -INFINITY;  // running (possibly stale) max, scaled domain
       float ell = 0.f;
-      bool ok = true;
       for (int j = 0; j < my_nkv; ++j) {
-        if (!warp_wait(bar(C::B_SFULL + t), j & 1, wd)) { ok = false; break; }
+        const uint32_t step = sn + j;
+        if (!warp_wait(bar(C::B_SFULL + t), step & 1, wd)) { ok = false; break; }
         tc_fence_after();
         uint32_t sr[kBN];
 #pragma unroll
@@ -460,7 +654,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (__any_sync(0xffffffffu, rescale_o)) {
           // The reference max rose (rare past the first tile): O(t) must hold P·V(t, j-1) before it
           // is rescaled, and the rescale must land before P·V(t, j) is issued.
-          if (!warp_wait(bar(C::B_PVDONE + t), (j - 1) & 1, wd)) { ok = false; break; }
+          if (!warp_wait(bar(C::B_PVDONE + t), (step - 1) & 1, wd)) { ok = false; break; }
           tc_fence_after();
           const float f = rescale_o ? alpha : 1.f;
 #pragma unroll
@@ -478,11 +672,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         mbar_arrive(bar(C::B_PFULL + t));
       }
       // ---- epilogue: O / ℓ -> dtype, LSE
-      if (ok && warp_wait(bar(C::B_PVDONE + t), (my_nkv - 1) & 1, wd)) {
+      if (ok && warp_wait(bar(C::B_PVDONE + t), (sn + my_nkv - 1) & 1, wd)) {
         tc_fence_after();
-        const bool valid = row < L;
+        const bool valid = row < U.L;
         const float inv = (ell > 0.f) ? 1.f / ell : 0.f;
-        const size_t obase = ((size_t)(tok0 + (valid ? row : 0)) * p.H + h) * D;
+        const size_t obase = ((size_t)(U.tok0 + (valid ? row : 0)) * p.H + U.h) * D;
         uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) + obase * 2;
 #pragma unroll
         for (int q = 0; q < D / 32; ++q) {
@@ -502,9 +696,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (valid) {
           const float lse = (ell > 0.f && m_ref != -INFINITY) ? (m_ref + __log2f(ell)) * 0.69314718055994531f
                                                              : -INFINITY;
-          p.lse[(size_t)(tok0 + row) * p.H + h] = lse;
+          p.lse[(size_t)(U.tok0 + row) * p.H + U.h] = lse;
         }
+      } else {
+        ok = false;
       }
+      sn += my_nkv;
     }
     __syncwarp();
   }

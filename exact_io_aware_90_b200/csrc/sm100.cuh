@@ -76,6 +76,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking probe: has the phase with the given parity completed?
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Shared abort state of one CTA: set by the first wait that gives up, so the
 // other roles stop waiting too.
 struct Watchdog {
@@ -132,6 +145,39 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
 // async-proxy reads (tensor-core operands written with st.shared).
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ---------------------------------------------------------------- cluster launch control
+// Asks the hardware scheduler to cancel the launch of a CTA of this grid that
+// has not started yet, so that this (already running) CTA can do its work
+// instead.  The 16-byte response is written to shared memory (16-byte
+// aligned) by the async proxy and completes 16 transaction bytes on the
+// mbarrier, which the caller armed with arrive.expect_tx.
+__device__ __forceinline__ void clc_try_cancel(uint32_t resp_smem, uint32_t bar) {
+  asm volatile("clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 [%0], [%1];"
+               ::"r"(resp_smem), "r"(bar)
+               : "memory");
+}
+
+// Decodes a response: true and the cancelled CTA's x index if the request
+// succeeded, false once no CTA is left to take (no further request may be
+// made after that).
+__device__ __forceinline__ bool clc_query(uint32_t resp_smem, int& ctaid_x) {
+  uint32_t ok = 0, x = 0, y = 0, z = 0;
+  asm volatile(
+      "{\n\t"
+      ".reg .pred p;\n\t"
+      ".reg .b128 r;\n\t"
+      "ld.shared.b128 r, [%4];\n\t"
+      "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, r;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t"
+      "@p clusterlaunchcontrol.query_cancel.get_first_ctaid.v4.b32.b128 {%1, %2, %3, _}, r;\n\t"
+      "}"
+      : "+r"(ok), "+r"(x), "+r"(y), "+r"(z)
+      : "r"(resp_smem)
+      : "memory");
+  ctaid_x = (int)x;
+  return ok != 0;
 }
 
 // ---------------------------------------------------------------- tensor memory
