@@ -197,6 +197,8 @@ __device__ __forceinline__ void red_add_v4_f32(float* p, float a, float b, float
 // (K-major, BQ rows); K dim = d.
 template <int D, int BQ, uint32_t IDESC>
 __device__ __forceinline__ void bwd_issue_kt(uint32_t d_tmem, uint64_t da, uint64_t db) {
+  da = opaque64(da);
+  db = opaque64(db);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
     const uint32_t oa = ((kk >> 2) * (kBK * 128) + (kk & 3) * 32) >> 4;
@@ -209,6 +211,7 @@ __device__ __forceinline__ void bwd_issue_kt(uint32_t d_tmem, uint64_t da, uint6
 // B = dO or Q MN-major (+2 KB per 16 query rows); K dim = BQ.
 template <int BQ, uint32_t IDESC>
 __device__ __forceinline__ void bwd_issue_acc(uint32_t d_tmem, uint32_t a_tmem, uint64_t db, uint32_t acc) {
+  db = opaque64(db);
 #pragma unroll
   for (int kk = 0; kk < BQ / 16; ++kk) mma_ts(d_tmem, a_tmem + kk * 8, db + ((kk * 2048) >> 4), IDESC, kk > 0 ? 1u : acc);
 }
@@ -216,6 +219,8 @@ __device__ __forceinline__ void bwd_issue_acc(uint32_t d_tmem, uint32_t a_tmem, 
 // dQ partial: K dim = the 128 keys, both operands MN-major (+2 KB per 16 keys).
 template <uint32_t IDESC>
 __device__ __forceinline__ void bwd_issue_dq(uint32_t d_tmem, uint64_t da, uint64_t db) {
+  da = opaque64(da);
+  db = opaque64(db);
 #pragma unroll
   for (int kk = 0; kk < kBK / 16; ++kk) mma_ss(d_tmem, da + ((kk * 2048) >> 4), db + ((kk * 2048) >> 4), IDESC, kk > 0 ? 1u : 0u);
 }
@@ -536,12 +541,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tc_fence_before();
           mbar_arrive(bar(C::B_DPFREE));
         }
+        // −D of these 32 queries.  At BQ = 128 they are read here with loads the compiler cannot hoist
+        // (all 128 values would not fit in registers beside Pᵀ); at BQ = 64 the compiler may schedule
+        // them early, which measures faster.
+        float nd[32];
+        if constexpr (BQ == 128) {
+#pragma unroll
+          for (int v = 0; v < 8; ++v) ld_shared_v4f(del_s + 32 * q + 4 * v, nd + 4 * v);
+        } else {
+#pragma unroll
+          for (int v = 0; v < 32; ++v) nd[v] = del_s[32 * q + v];
+        }
         uint32_t dsk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int col = 32 * q + 2 * i;
           const float2 dd = __fadd2_rn(make_float2(__uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1])),
-                                       make_float2(del_s[col], del_s[col + 1]));
+                                       make_float2(nd[2 * i], nd[2 * i + 1]));
           const float2 ds = __fmul2_rn(make_float2(pt[col], pt[col + 1]), dd);
           dsk[i] = pack2<BF16>(ds.x, ds.y);
         }
@@ -602,12 +618,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_arrive(bar(C::B_DQFREE));
       if constexpr (D == 128) {
         // lane = feature, columns = 64 queries: each warp instruction covers 32 consecutive features
-        float* base = p.dq_acc + ((size_t)(tok0 + i0) * p.H + h) * D + lrow;
+        // one address register stepped by the row stride (64 precomputed addresses would not fit in 128 registers)
+        uint64_t addr = reinterpret_cast<uint64_t>(p.dq_acc + ((size_t)(tok0 + i0) * p.H + h) * D + lrow);
         const int nq = min(64, L - i0);
-        const size_t stride = (size_t)p.H * D;
+        const uint64_t stride = (uint64_t)p.H * D * sizeof(float);
 #pragma unroll
-        for (int q = 0; q < 64; ++q)
-          if (q < nq) red_add_f32(base + q * stride, __uint_as_float(qr[q]));
+        for (int q = 0; q < 64; ++q) {
+          if (q < nq) red_add_f32(reinterpret_cast<float*>(addr), __uint_as_float(qr[q]));
+          addr = opaque64(addr + stride);
+        }
       } else {
         // lane = query row, columns = 64 features
         const int qrow = i0 + lrow;

@@ -119,14 +119,6 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const W
 // S = Q·Kᵀ for one 128 × 128 tile: D/16 MMAs of K = 16 along the head dimension.
 // Q and K are K-major with 128-byte rows; a 16-element step is +32 bytes inside a
 // swizzle atom, a 64-element step the next 16 KB atom column.
-// Returns x unchanged but opaque to the compiler, so descriptors derived from it
-// are formed at the issue site instead of being kept live across the MMA loop
-// (the MMA warp runs with 104 registers).
-__device__ __forceinline__ uint64_t opaque64(uint64_t x) {
-  asm volatile("mov.b64 %0, %0;" : "+l"(x));
-  return x;
-}
-
 template <int D, uint32_t IDESC>
 __device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint64_t dq, uint64_t dk) {
   dq = opaque64(dq);

@@ -147,6 +147,22 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Returns x unchanged but opaque to the compiler, so that shared-memory
+// descriptors derived from it (base + constant offset per MMA) are formed at
+// the issue site instead of being hoisted and kept live across a whole loop
+// in the register-starved MMA-issuing warp.
+__device__ __forceinline__ uint64_t opaque64(uint64_t x) {
+  asm volatile("mov.b64 %0, %0;" : "+l"(x));
+  return x;
+}
+
+// 16-byte shared-memory load that the compiler does not move across other volatile asm.
+__device__ __forceinline__ void ld_shared_v4f(const float* p, float* out) {
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(out[0]), "=f"(out[1]), "=f"(out[2]), "=f"(out[3])
+               : "r"(smem_u32(p)));
+}
+
 // ---------------------------------------------------------------- cluster launch control
 // Asks the hardware scheduler to cancel the launch of a CTA of this grid that
 // has not started yet, so that this (already running) CTA can do its work

@@ -193,3 +193,66 @@ def test_watchdog_gives_up_and_context_survives(fa):
     assert fa.fa_watchdog_selftest(20_000_000, stream) == fa.FA_ERR_TIMEOUT
     assert fa.fa_check_device_status(stream) == fa.FA_OK  # cleared
     _check_fwd(fa, workloads.random_inputs(1, 64, "bf16", seed=1, B=1, N=129, backward=False))
+
+
+def _fwd_on(fa, inp, stream):
+    dev = torch.device("cuda")
+    q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
+    cu = None if inp.cu_seqlens is None else inp.cu_seqlens.to(dev)
+    torch.cuda.synchronize()
+    kw = dict(causal=inp.causal, scale=inp.scale, cu_seqlens=cu, max_seqlen=inp.N if cu is not None else None,
+              batch=inp.B)
+    return (q, k, v, kw), lambda: fa.attention_forward(q, k, v, stream=stream, **kw)
+
+
+@pytest.mark.parametrize("varlen", [False, True])
+def test_persistent_scheduling_is_repeatable(fa, varlen):
+    """More units than SMs, so running CTAs take further units from the scheduler in an order that
+    changes from call to call; every unit is still computed whole by one CTA, so the outputs are
+    bit-identical across calls (a unit computed twice, skipped or mixed up between CTAs would show)."""
+    if varlen:
+        inp = workloads.random_inputs(8, 128, "bf16", seed=31, B=6, N=3000, causal=True, backward=False,
+                                      seqlens=[3000, 1, 0, 700, 2049, 129])
+    else:
+        inp = workloads.random_inputs(8, 128, "bf16", seed=30, B=2, N=4096, causal=True, backward=False)
+    stream = torch.cuda.current_stream().cuda_stream
+    _, run = _fwd_on(fa, inp, stream)
+    o0, l0 = run()
+    o0, l0 = o0.clone(), l0.clone()
+    for _ in range(3):
+        o, l = run()
+        assert fa.fa_check_device_status(stream) == fa.FA_OK
+        rows = torch.as_tensor(covered_rows(inp))
+        assert torch.equal(o[rows], o0[rows]) and torch.equal(l[rows], l0[rows])
+    rows = _sampled_rows(inp, 64, seed=5 + int(varlen))
+    cu = None if inp.cu_seqlens is None else inp.cu_seqlens.numpy()
+    O_ref, L_ref = oracle.attention_forward_rows(inp.q, inp.k, inp.v, rows, inp.scale, inp.causal, cu_seqlens=cu,
+                                                 B=inp.B, N=inp.N if cu is None else None)
+    assert max_abs(f64(o0[torch.as_tensor(rows)]), O_ref) <= O_TOL
+    assert max_abs(f64(l0[torch.as_tensor(rows)]), L_ref) <= LSE_TOL
+
+
+def test_concurrent_launches_on_two_streams(fa):
+    """Two forwards in flight at once on different streams: a CTA only ever takes units of its own
+    grid, so each result equals the same call run alone."""
+    a = workloads.random_inputs(8, 128, "bf16", seed=40, B=2, N=2048, causal=True, backward=False)
+    b = workloads.random_inputs(4, 64, "fp16", seed=41, B=3, N=1500, causal=False, backward=False)
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    _, run_a = _fwd_on(fa, a, s1.cuda_stream)
+    _, run_b = _fwd_on(fa, b, s2.cuda_stream)
+    # references: each call alone (synchronised before its outputs are read on the default stream)
+    out = run_a()
+    torch.cuda.synchronize()
+    ref_a = [t.clone() for t in out]
+    out = run_b()
+    torch.cuda.synchronize()
+    ref_b = [t.clone() for t in out]
+    for _ in range(3):
+        got_a = run_a()
+        got_b = run_b()
+        torch.cuda.synchronize()
+        assert fa.fa_check_device_status(s1.cuda_stream) == fa.FA_OK
+        assert all(torch.equal(x, y) for x, y in zip(got_a, ref_a))
+        assert all(torch.equal(x, y) for x, y in zip(got_b, ref_b))
+    O_ref, L_ref = oracle_forward(b)
+    assert max_abs(f64(ref_b[0]), O_ref) <= O_TOL and max_abs(f64(ref_b[1]), L_ref) <= LSE_TOL
