@@ -557,9 +557,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const uint32_t step = sn + j;
         if (!warp_wait(bar(C::B_SFULL + t), step & 1, wd)) { ok = false; break; }
         tc_fence_after();
+        // one 128-column load and one 64-column store per tile: fewer, larger tensor-memory accesses
+        // slow the MMAs running at the same time less than 32-column pieces of the same bytes
         uint32_t sr[kBN];
-#pragma unroll
-        for (int q = 0; q < kBN / 32; ++q) tmem_ld32(tS + 32u * q, reinterpret_cast<uint32_t(&)[32]>(sr[32 * q]));
+        tmem_ld128(tS, sr);
         tmem_wait_ld();
         float sv[kBN];
 #pragma unroll
@@ -592,36 +593,28 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         if (!split_p && !need_mask && PolyMask<D>::value != 0u) {
           // unmasked tile: part of the exponentials on the FMA pipe, interleaved with the MUFU ones
+          uint32_t pk[64];
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            uint32_t pk[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int idx = 64 * q + 2 * i;
-              const float2 x = __ffma2_rn(make_float2(sv[idx], sv[idx + 1]), c2, nm2);
-              float2 e;
-              if ((PolyMask<D>::value >> (i & 7)) & 1u) e = exp2_poly2(x);
-              else e = make_float2(ex2(x.x), ex2(x.y));
-              acc[i & 3] = __fadd2_rn(acc[i & 3], e);
-              pk[i] = pack2<BF16>(e.x, e.y);
-            }
-            tmem_st32(tS + 32u * q, pk);
+          for (int i = 0; i < 64; ++i) {
+            const float2 x = __ffma2_rn(make_float2(sv[2 * i], sv[2 * i + 1]), c2, nm2);
+            float2 e;
+            if ((PolyMask<D>::value >> (i & 7)) & 1u) e = exp2_poly2(x);
+            else e = make_float2(ex2(x.x), ex2(x.y));
+            acc[i & 3] = __fadd2_rn(acc[i & 3], e);
+            pk[i] = pack2<BF16>(e.x, e.y);
           }
+          tmem_st64(tS, pk);
         } else if (!split_p) {
           // P = 2^(c·s − m) on the MUFU (ex2(−inf) = 0 exactly), packed to 16 bits, written over S
+          uint32_t pk[64];
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            uint32_t pk[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int idx = 64 * q + 2 * i;
-              const float2 x = __ffma2_rn(make_float2(sv[idx], sv[idx + 1]), c2, nm2);
-              const float2 e = make_float2(ex2(x.x), ex2(x.y));
-              acc[i & 3] = __fadd2_rn(acc[i & 3], e);
-              pk[i] = pack2<BF16>(e.x, e.y);
-            }
-            tmem_st32(tS + 32u * q, pk);
+          for (int i = 0; i < 64; ++i) {
+            const float2 x = __ffma2_rn(make_float2(sv[2 * i], sv[2 * i + 1]), c2, nm2);
+            const float2 e = make_float2(ex2(x.x), ex2(x.y));
+            acc[i & 3] = __fadd2_rn(acc[i & 3], e);
+            pk[i] = pack2<BF16>(e.x, e.y);
           }
+          tmem_st64(tS, pk);
         } else {
           // P = hi + lo, both in the input dtype: hi in columns [0, 64), lo in [64, 128)
 #pragma unroll
