@@ -43,6 +43,19 @@ bool encode_tmap(CUtensorMap* map, const void* base, int T, int H, int d, bool b
   return r == CUDA_SUCCESS;
 }
 
+bool encode_tmap_f32(CUtensorMap* map, const void* base, int T, int H, int d, int rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T};
+  const cuuint64_t strides[2] = {(cuuint64_t)d * 4, (cuuint64_t)H * d * 4};
+  const cuuint32_t box[3] = {32, 1, (cuuint32_t)rows};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 static bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 static bool aligned4(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
@@ -147,7 +160,8 @@ int fa_bwd_main(const void* q, const void* k, const void* v, const float* lse, c
   // Q and dO stream in tiles of 64 rows at d = 128 and 128 rows at d = 64; K and V in 128-row tiles
   const int bq = (d == 128) ? 64 : 128;
   if (!encode_tmap(&a.tm_q, q, pb.T, H, d, pb.bf16, bq) || !encode_tmap(&a.tm_k, k, pb.T, H, d, pb.bf16, 128) ||
-      !encode_tmap(&a.tm_v, v, pb.T, H, d, pb.bf16, 128) || !encode_tmap(&a.tm_do, dO, pb.T, H, d, pb.bf16, bq))
+      !encode_tmap(&a.tm_v, v, pb.T, H, d, pb.bf16, 128) || !encode_tmap(&a.tm_do, dO, pb.T, H, d, pb.bf16, bq) ||
+      !encode_tmap_f32(&a.tm_dq, a.dq_acc, pb.T, H, d, bq))
     return FA_ERR_UNSUPPORTED;
   a.q = q;
   a.k = k;

@@ -147,7 +147,9 @@ struct BwdCfg {
   static constexpr int B_DQFULL = B_DSREADY + 1;
   static constexpr int B_DQFREE = B_DQFULL + 1;
   static constexpr int B_DSFREE = B_DQFREE + 1;   // [NDS]: dK and dQ have read dSᵀ buffer b
-  static constexpr int B_DKV = B_DSFREE + NDS;
+  static constexpr int B_DQSFREE = B_DSFREE + NDS;  // [2] dQ staging buffer b may be written
+  static constexpr int B_DQSFULL = B_DQSFREE + 2;   // [2] dQ staging buffer b written (128 arrivals)
+  static constexpr int B_DKV = B_DQSFULL + 2;
   static constexpr int B_DRAIN = B_DKV + 1;
   static constexpr int NBARS = B_DRAIN + 1;
   // shared memory
@@ -156,10 +158,16 @@ struct BwdCfg {
   static constexpr uint32_t OFF_Q = 2 * KV_TILE;
   static constexpr uint32_t OFF_DO = OFF_Q + STAGES * Q_TILE;
   static constexpr uint32_t OFF_DS = OFF_DO + STAGES * Q_TILE;
-  static constexpr uint32_t OFF_ROW = OFF_DS + NDS * DS_TILE;  // per stage: −lse·log2(e)[BQ], −D[BQ] (fp32)
+  // dQ partial staging for the TMA reduce-add: 2 buffers of D/32 boxes [BQ rows × 32 fp32], 128-byte swizzle
+  static constexpr int NBOX = D / 32;
+  static constexpr uint32_t DQ_BOX = BQ * 128;
+  static constexpr uint32_t DQ_TILE = NBOX * DQ_BOX;
+  static constexpr uint32_t OFF_DQS = OFF_DS + NDS * DS_TILE;
+  static constexpr uint32_t OFF_ROW = OFF_DQS + 2 * DQ_TILE;  // per stage: −lse·log2(e)[BQ], −D[BQ] (fp32)
   static constexpr uint32_t OFF_BAR = OFF_ROW + STAGES * 2 * BQ * 4;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
   static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   // registers per thread after setmaxnreg (block of 384 launched at 168: 3 × 168 = 504 per lane triple)
   static constexpr uint32_t REGS_CMP = 256;  // Pᵀ / dSᵀ warpgroup
   static constexpr uint32_t REGS_DQ = 128;   // dQ warpgroup
@@ -180,14 +188,6 @@ __device__ __forceinline__ void drain_wait_b(uint32_t bar, uint32_t parity, uint
 __device__ __forceinline__ bool warp_wait_b(uint32_t bar, uint32_t parity, const Watchdog& wd) {
   const bool ok = mbar_wait(bar, parity, wd);
   return __all_sync(0xffffffffu, ok);
-}
-
-__device__ __forceinline__ void red_add_f32(float* p, float v) {
-  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
-}
-
-__device__ __forceinline__ void red_add_v4_f32(float* p, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
 }
 
 // Products of one Q tile, issued by one elected lane.  Descriptor arguments
@@ -229,7 +229,7 @@ template <int D, bool BF16>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                       const BwdParams p) {
+                       const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using C = BwdCfg<D>;
   constexpr int BQ = C::BQ;
   // Sᵀ = K Qᵀ and dPᵀ = V dOᵀ: M = 128 keys, N = BQ, both operands K-major
@@ -308,6 +308,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(bar(C::B_DQFULL), 1);
     mbar_init(bar(C::B_DQFREE), 128);
     for (int b = 0; b < C::NDS; ++b) mbar_init(bar(C::B_DSFREE + b), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(C::B_DQSFREE + b), 1);
+      mbar_init(bar(C::B_DQSFULL + b), 128);
+    }
     mbar_init(bar(C::B_DKV), 1);
     mbar_init(bar(C::B_DRAIN), 1);
     *abort_flag = 0;
@@ -318,6 +322,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
     prefetch_tmap(&tm_do);
+    prefetch_tmap(&tm_dq);
   }
   tc_fence_before();
   __syncthreads();
@@ -605,6 +610,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t tDQ = tmem + lane_off + C::T_DQ;
     const uint32_t tDK = tmem + lane_off + C::T_DK;
     const int lrow = 32 * quarter + lane;  // tensor-memory lane of this thread
+    const bool issuer = (warp == 4 && lane == 0);
+    const uint32_t sDQS = s_base + C::OFF_DQS;
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
       const int i0 = (i_begin + it) * BQ;
@@ -616,29 +623,48 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(bar(C::B_DQFREE));
+      // The partial goes to the fp32 accumulator by TMA reduce-add from a shared-memory staging buffer
+      // (coalesced, asynchronous).  Buffer b = it & 1 is written once the reduce issued from it two
+      // steps ago has read it; the issuing thread signals that, and issues the next reduce when all
+      // 128 threads have written.  Rows past the end of the sequence hold exact zeros (P is 0 there),
+      // rows past T are clipped by the TMA unit.
+      const int b = it & 1;
+      const uint32_t u = (uint32_t)it >> 1;  // use of buffer b
+      const uint32_t buf = sDQS + b * C::DQ_TILE;
+      if (issuer) {
+        if (it >= 2) bulk_wait_group_read<1>();
+        mbar_arrive(bar(C::B_DQSFREE + b));
+      }
+      if (!warp_wait_b(bar(C::B_DQSFREE + b), u & 1, wd)) { ok = false; break; }
       if constexpr (D == 128) {
-        // lane = feature, columns = 64 queries: each warp instruction covers 32 consecutive features
-        // one address register stepped by the row stride (64 precomputed addresses would not fit in 128 registers)
-        uint64_t addr = reinterpret_cast<uint64_t>(p.dq_acc + ((size_t)(tok0 + i0) * p.H + h) * D + lrow);
-        const int nq = min(64, L - i0);
-        const uint64_t stride = (uint64_t)p.H * D * sizeof(float);
+        // dQᵀ: lane = feature 32·quarter + lane (box `quarter`), columns = 64 queries (box rows)
+        const uint32_t box = buf + quarter * C::DQ_BOX + ((lane & 3) << 2);
 #pragma unroll
-        for (int q = 0; q < 64; ++q) {
-          if (q < nq) red_add_f32(reinterpret_cast<float*>(addr), __uint_as_float(qr[q]));
-          addr = opaque64(addr + stride);
-        }
+        for (int q = 0; q < 64; ++q) st_shared_f32(box + q * 128 + ((((lane >> 2) ^ (q & 7))) << 4), qr[q]);
       } else {
-        // lane = query row, columns = 64 features
-        const int qrow = i0 + lrow;
-        if (qrow < L) {
-          float* base = p.dq_acc + ((size_t)(tok0 + qrow) * p.H + h) * D;
+        // dQ: lane = query row (box row), columns = 64 features (boxes 0 and 1)
 #pragma unroll
-          for (int f = 0; f < 64; f += 4)
-            red_add_v4_f32(base + f, __uint_as_float(qr[f]), __uint_as_float(qr[f + 1]), __uint_as_float(qr[f + 2]),
-                           __uint_as_float(qr[f + 3]));
+        for (int k = 0; k < 2; ++k)
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            st_shared_v4(buf + k * C::DQ_BOX + lrow * 128 + ((j ^ (lrow & 7)) << 4), qr[32 * k + 4 * j],
+                         qr[32 * k + 4 * j + 1], qr[32 * k + 4 * j + 2], qr[32 * k + 4 * j + 3]);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bar(C::B_DQSFULL + b));
+      bool fail = false;
+      if (issuer) {
+        if (mbar_wait(bar(C::B_DQSFULL + b), u & 1, wd)) {
+#pragma unroll
+          for (int k = 0; k < C::NBOX; ++k) tma_reduce_add_3d(&tm_dq, buf + k * C::DQ_BOX, 32 * k, h, tok0 + i0);
+          bulk_commit_group();
+        } else {
+          fail = true;
         }
       }
+      if (__any_sync(0xffffffffu, fail)) { ok = false; break; }  // the whole warp leaves together
     }
+    if (issuer) bulk_wait_group_all();  // every reduce performed before the kernel ends
     // ---- epilogue: dK rows (× scale)
     if (ok && warp_wait_b(bar(C::B_DKV), 0, wd)) {
       tc_fence_after();
@@ -748,7 +774,7 @@ static cudaError_t launch_main_t(const Problem& pb, const BwdArgs& a, cudaStream
   p.scale_log2 = pb.scale * 1.4426950408889634f;
   p.timeout_ns = pb.timeout_ns;
   const long long units = (long long)pb.B * pb.H * p.num_kblocks;
-  kern<<<dim3((unsigned)units), dim3(kBwdThreads), C::SMEM_BYTES, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, p);
+  kern<<<dim3((unsigned)units), dim3(kBwdThreads), C::SMEM_BYTES, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, a.tm_dq, p);
   return cudaPeekAtLastError();
 }
 

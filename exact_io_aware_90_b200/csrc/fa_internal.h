@@ -27,6 +27,7 @@ struct FwdArgs {
 
 struct BwdArgs {
   CUtensorMap tm_q, tm_k, tm_v, tm_do;
+  CUtensorMap tm_dq;  // the fp32 dQ accumulator, for TMA reduce-add
   const void* q;
   const void* k;
   const float* lse;
@@ -42,6 +43,10 @@ struct BwdArgs {
 // Encodes a [T, H, d] 16-bit tensor as a 3-D TMA map with 128-byte swizzle
 // and a box of 64 features × 1 head × `rows` tokens.  Returns false on failure.
 bool encode_tmap(CUtensorMap* map, const void* base, int T, int H, int d, bool bf16, int rows);
+
+// Encodes a [T, H, d] fp32 tensor as a 3-D TMA map with 128-byte swizzle and a
+// box of 32 features × 1 head × `rows` tokens.  Returns false on failure.
+bool encode_tmap_f32(CUtensorMap* map, const void* base, int T, int H, int d, int rows);
 
 cudaError_t launch_fwd(const Problem& pb, const FwdArgs& a, cudaStream_t stream);
 cudaError_t launch_bwd_pre(const Problem& pb, const BwdArgs& a, cudaStream_t stream);
