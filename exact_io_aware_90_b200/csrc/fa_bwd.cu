@@ -19,9 +19,10 @@
 //                         dSᵀ = Pᵀ ∘ (dPᵀ − D_i)                  (warps 0-3)
 //                         dK += dSᵀ Q_i         (dSᵀ read from tensor memory)
 //                         dQ_i partial = dS K_j (dSᵀ staged in shared memory)
-//                       and warps 4-7 add the dQ partial into the fp32
-//                       accumulator with vector reductions.  dK (× scale)
-//                       and dV are written once at the end.
+//                       and warps 4-7 stage the dQ partial in shared memory,
+//                       from where TMA reduce-adds it into the fp32
+//                       accumulator.  dK (× scale) and dV are written once
+//                       at the end.
 //   fa_bwd_post_kernel  dq = scale · accumulator, rounded to the dtype
 // All five MMAs are M = 128 (full tensor-core rate): at d = 128 the dQ
 // product is formed transposed, dQᵀ = K_jᵀ dSᵀ (M = d), at d = 64 directly
