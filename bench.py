@@ -317,6 +317,34 @@ def run_gpu(args, world, rank, local, pg):
     if st != fa.FA_OK:
         raise fa.FAError(st, "e2e steps")
 
+    # ---- the forward alone (inference use): same workload, same L2 flush, back-to-back steps
+    fwd_only = None
+    if backward:
+        for _ in range(args.warmup):
+            flush.fill_(1)
+            fwd()
+        torch.cuda.synchronize(dev)
+        fo_clocks = ClockSampler(dev)
+        if pg is not None:
+            pg.barrier()
+        torch.cuda.synchronize(dev)
+        fo_clocks.start()
+        fo = []
+        for _ in range(args.steps):
+            flush.fill_(1)  # outside the timed events
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fwd()
+            b.record(stream)
+            fo.append((a, b))
+        torch.cuda.synchronize(dev)
+        fo_clk = fo_clocks.stop()
+        st = fa.fa_check_device_status(sp)
+        if st != fa.FA_OK:
+            raise fa.FAError(st, "forward-only steps")
+        fo_ms = max_over_ranks(float(np.mean([x.elapsed_time(y) for x, y in fo])), pg, dev)
+        fwd_only = {"ms": round(fo_ms, 4), "tflops": round(flops_fwd / (fo_ms * 1e-3) / 1e12, 1), "clocks": fo_clk}
+
     # ---- roofline of the dominant kernel
     peaks = load_peaks()
     dom = max(per_kernel, key=per_kernel.get)
@@ -359,6 +387,10 @@ def run_gpu(args, world, rank, local, pg):
         "fwd_tflops": round(flops_fwd / (per_kernel["fa_fwd_kernel"] * 1e-3) / 1e12, 1),
         "fwd_frac_of_peak": round(flops_fwd / (per_kernel["fa_fwd_kernel"] * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
         "pct_of_peak": round(100.0 * value / world / peaks["bf16_tflops"], 2),
+        # the forward kernel timed in a forward-only loop (inference use; the fwd+bwd step above times it right
+        # after the previous step's backward)
+        "fwd_only": (None if fwd_only is None else
+                     dict(fwd_only, frac_of_peak=round(fwd_only["tflops"] / peaks["bf16_tflops"], 4))),
         "kernels": kernels,
         "roofline": roof,
         "e2e": {"value": round(world * flops_step / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
