@@ -36,6 +36,10 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+# NVIDIA's datasheet dense BF16 tensor figure for one B200 (its doubled figure assumes 2:4 sparsity);
+# reported beside the measured cuBLAS peak, which is the denominator of every `frac_of_peak`.
+NOMINAL_DENSE_BF16_TFLOPS = 2250.0
+NOMINAL_SOURCE = "NVIDIA B200 datasheet, dense BF16 (2.25 PFLOP/s; 4.5 with 2:4 sparsity)"
 METRIC = "attention TFLOP/s (fwd, fwd+bwd) on 1 B200 and % of dense bf16 tensor peak"
 DEFAULT_WORKLOAD = "causal_n8k_d128"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
@@ -390,7 +394,11 @@ def run_gpu(args, world, rank, local, pg):
         # the forward kernel timed in a forward-only loop (inference use; the fwd+bwd step above times it right
         # after the previous step's backward)
         "fwd_only": (None if fwd_only is None else
-                     dict(fwd_only, frac_of_peak=round(fwd_only["tflops"] / peaks["bf16_tflops"], 4))),
+                     dict(fwd_only, frac_of_peak=round(fwd_only["tflops"] / peaks["bf16_tflops"], 4),
+                          frac_of_sustained=round(fwd_only["tflops"] / peaks.get("bf16_tflops_sustained",
+                                                                                 peaks["bf16_tflops"]), 4),
+                          frac_of_nominal=round(fwd_only["tflops"] / NOMINAL_DENSE_BF16_TFLOPS, 4))),
+        "nominal_peak": {"tflops": NOMINAL_DENSE_BF16_TFLOPS, "source": NOMINAL_SOURCE},
         "kernels": kernels,
         "roofline": roof,
         "e2e": {"value": round(world * flops_step / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
