@@ -13,6 +13,10 @@ Parity status of each function (what pins it; see ``tests/test_oracle.py``):
                           to the rows.
 * online_blockwise_forward, online_softmax_stats, merge_softmax_stats
                           pinned: the pages' printed numbers.
+* decode_forward          pinned: the pages' hand example (last query row),
+                          the last row of causal self-attention, brute force.
+* split_kv_decode         pinned: equals decode_forward for every chunk size;
+                          chunk = 1 reduces to the page's per-element recurrence.
 """
 from .attention import *  # noqa: F401,F403
 from .attention import __all__  # noqa: F401

@@ -62,6 +62,8 @@ __all__ = [
     "online_softmax_stats",
     "merge_softmax_stats",
     "attention_flops",
+    "decode_forward",
+    "split_kv_decode",
 ]
 
 
@@ -356,3 +358,85 @@ def attention_flops(seqlens: Sequence[int], H: int, d: int, causal: bool, backwa
     if causal:
         f *= 0.5
     return f * 2.5 if backward else f
+
+
+# ----------------------------------------------------------------------------- decode (one query per sequence)
+
+
+def _key_segments(Tk: int, B: int, Nk: Optional[int], cu_seqlens_k) -> List[Tuple[int, int]]:
+    if cu_seqlens_k is not None:
+        cu = [int(c) for c in np.asarray(cu_seqlens_k).reshape(-1)]
+        return [(cu[b], cu[b + 1]) for b in range(len(cu) - 1)]
+    if Nk is None or B * Nk != Tk:
+        raise ValueError("dense key layout needs B·Nk == Tk")
+    return [(b * Nk, (b + 1) * Nk) for b in range(B)]
+
+
+def decode_forward(q, k, v, scale: float, cu_seqlens_k=None, B: Optional[int] = None, Nk: Optional[int] = None):
+    """Attention of one new query token per sequence over all keys of that sequence
+    (token-by-token decoding, the workload FlashAttention 短片讲解稿 "适用范围与关键结论"
+    sets apart): the same definition as ``attention_forward`` with a single query row
+    and no mask, since every cached key precedes or is the current token.
+
+    q: [B, H, d]; k, v: [Tk, H, d] with sequence b's keys at rows
+    [cu_seqlens_k[b], cu_seqlens_k[b+1]) (or b·Nk … without cu_seqlens_k).
+    Returns O [B, H, d] and LSE [B, H] (natural log) in float64; a sequence with
+    no key gets O = 0 and LSE = −∞.
+    """
+    Q, K, V = _f64(q), _f64(k), _f64(v)
+    Bq, H, d = Q.shape
+    segs = _key_segments(K.shape[0], Bq if B is None else B, Nk, cu_seqlens_k)
+    if len(segs) != Bq:
+        raise ValueError("one query per sequence")
+    O = np.zeros((Bq, H, d))
+    LSE = np.full((Bq, H), -np.inf)
+    for b, (lo, hi) in enumerate(segs):
+        if hi <= lo:
+            continue
+        for h in range(H):
+            s = (K[lo:hi, h] @ Q[b, h]) * scale          # [L] scores
+            m = s.max()
+            e = np.exp(s - m)
+            O[b, h] = (e @ V[lo:hi, h]) / e.sum()
+            LSE[b, h] = m + math.log(e.sum())
+    return O, LSE
+
+
+def split_kv_decode(q, k, v, scale: float, chunk: int, cu_seqlens_k=None, B: Optional[int] = None,
+                    Nk: Optional[int] = None, return_partials: bool = False):
+    """Decode by splitting each sequence's keys into chunks of ``chunk`` keys, each
+    reduced on its own to a partial (m_c, ℓ_c, Õ_c = Σ_j e^{s_j − m_c} v_j), then
+    merged in the form FlashAttention 与算子融合 gives for combining blocks
+    ("FlashAttention 的两个关键", online softmax):
+        m = max_c m_c,  ℓ = Σ_c ℓ_c·e^{m_c − m},  O = Σ_c Õ_c·e^{m_c − m} / ℓ
+    (the output partial sums scaled the same way as ℓ).  Chunks are merged one at
+    a time with ``merge_softmax_stats`` for (m, ℓ).  Mathematically equal to
+    ``decode_forward``; it exists to pin the merge the GPU path performs.
+    """
+    Q, K, V = _f64(q), _f64(k), _f64(v)
+    Bq, H, d = Q.shape
+    segs = _key_segments(K.shape[0], Bq if B is None else B, Nk, cu_seqlens_k)
+    O = np.zeros((Bq, H, d))
+    LSE = np.full((Bq, H), -np.inf)
+    partials = []
+    for b, (lo, hi) in enumerate(segs):
+        for h in range(H):
+            m, ell, acc = -math.inf, 0.0, np.zeros(d)
+            parts = []
+            for c0 in range(lo, hi, chunk):
+                c1 = min(hi, c0 + chunk)
+                s = (K[c0:c1, h] @ Q[b, h]) * scale
+                m_c = float(s.max())
+                e = np.exp(s - m_c)
+                l_c, O_c = float(e.sum()), e @ V[c0:c1, h]
+                parts.append((m_c, l_c, O_c))
+                m_new, ell = merge_softmax_stats(m, ell, m_c, l_c)
+                acc = (acc * math.exp(m - m_new) if m > -math.inf else 0.0) + O_c * math.exp(m_c - m_new)
+                m = m_new
+            partials.append(parts)
+            if ell > 0:
+                O[b, h] = acc / ell
+                LSE[b, h] = m + math.log(ell)
+    if return_partials:
+        return O, LSE, partials
+    return O, LSE

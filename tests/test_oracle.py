@@ -457,3 +457,123 @@ def test_pins_catch_planted_mistakes(monkeypatch):
         mp.setattr(A, "attention_backward", bwd_no_dk_scale)
         mp.setattr(oracle, "attention_backward", bwd_no_dk_scale)
         assert not _pins_pass()
+
+
+# ----------------------------------------------------------------------------- decode (one query per sequence)
+
+
+def _decode_pins_pass(decode, split=None):
+    """The decode pins, run against a given implementation (the oracle's, or a planted mistake)."""
+    try:
+        # the hand example: the one query row scores ln c_j against the four keys → O = 29, LSE = ln 10
+        ex, q, k, v, scale = _hand_qkv()
+        O, L = decode(q[:1, :, :], k, v, scale, B=1, Nk=4)
+        assert abs(O[0, 0, 0] - ex["full"]["result"]) < 1e-12
+        assert abs(L[0, 0] - math.log(ex["full"]["weight_total"])) < 1e-12
+        # the last row of causal self-attention (pinned above) is a decode step of the last token
+        rng = np.random.default_rng(7)
+        for Lk in (1, 5, 17):
+            Q, K, V = _rand(rng, Lk, 2, 4)
+            O_ref, L_ref = oracle.attention_forward(Q * 3.0, K, V, 0.37, causal=True)
+            O, L = decode(Q[Lk - 1:] * 3.0, K, V, 0.37, B=1, Nk=Lk)
+            assert np.abs(O[0] - O_ref[Lk - 1]).max() < 1e-12 and np.abs(L[0] - L_ref[Lk - 1]).max() < 1e-12
+        # brute force with scalar loops on a tiny packed batch, one sequence empty
+        q = rng.standard_normal((3, 1, 3))
+        k = rng.standard_normal((6, 1, 3))
+        v = rng.standard_normal((6, 1, 3))
+        cu = [0, 4, 4, 6]
+        O, L = decode(q, k, v, 0.8, cu_seqlens_k=cu)
+        for b in range(3):
+            lo, hi = cu[b], cu[b + 1]
+            if hi == lo:
+                assert np.all(O[b] == 0.0) and L[b, 0] == -math.inf
+                continue
+            w = [math.exp(0.8 * sum(q[b, 0, c] * k[j, 0, c] for c in range(3))) for j in range(lo, hi)]
+            tot = sum(w)
+            for c in range(3):
+                assert abs(O[b, 0, c] - sum(w[j - lo] * v[j, 0, c] for j in range(lo, hi)) / tot) < 1e-12
+            assert abs(L[b, 0] - math.log(tot)) < 1e-12
+        # large scores must not overflow (the max is subtracted first): every score is about 2400
+        q = np.full((1, 1, 2), 40.0)
+        k = 30.0 + rng.standard_normal((8, 1, 2))
+        v = rng.standard_normal((8, 1, 2))
+        O, L = decode(q, k, v, 1.0, B=1, Nk=8)
+        assert np.all(np.isfinite(O)) and np.isfinite(L[0, 0])
+        if split is not None:
+            q = rng.standard_normal((4, 3, 8))
+            k = rng.standard_normal((50, 3, 8))
+            v = rng.standard_normal((50, 3, 8))
+            cu = [0, 20, 20, 33, 50]
+            O_ref, L_ref = decode(q, k, v, 0.5, cu_seqlens_k=cu)
+            for chunk in (1, 2, 3, 7, 16, 20, 64):
+                O, L = split(q, k, v, 0.5, chunk, cu_seqlens_k=cu)
+                assert np.abs(O - O_ref).max() < 1e-12
+                fin = np.isfinite(L_ref)
+                assert np.all(fin == np.isfinite(L)) and np.abs(L[fin] - L_ref[fin]).max() < 1e-12
+        return True
+    except (AssertionError, FloatingPointError, ValueError, IndexError):
+        return False
+
+
+def test_decode_oracle_pins():
+    assert _decode_pins_pass(oracle.decode_forward, oracle.split_kv_decode)
+
+
+def test_split_kv_chunk_of_one_is_the_per_element_recurrence():
+    """With one key per chunk, the merged (m, ℓ) after each key are the page's running statistics."""
+    rng = np.random.default_rng(11)
+    q = rng.standard_normal((1, 1, 4))
+    k = rng.standard_normal((9, 1, 4))
+    v = rng.standard_normal((9, 1, 4))
+    scores = [0.5 * float(k[j, 0] @ q[0, 0]) for j in range(9)]
+    _, _, parts = oracle.split_kv_decode(q, k, v, 0.5, 1, B=1, Nk=9, return_partials=True)
+    stats = oracle.online_softmax_stats(scores, [1] * 9)
+    m, ell = -math.inf, 0.0
+    for j, ((m_c, l_c, O_c), (m_ref, l_ref)) in enumerate(zip(parts[0], stats)):
+        # one key: its own score is the max, the sum is e^0 = 1 and the partial output is that key's value
+        assert m_c == pytest.approx(scores[j], abs=1e-15) and l_c == 1.0
+        assert np.array_equal(O_c, v[j, 0])
+        m, ell = oracle.merge_softmax_stats(m, ell, m_c, l_c)
+        assert m == pytest.approx(m_ref, abs=1e-15) and ell == pytest.approx(l_ref, rel=1e-14)
+
+
+def test_decode_pins_catch_planted_mistakes():
+    def no_scale(q, k, v, scale, cu_seqlens_k=None, B=None, Nk=None):
+        return oracle.decode_forward(q, k, v, 1.0, cu_seqlens_k, B, Nk)
+
+    def no_max_shift(q, k, v, scale, cu_seqlens_k=None, B=None, Nk=None):
+        Q, K, V = (np.asarray(t, dtype=np.float64) for t in (q, k, v))
+        segs = A._key_segments(K.shape[0], Q.shape[0] if B is None else B, Nk, cu_seqlens_k)
+        O = np.zeros(Q.shape)
+        L = np.full(Q.shape[:2], -np.inf)
+        with np.errstate(over="raise"):
+            for b, (lo, hi) in enumerate(segs):
+                for h in range(Q.shape[1]):
+                    if hi > lo:
+                        e = np.exp((K[lo:hi, h] @ Q[b, h]) * scale)
+                        O[b, h] = e @ V[lo:hi, h] / e.sum()
+                        L[b, h] = math.log(e.sum())
+        return O, L
+
+    def drops_last_key(q, k, v, scale, cu_seqlens_k=None, B=None, Nk=None):
+        segs = A._key_segments(np.asarray(k).shape[0], np.asarray(q).shape[0] if B is None else B, Nk, cu_seqlens_k)
+        rows = [j for lo, hi in segs for j in range(lo, max(lo, hi - 1))]
+        cu = np.cumsum([0] + [max(0, hi - lo - 1) for lo, hi in segs])
+        return oracle.decode_forward(q, np.asarray(k)[rows], np.asarray(v)[rows], scale, cu_seqlens_k=cu)
+
+    def wrong_merge_sign(q, k, v, scale, chunk, cu_seqlens_k=None, B=None, Nk=None):
+        O, L, parts = oracle.split_kv_decode(q, k, v, scale, chunk, cu_seqlens_k, B, Nk, return_partials=True)
+        Ob = np.zeros_like(O)
+        for idx, ps in enumerate(parts):
+            b, h = divmod(idx, O.shape[1])
+            if not ps:
+                continue
+            m = max(p[0] for p in ps)
+            ell = sum(p[1] * math.exp(m - p[0]) for p in ps)   # the sign of the exponent flipped
+            Ob[b, h] = sum(p[2] * math.exp(m - p[0]) for p in ps) / ell
+        return Ob, L
+
+    assert not _decode_pins_pass(no_scale)
+    assert not _decode_pins_pass(no_max_shift)
+    assert not _decode_pins_pass(drops_last_key)
+    assert not _decode_pins_pass(oracle.decode_forward, wrong_merge_sign)
