@@ -414,6 +414,168 @@ def run_gpu(args, world, rank, local, pg):
 # ----------------------------------------------------------------------------- CPU oracle (baseline / reference arm)
 
 
+def run_gpu_decode(args, world, rank, local, pg):
+    """Decode workloads: one query per sequence over a device-resident K/V cache (HBM-bound)."""
+    import torch
+
+    import workloads
+    import exact_io_aware_90_b200 as fa
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    wname = args.workload
+    spec = workloads.DECODE_WORKLOADS[wname]
+    inp_h = workloads.make_decode_workload(wname)
+    if rank > 0:  # weak scaling: each rank its own seeded copy
+        inp_h = workloads.decode_inputs(inp_h.H, inp_h.d, inp_h.dtype, spec["seed"] + 1000 * rank, B=inp_h.B,
+                                        Nk=inp_h.Nk, seqlens=inp_h.seqlens if inp_h.cu_seqlens_k is not None else None)
+    B, H, Nk, d, Tk = inp_h.B, inp_h.H, inp_h.Nk, inp_h.d, inp_h.Tk
+    dt = fa.dtype_code(inp_h.q)
+    flops = 4.0 * H * d * float(sum(inp_h.seqlens))  # q·Kᵀ and p·V, 2 FLOP per multiply-add
+    elt = 2
+    algo_bytes = 2 * Tk * H * d * elt + 2 * B * H * d * elt + B * H * 4  # K, V once; q, o; lse
+    q, k, v = inp_h.q.to(dev), inp_h.k.to(dev), inp_h.v.to(dev)
+    cu = inp_h.cu_seqlens_k.to(dev) if inp_h.cu_seqlens_k is not None else None
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H), dtype=torch.float32, device=dev)
+    ws_bytes = fa.fa_decode_workspace_bytes(B, H, Nk, d)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def step():
+        st = fa.fa_decode(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, Nk, d,
+                          inp_h.scale, cu.data_ptr() if cu is not None else None, Tk, dt, ws.data_ptr(), ws_bytes, sp)
+        if st != fa.FA_OK:
+            raise fa.FAError(st, "fa_decode")
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(dev)
+    if pg is not None:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    evs = []
+    for _ in range(args.steps):
+        flush.fill_(1)  # outside the timed events: the cache is read from HBM every step
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        step()
+        b.record(stream)
+        evs.append((a, b))
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    st = fa.fa_check_device_status(sp)
+    if st != fa.FA_OK:
+        raise fa.FAError(st, "timed steps")
+    ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in evs])), pg, dev)
+    value = world * flops / (ms * 1e-3) / 1e12
+    # end to end through the public API: the new query in from pinned host memory, the output back (the cache
+    # stays resident on the device, as it does while generating)
+    hq = inp_h.q.pin_memory()
+    ho = torch.empty_like(hq).pin_memory()
+    hl = torch.empty((B, H), dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        fa.attention_decode(q, k, v, scale=inp_h.scale, cu_seqlens_k=cu, max_seqlen_k=Nk if cu is not None else None,
+                            out=o, lse=lse, workspace=ws, stream=sp)
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = max(1, min(args.steps, 10))
+    a.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(a.elapsed_time(b) / n_e2e, pg, dev)
+    peaks = load_peaks()
+    gbs = algo_bytes / (ms * 1e-3) / 1e9
+    out = {
+        "metric": METRIC + " (decode: one query per sequence)",
+        "value": round(value, 3),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": inp_h.dtype,
+        "data": "synthetic: i.i.d. N(0,1) q, k, v from a seeded CPU generator, rounded to the dtype",
+        "config": {"workload": wname, "B": B, "H": H, "Nk": Nk, "d": d, "varlen": cu is not None, "keys": Tk,
+                   "step": "decode", "flops_per_step": flops,
+                   "l2": "flushed before every step (256 MiB write, outside the events)",
+                   "parallelism": f"replicas x{world} (independent workloads per GPU)"},
+        "roofline": {"kernel": "fa_decode_split_kernel + fa_decode_merge_kernel", "bound": "hbm",
+                     "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None,
+                     "algorithmic_bytes": algo_bytes, "peak_source": peaks["source"]},
+        "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": int(hq.numel() * hq.element_size()),
+                "d2h_bytes_per_step": int(ho.numel() * ho.element_size() + hl.numel() * 4)},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline_decode(inp_h, budget_s=args.cpu_budget)
+    return out
+
+
+def decode_oracle_seq(inp, n):
+    """fp64 oracle decode of sequence n (all heads).  Returns (seconds, flops credited)."""
+    import oracle
+    lo = int(sum(inp.seqlens[:n]))
+    L = int(inp.seqlens[n])
+    t0 = time.perf_counter()
+    oracle.decode_forward(inp.q[n:n + 1], inp.k[lo:lo + L], inp.v[lo:lo + L], inp.scale, cu_seqlens_k=[0, L])
+    return time.perf_counter() - t0, 4.0 * inp.H * inp.d * L
+
+
+def cpu_baseline_decode(inp, budget_s=15.0):
+    """Whole sequences (all heads) through the oracle until about `budget_s` seconds of CPU work."""
+    tot_t, tot_f, n = 0.0, 0.0, 0
+    while n < inp.B and tot_t < budget_s:
+        dt, f = decode_oracle_seq(inp, n)
+        tot_t, tot_f, n = tot_t + dt, tot_f + f, n + 1
+    return {"value": round(tot_f / max(tot_t, 1e-9) / 1e12, 6), "unit": "TFLOP/s", "cores": blas_threads(),
+            "kind": "oracle", "sample": f"fp64 NumPy oracle decode of {n} whole sequence(s), all heads, {tot_t:.2f} s"}
+
+
+def run_reference_decode(args):
+    import workloads
+    inp = workloads.make_decode_workload(args.workload)
+    for _ in range(args.warmup):
+        decode_oracle_seq(inp, 0)
+    times, flops = [], 0.0
+    for _ in range(args.steps):
+        dt, f = decode_oracle_seq(inp, 0)
+        times.append(dt)
+        flops = f
+    ms = 1e3 * float(np.mean(times))
+    value = flops / (ms * 1e-3) / 1e12
+    return {
+        "impl": "reference", "metric": METRIC + " (decode: one query per sequence)", "value": round(value, 6),
+        "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms, 2), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "B": inp.B, "H": inp.H, "Nk": inp.Nk, "d": inp.d, "sample": "sequence 0"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": "fp64 NumPy oracle decode of sequence 0 (all heads) per step"},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
 def blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -462,6 +624,8 @@ def cpu_baseline(inp, budget_s=15.0):
 
 def run_reference(args, rank):
     import workloads
+    if args.workload in workloads.DECODE_WORKLOADS:
+        return run_reference_decode(args)
     spec = workloads.WORKLOADS[args.workload]
     inp = workloads.make_workload(args.workload, backward=spec["backward"])
     L = inp.seqlens[0]
@@ -516,7 +680,11 @@ def main():
         return 0
     world, rank, local, pg = dist_setup(args)
     try:
-        out = run_gpu(args, world, rank, local, pg)
+        import workloads
+        if args.workload in workloads.DECODE_WORKLOADS:
+            out = run_gpu_decode(args, world, rank, local, pg)
+        else:
+            out = run_gpu(args, world, rank, local, pg)
         if rank == 0:
             print(json.dumps(out), flush=True)
     finally:

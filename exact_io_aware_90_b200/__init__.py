@@ -9,11 +9,12 @@ GPU is present the calls raise.
 
 Raw ABI (same names and argument order as ``include/fa.h``; pointers are ints):
     fa_fwd, fa_bwd, fa_bwd_preprocess, fa_bwd_main, fa_bwd_postprocess,
-    fa_bwd_workspace_bytes, fa_bwd_noalloc, fa_check_device_status, fa_set_watchdog_ns,
-    fa_watchdog_selftest, fa_status_string, fa_version
+    fa_bwd_workspace_bytes, fa_bwd_noalloc, fa_decode, fa_decode_workspace_bytes,
+    fa_check_device_status, fa_set_watchdog_ns, fa_watchdog_selftest, fa_status_string, fa_version
 Torch wrappers:
     attention_forward(q, k, v, ...)          -> (o, lse)
     attention_backward(q, k, v, o, lse, do, ...) -> (dq, dk, dv)
+    attention_decode(q, k, v, ...)           -> (o, lse)   one query per sequence over a K/V cache
 """
 
 from __future__ import annotations
@@ -27,8 +28,8 @@ __all__ = [
     "FAError", "LIB_PATH", "lib", "FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA",
     "FA_ERR_TIMEOUT", "FA_BF16", "FA_FP16",
     "fa_fwd", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_postprocess", "fa_bwd_workspace_bytes",
-    "fa_bwd_noalloc", "FA_NOALLOC_SCRATCH_BYTES", "fa_check_device_status", "fa_set_watchdog_ns", "fa_watchdog_selftest", "fa_status_string", "fa_version",
-    "attention_forward", "attention_backward", "dtype_code",
+    "fa_bwd_noalloc", "FA_NOALLOC_SCRATCH_BYTES", "fa_decode", "fa_decode_workspace_bytes", "fa_check_device_status", "fa_set_watchdog_ns", "fa_watchdog_selftest", "fa_status_string", "fa_version",
+    "attention_forward", "attention_backward", "attention_decode", "dtype_code",
 ]
 
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = 0, 1, 2, 3, 4
@@ -59,6 +60,8 @@ def _load() -> ctypes.CDLL:
         "fa_bwd_main": (I, [P, P, P, P, P, P, P, I, I, I, I, F, I, P, I, I, P, S, P]),
         "fa_bwd_postprocess": (I, [P, I, I, I, I, F, P, I, I, P, S, P]),
         "fa_bwd_noalloc": (I, [P, P, P, P, P, P, P, P, P, I, I, I, I, F, I, P, I, I, P]),
+        "fa_decode_workspace_bytes": (S, [I, I, I, I]),
+        "fa_decode": (I, [P, P, P, P, P, I, I, I, I, F, P, I, I, P, S, P]),
         "fa_check_device_status": (I, [P]),
         "fa_set_watchdog_ns": (None, [U64]),
         "fa_watchdog_selftest": (I, [U64, P]),
@@ -115,6 +118,16 @@ def fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, c
     scratch (see include/fa.h)."""
     return lib.fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, cu_seqlens, total_tokens,
                               dtype, stream)
+
+
+def fa_decode_workspace_bytes(B, H, Nk, d) -> int:
+    return lib.fa_decode_workspace_bytes(B, H, Nk, d)
+
+
+def fa_decode(q, k, v, o, lse, B, H, Nk, d, scale, cu_seqlens_k, total_keys, dtype, workspace, workspace_bytes,
+              stream) -> int:
+    return lib.fa_decode(q, k, v, o, lse, B, H, Nk, d, scale, cu_seqlens_k, total_keys, dtype, workspace,
+                         workspace_bytes, stream)
 
 
 def fa_check_device_status(stream) -> int:
@@ -221,3 +234,45 @@ def attention_backward(q, k, v, o, lse, do, causal: bool = False, scale: Optiona
     if st != FA_OK:
         raise FAError(st, "fa_bwd")
     return dq, dk, dv
+
+
+def attention_decode(q, k, v, scale: Optional[float] = None, cu_seqlens_k=None, max_seqlen_k: Optional[int] = None,
+                     out=None, lse=None, workspace=None, stream=None):
+    """O [B, H, d] and LSE [B, H] of one query per sequence (q: [B, H, d]) over its keys in
+    k, v: [Tk, H, d] (see ``include/fa.h``).  Without ``cu_seqlens_k`` the Tk = B·Nk keys
+    form B sequences of Nk keys."""
+    import torch
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != q.dtype:
+            raise ValueError(f"{n} must be a contiguous CUDA tensor with q's dtype")
+    B, H, d = q.shape
+    Tk = k.shape[0]
+    if k.shape != (Tk, H, d) or v.shape != k.shape:
+        raise ValueError("k and v must be [Tk, H, d] with q's H and d")
+    if cu_seqlens_k is None:
+        if Tk % B:
+            raise ValueError("key count must be a multiple of the batch size")
+        Nk = Tk // B
+    else:
+        if int(cu_seqlens_k.numel()) != B + 1:
+            raise ValueError("cu_seqlens_k needs B + 1 entries")
+        if max_seqlen_k is None:
+            raise ValueError("max_seqlen_k is required with cu_seqlens_k")
+        Nk = int(max_seqlen_k)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    need = lib.fa_decode_workspace_bytes(B, H, Nk, d)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    st = lib.fa_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Nk, d, float(scale),
+                       _ptr(cu_seqlens_k), Tk, dtype_code(q), _ptr(workspace),
+                       workspace.numel() * workspace.element_size(), stream)
+    if st != FA_OK:
+        raise FAError(st, "fa_decode")
+    return out, lse

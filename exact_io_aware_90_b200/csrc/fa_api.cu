@@ -207,6 +207,35 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
                             stream);
 }
 
+size_t fa_decode_workspace_bytes(int B, int H, int Nk, int d) {
+  if (B < 1 || H < 1 || Nk < 1 || (d != 64 && d != 128)) return 0;
+  const size_t slots = (size_t)B * H * decode_chunks(Nk);
+  return align256(slots * d * sizeof(float)) + align256(slots * 2 * sizeof(float));
+}
+
+int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nk, int d,
+              float scale, const int32_t* cu_seqlens_k, int total_keys, int dtype, void* workspace,
+              size_t workspace_bytes_, fa_stream_t stream) {
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(lse)) return FA_ERR_INVALID_ARG;
+  Problem pb;
+  int st = make_problem(&pb, B, H, Nk, d, scale, 0, cu_seqlens_k, total_keys, dtype, true);
+  if (st != FA_OK) return st;
+  if (B > 65535 || H > 65535) return FA_ERR_UNSUPPORTED;  // grid y / z
+  const size_t need = fa_decode_workspace_bytes(B, H, Nk, d);
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes_ < need)
+    return FA_ERR_INVALID_ARG;
+  DecodeArgs a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.lse = lse;
+  const size_t slots = (size_t)B * H * decode_chunks(Nk);
+  a.part_o = reinterpret_cast<float*>(workspace);
+  a.part_ml = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + align256(slots * d * sizeof(float)));
+  return map_launch(launch_decode(pb, a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int fa_check_device_status(fa_stream_t stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
   int h = 0;

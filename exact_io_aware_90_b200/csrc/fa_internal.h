@@ -48,7 +48,21 @@ bool encode_tmap(CUtensorMap* map, const void* base, int T, int H, int d, bool b
 // box of 32 features × 1 head × `rows` tokens.  Returns false on failure.
 bool encode_tmap_f32(CUtensorMap* map, const void* base, int T, int H, int d, int rows);
 
+// Decode (one query per sequence, split-KV): keys per chunk, and its workspace.
+constexpr int kDecChunkKeys = 512;
+inline int decode_chunks(int Nk) { return (Nk + kDecChunkKeys - 1) / kDecChunkKeys; }
+struct DecodeArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  float* lse;
+  float* part_o;   // [B·H, chunks, d] fp32
+  float* part_ml;  // [B·H, chunks, 2] fp32
+};
+
 cudaError_t launch_fwd(const Problem& pb, const FwdArgs& a, cudaStream_t stream);
+cudaError_t launch_decode(const Problem& pb, const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_bwd_pre(const Problem& pb, const BwdArgs& a, cudaStream_t stream);
 cudaError_t launch_bwd_main(const Problem& pb, const BwdArgs& a, cudaStream_t stream);
 cudaError_t launch_bwd_post(const Problem& pb, const BwdArgs& a, cudaStream_t stream);

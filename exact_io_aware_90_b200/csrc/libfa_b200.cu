@@ -3,4 +3,5 @@
 #include "fa_api.cu"
 #include "fa_fwd.cu"
 #include "fa_bwd.cu"
+#include "fa_decode.cu"
 #include "fa_noalloc.cu"

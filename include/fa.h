@@ -177,6 +177,37 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
                    const int32_t* cu_seqlens, int total_tokens, int dtype, fa_stream_t stream);
 
 /*
+ * Decode: one new query token per sequence attends to every key of its
+ * sequence in a K/V cache (token-by-token generation, the workload
+ * "FlashAttention 短片讲解稿", segment "适用范围与关键结论", sets apart from
+ * training and prefill).  No mask: every cached key precedes or is the
+ * current token.
+ *   q, o       [B, H, d], one row per sequence (same dtype as k and v).
+ *   k, v       [total_keys, H, d]: sequence b's keys are rows
+ *              [cu_seqlens_k[b], cu_seqlens_k[b+1]) of a device int32
+ *              cu_seqlens_k (B+1 entries), or rows [b·Nk, (b+1)·Nk) when
+ *              cu_seqlens_k == NULL (total_keys must then equal B·Nk).  Nk
+ *              bounds every sequence's key count.
+ *   lse        fp32 [B, H], natural-log log-sum-exp of the scaled scores; a
+ *              sequence with no key gets o = 0 and lse = −inf.
+ * The keys of each (sequence, head) are split into chunks of 512 that are
+ * reduced in parallel to partial (max, sum, output) triples in `workspace`
+ * (device memory the caller owns, 256-byte aligned, at least
+ * fa_decode_workspace_bytes(B, H, Nk, d) bytes); a second kernel merges them
+ * with the block-merge rule of "FlashAttention 与算子融合" ("FlashAttention 的两个
+ * 关键": max of the maxima, sums and partial outputs rescaled to it).
+ * Arithmetic in fp32 on the CUDA cores (the single query makes this a stream
+ * over the cache, bound by memory bandwidth).  Errors as for fa_fwd; B and H
+ * above 65535 return FA_ERR_UNSUPPORTED.  The two kernels are enqueued on
+ * `stream`; nothing is allocated or synchronised.
+ */
+size_t fa_decode_workspace_bytes(int B, int H, int Nk, int d);
+int fa_decode(const void* q, const void* k, const void* v, void* o, float* lse,
+              int B, int H, int Nk, int d, float scale, const int32_t* cu_seqlens_k,
+              int total_keys, int dtype, void* workspace, size_t workspace_bytes,
+              fa_stream_t stream);
+
+/*
  * Synchronises `stream`, returns the device status word (FA_OK, or the first
  * FA_ERR_TIMEOUT / FA_ERR_INVALID_ARG a kernel recorded since the last call)
  * and clears it.  Returns FA_ERR_CUDA if the synchronisation itself failed.

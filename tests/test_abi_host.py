@@ -32,7 +32,7 @@ def test_header_declares_the_entry_points():
     names = _declared_functions()
     for n in ["fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_bwd_preprocess", "fa_bwd_main",
               "fa_bwd_postprocess", "fa_check_device_status", "fa_status_string", "fa_set_watchdog_ns",
-              "fa_watchdog_selftest", "fa_version"]:
+              "fa_watchdog_selftest", "fa_version", "fa_bwd_noalloc", "fa_decode", "fa_decode_workspace_bytes"]:
         assert n in names
 
 
@@ -99,6 +99,32 @@ def test_backward_rejects_invalid_arguments(fa):
     assert fa.fa_bwd_postprocess(P16, 2, 4, 256, 64, float("nan"), None, 512, 0, P16, ws, None) == fa.FA_ERR_INVALID_ARG
     assert fa.fa_bwd_main(P16, P16, P16, P16, P16, P16, P16, 2, 4, 256, 64, 0.125, 3, None, 512, 0, P16, ws,
                           None) == fa.FA_ERR_INVALID_ARG
+
+
+def test_decode_workspace_bytes(fa):
+    # per (sequence, head, 512-key chunk): d fp32 partial outputs + (m, ℓ), each part rounded up to 256 bytes
+    def up(x):
+        return (x + 255) // 256 * 256
+    slots = 16 * 16 * 16  # B = 16, H = 16, 8192 keys → 16 chunks
+    assert fa.fa_decode_workspace_bytes(16, 16, 8192, 128) == up(slots * 128 * 4) + up(slots * 2 * 4)
+    assert fa.fa_decode_workspace_bytes(1, 1, 513, 64) == up(2 * 64 * 4) + up(2 * 2 * 4)
+    assert fa.fa_decode_workspace_bytes(0, 16, 8192, 128) == 0
+    assert fa.fa_decode_workspace_bytes(1, 1, 64, 96) == 0
+
+
+def test_decode_rejects_invalid_arguments(fa):
+    ws = fa.fa_decode_workspace_bytes(2, 4, 256, 64)
+    good = dict(q=P16, k=P16, v=P16, o=P16, lse=P16, B=2, H=4, Nk=256, d=64, scale=0.125, cu_seqlens_k=None,
+                total_keys=512, dtype=0, workspace=P16, workspace_bytes=ws, stream=None)
+    for bad in [dict(d=96), dict(B=0), dict(Nk=0), dict(total_keys=511), dict(scale=float("nan")), dict(scale=0.0),
+                dict(dtype=3), dict(q=0), dict(k=P16 + 8), dict(lse=P16 + 2), dict(workspace=P16 + 16),
+                dict(workspace_bytes=ws - 1), dict(cu_seqlens_k=P16 + 2)]:
+        a = dict(good)
+        a.update(bad)
+        assert fa.fa_decode(**a) == fa.FA_ERR_INVALID_ARG, bad
+    a = dict(good)
+    a.update(B=70000, total_keys=70000 * 256, workspace_bytes=fa.fa_decode_workspace_bytes(70000, 4, 256, 64))
+    assert fa.fa_decode(**a) == fa.FA_ERR_UNSUPPORTED
 
 
 def test_missing_library_fails_loudly(tmp_path, monkeypatch):

@@ -20,6 +20,15 @@ varlen_causal_d128  32 sequences, lengths uniform in [128, 4096], H=32,
                     d=128, bf16, causal, fwd+bwd
 long_n128k_d128     B=1, H=8, N=131072, d=128, bf16, causal, forward only
 ==================  =========================================================
+
+Decode inputs (one query token per sequence over a K/V cache): q is
+[B, H, d], k and v are [Tk, H, d] with ``cu_seqlens_k`` (or Tk = B·Nk):
+
+==================  =========================================================
+decode_b16_kv8k     B=16, H=16, Nk=8192 keys each, d=128, bf16
+decode_varlen       64 sequences, key counts uniform in [512, 16384], H=16,
+                    d=128, bf16
+==================  =========================================================
 """
 
 from __future__ import annotations
@@ -144,3 +153,59 @@ def hand_example_inputs(dtype: str = "fp16", d: int = 64) -> AttnInputs:
     tdt = TORCH_DTYPES[dtype]
     return AttnInputs(q.to(tdt), k.to(tdt), v.to(tdt), None, None, [4], 1, 1, 4, d, scale, False, dtype,
                       "hand_example")
+
+
+DECODE_WORKLOADS = {
+    "decode_b16_kv8k": dict(B=16, H=16, Nk=8192, d=128, dtype="bf16", seed=1006),
+    "decode_varlen": dict(nseq=64, lmin=512, lmax=16384, H=16, d=128, dtype="bf16", seed=1007),
+}
+
+
+@dataclass
+class DecodeInputs:
+    q: torch.Tensor                      # [B, H, d]
+    k: torch.Tensor                      # [Tk, H, d]
+    v: torch.Tensor
+    cu_seqlens_k: Optional[torch.Tensor]  # int32 [B+1] or None
+    seqlens: List[int]                   # key count per sequence
+    B: int
+    H: int
+    Nk: int                              # maximum key count
+    d: int
+    scale: float
+    dtype: str
+    name: str = ""
+
+    @property
+    def Tk(self) -> int:
+        return int(self.k.shape[0])
+
+    def to(self, device) -> "DecodeInputs":
+        mv = lambda t: None if t is None else t.to(device)
+        return DecodeInputs(mv(self.q), mv(self.k), mv(self.v), mv(self.cu_seqlens_k), list(self.seqlens), self.B,
+                            self.H, self.Nk, self.d, self.scale, self.dtype, self.name)
+
+
+def decode_inputs(H: int, d: int, dtype: str, seed: int, *, B: int = 1, Nk: int = 0,
+                  seqlens: Optional[List[int]] = None, scale: Optional[float] = None, name: str = "") -> DecodeInputs:
+    """i.i.d. N(0,1) q (one row per sequence), k and v for a dense or packed (``seqlens``) cache."""
+    if seqlens is not None:
+        cu = cu_from_lengths(seqlens)
+        B, Tk, Nk = len(seqlens), int(cu[-1]), max(seqlens) if seqlens else 0
+    else:
+        cu, Tk, seqlens = None, B * Nk, [Nk] * B
+    g = torch.Generator().manual_seed(seed)
+    q = _randn(g, (B, H, d), dtype)
+    k = _randn(g, (Tk, H, d), dtype)
+    v = _randn(g, (Tk, H, d), dtype)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    return DecodeInputs(q, k, v, cu, list(seqlens), B, H, max(Nk, 1), d, float(scale), dtype, name)
+
+
+def make_decode_workload(name: str) -> DecodeInputs:
+    w = DECODE_WORKLOADS[name]
+    if "nseq" in w:
+        lens = varlen_lengths(w["nseq"], w["lmin"], w["lmax"], w["seed"])
+        return decode_inputs(w["H"], w["d"], w["dtype"], w["seed"], seqlens=lens, name=name)
+    return decode_inputs(w["H"], w["d"], w["dtype"], w["seed"], B=w["B"], Nk=w["Nk"], name=name)
