@@ -17,6 +17,13 @@ Parity status of each function (what pins it; see ``tests/test_oracle.py``):
                           the last row of causal self-attention, brute force.
 * split_kv_decode         pinned: equals decode_forward for every chunk size;
                           chunk = 1 reduces to the page's per-element recurrence.
+* philox4x32_10           pinned: the generator's published known-answer vectors.
+* dropout_keep_mask       pinned: scalar re-derivation of the element mapping,
+                          keep fraction within binomial bounds.
+* attention_forward_dropout, attention_backward_dropout
+                          pinned: p = 0 equals the plain oracle, unbiased over
+                          seeds, finite differences with the mask fixed, the
+                          D identity.
 """
 from .attention import *  # noqa: F401,F403
 from .attention import __all__  # noqa: F401

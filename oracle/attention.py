@@ -64,6 +64,11 @@ __all__ = [
     "attention_flops",
     "decode_forward",
     "split_kv_decode",
+    "philox4x32_10",
+    "dropout_threshold",
+    "dropout_keep_mask",
+    "attention_forward_dropout",
+    "attention_backward_dropout",
 ]
 
 
@@ -440,3 +445,118 @@ def split_kv_decode(q, k, v, scale: float, chunk: int, cu_seqlens_k=None, B: Opt
     if return_partials:
         return O, LSE, partials
     return O, LSE
+
+
+# ----------------------------------------------------------------------------- dropout on P
+
+
+_PHILOX_M = (0xD2511F53, 0xCD9E8D57)   # round multipliers
+_PHILOX_W = (0x9E3779B9, 0xBB67AE85)   # key schedule (Weyl) increments
+_U32 = 0xFFFFFFFF
+
+
+def philox4x32_10(counter, key):
+    """Philox4x32 with 10 rounds (Salmon, Moraes, Dror, Shaw: "Parallel random numbers: as easy as
+    1, 2, 3", SC 2011): a counter-based generator mapping a 128-bit counter and a 64-bit key to 128
+    random bits.  ``counter`` is 4 arrays (or ints) of uint32 words, ``key`` 2; broadcasting numpy
+    arrays are processed element-wise.  Each round multiplies words 0 and 2 by fixed constants
+    (full 64-bit products), and mixes the high halves with words 1, 3 and the round key; the key
+    is bumped by fixed increments between rounds."""
+    c = [np.asarray(x, dtype=np.uint64) & _U32 for x in counter]
+    k0 = np.asarray(key[0], dtype=np.uint64) & _U32
+    k1 = np.asarray(key[1], dtype=np.uint64) & _U32
+    for r in range(10):
+        if r > 0:
+            k0 = (k0 + _PHILOX_W[0]) & _U32
+            k1 = (k1 + _PHILOX_W[1]) & _U32
+        p0 = c[0] * np.uint64(_PHILOX_M[0])
+        p1 = c[2] * np.uint64(_PHILOX_M[1])
+        hi0, lo0 = p0 >> np.uint64(32), p0 & _U32
+        hi1, lo1 = p1 >> np.uint64(32), p1 & _U32
+        c = [hi1 ^ c[1] ^ k0, lo1, hi0 ^ c[3] ^ k1, lo0]
+    return [x.astype(np.uint64) for x in c]
+
+
+def dropout_threshold(p: float) -> int:
+    """Dropout decisions compare one random byte with t = round(256·p) (clamped to 0…255): the
+    element is kept when byte ≥ t, so the drop probability is t/256 and kept elements are scaled
+    by 256/(256 − t) (inverted dropout, the expectation of P unchanged)."""
+    if not (0.0 <= p < 1.0):
+        raise ValueError("dropout probability must be in [0, 1)")
+    return min(255, int(math.floor(p * 256.0 + 0.5)))
+
+
+def dropout_keep_mask(L: int, bh: int, seed: int, offset: int, t: int) -> np.ndarray:
+    """Keep mask [L, L] (query i, key j, positions inside one sequence) of the (sequence, head)
+    with global index bh = b·H + h.  One Philox call covers a 4×4 block: counter = (j / 4, i / 4,
+    bh, offset), key = the two 32-bit halves of ``seed``; element (i, j) uses byte j mod 4 of
+    output word i mod 4."""
+    i = np.arange(L)[:, None]
+    j = np.arange(L)[None, :]
+    words = philox4x32_10([j >> 2, i >> 2, np.full((1, 1), bh), np.full((1, 1), offset)],
+                          [seed & _U32, (seed >> 32) & _U32])
+    w = np.select([(i & 3) == r for r in range(4)], [np.broadcast_to(x, (L, L)) for x in words])
+    byte = (w >> (8 * (j & 3)).astype(np.uint64)) & np.uint64(0xFF)
+    return byte >= t
+
+
+def attention_forward_dropout(q, k, v, scale: float, causal: bool, dropout_p: float, seed: int, offset: int = 0,
+                              cu_seqlens=None, B: Optional[int] = None, N: Optional[int] = None):
+    """O = dropout(P) V with the keep mask of ``dropout_keep_mask``; LSE is that of the undropped
+    softmax (the statistic the backward needs to recompute P).  Dropout on the probabilities is
+    the ``dropout_p`` of the scaled-dot-product-attention interface (Flash Attention 优化, SDPA
+    signature)."""
+    Q, K, V = _f64(q), _f64(k), _f64(v)
+    T, H, d = Q.shape
+    t = dropout_threshold(dropout_p)
+    keep_scale = 256.0 / (256.0 - t)
+    if cu_seqlens is not None:
+        B = len(np.asarray(cu_seqlens).reshape(-1)) - 1
+    elif B is None:
+        B = 1
+    segs = sequence_segments(T, B, T // B if N is None else N, cu_seqlens)
+    O = np.zeros((T, H, d))
+    LSE = np.full((T, H), -np.inf)
+    for b, (lo, L) in enumerate(segs):
+        hi = lo + L
+        for h in range(H):
+            if L == 0:
+                continue
+            S = _scores(Q[lo:hi, h], K[lo:hi, h], scale, causal)
+            P, m, ell = _softmax_rows(S)
+            M = dropout_keep_mask(hi - lo, b * H + h, seed, offset, t)
+            O[lo:hi, h] = (P * M * keep_scale) @ V[lo:hi, h]
+            LSE[lo:hi, h] = m + np.log(ell)
+    return O, LSE
+
+
+def attention_backward_dropout(q, k, v, do, scale: float, causal: bool, dropout_p: float, seed: int,
+                               offset: int = 0, cu_seqlens=None, B: Optional[int] = None, N: Optional[int] = None):
+    """Gradients of ``attention_forward_dropout`` (the keep mask is a constant of the call): with
+    Z = M·s/(1 − p)·P, O = Z V:  dV = Zᵀ dO,  dP = (dO Vᵀ) ∘ M·s,  D_i = Σ_j P_ij dP_ij
+    (= Σ_c dO_ic O_ic),  dS = P ∘ (dP − D),  dQ = scale·dS K,  dK = scale·dSᵀ Q."""
+    Q, K, V, dO = _f64(q), _f64(k), _f64(v), _f64(do)
+    T, H, d = Q.shape
+    t = dropout_threshold(dropout_p)
+    keep_scale = 256.0 / (256.0 - t)
+    if cu_seqlens is not None:
+        B = len(np.asarray(cu_seqlens).reshape(-1)) - 1
+    elif B is None:
+        B = 1
+    segs = sequence_segments(T, B, T // B if N is None else N, cu_seqlens)
+    dQ, dK, dV = np.zeros_like(Q), np.zeros_like(K), np.zeros_like(V)
+    for b, (lo, L) in enumerate(segs):
+        hi = lo + L
+        for h in range(H):
+            if L == 0:
+                continue
+            S = _scores(Q[lo:hi, h], K[lo:hi, h], scale, causal)
+            P, _, _ = _softmax_rows(S)
+            Mk = dropout_keep_mask(hi - lo, b * H + h, seed, offset, t) * keep_scale
+            dV[lo:hi, h] = (P * Mk).T @ dO[lo:hi, h]
+            dP = (dO[lo:hi, h] @ V[lo:hi, h].T) * Mk
+            Dv = (P * dP).sum(axis=1)
+            dS = P * (dP - Dv[:, None])
+            dQ[lo:hi, h] = scale * dS @ K[lo:hi, h]
+            dK[lo:hi, h] = scale * dS.T @ Q[lo:hi, h]
+    return dQ, dK, dV

@@ -577,3 +577,111 @@ def test_decode_pins_catch_planted_mistakes():
     assert not _decode_pins_pass(no_max_shift)
     assert not _decode_pins_pass(drops_last_key)
     assert not _decode_pins_pass(oracle.decode_forward, wrong_merge_sign)
+
+
+# ----------------------------------------------------------------------------- dropout on P
+
+
+def test_philox_known_answers():
+    kat = _load("philox4x32_10_kat.json")
+    for vec in kat["vectors"]:
+        ctr = [int(x, 16) for x in vec["counter"]]
+        key = [int(x, 16) for x in vec["key"]]
+        got = [int(x) for x in oracle.philox4x32_10(ctr, key)]
+        assert got == [int(x, 16) for x in vec["output"]]
+
+
+def test_dropout_mask_mapping_scalar():
+    """Element (i, j): byte j mod 4 of word i mod 4 of Philox(counter (j/4, i/4, bh, offset), seed)."""
+    seed, bh, off, t = 0x1234_5678_9ABC_DEF0, 5, 3, 77
+    M = oracle.dropout_keep_mask(23, bh, seed, off, t)
+    for i in range(23):
+        for j in range(23):
+            w = [int(x) for x in oracle.philox4x32_10([j >> 2, i >> 2, bh, off], [seed & 0xFFFFFFFF, seed >> 32])]
+            byte = (w[i & 3] >> (8 * (j & 3))) & 0xFF
+            assert bool(M[i, j]) == (byte >= t)
+
+
+@pytest.mark.parametrize("p", [0.0, 0.1, 0.5, 0.9])
+def test_dropout_keep_fraction(p):
+    t = oracle.dropout_threshold(p)
+    M = oracle.dropout_keep_mask(512, 7, 99, 0, t)
+    keep = 1.0 - t / 256.0
+    n = M.size
+    assert abs(M.mean() - keep) <= 5.0 * math.sqrt(keep * (1 - keep) / n) + 1e-12
+    if p == 0.0:
+        assert M.all()
+
+
+def test_dropout_masks_differ_by_head_seed_offset():
+    t = oracle.dropout_threshold(0.5)
+    a = oracle.dropout_keep_mask(64, 0, 1, 0, t)
+    for other in (oracle.dropout_keep_mask(64, 1, 1, 0, t), oracle.dropout_keep_mask(64, 0, 2, 0, t),
+                  oracle.dropout_keep_mask(64, 0, 1, 1, t)):
+        assert 0.3 < (a != other).mean() < 0.7
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_dropout_zero_is_plain_attention(causal):
+    rng = np.random.default_rng(21)
+    q, k, v = _rand(rng, 30, 2, 8)
+    do = rng.standard_normal(q.shape)
+    cu = [0, 13, 30]
+    O1, L1 = oracle.attention_forward(q, k, v, 0.4, causal, cu_seqlens=cu)
+    O2, L2 = oracle.attention_forward_dropout(q, k, v, 0.4, causal, 0.0, 5, cu_seqlens=cu)
+    assert np.abs(O1 - O2).max() < 1e-12 and np.abs(L1 - L2).max() < 1e-12
+    g1 = oracle.attention_backward(q, k, v, do, 0.4, causal, cu_seqlens=cu)
+    g2 = oracle.attention_backward_dropout(q, k, v, do, 0.4, causal, 0.0, 5, cu_seqlens=cu)
+    for a, b in zip(g1, g2):
+        assert np.abs(a - b).max() < 1e-12
+
+
+def test_dropout_is_unbiased_over_seeds():
+    """Inverted dropout keeps the expectation: the mean of O over many seeds approaches the
+    undropped O (a missing 1/(1 − p) would leave it short by the keep probability)."""
+    rng = np.random.default_rng(3)
+    q, k, v = _rand(rng, 16, 1, 4)
+    O_ref, _ = oracle.attention_forward(q, k, v, 0.5, False)
+    acc = np.zeros_like(O_ref)
+    n = 400
+    for s in range(n):
+        acc += oracle.attention_forward_dropout(q, k, v, 0.5, False, 0.3, 1000 + s)[0]
+    assert np.abs(acc / n - O_ref).max() < 0.06
+    assert np.abs(acc / n * (1 - 77 / 256) - O_ref).max() > 0.05  # the unscaled mean would be visibly short
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_dropout_backward_finite_differences(causal):
+    rng = np.random.default_rng(8 + int(causal))
+    q, k, v = _rand(rng, 7, 1, 3)
+    do = rng.standard_normal(q.shape)
+    p, seed, scale = 0.3, 42, 0.7
+    f = lambda q_, k_, v_: float((oracle.attention_forward_dropout(q_, k_, v_, scale, causal, p, seed)[0] * do).sum())
+    dq, dk, dv = oracle.attention_backward_dropout(q, k, v, do, scale, causal, p, seed)
+    h = 1e-6
+    for arr, g in ((q, dq), (k, dk), (v, dv)):
+        num = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            a1, a2 = arr.copy(), arr.copy()
+            a1[idx] += h
+            a2[idx] -= h
+            args1 = [a1 if arr is x else x for x in (q, k, v)]
+            args2 = [a2 if arr is x else x for x in (q, k, v)]
+            num[idx] = (f(*args1) - f(*args2)) / (2 * h)
+        assert np.linalg.norm(num - g) <= 1e-6 * max(1.0, np.linalg.norm(g))
+
+
+def test_dropout_delta_identity():
+    """D_i = Σ_j P_ij dP_ij equals Σ_c dO_ic O_ic also with dropout (O is the dropped output)."""
+    rng = np.random.default_rng(4)
+    q, k, v = _rand(rng, 20, 1, 5)
+    do = rng.standard_normal(q.shape)
+    p, seed, scale = 0.2, 7, 0.5
+    O, _ = oracle.attention_forward_dropout(q, k, v, scale, True, p, seed)
+    t = oracle.dropout_threshold(p)
+    S = (q[:, 0] @ k[:, 0].T) * scale
+    S[np.triu_indices(20, 1)] = -np.inf
+    P = np.exp(S - S.max(axis=1, keepdims=True))
+    P /= P.sum(axis=1, keepdims=True)
+    dP = (do[:, 0] @ v[:, 0].T) * oracle.dropout_keep_mask(20, 0, seed, 0, t) * 256.0 / (256.0 - t)
+    assert np.abs((P * dP).sum(axis=1) - (do[:, 0] * O[:, 0]).sum(axis=1)).max() < 1e-12
