@@ -9,7 +9,7 @@ GPU is present the calls raise.
 
 Raw ABI (same names and argument order as ``include/fa.h``; pointers are ints):
     fa_fwd, fa_bwd, fa_bwd_preprocess, fa_bwd_main, fa_bwd_postprocess,
-    fa_bwd_workspace_bytes, fa_bwd_noalloc, fa_decode, fa_decode_workspace_bytes,
+    fa_bwd_workspace_bytes, fa_bwd_noalloc, fa_fwd_dropout, fa_bwd_dropout, fa_decode, fa_decode_workspace_bytes,
     fa_check_device_status, fa_set_watchdog_ns, fa_watchdog_selftest, fa_status_string, fa_version
 Torch wrappers:
     attention_forward(q, k, v, ...)          -> (o, lse)
@@ -28,7 +28,7 @@ __all__ = [
     "FAError", "LIB_PATH", "lib", "FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA",
     "FA_ERR_TIMEOUT", "FA_BF16", "FA_FP16",
     "fa_fwd", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_postprocess", "fa_bwd_workspace_bytes",
-    "fa_bwd_noalloc", "FA_NOALLOC_SCRATCH_BYTES", "fa_decode", "fa_decode_workspace_bytes", "fa_check_device_status", "fa_set_watchdog_ns", "fa_watchdog_selftest", "fa_status_string", "fa_version",
+    "fa_bwd_noalloc", "FA_NOALLOC_SCRATCH_BYTES", "fa_fwd_dropout", "fa_bwd_dropout", "fa_decode", "fa_decode_workspace_bytes", "fa_check_device_status", "fa_set_watchdog_ns", "fa_watchdog_selftest", "fa_status_string", "fa_version",
     "attention_forward", "attention_backward", "attention_decode", "dtype_code",
 ]
 
@@ -48,7 +48,7 @@ class FAError(RuntimeError):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m exact_io_aware_90_b200.build` "
+            f"{LIB_PATH} is missing: build it with `python exact_io_aware_90_b200/build.py` "
             "(nvcc, sm_100a). There is no fallback implementation.")
     L = ctypes.CDLL(LIB_PATH)
     P, I, F, S, U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_uint64
@@ -60,6 +60,9 @@ def _load() -> ctypes.CDLL:
         "fa_bwd_main": (I, [P, P, P, P, P, P, P, I, I, I, I, F, I, P, I, I, P, S, P]),
         "fa_bwd_postprocess": (I, [P, I, I, I, I, F, P, I, I, P, S, P]),
         "fa_bwd_noalloc": (I, [P, P, P, P, P, P, P, P, P, I, I, I, I, F, I, P, I, I, P]),
+        "fa_fwd_dropout": (I, [P, P, P, P, P, I, I, I, I, F, I, P, I, I, F, U64, ctypes.c_uint32, P]),
+        "fa_bwd_dropout": (I, [P, P, P, P, P, P, P, P, P, I, I, I, I, F, I, P, I, I, F, U64, ctypes.c_uint32, P, S,
+                               P]),
         "fa_decode_workspace_bytes": (S, [I, I, I, I]),
         "fa_decode": (I, [P, P, P, P, P, I, I, I, I, F, P, I, I, P, S, P]),
         "fa_check_device_status": (I, [P]),
@@ -118,6 +121,18 @@ def fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, c
     scratch (see include/fa.h)."""
     return lib.fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, cu_seqlens, total_tokens,
                               dtype, stream)
+
+
+def fa_fwd_dropout(q, k, v, o, lse, B, H, N, d, scale, causal, cu_seqlens, total_tokens, dtype, dropout_p, seed,
+                   offset, stream) -> int:
+    return lib.fa_fwd_dropout(q, k, v, o, lse, B, H, N, d, scale, causal, cu_seqlens, total_tokens, dtype, dropout_p,
+                              seed, offset, stream)
+
+
+def fa_bwd_dropout(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, cu_seqlens, total_tokens, dtype,
+                   dropout_p, seed, offset, workspace, workspace_bytes, stream) -> int:
+    return lib.fa_bwd_dropout(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, cu_seqlens, total_tokens,
+                              dtype, dropout_p, seed, offset, workspace, workspace_bytes, stream)
 
 
 def fa_decode_workspace_bytes(B, H, Nk, d) -> int:
@@ -187,8 +202,10 @@ def _check(t, name, q):
 
 def attention_forward(q, k, v, causal: bool = False, scale: Optional[float] = None, cu_seqlens=None,
                       max_seqlen: Optional[int] = None, batch: Optional[int] = None, out=None, lse=None,
-                      stream=None) -> Tuple["torch.Tensor", "torch.Tensor"]:
-    """O and LSE for q, k, v of shape [T, H, d] (see ``include/fa.h``)."""
+                      stream=None, dropout_p: float = 0.0, seed: int = 0,
+                      offset: int = 0) -> Tuple["torch.Tensor", "torch.Tensor"]:
+    """O and LSE for q, k, v of shape [T, H, d] (see ``include/fa.h``); ``dropout_p`` > 0 drops
+    probabilities with the in-kernel mask of (seed, offset)."""
     import torch
     for t, n in ((k, "k"), (v, "v")):
         _check(t, n, q)
@@ -202,8 +219,13 @@ def attention_forward(q, k, v, causal: bool = False, scale: Optional[float] = No
         lse = torch.empty((T, H), dtype=torch.float32, device=q.device)
     if stream is None:
         stream = torch.cuda.current_stream(q.device).cuda_stream
-    st = lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, d, float(scale), int(bool(causal)),
-                    _ptr(cu_seqlens), T, dtype_code(q), stream)
+    if dropout_p:
+        st = lib.fa_fwd_dropout(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, d, float(scale),
+                                int(bool(causal)), _ptr(cu_seqlens), T, dtype_code(q), float(dropout_p), int(seed),
+                                int(offset), stream)
+    else:
+        st = lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, d, float(scale), int(bool(causal)),
+                        _ptr(cu_seqlens), T, dtype_code(q), stream)
     if st != FA_OK:
         raise FAError(st, "fa_fwd")
     return out, lse
@@ -211,8 +233,8 @@ def attention_forward(q, k, v, causal: bool = False, scale: Optional[float] = No
 
 def attention_backward(q, k, v, o, lse, do, causal: bool = False, scale: Optional[float] = None, cu_seqlens=None,
                        max_seqlen: Optional[int] = None, batch: Optional[int] = None, dq=None, dk=None, dv=None,
-                       workspace=None, stream=None):
-    """dq, dk, dv for the forward that produced (o, lse)."""
+                       workspace=None, stream=None, dropout_p: float = 0.0, seed: int = 0, offset: int = 0):
+    """dq, dk, dv for the forward that produced (o, lse) (with the same dropout_p, seed, offset)."""
     import torch
     for t, n in ((k, "k"), (v, "v"), (o, "o"), (do, "do")):
         _check(t, n, q)
@@ -228,9 +250,15 @@ def attention_backward(q, k, v, o, lse, do, causal: bool = False, scale: Optiona
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     if stream is None:
         stream = torch.cuda.current_stream(q.device).cuda_stream
-    st = lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv), B, H, N,
-                    d, float(scale), int(bool(causal)), _ptr(cu_seqlens), T, dtype_code(q), _ptr(workspace),
-                    workspace.numel() * workspace.element_size(), stream)
+    if dropout_p:
+        st = lib.fa_bwd_dropout(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
+                                B, H, N, d, float(scale), int(bool(causal)), _ptr(cu_seqlens), T, dtype_code(q),
+                                float(dropout_p), int(seed), int(offset), _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), stream)
+    else:
+        st = lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv), B, H,
+                        N, d, float(scale), int(bool(causal)), _ptr(cu_seqlens), T, dtype_code(q), _ptr(workspace),
+                        workspace.numel() * workspace.element_size(), stream)
     if st != FA_OK:
         raise FAError(st, "fa_bwd")
     return dq, dk, dv

@@ -1,6 +1,7 @@
 """Builds libfa_b200.so in-tree with nvcc for sm_100a.
 
-Usage: python -m exact_io_aware_90_b200.build [--verbose-ptxas]
+Usage: python exact_io_aware_90_b200/build.py [--verbose-ptxas]   (by path: importing the package would load the
+existing library first)
 The library lands next to this file; the Python binding loads it from there.
 """
 from __future__ import annotations

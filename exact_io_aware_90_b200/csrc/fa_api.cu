@@ -86,6 +86,19 @@ static int make_problem(Problem* pb, int B, int H, int N, int d, float scale, in
   pb->cu_seqlens = cu;
   pb->bf16 = (dtype == FA_BF16);
   pb->timeout_ns = g_watchdog_ns;
+  pb->drop = Dropout{0u, 1.f, 0u, 0u, 0u};
+  return FA_OK;
+}
+
+// Dropout on P (see fa.h): threshold byte t = round(256·p) clamped to 255, keep scale 256/(256 − t).
+static int set_dropout(Problem* pb, float p, uint64_t seed, uint32_t offset) {
+  if (!(p >= 0.f && p < 1.f)) return FA_ERR_INVALID_ARG;  // also rejects NaN
+  const double t = std::floor((double)p * 256.0 + 0.5);
+  pb->drop.t = (uint32_t)(t > 255.0 ? 255.0 : t);
+  pb->drop.keep_scale = (float)(256.0 / (256.0 - (double)pb->drop.t));
+  pb->drop.seed_lo = (uint32_t)(seed & 0xFFFFFFFFull);
+  pb->drop.seed_hi = (uint32_t)(seed >> 32);
+  pb->drop.offset = offset;
   return FA_OK;
 }
 
@@ -107,16 +120,16 @@ static int map_launch(cudaError_t e) { return e == cudaSuccess ? FA_OK : FA_ERR_
 
 }  // namespace fa
 
-using namespace fa;
+namespace fa {
 
-extern "C" {
-
-int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
-           float scale, int causal, const int32_t* cu_seqlens, int total_tokens, int dtype, fa_stream_t stream) {
+static int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                    float scale, int causal, const int32_t* cu_seqlens, int total_tokens, int dtype, bool dropout,
+                    float dropout_p, uint64_t seed, uint32_t offset, fa_stream_t stream) {
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(lse)) return FA_ERR_INVALID_ARG;
   Problem pb;
   int st = make_problem(&pb, B, H, N, d, scale, causal, cu_seqlens, total_tokens, dtype, true);
   if (st != FA_OK) return st;
+  if (dropout && (st = set_dropout(&pb, dropout_p, seed, offset)) != FA_OK) return st;
   FwdArgs a;
   if (!encode_tmap(&a.tm_q, q, pb.T, H, d, pb.bf16, 128) || !encode_tmap(&a.tm_k, k, pb.T, H, d, pb.bf16, 128) ||
       !encode_tmap(&a.tm_v, v, pb.T, H, d, pb.bf16, 128))
@@ -124,6 +137,53 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   a.o = o;
   a.lse = lse;
   return map_launch(launch_fwd(pb, a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+static int bwd_main_impl(const void* q, const void* k, const void* v, const float* lse, const void* dO, void* dk,
+                         void* dv, int B, int H, int N, int d, float scale, int causal, const int32_t* cu_seqlens,
+                         int total_tokens, int dtype, bool dropout, float dropout_p, uint64_t seed, uint32_t offset,
+                         void* workspace, size_t workspace_bytes_, fa_stream_t stream) {
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned4(lse) || !aligned16(dO) || !aligned16(dk) ||
+      !aligned16(dv))
+    return FA_ERR_INVALID_ARG;
+  Problem pb;
+  int st = make_problem(&pb, B, H, N, d, scale, causal, cu_seqlens, total_tokens, dtype, true);
+  if (st != FA_OK) return st;
+  if (dropout && (st = set_dropout(&pb, dropout_p, seed, offset)) != FA_OK) return st;
+  BwdArgs a;
+  std::memset(&a, 0, sizeof(a));
+  if ((st = set_workspace(&a, workspace, workspace_bytes_, pb.T, H, d)) != FA_OK) return st;
+  // Q and dO stream in tiles of 64 rows at d = 128 and 128 rows at d = 64; K and V in 128-row tiles
+  const int bq = (d == 128) ? 64 : 128;
+  if (!encode_tmap(&a.tm_q, q, pb.T, H, d, pb.bf16, bq) || !encode_tmap(&a.tm_k, k, pb.T, H, d, pb.bf16, 128) ||
+      !encode_tmap(&a.tm_v, v, pb.T, H, d, pb.bf16, 128) || !encode_tmap(&a.tm_do, dO, pb.T, H, d, pb.bf16, bq) ||
+      !encode_tmap_f32(&a.tm_dq, a.dq_acc, pb.T, H, d, bq))
+    return FA_ERR_UNSUPPORTED;
+  a.q = q;
+  a.k = k;
+  a.lse = lse;
+  a.dO = dO;
+  a.dk = dk;
+  a.dv = dv;
+  return map_launch(launch_bwd_main(pb, a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" {
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+           float scale, int causal, const int32_t* cu_seqlens, int total_tokens, int dtype, fa_stream_t stream) {
+  return fwd_impl(q, k, v, o, lse, B, H, N, d, scale, causal, cu_seqlens, total_tokens, dtype, false, 0.f, 0, 0, stream);
+}
+
+int fa_fwd_dropout(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                   float scale, int causal, const int32_t* cu_seqlens, int total_tokens, int dtype, float dropout_p,
+                   uint64_t seed, uint32_t offset, fa_stream_t stream) {
+  return fwd_impl(q, k, v, o, lse, B, H, N, d, scale, causal, cu_seqlens, total_tokens, dtype, true, dropout_p, seed,
+                  offset, stream);
 }
 
 size_t fa_bwd_workspace_bytes(int total_tokens, int H, int d) {
@@ -148,28 +208,8 @@ int fa_bwd_preprocess(const void* o, const void* dO, int B, int H, int N, int d,
 int fa_bwd_main(const void* q, const void* k, const void* v, const float* lse, const void* dO, void* dk, void* dv,
                 int B, int H, int N, int d, float scale, int causal, const int32_t* cu_seqlens, int total_tokens,
                 int dtype, void* workspace, size_t workspace_bytes_, fa_stream_t stream) {
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned4(lse) || !aligned16(dO) || !aligned16(dk) ||
-      !aligned16(dv))
-    return FA_ERR_INVALID_ARG;
-  Problem pb;
-  int st = make_problem(&pb, B, H, N, d, scale, causal, cu_seqlens, total_tokens, dtype, true);
-  if (st != FA_OK) return st;
-  BwdArgs a;
-  std::memset(&a, 0, sizeof(a));
-  if ((st = set_workspace(&a, workspace, workspace_bytes_, pb.T, H, d)) != FA_OK) return st;
-  // Q and dO stream in tiles of 64 rows at d = 128 and 128 rows at d = 64; K and V in 128-row tiles
-  const int bq = (d == 128) ? 64 : 128;
-  if (!encode_tmap(&a.tm_q, q, pb.T, H, d, pb.bf16, bq) || !encode_tmap(&a.tm_k, k, pb.T, H, d, pb.bf16, 128) ||
-      !encode_tmap(&a.tm_v, v, pb.T, H, d, pb.bf16, 128) || !encode_tmap(&a.tm_do, dO, pb.T, H, d, pb.bf16, bq) ||
-      !encode_tmap_f32(&a.tm_dq, a.dq_acc, pb.T, H, d, bq))
-    return FA_ERR_UNSUPPORTED;
-  a.q = q;
-  a.k = k;
-  a.lse = lse;
-  a.dO = dO;
-  a.dk = dk;
-  a.dv = dv;
-  return map_launch(launch_bwd_main(pb, a, reinterpret_cast<cudaStream_t>(stream)));
+  return bwd_main_impl(q, k, v, lse, dO, dk, dv, B, H, N, d, scale, causal, cu_seqlens, total_tokens, dtype, false,
+                       0.f, 0, 0, workspace, workspace_bytes_, stream);
 }
 
 int fa_bwd_postprocess(void* dq, int B, int H, int N, int d, float scale, const int32_t* cu_seqlens,
@@ -202,6 +242,31 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
   if (st != FA_OK) return st;
   st = fa_bwd_main(q, k, v, lse, dO, dk, dv, B, H, N, d, scale, causal, cu_seqlens, total_tokens, dtype, workspace,
                    workspace_bytes_, stream);
+  if (st != FA_OK) return st;
+  return fa_bwd_postprocess(dq, B, H, N, d, scale, cu_seqlens, total_tokens, dtype, workspace, workspace_bytes_,
+                            stream);
+}
+
+int fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                   void* dq, void* dk, void* dv, int B, int H, int N, int d, float scale, int causal,
+                   const int32_t* cu_seqlens, int total_tokens, int dtype, float dropout_p, uint64_t seed,
+                   uint32_t offset, void* workspace, size_t workspace_bytes_, fa_stream_t stream) {
+  // validate everything before launching anything
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(lse) || !aligned16(dO) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_INVALID_ARG;
+  Problem pb;
+  int st = make_problem(&pb, B, H, N, d, scale, causal, cu_seqlens, total_tokens, dtype, true);
+  if (st != FA_OK) return st;
+  if ((st = set_dropout(&pb, dropout_p, seed, offset)) != FA_OK) return st;
+  BwdArgs a;
+  std::memset(&a, 0, sizeof(a));
+  if ((st = set_workspace(&a, workspace, workspace_bytes_, pb.T, H, d)) != FA_OK) return st;
+  // D = rowsum(dO ∘ O) holds with dropout too (O is the dropped output), so pre and post are shared
+  st = fa_bwd_preprocess(o, dO, B, H, N, d, cu_seqlens, total_tokens, dtype, workspace, workspace_bytes_, stream);
+  if (st != FA_OK) return st;
+  st = bwd_main_impl(q, k, v, lse, dO, dk, dv, B, H, N, d, scale, causal, cu_seqlens, total_tokens, dtype, true,
+                     dropout_p, seed, offset, workspace, workspace_bytes_, stream);
   if (st != FA_OK) return st;
   return fa_bwd_postprocess(dq, B, H, N, d, scale, cu_seqlens, total_tokens, dtype, workspace, workspace_bytes_,
                             stream);

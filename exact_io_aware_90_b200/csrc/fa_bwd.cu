@@ -111,6 +111,7 @@ struct BwdParams {
   float scale;
   float scale_log2;
   uint64_t timeout_ns;
+  Dropout drop;
 };
 
 constexpr int kBwdThreads = 384;  // 3 warpgroups
@@ -226,7 +227,7 @@ __device__ __forceinline__ void bwd_issue_dq(uint32_t d_tmem, uint64_t da, uint6
   for (int kk = 0; kk < kBK / 16; ++kk) mma_ss(d_tmem, da + ((kk * 2048) >> 4), db + ((kk * 2048) >> 4), IDESC, kk > 0 ? 1u : 0u);
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool DROP>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -497,9 +498,38 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int q_lo = p.causal ? key - i0 : 0;  // first visible column
       const int q_hi = (key < L) ? L - i0 : -1;  // one past the last visible column
       const bool full = __all_sync(0xffffffffu, q_lo <= 0 && q_hi >= BQ);  // no masking in this tile
+      // dropout: keep bits of this key for the BQ queries of the step (bit r of word w = query 32w + r),
+      // one Philox call per 4 queries; dV takes the dropped Pᵀ, dS the mask applied to dPᵀ
+      uint32_t qmask[BQ / 32];
+#pragma unroll
+      for (int w = 0; w < BQ / 32; ++w) qmask[w] = ~0u;
+      if constexpr (DROP) {
+        const uint32_t bh = (uint32_t)(b * p.H + h), kg = (uint32_t)key >> 2, ksel = 8u * ((uint32_t)key & 3u);
+#pragma unroll
+        for (int w = 0; w < BQ / 32; ++w) {
+          uint32_t mw = 0u;
+#pragma unroll 1
+          for (int g = 0; g < 8; ++g) {
+            const uint4 r4 = philox4x32_10(kg, (uint32_t)i0 / 4u + 8u * w + g, bh, p.drop.offset, p.drop.seed_lo,
+                                           p.drop.seed_hi);
+            if (((r4.x >> ksel) & 0xFFu) >= p.drop.t) mw |= 1u << (4 * g);
+            if (((r4.y >> ksel) & 0xFFu) >= p.drop.t) mw |= 1u << (4 * g + 1);
+            if (((r4.z >> ksel) & 0xFFu) >= p.drop.t) mw |= 1u << (4 * g + 2);
+            if (((r4.w >> ksel) & 0xFFu) >= p.drop.t) mw |= 1u << (4 * g + 3);
+          }
+          qmask[w] = mw;
+        }
+#pragma unroll
+        for (int w = 0; w < BQ / 32; ++w) asm volatile("" : "+r"(qmask[w]));  // materialised before Sᵀ is loaded
+      }
       if (!warp_wait_b(bar(C::B_SFULL), it & 1, wd)) { ok = false; break; }
       tc_fence_after();
       const float2 c2 = make_float2(c, c);
+      const float ks = DROP ? p.drop.keep_scale : 1.f;
+      auto mk = [&](int col) -> float {  // dropout factor of query column col (0 or 1/(1 − p))
+        if constexpr (!DROP) return 1.f;
+        return ((qmask[col >> 5] >> (col & 31)) & 1u) ? ks : 0.f;
+      };
       float pt[BQ];
       {
         uint32_t sr[BQ];
@@ -522,7 +552,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int q = 0; q < BQ / 64; ++q) {
         uint32_t pk[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) pk[i] = pack2<BF16>(pt[64 * q + 2 * i], pt[64 * q + 2 * i + 1]);
+        for (int i = 0; i < 32; ++i)
+          pk[i] = pack2<BF16>(pt[64 * q + 2 * i] * mk(64 * q + 2 * i), pt[64 * q + 2 * i + 1] * mk(64 * q + 2 * i + 1));
         tmem_st32(tST + 32u * q, pk);
       }
       tmem_wait_st();
@@ -562,8 +593,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int col = 32 * q + 2 * i;
-          const float2 dd = __fadd2_rn(make_float2(__uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1])),
-                                       make_float2(nd[2 * i], nd[2 * i + 1]));
+          const float2 dpv = make_float2(__uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1]));
+          const float2 dd = DROP ? __ffma2_rn(dpv, make_float2(mk(col), mk(col + 1)), make_float2(nd[2 * i], nd[2 * i + 1]))
+                                 : __fadd2_rn(dpv, make_float2(nd[2 * i], nd[2 * i + 1]));
           const float2 ds = __fmul2_rn(make_float2(pt[col], pt[col + 1]), dd);
           dsk[i] = pack2<BF16>(ds.x, ds.y);
         }
@@ -747,11 +779,11 @@ cudaError_t launch_bwd_post(const Problem& pb, const BwdArgs& a, cudaStream_t st
   return cudaPeekAtLastError();
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool DROP>
 static cudaError_t launch_main_t(const Problem& pb, const BwdArgs& a, cudaStream_t stream) {
   using C = BwdCfg<D>;
   static bool configured = false;
-  auto kern = fa_bwd_main_kernel<D, BF16>;
+  auto kern = fa_bwd_main_kernel<D, BF16, DROP>;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
@@ -774,14 +806,21 @@ static cudaError_t launch_main_t(const Problem& pb, const BwdArgs& a, cudaStream
   p.scale = pb.scale;
   p.scale_log2 = pb.scale * 1.4426950408889634f;
   p.timeout_ns = pb.timeout_ns;
+  p.drop = pb.drop;
   const long long units = (long long)pb.B * pb.H * p.num_kblocks;
   kern<<<dim3((unsigned)units), dim3(kBwdThreads), C::SMEM_BYTES, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, a.tm_dq, p);
   return cudaPeekAtLastError();
 }
 
+template <bool DROP>
+static cudaError_t launch_main_d(const Problem& pb, const BwdArgs& a, cudaStream_t stream) {
+  if (pb.d == 128)
+    return pb.bf16 ? launch_main_t<128, true, DROP>(pb, a, stream) : launch_main_t<128, false, DROP>(pb, a, stream);
+  return pb.bf16 ? launch_main_t<64, true, DROP>(pb, a, stream) : launch_main_t<64, false, DROP>(pb, a, stream);
+}
+
 cudaError_t launch_bwd_main(const Problem& pb, const BwdArgs& a, cudaStream_t stream) {
-  if (pb.d == 128) return pb.bf16 ? launch_main_t<128, true>(pb, a, stream) : launch_main_t<128, false>(pb, a, stream);
-  return pb.bf16 ? launch_main_t<64, true>(pb, a, stream) : launch_main_t<64, false>(pb, a, stream);
+  return pb.drop.t != 0u ? launch_main_d<true>(pb, a, stream) : launch_main_d<false>(pb, a, stream);
 }
 
 // ============================================================================ watchdog self-test

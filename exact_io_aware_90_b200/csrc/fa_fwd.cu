@@ -52,6 +52,7 @@ struct FwdParams {
   int heads_group;   // heads per L2 group in the unit order
   float scale_log2;  // scale · log2(e)
   uint64_t timeout_ns;
+  Dropout drop;
 };
 
 constexpr int kFwdThreads = 384;  // 3 warpgroups
@@ -144,7 +145,7 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint6
 // are [tok0, tok0 + L), head h; nkv[t] KV tiles for Q tile t (0 when the tile
 // lies past the end of the sequence), n_iter = max(nkv[0], nkv[1]).
 struct FwdUnit {
-  int tok0, L, q0, h;
+  int tok0, L, q0, h, b;
   int nkv[2];
   int n_iter;
 };
@@ -163,6 +164,7 @@ __device__ __forceinline__ bool decode_unit(const FwdParams& p, int unit, FwdUni
   const int qb = nqb - 1 - r / g_heads;
   const int bh = group * G + r % g_heads;
   const int b = bh / p.H;
+  u.b = b;
   u.h = bh - b * p.H;
   if (p.cu_seqlens != nullptr) {
     u.tok0 = __ldg(p.cu_seqlens + b);
@@ -194,7 +196,7 @@ __device__ __forceinline__ bool warp_test(uint32_t bar, uint32_t parity) {
   return __all_sync(0xffffffffu, mbar_test_wait(bar, parity));
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool DROP>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -555,6 +557,29 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       float ell = 0.f;
       for (int j = 0; j < my_nkv; ++j) {
         const uint32_t step = sn + j;
+        // dropout: keep bits of this row's 128 keys (bit c of word w = key 32w + c of the tile), one
+        // Philox call per 4 keys; ℓ takes the undropped values, P·V the dropped and rescaled ones
+        // (computed while S(t, j) is still on the tensor core)
+        uint32_t kmask[4] = {~0u, ~0u, ~0u, ~0u};
+        if constexpr (DROP) {
+          const uint32_t bh = (uint32_t)(U.b * p.H + U.h), qb = (uint32_t)row >> 2, rsel = (uint32_t)row & 3u;
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            uint32_t mw = 0u;
+#pragma unroll 1
+            for (int g = 0; g < 8; ++g) {
+              const uint4 r4 = philox4x32_10((uint32_t)(j * kBN) / 4u + 8u * w + g, qb, bh, p.drop.offset,
+                                             p.drop.seed_lo, p.drop.seed_hi);
+              const uint32_t word = rsel == 0 ? r4.x : rsel == 1 ? r4.y : rsel == 2 ? r4.z : r4.w;
+#pragma unroll
+              for (int c4 = 0; c4 < 4; ++c4)
+                if (((word >> (8 * c4)) & 0xFFu) >= p.drop.t) mw |= 1u << (4 * g + c4);
+            }
+            kmask[w] = mw;
+          }
+#pragma unroll
+          for (int w = 0; w < 4; ++w) asm volatile("" : "+r"(kmask[w]));  // materialised before S is loaded
+        }
         if (!warp_wait(bar(C::B_SFULL + t), step & 1, wd)) { ok = false; break; }
         tc_fence_after();
         // one 128-column load and one 64-column store per tile: fewer, larger tensor-memory accesses
@@ -591,6 +616,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
         const float2 nm2 = make_float2(neg_m, neg_m);
         float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        const float ks = DROP ? p.drop.keep_scale : 1.f;
+        auto dropped = [&](float2 e, int i) -> float2 {  // pair i = keys 2i, 2i + 1 of the tile
+          if constexpr (!DROP) return e;
+          const uint32_t bits = kmask[(2 * i) >> 5] >> ((2 * i) & 31);
+          return make_float2((bits & 1u) ? e.x * ks : 0.f, (bits & 2u) ? e.y * ks : 0.f);
+        };
         if (!split_p && !need_mask && PolyMask<D>::value != 0u) {
           // unmasked tile: part of the exponentials on the FMA pipe, interleaved with the MUFU ones
           uint32_t pk[64];
@@ -601,7 +632,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             if ((PolyMask<D>::value >> (i & 7)) & 1u) e = exp2_poly2(x);
             else e = make_float2(ex2(x.x), ex2(x.y));
             acc[i & 3] = __fadd2_rn(acc[i & 3], e);
-            pk[i] = pack2<BF16>(e.x, e.y);
+            const float2 ed = dropped(e, i);
+            pk[i] = pack2<BF16>(ed.x, ed.y);
           }
           tmem_st64(tS, pk);
         } else if (!split_p) {
@@ -612,7 +644,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             const float2 x = __ffma2_rn(make_float2(sv[2 * i], sv[2 * i + 1]), c2, nm2);
             const float2 e = make_float2(ex2(x.x), ex2(x.y));
             acc[i & 3] = __fadd2_rn(acc[i & 3], e);
-            pk[i] = pack2<BF16>(e.x, e.y);
+            const float2 ed = dropped(e, i);
+            pk[i] = pack2<BF16>(ed.x, ed.y);
           }
           tmem_st64(tS, pk);
         } else {
@@ -626,9 +659,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               const float2 x = __ffma2_rn(make_float2(sv[idx], sv[idx + 1]), c2, nm2);
               const float2 e = make_float2(ex2(x.x), ex2(x.y));
               acc[i & 3] = __fadd2_rn(acc[i & 3], e);
-              hi[i] = pack2<BF16>(e.x, e.y);
+              const float2 ed = dropped(e, 16 * q + i);
+              hi[i] = pack2<BF16>(ed.x, ed.y);
               const float2 hf = unpack2<BF16>(hi[i]);
-              lo[i] = pack2<BF16>(e.x - hf.x, e.y - hf.y);
+              lo[i] = pack2<BF16>(ed.x - hf.x, ed.y - hf.y);
             }
             tmem_st16(tS + 16u * q, hi);
             tmem_st16(tS + 64u + 16u * q, lo);
@@ -700,11 +734,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   }
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool DROP>
 static cudaError_t launch_fwd_t(const Problem& pb, const FwdArgs& a, cudaStream_t stream) {
   using C = FwdCfg<D>;
   static bool configured = false;  // per instantiation
-  auto kern = fa_fwd_kernel<D, BF16>;
+  auto kern = fa_fwd_kernel<D, BF16, DROP>;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
@@ -723,14 +757,21 @@ static cudaError_t launch_fwd_t(const Problem& pb, const FwdArgs& a, cudaStream_
   p.heads_group = 8;
   p.scale_log2 = pb.scale * 1.4426950408889634f;
   p.timeout_ns = pb.timeout_ns;
+  p.drop = pb.drop;
   const long long units = (long long)pb.B * pb.H * p.num_qblocks;
   kern<<<dim3((unsigned)units), dim3(kFwdThreads), C::SMEM_BYTES, stream>>>(a.tm_q, a.tm_k, a.tm_v, p);
   return cudaPeekAtLastError();
 }
 
+template <bool DROP>
+static cudaError_t launch_fwd_d(const Problem& pb, const FwdArgs& a, cudaStream_t stream) {
+  if (pb.d == 128)
+    return pb.bf16 ? launch_fwd_t<128, true, DROP>(pb, a, stream) : launch_fwd_t<128, false, DROP>(pb, a, stream);
+  return pb.bf16 ? launch_fwd_t<64, true, DROP>(pb, a, stream) : launch_fwd_t<64, false, DROP>(pb, a, stream);
+}
+
 cudaError_t launch_fwd(const Problem& pb, const FwdArgs& a, cudaStream_t stream) {
-  if (pb.d == 128) return pb.bf16 ? launch_fwd_t<128, true>(pb, a, stream) : launch_fwd_t<128, false>(pb, a, stream);
-  return pb.bf16 ? launch_fwd_t<64, true>(pb, a, stream) : launch_fwd_t<64, false>(pb, a, stream);
+  return pb.drop.t != 0u ? launch_fwd_d<true>(pb, a, stream) : launch_fwd_d<false>(pb, a, stream);
 }
 
 }  // namespace fa

@@ -9,6 +9,16 @@
 
 namespace fa {
 
+// Dropout on P: element (query i, key j) of the sequence/head with global index bh = b·H + h is kept
+// when byte (j mod 4) of word (i mod 4) of Philox(counter (j/4, i/4, bh, offset), key = seed) is at
+// least `t`; kept elements are scaled by keep_scale = 256/(256 − t).
+struct Dropout {
+  uint32_t t;         // threshold byte (0 = no dropout)
+  float keep_scale;
+  uint32_t seed_lo, seed_hi;
+  uint32_t offset;
+};
+
 // Work of one attention call, resolved on the host.
 struct Problem {
   int B, H, N, d, T;
@@ -17,6 +27,7 @@ struct Problem {
   const int32_t* cu_seqlens;  // device pointer or nullptr
   bool bf16;
   uint64_t timeout_ns;
+  Dropout drop;  // drop.t == 0: no dropout
 };
 
 struct FwdArgs {

@@ -191,6 +191,30 @@ __device__ __forceinline__ void ld_shared_v4f(const float* p, float* out) {
                : "r"(smem_u32(p)));
 }
 
+// ---------------------------------------------------------------- counter-based random numbers
+// Philox4x32 with 10 rounds (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy as 1, 2,
+// 3", SC 2011): 128 random bits from a 128-bit counter and a 64-bit key.  Each round takes the full
+// 64-bit products of words 0 and 2 with fixed multipliers and mixes their high halves with words 1,
+// 3 and the round key; the key is bumped by fixed increments between rounds.
+__device__ __forceinline__ uint4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3, uint32_t k0,
+                                               uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r > 0) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    const uint32_t hi0 = __umulhi(0xD2511F53u, c0), lo0 = 0xD2511F53u * c0;
+    const uint32_t hi1 = __umulhi(0xCD9E8D57u, c2), lo1 = 0xCD9E8D57u * c2;
+    const uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+    c0 = n0;
+    c1 = lo1;
+    c2 = n2;
+    c3 = lo0;
+  }
+  return make_uint4(c0, c1, c2, c3);
+}
+
 // ---------------------------------------------------------------- cluster launch control
 // Asks the hardware scheduler to cancel the launch of a CTA of this grid that
 // has not started yet, so that this (already running) CTA can do its work

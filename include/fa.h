@@ -177,6 +177,37 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
                    const int32_t* cu_seqlens, int total_tokens, int dtype, fa_stream_t stream);
 
 /*
+ * Dropout on the attention probabilities (the dropout_p of the SDPA
+ * interface, "Flash Attention 优化", SDPA signature): the forward uses
+ * O = (M ∘ P / (1 − p̂)) V with a keep mask M drawn inside the kernels, and
+ * the backward draws the same mask again instead of storing it.  LSE is that
+ * of the undropped softmax.  Otherwise as fa_fwd / fa_bwd.
+ *   dropout_p  in [0, 1); the decisions compare one random byte with
+ *              t = round(256·dropout_p) (clamped to 255): an element is kept
+ *              when the byte ≥ t, so p̂ = t/256 and kept probabilities are
+ *              scaled by 256/(256 − t).  t = 0 gives exactly fa_fwd / fa_bwd.
+ *   seed       64-bit key of the generator; offset  its fourth counter word
+ *              (advance it between calls that must draw different masks).
+ * Mask of element (query i, key j), positions counted from the start of the
+ * sequence, of sequence b and head h: byte (j mod 4) of output word (i mod 4)
+ * of Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC 2011) with counter
+ * (j/4, i/4, b·H + h, offset) and key (seed low 32 bits, seed high 32 bits).
+ * fa_bwd_dropout needs the same dropout_p, seed and offset as the forward.
+ * Errors as for fa_fwd / fa_bwd; dropout_p outside [0, 1) or NaN returns
+ * FA_ERR_INVALID_ARG.
+ */
+int fa_fwd_dropout(const void* q, const void* k, const void* v, void* o, float* lse,
+                   int B, int H, int N, int d, float scale, int causal,
+                   const int32_t* cu_seqlens, int total_tokens, int dtype,
+                   float dropout_p, uint64_t seed, uint32_t offset, fa_stream_t stream);
+int fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                   const void* dO, void* dq, void* dk, void* dv,
+                   int B, int H, int N, int d, float scale, int causal,
+                   const int32_t* cu_seqlens, int total_tokens, int dtype,
+                   float dropout_p, uint64_t seed, uint32_t offset,
+                   void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/*
  * Decode: one new query token per sequence attends to every key of its
  * sequence in a K/V cache (token-by-token generation, the workload
  * "FlashAttention 短片讲解稿", segment "适用范围与关键结论", sets apart from

@@ -32,7 +32,8 @@ def test_header_declares_the_entry_points():
     names = _declared_functions()
     for n in ["fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_bwd_preprocess", "fa_bwd_main",
               "fa_bwd_postprocess", "fa_check_device_status", "fa_status_string", "fa_set_watchdog_ns",
-              "fa_watchdog_selftest", "fa_version", "fa_bwd_noalloc", "fa_decode", "fa_decode_workspace_bytes"]:
+              "fa_watchdog_selftest", "fa_version", "fa_bwd_noalloc", "fa_decode", "fa_decode_workspace_bytes",
+              "fa_fwd_dropout", "fa_bwd_dropout"]:
         assert n in names
 
 
@@ -99,6 +100,16 @@ def test_backward_rejects_invalid_arguments(fa):
     assert fa.fa_bwd_postprocess(P16, 2, 4, 256, 64, float("nan"), None, 512, 0, P16, ws, None) == fa.FA_ERR_INVALID_ARG
     assert fa.fa_bwd_main(P16, P16, P16, P16, P16, P16, P16, 2, 4, 256, 64, 0.125, 3, None, 512, 0, P16, ws,
                           None) == fa.FA_ERR_INVALID_ARG
+
+
+def test_dropout_rejects_invalid_probability(fa):
+    args = [P16] * 5 + [2, 4, 256, 64, 0.125, 0, None, 512, 0]
+    for p in (-0.1, 1.0, 1.5, float("nan")):
+        assert fa.fa_fwd_dropout(*args, p, 1, 0, None) == fa.FA_ERR_INVALID_ARG
+    ws = fa.fa_bwd_workspace_bytes(512, 4, 64)
+    bargs = [P16] * 9 + [2, 4, 256, 64, 0.125, 0, None, 512, 0]
+    assert fa.fa_bwd_dropout(*bargs, 1.0, 1, 0, P16, ws, None) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_bwd_dropout(*bargs, 0.1, 1, 0, P16, ws - 1, None) == fa.FA_ERR_INVALID_ARG
 
 
 def test_decode_workspace_bytes(fa):
