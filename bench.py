@@ -64,14 +64,15 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
-def load_traffic(kernel, workload):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on this kernel source."""
+def load_traffic(kernel, workload, dropout_p=0.0):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on this kernel source
+    (entries of the dropout variant are keyed "<workload>+dropout<p>")."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
-    e = d.get(kernel, {}).get(workload)
+    e = d.get(kernel, {}).get(workload if dropout_p <= 0.0 else f"{workload}+dropout{dropout_p:g}")
     if not e or e.get("source_hash") != kernel_source_hash():
         return None
     return e.get("bytes_per_launch")
@@ -232,11 +233,32 @@ def run_gpu(args, world, rank, local, pg):
         check(fa.fa_bwd_postprocess(dq.data_ptr(), B, H, N, d, scale, cu_p, T, dt, ws.data_ptr(), ws_bytes, sp),
               "fa_bwd_postprocess")
 
-    stages = [("fa_fwd_kernel", fwd)]
-    if backward:
-        stages += [("fa_bwd_pre_kernel", bwd_pre), ("fa_bwd_main_kernel", bwd_main),
-                   ("fa_bwd_post_kernel", bwd_post)]
-    flops_of = {"fa_fwd_kernel": flops_fwd, "fa_bwd_main_kernel": flops_bwd}
+    drop_p, drop_seed, drop_off = float(args.dropout), 0x5EED, 0
+
+    def fwd_drop():
+        check(fa.fa_fwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, N, d,
+                                scale, causal, cu_p, T, dt, drop_p, drop_seed, drop_off, sp), "fa_fwd_dropout")
+
+    def bwd_drop():  # one call: D = rowsum(dO∘O), the main kernel, dQ conversion (three launches)
+        check(fa.fa_bwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                                dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, scale, causal, cu_p, T, dt,
+                                drop_p, drop_seed, drop_off, ws.data_ptr(), ws_bytes, sp), "fa_bwd_dropout")
+
+    if drop_p > 0.0:
+        stages = [("fa_fwd_kernel", fwd_drop)]
+        launches = {"fa_fwd_kernel": 1}
+        if backward:
+            stages += [("fa_bwd_dropout", bwd_drop)]
+            launches["fa_bwd_dropout"] = 3
+        flops_of = {"fa_fwd_kernel": flops_fwd, "fa_bwd_dropout": flops_bwd}
+    else:
+        stages = [("fa_fwd_kernel", fwd)]
+        if backward:
+            stages += [("fa_bwd_pre_kernel", bwd_pre), ("fa_bwd_main_kernel", bwd_main),
+                       ("fa_bwd_post_kernel", bwd_post)]
+        launches = {name: 1 for name, _ in stages}
+        flops_of = {"fa_fwd_kernel": flops_fwd, "fa_bwd_main_kernel": flops_bwd}
+    drop_kw = dict(dropout_p=drop_p, seed=drop_seed, offset=drop_off) if drop_p > 0.0 else {}
 
     def one_step(record):
         flush.fill_(1)  # outside the timed events
@@ -294,11 +316,11 @@ def run_gpu(args, world, rank, local, pg):
         if backward:
             do.copy_(hdo, non_blocking=True)
         fa.attention_forward(q, k, v, causal=bool(causal), scale=scale, cu_seqlens=cu,
-                             max_seqlen=N if cu is not None else None, batch=B, out=o, lse=lse, stream=sp)
+                             max_seqlen=N if cu is not None else None, batch=B, out=o, lse=lse, stream=sp, **drop_kw)
         if backward:
             fa.attention_backward(q, k, v, o, lse, do, causal=bool(causal), scale=scale, cu_seqlens=cu,
                                   max_seqlen=N if cu is not None else None, batch=B, dq=dq, dk=dk, dv=dv,
-                                  workspace=ws, stream=sp)
+                                  workspace=ws, stream=sp, **drop_kw)
         ho.copy_(o, non_blocking=True)
         hl.copy_(lse, non_blocking=True)
         if backward:
@@ -324,9 +346,10 @@ def run_gpu(args, world, rank, local, pg):
     # ---- the forward alone (inference use): same workload, same L2 flush, back-to-back steps
     fwd_only = None
     if backward:
+        fwd_fn = stages[0][1]
         for _ in range(args.warmup):
             flush.fill_(1)
-            fwd()
+            fwd_fn()
         torch.cuda.synchronize(dev)
         fo_clocks = ClockSampler(dev)
         if pg is not None:
@@ -338,7 +361,7 @@ def run_gpu(args, world, rank, local, pg):
             flush.fill_(1)  # outside the timed events
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
-            fwd()
+            fwd_fn()
             b.record(stream)
             fo.append((a, b))
         torch.cuda.synchronize(dev)
@@ -359,10 +382,12 @@ def run_gpu(args, world, rank, local, pg):
                 "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
                 "frac_of_sustained": round(achieved / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]), 4),
                 "peak_source": peaks["source"] + " (burst bf16; kernels timed one launch at a time)",
-                "traffic": load_traffic(dom, wname), "launch_ms": round(dom_ms, 4)}
+                "traffic": load_traffic(dom, wname, drop_p), "launch_ms": round(dom_ms, 4)}
+        if dom == "fa_bwd_dropout":
+            roof["note"] = "time of the whole dropout backward call (D = rowsum(dO∘O), main kernel, dQ conversion)"
     else:
         roof = {"kernel": dom, "bound": "hbm", "achieved": None, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": None, "traffic": load_traffic(dom, wname)}
+                "frac": None, "traffic": load_traffic(dom, wname, drop_p)}
     kernels = {}
     for name, ms in per_kernel.items():
         e = {"ms": round(ms, 4)}
@@ -387,7 +412,8 @@ def run_gpu(args, world, rank, local, pg):
         "config": {"workload": wname, "B": B, "H": H, "N": N, "d": d, "causal": bool(causal),
                    "varlen": inp_h.cu_seqlens is not None, "tokens": T, "step": "fwd+bwd" if backward else "fwd",
                    "flops_per_step": flops_step, "l2": "flushed before every step (256 MiB write, outside the events)",
-                   "parallelism": f"replicas x{world} (independent workloads per GPU)"},
+                   "parallelism": f"replicas x{world} (independent workloads per GPU)",
+                   "dropout_p": drop_p},
         "fwd_tflops": round(flops_fwd / (per_kernel["fa_fwd_kernel"] * 1e-3) / 1e12, 1),
         "fwd_frac_of_peak": round(flops_fwd / (per_kernel["fa_fwd_kernel"] * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
         "pct_of_peak": round(100.0 * value / world / peaks["bf16_tflops"], 2),
@@ -403,11 +429,12 @@ def run_gpu(args, world, rank, local, pg):
         "roofline": roof,
         "e2e": {"value": round(world * flops_step / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": len(stages) * args.steps,
+        "gpu_launches": sum(launches.values()) * args.steps,
         "clocks": clk,
     }
     if rank == 0 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(inp_h, budget_s=args.cpu_budget)
+        out["cpu_baseline"] = (cpu_baseline_dropout(inp_h, drop_p, budget_s=args.cpu_budget) if drop_p > 0.0 else
+                               cpu_baseline(inp_h, budget_s=args.cpu_budget))
     return out
 
 
@@ -516,7 +543,8 @@ def run_gpu_decode(args, world, rank, local, pg):
         "config": {"workload": wname, "B": B, "H": H, "Nk": Nk, "d": d, "varlen": cu is not None, "keys": Tk,
                    "step": "decode", "flops_per_step": flops,
                    "l2": "flushed before every step (256 MiB write, outside the events)",
-                   "parallelism": f"replicas x{world} (independent workloads per GPU)"},
+                   "parallelism": f"replicas x{world} (independent workloads per GPU)",
+                   "dropout_p": drop_p},
         "roofline": {"kernel": "fa_decode_split_kernel + fa_decode_merge_kernel", "bound": "hbm",
                      "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None,
@@ -622,12 +650,48 @@ def cpu_baseline(inp, budget_s=15.0):
                       f"sequence 0 ({L} query rows x all visible keys each), {tot_t:.2f} s"}
 
 
+def oracle_sample_dropout(inp, rows, p, head=0):
+    """fp64 dropout oracle forward+backward on one head of the first `rows` tokens of sequence 0 (a
+    sequence of that length).  Returns (seconds, flops by the GPU arm's convention)."""
+    import oracle
+    R = min(rows, inp.seqlens[0])
+    sl = (slice(0, R), slice(head, head + 1))
+    q, k, v = inp.q[sl], inp.k[sl], inp.v[sl]
+    t0 = time.perf_counter()
+    oracle.attention_forward_dropout(q, k, v, inp.scale, inp.causal, p, 0x5EED, 0, B=1, N=R)
+    if inp.do is not None:
+        oracle.attention_backward_dropout(q, k, v, inp.do[sl], inp.scale, inp.causal, p, 0x5EED, 0, B=1, N=R)
+    dt = time.perf_counter() - t0
+    pairs = R * (R + 1) / 2 if inp.causal else R * R
+    return dt, 4.0 * inp.d * pairs * (3.5 if inp.do is not None else 1.0)
+
+
+def dropout_sample_rows(inp, p, budget_s):
+    """Largest power-of-two prefix (from 256) whose dropout oracle run stays within about budget_s."""
+    R = 256
+    dt, _ = oracle_sample_dropout(inp, R, p)
+    while 2 * R <= inp.seqlens[0] and dt * 4 < budget_s:
+        R *= 2
+        dt, _ = oracle_sample_dropout(inp, R, p)
+    return R
+
+
+def cpu_baseline_dropout(inp, p, budget_s=15.0):
+    R = dropout_sample_rows(inp, p, budget_s / 2)
+    dt, f = oracle_sample_dropout(inp, R, p)
+    return {"value": round(f / dt / 1e12, 6), "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"fp64 NumPy dropout oracle (p = {p}), {'fwd+bwd' if inp.do is not None else 'fwd'} of one head "
+                      f"of the first {R} tokens of sequence 0 as a sequence of that length, {dt:.2f} s"}
+
+
 def run_reference(args, rank):
     import workloads
     if args.workload in workloads.DECODE_WORKLOADS:
         return run_reference_decode(args)
     spec = workloads.WORKLOADS[args.workload]
     inp = workloads.make_workload(args.workload, backward=spec["backward"])
+    if args.dropout > 0.0:
+        return run_reference_dropout(args, inp)
     L = inp.seqlens[0]
     # size each step so the whole run stays within ~3 minutes
     dt0, _ = oracle_sample(inp, 128)
@@ -659,6 +723,31 @@ def run_reference(args, rank):
     }
 
 
+def run_reference_dropout(args, inp):
+    p = float(args.dropout)
+    R = dropout_sample_rows(inp, p, 180.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_sample_dropout(inp, R, p)
+    times, flops = [], 0.0
+    for _ in range(args.steps):
+        dt, flops = oracle_sample_dropout(inp, R, p)
+        times.append(dt)
+    ms = 1e3 * float(np.mean(times))
+    value = flops / (ms * 1e-3) / 1e12
+    sample = (f"fp64 NumPy dropout oracle (p = {p}) {'fwd+bwd' if inp.do is not None else 'fwd'} of one head of the "
+              f"first {R} tokens of sequence 0 per step")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "B": inp.B, "H": inp.H, "N": inp.N, "d": inp.d,
+                   "causal": inp.causal, "dropout_p": p, "sample_tokens": R},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -668,6 +757,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--dropout", type=float, default=0.0,
+                    help="dropout probability on P (attention workloads; 0 = the plain step)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     args.steps = max(1, args.steps)

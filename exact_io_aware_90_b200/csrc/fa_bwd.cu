@@ -487,6 +487,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int kr = 32 * warp + lane;  // key row within the tile
     const int key = k0 + kr;          // position in the sequence
     const float c = p.scale_log2;
+    const uint32_t keep_bias = keep_flag_bias(p.drop.t);     // used by the dropout variant only
+    const uint32_t ks_bits = __float_as_uint(p.drop.keep_scale);
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
       const int i0 = (i_begin + it) * BQ;
@@ -498,37 +500,43 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int q_lo = p.causal ? key - i0 : 0;  // first visible column
       const int q_hi = (key < L) ? L - i0 : -1;  // one past the last visible column
       const bool full = __all_sync(0xffffffffu, q_lo <= 0 && q_hi >= BQ);  // no masking in this tile
-      // dropout: keep bits of this key for the BQ queries of the step (bit r of word w = query 32w + r),
-      // one Philox call per 4 queries; dV takes the dropped Pᵀ, dS the mask applied to dPᵀ
-      uint32_t qmask[BQ / 32];
-#pragma unroll
-      for (int w = 0; w < BQ / 32; ++w) qmask[w] = ~0u;
+      // dropout: the random bytes of this key for the BQ queries of the step, word g = queries 4g .. 4g+3
+      // (byte = query offset).  One Philox call covers the 4 keys of a lane quad (key mod 4 = lane mod 4)
+      // × 4 queries: each lane of the quad makes BQ/16 of the step's calls, reorders its call's bytes
+      // from (query word, key byte) to (key word, query byte), and the quad exchanges words.
+      uint32_t rw[DROP ? BQ / 4 : 1];
       if constexpr (DROP) {
-        const uint32_t bh = (uint32_t)(b * p.H + h), kg = (uint32_t)key >> 2, ksel = 8u * ((uint32_t)key & 3u);
+        const uint32_t bh = (uint32_t)(b * p.H + h), kg = (uint32_t)key >> 2;
+        const uint32_t g0 = (uint32_t)i0 / 4u + (uint32_t)(lane & 3);
 #pragma unroll
-        for (int w = 0; w < BQ / 32; ++w) {
-          uint32_t mw = 0u;
-#pragma unroll 1
-          for (int g = 0; g < 8; ++g) {
-            const uint4 r4 = philox4x32_10(kg, (uint32_t)i0 / 4u + 8u * w + g, bh, p.drop.offset, p.drop.seed_lo,
-                                           p.drop.seed_hi);
-            if (((r4.x >> ksel) & 0xFFu) >= p.drop.t) mw |= 1u << (4 * g);
-            if (((r4.y >> ksel) & 0xFFu) >= p.drop.t) mw |= 1u << (4 * g + 1);
-            if (((r4.z >> ksel) & 0xFFu) >= p.drop.t) mw |= 1u << (4 * g + 2);
-            if (((r4.w >> ksel) & 0xFFu) >= p.drop.t) mw |= 1u << (4 * g + 3);
-          }
-          qmask[w] = mw;
+        for (int m = 0; m < BQ / 16; ++m) {
+          const uint4 r4 = philox4x32_10(kg, g0 + 4u * m, bh, p.drop.offset, p.drop.seed_lo, p.drop.seed_hi);
+          const uint32_t a0 = prmt(r4.x, r4.y, 0x5140u), a1 = prmt(r4.x, r4.y, 0x7362u);
+          const uint32_t a2 = prmt(r4.z, r4.w, 0x5140u), a3 = prmt(r4.z, r4.w, 0x7362u);
+          uint32_t x[4] = {prmt(a0, a2, 0x5410u), prmt(a0, a2, 0x7632u), prmt(a1, a3, 0x5410u), prmt(a1, a3, 0x7632u)};
+          quad_transpose(x, lane);
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) rw[4 * m + c4] = x[c4];
         }
-#pragma unroll
-        for (int w = 0; w < BQ / 32; ++w) asm volatile("" : "+r"(qmask[w]));  // materialised before Sᵀ is loaded
       }
+      // words 4·m0 .. 4·(m0 + nm) − 1 of the step (held in registers: parking them in shared memory at
+      // d = 64, where it fits, removed the spills but measured slower)
+      auto drop_words = [&](int m0, int nm, uint32_t* out) {
+        if constexpr (DROP) {
+#pragma unroll
+          for (int k = 0; k < 4 * nm; ++k) out[k] = rw[4 * m0 + k];
+        }
+      };
       if (!warp_wait_b(bar(C::B_SFULL), it & 1, wd)) { ok = false; break; }
       tc_fence_after();
       const float2 c2 = make_float2(c, c);
-      const float ks = DROP ? p.drop.keep_scale : 1.f;
-      auto mk = [&](int col) -> float {  // dropout factor of query column col (0 or 1/(1 − p))
+      // dropout factor (0 or 1/(1 − p)) of the query whose random byte is byte c of word w
+      auto mk = [&](uint32_t w, int c) -> float {
         if constexpr (!DROP) return 1.f;
-        return ((qmask[col >> 5] >> (col & 31)) & 1u) ? ks : 0.f;
+        uint32_t e, o;
+        keep_flags(w, keep_bias, e, o);
+        const uint32_t sel = c == 0 ? 0x9999u : c == 1 ? 0xDDDDu : c == 2 ? 0xBBBBu : 0xFFFFu;
+        return __uint_as_float(prmt(e, o, sel) & ks_bits);  // the keep flag's sign fills all 32 bits
       };
       float pt[BQ];
       {
@@ -550,10 +558,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
 #pragma unroll
       for (int q = 0; q < BQ / 64; ++q) {
+        uint32_t wq[DROP ? 16 : 1];
+        drop_words(4 * q, 4, wq);  // queries 64q .. 64q + 63
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i)
-          pk[i] = pack2<BF16>(pt[64 * q + 2 * i] * mk(64 * q + 2 * i), pt[64 * q + 2 * i + 1] * mk(64 * q + 2 * i + 1));
+          pk[i] = pack2<BF16>(pt[64 * q + 2 * i] * mk(wq[DROP ? i >> 1 : 0], (2 * i) & 3),
+                              pt[64 * q + 2 * i + 1] * mk(wq[DROP ? i >> 1 : 0], (2 * i + 1) & 3));
         tmem_st32(tST + 32u * q, pk);
       }
       tmem_wait_st();
@@ -589,12 +600,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
           for (int v = 0; v < 32; ++v) nd[v] = del_s[32 * q + v];
         }
+        uint32_t wq[DROP ? 8 : 1];
+        drop_words(2 * q, 2, wq);  // queries 32q .. 32q + 31
         uint32_t dsk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int col = 32 * q + 2 * i;
           const float2 dpv = make_float2(__uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1]));
-          const float2 dd = DROP ? __ffma2_rn(dpv, make_float2(mk(col), mk(col + 1)), make_float2(nd[2 * i], nd[2 * i + 1]))
+          const uint32_t w = wq[DROP ? i >> 1 : 0];
+          const float2 dd = DROP ? __ffma2_rn(dpv, make_float2(mk(w, (2 * i) & 3), mk(w, (2 * i + 1) & 3)),
+                                              make_float2(nd[2 * i], nd[2 * i + 1]))
                                  : __fadd2_rn(dpv, make_float2(nd[2 * i], nd[2 * i + 1]));
           const float2 ds = __fmul2_rn(make_float2(pt[col], pt[col + 1]), dd);
           dsk[i] = pack2<BF16>(ds.x, ds.y);

@@ -531,6 +531,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const uint32_t tO = tmem + lane_off + 256u + (uint32_t)(D * t);
     const float c = p.scale_log2;
     const float2 c2 = make_float2(c, c);
+    const uint32_t keep_bias = keep_flag_bias(p.drop.t);  // used by the dropout variant only
     uint32_t un = 0;  // units read
     uint32_t sn = 0;  // S tiles of Q tile t consumed (all units)
     bool ok = true;
@@ -547,6 +548,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const int my_nkv = U.nkv[t];
       if (my_nkv == 0) continue;
       const int row = U.q0 + t * kBM + 32 * quarter + lane;  // position in the sequence
+      const uint32_t drop_bh = (uint32_t)(U.b * p.H + U.h);
       const int key_limit = p.causal ? min(U.L, row + 1) : U.L;
       // A tile whose rows see a single KV tile (the first 128 rows of a causal
       // sequence, or a sequence of at most 128 tokens) averages few values, so
@@ -557,28 +559,23 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       float ell = 0.f;
       for (int j = 0; j < my_nkv; ++j) {
         const uint32_t step = sn + j;
-        // dropout: keep bits of this row's 128 keys (bit c of word w = key 32w + c of the tile), one
-        // Philox call per 4 keys; ℓ takes the undropped values, P·V the dropped and rescaled ones
-        // (computed while S(t, j) is still on the tensor core)
-        uint32_t kmask[4] = {~0u, ~0u, ~0u, ~0u};
+        // dropout: the random bytes of this row's 128 keys, word g = keys 4g .. 4g+3 (byte = key offset).
+        // One Philox call covers 4 keys × the 4 rows of a lane quad (row mod 4 = lane mod 4): each lane
+        // of the quad makes 8 of the tile's 32 calls and the quad exchanges words, so no call is made
+        // twice.  Made while S(t, j) is still on the tensor core (measured faster than making each call
+        // just before its keys are packed).
+        uint32_t rw[DROP ? kBN / 4 : 1];
         if constexpr (DROP) {
-          const uint32_t bh = (uint32_t)(U.b * p.H + U.h), qb = (uint32_t)row >> 2, rsel = (uint32_t)row & 3u;
+          const uint32_t g0 = (uint32_t)(j * kBN) / 4u + (uint32_t)(lane & 3);
 #pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            uint32_t mw = 0u;
-#pragma unroll 1
-            for (int g = 0; g < 8; ++g) {
-              const uint4 r4 = philox4x32_10((uint32_t)(j * kBN) / 4u + 8u * w + g, qb, bh, p.drop.offset,
-                                             p.drop.seed_lo, p.drop.seed_hi);
-              const uint32_t word = rsel == 0 ? r4.x : rsel == 1 ? r4.y : rsel == 2 ? r4.z : r4.w;
+          for (int m = 0; m < kBN / 16; ++m) {
+            const uint4 r4 = philox4x32_10(g0 + 4u * m, (uint32_t)row >> 2, drop_bh, p.drop.offset,
+                                           p.drop.seed_lo, p.drop.seed_hi);
+            uint32_t x[4] = {r4.x, r4.y, r4.z, r4.w};
+            quad_transpose(x, lane);
 #pragma unroll
-              for (int c4 = 0; c4 < 4; ++c4)
-                if (((word >> (8 * c4)) & 0xFFu) >= p.drop.t) mw |= 1u << (4 * g + c4);
-            }
-            kmask[w] = mw;
+            for (int c4 = 0; c4 < 4; ++c4) rw[4 * m + c4] = x[c4];
           }
-#pragma unroll
-          for (int w = 0; w < 4; ++w) asm volatile("" : "+r"(kmask[w]));  // materialised before S is loaded
         }
         if (!warp_wait(bar(C::B_SFULL + t), step & 1, wd)) { ok = false; break; }
         tc_fence_after();
@@ -616,12 +613,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
         const float2 nm2 = make_float2(neg_m, neg_m);
         float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        const float ks = DROP ? p.drop.keep_scale : 1.f;
-        auto dropped = [&](float2 e, int i) -> float2 {  // pair i = keys 2i, 2i + 1 of the tile
-          if constexpr (!DROP) return e;
-          const uint32_t bits = kmask[(2 * i) >> 5] >> ((2 * i) & 31);
-          return make_float2((bits & 1u) ? e.x * ks : 0.f, (bits & 2u) ? e.y * ks : 0.f);
+        // pair i = keys 2i, 2i + 1 packed to 16 bits each: dropped keys zeroed (the 1/(1 − p) factor is
+        // applied to O at the end; ℓ takes the undropped values)
+        auto pair_mask = [&](int i) -> uint32_t {
+          if constexpr (!DROP) return ~0u;
+          uint32_t m01, m23;
+          keep_pair_masks(rw[i >> 1], keep_bias, m01, m23);
+          return (i & 1) ? m23 : m01;
         };
+        auto drop_pair = [&](uint32_t v, int i) -> uint32_t { return DROP ? v & pair_mask(i) : v; };
         if (!split_p && !need_mask && PolyMask<D>::value != 0u) {
           // unmasked tile: part of the exponentials on the FMA pipe, interleaved with the MUFU ones
           uint32_t pk[64];
@@ -632,8 +632,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             if ((PolyMask<D>::value >> (i & 7)) & 1u) e = exp2_poly2(x);
             else e = make_float2(ex2(x.x), ex2(x.y));
             acc[i & 3] = __fadd2_rn(acc[i & 3], e);
-            const float2 ed = dropped(e, i);
-            pk[i] = pack2<BF16>(ed.x, ed.y);
+            pk[i] = drop_pair(pack2<BF16>(e.x, e.y), i);
           }
           tmem_st64(tS, pk);
         } else if (!split_p) {
@@ -644,8 +643,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             const float2 x = __ffma2_rn(make_float2(sv[2 * i], sv[2 * i + 1]), c2, nm2);
             const float2 e = make_float2(ex2(x.x), ex2(x.y));
             acc[i & 3] = __fadd2_rn(acc[i & 3], e);
-            const float2 ed = dropped(e, i);
-            pk[i] = pack2<BF16>(ed.x, ed.y);
+            pk[i] = drop_pair(pack2<BF16>(e.x, e.y), i);
           }
           tmem_st64(tS, pk);
         } else {
@@ -659,10 +657,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               const float2 x = __ffma2_rn(make_float2(sv[idx], sv[idx + 1]), c2, nm2);
               const float2 e = make_float2(ex2(x.x), ex2(x.y));
               acc[i & 3] = __fadd2_rn(acc[i & 3], e);
-              const float2 ed = dropped(e, 16 * q + i);
-              hi[i] = pack2<BF16>(ed.x, ed.y);
-              const float2 hf = unpack2<BF16>(hi[i]);
-              lo[i] = pack2<BF16>(ed.x - hf.x, ed.y - hf.y);
+              const uint32_t h2 = pack2<BF16>(e.x, e.y);
+              const float2 hf = unpack2<BF16>(h2);
+              const uint32_t mk = pair_mask(16 * q + i);
+              hi[i] = h2 & mk;
+              lo[i] = pack2<BF16>(e.x - hf.x, e.y - hf.y) & mk;
             }
             tmem_st16(tS + 16u * q, hi);
             tmem_st16(tS + 64u + 16u * q, lo);
@@ -694,7 +693,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       if (ok && warp_wait(bar(C::B_PVDONE + t), (sn + my_nkv - 1) & 1, wd)) {
         tc_fence_after();
         const bool valid = row < U.L;
-        const float inv = (ell > 0.f) ? 1.f / ell : 0.f;
+        const float inv = (ell > 0.f) ? (DROP ? p.drop.keep_scale : 1.f) / ell : 0.f;
         const size_t obase = ((size_t)(U.tok0 + (valid ? row : 0)) * p.H + U.h) * D;
         uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) + obase * 2;
 #pragma unroll

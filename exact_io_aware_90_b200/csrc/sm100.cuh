@@ -204,15 +204,65 @@ __device__ __forceinline__ uint4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_
       k0 += 0x9E3779B9u;
       k1 += 0xBB67AE85u;
     }
-    const uint32_t hi0 = __umulhi(0xD2511F53u, c0), lo0 = 0xD2511F53u * c0;
-    const uint32_t hi1 = __umulhi(0xCD9E8D57u, c2), lo1 = 0xCD9E8D57u * c2;
-    const uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+    // one 32×32 → 64-bit product per multiplier gives both halves
+    const unsigned long long p0 = (unsigned long long)0xD2511F53u * c0;
+    const unsigned long long p1 = (unsigned long long)0xCD9E8D57u * c2;
+    const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ k0, n2 = (uint32_t)(p0 >> 32) ^ c3 ^ k1;
     c0 = n0;
-    c1 = lo1;
+    c1 = (uint32_t)p1;
     c2 = n2;
-    c3 = lo0;
+    c3 = (uint32_t)p0;
   }
   return make_uint4(c0, c1, c2, c3);
+}
+
+// Byte permute (PTX prmt, default mode): byte n of the result is byte (sel[4n+2:4n]) of {b, a}
+// (a = bytes 0–3, b = bytes 4–7); with sel bit 4n+3 set the selected byte's sign bit fills it.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// 4×4 transpose across the four lanes of a quad (lanes 4u .. 4u+3): on entry lane q holds x[r] meant
+// for lane r of its quad; on exit x[c] is what lane c held for lane q.  Two butterfly exchanges
+// (lane xor 1, then xor 2) of two words each, and selects to put the words in place.
+__device__ __forceinline__ void quad_transpose(uint32_t (&x)[4], int lane) {
+  const bool s = lane & 1, t = lane & 2;
+  // xor 1: keep the words for the rows with this lane's bit 0, pass the others to the partner
+  const uint32_t k0 = s ? x[1] : x[0], k1 = s ? x[3] : x[2];
+  const uint32_t r0 = __shfl_xor_sync(0xffffffffu, s ? x[0] : x[1], 1);
+  const uint32_t r1 = __shfl_xor_sync(0xffffffffu, s ? x[2] : x[3], 1);
+  // now (k0, k1) are this lane's words for rows s and 2 + s, (r0, r1) the partner's; xor 2 passes on
+  // the row with the other bit 1
+  const uint32_t a = t ? k1 : k0, b = t ? r1 : r0;
+  const uint32_t ra = __shfl_xor_sync(0xffffffffu, t ? k0 : k1, 2);
+  const uint32_t rb = __shfl_xor_sync(0xffffffffu, t ? r0 : r1, 2);
+  // from lanes q, q^1, q^2, q^3 in that order: slot c = (source lane) xor q
+  const uint32_t v0 = s ? b : a, v1 = s ? a : b, v2 = s ? rb : ra, v3 = s ? ra : rb;
+  x[0] = t ? v2 : v0;
+  x[1] = t ? v3 : v1;
+  x[2] = t ? v0 : v2;
+  x[3] = t ? v1 : v3;
+}
+
+// Dropout threshold t (0..255) in the form keep_flags wants: 0x8000 − 128·t in each 16-bit half.
+__host__ __device__ constexpr uint32_t keep_flag_bias(uint32_t t) { return 0x80008000u - (t << 7) - (t << 23); }
+
+// Keep flags of the four random bytes of w (byte ≥ t): bit 15 of *even = byte 0, bit 31 = byte 2;
+// bit 15 of *odd = byte 1, bit 31 = byte 3.  Each 16-bit half computes 0x8000 + 128·(byte − t), which
+// stays inside the half, so its top bit is the comparison.
+__device__ __forceinline__ void keep_flags(uint32_t w, uint32_t bias, uint32_t& even, uint32_t& odd) {
+  even = (w & 0x00FF00FFu) * 128u + bias;
+  odd = prmt(w, 0u, 0x4341u) * 128u + bias;
+}
+
+// Masks that zero the dropped keys of two packed 16-bit pairs: keys (0, 1) and (2, 3) of w.
+__device__ __forceinline__ void keep_pair_masks(uint32_t w, uint32_t bias, uint32_t& m01, uint32_t& m23) {
+  uint32_t e, o;
+  keep_flags(w, bias, e, o);
+  m01 = prmt(e, o, 0xDD99u);
+  m23 = prmt(e, o, 0xFFBBu);
 }
 
 // ---------------------------------------------------------------- cluster launch control
