@@ -39,6 +39,7 @@ sys.path.insert(0, ROOT)
 # NVIDIA's datasheet dense BF16 tensor figure for one B200 (its doubled figure assumes 2:4 sparsity);
 # reported beside the measured cuBLAS peak, which is the denominator of every `frac_of_peak`.
 NOMINAL_DENSE_BF16_TFLOPS = 2250.0
+FP8_OVER_BF16 = 2.0  # nominal dense e4m3 / bf16 tensor throughput (4.5 / 2.25 PFLOP/s)
 NOMINAL_SOURCE = "NVIDIA B200 datasheet, dense BF16 (2.25 PFLOP/s; 4.5 with 2:4 sparsity)"
 METRIC = "attention TFLOP/s (fwd, fwd+bwd) on 1 B200 and % of dense bf16 tensor peak"
 DEFAULT_WORKLOAD = "causal_n8k_d128"
@@ -543,8 +544,7 @@ def run_gpu_decode(args, world, rank, local, pg):
         "config": {"workload": wname, "B": B, "H": H, "Nk": Nk, "d": d, "varlen": cu is not None, "keys": Tk,
                    "step": "decode", "flops_per_step": flops,
                    "l2": "flushed before every step (256 MiB write, outside the events)",
-                   "parallelism": f"replicas x{world} (independent workloads per GPU)",
-                   "dropout_p": drop_p},
+                   "parallelism": f"replicas x{world} (independent workloads per GPU)"},
         "roofline": {"kernel": "fa_decode_split_kernel + fa_decode_merge_kernel", "bound": "hbm",
                      "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None,
@@ -557,6 +557,138 @@ def run_gpu_decode(args, world, rank, local, pg):
     }
     if rank == 0 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline_decode(inp_h, budget_s=args.cpu_budget)
+    return out
+
+
+def real_inputs(inp):
+    """e4m3 inputs as the float64 values they stand for (NumPy, so the oracle widens nothing through
+    float32: e4m3 × an fp32 descale needs up to 28 significand bits)."""
+    import workloads
+    ds = inp.extra["descale"]
+    return workloads.AttnInputs(workloads.real_values(inp.q, ds["q"]), workloads.real_values(inp.k, ds["k"]),
+                                workloads.real_values(inp.v, ds["v"]), None, inp.cu_seqlens, list(inp.seqlens),
+                                inp.B, inp.H, inp.N, inp.d, inp.scale, inp.causal, "f64", inp.name)
+
+
+def run_gpu_fp8(args, world, rank, local, pg):
+    """The forward with e4m3 inputs (per-tensor descales, bf16 output): TFLOP/s by the same FLOP
+    convention, against the e4m3 tensor peak."""
+    import torch
+
+    import workloads
+    import exact_io_aware_90_b200 as fa
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    wname = args.workload
+    spec = workloads.WORKLOADS[wname]
+    inp_h = workloads.make_workload(wname)
+    if rank > 0:  # weak scaling: each rank its own seeded copy
+        inp_h = workloads.random_inputs(inp_h.H, inp_h.d, "e4m3", spec["seed"] + 1000 * rank, B=inp_h.B, N=inp_h.N,
+                                        causal=inp_h.causal, backward=False)
+    B, H, N, d, T = inp_h.B, inp_h.H, inp_h.N, inp_h.d, inp_h.T
+    ds = inp_h.extra["descale"]
+    scale, causal = inp_h.scale, int(inp_h.causal)
+    flops = 4.0 * H * d * sum(float(L) * L for L in inp_h.seqlens) * (0.5 if causal else 1.0)
+    q, k, v = inp_h.q.to(dev), inp_h.k.to(dev), inp_h.v.to(dev)
+    o = torch.empty((T, H, d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((T, H), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def fwd():
+        st = fa.fa_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, N, d, scale,
+                           causal, None, T, ds["q"], ds["k"], ds["v"], sp)
+        if st != fa.FA_OK:
+            raise fa.FAError(st, "fa_fwd_fp8")
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        fwd()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(dev)
+    if pg is not None:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    evs = []
+    for _ in range(args.steps):
+        flush.fill_(1)  # outside the timed events
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fwd()
+        b.record(stream)
+        evs.append((a, b))
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    if pg is not None:
+        pg.barrier()
+    st = fa.fa_check_device_status(sp)
+    if st != fa.FA_OK:
+        raise fa.FAError(st, "timed steps")
+    ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in evs])), pg, dev)
+    value = world * flops / (ms * 1e-3) / 1e12
+    # end to end through the public API: e4m3 inputs from pinned host memory, O and LSE back
+    hq, hk, hv = inp_h.q.pin_memory(), inp_h.k.pin_memory(), inp_h.v.pin_memory()
+    ho = torch.empty((T, H, d), dtype=torch.bfloat16).pin_memory()
+    hl = torch.empty((T, H), dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        fa.attention_forward_fp8(q, k, v, ds["q"], ds["k"], ds["v"], causal=bool(causal), scale=scale, batch=B,
+                                 out=o, lse=lse, stream=sp)
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = max(1, min(args.steps, 5))
+    a.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(a.elapsed_time(b) / n_e2e, pg, dev)
+    peaks = load_peaks()
+    fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
+    out = {
+        "metric": METRIC + " (e4m3 inputs, forward)",
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e4m3",
+        "data": "synthetic: i.i.d. N(0,1) q, k, v from a seeded CPU generator, divided by amax/448 per tensor and "
+                "rounded to e4m3",
+        "config": {"workload": wname, "B": B, "H": H, "N": N, "d": d, "causal": bool(causal), "tokens": T,
+                   "step": "fwd", "flops_per_step": flops, "output": "bf16",
+                   "l2": "flushed before every step (256 MiB write, outside the events)",
+                   "parallelism": f"replicas x{world} (independent workloads per GPU)"},
+        "roofline": {"kernel": "fa_fwd_kernel (e4m3)", "bound": "tensor", "achieved": round(value / world, 1),
+                     "peak": round(fp8_peak, 1), "unit": "TFLOP/s", "frac": round(value / world / fp8_peak, 4),
+                     "frac_of_bf16_peak": round(value / world / peaks["bf16_tflops"], 4),
+                     "peak_source": peaks["source"] + f" (burst bf16) x {FP8_OVER_BF16:g}, the nominal e4m3/bf16 "
+                                                      "dense ratio (4.5 / 2.25 PFLOP/s)",
+                     "traffic": load_traffic("fa_fwd_kernel", wname), "launch_ms": round(ms, 4)},
+        "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": 3 * T * H * d,
+                "d2h_bytes_per_step": T * H * d * 2 + T * H * 4},
+        "gpu_launches": args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(real_inputs(inp_h), budget_s=args.cpu_budget)
+        out["cpu_baseline"]["sample"] += " (the real values of the e4m3 inputs)"
     return out
 
 
@@ -690,6 +822,10 @@ def run_reference(args, rank):
         return run_reference_decode(args)
     spec = workloads.WORKLOADS[args.workload]
     inp = workloads.make_workload(args.workload, backward=spec["backward"])
+    metric = METRIC
+    if inp.dtype == "e4m3":
+        inp = real_inputs(inp)
+        metric = METRIC + " (e4m3 inputs, forward)"
     if args.dropout > 0.0:
         return run_reference_dropout(args, inp)
     L = inp.seqlens[0]
@@ -712,7 +848,7 @@ def run_reference(args, rank):
     sample = (f"fp64 NumPy oracle {'fwd+bwd' if inp.do is not None else 'fwd'} of query rows [{L - rows}, {L}) of "
               f"one head of sequence 0 per step")
     return {
-        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "impl": "reference", "metric": metric, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": args.workload, "B": inp.B, "H": inp.H, "N": inp.N, "d": inp.d,
@@ -774,6 +910,8 @@ def main():
         import workloads
         if args.workload in workloads.DECODE_WORKLOADS:
             out = run_gpu_decode(args, world, rank, local, pg)
+        elif workloads.WORKLOADS[args.workload]["dtype"] == "e4m3":
+            out = run_gpu_fp8(args, world, rank, local, pg)
         else:
             out = run_gpu(args, world, rank, local, pg)
         if rank == 0:

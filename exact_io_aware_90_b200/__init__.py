@@ -9,12 +9,13 @@ GPU is present the calls raise.
 
 Raw ABI (same names and argument order as ``include/fa.h``; pointers are ints):
     fa_fwd, fa_bwd, fa_bwd_preprocess, fa_bwd_main, fa_bwd_postprocess,
-    fa_bwd_workspace_bytes, fa_bwd_noalloc, fa_fwd_dropout, fa_bwd_dropout, fa_decode, fa_decode_workspace_bytes,
-    fa_check_device_status, fa_set_watchdog_ns, fa_watchdog_selftest, fa_status_string, fa_version
+    fa_bwd_workspace_bytes, fa_bwd_noalloc, fa_fwd_dropout, fa_bwd_dropout, fa_fwd_fp8, fa_decode,
+    fa_decode_workspace_bytes, fa_check_device_status, fa_set_watchdog_ns, fa_watchdog_selftest, fa_status_string, fa_version
 Torch wrappers:
     attention_forward(q, k, v, ...)          -> (o, lse)
     attention_backward(q, k, v, o, lse, do, ...) -> (dq, dk, dv)
     attention_decode(q, k, v, ...)           -> (o, lse)   one query per sequence over a K/V cache
+    attention_forward_fp8(q8, k8, v8, descales, ...) -> (o bf16, lse)   e4m3 inputs
 """
 
 from __future__ import annotations
@@ -28,8 +29,8 @@ __all__ = [
     "FAError", "LIB_PATH", "lib", "FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA",
     "FA_ERR_TIMEOUT", "FA_BF16", "FA_FP16",
     "fa_fwd", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_postprocess", "fa_bwd_workspace_bytes",
-    "fa_bwd_noalloc", "FA_NOALLOC_SCRATCH_BYTES", "fa_fwd_dropout", "fa_bwd_dropout", "fa_decode", "fa_decode_workspace_bytes", "fa_check_device_status", "fa_set_watchdog_ns", "fa_watchdog_selftest", "fa_status_string", "fa_version",
-    "attention_forward", "attention_backward", "attention_decode", "dtype_code",
+    "fa_bwd_noalloc", "FA_NOALLOC_SCRATCH_BYTES", "fa_fwd_dropout", "fa_bwd_dropout", "fa_fwd_fp8", "fa_decode", "fa_decode_workspace_bytes", "fa_check_device_status", "fa_set_watchdog_ns", "fa_watchdog_selftest", "fa_status_string", "fa_version",
+    "attention_forward", "attention_backward", "attention_decode", "attention_forward_fp8", "dtype_code",
 ]
 
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = 0, 1, 2, 3, 4
@@ -63,6 +64,7 @@ def _load() -> ctypes.CDLL:
         "fa_fwd_dropout": (I, [P, P, P, P, P, I, I, I, I, F, I, P, I, I, F, U64, ctypes.c_uint32, P]),
         "fa_bwd_dropout": (I, [P, P, P, P, P, P, P, P, P, I, I, I, I, F, I, P, I, I, F, U64, ctypes.c_uint32, P, S,
                                P]),
+        "fa_fwd_fp8": (I, [P, P, P, P, P, I, I, I, I, F, I, P, I, F, F, F, P]),
         "fa_decode_workspace_bytes": (S, [I, I, I, I]),
         "fa_decode": (I, [P, P, P, P, P, I, I, I, I, F, P, I, I, P, S, P]),
         "fa_check_device_status": (I, [P]),
@@ -133,6 +135,12 @@ def fa_bwd_dropout(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, c
                    dropout_p, seed, offset, workspace, workspace_bytes, stream) -> int:
     return lib.fa_bwd_dropout(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, cu_seqlens, total_tokens,
                               dtype, dropout_p, seed, offset, workspace, workspace_bytes, stream)
+
+
+def fa_fwd_fp8(q, k, v, o, lse, B, H, N, d, scale, causal, cu_seqlens, total_tokens, q_descale, k_descale,
+               v_descale, stream) -> int:
+    return lib.fa_fwd_fp8(q, k, v, o, lse, B, H, N, d, scale, causal, cu_seqlens, total_tokens, q_descale, k_descale,
+                          v_descale, stream)
 
 
 def fa_decode_workspace_bytes(B, H, Nk, d) -> int:
@@ -262,6 +270,31 @@ def attention_backward(q, k, v, o, lse, do, causal: bool = False, scale: Optiona
     if st != FA_OK:
         raise FAError(st, "fa_bwd")
     return dq, dk, dv
+
+
+def attention_forward_fp8(q, k, v, q_descale: float, k_descale: float, v_descale: float, causal: bool = False,
+                          scale: Optional[float] = None, cu_seqlens=None, max_seqlen: Optional[int] = None,
+                          batch: Optional[int] = None, out=None, lse=None, stream=None):
+    """O (bf16) and LSE for e4m3 q, k, v of shape [T, H, 128] whose real values are the stored ones times
+    the descales (see ``include/fa.h``, fa_fwd_fp8)."""
+    import torch
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.float8_e4m3fn or t.shape != q.shape:
+            raise ValueError(f"{n} must be a contiguous CUDA float8_e4m3fn tensor shaped like q")
+    B, H, N, d, T = _shape(q, cu_seqlens, max_seqlen, batch)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((T, H, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((T, H), dtype=torch.float32, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    st = lib.fa_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, d, float(scale), int(bool(causal)),
+                        _ptr(cu_seqlens), T, float(q_descale), float(k_descale), float(v_descale), stream)
+    if st != FA_OK:
+        raise FAError(st, "fa_fwd_fp8")
+    return out, lse
 
 
 def attention_decode(q, k, v, scale: Optional[float] = None, cu_seqlens_k=None, max_seqlen_k: Optional[int] = None,

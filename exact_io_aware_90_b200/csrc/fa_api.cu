@@ -43,6 +43,20 @@ bool encode_tmap(CUtensorMap* map, const void* base, int T, int H, int d, bool b
   return r == CUDA_SUCCESS;
 }
 
+// e4m3 [T, H, d] as bytes: one 128-byte box per row (d = 128), 128-byte swizzle.
+bool encode_tmap_e4m3(CUtensorMap* map, const void* base, int T, int H, int d, int rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T};
+  const cuuint64_t strides[2] = {(cuuint64_t)d, (cuuint64_t)H * d};
+  const cuuint32_t box[3] = {128, 1, (cuuint32_t)rows};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool encode_tmap_f32(CUtensorMap* map, const void* base, int T, int H, int d, int rows) {
   EncodeTiledFn fn = get_encode_fn();
   if (fn == nullptr) return false;
@@ -87,6 +101,9 @@ static int make_problem(Problem* pb, int B, int H, int N, int d, float scale, in
   pb->bf16 = (dtype == FA_BF16);
   pb->timeout_ns = g_watchdog_ns;
   pb->drop = Dropout{0u, 1.f, 0u, 0u, 0u};
+  pb->fp8 = false;
+  pb->qk_descale = 1.f;
+  pb->v_descale = 1.f;
   return FA_OK;
 }
 
@@ -177,6 +194,30 @@ extern "C" {
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
            float scale, int causal, const int32_t* cu_seqlens, int total_tokens, int dtype, fa_stream_t stream) {
   return fwd_impl(q, k, v, o, lse, B, H, N, d, scale, causal, cu_seqlens, total_tokens, dtype, false, 0.f, 0, 0, stream);
+}
+
+int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+               float scale, int causal, const int32_t* cu_seqlens, int total_tokens, float q_descale,
+               float k_descale, float v_descale, fa_stream_t stream) {
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(lse)) return FA_ERR_INVALID_ARG;
+  Problem pb;
+  // sizes and scale are checked as for a bf16 call (the output is bf16)
+  int st = make_problem(&pb, B, H, N, d, scale, causal, cu_seqlens, total_tokens, FA_BF16, true);
+  if (st != FA_OK) return st;
+  for (float ds : {q_descale, k_descale, v_descale})
+    if (!std::isfinite(ds) || !(ds > 0.f)) return FA_ERR_INVALID_ARG;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  pb.fp8 = true;
+  pb.qk_descale = q_descale * k_descale;
+  pb.v_descale = v_descale;
+  if (!std::isfinite(pb.scale * pb.qk_descale) || !(pb.scale * pb.qk_descale > 0.f)) return FA_ERR_INVALID_ARG;
+  FwdArgs a;
+  if (!encode_tmap_e4m3(&a.tm_q, q, pb.T, H, d, 128) || !encode_tmap_e4m3(&a.tm_k, k, pb.T, H, d, 128) ||
+      !encode_tmap_e4m3(&a.tm_v, v, pb.T, H, d, 128))
+    return FA_ERR_UNSUPPORTED;
+  a.o = o;
+  a.lse = lse;
+  return map_launch(launch_fwd(pb, a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int fa_fwd_dropout(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,

@@ -37,6 +37,12 @@
 // expressed against the same, slightly stale reference, which leaves
 // O = Σ P V / Σ P unchanged (the rescaling argument of §5.2 run in reverse),
 // keeps every P ≤ 256, and makes the O rescale in tensor memory rare.
+//
+// e4m3 inputs (the FP8 instantiation, d = 128): Q, K, V tiles are 128-byte rows of 8-bit values
+// (16 KB per tile, deeper K/V rings), S and P·V run as kind::f8f6f4 MMAs of K = 32, the per-tensor
+// descales of q and k are folded into c and v's multiplies O in the epilogue, P is rounded to e4m3
+// (≤ 256 < 448, so no saturation) and packed four keys per tensor-memory column, and O is written
+// as bf16.
 #include "fa_internal.h"
 #include "sm100.cuh"
 
@@ -50,7 +56,8 @@ struct FwdParams {
   int causal;
   int num_qblocks;   // ceil(N / 256)
   int heads_group;   // heads per L2 group in the unit order
-  float scale_log2;  // scale · log2(e)
+  float scale_log2;  // scale · log2(e) (· the q and k descales for e4m3 inputs)
+  float o_scale;     // factor on O at the end: 1, or the v descale for e4m3 inputs
   uint64_t timeout_ns;
   Dropout drop;
 };
@@ -66,12 +73,14 @@ constexpr float kRescaleThreshold = 8.0f;
 template <int D> struct PolyMask { static constexpr uint32_t value = 0x00u; };
 template <> struct PolyMask<64> { static constexpr uint32_t value = 0x22u; };
 
-template <int D>
+// EB = bytes per input element: 2 (f16 / bf16) or 1 (e4m3).
+template <int D, int EB = 2>
 struct FwdCfg {
-  static constexpr int NCH = D / 64;                   // 128-byte feature chunks per row
-  static constexpr uint32_t TILE = kBM * D * 2;        // bytes of a 128-row tile
-  static constexpr int KSTAGES = (D == 128) ? 3 : 5;   // K ring depth
-  static constexpr int VSTAGES = (D == 128) ? 2 : 4;   // V ring depth
+  static constexpr int NCH = D * EB / 128;             // 128-byte feature chunks per row
+  static constexpr int CHUNK_ELEMS = 128 / EB;         // elements of a 128-byte chunk
+  static constexpr uint32_t TILE = kBM * D * EB;       // bytes of a 128-row tile
+  static constexpr int KSTAGES = (TILE == 32768) ? 3 : 5;  // K ring depth
+  static constexpr int VSTAGES = (TILE == 32768) ? 2 : 4;  // V ring depth
   // barrier indices
   static constexpr int B_QFULL = 0;                   // [2] Q tile t loaded
   static constexpr int B_QEMPTY = B_QFULL + 2;        // [2] last S of Q tile t in its unit done
@@ -117,28 +126,32 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const W
   return __all_sync(0xffffffffu, ok);
 }
 
-// S = Q·Kᵀ for one 128 × 128 tile: D/16 MMAs of K = 16 along the head dimension.
-// Q and K are K-major with 128-byte rows; a 16-element step is +32 bytes inside a
-// swizzle atom, a 64-element step the next 16 KB atom column.
-template <int D, uint32_t IDESC>
+// S = Q·Kᵀ for one 128 × 128 tile: one MMA per 32 bytes of the head dimension (K = 16
+// for 16-bit inputs, 32 for e4m3).  Q and K are K-major with 128-byte rows; a 32-byte step
+// stays inside a swizzle atom, the next 128 bytes are the next 16 KB atom column.
+template <int D, int EB, uint32_t IDESC>
 __device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint64_t dq, uint64_t dk) {
   dq = opaque64(dq);
   dk = opaque64(dk);
 #pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
+  for (int kk = 0; kk < D * EB / 32; ++kk) {
     const uint32_t off = ((kk >> 2) * (kBM * 128) + (kk & 3) * 32) >> 4;
-    mma_ss(s_tmem, dq + off, dk + off, IDESC, kk > 0 ? 1u : 0u);
+    if constexpr (EB == 1) mma_ss_f8(s_tmem, dq + off, dk + off, IDESC, kk > 0 ? 1u : 0u);
+    else mma_ss(s_tmem, dq + off, dk + off, IDESC, kk > 0 ? 1u : 0u);
   }
 }
 
-// O (+)= P·V for one tile: 8 MMAs of K = 16 keys; P is read from tensor memory
-// (8 columns of packed 16-bit values per step), V is MN-major (+2 KB per 16 keys).
-template <uint32_t IDESC>
+// O (+)= P·V for one tile: one MMA per 32 bytes of P's row (16 keys of 16 bits, or 32 of
+// e4m3), 8 tensor-memory columns each; V is MN-major, 128 bytes per key (+2 KB per 16 keys).
+template <int EB, uint32_t IDESC>
 __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint64_t dv, uint32_t acc) {
   dv = opaque64(dv);
+  constexpr int KPM = 32 / EB;  // keys per MMA
 #pragma unroll
-  for (int kk = 0; kk < kBN / 16; ++kk)
-    mma_ts(o_tmem, p_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), IDESC, kk > 0 ? 1u : acc);
+  for (int kk = 0; kk < kBN / KPM; ++kk) {
+    if constexpr (EB == 1) mma_ts_f8(o_tmem, p_tmem + kk * 8, dv + ((kk * KPM * 128) >> 4), IDESC, kk > 0 ? 1u : acc);
+    else mma_ts(o_tmem, p_tmem + kk * 8, dv + ((kk * KPM * 128) >> 4), IDESC, kk > 0 ? 1u : acc);
+  }
 }
 
 // A decoded work unit: query rows [q0, q0 + 256) of the sequence whose tokens
@@ -196,13 +209,18 @@ __device__ __forceinline__ bool warp_test(uint32_t bar, uint32_t parity) {
   return __all_sync(0xffffffffu, mbar_test_wait(bar, parity));
 }
 
-template <int D, bool BF16, bool DROP>
+// FP8: e4m3 Q, K, V (per-tensor descales folded into scale_log2 and o_scale), P rounded to e4m3 for
+// the P·V product, O written as bf16; BF16 is then true and names the output type.
+template <int D, bool BF16, bool DROP, bool FP8 = false>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using C = FwdCfg<D>;
-  constexpr uint32_t IDESC_S = idesc_f16(BF16, kBM, kBN, false, false);  // S = Q·Kᵀ, both K-major
-  constexpr uint32_t IDESC_O = idesc_f16(BF16, kBM, D, false, true);     // O += P·V, V MN-major
+  static_assert(!(FP8 && DROP), "dropout is not built for e4m3 inputs");
+  constexpr int EB = FP8 ? 1 : 2;
+  using C = FwdCfg<D, EB>;
+  // format code 0 is f16 for kind::f16 and e4m3 for kind::f8f6f4
+  constexpr uint32_t IDESC_S = idesc_f16(BF16 && !FP8, kBM, kBN, false, false);  // S = Q·Kᵀ, both K-major
+  constexpr uint32_t IDESC_O = idesc_f16(BF16 && !FP8, kBM, D, false, true);     // O += P·V, V MN-major
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -317,7 +335,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (elect_one()) {
           mbar_arrive_expect_tx(bar(C::B_QFULL + t), C::TILE);
           for (int c = 0; c < C::NCH; ++c)
-            tma_load_3d(sQ + t * C::TILE + c * (kBM * 128), &tm_q, bar(C::B_QFULL + t), c * 64, u.h,
+            tma_load_3d(sQ + t * C::TILE + c * (kBM * 128), &tm_q, bar(C::B_QFULL + t), c * C::CHUNK_ELEMS, u.h,
                         u.tok0 + u.q0 + t * kBM, pol_q);
         }
         __syncwarp();
@@ -331,7 +349,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (elect_one()) {
           mbar_arrive_expect_tx(bar(C::B_KFULL + s), C::TILE);
           for (int c = 0; c < C::NCH; ++c)
-            tma_load_3d(sK + s * C::TILE + c * (kBN * 128), &tm_k, bar(C::B_KFULL + s), c * 64, u.h,
+            tma_load_3d(sK + s * C::TILE + c * (kBN * 128), &tm_k, bar(C::B_KFULL + s), c * C::CHUNK_ELEMS, u.h,
                         u.tok0 + j * kBN, pol_kv);
         }
         __syncwarp();
@@ -345,7 +363,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (elect_one()) {
           mbar_arrive_expect_tx(bar(C::B_VFULL + s), C::TILE);
           for (int c = 0; c < C::NCH; ++c)
-            tma_load_3d(sV + s * C::TILE + c * (kBN * 128), &tm_v, bar(C::B_VFULL + s), c * 64, u.h,
+            tma_load_3d(sV + s * C::TILE + c * (kBN * 128), &tm_v, bar(C::B_VFULL + s), c * C::CHUNK_ELEMS, u.h,
                         u.tok0 + j * kBN, pol_kv);
         }
         __syncwarp();
@@ -412,7 +430,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         ++qn[t];
         tc_fence_after();
         if (elect_one()) {
-          issue_qk<D, IDESC_S>(tmem + 128u * t, dq_base + ((t * C::TILE) >> 4),
+          issue_qk<D, EB, IDESC_S>(tmem + 128u * t, dq_base + ((t * C::TILE) >> 4),
                                dk_base + (((kpos % C::KSTAGES) * C::TILE) >> 4));
           tc_commit(bar(C::B_SFULL + t));
           if (u.nkv[t] == 1) tc_commit(bar(C::B_QEMPTY + t));  // Q tile t is read by no later MMA of u
@@ -483,8 +501,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             }
             tc_fence_after();
             if (elect_one()) {
-              issue_pv<IDESC_O>(o_tmem, s_tmem, dv_s, j > 0 ? 1u : 0u);
-              if (U.nkv[t] == 1) issue_pv<IDESC_O>(o_tmem, s_tmem + 64u, dv_s, 1u);  // lo part of a split P
+              issue_pv<EB, IDESC_O>(o_tmem, s_tmem, dv_s, j > 0 ? 1u : 0u);
+              if (U.nkv[t] == 1) issue_pv<EB, IDESC_O>(o_tmem, s_tmem + 64u, dv_s, 1u);  // lo part of a split P
               tc_commit(bar(C::B_PVDONE + t));
             }
             __syncwarp();
@@ -492,7 +510,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               if (!k_wait(kpos1)) { ok = false; break; }
               tc_fence_after();
               if (elect_one()) {
-                issue_qk<D, IDESC_S>(s_tmem, dq_base + ((t * C::TILE) >> 4), dk_s1);
+                issue_qk<D, EB, IDESC_S>(s_tmem, dq_base + ((t * C::TILE) >> 4), dk_s1);
                 tc_commit(bar(C::B_SFULL + t));
                 if (j + 2 == U.nkv[t]) tc_commit(bar(C::B_QEMPTY + t));  // last S of Q tile t in this unit
               }
@@ -622,7 +640,45 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           return (i & 1) ? m23 : m01;
         };
         auto drop_pair = [&](uint32_t v, int i) -> uint32_t { return DROP ? v & pair_mask(i) : v; };
-        if (!split_p && !need_mask && PolyMask<D>::value != 0u) {
+        if constexpr (FP8) {
+          if (!split_p) {
+            // P = 2^(c·s − m) on the MUFU, rounded to e4m3, four keys per 32-bit column, written over S.
+            // (Moving a quarter of the exponentials to the FMA pipe, as at d = 64, measured 18 % slower
+            // here: the softmax warps are latency-bound, not MUFU-bound.)
+            uint32_t pk[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              float2 e[2];
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int pi = 2 * i + h;  // pair index
+                const float2 x = __ffma2_rn(make_float2(sv[2 * pi], sv[2 * pi + 1]), c2, nm2);
+                e[h] = make_float2(ex2(x.x), ex2(x.y));
+                acc[pi & 3] = __fadd2_rn(acc[pi & 3], e[h]);
+              }
+              pk[i] = pack4_e4m3(e[0].x, e[0].y, e[1].x, e[1].y);
+            }
+            tmem_st32(tS, pk);
+          } else {
+            // P = hi + lo, both e4m3: hi in columns [0, 32), lo in [64, 96)
+            uint32_t hi[32], lo[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float2 x0 = __ffma2_rn(make_float2(sv[4 * i], sv[4 * i + 1]), c2, nm2);
+              const float2 x1 = __ffma2_rn(make_float2(sv[4 * i + 2], sv[4 * i + 3]), c2, nm2);
+              const float2 e0 = make_float2(ex2(x0.x), ex2(x0.y));
+              const float2 e1 = make_float2(ex2(x1.x), ex2(x1.y));
+              acc[(2 * i) & 3] = __fadd2_rn(acc[(2 * i) & 3], e0);
+              acc[(2 * i + 1) & 3] = __fadd2_rn(acc[(2 * i + 1) & 3], e1);
+              hi[i] = pack4_e4m3(e0.x, e0.y, e1.x, e1.y);
+              const float2 h0 = unpack2_e4m3((uint16_t)(hi[i] & 0xFFFFu));
+              const float2 h1 = unpack2_e4m3((uint16_t)(hi[i] >> 16));
+              lo[i] = pack4_e4m3(e0.x - h0.x, e0.y - h0.y, e1.x - h1.x, e1.y - h1.y);
+            }
+            tmem_st32(tS, hi);
+            tmem_st32(tS + 64u, lo);
+          }
+        } else if (!split_p && !need_mask && PolyMask<D>::value != 0u) {
           // unmasked tile: part of the exponentials on the FMA pipe, interleaved with the MUFU ones
           uint32_t pk[64];
 #pragma unroll
@@ -693,7 +749,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       if (ok && warp_wait(bar(C::B_PVDONE + t), (sn + my_nkv - 1) & 1, wd)) {
         tc_fence_after();
         const bool valid = row < U.L;
-        const float inv = (ell > 0.f) ? (DROP ? p.drop.keep_scale : 1.f) / ell : 0.f;
+        const float inv = (ell > 0.f) ? p.o_scale / ell : 0.f;  // o_scale: 1/(1 − p) with dropout, v's descale for e4m3
         const size_t obase = ((size_t)(U.tok0 + (valid ? row : 0)) * p.H + U.h) * D;
         uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) + obase * 2;
 #pragma unroll
@@ -733,11 +789,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   }
 }
 
-template <int D, bool BF16, bool DROP>
+template <int D, bool BF16, bool DROP, bool FP8 = false>
 static cudaError_t launch_fwd_t(const Problem& pb, const FwdArgs& a, cudaStream_t stream) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, FP8 ? 1 : 2>;
   static bool configured = false;  // per instantiation
-  auto kern = fa_fwd_kernel<D, BF16, DROP>;
+  auto kern = fa_fwd_kernel<D, BF16, DROP, FP8>;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
@@ -754,7 +810,8 @@ static cudaError_t launch_fwd_t(const Problem& pb, const FwdArgs& a, cudaStream_
   p.causal = pb.causal;
   p.num_qblocks = (pb.N + 2 * kBM - 1) / (2 * kBM);
   p.heads_group = 8;
-  p.scale_log2 = pb.scale * 1.4426950408889634f;
+  p.scale_log2 = pb.scale * (pb.fp8 ? pb.qk_descale : 1.f) * 1.4426950408889634f;
+  p.o_scale = pb.drop.t != 0u ? pb.drop.keep_scale : (pb.fp8 ? pb.v_descale : 1.f);
   p.timeout_ns = pb.timeout_ns;
   p.drop = pb.drop;
   const long long units = (long long)pb.B * pb.H * p.num_qblocks;
@@ -770,6 +827,7 @@ static cudaError_t launch_fwd_d(const Problem& pb, const FwdArgs& a, cudaStream_
 }
 
 cudaError_t launch_fwd(const Problem& pb, const FwdArgs& a, cudaStream_t stream) {
+  if (pb.fp8) return launch_fwd_t<128, true, false, true>(pb, a, stream);  // e4m3 inputs: d = 128 only
   return pb.drop.t != 0u ? launch_fwd_d<true>(pb, a, stream) : launch_fwd_d<false>(pb, a, stream);
 }
 

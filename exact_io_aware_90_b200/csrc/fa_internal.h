@@ -28,6 +28,10 @@ struct Problem {
   bool bf16;
   uint64_t timeout_ns;
   Dropout drop;  // drop.t == 0: no dropout
+  // e4m3 inputs (forward only; output bf16): real value = stored value × descale
+  bool fp8;
+  float qk_descale;  // q descale × k descale
+  float v_descale;
 };
 
 struct FwdArgs {
@@ -57,6 +61,7 @@ bool encode_tmap(CUtensorMap* map, const void* base, int T, int H, int d, bool b
 
 // Encodes a [T, H, d] fp32 tensor as a 3-D TMA map with 128-byte swizzle and a
 // box of 32 features × 1 head × `rows` tokens.  Returns false on failure.
+bool encode_tmap_e4m3(CUtensorMap* map, const void* base, int T, int H, int d, int rows);
 bool encode_tmap_f32(CUtensorMap* map, const void* base, int T, int H, int d, int rows);
 
 // Decode (one query per sequence, split-KV): keys per chunk, and its workspace.

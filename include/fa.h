@@ -208,6 +208,29 @@ int fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o, c
                    void* workspace, size_t workspace_bytes, fa_stream_t stream);
 
 /*
+ * Forward with 8-bit floating-point inputs (the FP8 path the pages credit to
+ * FlashAttention-3, "Flash Attention 优化", 工程实践 "精度"): q, k, v are
+ * e4m3 (OCP FP8 E4M3: 1 sign, 4 exponent, 3 mantissa bits, bias 7, no
+ * infinities, ±448 largest), one byte per element, in the [T, H, d] layout
+ * of fa_fwd; the real value of an element is its e4m3 value × the tensor's
+ * descale.  Computes what fa_fwd computes for the real values: the descales
+ * of q and k are folded into the softmax scale, v's multiplies O at the end.
+ * The probabilities P are rounded to e4m3 before the P·V product (rows whose
+ * keys fit in one 128-key tile carry P as the sum of two e4m3 parts), the
+ * scores, the softmax statistics and O accumulate in fp32.
+ *   o     bf16 [T, H, d] (written); lse  fp32 [T, H] as for fa_fwd.
+ *   q_descale, k_descale, v_descale  finite and > 0.
+ * d must be 128 (FA_ERR_UNSUPPORTED otherwise).  Other errors as fa_fwd; a
+ * descale that is not finite and positive, or a scale·q_descale·k_descale
+ * that is not, returns FA_ERR_INVALID_ARG.  No backward: the e4m3 path is
+ * for inference.
+ */
+int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
+               int B, int H, int N, int d, float scale, int causal,
+               const int32_t* cu_seqlens, int total_tokens,
+               float q_descale, float k_descale, float v_descale, fa_stream_t stream);
+
+/*
  * Decode: one new query token per sequence attends to every key of its
  * sequence in a K/V cache (token-by-token generation, the workload
  * "FlashAttention 短片讲解稿", segment "适用范围与关键结论", sets apart from

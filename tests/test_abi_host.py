@@ -33,7 +33,7 @@ def test_header_declares_the_entry_points():
     for n in ["fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_bwd_preprocess", "fa_bwd_main",
               "fa_bwd_postprocess", "fa_check_device_status", "fa_status_string", "fa_set_watchdog_ns",
               "fa_watchdog_selftest", "fa_version", "fa_bwd_noalloc", "fa_decode", "fa_decode_workspace_bytes",
-              "fa_fwd_dropout", "fa_bwd_dropout"]:
+              "fa_fwd_dropout", "fa_bwd_dropout", "fa_fwd_fp8"]:
         assert n in names
 
 
@@ -110,6 +110,26 @@ def test_dropout_rejects_invalid_probability(fa):
     bargs = [P16] * 9 + [2, 4, 256, 64, 0.125, 0, None, 512, 0]
     assert fa.fa_bwd_dropout(*bargs, 1.0, 1, 0, P16, ws, None) == fa.FA_ERR_INVALID_ARG
     assert fa.fa_bwd_dropout(*bargs, 0.1, 1, 0, P16, ws - 1, None) == fa.FA_ERR_INVALID_ARG
+
+
+def test_fp8_rejects_invalid_arguments(fa):
+    args = [P16] * 5 + [2, 4, 256, 128, 0.125, 0, None, 512]
+    for ds in (0.0, -1.0, float("nan"), float("inf")):
+        assert fa.fa_fwd_fp8(*args, ds, 1.0, 1.0, None) == fa.FA_ERR_INVALID_ARG
+        assert fa.fa_fwd_fp8(*args, 1.0, ds, 1.0, None) == fa.FA_ERR_INVALID_ARG
+        assert fa.fa_fwd_fp8(*args, 1.0, 1.0, ds, None) == fa.FA_ERR_INVALID_ARG
+    # the folded softmax scale must stay finite
+    assert fa.fa_fwd_fp8(*args, 1e30, 1e30, 1.0, None) == fa.FA_ERR_INVALID_ARG
+    # e4m3 inputs are built for d = 128 only
+    assert fa.fa_fwd_fp8(*([P16] * 5 + [2, 4, 256, 64, 0.125, 0, None, 512]), 1.0, 1.0, 1.0, None) == \
+        fa.FA_ERR_UNSUPPORTED
+    # misaligned pointer, bad causal flag, token count mismatch
+    assert fa.fa_fwd_fp8(*([P16 + 8] + [P16] * 4 + [2, 4, 256, 128, 0.125, 0, None, 512]), 1.0, 1.0, 1.0, None) == \
+        fa.FA_ERR_INVALID_ARG
+    assert fa.fa_fwd_fp8(*([P16] * 5 + [2, 4, 256, 128, 0.125, 2, None, 512]), 1.0, 1.0, 1.0, None) == \
+        fa.FA_ERR_INVALID_ARG
+    assert fa.fa_fwd_fp8(*([P16] * 5 + [2, 4, 256, 128, 0.125, 0, None, 511]), 1.0, 1.0, 1.0, None) == \
+        fa.FA_ERR_INVALID_ARG
 
 
 def test_decode_workspace_bytes(fa):

@@ -100,27 +100,71 @@ def test_dropout_varlen(fa):
         assert rel_l2(f64(g)[rows], r[rows]) <= GRAD_TOL
 
 
+def _mask_case(causal):
+    """B = 2 sequences × H = 2 heads of N = 256 tokens, d = 128: two query tiles and two key tiles per
+    (sequence, head), and four values of the head index b·H + h in the Philox counter."""
+    B, H, N, d = 2, 2, 256, 128
+    g = torch.Generator().manual_seed(3)
+    q = torch.randn(B * N, H, d, generator=g).to(torch.bfloat16)
+    k = torch.randn(B * N, H, d, generator=g).to(torch.bfloat16)
+    visible = np.tril(np.ones((N, N), dtype=bool)) if causal else np.ones((N, N), dtype=bool)
+    return B, H, N, d, q, k, visible, 1.0 / math.sqrt(d), (0.375, 1234567, 9)
+
+
+def _window_eye(B, H, N, d, w0):
+    """[B·N, H, d] with token w0 + c of every sequence carrying e_c (c < d), all other tokens 0."""
+    x = torch.zeros(B * N, H, d, dtype=torch.bfloat16)
+    for b in range(B):
+        x[b * N + w0 + torch.arange(d), :, torch.arange(d)] = 1.0
+    return x
+
+
 @pytest.mark.parametrize("causal", [False, True])
 def test_dropout_mask_is_exact(fa, causal):
-    """V = identity (key j carries e_j): O row i is the dropped P row, so every kept and every dropped
-    element of the kernel's mask is visible and must equal the oracle's mask exactly."""
-    N, d = 64, 64
-    scale = 1.0 / math.sqrt(d)
-    g = torch.Generator().manual_seed(3)
-    q = torch.randn(N, 1, d, generator=g).to(torch.bfloat16)
-    k = torch.randn(N, 1, d, generator=g).to(torch.bfloat16)
-    v = torch.zeros(N, 1, d, dtype=torch.bfloat16)
-    v[torch.arange(N), 0, torch.arange(N)] = 1.0
+    """V carries e_c on key w0 + c: O[i, c] is the dropped, rescaled P[i, w0 + c], so every kept and
+    every dropped element of the forward kernel's mask over that key window is visible and must
+    equal the oracle's mask exactly (and hidden keys must give exact zeros)."""
+    B, H, N, d, q, k, visible, scale, (p, seed, off) = _mask_case(causal)
     dev = torch.device("cuda")
-    p, seed, off = 0.375, 1234567, 9
-    o, _ = fa.attention_forward(q.to(dev), k.to(dev), v.to(dev), causal=causal, scale=scale, dropout_p=p, seed=seed,
-                                offset=off)
     t = oracle.dropout_threshold(_p32(p))
-    keep = oracle.dropout_keep_mask(N, 0, seed, off, t)
-    visible = np.tril(np.ones((N, N), dtype=bool)) if causal else np.ones((N, N), dtype=bool)
-    got = f64(o)[:, 0, :N]
-    assert np.array_equal(got[visible] != 0.0, keep[visible])
-    assert np.all(got[~visible] == 0.0)
+    for w0 in (0, N - d):
+        v = _window_eye(B, H, N, d, w0)
+        o, _ = fa.attention_forward(q.to(dev), k.to(dev), v.to(dev), causal=causal, scale=scale, batch=B,
+                                    dropout_p=p, seed=seed, offset=off)
+        got = f64(o)
+        for b in range(B):
+            for h in range(H):
+                keep = oracle.dropout_keep_mask(N, b * H + h, seed, off, t)[:, w0:w0 + d]
+                vis = visible[:, w0:w0 + d]
+                gbh = got[b * N:(b + 1) * N, h, :]
+                assert np.array_equal(gbh[vis] != 0.0, keep[vis]), (w0, b, h)
+                assert np.all(gbh[~vis] == 0.0)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_dropout_backward_mask_is_exact(fa, causal):
+    """dO carries e_c on query w0 + c: dV[j, c] = (dropped, rescaled P)[w0 + c, j], so the backward
+    kernel's own regeneration of the mask is visible element by element over that query window."""
+    B, H, N, d, q, k, visible, scale, (p, seed, off) = _mask_case(causal)
+    dev = torch.device("cuda")
+    g = torch.Generator().manual_seed(4)
+    v = torch.randn(B * N, H, d, generator=g).to(torch.bfloat16)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    o, lse = fa.attention_forward(qd, kd, vd, causal=causal, scale=scale, batch=B, dropout_p=p, seed=seed,
+                                  offset=off)
+    t = oracle.dropout_threshold(_p32(p))
+    for w0 in (0, N - d):
+        do = _window_eye(B, H, N, d, w0).to(dev)
+        _, _, dv = fa.attention_backward(qd, kd, vd, o, lse, do, causal=causal, scale=scale, batch=B, dropout_p=p,
+                                         seed=seed, offset=off)
+        got = f64(dv)
+        for b in range(B):
+            for h in range(H):
+                keep = oracle.dropout_keep_mask(N, b * H + h, seed, off, t)[w0:w0 + d, :].T  # [key j, query c]
+                vis = visible[w0:w0 + d, :].T
+                gbh = got[b * N:(b + 1) * N, h, :]
+                assert np.array_equal(gbh[vis] != 0.0, keep[vis]), (w0, b, h)
+                assert np.all(gbh[~vis] == 0.0)
 
 
 def test_dropout_zero_is_plain(fa):

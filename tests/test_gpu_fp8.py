@@ -1,0 +1,163 @@
+"""GPU parity of the e4m3 forward (fa_fwd_fp8) against the fp64 oracle, through the C ABI.
+
+The inputs are e4m3 tensors with per-tensor descales (``workloads.random_inputs(..., "e4m3")``); the
+oracle computes the plain definition on the real values (stored value × descale).  The kernel's only
+rounding beyond fp32 is that of P to e4m3 before P·V (3 mantissa bits: relative error ≤ 2⁻⁴; values
+below the smallest subnormal 2⁻⁹ of the row's reference maximum flush, absolute error ≤ 2⁻¹⁰, and
+the softmax sum ℓ relative to that maximum is ≥ 1) and that of O to bf16.  So, per element,
+
+    |O − O_ref|_ic ≤ 2⁻⁴·Σ_j P_ij |v_jc| + Σ_j min(P_ij, 2⁻¹⁰)·|v_jc| + 2⁻⁸·|O_ref,ic| + 1e-4,
+
+and, the roundings being independent and centred, the RMS error over a tensor is at most about
+σ = 2⁻⁴/√3 · sqrt(mean Σ_j P_ij² v_jc²) (checked with a factor 1.5).  For random values that noise is
+a few percent of |O| per element, so a systematic error (a misapplied scale or descale) is caught by
+the least-squares factor of O on O_ref, which must be 1 within five standard errors σ/(rms O_ref·√n).
+LSE involves no e4m3 rounding: the plain 1e-3 bound.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from _gpu import LSE_TOL, f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fa():
+    from _lib import load_fa
+    m = load_fa()
+    if not torch.cuda.is_available():
+        pytest.fail("a CUDA device is required for the gpu-marked tests")
+    m.fa_set_watchdog_ns(2_000_000_000)
+    return m
+
+
+def _real(inp):
+    ds = inp.extra["descale"]
+    return (workloads.real_values(inp.q, ds["q"]), workloads.real_values(inp.k, ds["k"]),
+            workloads.real_values(inp.v, ds["v"]))
+
+
+def _run(fa, inp, **over):
+    dev = torch.device("cuda")
+    ds = dict(inp.extra["descale"], **over)
+    cu = None if inp.cu_seqlens is None else inp.cu_seqlens.to(dev)
+    o, lse = fa.attention_forward_fp8(inp.q.to(dev), inp.k.to(dev), inp.v.to(dev), ds["q"], ds["k"], ds["v"],
+                                      causal=inp.causal, scale=inp.scale, cu_seqlens=cu,
+                                      max_seqlen=inp.N if cu is not None else None, batch=inp.B)
+    assert fa.fa_check_device_status(torch.cuda.current_stream().cuda_stream) == fa.FA_OK
+    return o, lse
+
+
+def _seq_bounds(inp):
+    """(start, length) of every sequence."""
+    if inp.cu_seqlens is None:
+        return [(b * inp.N, inp.N) for b in range(inp.B)]
+    cu = inp.cu_seqlens.tolist()
+    return [(cu[b], cu[b + 1] - cu[b]) for b in range(len(cu) - 1)]
+
+
+def _rounding_terms(q, k, v, lse_ref, scale, causal, seqs, rows=None):
+    """For the chosen tokens (all heads): A = Σ_j P|v|, Bt = Σ_j min(P, 2⁻¹⁰)|v|, Q2 = Σ_j P²v², with P
+    from the oracle's LSE (P_ij = exp(scale·q_i·k_j − LSE_i) over the visible keys)."""
+    T, H, d = q.shape
+    A, Bt, Q2 = (np.zeros((T, H, d)) for _ in range(3))
+    want = np.ones(T, dtype=bool) if rows is None else np.isin(np.arange(T), rows)
+    for s0, L in seqs:
+        toks = [t for t in range(s0, s0 + L) if want[t]]
+        if not toks:
+            continue
+        ti = np.array(toks)
+        for h in range(H):
+            S = scale * q[ti, h, :] @ k[s0:s0 + L, h, :].T                      # [rows, L]
+            P = np.exp(S - lse_ref[ti, h][:, None])
+            if causal:
+                P = np.where(np.arange(L)[None, :] <= (ti - s0)[:, None], P, 0.0)
+            va = np.abs(v[s0:s0 + L, h, :])
+            A[ti, h] = P @ va
+            Bt[ti, h] = np.minimum(P, 2.0 ** -10) @ va
+            Q2[ti, h] = (P * P) @ (va * va)
+    return A, Bt, Q2
+
+
+def _check(inp, o, lse, rows=None):
+    q, k, v = _real(inp)
+    cu = None if inp.cu_seqlens is None else inp.cu_seqlens.numpy()
+    if rows is None:
+        O_ref, L_ref = oracle.attention_forward(q, k, v, inp.scale, inp.causal, cu_seqlens=cu, B=inp.B,
+                                                N=inp.N if cu is None else None)
+        sel = np.ones(inp.T, dtype=bool)
+    else:
+        O_r, L_r = oracle.attention_forward_rows(q, k, v, rows, inp.scale, inp.causal, cu_seqlens=cu, B=inp.B,
+                                                 N=inp.N if cu is None else None)
+        O_ref, L_ref = np.zeros(q.shape), np.zeros(q.shape[:2])
+        O_ref[rows], L_ref[rows] = O_r, L_r
+        sel = np.isin(np.arange(inp.T), rows)
+    A, Bt, Q2 = _rounding_terms(q, k, v, L_ref, inp.scale, inp.causal, _seq_bounds(inp), rows)
+    got, gl = f64(o)[sel], f64(lse)[sel]
+    err = np.abs(got - O_ref[sel])
+    bound = 2.0 ** -4 * A[sel] + Bt[sel] + 2.0 ** -8 * np.abs(O_ref[sel]) + 1e-4
+    worst = np.unravel_index(np.argmax(err - bound), err.shape) if err.size else None
+    assert np.all(err <= bound), (err[worst], bound[worst])
+    if err.size:
+        ref = O_ref[sel]
+        rms = math.sqrt(float(np.mean(err ** 2)))
+        rms_pred = 2.0 ** -4 / math.sqrt(3.0) * math.sqrt(float(np.mean(Q2[sel])))
+        rms_ref = math.sqrt(float(np.mean(ref ** 2)))
+        rms_out = 2.0 ** -9 * rms_ref
+        assert rms <= 1.5 * rms_pred + rms_out + 1e-5, (rms, rms_pred, rms_out)
+        # no systematic error: the least-squares factor of the output on the reference is 1 within five
+        # standard errors of the rounding noise (a misapplied scale or descale moves it by far more)
+        if rms_ref > 0:
+            alpha = float(np.sum(got * ref) / np.sum(ref * ref))
+            assert abs(alpha - 1.0) <= 5.0 * rms_pred / (rms_ref * math.sqrt(ref.size)) + 2.0 ** -10, alpha
+        assert float(np.max(np.abs(gl - L_ref[sel]))) <= LSE_TOL
+    return err
+
+
+@pytest.mark.parametrize("N", [1, 63, 129, 300, 700])
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp8_forward(fa, N, causal):
+    inp = workloads.random_inputs(2, 128, "e4m3", seed=500 + N + int(causal), B=2, N=N, causal=causal,
+                                  backward=False)
+    o, lse = _run(fa, inp)
+    assert o.dtype == torch.bfloat16
+    _check(inp, o, lse)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp8_varlen(fa, causal):
+    inp = workloads.random_inputs(3, 128, "e4m3", seed=77, seqlens=[5, 0, 257, 130, 1030], causal=causal,
+                                  backward=False)
+    o, lse = _run(fa, inp)
+    _check(inp, o, lse)
+
+
+def test_fp8_descales_fold_exactly(fa):
+    """Powers of two moved between the q and k descales leave every score unchanged, and doubling v's
+    descale doubles O: both exactly, since the kernel only multiplies by them."""
+    inp = workloads.random_inputs(2, 128, "e4m3", seed=9, B=1, N=520, causal=True, backward=False)
+    ds = inp.extra["descale"]
+    o1, l1 = _run(fa, inp)
+    o2, l2 = _run(fa, inp, q=ds["q"] * 4.0, k=ds["k"] / 4.0)
+    o3, l3 = _run(fa, inp, v=ds["v"] * 2.0)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    assert torch.equal(o3.float(), 2.0 * o1.float()) and torch.equal(l1, l3)
+
+
+def test_fp8_full_size_sampled_rows(fa):
+    """The measured workload (B=4, H=16, N=8192, d=128, causal), in the launch configuration the
+    benchmark times, on 48 seeded rows (all heads) against the oracle's row-restricted forward."""
+    inp = workloads.make_workload("causal_n8k_d128_fp8")
+    o, lse = _run(fa, inp)
+    rng = np.random.default_rng(5)
+    rows = np.sort(np.concatenate([rng.choice(inp.T, 40, replace=False), [0, 127, 128, 8191, 8192, 16383, 24576,
+                                                                             inp.T - 1]]))
+    rows = np.unique(rows)
+    _check(inp, o, lse, rows=rows)

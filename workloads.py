@@ -19,7 +19,14 @@ causal_n8k_d128     B=4, H=16, N=8192, d=128, bf16, causal, fwd+bwd
 varlen_causal_d128  32 sequences, lengths uniform in [128, 4096], H=32,
                     d=128, bf16, causal, fwd+bwd
 long_n128k_d128     B=1, H=8, N=131072, d=128, bf16, causal, forward only
+causal_n8k_d128_fp8 B=4, H=16, N=8192, d=128, e4m3 (per-tensor descales),
+                    causal, forward only
 ==================  =========================================================
+
+e4m3 inputs: each tensor is drawn in fp32, divided by its descale
+amax/448 (so its largest magnitude maps to e4m3's largest finite value) and
+rounded to float8_e4m3fn; ``extra["descale"]`` holds the three descales and
+the real value of an element is its e4m3 value times its tensor's descale.
 
 Decode inputs (one query token per sequence over a K/V cache): q is
 [B, H, d], k and v are [Tk, H, d] with ``cu_seqlens_k`` (or Tk = B·Nk):
@@ -47,6 +54,7 @@ WORKLOADS = {
     "varlen_causal_d128": dict(nseq=32, lmin=128, lmax=4096, H=32, d=128, dtype="bf16", causal=True,
                                backward=True, seed=1004),
     "long_n128k_d128": dict(B=1, H=8, N=131072, d=128, dtype="bf16", causal=True, backward=False, seed=1005),
+    "causal_n8k_d128_fp8": dict(B=4, H=16, N=8192, d=128, dtype="e4m3", causal=True, backward=False, seed=1008),
 }
 
 TORCH_DTYPES = {"bf16": torch.bfloat16, "fp16": torch.float16}
@@ -81,8 +89,23 @@ class AttnInputs:
                           self.dtype, self.name, dict(self.extra))
 
 
+E4M3_MAX = 448.0  # largest finite float8_e4m3fn value
+
+
 def _randn(g: torch.Generator, shape, dtype: str) -> torch.Tensor:
     return torch.randn(*shape, generator=g, dtype=torch.float32).to(TORCH_DTYPES[dtype])
+
+
+def _randn_e4m3(g: torch.Generator, shape):
+    """(e4m3 tensor, descale) with real values = e4m3 value × descale, descale = amax / 448."""
+    x = torch.randn(*shape, generator=g, dtype=torch.float32)
+    descale = float(np.float32(float(x.abs().max()) / E4M3_MAX))  # the fp32 value the C ABI receives
+    return (x / descale).to(torch.float8_e4m3fn), descale
+
+
+def real_values(t: torch.Tensor, descale: float = 1.0) -> np.ndarray:
+    """The values a stored tensor stands for, as float64 (e4m3 or 16-bit storage times its descale)."""
+    return t.detach().cpu().to(torch.float64).numpy() * float(descale)
 
 
 def varlen_lengths(nseq: int, lmin: int, lmax: int, seed: int) -> List[int]:
@@ -108,6 +131,16 @@ def random_inputs(H: int, d: int, dtype: str, seed: int, *, B: int = 1, N: int =
     else:
         cu, T, seqlens = None, B * N, [N] * B
     g = torch.Generator().manual_seed(seed)
+    extra = {}
+    if dtype == "e4m3":
+        if backward:
+            raise ValueError("e4m3 inputs are forward only")
+        (q, dq_), (k, dk_), (v, dv_) = (_randn_e4m3(g, (T, H, d)) for _ in range(3))
+        extra["descale"] = {"q": dq_, "k": dk_, "v": dv_}
+        if scale is None:
+            scale = 1.0 / math.sqrt(d)
+        return AttnInputs(q, k, v, None, cu, list(seqlens), B, H, N, d, float(scale), bool(causal), dtype, name,
+                          extra)
     q = _randn(g, (T, H, d), dtype)
     k = _randn(g, (T, H, d), dtype)
     v = _randn(g, (T, H, d), dtype)
