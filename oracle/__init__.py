@@ -17,6 +17,11 @@ Parity status of each function (what pins it; see ``tests/test_oracle.py``):
                           the last row of causal self-attention, brute force.
 * split_kv_decode         pinned: equals decode_forward for every chunk size;
                           chunk = 1 reduces to the page's per-element recurrence.
+* merge_attention_partials
+                          pinned: partials over disjoint key sets (any order, an empty
+                          one included) merge to decode_forward over all keys; identity
+                          and empty parts; no overflow at log-sum-exps near 1000.
+* ring_attention_forward  pinned: equals attention_forward for 1 … 6 ranks, causal and not.
 * philox4x32_10           pinned: the generator's published known-answer vectors.
 * dropout_keep_mask       pinned: scalar re-derivation of the element mapping,
                           keep fraction within binomial bounds.

@@ -64,6 +64,8 @@ __all__ = [
     "attention_flops",
     "decode_forward",
     "split_kv_decode",
+    "merge_attention_partials",
+    "ring_attention_forward",
     "philox4x32_10",
     "dropout_threshold",
     "dropout_keep_mask",
@@ -444,6 +446,64 @@ def split_kv_decode(q, k, v, scale: float, chunk: int, cu_seqlens_k=None, B: Opt
                 LSE[b, h] = m + math.log(ell)
     if return_partials:
         return O, LSE, partials
+    return O, LSE
+
+
+# ----------------------------------------------------------------------------- partial results: merge, ring schedule
+
+
+def merge_attention_partials(parts):
+    """Combine attention results of the same queries over disjoint sets of keys.
+
+    ``parts``: a list of (O_b, LSE_b) with O_b [..., d] normalised over its own keys and LSE_b [...]
+    their natural-log sum of exponentials (−∞ where a part saw no key).  This is the block-merge rule
+    of FlashAttention 与算子融合 ("FlashAttention 的两个关键", online softmax) for partials kept in
+    normalised form: a normalised part is the pair (m, ℓ) = (LSE_b, 1) with Õ_b = O_b, so
+        m = max_b LSE_b,  ℓ = Σ_b e^{LSE_b − m},  LSE = m + ln ℓ,  O = Σ_b e^{LSE_b − LSE} O_b.
+    Parts are merged one at a time, as the ring schedule produces them.  Returns (O, LSE) in float64.
+    """
+    O = np.array(_f64(parts[0][0]), dtype=np.float64)
+    L = np.array(_f64(parts[0][1]), dtype=np.float64)
+    for Ob, Lb in parts[1:]:
+        Ob, Lb = _f64(Ob), _f64(Lb)
+        m = np.maximum(L, Lb)
+        m_safe = np.where(np.isneginf(m), 0.0, m)          # both parts empty: keep LSE = −∞, O = 0
+        ea, eb = np.exp(L - m_safe), np.exp(Lb - m_safe)    # e^{−∞} = 0 drops an empty part
+        ell = ea + eb
+        L_new = np.where(ell > 0, m_safe + np.log(np.where(ell > 0, ell, 1.0)), -np.inf)
+        wa = np.where(ell > 0, ea / np.where(ell > 0, ell, 1.0), 0.0)
+        wb = np.where(ell > 0, eb / np.where(ell > 0, ell, 1.0), 0.0)
+        O = wa[..., None] * O + wb[..., None] * Ob
+        L = L_new
+    return O, L
+
+
+def ring_attention_forward(q, k, v, scale: float, causal: bool, world: int):
+    """Attention of one dense sequence [L, H, d] computed as ring (context-parallel) attention over
+    ``world`` ranks (FlashAttention 与算子融合, 工程实践: the ring of attention for very long
+    sequences, with FlashAttention as the compute core): rank r holds positions [r·S, (r+1)·S),
+    S = L / world, of q, k and v; at step t it holds the key/value shard of rank s = (r − t) mod
+    world, attends its queries to it — the causal diagonal block when s = r, every key when s < r,
+    nothing when s > r under the causal mask — and merges the block's (O, LSE) into its running
+    result with ``merge_attention_partials``.  Returns (O [L, H, d], LSE [L, H]) in float64,
+    equal to ``attention_forward`` of the whole sequence."""
+    Q, K, V = _f64(q), _f64(k), _f64(v)
+    L, H, d = Q.shape
+    if world < 1 or L % world:
+        raise ValueError("the sequence must split into `world` equal shards")
+    S = L // world
+    O = np.zeros((L, H, d))
+    LSE = np.full((L, H), -np.inf)
+    for r in range(world):
+        rows = slice(r * S, (r + 1) * S)
+        parts = []
+        for t in range(world):
+            s_ = (r - t) % world
+            if causal and s_ > r:
+                continue
+            cols = slice(s_ * S, (s_ + 1) * S)
+            parts.append(attention_forward(Q[rows], K[cols], V[cols], scale, causal and s_ == r))
+        O[rows], LSE[rows] = merge_attention_partials(parts)
     return O, LSE
 
 

@@ -685,3 +685,105 @@ def test_dropout_delta_identity():
     P /= P.sum(axis=1, keepdims=True)
     dP = (do[:, 0] @ v[:, 0].T) * oracle.dropout_keep_mask(20, 0, seed, 0, t) * 256.0 / (256.0 - t)
     assert np.abs((P * dP).sum(axis=1) - (do[:, 0] * O[:, 0]).sum(axis=1)).max() < 1e-12
+
+
+# ----------------------------------------------------------------------------- partial results: merge, ring schedule
+
+
+def _empty_part(shape):
+    return np.zeros(shape), np.full(shape[:-1], -np.inf)
+
+
+def _ring_pins_pass(merge, ring):
+    """The pins of merge_attention_partials and ring_attention_forward, run against a given pair of
+    implementations (the oracle's, or planted mistakes)."""
+    try:
+        rng = np.random.default_rng(21)
+        # (1) one query's partials over disjoint key sets (one of them empty) merge to its attention over
+        # all keys, whatever the order of the parts
+        q = rng.standard_normal((1, 2, 4))
+        k = rng.standard_normal((11, 2, 4))
+        v = rng.standard_normal((11, 2, 4))
+        full = oracle.decode_forward(q, k, v, 0.7, B=1, Nk=11)
+        sets = [[0, 3, 4], [], [1, 2, 5, 9], [6, 7, 8, 10]]
+        parts = [oracle.decode_forward(q, k[idx], v[idx], 0.7, B=1, Nk=len(idx)) if idx else _empty_part((1, 2, 4))
+                 for idx in sets]
+        for order in (parts, parts[::-1], [parts[2], parts[0], parts[3], parts[1]]):
+            O, L = merge(order)
+            assert np.allclose(O, full[0], atol=1e-13, rtol=0) and np.allclose(L, full[1], atol=1e-13, rtol=0)
+        # (2) one part comes back unchanged; an empty part changes nothing; two empty parts stay empty
+        for ps in ([full], [full, _empty_part((1, 2, 4))], [_empty_part((1, 2, 4)), full]):
+            O, L = merge(ps)
+            assert np.array_equal(O, full[0]) and np.array_equal(L, full[1])
+        O, L = merge([_empty_part((1, 2, 4)), _empty_part((1, 2, 4))])
+        assert np.all(O == 0.0) and np.all(np.isneginf(L))
+        # (3) log-sum-exps near 1000 (e^1000 overflows float64): shifting every part by 1000 shifts only LSE
+        with np.errstate(over="raise", invalid="raise"):
+            O, L = merge([(Ob, Lb + 1000.0) for Ob, Lb in parts])
+        assert np.allclose(O, full[0], atol=1e-13, rtol=0) and np.allclose(L, full[1] + 1000.0, atol=1e-12, rtol=0)
+        # (4) the ring schedule equals the definition for 1 … 6 ranks, causal and not
+        qq, kk, vv = (rng.standard_normal((12, 2, 4)) for _ in range(3))
+        for causal in (False, True):
+            O_ref, L_ref = oracle.attention_forward(qq, kk, vv, 0.5, causal)
+            for w in (1, 2, 3, 4, 6):
+                O, L = ring(qq, kk, vv, 0.5, causal, w)
+                assert np.allclose(O, O_ref, atol=1e-13, rtol=0) and np.allclose(L, L_ref, atol=1e-13, rtol=0)
+        return True
+    except (AssertionError, FloatingPointError):
+        return False
+
+
+def test_ring_and_merge_pins():
+    assert _ring_pins_pass(oracle.merge_attention_partials, oracle.ring_attention_forward)
+
+
+def test_ring_and_merge_pins_catch_planted_mistakes():
+    merge, ring = oracle.merge_attention_partials, oracle.ring_attention_forward
+
+    def merge_unshifted(ps):  # the weights e^{LSE_b} without the max shift
+        O, L = (np.asarray(ps[0][0], dtype=np.float64), np.asarray(ps[0][1], dtype=np.float64))
+        for Ob, Lb in ps[1:]:
+            s = np.exp(L) + np.exp(Lb)
+            O = (np.exp(L)[..., None] * O + np.exp(Lb)[..., None] * Ob) / s[..., None]
+            L = np.log(s)
+        return O, L
+
+    def merge_swapped(ps):  # each part weighted by the other part's share
+        O, L = ps[0]
+        for Ob, Lb in ps[1:]:
+            Ls = np.logaddexp(L, Lb)
+            O = np.exp(Lb - Ls)[..., None] * O + np.exp(L - Ls)[..., None] * Ob
+            L = Ls
+        return O, L
+
+    def merge_lse_max_only(ps):  # LSE taken as the larger part's, not the log of the sum
+        O, L = merge(ps)
+        return O, np.maximum.reduce([np.asarray(p[1]) for p in ps])
+
+    def ring_variant(skip, diag_causal):
+        def f(q, k, v, scale, causal, world):
+            L_, H, d = q.shape
+            S = L_ // world
+            O, LSE = np.zeros((L_, H, d)), np.full((L_, H), -np.inf)
+            for r in range(world):
+                rows, parts = slice(r * S, (r + 1) * S), []
+                for t in range(world):
+                    s_ = (r - t) % world
+                    if causal and skip(s_, r):
+                        continue
+                    cols = slice(s_ * S, (s_ + 1) * S)
+                    parts.append(oracle.attention_forward(q[rows], k[cols], v[cols], scale,
+                                                          causal and s_ == r and diag_causal))
+                if parts:  # a rank whose every shard is skipped keeps O = 0, LSE = −∞
+                    O[rows], LSE[rows] = merge(parts)
+            return O, LSE
+        return f
+
+    ring_sees_future = ring_variant(lambda s_, r: False, True)     # later shards not skipped
+    ring_skips_diagonal = ring_variant(lambda s_, r: s_ >= r, True)  # own shard skipped
+    ring_diag_unmasked = ring_variant(lambda s_, r: s_ > r, False)  # diagonal block without its mask
+    assert _ring_pins_pass(merge, ring_variant(lambda s_, r: s_ > r, True))  # the faithful restatement passes
+    for m in (merge_unshifted, merge_swapped, merge_lse_max_only):
+        assert not _ring_pins_pass(m, ring), m.__name__
+    for rv in (ring_sees_future, ring_skips_diagonal, ring_diag_unmasked):
+        assert not _ring_pins_pass(merge, rv)
