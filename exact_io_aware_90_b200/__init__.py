@@ -9,13 +9,15 @@ GPU is present the calls raise.
 
 Raw ABI (same names and argument order as ``include/fa.h``; pointers are ints):
     fa_fwd, fa_bwd, fa_bwd_preprocess, fa_bwd_main, fa_bwd_postprocess,
-    fa_bwd_workspace_bytes, fa_bwd_noalloc, fa_fwd_dropout, fa_bwd_dropout, fa_fwd_fp8, fa_decode,
+    fa_bwd_workspace_bytes, fa_bwd_noalloc, fa_fwd_dropout, fa_bwd_dropout, fa_fwd_fp8, fa_attn_merge, fa_decode,
     fa_decode_workspace_bytes, fa_check_device_status, fa_set_watchdog_ns, fa_watchdog_selftest, fa_status_string, fa_version
 Torch wrappers:
     attention_forward(q, k, v, ...)          -> (o, lse)
     attention_backward(q, k, v, o, lse, do, ...) -> (dq, dk, dv)
     attention_decode(q, k, v, ...)           -> (o, lse)   one query per sequence over a K/V cache
     attention_forward_fp8(q8, k8, v8, descales, ...) -> (o bf16, lse)   e4m3 inputs
+    attention_merge(acc_o, acc_lse, part_o, part_lse, ...)   merge a partial (O, LSE) into a running result
+Ring (context-parallel) attention over a process group: ``exact_io_aware_90_b200.ring``.
 """
 
 from __future__ import annotations
@@ -29,8 +31,8 @@ __all__ = [
     "FAError", "LIB_PATH", "lib", "FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA",
     "FA_ERR_TIMEOUT", "FA_BF16", "FA_FP16",
     "fa_fwd", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_postprocess", "fa_bwd_workspace_bytes",
-    "fa_bwd_noalloc", "FA_NOALLOC_SCRATCH_BYTES", "fa_fwd_dropout", "fa_bwd_dropout", "fa_fwd_fp8", "fa_decode", "fa_decode_workspace_bytes", "fa_check_device_status", "fa_set_watchdog_ns", "fa_watchdog_selftest", "fa_status_string", "fa_version",
-    "attention_forward", "attention_backward", "attention_decode", "attention_forward_fp8", "dtype_code",
+    "fa_bwd_noalloc", "FA_NOALLOC_SCRATCH_BYTES", "fa_fwd_dropout", "fa_bwd_dropout", "fa_fwd_fp8", "fa_attn_merge", "fa_decode", "fa_decode_workspace_bytes", "fa_check_device_status", "fa_set_watchdog_ns", "fa_watchdog_selftest", "fa_status_string", "fa_version",
+    "attention_forward", "attention_backward", "attention_decode", "attention_forward_fp8", "attention_merge", "dtype_code",
 ]
 
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = 0, 1, 2, 3, 4
@@ -65,6 +67,7 @@ def _load() -> ctypes.CDLL:
         "fa_bwd_dropout": (I, [P, P, P, P, P, P, P, P, P, I, I, I, I, F, I, P, I, I, F, U64, ctypes.c_uint32, P, S,
                                P]),
         "fa_fwd_fp8": (I, [P, P, P, P, P, I, I, I, I, F, I, P, I, F, F, F, P]),
+        "fa_attn_merge": (I, [P, P, P, P, P, I, I, I, I, I, P]),
         "fa_decode_workspace_bytes": (S, [I, I, I, I]),
         "fa_decode": (I, [P, P, P, P, P, I, I, I, I, F, P, I, I, P, S, P]),
         "fa_check_device_status": (I, [P]),
@@ -141,6 +144,10 @@ def fa_fwd_fp8(q, k, v, o, lse, B, H, N, d, scale, causal, cu_seqlens, total_tok
                v_descale, stream) -> int:
     return lib.fa_fwd_fp8(q, k, v, o, lse, B, H, N, d, scale, causal, cu_seqlens, total_tokens, q_descale, k_descale,
                           v_descale, stream)
+
+
+def fa_attn_merge(acc_o, acc_lse, part_o, part_lse, out, T, H, d, dtype, first, stream) -> int:
+    return lib.fa_attn_merge(acc_o, acc_lse, part_o, part_lse, out, T, H, d, dtype, first, stream)
 
 
 def fa_decode_workspace_bytes(B, H, Nk, d) -> int:
@@ -295,6 +302,28 @@ def attention_forward_fp8(q, k, v, q_descale: float, k_descale: float, v_descale
     if st != FA_OK:
         raise FAError(st, "fa_fwd_fp8")
     return out, lse
+
+
+def attention_merge(acc_o, acc_lse, part_o, part_lse, out=None, first: bool = False, stream=None):
+    """Merge the normalised partial (part_o [T, H, d] bf16/fp16, part_lse [T, H] fp32) into the running
+    result (acc_o fp32 [T, H, d], acc_lse fp32 [T, H]); with ``out`` the merged O goes there in
+    part_o's dtype (see ``include/fa.h``, fa_attn_merge)."""
+    import torch
+    T, H, d = part_o.shape
+    for t, n, dt in ((acc_o, "acc_o", torch.float32), (acc_lse, "acc_lse", torch.float32),
+                     (part_lse, "part_lse", torch.float32)):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != dt:
+            raise ValueError(f"{n} must be a contiguous CUDA {dt} tensor")
+    if acc_o.shape != part_o.shape or acc_lse.shape != (T, H) or part_lse.shape != (T, H):
+        raise ValueError("acc_o must be [T, H, d] and the LSE arrays [T, H], as part_o")
+    if out is not None and (out.shape != part_o.shape or out.dtype != part_o.dtype or not out.is_contiguous()):
+        raise ValueError("out must be a contiguous tensor like part_o")
+    if stream is None:
+        stream = torch.cuda.current_stream(part_o.device).cuda_stream
+    st = lib.fa_attn_merge(_ptr(acc_o), _ptr(acc_lse), _ptr(part_o), _ptr(part_lse), _ptr(out), T, H, d,
+                           dtype_code(part_o), int(bool(first)), stream)
+    if st != FA_OK:
+        raise FAError(st, "fa_attn_merge")
 
 
 def attention_decode(q, k, v, scale: Optional[float] = None, cu_seqlens_k=None, max_seqlen_k: Optional[int] = None,

@@ -17,7 +17,7 @@ ROOT = os.path.dirname(HERE)
 LIB_NAME = "libfa_b200.so"
 LIB_PATH = os.path.join(HERE, LIB_NAME)
 SOURCES = ["libfa_b200.cu"]
-DEPS = ["fa_api.cu", "fa_fwd.cu", "fa_bwd.cu", "fa_decode.cu", "fa_noalloc.cu"]
+DEPS = ["fa_api.cu", "fa_fwd.cu", "fa_bwd.cu", "fa_decode.cu", "fa_merge.cu", "fa_noalloc.cu"]
 HEADERS = ["fa_internal.h", "sm100.cuh", os.path.join("..", "..", "include", "fa.h")]
 
 

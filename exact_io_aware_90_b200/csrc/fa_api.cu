@@ -313,6 +313,17 @@ int fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o, c
                             stream);
 }
 
+int fa_attn_merge(float* acc_o, float* acc_lse, const void* part_o, const float* part_lse, void* out, int T, int H,
+                  int d, int dtype, int first, fa_stream_t stream) {
+  if (!aligned16(acc_o) || !aligned4(acc_lse) || !aligned16(part_o) || !aligned4(part_lse)) return FA_ERR_INVALID_ARG;
+  if (out != nullptr && !aligned16(out)) return FA_ERR_INVALID_ARG;
+  if (T < 1 || H < 1 || (d != 64 && d != 128) || (first != 0 && first != 1)) return FA_ERR_INVALID_ARG;
+  if (dtype != FA_BF16 && dtype != FA_FP16) return FA_ERR_INVALID_ARG;
+  if ((long long)T * H * d > (1LL << 40)) return FA_ERR_UNSUPPORTED;
+  return map_launch(launch_merge(acc_o, acc_lse, part_o, part_lse, out, (long long)T * H, d, dtype == FA_BF16, first,
+                                 reinterpret_cast<cudaStream_t>(stream)));
+}
+
 size_t fa_decode_workspace_bytes(int B, int H, int Nk, int d) {
   if (B < 1 || H < 1 || Nk < 1 || (d != 64 && d != 128)) return 0;
   const size_t slots = (size_t)B * H * decode_chunks(Nk);

@@ -4,4 +4,5 @@
 #include "fa_fwd.cu"
 #include "fa_bwd.cu"
 #include "fa_decode.cu"
+#include "fa_merge.cu"
 #include "fa_noalloc.cu"

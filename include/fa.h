@@ -231,6 +231,32 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
                float q_descale, float k_descale, float v_descale, fa_stream_t stream);
 
 /*
+ * Merge of normalised partial attention results: the same queries attended
+ * to disjoint key sets (the blocks a ring of ranks visits in ring /
+ * context-parallel attention, "FlashAttention 与算子融合", 工程实践 "与 CP
+ * 配合"), combined one part at a time by the block-merge rule of the same
+ * page ("FlashAttention 的两个关键", online softmax) written for normalised
+ * parts:  LSE' = ln(e^LSE_acc + e^LSE_b),
+ *         O'   = e^(LSE_acc − LSE')·O_acc + e^(LSE_b − LSE')·O_b.
+ * A part with LSE = −∞ (no key) changes nothing.
+ *   acc_o     fp32 [T, H, d], the running O (read unless first; written
+ *             unless out is given).
+ *   acc_lse   fp32 [T, H], the running LSE (read unless first; always
+ *             written with the merged LSE).
+ *   part_o    dtype [T, H, d] and part_lse fp32 [T, H]: the part, as fa_fwd
+ *             writes them.
+ *   out       NULL, or dtype [T, H, d]: the merged O is written here (rounded
+ *             to nearest even) instead of into acc_o — for the last part.
+ *   first     1: the running result is just this part (acc_o, acc_lse are
+ *             not read).
+ * acc_o, part_o, out 16-byte aligned, the LSE arrays 4-byte aligned; d ∈
+ * {64, 128}; errors as fa_fwd (FA_ERR_INVALID_ARG for bad arguments,
+ * FA_ERR_CUDA for a failed launch).  Asynchronous on `stream`.
+ */
+int fa_attn_merge(float* acc_o, float* acc_lse, const void* part_o, const float* part_lse, void* out,
+                  int T, int H, int d, int dtype, int first, fa_stream_t stream);
+
+/*
  * Decode: one new query token per sequence attends to every key of its
  * sequence in a K/V cache (token-by-token generation, the workload
  * "FlashAttention 短片讲解稿", segment "适用范围与关键结论", sets apart from

@@ -33,7 +33,7 @@ def test_header_declares_the_entry_points():
     for n in ["fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_bwd_preprocess", "fa_bwd_main",
               "fa_bwd_postprocess", "fa_check_device_status", "fa_status_string", "fa_set_watchdog_ns",
               "fa_watchdog_selftest", "fa_version", "fa_bwd_noalloc", "fa_decode", "fa_decode_workspace_bytes",
-              "fa_fwd_dropout", "fa_bwd_dropout", "fa_fwd_fp8"]:
+              "fa_fwd_dropout", "fa_bwd_dropout", "fa_fwd_fp8", "fa_attn_merge"]:
         assert n in names
 
 
@@ -130,6 +130,18 @@ def test_fp8_rejects_invalid_arguments(fa):
         fa.FA_ERR_INVALID_ARG
     assert fa.fa_fwd_fp8(*([P16] * 5 + [2, 4, 256, 128, 0.125, 0, None, 511]), 1.0, 1.0, 1.0, None) == \
         fa.FA_ERR_INVALID_ARG
+
+
+def test_merge_rejects_invalid_arguments(fa):
+    ok = [P16, P16, P16, P16, None, 64, 4, 128, 0, 0, None]
+    for i, bad in [(0, P16 + 4), (2, P16 + 8), (1, P16 + 2), (3, 0), (4, P16 + 8)]:
+        args = list(ok)
+        args[i] = bad
+        assert fa.fa_attn_merge(*args) == fa.FA_ERR_INVALID_ARG, i
+    for i, bad in [(5, 0), (6, 0), (7, 96), (8, 7), (9, 2)]:
+        args = list(ok)
+        args[i] = bad
+        assert fa.fa_attn_merge(*args) == fa.FA_ERR_INVALID_ARG, i
 
 
 def test_decode_workspace_bytes(fa):

@@ -1,0 +1,105 @@
+"""Host-side checks of ring (context-parallel) attention (no GPU).
+
+* The schedule: which shard each rank holds at each step and which blocks it computes.
+* The transport and the per-step bookkeeping over real process groups (gloo, world sizes 2 and 4):
+  each rank runs ``ring_attention_forward`` with the block and merge steps done by the fp64 oracle on
+  CPU tensors (injected through the driver's ``block_fn`` / ``merge_fn`` arguments, which default to
+  the CUDA kernels), and its shard of the result must equal the oracle's attention over the whole
+  sequence; the caller's K/V shards must come back untouched.
+"""
+
+import datetime
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("causal", [False, True])
+def test_ring_schedule(world, causal):
+    from exact_io_aware_90_b200.ring import ring_block
+    for r in range(world):
+        held = [ring_block(r, t, world, causal)[0] for t in range(world)]
+        # every shard passes through every rank exactly once, its own first, then r−1, r−2, …
+        assert held == [(r - t) % world for t in range(world)]
+        computed = {src for t in range(world) for src, kind in [ring_block(r, t, world, causal)] if kind}
+        assert computed == (set(range(r + 1)) if causal else set(range(world)))
+        kinds = {ring_block(r, t, world, causal)[0]: ring_block(r, t, world, causal)[1] for t in range(world)}
+        assert kinds[r] == ("causal" if causal else "full")
+        assert all(kinds[s] == "full" for s in range(r))
+
+
+def _oracle_block(q, k, v, causal, scale, out, lse):
+    import oracle
+    O, L = oracle.attention_forward(q.double().numpy(), k.double().numpy(), v.double().numpy(), scale, causal)
+    out.copy_(torch.from_numpy(O).to(out.dtype))
+    lse.copy_(torch.from_numpy(L).to(lse.dtype))
+
+
+def _oracle_merge(acc_o, acc_lse, part_o, part_lse, out, first):
+    import oracle
+    if first:
+        O, L = part_o.double().numpy(), part_lse.double().numpy()
+    else:
+        O, L = oracle.merge_attention_partials([(acc_o.double().numpy(), acc_lse.double().numpy()),
+                                                (part_o.double().numpy(), part_lse.double().numpy())])
+    acc_lse.copy_(torch.from_numpy(L).to(acc_lse.dtype))
+    (out if out is not None else acc_o).copy_(torch.from_numpy(O).to((out if out is not None else acc_o).dtype))
+
+
+def _rank_main(rank, world, port, causal, out_q):
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        import oracle
+        from exact_io_aware_90_b200.ring import ring_attention_forward
+        L, H, d = 24, 2, 8
+        g = np.random.default_rng(7)
+        q, k, v = (g.standard_normal((L, H, d)) for _ in range(3))
+        S = L // world
+        sl = slice(rank * S, (rank + 1) * S)
+        qs, ks, vs = (torch.from_numpy(x[sl].copy()).to(torch.float64) for x in (q, k, v))
+        k0, v0 = ks.clone(), vs.clone()
+        o, lse = ring_attention_forward(qs, ks, vs, causal=causal, scale=0.35, block_fn=_oracle_block,
+                                        merge_fn=_oracle_merge)
+        O_ref, L_ref = oracle.attention_forward(q, k, v, 0.35, causal)
+        err = max(float(np.abs(o.numpy() - O_ref[sl]).max()), float(np.abs(lse.numpy() - L_ref[sl]).max()))
+        untouched = bool(torch.equal(ks, k0) and torch.equal(vs, v0))
+        dist.barrier()
+        out_q.put((rank, err, untouched))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+@pytest.mark.parametrize("causal", [False, True])
+def test_ring_attention_gloo(world, causal):
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, causal, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = [q.get(timeout=180) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, err, untouched in got:
+        assert err < 1e-5, (rank, err)  # the running O and LSE are fp32 buffers, as on the GPU
+        assert untouched, rank
