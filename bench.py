@@ -56,10 +56,18 @@ def load_peaks():
     return dict(FALLBACK_PEAKS)
 
 
-def kernel_source_hash():
+# The source files each profiled kernel is built from: its own file and the two shared headers.
+KERNEL_SOURCES = {
+    "fa_fwd_kernel": ["fa_fwd.cu", "sm100.cuh", "fa_internal.h"],
+    "fa_bwd_main_kernel": ["fa_bwd.cu", "sm100.cuh", "fa_internal.h"],
+}
+
+
+def kernel_source_hash(kernel):
+    """Hash of the sources `kernel` is built from (every file under csrc/ for a kernel not listed)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "exact_io_aware_90_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(KERNEL_SOURCES.get(kernel, os.listdir(csrc))):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -74,7 +82,7 @@ def load_traffic(kernel, workload, dropout_p=0.0):
     with open(p) as f:
         d = json.load(f)
     e = d.get(kernel, {}).get(workload if dropout_p <= 0.0 else f"{workload}+dropout{dropout_p:g}")
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(kernel):
         return None
     return e.get("bytes_per_launch")
 
