@@ -22,6 +22,7 @@ Parity status of each function (what pins it; see ``tests/test_oracle.py``):
                           one included) merge to decode_forward over all keys; identity
                           and empty parts; no overflow at log-sum-exps near 1000.
 * ring_attention_forward  pinned: equals attention_forward for 1 … 6 ranks, causal and not.
+* ring_attention_backward pinned: equals attention_backward for 1 … 6 ranks, causal and not.
 * philox4x32_10           pinned: the generator's published known-answer vectors.
 * dropout_keep_mask       pinned: scalar re-derivation of the element mapping,
                           keep fraction within binomial bounds.

@@ -66,6 +66,7 @@ __all__ = [
     "split_kv_decode",
     "merge_attention_partials",
     "ring_attention_forward",
+    "ring_attention_backward",
     "philox4x32_10",
     "dropout_threshold",
     "dropout_keep_mask",
@@ -505,6 +506,41 @@ def ring_attention_forward(q, k, v, scale: float, causal: bool, world: int):
             parts.append(attention_forward(Q[rows], K[cols], V[cols], scale, causal and s_ == r))
         O[rows], LSE[rows] = merge_attention_partials(parts)
     return O, LSE
+
+
+def ring_attention_backward(q, k, v, do, scale: float, causal: bool, world: int):
+    """Gradients of ``ring_attention_forward`` computed on the same ring.  The probabilities of a block
+    (query shard r, key shard s) are recomputed from the global row statistic, P_rs = exp(scale·Q_r K_sᵀ
+    − LSE_r), as the tiled backward recomputes them from the saved LSE (FlashAttention 短片讲解稿,
+    "第三招 · 反向重计算"), with D_r = Σ_c dO_rc·O_rc of the global output; then, per block,
+        dS = P_rs ∘ (dO_r V_sᵀ − D_r),  dQ_r += scale·dS K_s,  dK_s += scale·dSᵀ Q_r,  dV_s += P_rsᵀ dO_r,
+    where dQ_r accumulates on rank r and dK_s, dV_s travel with the key/value shard s around the ring
+    and are home after one more step.  Returns (dQ, dK, dV) [L, H, d] in float64, equal to
+    ``attention_backward`` of the whole sequence."""
+    Q, K, V, dO = _f64(q), _f64(k), _f64(v), _f64(do)
+    L, H, d = Q.shape
+    if world < 1 or L % world:
+        raise ValueError("the sequence must split into `world` equal shards")
+    S = L // world
+    O, LSE = ring_attention_forward(Q, K, V, scale, causal, world)
+    D = (dO * O).sum(axis=-1)                                  # [L, H]
+    dQ, dK, dV = np.zeros_like(Q), np.zeros_like(K), np.zeros_like(V)
+    sh = lambda x, r: x[r * S:(r + 1) * S]
+    for r in range(world):
+        for t in range(world):
+            s_ = (r - t) % world
+            if causal and s_ > r:
+                continue
+            for h in range(H):
+                Qr, Ks, Vs, dOr = sh(Q, r)[:, h], sh(K, s_)[:, h], sh(V, s_)[:, h], sh(dO, r)[:, h]
+                P = np.exp((Qr @ Ks.T) * scale - sh(LSE, r)[:, h][:, None])
+                if causal and s_ == r:
+                    P[np.triu_indices(S, k=1)] = 0.0
+                dS = P * (dOr @ Vs.T - sh(D, r)[:, h][:, None])
+                dQ[r * S:(r + 1) * S, h] += scale * (dS @ Ks)
+                dK[s_ * S:(s_ + 1) * S, h] += scale * (dS.T @ Qr)
+                dV[s_ * S:(s_ + 1) * S, h] += P.T @ dOr
+    return dQ, dK, dV
 
 
 # ----------------------------------------------------------------------------- dropout on P

@@ -787,3 +787,46 @@ def test_ring_and_merge_pins_catch_planted_mistakes():
         assert not _ring_pins_pass(m, ring), m.__name__
     for rv in (ring_sees_future, ring_skips_diagonal, ring_diag_unmasked):
         assert not _ring_pins_pass(merge, rv)
+
+
+def test_ring_backward_equals_definition():
+    """The ring backward (blocks from the global LSE and D, dK/dV travelling with their shard) equals
+    the whole-sequence backward for 1 … 6 ranks, causal and not; dropping the causal skip, using the
+    block's own LSE instead of the global one, or leaving out D each breaks it."""
+    rng = np.random.default_rng(33)
+    q, k, v, do = (rng.standard_normal((12, 2, 4)) for _ in range(4))
+    for causal in (False, True):
+        ref = oracle.attention_backward(q, k, v, do, 0.45, causal)
+        for w in (1, 2, 3, 4, 6):
+            got = oracle.ring_attention_backward(q, k, v, do, 0.45, causal, w)
+            for a, b in zip(got, ref):
+                assert np.allclose(a, b, atol=1e-12, rtol=0)
+    # planted mistakes, checked against the same definition
+    def ring_bwd_variant(q, k, v, do, scale, causal, world, own_lse=False, no_skip=False, no_d=False):
+        Q, K, V, dO = (np.asarray(x, dtype=np.float64) for x in (q, k, v, do))
+        L, H, d = Q.shape
+        S = L // world
+        O, LSE = oracle.ring_attention_forward(Q, K, V, scale, causal, world)
+        D = 0.0 * O.sum(axis=-1) if no_d else (dO * O).sum(axis=-1)
+        dQ, dK, dV = np.zeros_like(Q), np.zeros_like(K), np.zeros_like(V)
+        for r in range(world):
+            for s_ in range(world):
+                if causal and s_ > r and not no_skip:
+                    continue
+                rows, cols = slice(r * S, (r + 1) * S), slice(s_ * S, (s_ + 1) * S)
+                for h in range(H):
+                    Sc = (Q[rows, h] @ K[cols, h].T) * scale
+                    if causal and s_ == r:
+                        Sc[np.triu_indices(S, k=1)] = -np.inf
+                    lse = np.log(np.exp(Sc).sum(axis=1)) if own_lse else LSE[rows, h]
+                    P = np.exp(Sc - lse[:, None])
+                    dS = P * (dO[rows, h] @ V[cols, h].T - D[rows, h][:, None])
+                    dQ[rows, h] += scale * (dS @ K[cols, h])
+                    dK[cols, h] += scale * (dS.T @ Q[rows, h])
+                    dV[cols, h] += P.T @ dO[rows, h]
+        return dQ, dK, dV
+    ref = oracle.attention_backward(q, k, v, do, 0.45, True)
+    ok = lambda got: all(np.allclose(a, b, atol=1e-9, rtol=0) for a, b in zip(got, ref))
+    assert ok(ring_bwd_variant(q, k, v, do, 0.45, True, 3))
+    for kw in (dict(own_lse=True), dict(no_skip=True), dict(no_d=True)):
+        assert not ok(ring_bwd_variant(q, k, v, do, 0.45, True, 3, **kw)), kw
