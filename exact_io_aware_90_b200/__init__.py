@@ -9,7 +9,7 @@ GPU is present the calls raise.
 
 Raw ABI (same names and argument order as ``include/fa.h``; pointers are ints):
     fa_fwd, fa_bwd, fa_bwd_preprocess, fa_bwd_main, fa_bwd_postprocess,
-    fa_bwd_workspace_bytes, fa_bwd_noalloc, fa_fwd_dropout, fa_bwd_dropout, fa_fwd_fp8, fa_attn_merge, fa_decode,
+    fa_bwd_workspace_bytes, fa_bwd_noalloc, fa_fwd_dropout, fa_bwd_dropout, fa_fwd_fp8, fa_attn_merge, fa_accumulate, fa_decode,
     fa_decode_workspace_bytes, fa_check_device_status, fa_set_watchdog_ns, fa_watchdog_selftest, fa_status_string, fa_version
 Torch wrappers:
     attention_forward(q, k, v, ...)          -> (o, lse)
@@ -31,7 +31,7 @@ __all__ = [
     "FAError", "LIB_PATH", "lib", "FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA",
     "FA_ERR_TIMEOUT", "FA_BF16", "FA_FP16",
     "fa_fwd", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_postprocess", "fa_bwd_workspace_bytes",
-    "fa_bwd_noalloc", "FA_NOALLOC_SCRATCH_BYTES", "fa_fwd_dropout", "fa_bwd_dropout", "fa_fwd_fp8", "fa_attn_merge", "fa_decode", "fa_decode_workspace_bytes", "fa_check_device_status", "fa_set_watchdog_ns", "fa_watchdog_selftest", "fa_status_string", "fa_version",
+    "fa_bwd_noalloc", "FA_NOALLOC_SCRATCH_BYTES", "fa_fwd_dropout", "fa_bwd_dropout", "fa_fwd_fp8", "fa_attn_merge", "fa_accumulate", "fa_decode", "fa_decode_workspace_bytes", "fa_check_device_status", "fa_set_watchdog_ns", "fa_watchdog_selftest", "fa_status_string", "fa_version",
     "attention_forward", "attention_backward", "attention_decode", "attention_forward_fp8", "attention_merge", "dtype_code",
 ]
 
@@ -68,6 +68,7 @@ def _load() -> ctypes.CDLL:
                                P]),
         "fa_fwd_fp8": (I, [P, P, P, P, P, I, I, I, I, F, I, P, I, F, F, F, P]),
         "fa_attn_merge": (I, [P, P, P, P, P, I, I, I, I, I, P]),
+        "fa_accumulate": (I, [P, P, P, ctypes.c_longlong, I, I, P]),
         "fa_decode_workspace_bytes": (S, [I, I, I, I]),
         "fa_decode": (I, [P, P, P, P, P, I, I, I, I, F, P, I, I, P, S, P]),
         "fa_check_device_status": (I, [P]),
@@ -148,6 +149,10 @@ def fa_fwd_fp8(q, k, v, o, lse, B, H, N, d, scale, causal, cu_seqlens, total_tok
 
 def fa_attn_merge(acc_o, acc_lse, part_o, part_lse, out, T, H, d, dtype, first, stream) -> int:
     return lib.fa_attn_merge(acc_o, acc_lse, part_o, part_lse, out, T, H, d, dtype, first, stream)
+
+
+def fa_accumulate(acc, part, out, n, dtype, first, stream) -> int:
+    return lib.fa_accumulate(acc, part, out, n, dtype, first, stream)
 
 
 def fa_decode_workspace_bytes(B, H, Nk, d) -> int:

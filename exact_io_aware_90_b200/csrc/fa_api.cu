@@ -324,6 +324,14 @@ int fa_attn_merge(float* acc_o, float* acc_lse, const void* part_o, const float*
                                  reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int fa_accumulate(float* acc, const void* part, void* out, long long n, int dtype, int first, fa_stream_t stream) {
+  if (!aligned16(acc) || (part != nullptr && !aligned16(part)) || (out != nullptr && !aligned16(out)))
+    return FA_ERR_INVALID_ARG;
+  if (n < 8 || (n & 7) != 0 || (first != 0 && first != 1)) return FA_ERR_INVALID_ARG;
+  if (dtype != FA_BF16 && dtype != FA_FP16) return FA_ERR_INVALID_ARG;
+  return map_launch(launch_accumulate(acc, part, out, n, dtype == FA_BF16, first, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 size_t fa_decode_workspace_bytes(int B, int H, int Nk, int d) {
   if (B < 1 || H < 1 || Nk < 1 || (d != 64 && d != 128)) return 0;
   const size_t slots = (size_t)B * H * decode_chunks(Nk);

@@ -82,6 +82,10 @@ cudaError_t launch_fwd(const Problem& pb, const FwdArgs& a, cudaStream_t stream)
 cudaError_t launch_merge(float* acc_o, float* acc_lse, const void* part_o, const float* part_lse, void* out,
                          long long rows, int d, bool bf16, int first, cudaStream_t stream);
 
+// acc (+)= part over n elements (n a multiple of 8), optionally written to `out` in the dtype (fa_merge.cu).
+cudaError_t launch_accumulate(float* acc, const void* part, void* out, long long n, bool bf16, int first,
+                              cudaStream_t stream);
+
 cudaError_t launch_decode(const Problem& pb, const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_bwd_pre(const Problem& pb, const BwdArgs& a, cudaStream_t stream);
 cudaError_t launch_bwd_main(const Problem& pb, const BwdArgs& a, cudaStream_t stream);

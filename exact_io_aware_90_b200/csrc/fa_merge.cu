@@ -1,4 +1,6 @@
-// fa_merge.cu — merge of normalised partial attention results of the same queries over disjoint key sets
+// fa_merge.cu — ring (context-parallel) attention's elementwise kernels.
+//
+// Merge of normalised partial attention results of the same queries over disjoint key sets
 // (the block-merge rule of "FlashAttention 与算子融合", "FlashAttention 的两个关键", online softmax:
 // m = max, ℓ = Σ ℓ_c·e^{m_c − m}, partial outputs scaled the same way), as ring / context-parallel
 // attention produces them one block at a time.  A normalised part (O_b, LSE_b) is the pair
@@ -9,6 +11,8 @@
 // 16-bit part, 32-byte loads and stores of the fp32 accumulator.
 #include "fa_internal.h"
 #include "sm100.cuh"
+
+#include <algorithm>
 
 namespace fa {
 
@@ -69,6 +73,54 @@ __global__ void __launch_bounds__(256) fa_merge_kernel(float* __restrict__ acc_o
     acc4[0] = make_float4(o[0], o[1], o[2], o[3]);
     acc4[1] = make_float4(o[4], o[5], o[6], o[7]);
   }
+}
+
+// Gradient accumulation for the ring backward: acc (+)= part over n elements (8 per thread), where
+// part is a dtype gradient partial (NULL: nothing added); with `out` the sum is written there in the
+// dtype instead of back into acc.  Elementwise, HBM-bound.
+template <bool BF16>
+__global__ void __launch_bounds__(256) fa_accum_kernel(float4* __restrict__ acc, const uint4* __restrict__ part,
+                                                        uint4* __restrict__ out, long long n8, int first) {
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (long long)gridDim.x * blockDim.x) {
+    float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (!first) {
+      const float4 a0 = acc[2 * i], a1 = acc[2 * i + 1];
+      v[0] = a0.x; v[1] = a0.y; v[2] = a0.z; v[3] = a0.w;
+      v[4] = a1.x; v[5] = a1.y; v[6] = a1.z; v[7] = a1.w;
+    }
+    if (part != nullptr) {
+      const uint4 pb = part[i];
+      const uint32_t pw[4] = {pb.x, pb.y, pb.z, pb.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 f = unpack2<BF16>(pw[k]);
+        v[2 * k] += f.x;
+        v[2 * k + 1] += f.y;
+      }
+    }
+    if (out != nullptr) {
+      out[i] = make_uint4(pack2<BF16>(v[0], v[1]), pack2<BF16>(v[2], v[3]), pack2<BF16>(v[4], v[5]),
+                          pack2<BF16>(v[6], v[7]));
+    } else {
+      acc[2 * i] = make_float4(v[0], v[1], v[2], v[3]);
+      acc[2 * i + 1] = make_float4(v[4], v[5], v[6], v[7]);
+    }
+  }
+}
+
+cudaError_t launch_accumulate(float* acc, const void* part, void* out, long long n, bool bf16, int first,
+                              cudaStream_t stream) {
+  const long long n8 = n / 8;
+  const unsigned blocks = (unsigned)std::min<long long>((n8 + 255) / 256, 148LL * 16);
+  if (bf16)
+    fa_accum_kernel<true><<<blocks, 256, 0, stream>>>(reinterpret_cast<float4*>(acc),
+                                                      reinterpret_cast<const uint4*>(part),
+                                                      reinterpret_cast<uint4*>(out), n8, first);
+  else
+    fa_accum_kernel<false><<<blocks, 256, 0, stream>>>(reinterpret_cast<float4*>(acc),
+                                                       reinterpret_cast<const uint4*>(part),
+                                                       reinterpret_cast<uint4*>(out), n8, first);
+  return cudaPeekAtLastError();
 }
 
 cudaError_t launch_merge(float* acc_o, float* acc_lse, const void* part_o, const float* part_lse, void* out,

@@ -8,7 +8,13 @@ to it with the library's forward kernel — the causal diagonal block when s = r
 nothing when s > r under the causal mask — then folds the block's (O, LSE) into its running result
 with the library's merge kernel (FlashAttention 与算子融合, 工程实践 "与 CP 配合": ring attention for
 very long sequences with FlashAttention as the compute core; the merge is the block-merge rule of the
-same page, "FlashAttention 的两个关键").  Forward only.
+same page, "FlashAttention 的两个关键").
+
+The backward runs the same ring.  A block's gradients come from the library's backward kernel given
+the global O and LSE of the rank's queries (P recomputed from the global LSE, D from the global O):
+its dQ part adds into the rank's fp32 dQ accumulator (the kernel's own reduce-add), its dK and dV
+parts add (fa_accumulate) into fp32 accumulators that travel with the key/value shard and are home
+after one more step.
 
 The per-rank state (``RingAttention``) is separate from the transport (``ring_attention_forward``),
 so the same per-step code runs under NCCL, under another backend, or with the ranks of a ring laid
@@ -20,7 +26,7 @@ from __future__ import annotations
 import math
 from typing import Callable, Optional, Tuple
 
-from . import attention_forward, attention_merge
+from . import FA_OK, FAError, attention_forward, attention_merge, dtype_code, lib
 
 
 def ring_block(rank: int, step: int, world: int, causal: bool) -> Tuple[int, Optional[str]]:
@@ -116,3 +122,115 @@ def ring_attention_forward(q, k, v, causal: bool = False, scale: Optional[float]
         if t < world - 1:
             cur_k, cur_v = bufs[t % 2]
     return ra.result()
+
+
+class RingAttentionBackward:
+    """One rank's backward state.  Call ``consume(step, k, v, dk_acc, dv_acc)`` with the shard held at
+    each step and the fp32 dK/dV accumulators travelling with it (``new_accumulators()`` makes the
+    rank's own, consumed at step 0), then ``finish(dk_acc, dv_acc)`` with the accumulators of its own
+    shard once they are home → (dq, dk, dv) in q's dtype.  o, lse: the ring forward's result."""
+
+    def __init__(self, q, o, lse, do, rank: int, world: int, causal: bool, scale: Optional[float] = None):
+        import torch
+        S, H, d = q.shape
+        self.q, self.o, self.lse, self.do = q, o, lse, do
+        self.rank, self.world, self.causal = rank, world, causal
+        self.S, self.H, self.d = S, H, d
+        self.scale = 1.0 / math.sqrt(d) if scale is None else scale
+        self.dt = dtype_code(q)
+        self.stream = torch.cuda.current_stream(q.device).cuda_stream
+        self.ws_bytes = lib.fa_bwd_workspace_bytes(S, H, d)
+        self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=q.device)
+        self.tmp_dk, self.tmp_dv = torch.empty_like(q), torch.empty_like(q)
+        # D = rowsum(dO ∘ O) of the global output and a zeroed dQ accumulator
+        self._check(lib.fa_bwd_preprocess(o.data_ptr(), do.data_ptr(), 1, H, S, d, None, S, self.dt, self.ws.data_ptr(),
+                                          self.ws_bytes, self.stream), "fa_bwd_preprocess")
+
+    @staticmethod
+    def _check(st, where):
+        if st != FA_OK:
+            raise FAError(st, where)
+
+    def new_accumulators(self):
+        import torch
+        return (torch.empty((self.S, self.H, self.d), dtype=torch.float32, device=self.q.device),
+                torch.empty((self.S, self.H, self.d), dtype=torch.float32, device=self.q.device))
+
+    def _acc(self, acc, part, out, first):
+        self._check(lib.fa_accumulate(acc.data_ptr(), None if part is None else part.data_ptr(),
+                                      None if out is None else out.data_ptr(), acc.numel(), self.dt, int(first),
+                                      self.stream), "fa_accumulate")
+
+    def consume(self, step: int, k, v, dk_acc, dv_acc) -> None:
+        _, kind = ring_block(self.rank, step, self.world, self.causal)
+        if kind is None:
+            return  # the accumulators pass on unchanged
+        self._check(lib.fa_bwd_main(self.q.data_ptr(), k.data_ptr(), v.data_ptr(), self.lse.data_ptr(),
+                                    self.do.data_ptr(), self.tmp_dk.data_ptr(), self.tmp_dv.data_ptr(), 1, self.H,
+                                    self.S, self.d, float(self.scale), int(kind == "causal"), None, self.S, self.dt,
+                                    self.ws.data_ptr(), self.ws_bytes, self.stream), "fa_bwd_main")
+        # step 0 is the rank's own shard, always computed: it starts the shard's accumulators
+        self._acc(dk_acc, self.tmp_dk, None, step == 0)
+        self._acc(dv_acc, self.tmp_dv, None, step == 0)
+
+    def finish(self, dk_acc, dv_acc):
+        import torch
+        dq = torch.empty_like(self.q)
+        self._check(lib.fa_bwd_postprocess(dq.data_ptr(), 1, self.H, self.S, self.d, float(self.scale), None, self.S,
+                                           self.dt, self.ws.data_ptr(), self.ws_bytes, self.stream),
+                    "fa_bwd_postprocess")
+        dk, dv = torch.empty_like(self.q), torch.empty_like(self.q)
+        self._acc(dk_acc, None, dk, False)
+        self._acc(dv_acc, None, dv, False)
+        return dq, dk, dv
+
+
+def ring_attention_backward(q, k, v, o, lse, do, causal: bool = False, scale: Optional[float] = None, group=None,
+                            state=None):
+    """dq, dk, dv of this rank's shards for the ring forward that produced (o, lse) on the same group.
+    ``state`` replaces the rank's RingAttentionBackward (an object with the same three methods)."""
+    import torch
+    import torch.distributed as dist
+
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    peer = (lambda r: r) if group is None else (lambda r: dist.get_global_rank(group, r))
+    nxt, prv = peer((rank + 1) % world), peer((rank - 1) % world)
+    rb = state if state is not None else RingAttentionBackward(q, o, lse, do, rank, world, causal, scale)
+    if world == 1:
+        acc = rb.new_accumulators()
+        rb.consume(0, k, v, *acc)
+        return rb.finish(*acc)
+    kv_bufs = [(torch.empty_like(k), torch.empty_like(v)) for _ in range(min(2, world - 1))]
+    acc_bufs = [rb.new_accumulators() for _ in range(2)]
+    cur_k, cur_v = k, v
+    cur_acc = rb.new_accumulators()
+    acc_reqs = []
+    for t in range(world):
+        kv_reqs = []
+        if t < world - 1:  # the next shard's K and V stream in while this block computes
+            rk, rv = kv_bufs[t % 2]
+            kv_reqs = dist.batch_isend_irecv([dist.P2POp(dist.isend, cur_k, nxt, group),
+                                              dist.P2POp(dist.isend, cur_v, nxt, group),
+                                              dist.P2POp(dist.irecv, rk, prv, group),
+                                              dist.P2POp(dist.irecv, rv, prv, group)])
+        for r in acc_reqs:  # this shard's accumulators have arrived
+            r.wait()
+        rb.consume(t, cur_k, cur_v, *cur_acc)
+        # the accumulators move on once this rank has added to them (after the last step: home)
+        nxt_acc = acc_bufs[t % 2]
+        acc_reqs = dist.batch_isend_irecv([dist.P2POp(dist.isend, cur_acc[0], nxt, group),
+                                           dist.P2POp(dist.isend, cur_acc[1], nxt, group),
+                                           dist.P2POp(dist.irecv, nxt_acc[0], prv, group),
+                                           dist.P2POp(dist.irecv, nxt_acc[1], prv, group)])
+        for r in kv_reqs:
+            r.wait()
+        if t < world - 1:
+            cur_k, cur_v = kv_bufs[t % 2]
+        # the buffers just sent may be reused two steps on, after the sends completed (waited below)
+        sent = cur_acc
+        cur_acc = nxt_acc
+        acc_bufs[t % 2] = sent
+    for r in acc_reqs:
+        r.wait()
+    return rb.finish(*cur_acc)

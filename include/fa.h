@@ -257,6 +257,20 @@ int fa_attn_merge(float* acc_o, float* acc_lse, const void* part_o, const float*
                   int T, int H, int d, int dtype, int first, fa_stream_t stream);
 
 /*
+ * Accumulation of gradient partials (the ring backward: the dK and dV
+ * contributions of each rank to a key/value shard add up in fp32 as the
+ * shard travels): over n elements,
+ *   v = (first ? 0 : acc[i]) + (part ? part[i] : 0);
+ *   out ? out[i] = dtype(v) (nearest even) : acc[i] = v.
+ *   acc   fp32 [n], 16-byte aligned; part, out  dtype [n] or NULL, 16-byte
+ *   aligned; n a positive multiple of 8.
+ * FA_ERR_INVALID_ARG for bad arguments, FA_ERR_CUDA for a failed launch.
+ * Asynchronous on `stream`.
+ */
+int fa_accumulate(float* acc, const void* part, void* out, long long n, int dtype, int first,
+                  fa_stream_t stream);
+
+/*
  * Decode: one new query token per sequence attends to every key of its
  * sequence in a K/V cache (token-by-token generation, the workload
  * "FlashAttention 短片讲解稿", segment "适用范围与关键结论", sets apart from

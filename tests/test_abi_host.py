@@ -33,7 +33,7 @@ def test_header_declares_the_entry_points():
     for n in ["fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_bwd_preprocess", "fa_bwd_main",
               "fa_bwd_postprocess", "fa_check_device_status", "fa_status_string", "fa_set_watchdog_ns",
               "fa_watchdog_selftest", "fa_version", "fa_bwd_noalloc", "fa_decode", "fa_decode_workspace_bytes",
-              "fa_fwd_dropout", "fa_bwd_dropout", "fa_fwd_fp8", "fa_attn_merge"]:
+              "fa_fwd_dropout", "fa_bwd_dropout", "fa_fwd_fp8", "fa_attn_merge", "fa_accumulate"]:
         assert n in names
 
 
@@ -142,6 +142,13 @@ def test_merge_rejects_invalid_arguments(fa):
         args = list(ok)
         args[i] = bad
         assert fa.fa_attn_merge(*args) == fa.FA_ERR_INVALID_ARG, i
+
+
+def test_accumulate_rejects_invalid_arguments(fa):
+    for args in ([P16 + 4, P16, None, 4096, 0, 0], [P16, P16 + 8, None, 4096, 0, 0], [P16, None, P16 + 2, 4096, 0, 0],
+                 [P16, P16, None, 4095, 0, 0], [P16, P16, None, 0, 0, 0], [P16, P16, None, 4096, 5, 0],
+                 [P16, P16, None, 4096, 0, 3]):
+        assert fa.fa_accumulate(*args, None) == fa.FA_ERR_INVALID_ARG, args
 
 
 def test_decode_workspace_bytes(fa):

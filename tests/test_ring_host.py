@@ -103,3 +103,85 @@ def test_ring_attention_gloo(world, causal):
     for rank, err, untouched in got:
         assert err < 1e-5, (rank, err)  # the running O and LSE are fp32 buffers, as on the GPU
         assert untouched, rank
+
+
+class _OracleBackwardState:
+    """The per-rank backward steps done by the fp64 oracle on CPU tensors (the same blocks as the
+    kernels: P from the global LSE, D from the global O)."""
+
+    def __init__(self, q, o, lse, do, rank, world, causal, scale):
+        self.q, self.o, self.lse, self.do = (x.double().numpy() for x in (q, o, lse, do))
+        self.rank, self.world, self.causal, self.scale = rank, world, causal, scale
+        self.D = (self.do * self.o).sum(axis=-1)
+        self.dq = np.zeros_like(self.q)
+
+    def new_accumulators(self):
+        return torch.zeros(self.q.shape, dtype=torch.float32), torch.zeros(self.q.shape, dtype=torch.float32)
+
+    def consume(self, step, k, v, dk_acc, dv_acc):
+        from exact_io_aware_90_b200.ring import ring_block
+        _, kind = ring_block(self.rank, step, self.world, self.causal)
+        if kind is None:
+            return
+        K, V = k.double().numpy(), v.double().numpy()
+        S = self.q.shape[0]
+        for h in range(self.q.shape[1]):
+            P = np.exp((self.q[:, h] @ K[:, h].T) * self.scale - self.lse[:, h][:, None])
+            if kind == "causal":
+                P[np.triu_indices(S, k=1)] = 0.0
+            dS = P * (self.do[:, h] @ V[:, h].T - self.D[:, h][:, None])
+            self.dq[:, h] += self.scale * (dS @ K[:, h])
+            dk_acc[:, h] += torch.from_numpy(self.scale * (dS.T @ self.q[:, h])).float()
+            dv_acc[:, h] += torch.from_numpy(P.T @ self.do[:, h]).float()
+
+    def finish(self, dk_acc, dv_acc):
+        return torch.from_numpy(self.dq), dk_acc.double(), dv_acc.double()
+
+
+def _rank_main_bwd(rank, world, port, causal, out_q):
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        import oracle
+        from exact_io_aware_90_b200.ring import ring_attention_backward
+        L, H, d = 24, 2, 8
+        g = np.random.default_rng(8)
+        q, k, v, do = (g.standard_normal((L, H, d)) for _ in range(4))
+        O, LSE = oracle.attention_forward(q, k, v, 0.35, causal)
+        S = L // world
+        sl = slice(rank * S, (rank + 1) * S)
+        t = lambda x: torch.from_numpy(np.ascontiguousarray(x[sl]))
+        state = _OracleBackwardState(t(q), t(O), t(LSE), t(do), rank, world, causal, 0.35)
+        ks, vs = t(k), t(v)
+        dq, dk, dv = ring_attention_backward(t(q), ks, vs, t(O), t(LSE), t(do), causal=causal, state=state)
+        ref = oracle.attention_backward(q, k, v, do, 0.35, causal)
+        err = max(float(np.abs(a.numpy() - b[sl]).max()) for a, b in zip((dq, dk, dv), ref))
+        dist.barrier()
+        out_q.put((rank, err, bool(torch.equal(ks, t(k)) and torch.equal(vs, t(v)))))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+@pytest.mark.parametrize("causal", [False, True])
+def test_ring_attention_backward_gloo(world, causal):
+    """The backward ring's transport over gloo: K/V shards and their travelling dK/dV accumulators
+    reach every rank in order and come home; every rank's gradients equal the oracle's over the whole
+    sequence (to the fp32 accumulators)."""
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main_bwd, args=(r, world, port, causal, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = [q.get(timeout=180) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, err, untouched in got:
+        assert err < 1e-5, (rank, err)
+        assert untouched, rank
