@@ -185,3 +185,40 @@ def test_ring_attention_backward_gloo(world, causal):
     for rank, err, untouched in got:
         assert err < 1e-5, (rank, err)
         assert untouched, rank
+
+
+def _rank_main_single(port, out_q):
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=0, world_size=1, timeout=datetime.timedelta(seconds=60))
+    try:
+        import oracle
+        from exact_io_aware_90_b200.ring import ring_attention_backward, ring_attention_forward
+        g = np.random.default_rng(9)
+        q, k, v, do = (g.standard_normal((16, 2, 8)) for _ in range(4))
+        t = lambda x: torch.from_numpy(np.ascontiguousarray(x))
+        o, lse = ring_attention_forward(t(q), t(k), t(v), causal=True, scale=0.3, block_fn=_oracle_block,
+                                        merge_fn=_oracle_merge)
+        O_ref, L_ref = oracle.attention_forward(q, k, v, 0.3, True)
+        state = _OracleBackwardState(t(q), o.double(), lse.double(), t(do), 0, 1, True, 0.3)
+        grads = ring_attention_backward(t(q), t(k), t(v), o, lse, t(do), causal=True, state=state)
+        ref = oracle.attention_backward(q, k, v, do, 0.3, True)
+        err = max([float(np.abs(o.numpy() - O_ref).max()), float(np.abs(lse.numpy() - L_ref).max())] +
+                  [float(np.abs(a.numpy() - b).max()) for a, b in zip(grads, ref)])
+        out_q.put(err)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_ring_single_rank_gloo():
+    """A ring of one rank: no exchange, the whole sequence is the rank's own (causal) block."""
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    p = ctx.Process(target=_rank_main_single, args=(_free_port(), q))
+    p.start()
+    err = q.get(timeout=120)
+    p.join(timeout=60)
+    assert p.exitcode == 0 and err < 1e-5, err
