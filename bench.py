@@ -62,6 +62,7 @@ def load_peaks():
 KERNEL_SOURCES = {
     "fa_fwd_kernel": ["fa_fwd.cu", "sm100.cuh", "fa_internal.h"],
     "fa_bwd_main_kernel": ["fa_bwd.cu", "sm100.cuh", "fa_internal.h"],
+    "fa_decode_split_kernel": ["fa_decode.cu", "sm100.cuh", "fa_internal.h"],
 }
 
 
@@ -590,7 +591,8 @@ def run_gpu_decode(args, world, rank, local, pg):
                    "parallelism": f"replicas x{world} (independent workloads per GPU)"},
         "roofline": {"kernel": "fa_decode_split_kernel + fa_decode_merge_kernel", "bound": "hbm",
                      "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None,
+                     "frac": round(gbs / peaks["hbm_gbs"], 4),
+                     "traffic": load_traffic("fa_decode_split_kernel", wname),  # the split kernel: the K/V stream
                      "algorithmic_bytes": algo_bytes, "peak_source": peaks["source"]},
         "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": int(hq.numel() * hq.element_size()),
