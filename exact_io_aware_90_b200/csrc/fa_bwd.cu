@@ -797,13 +797,10 @@ cudaError_t launch_bwd_post(const Problem& pb, const BwdArgs& a, cudaStream_t st
 template <int D, bool BF16, bool DROP>
 static cudaError_t launch_main_t(const Problem& pb, const BwdArgs& a, cudaStream_t stream) {
   using C = BwdCfg<D>;
-  static bool configured = false;
+  static std::atomic<unsigned long long> configured{0};  // per instantiation, one bit per device
   auto kern = fa_bwd_main_kernel<D, BF16, DROP>;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  if (cudaError_t e = set_smem_once(configured, reinterpret_cast<const void*>(kern), C::SMEM_BYTES); e != cudaSuccess)
+    return e;
   BwdParams p;
   p.lse = a.lse;
   p.delta = a.delta;

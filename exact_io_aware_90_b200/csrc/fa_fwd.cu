@@ -792,13 +792,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 template <int D, bool BF16, bool DROP, bool FP8 = false>
 static cudaError_t launch_fwd_t(const Problem& pb, const FwdArgs& a, cudaStream_t stream) {
   using C = FwdCfg<D, FP8 ? 1 : 2>;
-  static bool configured = false;  // per instantiation
+  static std::atomic<unsigned long long> configured{0};  // per instantiation, one bit per device
   auto kern = fa_fwd_kernel<D, BF16, DROP, FP8>;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  if (cudaError_t e = set_smem_once(configured, reinterpret_cast<const void*>(kern), C::SMEM_BYTES); e != cudaSuccess)
+    return e;
   FwdParams p;
   p.o = a.o;
   p.lse = a.lse;

@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cstddef>
+#include <atomic>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -18,6 +19,20 @@ struct Dropout {
   uint32_t seed_lo, seed_hi;
   uint32_t offset;
 };
+
+// Raises a kernel's dynamic shared-memory limit on the current device once per device: the attribute
+// belongs to the device's context, so a process driving several GPUs sets it on each.  `done` holds
+// one bit per device ordinal (ordinals from 64 on set it on every call).
+inline cudaError_t set_smem_once(std::atomic<unsigned long long>& done, const void* kern, int bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
+  if (bit != 0ull && (done.load(std::memory_order_acquire) & bit) != 0ull) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_release);
+  return e;
+}
 
 // Work of one attention call, resolved on the host.
 struct Problem {
