@@ -75,6 +75,23 @@ def test_reference_arm_json_line():
     assert d["steps"] == 2 and d["warmup"] == 3
 
 
+@pytest.mark.parametrize("extra, metric_tail", [(["--workload", "tiny_d64", "--dropout", "0.1"], ""),
+                                                 (["--workload", "decode_b16_kv8k"], "(decode: one query per sequence)")])
+def test_reference_arm_other_paths(extra, metric_tail):
+    """The reference arm of the dropout step and of decode: one contract line from the oracle."""
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "3"] + extra, capture_output=True, text=True, env=env, timeout=600)
+    assert r.returncode == 0, r.stderr
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["metric"].endswith(metric_tail)
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
+    if "--dropout" in extra:
+        assert d["config"]["dropout_p"] == 0.1 and "dropout oracle" in d["cpu_baseline"]["sample"]
+
+
 def test_reference_arm_other_ranks_exit_quietly():
     env = dict(os.environ, RANK="1", WORLD_SIZE="2")
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
