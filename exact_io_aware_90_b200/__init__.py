@@ -9,7 +9,8 @@ GPU is present the calls raise.
 
 Raw ABI (same names and argument order as ``include/fa.h``; pointers are ints):
     fa_fwd, fa_bwd, fa_bwd_preprocess, fa_bwd_main, fa_bwd_postprocess,
-    fa_bwd_workspace_bytes, fa_bwd_noalloc, fa_fwd_dropout, fa_bwd_dropout, fa_fwd_fp8, fa_attn_merge, fa_accumulate, fa_decode,
+    fa_bwd_workspace_bytes, fa_bwd_noalloc, fa_fwd_dropout, fa_bwd_dropout, fa_fwd_fp8, fa_fwd_fp8_per_head, fa_attn_merge, fa_accumulate,
+    fa_decode,
     fa_decode_workspace_bytes, fa_check_device_status, fa_set_watchdog_ns, fa_watchdog_selftest, fa_status_string, fa_version
 Torch wrappers:
     attention_forward(q, k, v, ...)          -> (o, lse)
@@ -31,7 +32,7 @@ __all__ = [
     "FAError", "LIB_PATH", "lib", "FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA",
     "FA_ERR_TIMEOUT", "FA_BF16", "FA_FP16",
     "fa_fwd", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_postprocess", "fa_bwd_workspace_bytes",
-    "fa_bwd_noalloc", "FA_NOALLOC_SCRATCH_BYTES", "fa_fwd_dropout", "fa_bwd_dropout", "fa_fwd_fp8", "fa_attn_merge", "fa_accumulate", "fa_decode", "fa_decode_workspace_bytes", "fa_check_device_status", "fa_set_watchdog_ns", "fa_watchdog_selftest", "fa_status_string", "fa_version",
+    "fa_bwd_noalloc", "FA_NOALLOC_SCRATCH_BYTES", "fa_fwd_dropout", "fa_bwd_dropout", "fa_fwd_fp8", "fa_fwd_fp8_per_head", "fa_attn_merge", "fa_accumulate", "fa_decode", "fa_decode_workspace_bytes", "fa_check_device_status", "fa_set_watchdog_ns", "fa_watchdog_selftest", "fa_status_string", "fa_version",
     "attention_forward", "attention_backward", "attention_decode", "attention_forward_fp8", "attention_merge", "dtype_code",
 ]
 
@@ -67,6 +68,7 @@ def _load() -> ctypes.CDLL:
         "fa_bwd_dropout": (I, [P, P, P, P, P, P, P, P, P, I, I, I, I, F, I, P, I, I, F, U64, ctypes.c_uint32, P, S,
                                P]),
         "fa_fwd_fp8": (I, [P, P, P, P, P, I, I, I, I, F, I, P, I, F, F, F, P]),
+        "fa_fwd_fp8_per_head": (I, [P, P, P, P, P, I, I, I, I, F, I, P, I, P, P, P, P]),
         "fa_attn_merge": (I, [P, P, P, P, P, I, I, I, I, I, P]),
         "fa_accumulate": (I, [P, P, P, ctypes.c_longlong, I, I, P]),
         "fa_decode_workspace_bytes": (S, [I, I, I, I]),
@@ -145,6 +147,12 @@ def fa_fwd_fp8(q, k, v, o, lse, B, H, N, d, scale, causal, cu_seqlens, total_tok
                v_descale, stream) -> int:
     return lib.fa_fwd_fp8(q, k, v, o, lse, B, H, N, d, scale, causal, cu_seqlens, total_tokens, q_descale, k_descale,
                           v_descale, stream)
+
+
+def fa_fwd_fp8_per_head(q, k, v, o, lse, B, H, N, d, scale, causal, cu_seqlens, total_tokens, q_descale, k_descale,
+                        v_descale, stream) -> int:
+    return lib.fa_fwd_fp8_per_head(q, k, v, o, lse, B, H, N, d, scale, causal, cu_seqlens, total_tokens, q_descale,
+                                   k_descale, v_descale, stream)
 
 
 def fa_attn_merge(acc_o, acc_lse, part_o, part_lse, out, T, H, d, dtype, first, stream) -> int:
@@ -288,7 +296,8 @@ def attention_forward_fp8(q, k, v, q_descale: float, k_descale: float, v_descale
                           scale: Optional[float] = None, cu_seqlens=None, max_seqlen: Optional[int] = None,
                           batch: Optional[int] = None, out=None, lse=None, stream=None):
     """O (bf16) and LSE for e4m3 q, k, v of shape [T, H, 128] whose real values are the stored ones times
-    the descales (see ``include/fa.h``, fa_fwd_fp8)."""
+    the descales: floats (one per tensor, fa_fwd_fp8) or fp32 CUDA tensors [B, H] (one per sequence and
+    head, fa_fwd_fp8_per_head); see ``include/fa.h``."""
     import torch
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.float8_e4m3fn or t.shape != q.shape:
@@ -302,8 +311,20 @@ def attention_forward_fp8(q, k, v, q_descale: float, k_descale: float, v_descale
         lse = torch.empty((T, H), dtype=torch.float32, device=q.device)
     if stream is None:
         stream = torch.cuda.current_stream(q.device).cuda_stream
-    st = lib.fa_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, d, float(scale), int(bool(causal)),
-                        _ptr(cu_seqlens), T, float(q_descale), float(k_descale), float(v_descale), stream)
+    per_head = [hasattr(x, "data_ptr") for x in (q_descale, k_descale, v_descale)]
+    if any(per_head):
+        if not all(per_head):
+            raise ValueError("the three descales must all be floats or all be [B, H] tensors")
+        for x in (q_descale, k_descale, v_descale):
+            if not x.is_cuda or x.dtype != torch.float32 or not x.is_contiguous() or x.numel() != B * H:
+                raise ValueError("per-head descales must be contiguous CUDA float32 tensors of B·H values")
+        st = lib.fa_fwd_fp8_per_head(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, d, float(scale),
+                                     int(bool(causal)), _ptr(cu_seqlens), T, _ptr(q_descale), _ptr(k_descale),
+                                     _ptr(v_descale), stream)
+    else:
+        st = lib.fa_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, d, float(scale),
+                            int(bool(causal)), _ptr(cu_seqlens), T, float(q_descale), float(k_descale), float(v_descale),
+                            stream)
     if st != FA_OK:
         raise FAError(st, "fa_fwd_fp8")
     return out, lse

@@ -58,6 +58,11 @@ struct FwdParams {
   int heads_group;   // heads per L2 group in the unit order
   float scale_log2;  // scale · log2(e) (· the q and k descales for e4m3 inputs)
   float o_scale;     // factor on O at the end: 1, or the v descale for e4m3 inputs
+  // e4m3 inputs with one descale per (sequence, head) (fp32 [B·H] device arrays, index b·H + h), or
+  // nullptr when the descales are per tensor (folded into scale_log2 and o_scale on the host)
+  const float* q_descale;
+  const float* k_descale;
+  const float* v_descale;
   uint64_t timeout_ns;
   Dropout drop;
 };
@@ -547,8 +552,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
     const uint32_t tS = tmem + lane_off + 128u * t;
     const uint32_t tO = tmem + lane_off + 256u + (uint32_t)(D * t);
-    const float c = p.scale_log2;
-    const float2 c2 = make_float2(c, c);
+    float c = p.scale_log2;  // per unit when the e4m3 descales are per (sequence, head)
+    float2 c2 = make_float2(c, c);
+    float o_scale_u = 1.f;   // the unit's v descale in that case (the FP8 instantiation only)
     const uint32_t keep_bias = keep_flag_bias(p.drop.t);  // used by the dropout variant only
     uint32_t un = 0;  // units read
     uint32_t sn = 0;  // S tiles of Q tile t consumed (all units)
@@ -567,6 +573,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       if (my_nkv == 0) continue;
       const int row = U.q0 + t * kBM + 32 * quarter + lane;  // position in the sequence
       const uint32_t drop_bh = (uint32_t)(U.b * p.H + U.h);
+      if constexpr (FP8) {
+        o_scale_u = p.o_scale;
+        if (p.q_descale != nullptr) {
+          const int bh = U.b * p.H + U.h;
+          c = p.scale_log2 * (__ldg(p.q_descale + bh) * __ldg(p.k_descale + bh));
+          c2 = make_float2(c, c);
+          o_scale_u = __ldg(p.v_descale + bh);
+        }
+      }
       const int key_limit = p.causal ? min(U.L, row + 1) : U.L;
       // A tile whose rows see a single KV tile (the first 128 rows of a causal
       // sequence, or a sequence of at most 128 tokens) averages few values, so
@@ -749,7 +764,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       if (ok && warp_wait(bar(C::B_PVDONE + t), (sn + my_nkv - 1) & 1, wd)) {
         tc_fence_after();
         const bool valid = row < U.L;
-        const float inv = (ell > 0.f) ? p.o_scale / ell : 0.f;  // o_scale: 1/(1 − p) with dropout, v's descale for e4m3
+        // o_scale: 1/(1 − p) with dropout, v's descale for e4m3
+        const float inv = (ell > 0.f) ? (FP8 ? o_scale_u : p.o_scale) / ell : 0.f;
         const size_t obase = ((size_t)(U.tok0 + (valid ? row : 0)) * p.H + U.h) * D;
         uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) + obase * 2;
 #pragma unroll
@@ -809,6 +825,9 @@ static cudaError_t launch_fwd_t(const Problem& pb, const FwdArgs& a, cudaStream_
   p.heads_group = 8;
   p.scale_log2 = pb.scale * (pb.fp8 ? pb.qk_descale : 1.f) * 1.4426950408889634f;
   p.o_scale = pb.drop.t != 0u ? pb.drop.keep_scale : (pb.fp8 ? pb.v_descale : 1.f);
+  p.q_descale = pb.q_descale_bh;
+  p.k_descale = pb.k_descale_bh;
+  p.v_descale = pb.v_descale_bh;
   p.timeout_ns = pb.timeout_ns;
   p.drop = pb.drop;
   const long long units = (long long)pb.B * pb.H * p.num_qblocks;

@@ -47,6 +47,10 @@ struct Problem {
   bool fp8;
   float qk_descale;  // q descale × k descale
   float v_descale;
+  // or one descale per (sequence, head): fp32 [B·H] device arrays (nullptr: per tensor)
+  const float* q_descale_bh;
+  const float* k_descale_bh;
+  const float* v_descale_bh;
 };
 
 struct FwdArgs {

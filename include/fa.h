@@ -231,6 +231,21 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
                float q_descale, float k_descale, float v_descale, fa_stream_t stream);
 
 /*
+ * fa_fwd_fp8 with one descale per (sequence, head) instead of per tensor:
+ * q_descale, k_descale, v_descale are fp32 device arrays [B·H] (index b·H + h,
+ * b the sequence), 4-byte aligned, read by the kernel (values are not
+ * checked on the host: each must be finite and > 0, else the output is
+ * undefined).  The descales of (b, h) are folded into that unit's softmax
+ * constant and output factor, exactly as the per-tensor ones are.  Errors as
+ * fa_fwd_fp8 (a null or misaligned descale array: FA_ERR_INVALID_ARG).
+ */
+int fa_fwd_fp8_per_head(const void* q, const void* k, const void* v, void* o, float* lse,
+                        int B, int H, int N, int d, float scale, int causal,
+                        const int32_t* cu_seqlens, int total_tokens,
+                        const float* q_descale, const float* k_descale, const float* v_descale,
+                        fa_stream_t stream);
+
+/*
  * Merge of normalised partial attention results: the same queries attended
  * to disjoint key sets (the blocks a ring of ranks visits in ring /
  * context-parallel attention, "FlashAttention 与算子融合", 工程实践 "与 CP

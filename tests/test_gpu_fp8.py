@@ -39,6 +39,9 @@ def fa():
 
 
 def _real(inp):
+    if "descale_bh" in inp.extra:  # one descale per (sequence, head)
+        ds, segs = inp.extra["descale_bh"], _seq_bounds(inp)
+        return tuple(workloads.real_values(t, ds[n], segs) for t, n in ((inp.q, "q"), (inp.k, "k"), (inp.v, "v")))
     ds = inp.extra["descale"]
     return (workloads.real_values(inp.q, ds["q"]), workloads.real_values(inp.k, ds["k"]),
             workloads.real_values(inp.v, ds["v"]))
@@ -46,7 +49,11 @@ def _real(inp):
 
 def _run(fa, inp, **over):
     dev = torch.device("cuda")
-    ds = dict(inp.extra["descale"], **over)
+    if "descale_bh" in inp.extra:
+        ds = {n: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(dev)
+              for n, a in inp.extra["descale_bh"].items()}
+    else:
+        ds = dict(inp.extra["descale"], **over)
     cu = None if inp.cu_seqlens is None else inp.cu_seqlens.to(dev)
     o, lse = fa.attention_forward_fp8(inp.q.to(dev), inp.k.to(dev), inp.v.to(dev), ds["q"], ds["k"], ds["v"],
                                       causal=inp.causal, scale=inp.scale, cu_seqlens=cu,
@@ -161,3 +168,28 @@ def test_fp8_full_size_sampled_rows(fa):
                                                                              inp.T - 1]]))
     rows = np.unique(rows)
     _check(inp, o, lse, rows=rows)
+
+
+@pytest.mark.parametrize("varlen", [False, True])
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp8_per_head_descales(fa, causal, varlen):
+    """One descale per (sequence, head) (fa_fwd_fp8_per_head): heads and sequences drawn at magnitudes
+    a factor 2 apart, each quantised with its own amax/448, so a kernel that used one descale for all
+    would be far off; checked under the same e4m3 bounds against the oracle on the real values."""
+    H, d = 3, 128
+    seqlens = [200, 0, 513, 64] if varlen else [384, 384]
+    B, N = len(seqlens), max(seqlens)
+    cu = workloads.cu_from_lengths(seqlens) if varlen else None
+    segs = [(int(sum(seqlens[:b])), L) for b, L in enumerate(seqlens)]
+    T = sum(seqlens)
+    g = torch.Generator().manual_seed(61 + int(causal) + 2 * int(varlen))
+    mag = torch.ones(T, H, 1)
+    for b, (s0, L) in enumerate(segs):
+        mag[s0:s0 + L] = (2.0 ** torch.arange(H, dtype=torch.float32))[None, :, None] * (b + 1)
+    q8, dq = workloads.quantize_e4m3_per_head(torch.randn(T, H, d, generator=g) * mag, segs)
+    k8, dk = workloads.quantize_e4m3_per_head(torch.randn(T, H, d, generator=g) * mag, segs)
+    v8, dv = workloads.quantize_e4m3_per_head(torch.randn(T, H, d, generator=g) * mag, segs)
+    inp = workloads.AttnInputs(q8, k8, v8, None, cu, seqlens, B, H, N, d, 0.25 / math.sqrt(d), causal, "e4m3",
+                               "per_head", {"descale_bh": {"q": dq, "k": dk, "v": dv}})
+    o, lse = _run(fa, inp)
+    _check(inp, o, lse)

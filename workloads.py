@@ -103,9 +103,32 @@ def _randn_e4m3(g: torch.Generator, shape):
     return (x / descale).to(torch.float8_e4m3fn), descale
 
 
-def real_values(t: torch.Tensor, descale: float = 1.0) -> np.ndarray:
-    """The values a stored tensor stands for, as float64 (e4m3 or 16-bit storage times its descale)."""
-    return t.detach().cpu().to(torch.float64).numpy() * float(descale)
+def real_values(t: torch.Tensor, descale=1.0, segments=None) -> np.ndarray:
+    """The values a stored tensor stands for, as float64 (e4m3 or 16-bit storage times its descale):
+    ``descale`` a float, or a [B, H] array with ``segments`` the (start, length) of each sequence."""
+    x = t.detach().cpu().to(torch.float64).numpy()
+    if segments is None:
+        return x * float(descale)
+    ds = np.asarray(descale, dtype=np.float64)
+    out = x.copy()
+    for b, (s0, L) in enumerate(segments):
+        out[s0:s0 + L] *= ds[b][None, :, None]
+    return out
+
+
+def quantize_e4m3_per_head(x: torch.Tensor, segments):
+    """fp32 [T, H, d] → (e4m3 tensor, fp32 descales [B, H]): each (sequence, head) divided by its own
+    amax/448 (rounded to fp32) and rounded to e4m3."""
+    T, H, _ = x.shape
+    ds = np.ones((len(segments), H), dtype=np.float32)
+    y = torch.empty_like(x)
+    for b, (s0, L) in enumerate(segments):
+        if L == 0:
+            continue
+        amax = x[s0:s0 + L].abs().amax(dim=(0, 2))                      # [H]
+        ds[b] = (amax / E4M3_MAX).numpy().astype(np.float32)
+        y[s0:s0 + L] = x[s0:s0 + L] / torch.from_numpy(ds[b])[None, :, None]
+    return y.to(torch.float8_e4m3fn), ds
 
 
 def varlen_lengths(nseq: int, lmin: int, lmax: int, seed: int) -> List[int]:
