@@ -933,6 +933,13 @@ def main():
     ap.add_argument("--dropout", type=float, default=0.0,
                     help="dropout probability on P (attention workloads; 0 = the plain step)")
     args = ap.parse_args()
+    if not (0.0 <= args.dropout < 1.0):
+        ap.error("--dropout must be in [0, 1)")
+    if args.dropout > 0.0:
+        import workloads
+        spec = workloads.WORKLOADS.get(args.workload)
+        if spec is None or spec["dtype"] == "e4m3":
+            ap.error("--dropout applies to the 16-bit attention workloads only (not decode or e4m3)")
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     args.steps = max(1, args.steps)
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -98,3 +98,12 @@ def test_reference_arm_other_ranks_exit_quietly():
                         "tiny_d64", "--steps", "1", "--warmup", "3"], capture_output=True, text=True, env=env,
                        timeout=300)
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+@pytest.mark.parametrize("extra", [["--workload", "decode_b16_kv8k", "--dropout", "0.1"],
+                                   ["--workload", "causal_n8k_d128_fp8", "--dropout", "0.1"],
+                                   ["--dropout", "1.5"]])
+def test_bench_rejects_dropout_where_it_does_not_apply(extra):
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference"] + extra,
+                       capture_output=True, text=True, timeout=120)
+    assert r.returncode == 2 and "--dropout" in r.stderr and r.stdout.strip() == ""
