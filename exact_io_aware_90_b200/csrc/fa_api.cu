@@ -171,11 +171,11 @@ static int bwd_main_impl(const void* q, const void* k, const void* v, const floa
   BwdArgs a;
   std::memset(&a, 0, sizeof(a));
   if ((st = set_workspace(&a, workspace, workspace_bytes_, pb.T, H, d)) != FA_OK) return st;
-  // Q and dO stream in tiles of 64 rows at d = 128 and 128 rows at d = 64; K and V in 128-row tiles
-  const int bq = (d == 128) ? 64 : 128;
+  // Q and dO stream in tiles of bq rows (the main kernel's query step); K and V in 128-row tiles
+  const int bq = bwd_q_tile_rows(d, dropout);
   if (!encode_tmap(&a.tm_q, q, pb.T, H, d, pb.bf16, bq) || !encode_tmap(&a.tm_k, k, pb.T, H, d, pb.bf16, 128) ||
       !encode_tmap(&a.tm_v, v, pb.T, H, d, pb.bf16, 128) || !encode_tmap(&a.tm_do, dO, pb.T, H, d, pb.bf16, bq) ||
-      !encode_tmap_f32(&a.tm_dq, a.dq_acc, pb.T, H, d, bq))
+      !encode_tmap_f32(&a.tm_dq, a.dq_acc, pb.T, H, d, bwd_dq_box_rows(d, dropout)))
     return FA_ERR_UNSUPPORTED;
   a.q = q;
   a.k = k;

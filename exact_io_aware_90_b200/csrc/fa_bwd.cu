@@ -746,6 +746,514 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
 }
 
+// ============================================================================ main kernel at d = 128, 128-query steps
+//
+// Same work unit and equations as fa_bwd_main_kernel, but every Q step covers 128 query rows, so the
+// score, dP, dV, dK and dQ products are all 128 × 128 × 128 (N = 128: at N = 64 the tensor core is
+// starved by its shared-memory operand reads).  Two compute warpgroups form Pᵀ and dSᵀ concurrently,
+// one per 64-query half of the step (thread = key row, as before).  Tensor memory cannot hold Sᵀ and
+// dPᵀ of such a step beside dK and dV (128 columns each) plus a dQ partial, so columns are reused
+// within the step:
+//   [0, 128)    Sᵀ; once both halves are read, Pᵀ is packed into [0, 64) (half a in [32a, 32a + 32))
+//               and later dSᵀ into [64, 128) (half a in [64 + 32a, ...))
+//   [128, 256)  dPᵀ; once both halves are read, dQᵀ = Kᵀ dSᵀ [128 features × 128 queries]
+//   [256, 384)  dK,  [384, 512)  dV
+// The two warpgroups tell each other "my half of Sᵀ is in registers" through an mbarrier before
+// packing over the other half's columns.  MMA issue order per step i (one thread; tcgen05 MMAs of one
+// thread run in issue order, so each product below has read its tensor-memory operand before a later
+// one overwrites it):
+//   dV(0) after Pᵀ(0), dV(1) after Pᵀ(1); dK after dSᵀ; Sᵀ(i+1) right behind it (it depends on no
+//   read-out); dQᵀ; dPᵀ(i+1) once the dQ warpgroup has read dQᵀ out of [128, 256).
+// The dQ partial goes from tensor memory to the fp32 accumulator through shared memory: each warp of
+// the dQ warpgroup stages its 32 features × 32 queries as one TMA box (two boxes per warp, used in
+// turn) and adds it into the accumulator with a TMA reduce-add (per-thread red.global.add of the same
+// data measured far slower).
+constexpr int kBwd128Threads = 512;  // 4 warpgroups
+
+struct Bq128 {
+  static constexpr int D = 128, BQ = 128;
+  static constexpr uint32_t CHUNK = 128 * 128;  // [128 rows × 64 features], 128-byte swizzle
+  static constexpr uint32_t TILE = 2 * CHUNK;   // [128 rows × 128 features]
+  // tensor memory columns
+  static constexpr uint32_t T_S = 0, T_P = 0, T_DS = 64, T_DP = 128, T_DQ = 128, T_DK = 256, T_DV = 384;
+  // barriers
+  static constexpr int B_KV = 0;
+  static constexpr int B_QFULL = 1;     // [2] Q tile of stage s landed
+  static constexpr int B_QEMPTY = 3;    // [2] Q tile and row terms of stage s no longer read
+  static constexpr int B_ROWFULL = 5;   // [2] −LSE·log2 e and −D of stage s written (32 arrivals)
+  static constexpr int B_DOFULL = 7;
+  static constexpr int B_DOEMPTY = 8;
+  static constexpr int B_SFULL = 9;
+  static constexpr int B_DPFULL = 10;
+  static constexpr int B_SREAD = 11;    // both halves of Sᵀ in registers (256 arrivals)
+  static constexpr int B_PREADY = 12;   // [2] half a of Pᵀ in tensor memory (128 arrivals)
+  static constexpr int B_DSREADY = 14;  // [2] half a of dSᵀ in tensor and shared memory, its dPᵀ read (128 arrivals)
+  static constexpr int B_DQFULL = 16;
+  static constexpr int B_DQFREE = 17;   // dQᵀ read out of [128, 256) (128 arrivals)
+  static constexpr int B_DKV = 18;
+  static constexpr int B_DRAIN = 19;
+  static constexpr int NBARS = 20;
+  // shared memory: K, V resident; Q double-buffered; dO single (its next tile loads once dV has read
+  // it, well before the next dPᵀ); dSᵀ as two [128 keys × 64 queries] chunks (B operand of dQᵀ)
+  static constexpr uint32_t OFF_K = 0;
+  static constexpr uint32_t OFF_V = TILE;
+  static constexpr uint32_t OFF_Q = 2 * TILE;
+  static constexpr uint32_t OFF_DO = 4 * TILE;
+  static constexpr uint32_t OFF_DS = 5 * TILE;
+  static constexpr uint32_t OFF_DQS = 6 * TILE;  // dQ staging: per dQ warp two boxes [32 queries × 32 fp32]
+  static constexpr uint32_t DQ_BOX = 32 * 128;
+  static constexpr uint32_t OFF_ROW = OFF_DQS + 8 * DQ_BOX;  // per stage: −LSE·log2 e [128], −D [128] (fp32)
+  static constexpr uint32_t OFF_BAR = OFF_ROW + 2 * 2 * BQ * 4;
+  static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
+  // no alignment slack: the dynamic shared memory is declared 1024-byte aligned (checked at run time)
+  static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  // registers per thread after setmaxnreg: the block is launched at 128 (512 threads), so the four
+  // warpgroups' shares must add up to at most 4 × 128
+  static constexpr uint32_t REGS_LAUNCH = 128;  // 65536 registers / 512 threads (ptxas reports 128)
+  static constexpr uint32_t REGS_CMP = 152, REGS_DQ = 152, REGS_IO = 56;
+  static_assert(2 * REGS_CMP + REGS_DQ + REGS_IO <= 4 * REGS_LAUNCH, "register budget");
+};
+
+// dQᵀ = Kᵀ dSᵀ: A = K MN-major (M = 128 features), B = dSᵀ MN-major (N = 128 queries, two 64-query
+// chunks 16 KB apart), K dim = the 128 keys (+2 KB per 16 keys in both operands).
+template <uint32_t IDESC>
+__device__ __forceinline__ void bwd_issue_dq128(uint32_t d_tmem, uint64_t da, uint64_t db) {
+  da = opaque64(da);
+  db = opaque64(db);
+#pragma unroll
+  for (int kk = 0; kk < kBK / 16; ++kk) mma_ss(d_tmem, da + ((kk * 2048) >> 4), db + ((kk * 2048) >> 4), IDESC, kk > 0 ? 1u : 0u);
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(kBwd128Threads, 1)
+    fa_bwd_main_q128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                            const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                            const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
+  using C = Bq128;
+  constexpr int BQ = C::BQ;
+  constexpr uint32_t IDESC_ST = idesc_f16(BF16, kBK, BQ, false, false);    // Sᵀ = K Qᵀ, dPᵀ = V dOᵀ
+  constexpr uint32_t IDESC_DKV = idesc_f16(BF16, kBK, C::D, false, true);  // dV += Pᵀ dO, dK += dSᵀ Q
+  constexpr uint32_t IDESC_DQ = idesc_f16(BF16, C::D, BQ, true, true);     // dQᵀ = Kᵀ dSᵀ
+
+  extern __shared__ __align__(1024) uint8_t smem_aligned[];
+  uint8_t* smem = smem_aligned;
+  const uint32_t s_base = smem_u32(smem);
+  if ((s_base & 1023u) != 0u) {  // the 128-byte-swizzled tiles need 1024-byte alignment
+    if (threadIdx.x == 0) record_status(2);
+    return;
+  }
+  const uint32_t sK = s_base + C::OFF_K;
+  const uint32_t sV = s_base + C::OFF_V;
+  const uint32_t sQ = s_base + C::OFF_Q;
+  const uint32_t sDO = s_base + C::OFF_DO;
+  const uint32_t sDS = s_base + C::OFF_DS;
+  float* row_buf = reinterpret_cast<float*>(smem + C::OFF_ROW);
+  const uint32_t bar0 = s_base + C::OFF_BAR;
+  auto bar = [&](int i) -> uint32_t { return bar0 + 8u * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  int* abort_flag = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work unit: heads in groups, heaviest key tiles (the first ones when causal) first
+  const int BH = p.B * p.H;
+  const int nkb = p.num_kblocks;
+  const int G = p.heads_group;
+  const int unit = blockIdx.x;
+  const int group = unit / (G * nkb);
+  const int g_heads = min(G, BH - group * G);
+  const int r = unit - group * G * nkb;
+  const int kb = r / g_heads;
+  const int bh = group * G + r % g_heads;
+  const int b = bh / p.H;
+  const int h = bh - b * p.H;
+
+  int tok0, L;
+  if (p.cu_seqlens != nullptr) {
+    tok0 = __ldg(p.cu_seqlens + b);
+    const int end = __ldg(p.cu_seqlens + b + 1);
+    L = end - tok0;
+    if (tok0 < 0 || L < 0 || end > p.T || L > p.N) {
+      if (threadIdx.x == 0) record_status(1);
+      return;
+    }
+  } else {
+    tok0 = b * p.N;
+    L = p.N;
+  }
+  const int k0 = kb * kBK;
+  if (k0 >= L) return;
+  const int nq_all = (L + BQ - 1) / BQ;
+  const int i_begin = p.causal ? k0 / BQ : 0;
+  const int n_it = nq_all - i_begin;  // ≥ 1
+
+  if (warp == 13) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 0) {
+    mbar_init(bar(C::B_KV), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(C::B_QFULL + s), 1);
+      mbar_init(bar(C::B_QEMPTY + s), 1);
+      mbar_init(bar(C::B_ROWFULL + s), 32);
+      mbar_init(bar(C::B_PREADY + s), 128);
+      mbar_init(bar(C::B_DSREADY + s), 128);
+    }
+    mbar_init(bar(C::B_DOFULL), 1);
+    mbar_init(bar(C::B_DOEMPTY), 1);
+    mbar_init(bar(C::B_SFULL), 1);
+    mbar_init(bar(C::B_DPFULL), 1);
+    mbar_init(bar(C::B_SREAD), 256);
+    mbar_init(bar(C::B_DQFULL), 1);
+    mbar_init(bar(C::B_DQFREE), 128);
+    mbar_init(bar(C::B_DKV), 1);
+    mbar_init(bar(C::B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 12 && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    prefetch_tmap(&tm_do);
+    prefetch_tmap(&tm_dq);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Watchdog wd{abort_flag, p.timeout_ns};
+
+  if (warp >= 12) {
+    regs_set<C::REGS_IO, C::REGS_LAUNCH>();
+    if (warp == 12) {
+      // ================================================================ TMA producer (+ row terms)
+      const uint64_t pol_kv = l2_policy_evict_first();
+      const uint64_t pol_q = l2_policy_evict_last();
+      if (elect_one()) {
+        mbar_arrive_expect_tx(bar(C::B_KV), 2 * C::TILE);
+        for (int c = 0; c < 2; ++c) {
+          tma_load_3d(sK + c * C::CHUNK, &tm_k, bar(C::B_KV), c * 64, h, tok0 + k0, pol_kv);
+          tma_load_3d(sV + c * C::CHUNK, &tm_v, bar(C::B_KV), c * 64, h, tok0 + k0, pol_kv);
+        }
+      }
+      __syncwarp();
+      int q_issued = 0, do_issued = 0;
+      const float LOG2E = 1.4426950408889634f;
+      for (int it = 0; it < n_it; ++it) {
+        const int s = it & 1;
+        const int i0 = (i_begin + it) * BQ;
+        if (it >= 2 && !warp_wait_b(bar(C::B_QEMPTY + s), ((it >> 1) - 1) & 1, wd)) break;
+        if (elect_one()) {
+          mbar_arrive_expect_tx(bar(C::B_QFULL + s), C::TILE);
+          for (int c = 0; c < 2; ++c)
+            tma_load_3d(sQ + s * C::TILE + c * C::CHUNK, &tm_q, bar(C::B_QFULL + s), c * 64, h, tok0 + i0, pol_q);
+        }
+        __syncwarp();
+        q_issued = it + 1;
+        // −LSE·log2 e and −D of the step's query rows; rows past the sequence get 0
+        float* lse_s = row_buf + s * 2 * BQ;
+        float* del_s = lse_s + BQ;
+        for (int q = lane; q < BQ; q += 32) {
+          const int qrow = i0 + q;
+          const bool v = qrow < L;
+          lse_s[q] = v ? -__ldg(p.lse + (size_t)(tok0 + qrow) * p.H + h) * LOG2E : 0.f;
+          del_s[q] = v ? -__ldg(p.delta + (size_t)(tok0 + qrow) * p.H + h) : 0.f;
+        }
+        mbar_arrive(bar(C::B_ROWFULL + s));  // release: the stores above are visible to waiters
+        // dO of this step, once dV of the previous step has read the single buffer
+        if (it >= 1 && !warp_wait_b(bar(C::B_DOEMPTY), (it - 1) & 1, wd)) break;
+        if (elect_one()) {
+          mbar_arrive_expect_tx(bar(C::B_DOFULL), C::TILE);
+          for (int c = 0; c < 2; ++c)
+            tma_load_3d(sDO + c * C::CHUNK, &tm_do, bar(C::B_DOFULL), c * 64, h, tok0 + i0, pol_q);
+        }
+        __syncwarp();
+        do_issued = it + 1;
+      }
+      if (elect_one()) {
+        drain_wait_b(bar(C::B_KV), 0, p.timeout_ns);
+        for (int it = max(0, q_issued - 2); it < q_issued; ++it)
+          drain_wait_b(bar(C::B_QFULL + (it & 1)), (it >> 1) & 1, p.timeout_ns);
+        if (do_issued > 0) drain_wait_b(bar(C::B_DOFULL), (do_issued - 1) & 1, p.timeout_ns);
+      }
+      __syncwarp();
+    } else if (warp == 13) {
+      // ================================================================ MMA issuer
+      const uint32_t tS = tmem + C::T_S, tP = tmem + C::T_P, tDQ = tmem + C::T_DQ, tDP = tmem + C::T_DP;
+      const uint32_t tDS = tmem + C::T_DS, tDK = tmem + C::T_DK, tDV = tmem + C::T_DV;
+      const uint64_t dK_kmaj = sdesc_sw128(sK, 16, 1024), dV_kmaj = sdesc_sw128(sV, 16, 1024);
+      const uint64_t dQ_kmaj = sdesc_sw128(sQ, 16, 1024), dDO_kmaj = sdesc_sw128(sDO, 16, 1024);
+      const uint64_t dQ_mn = sdesc_sw128(sQ, C::CHUNK, 1024), dDO_mn = sdesc_sw128(sDO, C::CHUNK, 1024);
+      const uint64_t dKt_mn = sdesc_sw128(sK, C::CHUNK, 1024);  // Kᵀ: MN-major A of dQᵀ (features contiguous)
+      const uint64_t dDS_mn = sdesc_sw128(sDS, C::CHUNK, 1024);  // dSᵀ: MN-major B of dQᵀ (queries contiguous)
+      constexpr uint32_t TILE16 = C::TILE >> 4;
+      constexpr uint32_t HALF16 = (64 * 128) >> 4;  // 64 rows of a chunk: query half 1 of Q / dO
+      bool ok = warp_wait_b(bar(C::B_KV), 0, wd) && warp_wait_b(bar(C::B_QFULL + 0), 0, wd) &&
+                warp_wait_b(bar(C::B_DOFULL), 0, wd);
+      if (ok) {
+        tc_fence_after();
+        if (elect_one()) {
+          bwd_issue_kt<C::D, BQ, IDESC_ST>(tS, dK_kmaj, dQ_kmaj);
+          tc_commit(bar(C::B_SFULL));
+          bwd_issue_kt<C::D, BQ, IDESC_ST>(tDP, dV_kmaj, dDO_kmaj);
+          tc_commit(bar(C::B_DPFULL));
+        }
+        __syncwarp();
+      }
+      for (int it = 0; ok && it < n_it; ++it) {
+        const int s = it & 1;
+        const bool more = it + 1 < n_it;
+        const int s1 = (it + 1) & 1;
+        // dV += Pᵀ(a) dO(a), as each half of Pᵀ is formed
+        if (!warp_wait_b(bar(C::B_PREADY + 0), it & 1, wd)) break;
+        tc_fence_after();
+        if (elect_one()) bwd_issue_acc<64, IDESC_DKV>(tDV, tP, dDO_mn, it > 0 ? 1u : 0u);
+        __syncwarp();
+        if (!warp_wait_b(bar(C::B_PREADY + 1), it & 1, wd)) break;
+        tc_fence_after();
+        if (elect_one()) {
+          bwd_issue_acc<64, IDESC_DKV>(tDV, tP + 32u, dDO_mn + HALF16, 1u);
+          tc_commit(bar(C::B_DOEMPTY));  // dO of this step is read by no later MMA
+        }
+        __syncwarp();
+        // dK += dSᵀ Q once both halves of dSᵀ are formed, then Sᵀ of the next step over [0, 128) right
+        // behind it (Pᵀ and dSᵀ there are read by the dV and dK MMAs, which run first)
+        if (!warp_wait_b(bar(C::B_DSREADY + 0), it & 1, wd) || !warp_wait_b(bar(C::B_DSREADY + 1), it & 1, wd)) break;
+        tc_fence_after();
+        if (elect_one()) bwd_issue_acc<BQ, IDESC_DKV>(tDK, tDS, dQ_mn + s * TILE16, it > 0 ? 1u : 0u);
+        __syncwarp();
+        if (more) {
+          if (!warp_wait_b(bar(C::B_QFULL + s1), ((it + 1) >> 1) & 1, wd)) break;
+          tc_fence_after();
+          if (elect_one()) {
+            bwd_issue_kt<C::D, BQ, IDESC_ST>(tS, dK_kmaj, dQ_kmaj + s1 * TILE16);
+            tc_commit(bar(C::B_SFULL));
+          }
+          __syncwarp();
+        }
+        // dQᵀ = Kᵀ dSᵀ over [128, 256): both halves of dPᵀ have been read out (dSᵀ ready)
+        if (elect_one()) {
+          bwd_issue_dq128<IDESC_DQ>(tDQ, dKt_mn, dDS_mn);
+          tc_commit(bar(C::B_DQFULL));
+          tc_commit(bar(C::B_QEMPTY + s));  // Q and row terms of this step no longer read
+        }
+        __syncwarp();
+        // dPᵀ of the next step over [128, 256) once dQᵀ has been read out
+        if (more) {
+          if (!warp_wait_b(bar(C::B_DQFREE), it & 1, wd) || !warp_wait_b(bar(C::B_DOFULL), (it + 1) & 1, wd))
+            break;
+          tc_fence_after();
+          if (elect_one()) {
+            bwd_issue_kt<C::D, BQ, IDESC_ST>(tDP, dV_kmaj, dDO_kmaj);
+            tc_commit(bar(C::B_DPFULL));
+          }
+          __syncwarp();
+        }
+      }
+      if (elect_one()) {
+        tc_commit(bar(C::B_DKV));
+        tc_commit(bar(C::B_DRAIN));
+        drain_wait_b(bar(C::B_DRAIN), 0, p.timeout_ns);
+      }
+      __syncwarp();
+    }
+  } else if (warp < 8) {
+    // ================================================================ Pᵀ / dSᵀ warpgroups (thread = key row)
+    // warpgroup a forms query half a (64 queries) of each step
+    regs_set<C::REGS_CMP, C::REGS_LAUNCH>();
+    const int a = warp >> 2;
+    const int quarter = warp & 3;
+    const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
+    const uint32_t tS = tmem + lane_off + C::T_S + 64u * a;    // this half of Sᵀ
+    const uint32_t tP = tmem + lane_off + C::T_P + 32u * a;    // this half of Pᵀ (packed)
+    const uint32_t tDP = tmem + lane_off + C::T_DP + 64u * a;  // this half of dPᵀ
+    const uint32_t tDS = tmem + lane_off + C::T_DS + 32u * a;  // this half of dSᵀ (packed, over Sᵀ)
+    const uint32_t tDV = tmem + lane_off + C::T_DV + 64u * a;  // dV columns this warpgroup writes out
+    const int kr = 32 * quarter + lane;  // key row within the tile
+    const int key = k0 + kr;             // position in the sequence
+    const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
+    uint8_t* ds_row = smem + C::OFF_DS + a * C::CHUNK + kr * 128;
+    bool ok = true;
+    for (int it = 0; it < n_it; ++it) {
+      const int i0 = (i_begin + it) * BQ + 64 * a;  // first query of this half
+      const int s = it & 1;
+      if (!warp_wait_b(bar(C::B_ROWFULL + s), (it >> 1) & 1, wd)) { ok = false; break; }
+      const float* lse_h = row_buf + s * 2 * BQ + 64 * a;
+      const float* del_h = lse_h + BQ;
+      // visible queries for this key: q >= key (causal) and q < L; key < L
+      const int q_lo = p.causal ? key - i0 : 0;  // first visible column of the half
+      const int q_hi = (key < L) ? L - i0 : -1;  // one past the last visible column
+      const bool full = __all_sync(0xffffffffu, q_lo <= 0 && q_hi >= 64);
+      // ---- Pᵀ = 2^(c·Sᵀ − LSE·log2 e), masked
+      if (!warp_wait_b(bar(C::B_SFULL), it & 1, wd)) { ok = false; break; }
+      tc_fence_after();
+      // Pᵀ is kept in registers only in its packed 16-bit form (the values the dV product uses), which
+      // leaves registers for the dQ warpgroup to take its whole partial out of tensor memory at once
+      uint32_t pk[32];
+      {
+        uint32_t sr[64];
+        tmem_ld64(tS, sr);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar(C::B_SREAD));
+        float pt[64];
+#pragma unroll
+        for (int i = 0; i < 64; i += 2) {
+          const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), c2,
+                                      make_float2(lse_h[i], lse_h[i + 1]));
+          pt[i] = ex2(x.x);
+          pt[i + 1] = ex2(x.y);
+        }
+        if (!full) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) pt[i] = (i >= q_lo && i < q_hi) ? pt[i] : 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) pk[i] = pack2<BF16>(pt[2 * i], pt[2 * i + 1]);
+      }
+      // packed over [32a, 32a + 32): for a = 1 those are Sᵀ columns of half 0, so both halves must have
+      // been read first
+      if (!warp_wait_b(bar(C::B_SREAD), it & 1, wd)) { ok = false; break; }
+      tc_fence_after();
+      tmem_st32(tP, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(C::B_PREADY + a));
+      // ---- dSᵀ = Pᵀ ∘ (dPᵀ − D)
+      if (!warp_wait_b(bar(C::B_DPFULL), it & 1, wd)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t dsk[32];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        uint32_t dr[32];
+        tmem_ld32(tDP + 32u * q, dr);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int col = 32 * q + 2 * i;
+          const float2 dpv = make_float2(__uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1]));
+          const float2 dd = __fadd2_rn(dpv, make_float2(del_h[col], del_h[col + 1]));
+          const float2 ds = __fmul2_rn(unpack2<BF16>(pk[col >> 1]), dd);
+          dsk[16 * q + i] = pack2<BF16>(ds.x, ds.y);
+        }
+      }
+      // into shared-memory chunk a as a 128-byte swizzled row (B operand of dQᵀ), and packed into tensor
+      // memory over Sᵀ columns both warpgroups have read (A operand of dK)
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        *reinterpret_cast<uint4*>(ds_row + ((j ^ (kr & 7)) << 4)) =
+            make_uint4(dsk[4 * j], dsk[4 * j + 1], dsk[4 * j + 2], dsk[4 * j + 3]);
+      fence_proxy_async_smem();
+      tmem_st32(tDS, dsk);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(C::B_DSREADY + a));
+    }
+    // ---- epilogue: dV rows of this tile, columns [64a, 64a + 64)
+    if (ok && warp_wait_b(bar(C::B_DKV), 0, wd)) {
+      tc_fence_after();
+      const bool valid = key < L;
+      uint8_t* dst = reinterpret_cast<uint8_t*>(p.dv) +
+                     (((size_t)(tok0 + (valid ? key : 0)) * p.H + h) * C::D + 64 * a) * 2;
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        uint32_t r32[32];
+        tmem_ld32(tDV + 32u * q, r32);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[i] = pack2<BF16>(__uint_as_float(r32[2 * i]), __uint_as_float(r32[2 * i + 1]));
+        if (valid) {
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            st_global_v4(dst + q * 64 + v4 * 16, pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ================================================================ dQ warpgroup (warps 8-11; thread = feature)
+    regs_set<C::REGS_DQ, C::REGS_LAUNCH>();
+    const int quarter = warp & 3;
+    const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
+    const uint32_t tDQ = tmem + lane_off + C::T_DQ;
+    const uint32_t tDK = tmem + lane_off + C::T_DK;
+    // this warp's two staging boxes: row q = query, 32 fp32 features in 16-byte chunks swizzled by q mod 8
+    const uint32_t box_base = s_base + C::OFF_DQS + quarter * 2 * C::DQ_BOX;
+    bool ok = true;
+    uint32_t pieces = 0;  // boxes staged so far (box = pieces mod 2)
+    for (int it = 0; it < n_it; ++it) {
+      const int i0 = (i_begin + it) * BQ;
+      if (!warp_wait_b(bar(C::B_DQFULL), it & 1, wd)) { ok = false; break; }
+      tc_fence_after();
+      // the whole partial into registers (lane = feature 32·quarter + lane, columns = queries), so the
+      // next dPᵀ may overwrite [128, 256) at once; staging and the reduce-adds follow at their own pace
+      uint32_t qr[128];
+      tmem_ld64(tDQ, reinterpret_cast<uint32_t(&)[64]>(qr[0]));
+      tmem_ld64(tDQ + 64u, reinterpret_cast<uint32_t(&)[64]>(qr[64]));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar(C::B_DQFREE));
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int q0 = i0 + 32 * c;
+        if (q0 >= L) break;  // the rest of the step lies past the sequence: nothing to add
+        const uint32_t bx = box_base + (pieces & 1u) * C::DQ_BOX;
+        // the box may be rewritten once the reduce issued from it two pieces ago has read it
+        if (lane == 0) bulk_wait_group_read<1>();
+        __syncwarp();
+#pragma unroll
+        for (int q = 0; q < 32; ++q)
+          st_shared_f32(bx + q * 128 + (((lane >> 2) ^ (q & 7)) << 4) + ((lane & 3) << 2), qr[32 * c + q]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        // rows past the sequence hold exact zeros (P is 0 there); rows past T are clipped by the TMA unit
+        if (lane == 0) {
+          tma_reduce_add_3d(&tm_dq, bx, 32 * quarter, h, tok0 + q0);
+          bulk_commit_group();
+        }
+        __syncwarp();
+        ++pieces;
+      }
+    }
+    if (lane == 0) bulk_wait_group_all();  // every reduce performed before the kernel ends
+    // ---- epilogue: dK rows (× scale)
+    if (ok && warp_wait_b(bar(C::B_DKV), 0, wd)) {
+      tc_fence_after();
+      const int key = k0 + 32 * quarter + lane;
+      const bool valid = key < L;
+      uint8_t* dst = reinterpret_cast<uint8_t*>(p.dk) + (((size_t)(tok0 + (valid ? key : 0)) * p.H + h) * C::D) * 2;
+#pragma unroll
+      for (int q = 0; q < C::D / 32; ++q) {
+        uint32_t r32[32];
+        tmem_ld32(tDK + 32u * q, r32);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pk[i] = pack2<BF16>(__uint_as_float(r32[2 * i]) * p.scale, __uint_as_float(r32[2 * i + 1]) * p.scale);
+        if (valid) {
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            st_global_v4(dst + q * 64 + v4 * 16, pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+        }
+      }
+    }
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 13) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 // ============================================================================ launchers
 
 static int num_sms() {
@@ -824,12 +1332,50 @@ static cudaError_t launch_main_t(const Problem& pb, const BwdArgs& a, cudaStream
   return cudaPeekAtLastError();
 }
 
+template <bool BF16>
+static cudaError_t launch_main_q128_t(const Problem& pb, const BwdArgs& a, cudaStream_t stream) {
+  static std::atomic<unsigned long long> configured{0};  // per instantiation, one bit per device
+  auto kern = fa_bwd_main_q128_kernel<BF16>;
+  if (cudaError_t e = set_smem_once(configured, reinterpret_cast<const void*>(kern), Bq128::SMEM_BYTES);
+      e != cudaSuccess)
+    return e;
+  BwdParams p;
+  p.lse = a.lse;
+  p.delta = a.delta;
+  p.dq_acc = a.dq_acc;
+  p.dk = a.dk;
+  p.dv = a.dv;
+  p.cu_seqlens = pb.cu_seqlens;
+  p.B = pb.B;
+  p.H = pb.H;
+  p.N = pb.N;
+  p.T = pb.T;
+  p.causal = pb.causal;
+  p.num_kblocks = (pb.N + kBK - 1) / kBK;
+  p.heads_group = 8;
+  p.scale = pb.scale;
+  p.scale_log2 = pb.scale * 1.4426950408889634f;
+  p.timeout_ns = pb.timeout_ns;
+  p.drop = pb.drop;
+  const long long units = (long long)pb.B * pb.H * p.num_kblocks;
+  kern<<<dim3((unsigned)units), dim3(kBwd128Threads), Bq128::SMEM_BYTES, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do,
+                                                                                     a.tm_dq, p);
+  return cudaPeekAtLastError();
+}
+
 template <bool DROP>
 static cudaError_t launch_main_d(const Problem& pb, const BwdArgs& a, cudaStream_t stream) {
-  if (pb.d == 128)
+  if (pb.d == 128) {
+    if constexpr (!DROP) return pb.bf16 ? launch_main_q128_t<true>(pb, a, stream) : launch_main_q128_t<false>(pb, a, stream);
     return pb.bf16 ? launch_main_t<128, true, DROP>(pb, a, stream) : launch_main_t<128, false, DROP>(pb, a, stream);
+  }
   return pb.bf16 ? launch_main_t<64, true, DROP>(pb, a, stream) : launch_main_t<64, false, DROP>(pb, a, stream);
 }
+
+// Rows per Q / dO tile the main kernel loads, and per box of its dQ reduce-adds (the host encodes the
+// tensor maps with these box heights).
+int bwd_q_tile_rows(int d, bool dropout) { return (d == 128 && dropout) ? 64 : 128; }
+int bwd_dq_box_rows(int d, bool dropout) { return d == 128 ? (dropout ? 64 : 32) : 128; }
 
 cudaError_t launch_bwd_main(const Problem& pb, const BwdArgs& a, cudaStream_t stream) {
   return pb.drop.t != 0u ? launch_main_d<true>(pb, a, stream) : launch_main_d<false>(pb, a, stream);

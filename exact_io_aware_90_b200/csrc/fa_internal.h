@@ -108,6 +108,8 @@ cudaError_t launch_accumulate(float* acc, const void* part, void* out, long long
 cudaError_t launch_decode(const Problem& pb, const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_bwd_pre(const Problem& pb, const BwdArgs& a, cudaStream_t stream);
 cudaError_t launch_bwd_main(const Problem& pb, const BwdArgs& a, cudaStream_t stream);
+int bwd_q_tile_rows(int d, bool dropout);
+int bwd_dq_box_rows(int d, bool dropout);
 cudaError_t launch_bwd_post(const Problem& pb, const BwdArgs& a, cudaStream_t stream);
 cudaError_t launch_watchdog_selftest(uint64_t timeout_ns, cudaStream_t stream);
 
