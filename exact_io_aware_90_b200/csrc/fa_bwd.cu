@@ -192,6 +192,11 @@ __device__ __forceinline__ bool warp_wait_b(uint32_t bar, uint32_t parity, const
   return __all_sync(0xffffffffu, ok);
 }
 
+// Warp-uniform non-blocking probe of one barrier phase.
+__device__ __forceinline__ bool warp_test_b(uint32_t bar, uint32_t parity) {
+  return __all_sync(0xffffffffu, mbar_test_wait(bar, parity));
+}
+
 // Products of one Q tile, issued by one elected lane.  Descriptor arguments
 // are pre-built bases; per 16-element K step only a constant start-address
 // offset (16-byte units) is added.
@@ -752,30 +757,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 // score, dP, dV, dK and dQ products are all 128 × 128 × 128 (N = 128: at N = 64 the tensor core is
 // starved by its shared-memory operand reads).  Two compute warpgroups form Pᵀ and dSᵀ concurrently,
 // one per 64-query half of the step (thread = key row, as before).  Tensor memory cannot hold Sᵀ and
-// dPᵀ of such a step beside dK and dV (128 columns each) plus a dQ partial, so columns are reused
-// within the step:
-//   [0, 128)    Sᵀ; once both halves are read, Pᵀ is packed into [0, 64) (half a in [32a, 32a + 32))
-//               and later dSᵀ into [64, 128) (half a in [64 + 32a, ...))
-//   [128, 256)  dPᵀ; once both halves are read, dQᵀ = Kᵀ dSᵀ [128 features × 128 queries]
+// dPᵀ of a step beside dK and dV (128 columns each) plus a dQ partial, so columns are reused:
+//   [0, 128)    Sᵀ(j); once both halves are in registers, dQᵀ(j − 1) = Kᵀ dSᵀ(j − 1) [128 features ×
+//               128 queries]; once that has been read out, Pᵀ(j) packed into [0, 64) (half a in
+//               [32a, 32a + 32))
+//   [128, 256)  dPᵀ(j); once both halves are in registers, dSᵀ(j) packed into [128, 192)
 //   [256, 384)  dK,  [384, 512)  dV
-// The two warpgroups tell each other "my half of Sᵀ is in registers" through an mbarrier before
-// packing over the other half's columns.  MMA issue order per step i (one thread; tcgen05 MMAs of one
-// thread run in issue order, so each product below has read its tensor-memory operand before a later
-// one overwrites it):
-//   dV(0) after Pᵀ(0), dV(1) after Pᵀ(1); dK after dSᵀ; Sᵀ(i+1) right behind it (it depends on no
-//   read-out); dQᵀ; dPᵀ(i+1) once the dQ warpgroup has read dQᵀ out of [128, 256).
-// The dQ partial goes from tensor memory to the fp32 accumulator through shared memory: each warp of
-// the dQ warpgroup stages its 32 features × 32 queries as one TMA box (two boxes per warp, used in
+// The two warpgroups tell each other "my half of Sᵀ (dPᵀ) is in registers" through an mbarrier before
+// anything is written over the other half's columns.  MMA issue order per step j (one thread; tcgen05
+// MMAs of one thread run in issue order, so each product has read its tensor-memory operand before a
+// later one overwrites it):
+//   dV(j) after Pᵀ(j); Sᵀ(j + 1) right behind it (so it is computed while dSᵀ(j) is formed); dK(j)
+//   after dSᵀ(j); dQᵀ(j) once Sᵀ(j + 1) has been read; dPᵀ(j + 1).
+// The dQ partial goes from tensor memory to the fp32 accumulator through shared memory: the dQ
+// warpgroup takes the whole partial into registers at once (so [0, 128) is released early), then each
+// of its warps stages 32 features × 32 queries at a time as one TMA box (two boxes per warp, used in
 // turn) and adds it into the accumulator with a TMA reduce-add (per-thread red.global.add of the same
 // data measured far slower).
 constexpr int kBwd128Threads = 512;  // 4 warpgroups
+// Column pairs i (of 32 per query half) with bit (i % 8) set take the FMA-pipe exp2 in unmasked halves.
+constexpr uint32_t kBwd128PolyMask = 0x00u;
 
 struct Bq128 {
   static constexpr int D = 128, BQ = 128;
   static constexpr uint32_t CHUNK = 128 * 128;  // [128 rows × 64 features], 128-byte swizzle
   static constexpr uint32_t TILE = 2 * CHUNK;   // [128 rows × 128 features]
   // tensor memory columns
-  static constexpr uint32_t T_S = 0, T_P = 0, T_DS = 64, T_DP = 128, T_DQ = 128, T_DK = 256, T_DV = 384;
+  static constexpr uint32_t T_S = 0, T_P = 0, T_DQ = 0, T_DP = 128, T_DS = 128, T_DK = 256, T_DV = 384;
   // barriers
   static constexpr int B_KV = 0;
   static constexpr int B_QFULL = 1;     // [2] Q tile of stage s landed
@@ -786,13 +794,14 @@ struct Bq128 {
   static constexpr int B_SFULL = 9;
   static constexpr int B_DPFULL = 10;
   static constexpr int B_SREAD = 11;    // both halves of Sᵀ in registers (256 arrivals)
-  static constexpr int B_PREADY = 12;   // [2] half a of Pᵀ in tensor memory (128 arrivals)
-  static constexpr int B_DSREADY = 14;  // [2] half a of dSᵀ in tensor and shared memory, its dPᵀ read (128 arrivals)
-  static constexpr int B_DQFULL = 16;
-  static constexpr int B_DQFREE = 17;   // dQᵀ read out of [128, 256) (128 arrivals)
-  static constexpr int B_DKV = 18;
-  static constexpr int B_DRAIN = 19;
-  static constexpr int NBARS = 20;
+  static constexpr int B_DPREAD = 12;   // both halves of dPᵀ in registers (256 arrivals)
+  static constexpr int B_PREADY = 13;   // [2] half a of Pᵀ in tensor memory (128 arrivals)
+  static constexpr int B_DSREADY = 15;  // [2] half a of dSᵀ in tensor and shared memory (128 arrivals)
+  static constexpr int B_DQFULL = 17;
+  static constexpr int B_DQFREE = 18;   // dQᵀ read out of [0, 128) (128 arrivals)
+  static constexpr int B_DKV = 19;
+  static constexpr int B_DRAIN = 20;
+  static constexpr int NBARS = 21;
   // shared memory: K, V resident; Q double-buffered; dO single (its next tile loads once dV has read
   // it, well before the next dPᵀ); dSᵀ as two [128 keys × 64 queries] chunks (B operand of dQᵀ)
   static constexpr uint32_t OFF_K = 0;
@@ -907,6 +916,7 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
     mbar_init(bar(C::B_SFULL), 1);
     mbar_init(bar(C::B_DPFULL), 1);
     mbar_init(bar(C::B_SREAD), 256);
+    mbar_init(bar(C::B_DPREAD), 256);
     mbar_init(bar(C::B_DQFULL), 1);
     mbar_init(bar(C::B_DQFREE), 128);
     mbar_init(bar(C::B_DKV), 1);
@@ -929,8 +939,27 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
 
   if (warp >= 12) {
     regs_set<C::REGS_IO, C::REGS_LAUNCH>();
-    if (warp == 12) {
-      // ================================================================ TMA producer (+ row terms)
+    if (warp == 14) {
+      // ================================================================ row terms
+      // −LSE·log2 e and −D of each step's query rows into the stage of its Q tile (rows past the
+      // sequence get 0).  A warp of its own: these strided loads would otherwise hold up the TMA issue.
+      const float LOG2E = 1.4426950408889634f;
+      for (int it = 0; it < n_it; ++it) {
+        const int s = it & 1;
+        const int i0 = (i_begin + it) * BQ;
+        if (it >= 2 && !warp_wait_b(bar(C::B_QEMPTY + s), ((it >> 1) - 1) & 1, wd)) break;
+        float* lse_s = row_buf + s * 2 * BQ;
+        float* del_s = lse_s + BQ;
+        for (int q = lane; q < BQ; q += 32) {
+          const int qrow = i0 + q;
+          const bool v = qrow < L;
+          lse_s[q] = v ? -__ldg(p.lse + (size_t)(tok0 + qrow) * p.H + h) * LOG2E : 0.f;
+          del_s[q] = v ? -__ldg(p.delta + (size_t)(tok0 + qrow) * p.H + h) : 0.f;
+        }
+        mbar_arrive(bar(C::B_ROWFULL + s));  // release: the stores above are visible to waiters
+      }
+    } else if (warp == 12) {
+      // ================================================================ TMA producer
       const uint64_t pol_kv = l2_policy_evict_first();
       const uint64_t pol_q = l2_policy_evict_last();
       if (elect_one()) {
@@ -942,7 +971,6 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
       }
       __syncwarp();
       int q_issued = 0, do_issued = 0;
-      const float LOG2E = 1.4426950408889634f;
       for (int it = 0; it < n_it; ++it) {
         const int s = it & 1;
         const int i0 = (i_begin + it) * BQ;
@@ -954,16 +982,6 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
         }
         __syncwarp();
         q_issued = it + 1;
-        // −LSE·log2 e and −D of the step's query rows; rows past the sequence get 0
-        float* lse_s = row_buf + s * 2 * BQ;
-        float* del_s = lse_s + BQ;
-        for (int q = lane; q < BQ; q += 32) {
-          const int qrow = i0 + q;
-          const bool v = qrow < L;
-          lse_s[q] = v ? -__ldg(p.lse + (size_t)(tok0 + qrow) * p.H + h) * LOG2E : 0.f;
-          del_s[q] = v ? -__ldg(p.delta + (size_t)(tok0 + qrow) * p.H + h) : 0.f;
-        }
-        mbar_arrive(bar(C::B_ROWFULL + s));  // release: the stores above are visible to waiters
         // dO of this step, once dV of the previous step has read the single buffer
         if (it >= 1 && !warp_wait_b(bar(C::B_DOEMPTY), (it - 1) & 1, wd)) break;
         if (elect_one()) {
@@ -1020,14 +1038,12 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
           tc_commit(bar(C::B_DOEMPTY));  // dO of this step is read by no later MMA
         }
         __syncwarp();
-        // dK += dSᵀ Q once both halves of dSᵀ are formed, then Sᵀ of the next step over [0, 128) right
-        // behind it (Pᵀ and dSᵀ there are read by the dV and dK MMAs, which run first)
-        if (!warp_wait_b(bar(C::B_DSREADY + 0), it & 1, wd) || !warp_wait_b(bar(C::B_DSREADY + 1), it & 1, wd)) break;
-        tc_fence_after();
-        if (elect_one()) bwd_issue_acc<BQ, IDESC_DKV>(tDK, tDS, dQ_mn + s * TILE16, it > 0 ? 1u : 0u);
-        __syncwarp();
+        // Sᵀ of the next step over [0, 128): Pᵀ there is read by the dV MMAs above, which run first, and
+        // dQᵀ of the previous step has been read out
         if (more) {
-          if (!warp_wait_b(bar(C::B_QFULL + s1), ((it + 1) >> 1) & 1, wd)) break;
+          if (!warp_wait_b(bar(C::B_QFULL + s1), ((it + 1) >> 1) & 1, wd) ||
+              (it > 0 && !warp_wait_b(bar(C::B_DQFREE), (it - 1) & 1, wd)))
+            break;
           tc_fence_after();
           if (elect_one()) {
             bwd_issue_kt<C::D, BQ, IDESC_ST>(tS, dK_kmaj, dQ_kmaj + s1 * TILE16);
@@ -1035,17 +1051,38 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
           }
           __syncwarp();
         }
-        // dQᵀ = Kᵀ dSᵀ over [128, 256): both halves of dPᵀ have been read out (dSᵀ ready)
+        // dK += dSᵀ Q once both halves of dSᵀ are formed, and dQᵀ = Kᵀ dSᵀ over [0, 128) once both halves
+        // of the next Sᵀ are in registers (the last step's [0, 128) holds only Pᵀ, read by its dV MMAs
+        // above).  dQᵀ goes first when it can: the next Pᵀ is written over [0, 64) only after dQᵀ has been
+        // read out; otherwise dK fills the tensor core while the next Sᵀ is being read.
+        if (!warp_wait_b(bar(C::B_DSREADY + 0), it & 1, wd) || !warp_wait_b(bar(C::B_DSREADY + 1), it & 1, wd)) break;
+        tc_fence_after();
+        const bool dq_first = !more;
+        if (dq_first) {
+          tc_fence_after();
+          if (elect_one()) {
+            bwd_issue_dq128<IDESC_DQ>(tDQ, dKt_mn, dDS_mn);
+            tc_commit(bar(C::B_DQFULL));
+          }
+          __syncwarp();
+        }
         if (elect_one()) {
-          bwd_issue_dq128<IDESC_DQ>(tDQ, dKt_mn, dDS_mn);
-          tc_commit(bar(C::B_DQFULL));
+          bwd_issue_acc<BQ, IDESC_DKV>(tDK, tDS, dQ_mn + s * TILE16, it > 0 ? 1u : 0u);
           tc_commit(bar(C::B_QEMPTY + s));  // Q and row terms of this step no longer read
         }
         __syncwarp();
-        // dPᵀ of the next step over [128, 256) once dQᵀ has been read out
+        if (!dq_first) {
+          if (!warp_wait_b(bar(C::B_SREAD), (it + 1) & 1, wd)) break;
+          tc_fence_after();
+          if (elect_one()) {
+            bwd_issue_dq128<IDESC_DQ>(tDQ, dKt_mn, dDS_mn);
+            tc_commit(bar(C::B_DQFULL));
+          }
+          __syncwarp();
+        }
+        // dPᵀ of the next step over [128, 256) (dSᵀ there is read by dK, issued above)
         if (more) {
-          if (!warp_wait_b(bar(C::B_DQFREE), it & 1, wd) || !warp_wait_b(bar(C::B_DOFULL), (it + 1) & 1, wd))
-            break;
+          if (!warp_wait_b(bar(C::B_DOFULL), (it + 1) & 1, wd)) break;
           tc_fence_after();
           if (elect_one()) {
             bwd_issue_kt<C::D, BQ, IDESC_ST>(tDP, dV_kmaj, dDO_kmaj);
@@ -1071,7 +1108,7 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
     const uint32_t tS = tmem + lane_off + C::T_S + 64u * a;    // this half of Sᵀ
     const uint32_t tP = tmem + lane_off + C::T_P + 32u * a;    // this half of Pᵀ (packed)
     const uint32_t tDP = tmem + lane_off + C::T_DP + 64u * a;  // this half of dPᵀ
-    const uint32_t tDS = tmem + lane_off + C::T_DS + 32u * a;  // this half of dSᵀ (packed, over Sᵀ)
+    const uint32_t tDS = tmem + lane_off + C::T_DS + 32u * a;  // this half of dSᵀ (packed, over dPᵀ)
     const uint32_t tDV = tmem + lane_off + C::T_DV + 64u * a;  // dV columns this warpgroup writes out
     const int kr = 32 * quarter + lane;  // key row within the tile
     const int key = k0 + kr;             // position in the sequence
@@ -1105,8 +1142,14 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
         for (int i = 0; i < 64; i += 2) {
           const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), c2,
                                       make_float2(lse_h[i], lse_h[i + 1]));
-          pt[i] = ex2(x.x);
-          pt[i + 1] = ex2(x.y);
+          if (((kBwd128PolyMask >> ((i >> 1) & 7)) & 1u) && full) {
+            const float2 e = exp2_poly2(x);
+            pt[i] = e.x;
+            pt[i + 1] = e.y;
+          } else {
+            pt[i] = ex2(x.x);
+            pt[i + 1] = ex2(x.y);
+          }
         }
         if (!full) {
 #pragma unroll
@@ -1116,8 +1159,11 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
         for (int i = 0; i < 32; ++i) pk[i] = pack2<BF16>(pt[2 * i], pt[2 * i + 1]);
       }
       // packed over [32a, 32a + 32): for a = 1 those are Sᵀ columns of half 0, so both halves must have
-      // been read first
-      if (!warp_wait_b(bar(C::B_SREAD), it & 1, wd)) { ok = false; break; }
+      // been read first, and dQᵀ of the previous step (written there after that) must have been read out
+      if (!warp_wait_b(bar(C::B_SREAD), it & 1, wd) || (it > 0 && !warp_wait_b(bar(C::B_DQFREE), (it - 1) & 1, wd))) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       tmem_st32(tP, pk);
       tmem_wait_st();
@@ -1141,13 +1187,18 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
           dsk[16 * q + i] = pack2<BF16>(ds.x, ds.y);
         }
       }
-      // into shared-memory chunk a as a 128-byte swizzled row (B operand of dQᵀ), and packed into tensor
-      // memory over Sᵀ columns both warpgroups have read (A operand of dK)
+      tc_fence_before();
+      mbar_arrive(bar(C::B_DPREAD));
+      // into shared-memory chunk a as a 128-byte swizzled row (B operand of dQᵀ)
 #pragma unroll
       for (int j = 0; j < 8; ++j)
         *reinterpret_cast<uint4*>(ds_row + ((j ^ (kr & 7)) << 4)) =
             make_uint4(dsk[4 * j], dsk[4 * j + 1], dsk[4 * j + 2], dsk[4 * j + 3]);
       fence_proxy_async_smem();
+      // packed over [128 + 32a, ...) (A operand of dK): for a = 1 those are dPᵀ columns of half 0, so both
+      // halves must have been read first
+      if (!warp_wait_b(bar(C::B_DPREAD), it & 1, wd)) { ok = false; break; }
+      tc_fence_after();
       tmem_st32(tDS, dsk);
       tmem_wait_st();
       tc_fence_before();
@@ -1190,8 +1241,8 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
       const int i0 = (i_begin + it) * BQ;
       if (!warp_wait_b(bar(C::B_DQFULL), it & 1, wd)) { ok = false; break; }
       tc_fence_after();
-      // the whole partial into registers (lane = feature 32·quarter + lane, columns = queries), so the
-      // next dPᵀ may overwrite [128, 256) at once; staging and the reduce-adds follow at their own pace
+      // the whole partial into registers (lane = feature 32·quarter + lane, columns = queries), so that
+      // [0, 128) is released at once; staging and the reduce-adds follow at their own pace
       uint32_t qr[128];
       tmem_ld64(tDQ, reinterpret_cast<uint32_t(&)[64]>(qr[0]));
       tmem_ld64(tDQ + 64u, reinterpret_cast<uint32_t(&)[64]>(qr[64]));

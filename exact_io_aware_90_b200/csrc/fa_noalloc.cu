@@ -15,15 +15,16 @@
 //     library routine;
 //   * problems whose workspace exceeds FA_NOALLOC_SCRATCH_BYTES are rejected
 //     with FA_ERR_UNSUPPORTED before anything is launched;
-//   * every call shares the one array per device and it keeps the last
-//     call's contents; the backward's first kernel zeroes what must start at
-//     zero, so stale contents do no harm, but two calls whose kernels overlap
+//   * every call on a device (in one CUDA context) shares the one array, which keeps the last
+//     call's contents; the backward's first kernel zeroes what must start
+//     at zero, so stale contents do no harm, but two calls whose kernels overlap
 //     on the GPU (different streams, no ordering) race on the array;
-//   * the first call on a device looks up the array's device address
-//     (cudaGetSymbolAddress, with that device current); make that first call
+//   * every call looks up the array's device address in the context current
+//     on the calling thread: a __device__ array has one copy per CUDA context,
+//     so an address cached per device ordinal would be wrong for a caller on a
+//     non-primary context, or after cudaDeviceReset.  The first lookup in a
+//     context may load the library's device code into it; make that first call
 //     before any stream capture.
-#include <mutex>
-
 #include "../../include/fa.h"
 #include "fa_internal.h"
 
@@ -33,22 +34,13 @@ namespace fa {
 // for the device array: its device address comes from cudaGetSymbolAddress.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-static void* g_noalloc_ptr[kMaxDevices] = {};
-static std::mutex g_noalloc_mu;
-
-// Device address of the scratch array on the current device, looked up once
-// per device.  Returns nullptr if the lookup fails.
-static void* noalloc_scratch_for_current_device() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return nullptr;
-    g_noalloc_ptr[dev] = p;
-  }
-  return g_noalloc_ptr[dev];
+// Device address of the scratch array in the calling thread's current context,
+// or nullptr if the lookup fails.  Looked up on every call (cheap once the
+// module is loaded), so it always belongs to the context the kernels run in.
+static void* noalloc_scratch_for_current_context() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+  return p;
 }
 
 }  // namespace fa
@@ -60,7 +52,7 @@ extern "C" int fa_bwd_noalloc(const void* q, const void* k, const void* v, const
   const size_t need = fa_bwd_workspace_bytes(total_tokens, H, d);
   if (need == 0) return FA_ERR_INVALID_ARG;
   if (need > (size_t)FA_NOALLOC_SCRATCH_BYTES) return FA_ERR_UNSUPPORTED;
-  void* scratch = fa::noalloc_scratch_for_current_device();
+  void* scratch = fa::noalloc_scratch_for_current_context();
   if (scratch == nullptr) return FA_ERR_CUDA;
   return fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, scale, causal, cu_seqlens, total_tokens, dtype, scratch,
                 (size_t)FA_NOALLOC_SCRATCH_BYTES, stream);

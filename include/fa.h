@@ -161,15 +161,20 @@ int fa_bwd_postprocess(void* dq, int B, int H, int N, int d, float scale,
  * the dQ accumulator and D live in a static device array of
  * FA_NOALLOC_SCRATCH_BYTES inside the library.  Nothing is allocated or freed.
  *   - Returns FA_ERR_UNSUPPORTED, launching nothing, when the problem needs more
- *     scratch than that: fa_bwd_workspace_bytes(total_tokens, H, d) must not
- *     exceed FA_NOALLOC_SCRATCH_BYTES (about 63k token-heads at d = 128,
- *     126k at d = 64).
+ *     scratch than that.  The rule is exactly fa_bwd_workspace_bytes(total_tokens,
+ *     H, d) <= FA_NOALLOC_SCRATCH_BYTES, which holds up to total_tokens·H =
+ *     floor(FA_NOALLOC_SCRATCH_BYTES / (4·d + 4)) token-heads: 65,027 at
+ *     d = 128 and 129,055 at d = 64.
  *   - All calls on a device share the one array, which keeps the last call's
  *     contents (the first kernel of every call zeroes what must start at zero).
  *     Calls whose kernels overlap on the GPU — e.g. on two streams with no
  *     ordering between them — race on the array and give wrong results.
- *   - The first call on a device looks up the array's device address with that
- *     device current; make that first call before any stream capture.
+ *   - Every call looks up the array's device address in the CUDA context that
+ *     is current on the calling thread (a __device__ array has one copy per
+ *     context), so callers on a non-primary context, or after cudaDeviceReset,
+ *     get their own context's array.  The first lookup in a context may load
+ *     the library's device code into it; make that first call before any
+ *     stream capture.
  */
 int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
                    const void* dO, void* dq, void* dk, void* dv,

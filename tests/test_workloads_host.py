@@ -47,6 +47,19 @@ def test_e4m3_per_head_quantisation():
     assert math.isclose(float(ds[0, 1] / ds[0, 0]), 8.0, rel_tol=0.5)
 
 
+def test_e4m3_quantisers_zero_heads_and_gaps():
+    """An all-zero (sequence, head) keeps descale 1 and stores exact zeros (descale 0 would make NaN
+    codes and break the kernels' 'finite and > 0' contract); tokens outside every segment are 0."""
+    x = torch.randn(40, 2, 128, generator=torch.Generator().manual_seed(9))
+    x[0:10, 1] = 0.0                                                   # head 1 of sequence 0 is all zero
+    segs = [(0, 10), (10, 20)]                                         # tokens 30..39 belong to no segment
+    q8, ds = workloads.quantize_e4m3_per_head(x, segs)
+    assert ds[0, 1] == 1.0 and np.all(np.isfinite(ds)) and np.all(ds > 0)
+    stored = q8.float()
+    assert torch.all(torch.isfinite(stored))
+    assert torch.all(stored[0:10, 1] == 0) and torch.all(stored[30:] == 0)
+
+
 def test_generators_are_deterministic():
     for name in ("tiny_d64", "mha_n4k_d64"):
         a, b = workloads.make_workload(name), workloads.make_workload(name)

@@ -5,18 +5,20 @@ GPU's memory and hands them only their input and output buffers, or must not
 call cudaMalloc at all (it can synchronise the device and can fail under a
 fixed memory budget).  fa_bwd_noalloc lets them run the backward with its
 workspace in the library's own static device array instead of a buffer they
-would have to allocate.  These tests call it through the C ABI and check it
-gives the same gradients as fa_bwd with a caller-provided workspace, on two
-calls in a row (the array keeps the previous call's contents, so the second
-call shows that stale scratch does no harm).  This file is named to be
-collected last.
+would have to allocate.  These tests call it through the C ABI and check that
+it gives the same gradients as fa_bwd with a caller-provided workspace and,
+within the gradient tolerance, as the fp64 oracle, on two calls in a row (the
+array keeps the previous call's contents, so the second call shows that stale
+scratch does no harm); and that, once the library is loaded, the calls change
+neither the device's free memory nor PyTorch's allocations.  This file is
+named to be collected last.
 """
 
 import pytest
 import torch
 
 import workloads
-from _gpu import GRAD_TOL, f64, rel_l2
+from _gpu import GRAD_TOL, covered_rows, f64, oracle_backward, rel_l2
 
 pytestmark = pytest.mark.gpu
 
@@ -58,16 +60,29 @@ def test_noalloc_matches_workspace_backward_twice(fa, d, causal, dtype, seqlens)
     assert st == fa.FA_OK
     assert fa.fa_check_device_status(stream) == fa.FA_OK
     assert ws_bytes <= fa.FA_NOALLOC_SCRATCH_BYTES
+    rows = covered_rows(inp)
+    oracle_grads = oracle_backward(inp)
+    outs = [[torch.full_like(q, float("nan")) for _ in range(3)] for _ in range(2)]
+    torch.cuda.synchronize()
+    free_before = torch.cuda.mem_get_info()[0]
+    torch_before = torch.cuda.memory_allocated()
     for call in range(2):
-        got = [torch.full_like(q, float("nan")) for _ in range(3)]
+        got = outs[call]
         st = fa.fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), *(_ptr(t) for t in got),
                                B, H, N, d, inp.scale, int(causal), _ptr(cu), T, code, stream)
         assert st == fa.FA_OK, fa.fa_status_string(st)
         assert fa.fa_check_device_status(stream) == fa.FA_OK
-        rows = torch.arange(int(inp.cu_seqlens[-1])) if cu is not None else torch.arange(T)
-        for name, g, r in zip(("dq", "dk", "dv"), got, ref):
-            e = rel_l2(f64(g[rows]), f64(r[rows]))
-            assert e <= GRAD_TOL, (call, name, e)
+    # nothing was allocated by the two calls (the library and its static array were loaded by the
+    # first fa_bwd call above)
+    assert torch.cuda.mem_get_info()[0] == free_before
+    assert torch.cuda.memory_allocated() == torch_before
+    for call in range(2):
+        for name, g, r, ro in zip(("dq", "dk", "dv"), outs[call], ref, oracle_grads):
+            a = f64(g)[rows]
+            e = rel_l2(a, f64(r)[rows])
+            assert e <= GRAD_TOL, (call, name, "vs fa_bwd", e)
+            e = rel_l2(a, ro[rows])
+            assert e <= GRAD_TOL, (call, name, "vs oracle", e)
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch(fa):

@@ -100,6 +100,8 @@ def _randn_e4m3(g: torch.Generator, shape):
     """(e4m3 tensor, descale) with real values = e4m3 value × descale, descale = amax / 448."""
     x = torch.randn(*shape, generator=g, dtype=torch.float32)
     descale = float(np.float32(float(x.abs().max()) / E4M3_MAX))  # the fp32 value the C ABI receives
+    if not descale > 0.0:
+        descale = 1.0  # an all-zero tensor keeps descale 1 (the C ABI wants it finite and > 0)
     return (x / descale).to(torch.float8_e4m3fn), descale
 
 
@@ -121,12 +123,13 @@ def quantize_e4m3_per_head(x: torch.Tensor, segments):
     amax/448 (rounded to fp32) and rounded to e4m3."""
     T, H, _ = x.shape
     ds = np.ones((len(segments), H), dtype=np.float32)
-    y = torch.empty_like(x)
+    y = torch.zeros_like(x)  # tokens outside every segment stay 0
     for b, (s0, L) in enumerate(segments):
         if L == 0:
             continue
         amax = x[s0:s0 + L].abs().amax(dim=(0, 2))                      # [H]
-        ds[b] = (amax / E4M3_MAX).numpy().astype(np.float32)
+        d = (amax / E4M3_MAX).numpy().astype(np.float32)
+        ds[b] = np.where(d > 0, d, np.float32(1.0))  # an all-zero head keeps descale 1 (finite and > 0)
         y[s0:s0 + L] = x[s0:s0 + L] / torch.from_numpy(ds[b])[None, :, None]
     return y.to(torch.float8_e4m3fn), ds
 
