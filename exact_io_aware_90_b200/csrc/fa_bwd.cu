@@ -785,23 +785,29 @@ struct Bq128 {
   // tensor memory columns
   static constexpr uint32_t T_S = 0, T_P = 0, T_DQ = 0, T_DP = 128, T_DS = 128, T_DK = 256, T_DV = 384;
   // barriers
-  static constexpr int B_KV = 0;
-  static constexpr int B_QFULL = 1;     // [2] Q tile of stage s landed
-  static constexpr int B_QEMPTY = 3;    // [2] Q tile and row terms of stage s no longer read
-  static constexpr int B_ROWFULL = 5;   // [2] −LSE·log2 e and −D of stage s written (32 arrivals)
-  static constexpr int B_DOFULL = 7;
-  static constexpr int B_DOEMPTY = 8;
-  static constexpr int B_SFULL = 9;
-  static constexpr int B_DPFULL = 10;
-  static constexpr int B_SREAD = 11;    // both halves of Sᵀ in registers (256 arrivals)
-  static constexpr int B_DPREAD = 12;   // both halves of dPᵀ in registers (256 arrivals)
-  static constexpr int B_PREADY = 13;   // [2] half a of Pᵀ in tensor memory (128 arrivals)
-  static constexpr int B_DSREADY = 15;  // [2] half a of dSᵀ in tensor and shared memory (128 arrivals)
-  static constexpr int B_DQFULL = 17;
-  static constexpr int B_DQFREE = 18;   // dQᵀ read out of [0, 128) (128 arrivals)
-  static constexpr int B_DKV = 19;
-  static constexpr int B_DRAIN = 20;
-  static constexpr int NBARS = 21;
+  static constexpr int B_KVFULL = 0;    // K, V of the unit landed
+  static constexpr int B_KVEMPTY = 1;   // K, V no longer read (the unit's last MMAs done)
+  static constexpr int B_QFULL = 2;     // [2] Q tile of stage s landed
+  static constexpr int B_QEMPTY = 4;    // [2] Q tile and row terms of stage s no longer read
+  static constexpr int B_ROWFULL = 6;   // [2] −LSE·log2 e and −D of stage s written (32 arrivals)
+  static constexpr int B_DOFULL = 8;
+  static constexpr int B_DOEMPTY = 9;
+  static constexpr int B_SFULL = 10;
+  static constexpr int B_DPFULL = 11;
+  static constexpr int B_SREAD = 12;    // both halves of Sᵀ in registers (256 arrivals)
+  static constexpr int B_DPREAD = 13;   // both halves of dPᵀ in registers (256 arrivals)
+  static constexpr int B_PREADY = 14;   // [2] half a of Pᵀ in tensor memory (128 arrivals)
+  static constexpr int B_DSREADY = 16;  // [2] half a of dSᵀ in tensor and shared memory (128 arrivals)
+  static constexpr int B_DQFULL = 18;
+  static constexpr int B_DQFREE = 19;   // dQᵀ read out of [0, 128) (128 arrivals)
+  static constexpr int B_DKV = 20;      // dK, dV of the unit complete
+  static constexpr int B_DKVFREE = 21;  // dK, dV read out of tensor memory (128 arrivals)
+  static constexpr int B_UFULL = 22;    // [2] work-unit ring slot written
+  static constexpr int B_UEMPTY = 24;   // [2] slot read by every reader warp
+  static constexpr int B_CLC = 26;      // scheduler response landed
+  static constexpr int B_DRAIN = 27;
+  static constexpr int NBARS = 28;
+  static constexpr int UNIT_READERS = 14;  // compute warps 0-7, dQ warps 8-11, MMA warp 13, row-term warp 14
   // shared memory: K, V resident; Q double-buffered; dO single (its next tile loads once dV has read
   // it, well before the next dPᵀ); dSᵀ as two [128 keys × 64 queries] chunks (B operand of dQᵀ)
   static constexpr uint32_t OFF_K = 0;
@@ -812,8 +818,9 @@ struct Bq128 {
   static constexpr uint32_t OFF_DQS = 6 * TILE;  // dQ staging: per dQ warp two boxes [32 queries × 32 fp32]
   static constexpr uint32_t DQ_BOX = 32 * 128;
   static constexpr uint32_t OFF_ROW = OFF_DQS + 8 * DQ_BOX;  // per stage: −LSE·log2 e [128], −D [128] (fp32)
-  static constexpr uint32_t OFF_BAR = OFF_ROW + 2 * 2 * BQ * 4;
-  static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
+  static constexpr uint32_t OFF_CLC = OFF_ROW + 2 * 2 * BQ * 4;  // 16-byte scheduler response
+  static constexpr uint32_t OFF_BAR = OFF_CLC + 16;
+  static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;  // TMEM base, abort flag, unit ring [2]
   // no alignment slack: the dynamic shared memory is declared 1024-byte aligned (checked at run time)
   static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -832,6 +839,46 @@ __device__ __forceinline__ void bwd_issue_dq128(uint32_t d_tmem, uint64_t da, ui
   db = opaque64(db);
 #pragma unroll
   for (int kk = 0; kk < kBK / 16; ++kk) mma_ss(d_tmem, da + ((kk * 2048) >> 4), db + ((kk * 2048) >> 4), IDESC, kk > 0 ? 1u : 0u);
+}
+
+// A decoded work unit of the backward: key tile [k0, k0 + 128) of the sequence whose tokens are
+// [tok0, tok0 + L), head h; n_it Q steps from query tile i_begin.
+struct BwdUnit {
+  int tok0, L, k0, h, i_begin, n_it;
+};
+
+// Unit order: heads in groups (K, V, Q and dO of a group stay in L2), heaviest key tiles (the first
+// ones when causal) first inside a group.  Returns false for a unit whose key tile lies past the end of
+// its sequence; invalid sequence bounds are recorded as FA_ERR_INVALID_ARG (when `record`) and the
+// unit is skipped.
+__device__ __forceinline__ bool decode_bwd_unit(const BwdParams& p, int unit, BwdUnit& u, bool record) {
+  const int BH = p.B * p.H;
+  const int nkb = p.num_kblocks;
+  const int G = p.heads_group;
+  const int group = unit / (G * nkb);
+  const int g_heads = min(G, BH - group * G);
+  const int r = unit - group * G * nkb;
+  const int kb = r / g_heads;
+  const int bh = group * G + r % g_heads;
+  const int b = bh / p.H;
+  u.h = bh - b * p.H;
+  if (p.cu_seqlens != nullptr) {
+    u.tok0 = __ldg(p.cu_seqlens + b);
+    const int end = __ldg(p.cu_seqlens + b + 1);
+    u.L = end - u.tok0;
+    if (u.tok0 < 0 || u.L < 0 || end > p.T || u.L > p.N) {
+      if (record) record_status(1);
+      return false;
+    }
+  } else {
+    u.tok0 = b * p.N;
+    u.L = p.N;
+  }
+  u.k0 = kb * kBK;
+  if (u.k0 >= u.L) return false;
+  u.i_begin = p.causal ? u.k0 / 128 : 0;
+  u.n_it = (u.L + 127) / 128 - u.i_begin;  // ≥ 1
+  return true;
 }
 
 template <bool BF16>
@@ -857,59 +904,33 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
   const uint32_t sQ = s_base + C::OFF_Q;
   const uint32_t sDO = s_base + C::OFF_DO;
   const uint32_t sDS = s_base + C::OFF_DS;
+  const uint32_t clc_resp = s_base + C::OFF_CLC;
   float* row_buf = reinterpret_cast<float*>(smem + C::OFF_ROW);
   const uint32_t bar0 = s_base + C::OFF_BAR;
   auto bar = [&](int i) -> uint32_t { return bar0 + 8u * i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   int* abort_flag = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
+  volatile int* unit_ring = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work unit: heads in groups, heaviest key tiles (the first ones when causal) first
-  const int BH = p.B * p.H;
-  const int nkb = p.num_kblocks;
-  const int G = p.heads_group;
-  const int unit = blockIdx.x;
-  const int group = unit / (G * nkb);
-  const int g_heads = min(G, BH - group * G);
-  const int r = unit - group * G * nkb;
-  const int kb = r / g_heads;
-  const int bh = group * G + r % g_heads;
-  const int b = bh / p.H;
-  const int h = bh - b * p.H;
-
-  int tok0, L;
-  if (p.cu_seqlens != nullptr) {
-    tok0 = __ldg(p.cu_seqlens + b);
-    const int end = __ldg(p.cu_seqlens + b + 1);
-    L = end - tok0;
-    if (tok0 < 0 || L < 0 || end > p.T || L > p.N) {
-      if (threadIdx.x == 0) record_status(1);
-      return;
-    }
-  } else {
-    tok0 = b * p.N;
-    L = p.N;
-  }
-  const int k0 = kb * kBK;
-  if (k0 >= L) return;
-  const int nq_all = (L + BQ - 1) / BQ;
-  const int i_begin = p.causal ? k0 / BQ : 0;
-  const int n_it = nq_all - i_begin;  // ≥ 1
-
+  // ---- set-up, once per CTA: the CTA then runs work units until none is left
   if (warp == 13) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
   if (threadIdx.x == 0) {
-    mbar_init(bar(C::B_KV), 1);
+    mbar_init(bar(C::B_KVFULL), 1);
+    mbar_init(bar(C::B_KVEMPTY), 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(C::B_QFULL + s), 1);
       mbar_init(bar(C::B_QEMPTY + s), 1);
       mbar_init(bar(C::B_ROWFULL + s), 32);
       mbar_init(bar(C::B_PREADY + s), 128);
       mbar_init(bar(C::B_DSREADY + s), 128);
+      mbar_init(bar(C::B_UFULL + s), 1);
+      mbar_init(bar(C::B_UEMPTY + s), C::UNIT_READERS);
     }
     mbar_init(bar(C::B_DOFULL), 1);
     mbar_init(bar(C::B_DOEMPTY), 1);
@@ -920,6 +941,8 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
     mbar_init(bar(C::B_DQFULL), 1);
     mbar_init(bar(C::B_DQFREE), 128);
     mbar_init(bar(C::B_DKV), 1);
+    mbar_init(bar(C::B_DKVFREE), 128);
+    mbar_init(bar(C::B_CLC), 1);
     mbar_init(bar(C::B_DRAIN), 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -937,68 +960,157 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
   const uint32_t tmem = *tmem_slot;
   const Watchdog wd{abort_flag, p.timeout_ns};
 
+  // Reads the next unit from the ring (every reader warp; one lane arrives for the warp).
+  uint32_t un = 0;  // units read by this warp
+  auto read_unit = [&](int& unit) -> bool {
+    const int s = un & 1;
+    if (!warp_wait_b(bar(C::B_UFULL + s), (un >> 1) & 1, wd)) return false;
+    unit = unit_ring[s];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar(C::B_UEMPTY + s));
+    __syncwarp();
+    ++un;
+    return true;
+  };
+
   if (warp >= 12) {
     regs_set<C::REGS_IO, C::REGS_LAUNCH>();
-    if (warp == 14) {
+    if (warp == 12) {
+      // ================================================================ scheduler and TMA producer
+      // Units come from the hardware scheduler: this CTA's own index first, then, one at a time, the
+      // index of a CTA of the grid that has not started yet, whose launch is cancelled.  The next unit
+      // is fetched while the current one is loaded, so that its K and V can be prefetched into L2.
+      const uint64_t pol_kv = l2_policy_evict_first();
+      const uint64_t pol_q = l2_policy_evict_last();
+      uint32_t pub = 0;               // units published
+      uint32_t kvn = 0, qn = 0, don = 0;  // K/V, Q and dO tiles loaded so far
+      uint32_t c_issued = 0, c_done = 0;  // cancellation requests / responses
+      bool can_steal = true, ok = true;
+      auto steal = [&]() -> int {
+        if (!can_steal) return -1;
+        if (elect_one()) {
+          mbar_arrive_expect_tx(bar(C::B_CLC), 16);
+          clc_try_cancel(clc_resp, bar(C::B_CLC));
+        }
+        __syncwarp();
+        ++c_issued;
+        if (!warp_wait_b(bar(C::B_CLC), c_done & 1, wd)) {
+          ok = false;
+          return -1;
+        }
+        ++c_done;
+        int x = -1;
+        const bool got = clc_query(clc_resp, x);
+        fence_proxy_async_smem();  // the read above before the next response overwrites it
+        __syncwarp();
+        if (!got) {
+          can_steal = false;  // no CTA left; no further request may be made
+          return -1;
+        }
+        return x;
+      };
+      // the next unit with work, from `unit` on (-1: none left)
+      auto next_valid = [&](int unit, BwdUnit& u) -> int {
+        while (unit >= 0 && !decode_bwd_unit(p, unit, u, true)) unit = steal();
+        return unit;
+      };
+      auto publish = [&](int unit) -> bool {
+        const int s = pub & 1;
+        if (pub >= 2 && !warp_wait_b(bar(C::B_UEMPTY + s), ((pub >> 1) - 1) & 1, wd)) return false;
+        if (elect_one()) {
+          unit_ring[s] = unit;
+          mbar_arrive(bar(C::B_UFULL + s));  // release: the store is visible once the phase flips
+        }
+        __syncwarp();
+        ++pub;
+        return true;
+      };
+      BwdUnit U, N;
+      int cur = next_valid(blockIdx.x, U);
+      while (ok && cur >= 0) {
+        if (!publish(cur)) break;
+        // K and V of this unit, once the previous unit's last MMAs have read the buffers
+        if (kvn > 0 && !warp_wait_b(bar(C::B_KVEMPTY), (kvn - 1) & 1, wd)) break;
+        if (elect_one()) {
+          mbar_arrive_expect_tx(bar(C::B_KVFULL), 2 * C::TILE);
+          for (int c = 0; c < 2; ++c) {
+            tma_load_3d(sK + c * C::CHUNK, &tm_k, bar(C::B_KVFULL), c * 64, U.h, U.tok0 + U.k0, pol_kv);
+            tma_load_3d(sV + c * C::CHUNK, &tm_v, bar(C::B_KVFULL), c * 64, U.h, U.tok0 + U.k0, pol_kv);
+          }
+        }
+        __syncwarp();
+        ++kvn;
+        // the next unit, its K and V on their way into L2
+        const int nxt = next_valid(steal(), N);
+        if (nxt >= 0 && elect_one()) {
+          for (int c = 0; c < 2; ++c) {
+            tma_prefetch_l2_3d(&tm_k, c * 64, N.h, N.tok0 + N.k0);
+            tma_prefetch_l2_3d(&tm_v, c * 64, N.h, N.tok0 + N.k0);
+          }
+        }
+        __syncwarp();
+        for (int it = 0; ok && it < U.n_it; ++it) {
+          const int i0 = (U.i_begin + it) * BQ;
+          const int s = qn & 1;
+          if (qn >= 2 && !warp_wait_b(bar(C::B_QEMPTY + s), ((qn >> 1) - 1) & 1, wd)) { ok = false; break; }
+          if (elect_one()) {
+            mbar_arrive_expect_tx(bar(C::B_QFULL + s), C::TILE);
+            for (int c = 0; c < 2; ++c)
+              tma_load_3d(sQ + s * C::TILE + c * C::CHUNK, &tm_q, bar(C::B_QFULL + s), c * 64, U.h, U.tok0 + i0,
+                          pol_q);
+          }
+          __syncwarp();
+          ++qn;
+          // dO of this step, once dV of the previous step has read the single buffer
+          if (don > 0 && !warp_wait_b(bar(C::B_DOEMPTY), (don - 1) & 1, wd)) { ok = false; break; }
+          if (elect_one()) {
+            mbar_arrive_expect_tx(bar(C::B_DOFULL), C::TILE);
+            for (int c = 0; c < 2; ++c)
+              tma_load_3d(sDO + c * C::CHUNK, &tm_do, bar(C::B_DOFULL), c * 64, U.h, U.tok0 + i0, pol_q);
+          }
+          __syncwarp();
+          ++don;
+        }
+        cur = nxt;
+        U = N;
+      }
+      if (ok) publish(-1);  // no unit left
+      // Let every load and scheduler response this warp asked for land before the CTA can exit.
+      if (elect_one()) {
+        if (c_issued > c_done) drain_wait_b(bar(C::B_CLC), c_done & 1, p.timeout_ns);
+        if (kvn > 0) drain_wait_b(bar(C::B_KVFULL), (kvn - 1) & 1, p.timeout_ns);
+        for (uint32_t i = qn > 2 ? qn - 2 : 0u; i < qn; ++i)
+          drain_wait_b(bar(C::B_QFULL + (i & 1)), (i >> 1) & 1, p.timeout_ns);
+        if (don > 0) drain_wait_b(bar(C::B_DOFULL), (don - 1) & 1, p.timeout_ns);
+      }
+      __syncwarp();
+    } else if (warp == 14) {
       // ================================================================ row terms
       // −LSE·log2 e and −D of each step's query rows into the stage of its Q tile (rows past the
       // sequence get 0).  A warp of its own: these strided loads would otherwise hold up the TMA issue.
       const float LOG2E = 1.4426950408889634f;
-      for (int it = 0; it < n_it; ++it) {
-        const int s = it & 1;
-        const int i0 = (i_begin + it) * BQ;
-        if (it >= 2 && !warp_wait_b(bar(C::B_QEMPTY + s), ((it >> 1) - 1) & 1, wd)) break;
-        float* lse_s = row_buf + s * 2 * BQ;
-        float* del_s = lse_s + BQ;
-        for (int q = lane; q < BQ; q += 32) {
-          const int qrow = i0 + q;
-          const bool v = qrow < L;
-          lse_s[q] = v ? -__ldg(p.lse + (size_t)(tok0 + qrow) * p.H + h) * LOG2E : 0.f;
-          del_s[q] = v ? -__ldg(p.delta + (size_t)(tok0 + qrow) * p.H + h) : 0.f;
+      uint32_t g = 0;  // steps so far (all units)
+      int unit;
+      while (read_unit(unit) && unit >= 0) {
+        BwdUnit U;
+        decode_bwd_unit(p, unit, U, false);
+        bool ok = true;
+        for (int it = 0; it < U.n_it; ++it, ++g) {
+          const int s = g & 1;
+          const int i0 = (U.i_begin + it) * BQ;
+          if (g >= 2 && !warp_wait_b(bar(C::B_QEMPTY + s), ((g >> 1) - 1) & 1, wd)) { ok = false; break; }
+          float* lse_s = row_buf + s * 2 * BQ;
+          float* del_s = lse_s + BQ;
+          for (int q = lane; q < BQ; q += 32) {
+            const int qrow = i0 + q;
+            const bool v = qrow < U.L;
+            lse_s[q] = v ? -__ldg(p.lse + (size_t)(U.tok0 + qrow) * p.H + U.h) * LOG2E : 0.f;
+            del_s[q] = v ? -__ldg(p.delta + (size_t)(U.tok0 + qrow) * p.H + U.h) : 0.f;
+          }
+          mbar_arrive(bar(C::B_ROWFULL + s));  // release: the stores above are visible to waiters
         }
-        mbar_arrive(bar(C::B_ROWFULL + s));  // release: the stores above are visible to waiters
+        if (!ok) break;
       }
-    } else if (warp == 12) {
-      // ================================================================ TMA producer
-      const uint64_t pol_kv = l2_policy_evict_first();
-      const uint64_t pol_q = l2_policy_evict_last();
-      if (elect_one()) {
-        mbar_arrive_expect_tx(bar(C::B_KV), 2 * C::TILE);
-        for (int c = 0; c < 2; ++c) {
-          tma_load_3d(sK + c * C::CHUNK, &tm_k, bar(C::B_KV), c * 64, h, tok0 + k0, pol_kv);
-          tma_load_3d(sV + c * C::CHUNK, &tm_v, bar(C::B_KV), c * 64, h, tok0 + k0, pol_kv);
-        }
-      }
-      __syncwarp();
-      int q_issued = 0, do_issued = 0;
-      for (int it = 0; it < n_it; ++it) {
-        const int s = it & 1;
-        const int i0 = (i_begin + it) * BQ;
-        if (it >= 2 && !warp_wait_b(bar(C::B_QEMPTY + s), ((it >> 1) - 1) & 1, wd)) break;
-        if (elect_one()) {
-          mbar_arrive_expect_tx(bar(C::B_QFULL + s), C::TILE);
-          for (int c = 0; c < 2; ++c)
-            tma_load_3d(sQ + s * C::TILE + c * C::CHUNK, &tm_q, bar(C::B_QFULL + s), c * 64, h, tok0 + i0, pol_q);
-        }
-        __syncwarp();
-        q_issued = it + 1;
-        // dO of this step, once dV of the previous step has read the single buffer
-        if (it >= 1 && !warp_wait_b(bar(C::B_DOEMPTY), (it - 1) & 1, wd)) break;
-        if (elect_one()) {
-          mbar_arrive_expect_tx(bar(C::B_DOFULL), C::TILE);
-          for (int c = 0; c < 2; ++c)
-            tma_load_3d(sDO + c * C::CHUNK, &tm_do, bar(C::B_DOFULL), c * 64, h, tok0 + i0, pol_q);
-        }
-        __syncwarp();
-        do_issued = it + 1;
-      }
-      if (elect_one()) {
-        drain_wait_b(bar(C::B_KV), 0, p.timeout_ns);
-        for (int it = max(0, q_issued - 2); it < q_issued; ++it)
-          drain_wait_b(bar(C::B_QFULL + (it & 1)), (it >> 1) & 1, p.timeout_ns);
-        if (do_issued > 0) drain_wait_b(bar(C::B_DOFULL), (do_issued - 1) & 1, p.timeout_ns);
-      }
-      __syncwarp();
     } else if (warp == 13) {
       // ================================================================ MMA issuer
       const uint32_t tS = tmem + C::T_S, tP = tmem + C::T_P, tDQ = tmem + C::T_DQ, tDP = tmem + C::T_DP;
@@ -1010,89 +1122,110 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
       const uint64_t dDS_mn = sdesc_sw128(sDS, C::CHUNK, 1024);  // dSᵀ: MN-major B of dQᵀ (queries contiguous)
       constexpr uint32_t TILE16 = C::TILE >> 4;
       constexpr uint32_t HALF16 = (64 * 128) >> 4;  // 64 rows of a chunk: query half 1 of Q / dO
-      bool ok = warp_wait_b(bar(C::B_KV), 0, wd) && warp_wait_b(bar(C::B_QFULL + 0), 0, wd) &&
-                warp_wait_b(bar(C::B_DOFULL), 0, wd);
-      if (ok) {
+      uint32_t g = 0;   // steps so far (all units); step g uses Q stage g mod 2 and the g-th dO tile
+      uint32_t u = 0;   // units so far
+      bool ok = true;
+      int unit;
+      while (ok && read_unit(unit) && unit >= 0) {
+        BwdUnit U;
+        decode_bwd_unit(p, unit, U, false);
+        // Sᵀ and dPᵀ of the unit's first step: K and V in shared memory; [0, 128) released by the read-out
+        // of the previous unit's last dQᵀ ([128, 256) was read by its last dK, issued before)
+        ok = warp_wait_b(bar(C::B_KVFULL), u & 1, wd) && warp_wait_b(bar(C::B_QFULL + (g & 1)), (g >> 1) & 1, wd) &&
+             (g == 0 || warp_wait_b(bar(C::B_DQFREE), (g - 1) & 1, wd)) && warp_wait_b(bar(C::B_DOFULL), g & 1, wd);
+        if (!ok) break;
         tc_fence_after();
         if (elect_one()) {
-          bwd_issue_kt<C::D, BQ, IDESC_ST>(tS, dK_kmaj, dQ_kmaj);
+          bwd_issue_kt<C::D, BQ, IDESC_ST>(tS, dK_kmaj, dQ_kmaj + (g & 1) * TILE16);
           tc_commit(bar(C::B_SFULL));
           bwd_issue_kt<C::D, BQ, IDESC_ST>(tDP, dV_kmaj, dDO_kmaj);
           tc_commit(bar(C::B_DPFULL));
         }
         __syncwarp();
-      }
-      for (int it = 0; ok && it < n_it; ++it) {
-        const int s = it & 1;
-        const bool more = it + 1 < n_it;
-        const int s1 = (it + 1) & 1;
-        // dV += Pᵀ(a) dO(a), as each half of Pᵀ is formed
-        if (!warp_wait_b(bar(C::B_PREADY + 0), it & 1, wd)) break;
-        tc_fence_after();
-        if (elect_one()) bwd_issue_acc<64, IDESC_DKV>(tDV, tP, dDO_mn, it > 0 ? 1u : 0u);
-        __syncwarp();
-        if (!warp_wait_b(bar(C::B_PREADY + 1), it & 1, wd)) break;
-        tc_fence_after();
-        if (elect_one()) {
-          bwd_issue_acc<64, IDESC_DKV>(tDV, tP + 32u, dDO_mn + HALF16, 1u);
-          tc_commit(bar(C::B_DOEMPTY));  // dO of this step is read by no later MMA
-        }
-        __syncwarp();
-        // Sᵀ of the next step over [0, 128): Pᵀ there is read by the dV MMAs above, which run first, and
-        // dQᵀ of the previous step has been read out
-        if (more) {
-          if (!warp_wait_b(bar(C::B_QFULL + s1), ((it + 1) >> 1) & 1, wd) ||
-              (it > 0 && !warp_wait_b(bar(C::B_DQFREE), (it - 1) & 1, wd)))
+        // dK and dV of the previous unit must have been read out before this unit's first products
+        // (accumulate = 0) overwrite them
+        if (u > 0 && !warp_wait_b(bar(C::B_DKVFREE), (u - 1) & 1, wd)) { ok = false; break; }
+        for (int it = 0; it < U.n_it; ++it, ++g) {
+          const int s = g & 1;
+          const bool more = it + 1 < U.n_it;
+          const uint32_t g1 = g + 1;
+          // dV += Pᵀ(a) dO(a), as each half of Pᵀ is formed
+          if (!warp_wait_b(bar(C::B_PREADY + 0), g & 1, wd)) { ok = false; break; }
+          tc_fence_after();
+          if (elect_one()) bwd_issue_acc<64, IDESC_DKV>(tDV, tP, dDO_mn, it > 0 ? 1u : 0u);
+          __syncwarp();
+          if (!warp_wait_b(bar(C::B_PREADY + 1), g & 1, wd)) { ok = false; break; }
+          tc_fence_after();
+          if (elect_one()) {
+            bwd_issue_acc<64, IDESC_DKV>(tDV, tP + 32u, dDO_mn + HALF16, 1u);
+            tc_commit(bar(C::B_DOEMPTY));  // dO of this step is read by no later MMA
+          }
+          __syncwarp();
+          // Sᵀ of the next step over [0, 128): Pᵀ there is read by the dV MMAs above, which run first, and
+          // dQᵀ of the previous step has been read out
+          if (more) {
+            if (!warp_wait_b(bar(C::B_QFULL + (g1 & 1)), (g1 >> 1) & 1, wd) ||
+                (g > 0 && !warp_wait_b(bar(C::B_DQFREE), (g - 1) & 1, wd))) { ok = false; break; }
+            tc_fence_after();
+            if (elect_one()) {
+              bwd_issue_kt<C::D, BQ, IDESC_ST>(tS, dK_kmaj, dQ_kmaj + (g1 & 1) * TILE16);
+              tc_commit(bar(C::B_SFULL));
+            }
+            __syncwarp();
+          }
+          // dK += dSᵀ Q once both halves of dSᵀ are formed, and dQᵀ = Kᵀ dSᵀ over [0, 128) once both
+          // halves of the next Sᵀ are in registers (a unit's last step: [0, 128) holds only Pᵀ, read by
+          // its dV MMAs above).  dQᵀ goes first when it can: the next Pᵀ is written over [0, 64) only after
+          // dQᵀ has been read out; otherwise dK fills the tensor core while the next Sᵀ is being read.
+          if (!warp_wait_b(bar(C::B_DSREADY + 0), g & 1, wd) || !warp_wait_b(bar(C::B_DSREADY + 1), g & 1, wd)) {
+            ok = false;
             break;
+          }
           tc_fence_after();
+          const bool dq_first = !more || warp_test_b(bar(C::B_SREAD), g1 & 1);
+          if (dq_first) {
+            tc_fence_after();
+            if (elect_one()) {
+              bwd_issue_dq128<IDESC_DQ>(tDQ, dKt_mn, dDS_mn);
+              tc_commit(bar(C::B_DQFULL));
+            }
+            __syncwarp();
+          }
           if (elect_one()) {
-            bwd_issue_kt<C::D, BQ, IDESC_ST>(tS, dK_kmaj, dQ_kmaj + s1 * TILE16);
-            tc_commit(bar(C::B_SFULL));
+            bwd_issue_acc<BQ, IDESC_DKV>(tDK, tDS, dQ_mn + s * TILE16, it > 0 ? 1u : 0u);
+            tc_commit(bar(C::B_QEMPTY + s));  // Q and row terms of this step no longer read
           }
           __syncwarp();
-        }
-        // dK += dSᵀ Q once both halves of dSᵀ are formed, and dQᵀ = Kᵀ dSᵀ over [0, 128) once both halves
-        // of the next Sᵀ are in registers (the last step's [0, 128) holds only Pᵀ, read by its dV MMAs
-        // above).  dQᵀ goes first when it can: the next Pᵀ is written over [0, 64) only after dQᵀ has been
-        // read out; otherwise dK fills the tensor core while the next Sᵀ is being read.
-        if (!warp_wait_b(bar(C::B_DSREADY + 0), it & 1, wd) || !warp_wait_b(bar(C::B_DSREADY + 1), it & 1, wd)) break;
-        tc_fence_after();
-        const bool dq_first = !more;
-        if (dq_first) {
-          tc_fence_after();
-          if (elect_one()) {
-            bwd_issue_dq128<IDESC_DQ>(tDQ, dKt_mn, dDS_mn);
-            tc_commit(bar(C::B_DQFULL));
+          if (!dq_first) {
+            if (!warp_wait_b(bar(C::B_SREAD), g1 & 1, wd)) { ok = false; break; }
+            tc_fence_after();
+            if (elect_one()) {
+              bwd_issue_dq128<IDESC_DQ>(tDQ, dKt_mn, dDS_mn);
+              tc_commit(bar(C::B_DQFULL));
+            }
+            __syncwarp();
           }
-          __syncwarp();
+          // dPᵀ of the next step over [128, 256) (dSᵀ there is read by dK, issued above)
+          if (more) {
+            if (!warp_wait_b(bar(C::B_DOFULL), g1 & 1, wd)) { ok = false; break; }
+            tc_fence_after();
+            if (elect_one()) {
+              bwd_issue_kt<C::D, BQ, IDESC_ST>(tDP, dV_kmaj, dDO_kmaj);
+              tc_commit(bar(C::B_DPFULL));
+            }
+            __syncwarp();
+          }
         }
+        if (!ok) break;
         if (elect_one()) {
-          bwd_issue_acc<BQ, IDESC_DKV>(tDK, tDS, dQ_mn + s * TILE16, it > 0 ? 1u : 0u);
-          tc_commit(bar(C::B_QEMPTY + s));  // Q and row terms of this step no longer read
+          tc_commit(bar(C::B_DKV));      // dK, dV of the unit complete
+          tc_commit(bar(C::B_KVEMPTY));  // K and V no longer read
         }
         __syncwarp();
-        if (!dq_first) {
-          if (!warp_wait_b(bar(C::B_SREAD), (it + 1) & 1, wd)) break;
-          tc_fence_after();
-          if (elect_one()) {
-            bwd_issue_dq128<IDESC_DQ>(tDQ, dKt_mn, dDS_mn);
-            tc_commit(bar(C::B_DQFULL));
-          }
-          __syncwarp();
-        }
-        // dPᵀ of the next step over [128, 256) (dSᵀ there is read by dK, issued above)
-        if (more) {
-          if (!warp_wait_b(bar(C::B_DOFULL), (it + 1) & 1, wd)) break;
-          tc_fence_after();
-          if (elect_one()) {
-            bwd_issue_kt<C::D, BQ, IDESC_ST>(tDP, dV_kmaj, dDO_kmaj);
-            tc_commit(bar(C::B_DPFULL));
-          }
-          __syncwarp();
-        }
+        ++u;
       }
+      // every MMA issued so far must finish before tensor memory is released
       if (elect_one()) {
-        tc_commit(bar(C::B_DKV));
         tc_commit(bar(C::B_DRAIN));
         drain_wait_b(bar(C::B_DRAIN), 0, p.timeout_ns);
       }
@@ -1109,194 +1242,192 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
     const uint32_t tP = tmem + lane_off + C::T_P + 32u * a;    // this half of Pᵀ (packed)
     const uint32_t tDP = tmem + lane_off + C::T_DP + 64u * a;  // this half of dPᵀ
     const uint32_t tDS = tmem + lane_off + C::T_DS + 32u * a;  // this half of dSᵀ (packed, over dPᵀ)
-    const uint32_t tDV = tmem + lane_off + C::T_DV + 64u * a;  // dV columns this warpgroup writes out
     const int kr = 32 * quarter + lane;  // key row within the tile
-    const int key = k0 + kr;             // position in the sequence
     const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
     uint8_t* ds_row = smem + C::OFF_DS + a * C::CHUNK + kr * 128;
+    uint32_t g = 0;  // steps so far (all units)
     bool ok = true;
-    for (int it = 0; it < n_it; ++it) {
-      const int i0 = (i_begin + it) * BQ + 64 * a;  // first query of this half
-      const int s = it & 1;
-      if (!warp_wait_b(bar(C::B_ROWFULL + s), (it >> 1) & 1, wd)) { ok = false; break; }
-      const float* lse_h = row_buf + s * 2 * BQ + 64 * a;
-      const float* del_h = lse_h + BQ;
-      // visible queries for this key: q >= key (causal) and q < L; key < L
-      const int q_lo = p.causal ? key - i0 : 0;  // first visible column of the half
-      const int q_hi = (key < L) ? L - i0 : -1;  // one past the last visible column
-      const bool full = __all_sync(0xffffffffu, q_lo <= 0 && q_hi >= 64);
-      // ---- Pᵀ = 2^(c·Sᵀ − LSE·log2 e), masked
-      if (!warp_wait_b(bar(C::B_SFULL), it & 1, wd)) { ok = false; break; }
-      tc_fence_after();
-      // Pᵀ is kept in registers only in its packed 16-bit form (the values the dV product uses), which
-      // leaves registers for the dQ warpgroup to take its whole partial out of tensor memory at once
-      uint32_t pk[32];
-      {
-        uint32_t sr[64];
-        tmem_ld64(tS, sr);
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(bar(C::B_SREAD));
-        float pt[64];
+    int unit;
+    while (ok && read_unit(unit) && unit >= 0) {
+      BwdUnit U;
+      decode_bwd_unit(p, unit, U, false);
+      const int key = U.k0 + kr;  // position in the sequence
+      for (int it = 0; it < U.n_it; ++it, ++g) {
+        const int i0 = (U.i_begin + it) * BQ + 64 * a;  // first query of this half
+        const int s = g & 1;
+        if (!warp_wait_b(bar(C::B_ROWFULL + s), (g >> 1) & 1, wd)) { ok = false; break; }
+        const float* lse_h = row_buf + s * 2 * BQ + 64 * a;
+        const float* del_h = lse_h + BQ;
+        // visible queries for this key: q >= key (causal) and q < L; key < L
+        const int q_lo = p.causal ? key - i0 : 0;    // first visible column of the half
+        const int q_hi = (key < U.L) ? U.L - i0 : -1;  // one past the last visible column
+        const bool full = __all_sync(0xffffffffu, q_lo <= 0 && q_hi >= 64);
+        // ---- Pᵀ = 2^(c·Sᵀ − LSE·log2 e), masked
+        if (!warp_wait_b(bar(C::B_SFULL), g & 1, wd)) { ok = false; break; }
+        tc_fence_after();
+        // Pᵀ is kept in registers only in its packed 16-bit form (the values the dV product uses), which
+        // leaves registers for the dQ warpgroup to take its whole partial out of tensor memory at once
+        uint32_t pk[32];
+        {
+          uint32_t sr[64];
+          tmem_ld64(tS, sr);
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(bar(C::B_SREAD));
+          float pt[64];
 #pragma unroll
-        for (int i = 0; i < 64; i += 2) {
-          const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), c2,
-                                      make_float2(lse_h[i], lse_h[i + 1]));
-          if (((kBwd128PolyMask >> ((i >> 1) & 7)) & 1u) && full) {
-            const float2 e = exp2_poly2(x);
-            pt[i] = e.x;
-            pt[i + 1] = e.y;
-          } else {
+          for (int i = 0; i < 64; i += 2) {
+            const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), c2,
+                                        make_float2(lse_h[i], lse_h[i + 1]));
             pt[i] = ex2(x.x);
             pt[i + 1] = ex2(x.y);
           }
+          if (!full) {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) pt[i] = (i >= q_lo && i < q_hi) ? pt[i] : 0.f;
+          }
+#pragma unroll
+          for (int i = 0; i < 32; ++i) pk[i] = pack2<BF16>(pt[2 * i], pt[2 * i + 1]);
         }
-        if (!full) {
-#pragma unroll
-          for (int i = 0; i < 64; ++i) pt[i] = (i >= q_lo && i < q_hi) ? pt[i] : 0.f;
+        // packed over [32a, 32a + 32): for a = 1 those are Sᵀ columns of half 0, so both halves must have
+        // been read first, and dQᵀ of the previous step (written there after that) must have been read out
+        if (!warp_wait_b(bar(C::B_SREAD), g & 1, wd) || (g > 0 && !warp_wait_b(bar(C::B_DQFREE), (g - 1) & 1, wd))) {
+          ok = false;
+          break;
         }
+        tc_fence_after();
+        tmem_st32(tP, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(C::B_PREADY + a));
+        // ---- dSᵀ = Pᵀ ∘ (dPᵀ − D)
+        if (!warp_wait_b(bar(C::B_DPFULL), g & 1, wd)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t dsk[32];
+        {
+          uint32_t dr[64];
+          tmem_ld64(tDP, dr);
+          tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) pk[i] = pack2<BF16>(pt[2 * i], pt[2 * i + 1]);
-      }
-      // packed over [32a, 32a + 32): for a = 1 those are Sᵀ columns of half 0, so both halves must have
-      // been read first, and dQᵀ of the previous step (written there after that) must have been read out
-      if (!warp_wait_b(bar(C::B_SREAD), it & 1, wd) || (it > 0 && !warp_wait_b(bar(C::B_DQFREE), (it - 1) & 1, wd))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      tmem_st32(tP, pk);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(C::B_PREADY + a));
-      // ---- dSᵀ = Pᵀ ∘ (dPᵀ − D)
-      if (!warp_wait_b(bar(C::B_DPFULL), it & 1, wd)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t dsk[32];
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        uint32_t dr[32];
-        tmem_ld32(tDP + 32u * q, dr);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int col = 32 * q + 2 * i;
-          const float2 dpv = make_float2(__uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1]));
-          const float2 dd = __fadd2_rn(dpv, make_float2(del_h[col], del_h[col + 1]));
-          const float2 ds = __fmul2_rn(unpack2<BF16>(pk[col >> 1]), dd);
-          dsk[16 * q + i] = pack2<BF16>(ds.x, ds.y);
+          for (int i = 0; i < 32; ++i) {
+            const float2 dpv = make_float2(__uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1]));
+            const float2 dd = __fadd2_rn(dpv, make_float2(del_h[2 * i], del_h[2 * i + 1]));
+            const float2 ds = __fmul2_rn(unpack2<BF16>(pk[i]), dd);
+            dsk[i] = pack2<BF16>(ds.x, ds.y);
+          }
         }
-      }
-      tc_fence_before();
-      mbar_arrive(bar(C::B_DPREAD));
-      // into shared-memory chunk a as a 128-byte swizzled row (B operand of dQᵀ)
+        tc_fence_before();
+        mbar_arrive(bar(C::B_DPREAD));
+        // into shared-memory chunk a as a 128-byte swizzled row (B operand of dQᵀ)
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        *reinterpret_cast<uint4*>(ds_row + ((j ^ (kr & 7)) << 4)) =
-            make_uint4(dsk[4 * j], dsk[4 * j + 1], dsk[4 * j + 2], dsk[4 * j + 3]);
-      fence_proxy_async_smem();
-      // packed over [128 + 32a, ...) (A operand of dK): for a = 1 those are dPᵀ columns of half 0, so both
-      // halves must have been read first
-      if (!warp_wait_b(bar(C::B_DPREAD), it & 1, wd)) { ok = false; break; }
-      tc_fence_after();
-      tmem_st32(tDS, dsk);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(C::B_DSREADY + a));
-    }
-    // ---- epilogue: dV rows of this tile, columns [64a, 64a + 64)
-    if (ok && warp_wait_b(bar(C::B_DKV), 0, wd)) {
-      tc_fence_after();
-      const bool valid = key < L;
-      uint8_t* dst = reinterpret_cast<uint8_t*>(p.dv) +
-                     (((size_t)(tok0 + (valid ? key : 0)) * p.H + h) * C::D + 64 * a) * 2;
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        uint32_t r32[32];
-        tmem_ld32(tDV + 32u * q, r32);
-        tmem_wait_ld();
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = pack2<BF16>(__uint_as_float(r32[2 * i]), __uint_as_float(r32[2 * i + 1]));
-        if (valid) {
-#pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            st_global_v4(dst + q * 64 + v4 * 16, pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
-        }
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<uint4*>(ds_row + ((j ^ (kr & 7)) << 4)) =
+              make_uint4(dsk[4 * j], dsk[4 * j + 1], dsk[4 * j + 2], dsk[4 * j + 3]);
+        fence_proxy_async_smem();
+        // packed over [128 + 32a, ...) (A operand of dK): for a = 1 those are dPᵀ columns of half 0, so both
+        // halves must have been read first
+        if (!warp_wait_b(bar(C::B_DPREAD), g & 1, wd)) { ok = false; break; }
+        tc_fence_after();
+        tmem_st32(tDS, dsk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(C::B_DSREADY + a));
       }
     }
     __syncwarp();
   } else {
-    // ================================================================ dQ warpgroup (warps 8-11; thread = feature)
+    // ================================================================ dQ warpgroup (warps 8-11)
+    // Per step, thread = feature of the dQ partial; per unit, thread = key row of the dK and dV epilogue.
     regs_set<C::REGS_DQ, C::REGS_LAUNCH>();
     const int quarter = warp & 3;
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
     const uint32_t tDQ = tmem + lane_off + C::T_DQ;
     const uint32_t tDK = tmem + lane_off + C::T_DK;
+    const uint32_t tDV = tmem + lane_off + C::T_DV;
     // this warp's two staging boxes: row q = query, 32 fp32 features in 16-byte chunks swizzled by q mod 8
     const uint32_t box_base = s_base + C::OFF_DQS + quarter * 2 * C::DQ_BOX;
-    bool ok = true;
+    uint32_t g = 0;       // steps so far (all units)
+    uint32_t u = 0;       // units so far
     uint32_t pieces = 0;  // boxes staged so far (box = pieces mod 2)
-    for (int it = 0; it < n_it; ++it) {
-      const int i0 = (i_begin + it) * BQ;
-      if (!warp_wait_b(bar(C::B_DQFULL), it & 1, wd)) { ok = false; break; }
-      tc_fence_after();
-      // the whole partial into registers (lane = feature 32·quarter + lane, columns = queries), so that
-      // [0, 128) is released at once; staging and the reduce-adds follow at their own pace
-      uint32_t qr[128];
-      tmem_ld64(tDQ, reinterpret_cast<uint32_t(&)[64]>(qr[0]));
-      tmem_ld64(tDQ + 64u, reinterpret_cast<uint32_t(&)[64]>(qr[64]));
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar(C::B_DQFREE));
+    bool ok = true;
+    int unit;
+    while (ok && read_unit(unit) && unit >= 0) {
+      BwdUnit U;
+      decode_bwd_unit(p, unit, U, false);
+      for (int it = 0; it < U.n_it; ++it, ++g) {
+        const int i0 = (U.i_begin + it) * BQ;
+        if (!warp_wait_b(bar(C::B_DQFULL), g & 1, wd)) { ok = false; break; }
+        tc_fence_after();
+        // the whole partial into registers (lane = feature 32·quarter + lane, columns = queries), so that
+        // [0, 128) is released at once; staging and the reduce-adds follow at their own pace
+        uint32_t qr[128];
+        tmem_ld64(tDQ, reinterpret_cast<uint32_t(&)[64]>(qr[0]));
+        tmem_ld64(tDQ + 64u, reinterpret_cast<uint32_t(&)[64]>(qr[64]));
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar(C::B_DQFREE));
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int q0 = i0 + 32 * c;
-        if (q0 >= L) break;  // the rest of the step lies past the sequence: nothing to add
-        const uint32_t bx = box_base + (pieces & 1u) * C::DQ_BOX;
-        // the box may be rewritten once the reduce issued from it two pieces ago has read it
-        if (lane == 0) bulk_wait_group_read<1>();
-        __syncwarp();
+        for (int c = 0; c < 4; ++c) {
+          const int q0 = i0 + 32 * c;
+          if (q0 >= U.L) break;  // the rest of the step lies past the sequence: nothing to add
+          const uint32_t bx = box_base + (pieces & 1u) * C::DQ_BOX;
+          // the box may be rewritten once the reduce issued from it two pieces ago has read it
+          if (lane == 0) bulk_wait_group_read<1>();
+          __syncwarp();
 #pragma unroll
-        for (int q = 0; q < 32; ++q)
-          st_shared_f32(bx + q * 128 + (((lane >> 2) ^ (q & 7)) << 4) + ((lane & 3) << 2), qr[32 * c + q]);
-        fence_proxy_async_smem();
-        __syncwarp();
-        // rows past the sequence hold exact zeros (P is 0 there); rows past T are clipped by the TMA unit
-        if (lane == 0) {
-          tma_reduce_add_3d(&tm_dq, bx, 32 * quarter, h, tok0 + q0);
-          bulk_commit_group();
+          for (int q = 0; q < 32; ++q)
+            st_shared_f32(bx + q * 128 + (((lane >> 2) ^ (q & 7)) << 4) + ((lane & 3) << 2), qr[32 * c + q]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          // rows past the sequence hold exact zeros (P is 0 there); rows past T are clipped by the TMA unit
+          if (lane == 0) {
+            tma_reduce_add_3d(&tm_dq, bx, 32 * quarter, U.h, U.tok0 + q0);
+            bulk_commit_group();
+          }
+          __syncwarp();
+          ++pieces;
         }
-        __syncwarp();
-        ++pieces;
       }
+      if (!ok) break;
+      // ---- epilogue of the unit: dK (× scale) and dV rows of the key tile, read out of tensor memory
+      // (released to the next unit's first products as soon as they are in registers) and stored
+      if (!warp_wait_b(bar(C::B_DKV), u & 1, wd)) { ok = false; break; }
+      tc_fence_after();
+      const int key = U.k0 + 32 * quarter + lane;
+      const bool valid = key < U.L;
+      uint8_t* dk_row = reinterpret_cast<uint8_t*>(p.dk) + (((size_t)(U.tok0 + (valid ? key : 0)) * p.H + U.h) * C::D) * 2;
+      uint8_t* dv_row = reinterpret_cast<uint8_t*>(p.dv) + (((size_t)(U.tok0 + (valid ? key : 0)) * p.H + U.h) * C::D) * 2;
+#pragma unroll 1
+      for (int t = 0; t < 2; ++t) {  // dK, then dV
+        const float f = t == 0 ? p.scale : 1.f;
+        uint8_t* row = t == 0 ? dk_row : dv_row;
+#pragma unroll
+        for (int q = 0; q < C::D / 32; ++q) {
+          uint32_t r32[32];
+          tmem_ld32((t == 0 ? tDK : tDV) + 32u * q, r32);
+          tmem_wait_ld();
+          if (t == 1 && q == C::D / 32 - 1) {
+            tc_fence_before();
+            mbar_arrive(bar(C::B_DKVFREE));  // dK and dV read out: the next unit may overwrite them
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack2<BF16>(__uint_as_float(r32[2 * i]) * f, __uint_as_float(r32[2 * i + 1]) * f);
+          if (valid) {
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              st_global_v4(row + q * 64 + v4 * 16, pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+          }
+        }
+      }
+      ++u;
     }
     if (lane == 0) bulk_wait_group_all();  // every reduce performed before the kernel ends
-    // ---- epilogue: dK rows (× scale)
-    if (ok && warp_wait_b(bar(C::B_DKV), 0, wd)) {
-      tc_fence_after();
-      const int key = k0 + 32 * quarter + lane;
-      const bool valid = key < L;
-      uint8_t* dst = reinterpret_cast<uint8_t*>(p.dk) + (((size_t)(tok0 + (valid ? key : 0)) * p.H + h) * C::D) * 2;
-#pragma unroll
-      for (int q = 0; q < C::D / 32; ++q) {
-        uint32_t r32[32];
-        tmem_ld32(tDK + 32u * q, r32);
-        tmem_wait_ld();
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pk[i] = pack2<BF16>(__uint_as_float(r32[2 * i]) * p.scale, __uint_as_float(r32[2 * i + 1]) * p.scale);
-        if (valid) {
-#pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            st_global_v4(dst + q * 64 + v4 * 16, pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
-        }
-      }
-    }
     __syncwarp();
   }
 
+  // ---- tear-down
   tc_fence_before();
   __syncthreads();
   if (warp == 13) {
