@@ -21,8 +21,14 @@ Parity status of each function (what pins it; see ``tests/test_oracle.py``):
                           pinned: partials over disjoint key sets (any order, an empty
                           one included) merge to decode_forward over all keys; identity
                           and empty parts; no overflow at log-sum-exps near 1000.
-* ring_attention_forward  pinned: equals attention_forward for 1 … 6 ranks, causal and not.
-* ring_attention_backward pinned: equals attention_backward for 1 … 6 ranks, causal and not.
+* ring_attention_forward  pinned: equals attention_forward for 1 … 6 ranks, causal and not,
+                          in the contiguous and the zigzag layout.
+* ring_attention_backward pinned: equals attention_backward for 1 … 6 ranks, causal and not,
+                          in both layouts.
+* zigzag_chunks, ring_blocks
+                          pinned: the zigzag ring covers every visible (query, key) chunk
+                          pair exactly once, gives every rank the same causal work, and
+                          the contiguous schedule does not.
 * philox4x32_10           pinned: the generator's published known-answer vectors.
 * dropout_keep_mask       pinned: scalar re-derivation of the element mapping,
                           keep fraction within binomial bounds.

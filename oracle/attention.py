@@ -65,6 +65,8 @@ __all__ = [
     "decode_forward",
     "split_kv_decode",
     "merge_attention_partials",
+    "zigzag_chunks",
+    "ring_blocks",
     "ring_attention_forward",
     "ring_attention_backward",
     "philox4x32_10",
@@ -479,67 +481,109 @@ def merge_attention_partials(parts):
     return O, L
 
 
-def ring_attention_forward(q, k, v, scale: float, causal: bool, world: int):
+def zigzag_chunks(rank: int, world: int):
+    """Global chunk indices held by `rank` in the load-balanced ring layout: the sequence is cut into
+    2·world equal chunks and rank r holds chunks r and 2·world − 1 − r (one from each end), so that under
+    the causal mask every rank attends to as many keys as every other.  The pages name ring attention for
+    very long sequences (FlashAttention 与算子融合, 工程实践 "与 CP 配合") but no shard order; this is the
+    reading taken for a balanced one."""
+    return (rank, 2 * world - 1 - rank)
+
+
+def ring_blocks(rank: int, step: int, world: int, causal: bool, layout: str = "contiguous"):
+    """The blocks rank `rank` computes at ring step `step`: a list of (query part, key part, causal
+    diagonal?) over the parts of its own shard and of the shard it holds, that of rank
+    s = (rank − step) mod world.  "contiguous": one part per shard (rank r holds positions [r·S, (r+1)·S));
+    the block is the diagonal when s = r, skipped when s > r under the causal mask.  "zigzag": two parts
+    per shard (``zigzag_chunks``); chunk pair (qc, kc) is the diagonal when qc = kc, skipped when
+    kc > qc under the causal mask."""
+    s_ = (rank - step) % world
+    if layout == "contiguous":
+        if causal and s_ > rank:
+            return []
+        return [(0, 0, causal and s_ == rank)]
+    if layout != "zigzag":
+        raise ValueError("layout must be 'contiguous' or 'zigzag'")
+    out = []
+    for qi, qc in enumerate(zigzag_chunks(rank, world)):
+        for ki, kc in enumerate(zigzag_chunks(s_, world)):
+            if causal and kc > qc:
+                continue
+            out.append((qi, ki, causal and kc == qc))
+    return out
+
+
+def _ring_parts(L: int, world: int, layout: str):
+    """Row ranges of each rank's parts in the global sequence: parts[r] = [(start, stop), ...]."""
+    if layout == "contiguous":
+        if world < 1 or L % world:
+            raise ValueError("the sequence must split into `world` equal shards")
+        S = L // world
+        return [[(r * S, (r + 1) * S)] for r in range(world)]
+    if world < 1 or L % (2 * world):
+        raise ValueError("the zigzag layout splits the sequence into 2·world equal chunks")
+    C = L // (2 * world)
+    return [[(c * C, (c + 1) * C) for c in zigzag_chunks(r, world)] for r in range(world)]
+
+
+def ring_attention_forward(q, k, v, scale: float, causal: bool, world: int, layout: str = "contiguous"):
     """Attention of one dense sequence [L, H, d] computed as ring (context-parallel) attention over
     ``world`` ranks (FlashAttention 与算子融合, 工程实践: the ring of attention for very long
     sequences, with FlashAttention as the compute core): rank r holds positions [r·S, (r+1)·S),
     S = L / world, of q, k and v; at step t it holds the key/value shard of rank s = (r − t) mod
     world, attends its queries to it — the causal diagonal block when s = r, every key when s < r,
     nothing when s > r under the causal mask — and merges the block's (O, LSE) into its running
-    result with ``merge_attention_partials``.  Returns (O [L, H, d], LSE [L, H]) in float64,
-    equal to ``attention_forward`` of the whole sequence."""
+    result with ``merge_attention_partials``.  With ``layout="zigzag"`` each rank holds two chunks
+    (``zigzag_chunks``) and computes the blocks ``ring_blocks`` lists, one running result per chunk.
+    Returns (O [L, H, d], LSE [L, H]) in float64 in the sequence's own order, equal to
+    ``attention_forward`` of the whole sequence."""
     Q, K, V = _f64(q), _f64(k), _f64(v)
     L, H, d = Q.shape
-    if world < 1 or L % world:
-        raise ValueError("the sequence must split into `world` equal shards")
-    S = L // world
+    parts_of = _ring_parts(L, world, layout)
     O = np.zeros((L, H, d))
     LSE = np.full((L, H), -np.inf)
     for r in range(world):
-        rows = slice(r * S, (r + 1) * S)
-        parts = []
+        partials = [[] for _ in parts_of[r]]
         for t in range(world):
             s_ = (r - t) % world
-            if causal and s_ > r:
-                continue
-            cols = slice(s_ * S, (s_ + 1) * S)
-            parts.append(attention_forward(Q[rows], K[cols], V[cols], scale, causal and s_ == r))
-        O[rows], LSE[rows] = merge_attention_partials(parts)
+            for qi, ki, diag in ring_blocks(r, t, world, causal, layout):
+                rows, cols = slice(*parts_of[r][qi]), slice(*parts_of[s_][ki])
+                partials[qi].append(attention_forward(Q[rows], K[cols], V[cols], scale, diag))
+        for qi, (a, b) in enumerate(parts_of[r]):
+            O[a:b], LSE[a:b] = merge_attention_partials(partials[qi])
     return O, LSE
 
 
-def ring_attention_backward(q, k, v, do, scale: float, causal: bool, world: int):
+def ring_attention_backward(q, k, v, do, scale: float, causal: bool, world: int, layout: str = "contiguous"):
     """Gradients of ``ring_attention_forward`` computed on the same ring.  The probabilities of a block
     (query shard r, key shard s) are recomputed from the global row statistic, P_rs = exp(scale·Q_r K_sᵀ
     − LSE_r), as the tiled backward recomputes them from the saved LSE (FlashAttention 短片讲解稿,
     "第三招 · 反向重计算"), with D_r = Σ_c dO_rc·O_rc of the global output; then, per block,
         dS = P_rs ∘ (dO_r V_sᵀ − D_r),  dQ_r += scale·dS K_s,  dK_s += scale·dSᵀ Q_r,  dV_s += P_rsᵀ dO_r,
     where dQ_r accumulates on rank r and dK_s, dV_s travel with the key/value shard s around the ring
-    and are home after one more step.  Returns (dQ, dK, dV) [L, H, d] in float64, equal to
-    ``attention_backward`` of the whole sequence."""
+    and are home after one more step.  ``layout`` as in ``ring_attention_forward`` (blocks are then
+    pairs of chunks).  Returns (dQ, dK, dV) [L, H, d] in float64, equal to ``attention_backward`` of
+    the whole sequence."""
     Q, K, V, dO = _f64(q), _f64(k), _f64(v), _f64(do)
     L, H, d = Q.shape
-    if world < 1 or L % world:
-        raise ValueError("the sequence must split into `world` equal shards")
-    S = L // world
-    O, LSE = ring_attention_forward(Q, K, V, scale, causal, world)
+    parts_of = _ring_parts(L, world, layout)
+    O, LSE = ring_attention_forward(Q, K, V, scale, causal, world, layout)
     D = (dO * O).sum(axis=-1)                                  # [L, H]
     dQ, dK, dV = np.zeros_like(Q), np.zeros_like(K), np.zeros_like(V)
-    sh = lambda x, r: x[r * S:(r + 1) * S]
     for r in range(world):
         for t in range(world):
             s_ = (r - t) % world
-            if causal and s_ > r:
-                continue
-            for h in range(H):
-                Qr, Ks, Vs, dOr = sh(Q, r)[:, h], sh(K, s_)[:, h], sh(V, s_)[:, h], sh(dO, r)[:, h]
-                P = np.exp((Qr @ Ks.T) * scale - sh(LSE, r)[:, h][:, None])
-                if causal and s_ == r:
-                    P[np.triu_indices(S, k=1)] = 0.0
-                dS = P * (dOr @ Vs.T - sh(D, r)[:, h][:, None])
-                dQ[r * S:(r + 1) * S, h] += scale * (dS @ Ks)
-                dK[s_ * S:(s_ + 1) * S, h] += scale * (dS.T @ Qr)
-                dV[s_ * S:(s_ + 1) * S, h] += P.T @ dOr
+            for qi, ki, diag in ring_blocks(r, t, world, causal, layout):
+                rows, cols = slice(*parts_of[r][qi]), slice(*parts_of[s_][ki])
+                for h in range(H):
+                    Qr, Ks, Vs, dOr = Q[rows, h], K[cols, h], V[cols, h], dO[rows, h]
+                    P = np.exp((Qr @ Ks.T) * scale - LSE[rows, h][:, None])
+                    if diag:
+                        P[np.triu_indices(P.shape[0], k=1)] = 0.0
+                    dS = P * (dOr @ Vs.T - D[rows, h][:, None])
+                    dQ[rows, h] += scale * (dS @ Ks)
+                    dK[cols, h] += scale * (dS.T @ Qr)
+                    dV[cols, h] += P.T @ dOr
     return dQ, dK, dV
 
 

@@ -830,3 +830,111 @@ def test_ring_backward_equals_definition():
     assert ok(ring_bwd_variant(q, k, v, do, 0.45, True, 3))
     for kw in (dict(own_lse=True), dict(no_skip=True), dict(no_d=True)):
         assert not ok(ring_bwd_variant(q, k, v, do, 0.45, True, 3, **kw)), kw
+
+
+# ----------------------------------------------------------------------------- load-balanced (zigzag) ring
+
+
+def _zigzag_pins_pass(ring_fwd, ring_bwd, blocks):
+    """Pins of the zigzag ring layout against the whole-sequence definition and the work balance."""
+    rng = np.random.default_rng(77)
+    H, d = 2, 4
+    for w in (1, 2, 3, 4, 6):
+        L = 2 * w * 3  # 3 tokens per chunk
+        q, k, v, do = (rng.standard_normal((L, H, d)) for _ in range(4))
+        for causal in (False, True):
+            O, LSE = oracle.attention_forward(q, k, v, 0.6, causal)
+            Oz, Lz = ring_fwd(q, k, v, 0.6, causal, w, "zigzag")
+            if not (np.allclose(Oz, O, atol=1e-12) and np.allclose(Lz, LSE, atol=1e-12)):
+                return False
+            g = oracle.attention_backward(q, k, v, do, 0.6, causal)
+            gz = ring_bwd(q, k, v, do, 0.6, causal, w, "zigzag")
+            if not all(np.allclose(a, b, atol=1e-11) for a, b in zip(gz, g)):
+                return False
+        # every visible chunk pair is computed exactly once over the ring, and under the causal mask
+        # every rank attends to the same number of (query, key) pairs
+        C = 3
+        work = []
+        for causal in (False, True):
+            seen = {}
+            for r in range(w):
+                pairs = 0
+                for t in range(w):
+                    s_ = (r - t) % w
+                    for qi, ki, diag in blocks(r, t, w, causal, "zigzag"):
+                        qc, kc = oracle.zigzag_chunks(r, w)[qi], oracle.zigzag_chunks(s_, w)[ki]
+                        seen[(qc, kc)] = seen.get((qc, kc), 0) + 1
+                        if diag != (causal and qc == kc):
+                            return False
+                        pairs += C * (C + 1) // 2 if diag else C * C
+                work.append((causal, pairs))
+            want = {(a, b) for a in range(2 * w) for b in range(2 * w) if not causal or b <= a}
+            if set(seen) != want or any(n != 1 for n in seen.values()):
+                return False
+        causal_work = [p for c, p in work if c]
+        if len(set(causal_work)) != 1:
+            return False
+    return True
+
+
+def test_zigzag_ring_pins():
+    assert _zigzag_pins_pass(oracle.ring_attention_forward, oracle.ring_attention_backward, oracle.ring_blocks)
+
+
+def test_contiguous_ring_is_unbalanced_under_the_causal_mask():
+    """The reason for the zigzag layout: with contiguous shards rank W-1 does W blocks, rank 0 one."""
+    w = 4
+    n = [len([1 for t in range(w) for _ in oracle.ring_blocks(r, t, w, True)]) for r in range(w)]
+    assert n == [1, 2, 3, 4]
+    z = [sum(2 if not diag else 1 for t in range(w) for (_, _, diag) in oracle.ring_blocks(r, t, w, True, "zigzag"))
+         for r in range(w)]
+    assert len(set(z)) == 1  # full blocks count 2 half-blocks, diagonal ones 1: equal for every rank
+
+
+def test_zigzag_pins_catch_planted_mistakes():
+    def blocks_variant(chunks, skip_side="greater", diag_rule=True):
+        def blocks(rank, step, world, causal, layout="contiguous"):
+            s_ = (rank - step) % world
+            out = []
+            for qi, qc in enumerate(chunks(rank, world)):
+                for ki, kc in enumerate(chunks(s_, world)):
+                    if causal and ((kc > qc) if skip_side == "greater" else (kc < qc)):
+                        continue
+                    out.append((qi, ki, causal and kc == qc if diag_rule else False))
+            return out
+        return blocks
+
+    def ring_pair(chunks, **kw):
+        blocks = blocks_variant(chunks, **kw)
+
+        def parts(L, world):
+            C = L // (2 * world)
+            return [[(c * C, (c + 1) * C) for c in chunks(r, world)] for r in range(world)]
+
+        def fwd(q, k, v, scale, causal, world, layout):
+            Q, K, V = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+            L, H, d = Q.shape
+            po = parts(L, world)
+            O, LSE = np.zeros((L, H, d)), np.full((L, H), -np.inf)
+            for r in range(world):
+                acc = [[] for _ in po[r]]
+                for t in range(world):
+                    s_ = (r - t) % world
+                    for qi, ki, diag in blocks(r, t, world, causal):
+                        rows, cols = slice(*po[r][qi]), slice(*po[s_][ki])
+                        acc[qi].append(oracle.attention_forward(Q[rows], K[cols], V[cols], scale, diag))
+                for qi, (a, b) in enumerate(po[r]):
+                    if acc[qi]:
+                        O[a:b], LSE[a:b] = oracle.merge_attention_partials(acc[qi])
+            return O, LSE
+
+        def bwd(q, k, v, do, scale, causal, world, layout):
+            return oracle.ring_attention_backward(q, k, v, do, scale, causal, world, layout)
+        return fwd, bwd, blocks
+
+    good = ring_pair(oracle.zigzag_chunks)
+    assert _zigzag_pins_pass(*good)  # the restatement passes
+    shifted = lambda r, w: (r, (2 * w - 2 - r) % (2 * w))  # the second chunk off by one
+    for bad in (ring_pair(shifted), ring_pair(oracle.zigzag_chunks, skip_side="less"),
+                ring_pair(oracle.zigzag_chunks, diag_rule=False)):
+        assert not _zigzag_pins_pass(*bad)
