@@ -19,6 +19,14 @@ after one more step.
 The per-rank state (``RingAttention``) is separate from the transport (``ring_attention_forward``),
 so the same per-step code runs under NCCL, under another backend, or with the ranks of a ring laid
 side by side in one process.
+
+Shard layouts (``layout``): "contiguous" as above, or "zigzag" for a balanced causal ring — the
+sequence is cut into 2W equal chunks and rank r holds chunks r and 2W − 1 − r (one from each end,
+concatenated in that order).  A block is then a pair of chunks (the rank's query chunk, the held
+shard's key chunk): the causal diagonal when they are the same chunk, full when the key chunk comes
+first, skipped when it comes later.  Every rank computes the same number of full blocks per step
+(two), where with contiguous shards rank W − 1 computes W blocks and rank 0 one.
+``zigzag_shard`` / ``zigzag_unshard`` convert between a whole sequence and the ranks' shards.
 """
 
 from __future__ import annotations
@@ -27,6 +35,56 @@ import math
 from typing import Callable, Optional, Tuple
 
 from . import FA_OK, FAError, attention_forward, attention_merge, dtype_code, lib
+
+
+def zigzag_chunks(rank: int, world: int) -> Tuple[int, int]:
+    """Global chunk indices (of 2·world) held by `rank` in the zigzag layout, in shard order."""
+    return rank, 2 * world - 1 - rank
+
+
+def zigzag_shard(x, rank: int, world: int):
+    """Rank `rank`'s zigzag shard [2C, ...] of a whole sequence x [L, ...] (L = 2·world·C)."""
+    import torch
+    C = x.shape[0] // (2 * world)
+    a, b = zigzag_chunks(rank, world)
+    return torch.cat([x[a * C:(a + 1) * C], x[b * C:(b + 1) * C]]).contiguous()
+
+
+def zigzag_unshard(shards):
+    """The whole sequence from the ranks' zigzag shards (the inverse of ``zigzag_shard``)."""
+    import torch
+    world = len(shards)
+    C = shards[0].shape[0] // 2
+    chunks = [None] * (2 * world)
+    for r, sh in enumerate(shards):
+        a, b = zigzag_chunks(r, world)
+        chunks[a], chunks[b] = sh[:C], sh[C:]
+    return torch.cat(chunks)
+
+
+def ring_blocks(rank: int, step: int, world: int, causal: bool, layout: str = "contiguous"):
+    """The blocks rank `rank` computes at step `step` on the shard of rank (rank − step) mod world:
+    a list of (query part, key part, kind) with kind "causal" (a diagonal block) or "full"; parts index
+    the halves of a zigzag shard, or are 0 (the whole shard) in the contiguous layout."""
+    if layout == "contiguous":
+        _, kind = ring_block(rank, step, world, causal)
+        return [] if kind is None else [(0, 0, kind)]
+    if layout != "zigzag":
+        raise ValueError("layout must be 'contiguous' or 'zigzag'")
+    src = (rank - step) % world
+    out = []
+    for qi, qc in enumerate(zigzag_chunks(rank, world)):
+        for ki, kc in enumerate(zigzag_chunks(src, world)):
+            if causal and kc > qc:
+                continue
+            out.append((qi, ki, "causal" if causal and kc == qc else "full"))
+    return out
+
+
+def _part(x, i: int, nparts: int):
+    """Part i of nparts equal row ranges of x (a contiguous view)."""
+    n = x.shape[0] // nparts
+    return x[i * n:(i + 1) * n]
 
 
 def ring_block(rank: int, step: int, world: int, causal: bool) -> Tuple[int, Optional[str]]:
@@ -53,51 +111,61 @@ class RingAttention:
     0 … world−1 (in order), then ``result()`` → (O [S, H, d] in q's dtype, LSE [S, H] fp32).
 
     ``block_fn(q, k, v, causal, scale, out, lse)`` computes one block and ``merge_fn(acc_o, acc_lse,
-    part_o, part_lse, out, first)`` folds it in; both default to the library's kernels.
+    part_o, part_lse, out, first)`` folds it in; both default to the library's kernels.  ``layout``:
+    "contiguous" or "zigzag" (see the module docstring); each query part keeps its own running result.
     """
 
     def __init__(self, q, rank: int, world: int, causal: bool, scale: Optional[float] = None,
-                 block_fn: Optional[Callable] = None, merge_fn: Optional[Callable] = None):
+                 block_fn: Optional[Callable] = None, merge_fn: Optional[Callable] = None,
+                 layout: str = "contiguous"):
         import torch
         S, H, d = q.shape
-        self.q, self.rank, self.world, self.causal = q, rank, world, causal
+        self.q, self.rank, self.world, self.causal, self.layout = q, rank, world, causal, layout
+        self.np = 1 if layout == "contiguous" else 2  # query / key parts per shard
+        if S % self.np:
+            raise ValueError("a zigzag shard holds two equal chunks")
         self.scale = 1.0 / math.sqrt(d) if scale is None else scale
         self.block_fn = block_fn or _default_block
         self.merge_fn = merge_fn or _default_merge
-        steps = [t for t in range(world) if ring_block(rank, t, world, causal)[1] is not None]
-        self.last = steps[-1]
-        self.n_parts = len(steps)
-        self.done = 0
+        # per query part: the blocks that feed it, in ring order (the last writes the output dtype)
+        self.feeds = [[(t, ki, kind) for t in range(world) for qi, ki, kind in ring_blocks(rank, t, world, causal,
+                                                                                           layout) if qi == p]
+                      for p in range(self.np)]
+        self.done = [0] * self.np
         self.out = torch.empty_like(q)
         self.lse = torch.empty((S, H), dtype=torch.float32, device=q.device)  # the running LSE, then the result
-        if self.n_parts > 1:
+        if any(len(f) > 1 for f in self.feeds):
             self.acc_o = torch.empty((S, H, d), dtype=torch.float32, device=q.device)
             self.part_o = torch.empty_like(q)
             self.part_lse = torch.empty((S, H), dtype=torch.float32, device=q.device)
 
     def consume(self, step: int, k, v) -> None:
-        _, kind = ring_block(self.rank, step, self.world, self.causal)
-        if kind is None:
-            return
-        causal = kind == "causal"
-        if self.n_parts == 1:  # one block: it is the result
-            self.block_fn(self.q, k, v, causal, self.scale, self.out, self.lse)
-        else:
-            self.block_fn(self.q, k, v, causal, self.scale, self.part_o, self.part_lse)
-            self.merge_fn(self.acc_o, self.lse, self.part_o, self.part_lse,
-                          self.out if step == self.last else None, self.done == 0)
-        self.done += 1
+        n = self.np
+        for qi, ki, kind in ring_blocks(self.rank, step, self.world, self.causal, self.layout):
+            q, kk, vv = _part(self.q, qi, n), _part(k, ki, n), _part(v, ki, n)
+            out, lse = _part(self.out, qi, n), _part(self.lse, qi, n)
+            causal = kind == "causal"
+            if len(self.feeds[qi]) == 1:  # one block: it is the result
+                self.block_fn(q, kk, vv, causal, self.scale, out, lse)
+            else:
+                po, pl = _part(self.part_o, qi, n), _part(self.part_lse, qi, n)
+                self.block_fn(q, kk, vv, causal, self.scale, po, pl)
+                last = self.done[qi] == len(self.feeds[qi]) - 1
+                self.merge_fn(_part(self.acc_o, qi, n), lse, po, pl, out if last else None, self.done[qi] == 0)
+            self.done[qi] += 1
 
     def result(self):
-        if self.done != self.n_parts:
+        if any(dn != len(f) for dn, f in zip(self.done, self.feeds)):
             raise RuntimeError("not every step's shard has been consumed")
         return self.out, self.lse
 
 
 def ring_attention_forward(q, k, v, causal: bool = False, scale: Optional[float] = None, group=None,
-                           block_fn: Optional[Callable] = None, merge_fn: Optional[Callable] = None):
-    """O and LSE of this rank's queries; q, k, v are this rank's contiguous shard [S, H, d] of one
-    sequence of W·S tokens, W the size of ``group`` (the default process group when None)."""
+                           block_fn: Optional[Callable] = None, merge_fn: Optional[Callable] = None,
+                           layout: str = "contiguous"):
+    """O and LSE of this rank's queries; q, k, v are this rank's shard [S, H, d] of one sequence of W·S
+    tokens (``layout``: contiguous, or zigzag as made by ``zigzag_shard``), W the size of ``group``
+    (the default process group when None)."""
     import torch
     import torch.distributed as dist
 
@@ -105,7 +173,7 @@ def ring_attention_forward(q, k, v, causal: bool = False, scale: Optional[float]
     rank = dist.get_rank(group)
     peer = (lambda r: r) if group is None else (lambda r: dist.get_global_rank(group, r))
     nxt, prv = peer((rank + 1) % world), peer((rank - 1) % world)
-    ra = RingAttention(q, rank, world, causal, scale, block_fn, merge_fn)
+    ra = RingAttention(q, rank, world, causal, scale, block_fn, merge_fn, layout)
     # received shards alternate between two buffers, so the caller's k and v are only ever sent
     bufs = [(torch.empty_like(k), torch.empty_like(v)) for _ in range(min(2, world - 1))]
     cur_k, cur_v = k, v
@@ -128,23 +196,32 @@ class RingAttentionBackward:
     """One rank's backward state.  Call ``consume(step, k, v, dk_acc, dv_acc)`` with the shard held at
     each step and the fp32 dK/dV accumulators travelling with it (``new_accumulators()`` makes the
     rank's own, consumed at step 0), then ``finish(dk_acc, dv_acc)`` with the accumulators of its own
-    shard once they are home → (dq, dk, dv) in q's dtype.  o, lse: the ring forward's result."""
+    shard once they are home → (dq, dk, dv) in q's dtype.  o, lse: the ring forward's result; ``layout``
+    as for the forward (each query part of a zigzag shard has its own dQ accumulator)."""
 
-    def __init__(self, q, o, lse, do, rank: int, world: int, causal: bool, scale: Optional[float] = None):
+    def __init__(self, q, o, lse, do, rank: int, world: int, causal: bool, scale: Optional[float] = None,
+                 layout: str = "contiguous"):
         import torch
         S, H, d = q.shape
         self.q, self.o, self.lse, self.do = q, o, lse, do
-        self.rank, self.world, self.causal = rank, world, causal
+        self.rank, self.world, self.causal, self.layout = rank, world, causal, layout
+        self.np = 1 if layout == "contiguous" else 2
+        if S % self.np:
+            raise ValueError("a zigzag shard holds two equal chunks")
         self.S, self.H, self.d = S, H, d
+        self.C = S // self.np  # rows of a part
         self.scale = 1.0 / math.sqrt(d) if scale is None else scale
         self.dt = dtype_code(q)
         self.stream = torch.cuda.current_stream(q.device).cuda_stream
-        self.ws_bytes = lib.fa_bwd_workspace_bytes(S, H, d)
-        self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=q.device)
-        self.tmp_dk, self.tmp_dv = torch.empty_like(q), torch.empty_like(q)
-        # D = rowsum(dO ∘ O) of the global output and a zeroed dQ accumulator
-        self._check(lib.fa_bwd_preprocess(o.data_ptr(), do.data_ptr(), 1, H, S, d, None, S, self.dt, self.ws.data_ptr(),
-                                          self.ws_bytes, self.stream), "fa_bwd_preprocess")
+        self.ws_bytes = lib.fa_bwd_workspace_bytes(self.C, H, d)
+        self.ws = [torch.empty(self.ws_bytes, dtype=torch.uint8, device=q.device) for _ in range(self.np)]
+        tmp = torch.empty((self.C, H, d), dtype=q.dtype, device=q.device)
+        self.tmp_dk, self.tmp_dv = tmp, torch.empty_like(tmp)
+        # per query part: D = rowsum(dO ∘ O) of the global output and a zeroed dQ accumulator
+        for i in range(self.np):
+            self._check(lib.fa_bwd_preprocess(_part(o, i, self.np).data_ptr(), _part(do, i, self.np).data_ptr(), 1, H,
+                                              self.C, d, None, self.C, self.dt, self.ws[i].data_ptr(), self.ws_bytes,
+                                              self.stream), "fa_bwd_preprocess")
 
     @staticmethod
     def _check(st, where):
@@ -162,23 +239,29 @@ class RingAttentionBackward:
                                       self.stream), "fa_accumulate")
 
     def consume(self, step: int, k, v, dk_acc, dv_acc) -> None:
-        _, kind = ring_block(self.rank, step, self.world, self.causal)
-        if kind is None:
-            return  # the accumulators pass on unchanged
-        self._check(lib.fa_bwd_main(self.q.data_ptr(), k.data_ptr(), v.data_ptr(), self.lse.data_ptr(),
-                                    self.do.data_ptr(), self.tmp_dk.data_ptr(), self.tmp_dv.data_ptr(), 1, self.H,
-                                    self.S, self.d, float(self.scale), int(kind == "causal"), None, self.S, self.dt,
-                                    self.ws.data_ptr(), self.ws_bytes, self.stream), "fa_bwd_main")
-        # step 0 is the rank's own shard, always computed: it starts the shard's accumulators
-        self._acc(dk_acc, self.tmp_dk, None, step == 0)
-        self._acc(dv_acc, self.tmp_dv, None, step == 0)
+        n, started = self.np, set()
+        for qi, ki, kind in ring_blocks(self.rank, step, self.world, self.causal, self.layout):
+            self._check(lib.fa_bwd_main(_part(self.q, qi, n).data_ptr(), _part(k, ki, n).data_ptr(),
+                                        _part(v, ki, n).data_ptr(), _part(self.lse, qi, n).data_ptr(),
+                                        _part(self.do, qi, n).data_ptr(), self.tmp_dk.data_ptr(),
+                                        self.tmp_dv.data_ptr(), 1, self.H, self.C, self.d, float(self.scale),
+                                        int(kind == "causal"), None, self.C, self.dt, self.ws[qi].data_ptr(),
+                                        self.ws_bytes, self.stream), "fa_bwd_main")
+            # step 0 is the rank's own shard, whose every key part is computed: the first block on a key
+            # part starts the shard's accumulators there
+            first = step == 0 and ki not in started
+            started.add(ki)
+            self._acc(_part(dk_acc, ki, n), self.tmp_dk, None, first)
+            self._acc(_part(dv_acc, ki, n), self.tmp_dv, None, first)
+        # (a step with no block passes the accumulators on unchanged)
 
     def finish(self, dk_acc, dv_acc):
         import torch
         dq = torch.empty_like(self.q)
-        self._check(lib.fa_bwd_postprocess(dq.data_ptr(), 1, self.H, self.S, self.d, float(self.scale), None, self.S,
-                                           self.dt, self.ws.data_ptr(), self.ws_bytes, self.stream),
-                    "fa_bwd_postprocess")
+        for i in range(self.np):
+            self._check(lib.fa_bwd_postprocess(_part(dq, i, self.np).data_ptr(), 1, self.H, self.C, self.d,
+                                               float(self.scale), None, self.C, self.dt, self.ws[i].data_ptr(),
+                                               self.ws_bytes, self.stream), "fa_bwd_postprocess")
         dk, dv = torch.empty_like(self.q), torch.empty_like(self.q)
         self._acc(dk_acc, None, dk, False)
         self._acc(dv_acc, None, dv, False)
@@ -186,9 +269,10 @@ class RingAttentionBackward:
 
 
 def ring_attention_backward(q, k, v, o, lse, do, causal: bool = False, scale: Optional[float] = None, group=None,
-                            state=None):
-    """dq, dk, dv of this rank's shards for the ring forward that produced (o, lse) on the same group.
-    ``state`` replaces the rank's RingAttentionBackward (an object with the same three methods)."""
+                            state=None, layout: str = "contiguous"):
+    """dq, dk, dv of this rank's shards for the ring forward that produced (o, lse) on the same group
+    (with the same ``layout``).  ``state`` replaces the rank's RingAttentionBackward (an object with the
+    same three methods)."""
     import torch
     import torch.distributed as dist
 
@@ -196,7 +280,7 @@ def ring_attention_backward(q, k, v, o, lse, do, causal: bool = False, scale: Op
     rank = dist.get_rank(group)
     peer = (lambda r: r) if group is None else (lambda r: dist.get_global_rank(group, r))
     nxt, prv = peer((rank + 1) % world), peer((rank - 1) % world)
-    rb = state if state is not None else RingAttentionBackward(q, o, lse, do, rank, world, causal, scale)
+    rb = state if state is not None else RingAttentionBackward(q, o, lse, do, rank, world, causal, scale, layout)
     if world == 1:
         acc = rb.new_accumulators()
         rb.consume(0, k, v, *acc)

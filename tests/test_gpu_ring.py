@@ -159,3 +159,52 @@ def test_ring_attention_backward_matches_single_call(fa):
     g_one = fa.attention_backward(q, k, v, o1, l1, do, causal=True, scale=inp.scale)
     for a, b, r in zip(g_ring, g_one, ref):
         assert rel_l2(f64(a), r) <= GRAD_TOL and rel_l2(f64(a), f64(b)) <= GRAD_TOL
+
+
+# ----------------------------------------------------------------------------- load-balanced (zigzag) layout
+
+
+def _ring_zigzag(q, k, v, do, world, causal, scale):
+    """The zigzag ring, forward and (with do) backward, ranks side by side; results in sequence order."""
+    from exact_io_aware_90_b200.ring import RingAttention, RingAttentionBackward, zigzag_shard, zigzag_unshard
+    sh = lambda x, r: zigzag_shard(x, r, world)
+    ras = [RingAttention(sh(q, r), r, world, causal, scale, layout="zigzag") for r in range(world)]
+    held = [(sh(k, r), sh(v, r)) for r in range(world)]
+    for t in range(world):
+        for r in range(world):
+            ras[r].consume(t, *held[r])
+        held = [held[(r - 1) % world] for r in range(world)]
+    outs = [ra.result() for ra in ras]
+    o, lse = zigzag_unshard([x for x, _ in outs]), zigzag_unshard([x for _, x in outs])
+    if do is None:
+        return o, lse, None
+    rbs = [RingAttentionBackward(sh(q, r), outs[r][0], outs[r][1], sh(do, r), r, world, causal, scale,
+                                 layout="zigzag") for r in range(world)]
+    held = [(sh(k, r), sh(v, r)) + rbs[r].new_accumulators() for r in range(world)]
+    for t in range(world):
+        for r in range(world):
+            rbs[r].consume(t, *held[r])
+        held = [held[(r - 1) % world] for r in range(world)]
+    grads = [rbs[r].finish(held[r][2], held[r][3]) for r in range(world)]
+    return o, lse, [zigzag_unshard([g[i] for g in grads]) for i in range(3)]
+
+
+@pytest.mark.parametrize("world", [2, 4])
+@pytest.mark.parametrize("C", [64, 150])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_zigzag_ring_emulated(fa, world, C, d, causal):
+    """The load-balanced ring (chunks r and 2W−1−r per rank, chunk-pair blocks) against the oracle's
+    attention and gradients over the whole sequence."""
+    from _gpu import GRAD_TOL, rel_l2
+    L = 2 * world * C
+    inp = workloads.random_inputs(2, d, "bf16", seed=970 + world + C + d + int(causal), B=1, N=L, causal=causal)
+    dev = torch.device("cuda")
+    q, k, v, do = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev), inp.do.to(dev)
+    o, lse, grads = _ring_zigzag(q, k, v, do, world, causal, inp.scale)
+    O_ref, L_ref = oracle.attention_forward(inp.q, inp.k, inp.v, inp.scale, causal)
+    assert max_abs(f64(o), O_ref) <= O_TOL
+    assert max_abs(f64(lse), L_ref) <= LSE_TOL
+    ref = oracle.attention_backward(inp.q, inp.k, inp.v, inp.do, inp.scale, causal)
+    for name, g, r in zip(("dq", "dk", "dv"), grads, ref):
+        assert rel_l2(f64(g), r) <= GRAD_TOL, (name, rel_l2(f64(g), r))

@@ -109,9 +109,10 @@ class _OracleBackwardState:
     """The per-rank backward steps done by the fp64 oracle on CPU tensors (the same blocks as the
     kernels: P from the global LSE, D from the global O)."""
 
-    def __init__(self, q, o, lse, do, rank, world, causal, scale):
+    def __init__(self, q, o, lse, do, rank, world, causal, scale, layout="contiguous"):
         self.q, self.o, self.lse, self.do = (x.double().numpy() for x in (q, o, lse, do))
-        self.rank, self.world, self.causal, self.scale = rank, world, causal, scale
+        self.rank, self.world, self.causal, self.scale, self.layout = rank, world, causal, scale, layout
+        self.np = 1 if layout == "contiguous" else 2
         self.D = (self.do * self.o).sum(axis=-1)
         self.dq = np.zeros_like(self.q)
 
@@ -119,20 +120,20 @@ class _OracleBackwardState:
         return torch.zeros(self.q.shape, dtype=torch.float32), torch.zeros(self.q.shape, dtype=torch.float32)
 
     def consume(self, step, k, v, dk_acc, dv_acc):
-        from exact_io_aware_90_b200.ring import ring_block
-        _, kind = ring_block(self.rank, step, self.world, self.causal)
-        if kind is None:
-            return
+        from exact_io_aware_90_b200.ring import ring_blocks
         K, V = k.double().numpy(), v.double().numpy()
-        S = self.q.shape[0]
-        for h in range(self.q.shape[1]):
-            P = np.exp((self.q[:, h] @ K[:, h].T) * self.scale - self.lse[:, h][:, None])
-            if kind == "causal":
-                P[np.triu_indices(S, k=1)] = 0.0
-            dS = P * (self.do[:, h] @ V[:, h].T - self.D[:, h][:, None])
-            self.dq[:, h] += self.scale * (dS @ K[:, h])
-            dk_acc[:, h] += torch.from_numpy(self.scale * (dS.T @ self.q[:, h])).float()
-            dv_acc[:, h] += torch.from_numpy(P.T @ self.do[:, h]).float()
+        C = self.q.shape[0] // self.np
+        for qi, ki, kind in ring_blocks(self.rank, step, self.world, self.causal, self.layout):
+            rq, rk = slice(qi * C, (qi + 1) * C), slice(ki * C, (ki + 1) * C)
+            for h in range(self.q.shape[1]):
+                Q, Kp, Vp, dO = self.q[rq, h], K[rk, h], V[rk, h], self.do[rq, h]
+                P = np.exp((Q @ Kp.T) * self.scale - self.lse[rq, h][:, None])
+                if kind == "causal":
+                    P[np.triu_indices(C, k=1)] = 0.0
+                dS = P * (dO @ Vp.T - self.D[rq, h][:, None])
+                self.dq[rq, h] += self.scale * (dS @ Kp)
+                dk_acc[rk, h] += torch.from_numpy(self.scale * (dS.T @ Q)).float()
+                dv_acc[rk, h] += torch.from_numpy(P.T @ dO).float()
 
     def finish(self, dk_acc, dv_acc):
         return torch.from_numpy(self.dq), dk_acc.double(), dv_acc.double()
@@ -222,3 +223,89 @@ def test_ring_single_rank_gloo():
     err = q.get(timeout=120)
     p.join(timeout=60)
     assert p.exitcode == 0 and err < 1e-5, err
+
+
+# ----------------------------------------------------------------------------- load-balanced (zigzag) layout
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("causal", [False, True])
+def test_zigzag_schedule(world, causal):
+    """Every visible (query chunk, key chunk) pair is computed exactly once over the ring, with the
+    diagonal pairs causal; under the causal mask every rank computes two full blocks per step (the
+    diagonal ones of step 0 counting half each); the shards cut a sequence and put it back."""
+    from exact_io_aware_90_b200.ring import ring_blocks, zigzag_chunks, zigzag_shard, zigzag_unshard
+    seen = {}
+    for r in range(world):
+        work = []
+        for t in range(world):
+            src = (r - t) % world
+            w_t = 0.0
+            for qi, ki, kind in ring_blocks(r, t, world, causal, "zigzag"):
+                qc, kc = zigzag_chunks(r, world)[qi], zigzag_chunks(src, world)[ki]
+                seen[(qc, kc)] = seen.get((qc, kc), 0) + 1
+                assert kind == ("causal" if causal and qc == kc else "full")
+                w_t += 0.5 if kind == "causal" else 1.0
+            work.append(w_t)
+        if causal:
+            assert work == [2.0] * world
+    want = {(a, b) for a in range(2 * world) for b in range(2 * world) if not causal or b <= a}
+    assert set(seen) == want and all(n == 1 for n in seen.values())
+    x = torch.arange(2 * world * 3 * 2, dtype=torch.float32).reshape(2 * world * 3, 2)
+    shards = [zigzag_shard(x, r, world) for r in range(world)]
+    assert torch.equal(zigzag_unshard(shards), x)
+    assert torch.equal(shards[0][:3], x[:3]) and torch.equal(shards[0][3:], x[-3:])
+
+
+def _rank_main_zigzag(rank, world, port, causal, out_q):
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        import oracle
+        from exact_io_aware_90_b200.ring import ring_attention_backward, ring_attention_forward, zigzag_shard
+        L, H, d = 2 * world * 5, 2, 8
+        g = np.random.default_rng(17)
+        q, k, v, do = (torch.from_numpy(g.standard_normal((L, H, d))) for _ in range(4))
+        sh = lambda x: zigzag_shard(x, rank, world)
+        ks, vs = sh(k), sh(v)
+        k0, v0 = ks.clone(), vs.clone()
+        o, lse = ring_attention_forward(sh(q), ks, vs, causal=causal, scale=0.35, block_fn=_oracle_block,
+                                        merge_fn=_oracle_merge, layout="zigzag")
+        O_ref, L_ref = oracle.attention_forward(q.numpy(), k.numpy(), v.numpy(), 0.35, causal)
+        t = lambda x: torch.from_numpy(np.ascontiguousarray(x))
+        err = max(float(np.abs(o.numpy() - sh(t(O_ref)).numpy()).max()),
+                  float(np.abs(lse.numpy() - sh(t(L_ref)).numpy()).max()))
+        state = _OracleBackwardState(sh(q), sh(t(O_ref)), sh(t(L_ref)), sh(do), rank, world, causal, 0.35, "zigzag")
+        grads = ring_attention_backward(sh(q), ks, vs, sh(t(O_ref)), sh(t(L_ref)), sh(do), causal=causal,
+                                        state=state, layout="zigzag")
+        ref = oracle.attention_backward(q.numpy(), k.numpy(), v.numpy(), do.numpy(), 0.35, causal)
+        gerr = max(float(np.abs(a.numpy() - sh(t(b)).numpy()).max()) for a, b in zip(grads, ref))
+        untouched = bool(torch.equal(ks, k0) and torch.equal(vs, v0))
+        dist.barrier()
+        out_q.put((rank, err, gerr, untouched))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+@pytest.mark.parametrize("causal", [False, True])
+def test_zigzag_ring_gloo(world, causal):
+    """The zigzag ring's forward and backward over gloo (oracle steps injected): every rank's shard of
+    O, LSE and the gradients equals the oracle's over the whole sequence, cut the same way."""
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main_zigzag, args=(r, world, port, causal, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = [q.get(timeout=180) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, err, gerr, untouched in got:
+        assert err < 1e-5 and gerr < 1e-5, (rank, err, gerr)
+        assert untouched, rank
