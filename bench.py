@@ -62,7 +62,9 @@ def load_peaks():
 KERNEL_SOURCES = {
     "fa_fwd_kernel": ["fa_fwd.cu", "sm100.cuh", "fa_internal.h"],
     "fa_bwd_main_kernel": ["fa_bwd.cu", "sm100.cuh", "fa_internal.h"],
+    "fa_bwd_dropout": ["fa_bwd.cu", "sm100.cuh", "fa_internal.h"],
     "fa_decode_split_kernel": ["fa_decode.cu", "sm100.cuh", "fa_internal.h"],
+    "fa_merge_kernel": ["fa_merge.cu", "sm100.cuh", "fa_internal.h"],
 }
 
 
@@ -605,6 +607,105 @@ def run_gpu_decode(args, world, rank, local, pg):
     return out
 
 
+MERGE_WORKLOADS = {"ring_merge_t32k_h16_d128": dict(T=32768, H=16, d=128, dtype="bf16", seed=1009)}
+
+
+def run_gpu_merge(args, world, rank, local, pg):
+    """The ring path's elementwise kernels (HBM-bound) at the headline's token count: the merge of a
+    normalised block result into the fp32 running (O, LSE), the last merge straight into the output dtype,
+    and the fp32 accumulation of a dK/dV block part.  GB/s of algorithmic bytes against the HBM peak."""
+    import torch
+
+    import exact_io_aware_90_b200 as fa
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    w = MERGE_WORKLOADS[args.workload]
+    T, H, d = w["T"], w["H"], w["d"]
+    g = torch.Generator().manual_seed(w["seed"] + 1000 * rank)
+    tdt = torch.bfloat16 if w["dtype"] == "bf16" else torch.float16
+    part_o = torch.randn(T, H, d, generator=g).to(tdt).to(dev)
+    part_lse = torch.randn(T, H, generator=g).to(dev)
+    acc_o = torch.randn(T, H, d, generator=g).to(dev)
+    acc_lse = torch.randn(T, H, generator=g).to(dev)
+    out_o = torch.empty_like(part_o)
+    acc = torch.randn(T * H * d, generator=g).to(dev)
+    dt = fa.dtype_code(part_o)
+    n, rows = T * H * d, T * H
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def merge(first_out):
+        st = fa.fa_attn_merge(acc_o.data_ptr(), acc_lse.data_ptr(), part_o.data_ptr(), part_lse.data_ptr(),
+                              out_o.data_ptr() if first_out else None, T, H, d, dt, 0, sp)
+        if st != fa.FA_OK:
+            raise fa.FAError(st, "fa_attn_merge")
+
+    def accumulate():
+        st = fa.fa_accumulate(acc.data_ptr(), part_o.data_ptr(), None, n, dt, 0, sp)
+        if st != fa.FA_OK:
+            raise fa.FAError(st, "fa_accumulate")
+
+    # algorithmic bytes per launch: a running merge reads the part (2 B) and the fp32 accumulator and writes
+    # it back (4 + 4 B) per element, and per row reads the part LSE and reads and writes the running LSE;
+    # the last merge writes the output dtype (2 B) instead of the accumulator; the accumulation reads the
+    # fp32 accumulator and the part and writes the accumulator back
+    kernels = [("fa_merge_kernel (running)", lambda: merge(False), n * 10 + rows * 12),
+               ("fa_merge_kernel (last)", lambda: merge(True), n * 8 + rows * 12),
+               ("fa_accum_kernel", accumulate, n * 10)]
+    for _ in range(args.warmup):
+        for _, fn, _ in kernels:
+            flush.fill_(1)
+            fn()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(dev)
+    if pg is not None:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    times = {name: [] for name, _, _ in kernels}
+    for _ in range(args.steps):
+        for name, fn, _ in kernels:
+            flush.fill_(1)  # outside the timed events
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            times[name].append((a, b))
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    st = fa.fa_check_device_status(sp)
+    if st != fa.FA_OK:
+        raise fa.FAError(st, "timed steps")
+    peaks = load_peaks()
+    per = {}
+    for name, _, nbytes in kernels:
+        ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in times[name]])), pg, dev)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        per[name] = {"ms": round(ms, 4), "bytes": nbytes, "gbs": round(gbs, 1), "frac": round(gbs / peaks["hbm_gbs"], 4)}
+    step_ms = sum(v["ms"] for v in per.values())
+    step_bytes = sum(nb for _, _, nb in kernels)
+    value = world * step_bytes / (step_ms * 1e-3) / 1e9
+    dom = max(per, key=lambda k: per[k]["ms"])
+    return {
+        "metric": "ring-merge kernels: algorithmic HBM GB/s", "value": round(value, 1), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w["dtype"],
+        "data": "synthetic: N(0,1) partial O and running O/LSE from a seeded CPU generator",
+        "config": {"workload": args.workload, "T": T, "H": H, "d": d, "step": "merge (running) + merge (last) + "
+                   "accumulate", "l2": "flushed before every launch (256 MiB write, outside the events)",
+                   "parallelism": f"replicas x{world} (independent workloads per GPU)"},
+        "kernels": per,
+        "roofline": {"kernel": dom, "bound": "hbm", "achieved": per[dom]["gbs"], "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": per[dom]["frac"], "traffic": load_traffic("fa_merge_kernel", args.workload),
+                     "peak_source": peaks["source"]},
+        "e2e": None,
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk,
+    }
+
+
 def real_inputs(inp):
     """e4m3 inputs as the float64 values they stand for (NumPy, so the oracle widens nothing through
     float32: e4m3 × an fp32 descale needs up to 28 significand bits)."""
@@ -745,7 +846,7 @@ def cpu_baseline_decode(inp, budget_s=15.0):
     while n < inp.B and tot_t < budget_s:
         dt, f = decode_oracle_seq(inp, n)
         tot_t, tot_f, n = tot_t + dt, tot_f + f, n + 1
-    return {"value": round(tot_f / max(tot_t, 1e-9) / 1e12, 6), "unit": "TFLOP/s", "cores": blas_threads(),
+    return {"value": round(tot_f / max(tot_t, 1e-9) / 1e12, 6), "unit": "TFLOP/s", **host_threads(),
             "kind": "oracle", "sample": f"fp64 NumPy oracle decode of {n} whole sequence(s), all heads, {tot_t:.2f} s"}
 
 
@@ -767,7 +868,7 @@ def run_reference_decode(args):
         "ms_per_step": round(ms, 2), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic",
         "config": {"workload": args.workload, "B": inp.B, "H": inp.H, "Nk": inp.Nk, "d": inp.d, "sample": "sequence 0"},
-        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", **host_threads(), "kind": "oracle",
                          "sample": "fp64 NumPy oracle decode of sequence 0 (all heads) per step"},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -782,6 +883,13 @@ def blas_threads():
     except Exception:
         pass
     return len(os.sched_getaffinity(0))
+
+
+def host_threads():
+    """The oracle's thread counts: `cores` = the threads its work ran on (NumPy's BLAS pool; the rest of
+    the oracle is single-threaded), beside the cores this process may run on and the BLAS pool size."""
+    n = blas_threads()
+    return {"cores": n, "cores_available": len(os.sched_getaffinity(0)), "blas_threads": n}
 
 
 def oracle_sample(inp, rows, head=0):
@@ -814,7 +922,7 @@ def cpu_baseline(inp, budget_s=15.0):
         heads += 1
         if tot_t >= budget_s:
             break
-    return {"value": round(tot_f / tot_t / 1e12, 6), "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+    return {"value": round(tot_f / tot_t / 1e12, 6), "unit": "TFLOP/s", **host_threads(), "kind": "oracle",
             "sample": f"fp64 NumPy oracle, {'fwd+bwd' if inp.do is not None else 'fwd'} of {heads} whole head(s) of "
                       f"sequence 0 ({L} query rows x all visible keys each), {tot_t:.2f} s"}
 
@@ -848,15 +956,48 @@ def dropout_sample_rows(inp, p, budget_s):
 def cpu_baseline_dropout(inp, p, budget_s=15.0):
     R = dropout_sample_rows(inp, p, budget_s / 2)
     dt, f = oracle_sample_dropout(inp, R, p)
-    return {"value": round(f / dt / 1e12, 6), "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+    return {"value": round(f / dt / 1e12, 6), "unit": "TFLOP/s", **host_threads(), "kind": "oracle",
             "sample": f"fp64 NumPy dropout oracle (p = {p}), {'fwd+bwd' if inp.do is not None else 'fwd'} of one head "
                       f"of the first {R} tokens of sequence 0 as a sequence of that length, {dt:.2f} s"}
+
+
+def run_reference_merge(args):
+    """The oracle's merge of two normalised partials on a bounded sample of (token, head) rows per step."""
+    import torch
+
+    import oracle
+    w = MERGE_WORKLOADS[args.workload]
+    rows, d = 65536, w["d"]  # 1/8 of the workload's 524 288 rows per step
+    g = torch.Generator().manual_seed(w["seed"])
+    a_o, b_o = (torch.randn(rows, d, generator=g).double().numpy() for _ in range(2))
+    a_l, b_l = (torch.randn(rows, generator=g).double().numpy() for _ in range(2))
+    for _ in range(args.warmup):
+        oracle.merge_attention_partials([(a_o, a_l), (b_o, b_l)])
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.merge_attention_partials([(a_o, a_l), (b_o, b_l)])
+        times.append(time.perf_counter() - t0)
+    ms = 1e3 * float(np.mean(times))
+    nbytes = rows * d * 10 + rows * 12  # the GPU arm's count for a running merge of as many rows
+    value = nbytes / (ms * 1e-3) / 1e9
+    return {
+        "impl": "reference", "metric": "ring-merge kernels: algorithmic HBM GB/s", "value": round(value, 3),
+        "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "sample_rows": rows, "d": d},
+        "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", **host_threads(), "kind": "oracle",
+                         "sample": f"fp64 NumPy oracle merge of two normalised partials over {rows} rows per step"},
+        "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
 
 
 def run_reference(args, rank):
     import workloads
     if args.workload in workloads.DECODE_WORKLOADS:
         return run_reference_decode(args)
+    if args.workload in MERGE_WORKLOADS:
+        return run_reference_merge(args)
     spec = workloads.WORKLOADS[args.workload]
     inp = workloads.make_workload(args.workload, backward=spec["backward"])
     metric = METRIC
@@ -890,7 +1031,7 @@ def run_reference(args, rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": args.workload, "B": inp.B, "H": inp.H, "N": inp.N, "d": inp.d,
                    "causal": inp.causal, "sample_rows": rows},
-        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", **host_threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -915,10 +1056,48 @@ def run_reference_dropout(args, inp):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": args.workload, "B": inp.B, "H": inp.H, "N": inp.N, "d": inp.d,
                    "causal": inp.causal, "dropout_p": p, "sample_tokens": R},
-        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", **host_threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
+
+
+# The five workloads the headline metric is quoted on (the default workload is the headline itself); each
+# is measured by the same step as the headline, with fewer steps, and summarised in the `configs` object.
+CONFIG_WORKLOADS = ["tiny_d64", "mha_n4k_d64", "causal_n8k_d128", "varlen_causal_d128", "long_n128k_d128"]
+
+
+def config_summary(r):
+    """Compact per-workload entry: step time, TFLOP/s and fraction of the measured peak, per kernel."""
+    peaks = load_peaks()
+    e = {"workload": r["config"]["workload"], "step": r["config"]["step"], "dtype": r["dtype"],
+         "ms_per_step": r["ms_per_step"], "tflops": round(r["value"] / r["n_gpus"], 1),
+         "frac_of_peak": round(r["value"] / r["n_gpus"] / peaks["bf16_tflops"], 4),
+         "kernels": r.get("kernels"), "clocks": r.get("clocks")}
+    if r["config"].get("dropout_p"):
+        e["dropout_p"] = r["config"]["dropout_p"]
+    if r["config"]["workload"] == "tiny_d64":
+        e["us_per_step"] = round(1e3 * r["ms_per_step"], 1)  # launch-latency bound: no roofline claim
+    return e
+
+
+def run_configs(args, world, rank, local, pg, headline):
+    """The other spec workloads and the dropout step, measured after the headline."""
+    import copy
+    out = {}
+    for name in CONFIG_WORKLOADS + ["causal_n8k_d128+dropout0.1"]:
+        if name == headline["config"]["workload"] and not headline["config"].get("dropout_p"):
+            out[name] = config_summary(headline)
+            continue
+        a = copy.copy(args)
+        a.workload, a.dropout = (name.split("+")[0], 0.1) if "+dropout" in name else (name, 0.0)
+        a.steps = min(args.steps, 5)
+        a.no_cpu_baseline = True
+        try:
+            out[name] = config_summary(run_gpu(a, world, rank, local, pg))
+        except Exception as exc:  # a failed extra config must not lose the headline line
+            out[name] = {"workload": name, "error": f"{type(exc).__name__}: {exc}"}
+    return out
 
 
 def main():
@@ -932,6 +1111,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--dropout", type=float, default=0.0,
                     help="dropout probability on P (attention workloads; 0 = the plain step)")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other workloads' summary (the `configs` object of the default line)")
     args = ap.parse_args()
     if not (0.0 <= args.dropout < 1.0):
         ap.error("--dropout must be in [0, 1)")
@@ -954,10 +1135,14 @@ def main():
         import workloads
         if args.workload in workloads.DECODE_WORKLOADS:
             out = run_gpu_decode(args, world, rank, local, pg)
+        elif args.workload in MERGE_WORKLOADS:
+            out = run_gpu_merge(args, world, rank, local, pg)
         elif workloads.WORKLOADS[args.workload]["dtype"] == "e4m3":
             out = run_gpu_fp8(args, world, rank, local, pg)
         else:
             out = run_gpu(args, world, rank, local, pg)
+            if args.workload == DEFAULT_WORKLOAD and args.dropout == 0.0 and not args.no_configs:
+                out["configs"] = run_configs(args, world, rank, local, pg, out)
         if rank == 0:
             print(json.dumps(out), flush=True)
     finally:
