@@ -778,12 +778,18 @@ constexpr int kBwd128Threads = 512;  // 4 warpgroups
 // Column pairs i (of 32 per query half) with bit (i % 8) set take the FMA-pipe exp2 in unmasked halves.
 constexpr uint32_t kBwd128PolyMask = 0x00u;
 
+template <int D>
 struct Bq128 {
-  static constexpr int D = 128, BQ = 128;
+  static constexpr int BQ = 128;
+  static constexpr int NCH = D / 64;           // 64-feature (128-byte) chunks per row
   static constexpr uint32_t CHUNK = 128 * 128;  // [128 rows × 64 features], 128-byte swizzle
-  static constexpr uint32_t TILE = 2 * CHUNK;   // [128 rows × 128 features]
+  static constexpr uint32_t TILE = NCH * CHUNK;  // [128 rows × D features]
+  // d = 64: dQ (= dS K, lane = query) has tensor-memory columns of its own; d = 128: dQᵀ (= Kᵀ dSᵀ,
+  // lane = feature) is written over Sᵀ once the next Sᵀ is in registers
+  static constexpr bool DQ_OWN = (D == 64);
   // tensor memory columns
-  static constexpr uint32_t T_S = 0, T_P = 0, T_DQ = 0, T_DP = 128, T_DS = 128, T_DK = 256, T_DV = 384;
+  static constexpr uint32_t T_S = 0, T_P = 0, T_DP = 128, T_DS = 128, T_DK = 256, T_DV = 256 + D;
+  static constexpr uint32_t T_DQ = DQ_OWN ? 256 + 2 * D : 0;
   // barriers
   static constexpr int B_KVFULL = 0;    // K, V of the unit landed
   static constexpr int B_KVEMPTY = 1;   // K, V no longer read (the unit's last MMAs done)
@@ -799,7 +805,7 @@ struct Bq128 {
   static constexpr int B_PREADY = 14;   // [2] half a of Pᵀ in tensor memory (128 arrivals)
   static constexpr int B_DSREADY = 16;  // [2] half a of dSᵀ in tensor and shared memory (128 arrivals)
   static constexpr int B_DQFULL = 18;
-  static constexpr int B_DQFREE = 19;   // dQᵀ read out of [0, 128) (128 arrivals)
+  static constexpr int B_DQFREE = 19;   // the dQ partial read out of tensor memory (128 arrivals)
   static constexpr int B_DKV = 20;      // dK, dV of the unit complete
   static constexpr int B_DKVFREE = 21;  // dK, dV read out of tensor memory (128 arrivals)
   static constexpr int B_UFULL = 22;    // [2] work-unit ring slot written
@@ -809,13 +815,13 @@ struct Bq128 {
   static constexpr int NBARS = 28;
   static constexpr int UNIT_READERS = 14;  // compute warps 0-7, dQ warps 8-11, MMA warp 13, row-term warp 14
   // shared memory: K, V resident; Q double-buffered; dO single (its next tile loads once dV has read
-  // it, well before the next dPᵀ); dSᵀ as two [128 keys × 64 queries] chunks (B operand of dQᵀ)
+  // it, well before the next dPᵀ); dSᵀ as two [128 keys × 64 queries] chunks (operand of the dQ product)
   static constexpr uint32_t OFF_K = 0;
   static constexpr uint32_t OFF_V = TILE;
   static constexpr uint32_t OFF_Q = 2 * TILE;
   static constexpr uint32_t OFF_DO = 4 * TILE;
   static constexpr uint32_t OFF_DS = 5 * TILE;
-  static constexpr uint32_t OFF_DQS = 6 * TILE;  // dQ staging: per dQ warp two boxes [32 queries × 32 fp32]
+  static constexpr uint32_t OFF_DQS = OFF_DS + 2 * CHUNK;  // dQ staging: per dQ warp two boxes [32 rows × 32 fp32]
   static constexpr uint32_t DQ_BOX = 32 * 128;
   static constexpr uint32_t OFF_ROW = OFF_DQS + 8 * DQ_BOX;  // per stage: −LSE·log2 e [128], −D [128] (fp32)
   static constexpr uint32_t OFF_CLC = OFF_ROW + 2 * 2 * BQ * 4;  // 16-byte scheduler response
@@ -881,16 +887,18 @@ __device__ __forceinline__ bool decode_bwd_unit(const BwdParams& p, int unit, Bw
   return true;
 }
 
-template <bool BF16>
+template <int D, bool BF16>
 __global__ void __launch_bounds__(kBwd128Threads, 1)
     fa_bwd_main_q128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                             const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
-  using C = Bq128;
+  using C = Bq128<D>;
   constexpr int BQ = C::BQ;
-  constexpr uint32_t IDESC_ST = idesc_f16(BF16, kBK, BQ, false, false);    // Sᵀ = K Qᵀ, dPᵀ = V dOᵀ
-  constexpr uint32_t IDESC_DKV = idesc_f16(BF16, kBK, C::D, false, true);  // dV += Pᵀ dO, dK += dSᵀ Q
-  constexpr uint32_t IDESC_DQ = idesc_f16(BF16, C::D, BQ, true, true);     // dQᵀ = Kᵀ dSᵀ
+  constexpr uint32_t IDESC_ST = idesc_f16(BF16, kBK, BQ, false, false);  // Sᵀ = K Qᵀ, dPᵀ = V dOᵀ
+  constexpr uint32_t IDESC_DKV = idesc_f16(BF16, kBK, D, false, true);   // dV += Pᵀ dO, dK += dSᵀ Q
+  // d = 128: dQᵀ = Kᵀ dSᵀ (M = 128 features, N = 128 queries); d = 64: dQ = dS K (M = 128 queries,
+  // N = 64 features); both operands MN-major
+  constexpr uint32_t IDESC_DQ = C::DQ_OWN ? idesc_f16(BF16, BQ, D, true, true) : idesc_f16(BF16, D, BQ, true, true);
 
   extern __shared__ __align__(1024) uint8_t smem_aligned[];
   uint8_t* smem = smem_aligned;
@@ -1033,7 +1041,7 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
         if (kvn > 0 && !warp_wait_b(bar(C::B_KVEMPTY), (kvn - 1) & 1, wd)) break;
         if (elect_one()) {
           mbar_arrive_expect_tx(bar(C::B_KVFULL), 2 * C::TILE);
-          for (int c = 0; c < 2; ++c) {
+          for (int c = 0; c < C::NCH; ++c) {
             tma_load_3d(sK + c * C::CHUNK, &tm_k, bar(C::B_KVFULL), c * 64, U.h, U.tok0 + U.k0, pol_kv);
             tma_load_3d(sV + c * C::CHUNK, &tm_v, bar(C::B_KVFULL), c * 64, U.h, U.tok0 + U.k0, pol_kv);
           }
@@ -1043,7 +1051,7 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
         // the next unit, its K and V on their way into L2
         const int nxt = next_valid(steal(), N);
         if (nxt >= 0 && elect_one()) {
-          for (int c = 0; c < 2; ++c) {
+          for (int c = 0; c < C::NCH; ++c) {
             tma_prefetch_l2_3d(&tm_k, c * 64, N.h, N.tok0 + N.k0);
             tma_prefetch_l2_3d(&tm_v, c * 64, N.h, N.tok0 + N.k0);
           }
@@ -1055,7 +1063,7 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
           if (qn >= 2 && !warp_wait_b(bar(C::B_QEMPTY + s), ((qn >> 1) - 1) & 1, wd)) { ok = false; break; }
           if (elect_one()) {
             mbar_arrive_expect_tx(bar(C::B_QFULL + s), C::TILE);
-            for (int c = 0; c < 2; ++c)
+            for (int c = 0; c < C::NCH; ++c)
               tma_load_3d(sQ + s * C::TILE + c * C::CHUNK, &tm_q, bar(C::B_QFULL + s), c * 64, U.h, U.tok0 + i0,
                           pol_q);
           }
@@ -1065,7 +1073,7 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
           if (don > 0 && !warp_wait_b(bar(C::B_DOEMPTY), (don - 1) & 1, wd)) { ok = false; break; }
           if (elect_one()) {
             mbar_arrive_expect_tx(bar(C::B_DOFULL), C::TILE);
-            for (int c = 0; c < 2; ++c)
+            for (int c = 0; c < C::NCH; ++c)
               tma_load_3d(sDO + c * C::CHUNK, &tm_do, bar(C::B_DOFULL), c * 64, U.h, U.tok0 + i0, pol_q);
           }
           __syncwarp();
@@ -1118,8 +1126,10 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
       const uint64_t dK_kmaj = sdesc_sw128(sK, 16, 1024), dV_kmaj = sdesc_sw128(sV, 16, 1024);
       const uint64_t dQ_kmaj = sdesc_sw128(sQ, 16, 1024), dDO_kmaj = sdesc_sw128(sDO, 16, 1024);
       const uint64_t dQ_mn = sdesc_sw128(sQ, C::CHUNK, 1024), dDO_mn = sdesc_sw128(sDO, C::CHUNK, 1024);
-      const uint64_t dKt_mn = sdesc_sw128(sK, C::CHUNK, 1024);  // Kᵀ: MN-major A of dQᵀ (features contiguous)
-      const uint64_t dDS_mn = sdesc_sw128(sDS, C::CHUNK, 1024);  // dSᵀ: MN-major B of dQᵀ (queries contiguous)
+      // dQ operands, both MN-major, +2 KB per 16 keys: d = 128: A = Kᵀ (features contiguous), B = dSᵀ
+      // (queries contiguous, two 64-query chunks); d = 64: A = dS (queries contiguous), B = K
+      const uint64_t dK_mn = sdesc_sw128(sK, C::CHUNK, 1024), dDS_mn = sdesc_sw128(sDS, C::CHUNK, 1024);
+      const uint64_t dq_a = C::DQ_OWN ? dDS_mn : dK_mn, dq_b = C::DQ_OWN ? dK_mn : dDS_mn;
       constexpr uint32_t TILE16 = C::TILE >> 4;
       constexpr uint32_t HALF16 = (64 * 128) >> 4;  // 64 rows of a chunk: query half 1 of Q / dO
       uint32_t g = 0;   // steps so far (all units); step g uses Q stage g mod 2 and the g-th dO tile
@@ -1132,13 +1142,14 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
         // Sᵀ and dPᵀ of the unit's first step: K and V in shared memory; [0, 128) released by the read-out
         // of the previous unit's last dQᵀ ([128, 256) was read by its last dK, issued before)
         ok = warp_wait_b(bar(C::B_KVFULL), u & 1, wd) && warp_wait_b(bar(C::B_QFULL + (g & 1)), (g >> 1) & 1, wd) &&
-             (g == 0 || warp_wait_b(bar(C::B_DQFREE), (g - 1) & 1, wd)) && warp_wait_b(bar(C::B_DOFULL), g & 1, wd);
+             (C::DQ_OWN || g == 0 || warp_wait_b(bar(C::B_DQFREE), (g - 1) & 1, wd)) &&
+             warp_wait_b(bar(C::B_DOFULL), g & 1, wd);
         if (!ok) break;
         tc_fence_after();
         if (elect_one()) {
-          bwd_issue_kt<C::D, BQ, IDESC_ST>(tS, dK_kmaj, dQ_kmaj + (g & 1) * TILE16);
+          bwd_issue_kt<D, BQ, IDESC_ST>(tS, dK_kmaj, dQ_kmaj + (g & 1) * TILE16);
           tc_commit(bar(C::B_SFULL));
-          bwd_issue_kt<C::D, BQ, IDESC_ST>(tDP, dV_kmaj, dDO_kmaj);
+          bwd_issue_kt<D, BQ, IDESC_ST>(tDP, dV_kmaj, dDO_kmaj);
           tc_commit(bar(C::B_DPFULL));
         }
         __syncwarp();
@@ -1165,10 +1176,10 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
           // dQᵀ of the previous step has been read out
           if (more) {
             if (!warp_wait_b(bar(C::B_QFULL + (g1 & 1)), (g1 >> 1) & 1, wd) ||
-                (g > 0 && !warp_wait_b(bar(C::B_DQFREE), (g - 1) & 1, wd))) { ok = false; break; }
+                (!C::DQ_OWN && g > 0 && !warp_wait_b(bar(C::B_DQFREE), (g - 1) & 1, wd))) { ok = false; break; }
             tc_fence_after();
             if (elect_one()) {
-              bwd_issue_kt<C::D, BQ, IDESC_ST>(tS, dK_kmaj, dQ_kmaj + (g1 & 1) * TILE16);
+              bwd_issue_kt<D, BQ, IDESC_ST>(tS, dK_kmaj, dQ_kmaj + (g1 & 1) * TILE16);
               tc_commit(bar(C::B_SFULL));
             }
             __syncwarp();
@@ -1182,11 +1193,13 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
             break;
           }
           tc_fence_after();
-          const bool dq_first = !more || warp_test_b(bar(C::B_SREAD), g1 & 1);
+          // (d = 64: dQ has columns of its own, free once the previous dQ has been read out)
+          const bool dq_first = C::DQ_OWN || !more || warp_test_b(bar(C::B_SREAD), g1 & 1);
+          if (C::DQ_OWN && g > 0 && !warp_wait_b(bar(C::B_DQFREE), (g - 1) & 1, wd)) { ok = false; break; }
           if (dq_first) {
             tc_fence_after();
             if (elect_one()) {
-              bwd_issue_dq128<IDESC_DQ>(tDQ, dKt_mn, dDS_mn);
+              bwd_issue_dq128<IDESC_DQ>(tDQ, dq_a, dq_b);
               tc_commit(bar(C::B_DQFULL));
             }
             __syncwarp();
@@ -1200,7 +1213,7 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
             if (!warp_wait_b(bar(C::B_SREAD), g1 & 1, wd)) { ok = false; break; }
             tc_fence_after();
             if (elect_one()) {
-              bwd_issue_dq128<IDESC_DQ>(tDQ, dKt_mn, dDS_mn);
+              bwd_issue_dq128<IDESC_DQ>(tDQ, dq_a, dq_b);
               tc_commit(bar(C::B_DQFULL));
             }
             __syncwarp();
@@ -1210,7 +1223,7 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
             if (!warp_wait_b(bar(C::B_DOFULL), g1 & 1, wd)) { ok = false; break; }
             tc_fence_after();
             if (elect_one()) {
-              bwd_issue_kt<C::D, BQ, IDESC_ST>(tDP, dV_kmaj, dDO_kmaj);
+              bwd_issue_kt<D, BQ, IDESC_ST>(tDP, dV_kmaj, dDO_kmaj);
               tc_commit(bar(C::B_DPFULL));
             }
             __syncwarp();
@@ -1291,7 +1304,8 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
         }
         // packed over [32a, 32a + 32): for a = 1 those are Sᵀ columns of half 0, so both halves must have
         // been read first, and dQᵀ of the previous step (written there after that) must have been read out
-        if (!warp_wait_b(bar(C::B_SREAD), g & 1, wd) || (g > 0 && !warp_wait_b(bar(C::B_DQFREE), (g - 1) & 1, wd))) {
+        if (!warp_wait_b(bar(C::B_SREAD), g & 1, wd) ||
+            (!C::DQ_OWN && g > 0 && !warp_wait_b(bar(C::B_DQFREE), (g - 1) & 1, wd))) {
           ok = false;
           break;
         }
@@ -1358,34 +1372,67 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
         const int i0 = (U.i_begin + it) * BQ;
         if (!warp_wait_b(bar(C::B_DQFULL), g & 1, wd)) { ok = false; break; }
         tc_fence_after();
-        // the whole partial into registers (lane = feature 32·quarter + lane, columns = queries), so that
-        // [0, 128) is released at once; staging and the reduce-adds follow at their own pace
-        uint32_t qr[128];
-        tmem_ld64(tDQ, reinterpret_cast<uint32_t(&)[64]>(qr[0]));
-        tmem_ld64(tDQ + 64u, reinterpret_cast<uint32_t(&)[64]>(qr[64]));
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(bar(C::B_DQFREE));
+        if constexpr (!C::DQ_OWN) {
+          // dQᵀ: the whole partial into registers (lane = feature 32·quarter + lane, columns = queries), so
+          // that [0, 128) is released at once; staging and the reduce-adds follow at their own pace
+          uint32_t qr[128];
+          tmem_ld64(tDQ, reinterpret_cast<uint32_t(&)[64]>(qr[0]));
+          tmem_ld64(tDQ + 64u, reinterpret_cast<uint32_t(&)[64]>(qr[64]));
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(bar(C::B_DQFREE));
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int q0 = i0 + 32 * c;
-          if (q0 >= U.L) break;  // the rest of the step lies past the sequence: nothing to add
-          const uint32_t bx = box_base + (pieces & 1u) * C::DQ_BOX;
-          // the box may be rewritten once the reduce issued from it two pieces ago has read it
-          if (lane == 0) bulk_wait_group_read<1>();
-          __syncwarp();
+          for (int c = 0; c < 4; ++c) {
+            const int q0 = i0 + 32 * c;
+            if (q0 >= U.L) break;  // the rest of the step lies past the sequence: nothing to add
+            const uint32_t bx = box_base + (pieces & 1u) * C::DQ_BOX;
+            // the box may be rewritten once the reduce issued from it two pieces ago has read it
+            if (lane == 0) bulk_wait_group_read<1>();
+            __syncwarp();
 #pragma unroll
-          for (int q = 0; q < 32; ++q)
-            st_shared_f32(bx + q * 128 + (((lane >> 2) ^ (q & 7)) << 4) + ((lane & 3) << 2), qr[32 * c + q]);
-          fence_proxy_async_smem();
-          __syncwarp();
-          // rows past the sequence hold exact zeros (P is 0 there); rows past T are clipped by the TMA unit
-          if (lane == 0) {
-            tma_reduce_add_3d(&tm_dq, bx, 32 * quarter, U.h, U.tok0 + q0);
-            bulk_commit_group();
+            for (int q = 0; q < 32; ++q)
+              st_shared_f32(bx + q * 128 + (((lane >> 2) ^ (q & 7)) << 4) + ((lane & 3) << 2), qr[32 * c + q]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            // rows past the sequence hold exact zeros (P is 0 there); rows past T are clipped by the TMA unit
+            if (lane == 0) {
+              tma_reduce_add_3d(&tm_dq, bx, 32 * quarter, U.h, U.tok0 + q0);
+              bulk_commit_group();
+            }
+            __syncwarp();
+            ++pieces;
           }
-          __syncwarp();
-          ++pieces;
+        } else {
+          // dQ: lane = query 32·quarter + lane of the step, columns = the 64 features; this warp's 32 query
+          // rows go out as two boxes of 32 features
+          uint32_t qr[64];
+          tmem_ld64(tDQ, qr);
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(bar(C::B_DQFREE));
+          const int q0 = i0 + 32 * quarter;
+          if (q0 < U.L) {
+            // both boxes may be rewritten once the reduces issued from them last step have read them
+            if (lane == 0) bulk_wait_group_read<0>();
+            __syncwarp();
+#pragma unroll
+            for (int bx_i = 0; bx_i < 2; ++bx_i) {
+              const uint32_t row = box_base + bx_i * C::DQ_BOX + lane * 128;
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                st_shared_v4(row + ((j ^ (lane & 7)) << 4), qr[32 * bx_i + 4 * j], qr[32 * bx_i + 4 * j + 1],
+                             qr[32 * bx_i + 4 * j + 2], qr[32 * bx_i + 4 * j + 3]);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            // rows past the sequence hold exact zeros (P is 0 there); rows past T are clipped by the TMA unit
+            if (lane == 0) {
+              tma_reduce_add_3d(&tm_dq, box_base, 0, U.h, U.tok0 + q0);
+              tma_reduce_add_3d(&tm_dq, box_base + C::DQ_BOX, 32, U.h, U.tok0 + q0);
+              bulk_commit_group();
+            }
+            __syncwarp();
+          }
         }
       }
       if (!ok) break;
@@ -1395,18 +1442,18 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
       tc_fence_after();
       const int key = U.k0 + 32 * quarter + lane;
       const bool valid = key < U.L;
-      uint8_t* dk_row = reinterpret_cast<uint8_t*>(p.dk) + (((size_t)(U.tok0 + (valid ? key : 0)) * p.H + U.h) * C::D) * 2;
-      uint8_t* dv_row = reinterpret_cast<uint8_t*>(p.dv) + (((size_t)(U.tok0 + (valid ? key : 0)) * p.H + U.h) * C::D) * 2;
+      uint8_t* dk_row = reinterpret_cast<uint8_t*>(p.dk) + (((size_t)(U.tok0 + (valid ? key : 0)) * p.H + U.h) * D) * 2;
+      uint8_t* dv_row = reinterpret_cast<uint8_t*>(p.dv) + (((size_t)(U.tok0 + (valid ? key : 0)) * p.H + U.h) * D) * 2;
 #pragma unroll 1
       for (int t = 0; t < 2; ++t) {  // dK, then dV
         const float f = t == 0 ? p.scale : 1.f;
         uint8_t* row = t == 0 ? dk_row : dv_row;
 #pragma unroll
-        for (int q = 0; q < C::D / 32; ++q) {
+        for (int q = 0; q < D / 32; ++q) {
           uint32_t r32[32];
           tmem_ld32((t == 0 ? tDK : tDV) + 32u * q, r32);
           tmem_wait_ld();
-          if (t == 1 && q == C::D / 32 - 1) {
+          if (t == 1 && q == D / 32 - 1) {
             tc_fence_before();
             mbar_arrive(bar(C::B_DKVFREE));  // dK and dV read out: the next unit may overwrite them
           }
@@ -1514,11 +1561,11 @@ static cudaError_t launch_main_t(const Problem& pb, const BwdArgs& a, cudaStream
   return cudaPeekAtLastError();
 }
 
-template <bool BF16>
+template <int D, bool BF16>
 static cudaError_t launch_main_q128_t(const Problem& pb, const BwdArgs& a, cudaStream_t stream) {
   static std::atomic<unsigned long long> configured{0};  // per instantiation, one bit per device
-  auto kern = fa_bwd_main_q128_kernel<BF16>;
-  if (cudaError_t e = set_smem_once(configured, reinterpret_cast<const void*>(kern), Bq128::SMEM_BYTES);
+  auto kern = fa_bwd_main_q128_kernel<D, BF16>;
+  if (cudaError_t e = set_smem_once(configured, reinterpret_cast<const void*>(kern), Bq128<D>::SMEM_BYTES);
       e != cudaSuccess)
     return e;
   BwdParams p;
@@ -1540,24 +1587,27 @@ static cudaError_t launch_main_q128_t(const Problem& pb, const BwdArgs& a, cudaS
   p.timeout_ns = pb.timeout_ns;
   p.drop = pb.drop;
   const long long units = (long long)pb.B * pb.H * p.num_kblocks;
-  kern<<<dim3((unsigned)units), dim3(kBwd128Threads), Bq128::SMEM_BYTES, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do,
+  kern<<<dim3((unsigned)units), dim3(kBwd128Threads), Bq128<D>::SMEM_BYTES, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do,
                                                                                      a.tm_dq, p);
   return cudaPeekAtLastError();
 }
 
 template <bool DROP>
 static cudaError_t launch_main_d(const Problem& pb, const BwdArgs& a, cudaStream_t stream) {
-  if (pb.d == 128) {
-    if constexpr (!DROP) return pb.bf16 ? launch_main_q128_t<true>(pb, a, stream) : launch_main_q128_t<false>(pb, a, stream);
-    return pb.bf16 ? launch_main_t<128, true, DROP>(pb, a, stream) : launch_main_t<128, false, DROP>(pb, a, stream);
+  if constexpr (!DROP) {
+    if (pb.d == 128)
+      return pb.bf16 ? launch_main_q128_t<128, true>(pb, a, stream) : launch_main_q128_t<128, false>(pb, a, stream);
+    return pb.bf16 ? launch_main_q128_t<64, true>(pb, a, stream) : launch_main_q128_t<64, false>(pb, a, stream);
   }
+  if (pb.d == 128)
+    return pb.bf16 ? launch_main_t<128, true, DROP>(pb, a, stream) : launch_main_t<128, false, DROP>(pb, a, stream);
   return pb.bf16 ? launch_main_t<64, true, DROP>(pb, a, stream) : launch_main_t<64, false, DROP>(pb, a, stream);
 }
 
 // Rows per Q / dO tile the main kernel loads, and per box of its dQ reduce-adds (the host encodes the
 // tensor maps with these box heights).
 int bwd_q_tile_rows(int d, bool dropout) { return (d == 128 && dropout) ? 64 : 128; }
-int bwd_dq_box_rows(int d, bool dropout) { return d == 128 ? (dropout ? 64 : 32) : 128; }
+int bwd_dq_box_rows(int d, bool dropout) { return dropout ? (d == 128 ? 64 : 128) : 32; }
 
 cudaError_t launch_bwd_main(const Problem& pb, const BwdArgs& a, cudaStream_t stream) {
   return pb.drop.t != 0u ? launch_main_d<true>(pb, a, stream) : launch_main_d<false>(pb, a, stream);
