@@ -1303,8 +1303,9 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
           for (int i = 0; i < 32; ++i) pk[i] = pack2<BF16>(pt[2 * i], pt[2 * i + 1]);
         }
         // packed over [32a, 32a + 32): for a = 1 those are Sᵀ columns of half 0, so both halves must have
-        // been read first, and dQᵀ of the previous step (written there after that) must have been read out
-        if (!warp_wait_b(bar(C::B_SREAD), g & 1, wd) ||
+        // been read first (half 0 packs over its own columns), and at d = 128 dQᵀ of the previous step
+        // (written over Sᵀ after that) must have been read out
+        if ((a == 1 && !warp_wait_b(bar(C::B_SREAD), g & 1, wd)) ||
             (!C::DQ_OWN && g > 0 && !warp_wait_b(bar(C::B_DQFREE), (g - 1) & 1, wd))) {
           ok = false;
           break;
@@ -1339,8 +1340,8 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
               make_uint4(dsk[4 * j], dsk[4 * j + 1], dsk[4 * j + 2], dsk[4 * j + 3]);
         fence_proxy_async_smem();
         // packed over [128 + 32a, ...) (A operand of dK): for a = 1 those are dPᵀ columns of half 0, so both
-        // halves must have been read first
-        if (!warp_wait_b(bar(C::B_DPREAD), g & 1, wd)) { ok = false; break; }
+        // halves must have been read first (half 0 packs over its own columns)
+        if (a == 1 && !warp_wait_b(bar(C::B_DPREAD), g & 1, wd)) { ok = false; break; }
         tc_fence_after();
         tmem_st32(tDS, dsk);
         tmem_wait_st();
