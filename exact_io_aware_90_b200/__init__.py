@@ -69,6 +69,7 @@ def _load() -> ctypes.CDLL:
                                P]),
         "fa_fwd_fp8": (I, [P, P, P, P, P, I, I, I, I, F, I, P, I, F, F, F, P]),
         "fa_fwd_fp8_per_head": (I, [P, P, P, P, P, I, I, I, I, F, I, P, I, P, P, P, P]),
+        "fa_fwd_fp8_per_block": (I, [P, P, P, P, P, I, I, I, I, F, I, P, I, P, P, P, I, P]),
         "fa_attn_merge": (I, [P, P, P, P, P, I, I, I, I, I, P]),
         "fa_accumulate": (I, [P, P, P, ctypes.c_longlong, I, I, P]),
         "fa_decode_workspace_bytes": (S, [I, I, I, I]),
@@ -153,6 +154,12 @@ def fa_fwd_fp8_per_head(q, k, v, o, lse, B, H, N, d, scale, causal, cu_seqlens, 
                         v_descale, stream) -> int:
     return lib.fa_fwd_fp8_per_head(q, k, v, o, lse, B, H, N, d, scale, causal, cu_seqlens, total_tokens, q_descale,
                                    k_descale, v_descale, stream)
+
+
+def fa_fwd_fp8_per_block(q, k, v, o, lse, B, H, N, d, scale, causal, cu_seqlens, total_tokens, q_descale, k_descale,
+                         v_descale, num_blocks, stream) -> int:
+    return lib.fa_fwd_fp8_per_block(q, k, v, o, lse, B, H, N, d, scale, causal, cu_seqlens, total_tokens, q_descale,
+                                    k_descale, v_descale, num_blocks, stream)
 
 
 def fa_attn_merge(acc_o, acc_lse, part_o, part_lse, out, T, H, d, dtype, first, stream) -> int:
@@ -294,10 +301,11 @@ def attention_backward(q, k, v, o, lse, do, causal: bool = False, scale: Optiona
 
 def attention_forward_fp8(q, k, v, q_descale: float, k_descale: float, v_descale: float, causal: bool = False,
                           scale: Optional[float] = None, cu_seqlens=None, max_seqlen: Optional[int] = None,
-                          batch: Optional[int] = None, out=None, lse=None, stream=None):
+                          batch: Optional[int] = None, out=None, lse=None, stream=None, per_block: bool = False):
     """O (bf16) and LSE for e4m3 q, k, v of shape [T, H, 128] whose real values are the stored ones times
-    the descales: floats (one per tensor, fa_fwd_fp8) or fp32 CUDA tensors [B, H] (one per sequence and
-    head, fa_fwd_fp8_per_head); see ``include/fa.h``."""
+    the descales: floats (one per tensor, fa_fwd_fp8), fp32 CUDA tensors [B, H] (one per sequence and
+    head, fa_fwd_fp8_per_head) or, with ``per_block``, fp32 CUDA tensors [num_blocks, H] (one per
+    128-token block of each sequence and head, fa_fwd_fp8_per_block); see ``include/fa.h``."""
     import torch
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.float8_e4m3fn or t.shape != q.shape:
@@ -312,7 +320,17 @@ def attention_forward_fp8(q, k, v, q_descale: float, k_descale: float, v_descale
     if stream is None:
         stream = torch.cuda.current_stream(q.device).cuda_stream
     per_head = [hasattr(x, "data_ptr") for x in (q_descale, k_descale, v_descale)]
-    if any(per_head):
+    if per_block:
+        if not all(per_head):
+            raise ValueError("per-block descales must be [num_blocks, H] tensors")
+        nb = q_descale.numel() // H
+        for x in (q_descale, k_descale, v_descale):
+            if not x.is_cuda or x.dtype != torch.float32 or not x.is_contiguous() or x.numel() != nb * H or nb < 1:
+                raise ValueError("per-block descales must be contiguous CUDA float32 tensors of num_blocks·H values")
+        st = lib.fa_fwd_fp8_per_block(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, d, float(scale),
+                                      int(bool(causal)), _ptr(cu_seqlens), T, _ptr(q_descale), _ptr(k_descale),
+                                      _ptr(v_descale), nb, stream)
+    elif any(per_head):
         if not all(per_head):
             raise ValueError("the three descales must all be floats or all be [B, H] tensors")
         for x in (q_descale, k_descale, v_descale):

@@ -105,6 +105,7 @@ static int make_problem(Problem* pb, int B, int H, int N, int d, float scale, in
   pb->qk_descale = 1.f;
   pb->v_descale = 1.f;
   pb->q_descale_bh = pb->k_descale_bh = pb->v_descale_bh = nullptr;
+  pb->descale_blocks = 0;
   return FA_OK;
 }
 
@@ -234,6 +235,33 @@ int fa_fwd_fp8_per_head(const void* q, const void* k, const void* v, void* o, fl
   pb.q_descale_bh = q_descale;
   pb.k_descale_bh = k_descale;
   pb.v_descale_bh = v_descale;
+  FwdArgs a;
+  if (!encode_tmap_e4m3(&a.tm_q, q, pb.T, H, d, 128) || !encode_tmap_e4m3(&a.tm_k, k, pb.T, H, d, 128) ||
+      !encode_tmap_e4m3(&a.tm_v, v, pb.T, H, d, 128))
+    return FA_ERR_UNSUPPORTED;
+  a.o = o;
+  a.lse = lse;
+  return map_launch(launch_fwd(pb, a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int fa_fwd_fp8_per_block(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+                         int d, float scale, int causal, const int32_t* cu_seqlens, int total_tokens,
+                         const float* q_descale, const float* k_descale, const float* v_descale, int num_blocks,
+                         fa_stream_t stream) {
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(lse)) return FA_ERR_INVALID_ARG;
+  if (!aligned4(q_descale) || !aligned4(k_descale) || !aligned4(v_descale)) return FA_ERR_INVALID_ARG;
+  Problem pb;
+  int st = make_problem(&pb, B, H, N, d, scale, causal, cu_seqlens, total_tokens, FA_BF16, true);
+  if (st != FA_OK) return st;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  // dense: every sequence has ceil(N / 128) blocks; varlen: checked per sequence on the device
+  const long long dense_blocks = (long long)B * ((N + 127) / 128);
+  if (num_blocks < 1 || (cu_seqlens == nullptr && num_blocks < dense_blocks)) return FA_ERR_INVALID_ARG;
+  pb.fp8 = true;
+  pb.q_descale_bh = q_descale;
+  pb.k_descale_bh = k_descale;
+  pb.v_descale_bh = v_descale;
+  pb.descale_blocks = num_blocks;
   FwdArgs a;
   if (!encode_tmap_e4m3(&a.tm_q, q, pb.T, H, d, 128) || !encode_tmap_e4m3(&a.tm_k, k, pb.T, H, d, 128) ||
       !encode_tmap_e4m3(&a.tm_v, v, pb.T, H, d, 128))

@@ -63,6 +63,9 @@ struct FwdParams {
   const float* q_descale;
   const float* k_descale;
   const float* v_descale;
+  // > 0: the descale arrays hold one value per (128-token block, head) instead, [num_blocks·H], the
+  // blocks of each sequence numbered after those of the sequences before it
+  int descale_blocks;
   uint64_t timeout_ns;
   Dropout drop;
 };
@@ -77,6 +80,10 @@ constexpr float kRescaleThreshold = 8.0f;
 // the tile, so part of them moves to the FMA pipe.
 template <int D> struct PolyMask { static constexpr uint32_t value = 0x00u; };
 template <> struct PolyMask<64> { static constexpr uint32_t value = 0x22u; };
+// The e4m3 instantiation (d = 128, MMAs at twice the 16-bit rate): the same quarter, in every tile (the
+// polynomial clamps its input at −126, so a masked key's 2^-126 rounds to e4m3 zero and adds nothing
+// visible to ℓ).
+constexpr uint32_t kFp8PolyMask = 0x22u;
 
 // EB = bytes per input element: 2 (f16 / bf16) or 1 (e4m3).
 template <int D, int EB = 2>
@@ -207,6 +214,27 @@ __device__ __forceinline__ bool decode_unit(const FwdParams& p, int unit, FwdUni
   }
   u.n_iter = max(u.nkv[0], u.nkv[1]);
   return true;
+}
+
+// First per-block descale block of the unit's sequence: the ceil(L / 128) blocks of every sequence
+// before it, summed across the warp (warp-collective; every lane gets the sum).
+__device__ __forceinline__ int descale_block0(const FwdParams& p, const FwdUnit& u, int lane) {
+  if (p.cu_seqlens == nullptr) return u.b * ((p.N + kBN - 1) / kBN);
+  int n = 0;
+  for (int b = lane; b < u.b; b += 32) {
+    const int L = __ldg(p.cu_seqlens + b + 1) - __ldg(p.cu_seqlens + b);
+    n += (max(L, 0) + kBN - 1) / kBN;
+  }
+  return __reduce_add_sync(0xffffffffu, n);
+}
+
+// Per-block descales: the unit's blocks must lie inside the arrays (inconsistent offsets are reported
+// and the unit skipped, as decode_unit does for a bad sequence).
+__device__ __forceinline__ bool descale_blocks_ok(const FwdParams& p, const FwdUnit& u, int lane) {
+  if (p.descale_blocks <= 0) return true;
+  const bool ok = descale_block0(p, u, lane) + (u.L + kBN - 1) / kBN <= p.descale_blocks;
+  if (!ok && lane == 0) record_status(1);
+  return ok;
 }
 
 // Warp-uniform non-blocking probe of one barrier phase.
@@ -378,11 +406,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       int unit = blockIdx.x;
       while (ok) {
         FwdUnit U;
-        bool have = decode_unit(p, unit, U);
+        bool have = decode_unit(p, unit, U) && (!FP8 || descale_blocks_ok(p, U, lane));
         while (!have) {  // a unit past the end of its sequence: take the next one
           unit = steal();
           if (unit < 0) break;
-          have = decode_unit(p, unit, U);
+          have = decode_unit(p, unit, U) && (!FP8 || descale_blocks_ok(p, U, lane));
         }
         if (!have) break;
         ok = publish(unit) && load_q(U, 0) && load_k(U, 0) && (U.nkv[1] == 0 || load_q(U, 1)) && load_v(U, 0);
@@ -555,6 +583,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     float c = p.scale_log2;  // per unit when the e4m3 descales are per (sequence, head)
     float2 c2 = make_float2(c, c);
     float o_scale_u = 1.f;   // the unit's v descale in that case (the FP8 instantiation only)
+    float kd_next = 1.f, vd_next = 1.f;  // per-block descales of the next KV tile, loaded a tile ahead
     const uint32_t keep_bias = keep_flag_bias(p.drop.t);  // used by the dropout variant only
     uint32_t un = 0;  // units read
     uint32_t sn = 0;  // S tiles of Q tile t consumed (all units)
@@ -573,9 +602,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       if (my_nkv == 0) continue;
       const int row = U.q0 + t * kBM + 32 * quarter + lane;  // position in the sequence
       const uint32_t drop_bh = (uint32_t)(U.b * p.H + U.h);
+      int blk0 = 0;  // first descale block of this sequence (per-block descales)
       if constexpr (FP8) {
         o_scale_u = p.o_scale;
-        if (p.q_descale != nullptr) {
+        if (p.descale_blocks > 0) {
+          // the producer published the unit only if its blocks lie inside the arrays
+          blk0 = descale_block0(p, U, lane);
+          // q's descale is that of the 128-row block this Q tile is; k's and v's change per KV tile
+          c = p.scale_log2 * __ldg(p.q_descale + (size_t)(blk0 + (U.q0 + t * kBM) / kBM) * p.H + U.h);
+          o_scale_u = 1.f;
+          kd_next = __ldg(p.k_descale + (size_t)blk0 * p.H + U.h);
+          vd_next = __ldg(p.v_descale + (size_t)blk0 * p.H + U.h);
+        } else if (p.q_descale != nullptr) {
           const int bh = U.b * p.H + U.h;
           c = p.scale_log2 * (__ldg(p.q_descale + bh) * __ldg(p.k_descale + bh));
           c2 = make_float2(c, c);
@@ -610,6 +648,23 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             for (int c4 = 0; c4 < 4; ++c4) rw[4 * m + c4] = x[c4];
           }
         }
+        // per-block e4m3 descales of KV tile j: k's folds into this tile's c, v's into P: the tile's P is
+        // formed as 2^(c·s − m + log2 v_descale), ℓ takes it divided by v_descale, and m tracks the
+        // maximum of c·s + log2 v_descale, so that P stays ≤ 256 and O = Σ P V / ℓ needs no factor
+        float lv = 0.f, inv_vd = 1.f;
+        if constexpr (FP8) {
+          if (p.descale_blocks > 0) {
+            const float kd = kd_next, vd = vd_next;
+            if (j + 1 < my_nkv) {  // the next tile's, so that the loads are in flight during this tile
+              const size_t bi = (size_t)(blk0 + j + 1) * p.H + U.h;
+              kd_next = __ldg(p.k_descale + bi);
+              vd_next = __ldg(p.v_descale + bi);
+            }
+            c2 = make_float2(c * kd, c * kd);
+            lv = __log2f(vd);
+            inv_vd = 1.f / vd;
+          }
+        }
         if (!warp_wait(bar(C::B_SFULL + t), step & 1, wd)) { ok = false; break; }
         tc_fence_after();
         // one 128-column load and one 64-column store per tile: fewer, larger tensor-memory accesses
@@ -635,7 +690,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
           for (int k = 0; k < 8; ++k) mx[k] = max3f(mx[k], sv[i + k], sv[i + k + 8]);
         }
-        const float m_tile = max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * c;
+        const float m_tile =
+            max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * c2.x + lv;
         // raise the reference max only when the tile max exceeds it by more than the threshold
         const float m_new = (m_tile > m_ref + kRescaleThreshold) ? m_tile : m_ref;
         const float alpha = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - m_new);
@@ -643,7 +699,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         ell *= alpha;
         m_ref = m_new;
         // a row that has seen no visible key yet keeps m = -inf; its P is 0 either way
-        const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
+        const float neg_m = ((m_ref == -INFINITY) ? 0.f : -m_ref) + lv;
         const float2 nm2 = make_float2(neg_m, neg_m);
         float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         // pair i = keys 2i, 2i + 1 packed to 16 bits each: dropped keys zeroed (the 1/(1 − p) factor is
@@ -657,9 +713,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         auto drop_pair = [&](uint32_t v, int i) -> uint32_t { return DROP ? v & pair_mask(i) : v; };
         if constexpr (FP8) {
           if (!split_p) {
-            // P = 2^(c·s − m) on the MUFU, rounded to e4m3, four keys per 32-bit column, written over S.
-            // (Moving a quarter of the exponentials to the FMA pipe, as at d = 64, measured 18 % slower
-            // here: the softmax warps are latency-bound, not MUFU-bound.)
+            // P = 2^(c·s − m), rounded to e4m3, four keys per 32-bit column, written over S.  The MMAs
+            // take half as long as at 16 bits, so the exponentials bound the tile: a quarter of them go
+            // to the FMA-pipe polynomial (measured 4.8 % faster than all on the MUFU; 1/8 and 3/8 gain
+            // less).
             uint32_t pk[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
@@ -668,7 +725,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               for (int h = 0; h < 2; ++h) {
                 const int pi = 2 * i + h;  // pair index
                 const float2 x = __ffma2_rn(make_float2(sv[2 * pi], sv[2 * pi + 1]), c2, nm2);
-                e[h] = make_float2(ex2(x.x), ex2(x.y));
+                e[h] = ((kFp8PolyMask >> (pi & 7)) & 1u) ? exp2_poly2(x) : make_float2(ex2(x.x), ex2(x.y));
                 acc[pi & 3] = __fadd2_rn(acc[pi & 3], e[h]);
               }
               pk[i] = pack4_e4m3(e[0].x, e[0].y, e[1].x, e[1].y);
@@ -739,7 +796,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           }
         }
         const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
-        ell += a.x + a.y;
+        if constexpr (FP8) ell += (a.x + a.y) * inv_vd;
+        else ell += a.x + a.y;
         if (__any_sync(0xffffffffu, rescale_o)) {
           // The reference max rose (rare past the first tile): O(t) must hold P·V(t, j-1) before it
           // is rescaled, and the rescale must land before P·V(t, j) is issued.
@@ -828,6 +886,7 @@ static cudaError_t launch_fwd_t(const Problem& pb, const FwdArgs& a, cudaStream_
   p.q_descale = pb.q_descale_bh;
   p.k_descale = pb.k_descale_bh;
   p.v_descale = pb.v_descale_bh;
+  p.descale_blocks = pb.descale_blocks;
   p.timeout_ns = pb.timeout_ns;
   p.drop = pb.drop;
   const long long units = (long long)pb.B * pb.H * p.num_qblocks;

@@ -47,10 +47,12 @@ struct Problem {
   bool fp8;
   float qk_descale;  // q descale × k descale
   float v_descale;
-  // or one descale per (sequence, head): fp32 [B·H] device arrays (nullptr: per tensor)
+  // or one descale per (sequence, head): fp32 [B·H] device arrays (nullptr: per tensor), or, when
+  // descale_blocks > 0, one per (128-token block, head): fp32 [descale_blocks·H] device arrays
   const float* q_descale_bh;
   const float* k_descale_bh;
   const float* v_descale_bh;
+  int descale_blocks;
 };
 
 struct FwdArgs {

@@ -251,6 +251,35 @@ int fa_fwd_fp8_per_head(const void* q, const void* k, const void* v, void* o, fl
                         fa_stream_t stream);
 
 /*
+ * fa_fwd_fp8 with one descale per (128-token block, head): the blocks of a
+ * sequence are its tokens [128i, 128i + 128) (the last one ragged), numbered
+ * sequence after sequence, so block i of sequence b is number
+ * n_b + i with n_b = Σ_{b' < b} ceil(L_b' / 128) (dense: b·ceil(N/128) + i).
+ * q_descale, k_descale, v_descale are fp32 device arrays [num_blocks·H],
+ * index (n_b + i)·H + h, 4-byte aligned, read by the kernel (values are not
+ * checked on the host: each must be finite and > 0, else the output is
+ * undefined).  The real value of element (token, h, c) is its e4m3 value ×
+ * the descale of its block and head.
+ * A query tile is one block, so q's descale is folded into its softmax
+ * constant; k's is folded into the constant of each key tile; v's enters the
+ * exponent of each key tile's P as log2(v descale), so the rounded P already
+ * carries it, and the softmax sum takes each tile's P divided by it (the row
+ * maximum tracked is that of scale·s + log2 v descale, which keeps every P
+ * ≤ 256 and leaves O = Σ P V / Σ P unchanged).
+ *   num_blocks  the arrays' length / H: ≥ B·ceil(N/128) for a dense batch
+ *               (FA_ERR_INVALID_ARG otherwise); with cu_seqlens each
+ *               sequence is checked on the device, and one whose blocks
+ *               would lie past num_blocks is skipped and reported as
+ *               inconsistent offsets are (fa_check_device_status).
+ * Other errors as fa_fwd_fp8_per_head.
+ */
+int fa_fwd_fp8_per_block(const void* q, const void* k, const void* v, void* o, float* lse,
+                         int B, int H, int N, int d, float scale, int causal,
+                         const int32_t* cu_seqlens, int total_tokens,
+                         const float* q_descale, const float* k_descale, const float* v_descale,
+                         int num_blocks, fa_stream_t stream);
+
+/*
  * Merge of normalised partial attention results: the same queries attended
  * to disjoint key sets (the blocks a ring of ranks visits in ring /
  * context-parallel attention, "FlashAttention 与算子融合", 工程实践 "与 CP

@@ -33,7 +33,8 @@ def test_header_declares_the_entry_points():
     for n in ["fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_bwd_preprocess", "fa_bwd_main",
               "fa_bwd_postprocess", "fa_check_device_status", "fa_status_string", "fa_set_watchdog_ns",
               "fa_watchdog_selftest", "fa_version", "fa_bwd_noalloc", "fa_decode", "fa_decode_workspace_bytes",
-              "fa_fwd_dropout", "fa_bwd_dropout", "fa_fwd_fp8", "fa_fwd_fp8_per_head", "fa_attn_merge",
+              "fa_fwd_dropout", "fa_bwd_dropout", "fa_fwd_fp8", "fa_fwd_fp8_per_head", "fa_fwd_fp8_per_block",
+              "fa_attn_merge",
               "fa_accumulate"]:
         assert n in names
 
@@ -142,6 +143,21 @@ def test_fp8_per_head_rejects_invalid_arguments(fa):
     assert fa.fa_fwd_fp8_per_head(*([P16] * 5 + [2, 4, 256, 64, 0.125, 0, None, 512]), P16, P16, P16, None) == \
         fa.FA_ERR_UNSUPPORTED
     assert fa.fa_fwd_fp8_per_head(*([P16] * 5 + [2, 4, 256, 128, 0.125, 0, None, 511]), P16, P16, P16, None) == \
+        fa.FA_ERR_INVALID_ARG
+
+
+def test_fp8_per_block_rejects_invalid_arguments(fa):
+    base = [P16] * 5 + [2, 4, 256, 128, 0.125, 0, None, 512]
+    for i, bad in [(0, None), (1, P16 + 2), (2, None)]:  # q, k, v descale arrays: null or misaligned
+        ds = [P16, P16, P16]
+        ds[i] = bad
+        assert fa.fa_fwd_fp8_per_block(*base, *ds, 4, None) == fa.FA_ERR_INVALID_ARG
+    # a dense batch of 2 × 256 tokens has 2·2 blocks: 3 is too few, 0 is never valid
+    assert fa.fa_fwd_fp8_per_block(*base, P16, P16, P16, 3, None) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_fwd_fp8_per_block(*base, P16, P16, P16, 0, None) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_fwd_fp8_per_block(*([P16] * 5 + [2, 4, 256, 64, 0.125, 0, None, 512]), P16, P16, P16, 4, None) == \
+        fa.FA_ERR_UNSUPPORTED
+    assert fa.fa_fwd_fp8_per_block(*([P16] * 5 + [2, 4, 256, 128, 0.125, 0, None, 511]), P16, P16, P16, 4, None) == \
         fa.FA_ERR_INVALID_ARG
 
 

@@ -39,6 +39,9 @@ def fa():
 
 
 def _real(inp):
+    if "descale_blk" in inp.extra:  # one descale per (128-token block, head)
+        ds, segs = inp.extra["descale_blk"], workloads.block_segments(_seq_bounds(inp))
+        return tuple(workloads.real_values(t, ds[n], segs) for t, n in ((inp.q, "q"), (inp.k, "k"), (inp.v, "v")))
     if "descale_bh" in inp.extra:  # one descale per (sequence, head)
         ds, segs = inp.extra["descale_bh"], _seq_bounds(inp)
         return tuple(workloads.real_values(t, ds[n], segs) for t, n in ((inp.q, "q"), (inp.k, "k"), (inp.v, "v")))
@@ -49,17 +52,30 @@ def _real(inp):
 
 def _run(fa, inp, **over):
     dev = torch.device("cuda")
-    if "descale_bh" in inp.extra:
+    per_block = "descale_blk" in inp.extra
+    if per_block or "descale_bh" in inp.extra:
         ds = {n: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(dev)
-              for n, a in inp.extra["descale_bh"].items()}
+              for n, a in inp.extra["descale_blk" if per_block else "descale_bh"].items()}
     else:
         ds = dict(inp.extra["descale"], **over)
     cu = None if inp.cu_seqlens is None else inp.cu_seqlens.to(dev)
     o, lse = fa.attention_forward_fp8(inp.q.to(dev), inp.k.to(dev), inp.v.to(dev), ds["q"], ds["k"], ds["v"],
                                       causal=inp.causal, scale=inp.scale, cu_seqlens=cu,
-                                      max_seqlen=inp.N if cu is not None else None, batch=inp.B)
+                                      max_seqlen=inp.N if cu is not None else None, batch=inp.B,
+                                      per_block=per_block)
     assert fa.fa_check_device_status(torch.cuda.current_stream().cuda_stream) == fa.FA_OK
     return o, lse
+
+
+def _v_descale_per_token(inp):
+    """[T, H] descale of v at every token (None when v has one descale per tensor or per sequence, where
+    the plain bound below applies)."""
+    if "descale_blk" not in inp.extra:
+        return None
+    out = np.ones((inp.T, inp.H))
+    for (s0, L), ds in zip(workloads.block_segments(_seq_bounds(inp)), inp.extra["descale_blk"]["v"]):
+        out[s0:s0 + L] = ds[None, :]
+    return out
 
 
 def _seq_bounds(inp):
@@ -70,9 +86,13 @@ def _seq_bounds(inp):
     return [(cu[b], cu[b + 1] - cu[b]) for b in range(len(cu) - 1)]
 
 
-def _rounding_terms(q, k, v, lse_ref, scale, causal, seqs, rows=None):
+def _rounding_terms(q, k, v, lse_ref, scale, causal, seqs, rows=None, vd=None):
     """For the chosen tokens (all heads): A = Σ_j P|v|, Bt = Σ_j min(P, 2⁻¹⁰)|v|, Q2 = Σ_j P²v², with P
-    from the oracle's LSE (P_ij = exp(scale·q_i·k_j − LSE_i) over the visible keys)."""
+    from the oracle's LSE (P_ij = exp(scale·q_i·k_j − LSE_i) over the visible keys).
+
+    With v descales that differ between key blocks (``vd`` [T, H], the descale of each key) the kernel
+    rounds P_ij·vd_j / W_i, with W_i ≤ M_i = max_j P_ij·vd_j (its row maximum is that of the weighted
+    values), so the flush term becomes Bt = Σ_j min(P_ij|v_j|, 2⁻¹⁰·M_i·|v_j| / vd_j)."""
     T, H, d = q.shape
     A, Bt, Q2 = (np.zeros((T, H, d)) for _ in range(3))
     want = np.ones(T, dtype=bool) if rows is None else np.isin(np.arange(T), rows)
@@ -88,7 +108,13 @@ def _rounding_terms(q, k, v, lse_ref, scale, causal, seqs, rows=None):
                 P = np.where(np.arange(L)[None, :] <= (ti - s0)[:, None], P, 0.0)
             va = np.abs(v[s0:s0 + L, h, :])
             A[ti, h] = P @ va
-            Bt[ti, h] = np.minimum(P, 2.0 ** -10) @ va
+            if vd is None:
+                Bt[ti, h] = np.minimum(P, 2.0 ** -10) @ va
+            else:
+                w = vd[s0:s0 + L, h]                                              # [L]
+                M = np.max(P * w[None, :], axis=1, keepdims=True)                 # [rows, 1]
+                Bt[ti, h] = np.sum(np.minimum(P[:, :, None] * va[None], 2.0 ** -10 * M[:, :, None]
+                                              * (va / w[:, None])[None]), axis=1)
             Q2[ti, h] = (P * P) @ (va * va)
     return A, Bt, Q2
 
@@ -106,7 +132,8 @@ def _check(inp, o, lse, rows=None):
         O_ref, L_ref = np.zeros(q.shape), np.zeros(q.shape[:2])
         O_ref[rows], L_ref[rows] = O_r, L_r
         sel = np.isin(np.arange(inp.T), rows)
-    A, Bt, Q2 = _rounding_terms(q, k, v, L_ref, inp.scale, inp.causal, _seq_bounds(inp), rows)
+    A, Bt, Q2 = _rounding_terms(q, k, v, L_ref, inp.scale, inp.causal, _seq_bounds(inp), rows,
+                                vd=_v_descale_per_token(inp))
     got, gl = f64(o)[sel], f64(lse)[sel]
     err = np.abs(got - O_ref[sel])
     bound = 2.0 ** -4 * A[sel] + Bt[sel] + 2.0 ** -8 * np.abs(O_ref[sel]) + 1e-4
@@ -193,3 +220,78 @@ def test_fp8_per_head_descales(fa, causal, varlen):
                                "per_head", {"descale_bh": {"q": dq, "k": dk, "v": dv}})
     o, lse = _run(fa, inp)
     _check(inp, o, lse)
+
+
+def _per_block_inputs(seqlens, varlen, causal, seed, H=3, d=128):
+    """e4m3 inputs with one descale per (128-token block, head): every block and head drawn at its own
+    magnitude (factors of 2 and 3 apart along heads and blocks, so that one descale per sequence would
+    be far off) and quantised with its own amax/448."""
+    B, N = len(seqlens), max(seqlens)
+    cu = workloads.cu_from_lengths(seqlens) if varlen else None
+    segs = [(int(sum(seqlens[:b])), L) for b, L in enumerate(seqlens)]
+    T = sum(seqlens)
+    g = torch.Generator().manual_seed(seed)
+    mags = []
+    for name in ("q", "k", "v"):
+        mag = torch.ones(T, H, 1)
+        for n, (s0, L) in enumerate(workloads.block_segments(segs)):
+            mag[s0:s0 + L] = (2.0 ** torch.arange(H, dtype=torch.float32))[None, :, None] * (1 + (n + len(name)) % 3)
+        mags.append(mag)
+    (q8, dq), (k8, dk), (v8, dv) = (workloads.quantize_e4m3_per_block(torch.randn(T, H, d, generator=g) * m, segs)
+                                    for m in mags)
+    return workloads.AttnInputs(q8, k8, v8, None, cu, seqlens, B, H, N, d, 0.25 / math.sqrt(d), causal, "e4m3",
+                                "per_block", {"descale_blk": {"q": dq, "k": dk, "v": dv}})
+
+
+@pytest.mark.parametrize("varlen", [False, True])
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp8_per_block_descales(fa, causal, varlen):
+    """One descale per (128-token block, head) (fa_fwd_fp8_per_block): q's per query tile, k's per key
+    tile, v's carried in P, against the oracle on the real values under the e4m3 bounds (the flush term
+    with the weighted row maximum).  The lengths leave ragged last blocks, an empty sequence, and a
+    sequence of one tile."""
+    seqlens = [200, 0, 513, 64] if varlen else [384, 384]
+    inp = _per_block_inputs(seqlens, varlen, causal, seed=71 + int(causal) + 2 * int(varlen))
+    o, lse = _run(fa, inp)
+    _check(inp, o, lse)
+
+
+def test_fp8_per_block_equal_descales_match_per_tensor(fa):
+    """Per-block descales that are all equal compute exactly what the per-tensor call computes (the
+    same folded constant, log2 of the descale added to m and subtracted again through ℓ): compared
+    against fa_fwd_fp8 within the e4m3 rounding of a different but equivalent exponent split."""
+    inp = workloads.random_inputs(2, 128, "e4m3", seed=19, B=2, N=700, causal=True, backward=False)
+    ds = inp.extra["descale"]
+    nb = 2 * ((700 + 127) // 128)
+    blk = {n: np.full((nb, 2), np.float32(ds[n]), dtype=np.float32) for n in ("q", "k", "v")}
+    o1, l1 = _run(fa, inp)
+    pb = workloads.AttnInputs(inp.q, inp.k, inp.v, None, None, inp.seqlens, inp.B, inp.H, inp.N, inp.d, inp.scale,
+                              inp.causal, "e4m3", "per_block", {"descale_blk": blk})
+    o2, l2 = _run(fa, pb)
+    _check(pb, o2, l2)
+    assert float((o1.float() - o2.float()).abs().max()) <= 2.0 ** -3 * float(o1.float().abs().max())
+    assert float((l1 - l2).abs().max()) <= 1e-4
+
+
+def test_fp8_per_block_too_few_blocks_is_reported(fa):
+    """Varlen with descale arrays one block short: the host cannot count the blocks, so the kernel finds
+    the last sequence's blocks past the arrays, skips that sequence and records FA_ERR_INVALID_ARG; the
+    other sequences are computed as usual."""
+    seqlens = [130, 300]
+    inp = _per_block_inputs(seqlens, True, True, seed=5)
+    dev = torch.device("cuda")
+    ds = {n: torch.from_numpy(np.ascontiguousarray(a[:-1], dtype=np.float32)).to(dev)
+          for n, a in inp.extra["descale_blk"].items()}
+    o = torch.full((inp.T, inp.H, inp.d), 7.0, dtype=torch.bfloat16, device=dev)
+    lse = torch.full((inp.T, inp.H), 7.0, dtype=torch.float32, device=dev)
+    fa.attention_forward_fp8(inp.q.to(dev), inp.k.to(dev), inp.v.to(dev), ds["q"], ds["k"], ds["v"], causal=True,
+                             scale=inp.scale, cu_seqlens=inp.cu_seqlens.to(dev), max_seqlen=inp.N, batch=inp.B,
+                             out=o, lse=lse, per_block=True)
+    stream = torch.cuda.current_stream().cuda_stream
+    assert fa.fa_check_device_status(stream) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_check_device_status(stream) == fa.FA_OK  # reading the status clears it
+    assert bool((o[130:].float() == 7.0).all()) and bool((lse[130:] == 7.0).all())  # skipped: untouched
+    q, k, v = _real(inp)
+    O_ref, L_ref = oracle.attention_forward(q[:130], k[:130], v[:130], inp.scale, True, B=1, N=130)
+    assert float(np.max(np.abs(f64(lse[:130]) - L_ref))) <= LSE_TOL
+    assert float(np.max(np.abs(f64(o[:130]) - O_ref))) <= 0.1 * float(np.max(np.abs(O_ref)))

@@ -68,3 +68,25 @@ def test_generators_are_deterministic():
     assert lens == workloads.varlen_lengths(32, 128, 4096, 1004) and min(lens) >= 128 and max(lens) <= 4096
     cu = workloads.cu_from_lengths(lens)
     assert cu.dtype == torch.int32 and int(cu[0]) == 0 and int(cu[-1]) == sum(lens)
+
+
+def test_e4m3_per_block_quantisation():
+    """Per-block descales: the blocks of each sequence are its tokens [128i, 128i + 128) (the last one
+    ragged), numbered sequence after sequence; each (block, head) has its largest stored magnitude at
+    448, and stored × descale reproduces the source within e4m3's rounding."""
+    assert workloads.block_segments([(0, 200), (200, 0), (200, 513), (713, 64)]) == \
+        [(0, 128), (128, 72), (200, 128), (328, 128), (456, 128), (584, 128), (712, 1), (713, 64)]
+    g = torch.Generator().manual_seed(4)
+    segs = [(0, 200), (200, 0), (200, 300)]
+    x = torch.randn(500, 2, 128, generator=g)
+    x[128:200] *= 16.0                                                # the second block of sequence 0
+    q8, ds = workloads.quantize_e4m3_per_block(x, segs)
+    blocks = workloads.block_segments(segs)
+    assert ds.shape == (len(blocks), 2) == (5, 2)
+    for n, (s0, L) in enumerate(blocks):
+        assert torch.all(q8[s0:s0 + L].float().abs().amax(dim=(0, 2)) == workloads.E4M3_MAX)
+    assert math.isclose(float(ds[1, 0] / ds[0, 0]), 16.0, rel_tol=0.5)
+    real = workloads.real_values(q8, ds, blocks)
+    dsrow = np.concatenate([np.repeat(ds[n][None, :], L, axis=0) for n, (s0, L) in enumerate(blocks)])[:, :, None]
+    src = x.double().numpy()
+    assert np.all(np.abs(real - src) <= (2.0 ** -4 * np.abs(src) + 2.0 ** -10 * dsrow) * (1 + 1e-6))

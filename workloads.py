@@ -107,7 +107,8 @@ def _randn_e4m3(g: torch.Generator, shape):
 
 def real_values(t: torch.Tensor, descale=1.0, segments=None) -> np.ndarray:
     """The values a stored tensor stands for, as float64 (e4m3 or 16-bit storage times its descale):
-    ``descale`` a float, or a [B, H] array with ``segments`` the (start, length) of each sequence."""
+    ``descale`` a float, or an [S, H] array with ``segments`` the (start, length) of each of the S
+    token ranges it covers (sequences, or the 128-token blocks of ``block_segments``)."""
     x = t.detach().cpu().to(torch.float64).numpy()
     if segments is None:
         return x * float(descale)
@@ -132,6 +133,19 @@ def quantize_e4m3_per_head(x: torch.Tensor, segments):
         ds[b] = np.where(d > 0, d, np.float32(1.0))  # an all-zero head keeps descale 1 (finite and > 0)
         y[s0:s0 + L] = x[s0:s0 + L] / torch.from_numpy(ds[b])[None, :, None]
     return y.to(torch.float8_e4m3fn), ds
+
+
+def block_segments(segments, block: int = 128):
+    """(start, length) of every 128-token block, sequence after sequence: block i of a sequence is its
+    tokens [128i, 128i + 128), the last one ragged (the numbering of per-block e4m3 descales)."""
+    return [(s0 + i, min(block, L - i)) for s0, L in segments for i in range(0, L, block)]
+
+
+def quantize_e4m3_per_block(x: torch.Tensor, segments):
+    """fp32 [T, H, d] → (e4m3 tensor, fp32 descales [num_blocks, H]): each (128-token block, head) of
+    every sequence divided by its own amax/448 and rounded to e4m3; the real values follow from
+    ``real_values(t, descales, block_segments(segments))``."""
+    return quantize_e4m3_per_head(x, block_segments(segments))
 
 
 def varlen_lengths(nseq: int, lmin: int, lmax: int, seed: int) -> List[int]:
