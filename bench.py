@@ -1097,7 +1097,38 @@ def run_configs(args, world, rank, local, pg, headline):
             out[name] = config_summary(run_gpu(a, world, rank, local, pg))
         except Exception as exc:  # a failed extra config must not lose the headline line
             out[name] = {"workload": name, "error": f"{type(exc).__name__}: {exc}"}
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        for name, e in out.items():
+            if "error" not in e and name != headline["config"]["workload"]:
+                e["cpu_baseline"] = config_cpu_baseline(name)
     return out
+
+
+def config_cpu_baseline(name, budget_s=4.0):
+    """The oracle on a short sample of one extra workload (the headline has its own cpu_baseline): the
+    last `rows` query rows of head 0 of sequence 0 (the rows with the most visible keys), `rows` doubled
+    from 64 until the run takes about a quarter of `budget_s`, then timed once."""
+    import workloads
+    wl, p = (name.split("+")[0], 0.1) if "+dropout" in name else (name, 0.0)
+    inp = workloads.make_workload(wl)
+    L = inp.seqlens[0]
+    if p > 0.0:
+        R = dropout_sample_rows(inp, p, budget_s / 2)
+        dt, f = oracle_sample_dropout(inp, R, p)
+        sample = f"fp64 NumPy dropout oracle (p = {p}), one head of the first {R} tokens of sequence 0"
+    else:
+        rows = min(64, L)
+        dt, f = oracle_sample(inp, rows)
+        while rows < L and dt * 4 < budget_s:
+            rows = min(2 * rows, L)
+            dt, f = oracle_sample(inp, rows)
+        reps = max(1, int(0.25 * budget_s / max(dt, 1e-6)))  # a tiny sample is repeated to a measurable time
+        if reps > 1:
+            dt = sum(oracle_sample(inp, rows)[0] for _ in range(reps)) / reps
+        sample = (f"fp64 NumPy oracle, {'fwd+bwd' if inp.do is not None else 'fwd'} of the last {rows} query rows "
+                  f"of head 0 of sequence 0 ({L} tokens), {dt:.4f} s per run, {reps} run(s)")
+    return {"value": round(f / dt / 1e12, 6), "unit": "TFLOP/s", **host_threads(), "kind": "oracle",
+            "sample": sample}
 
 
 def main():
