@@ -861,9 +861,22 @@ __device__ __forceinline__ bool decode_bwd_unit(const BwdParams& p, int unit, Bw
   const int BH = p.B * p.H;
   const int nkb = p.num_kblocks;
   const int G = p.heads_group;
-  const int group = unit / (G * nkb);
-  const int g_heads = min(G, BH - group * G);
-  const int r = unit - group * G * nkb;
+  // Head groups run from the last (sequence, head) to the first: the preprocess kernel zeroes the dQ
+  // accumulator in token order, so the last sequences' accumulator lines are the ones still in L2 when
+  // this kernel starts, and the postprocess kernel, reading in token order, finds the lines this
+  // kernel reduced into last still in L2.  A partial last group (fewer than G heads) comes first.
+  const int full = BH / G, rem = BH - full * G;
+  int group, g_heads, r;
+  if (unit < rem * nkb) {
+    group = full;
+    g_heads = rem;
+    r = unit;
+  } else {
+    const int u2 = unit - rem * nkb;
+    group = full - 1 - u2 / (G * nkb);
+    g_heads = G;
+    r = u2 - (full - 1 - group) * G * nkb;
+  }
   const int kb = r / g_heads;
   const int bh = group * G + r % g_heads;
   const int b = bh / p.H;
