@@ -295,3 +295,14 @@ def test_fp8_per_block_too_few_blocks_is_reported(fa):
     O_ref, L_ref = oracle.attention_forward(q[:130], k[:130], v[:130], inp.scale, True, B=1, N=130)
     assert float(np.max(np.abs(f64(lse[:130]) - L_ref))) <= LSE_TOL
     assert float(np.max(np.abs(f64(o[:130]) - O_ref))) <= 0.1 * float(np.max(np.abs(O_ref)))
+
+
+def test_fp8_per_block_many_sequences(fa):
+    """Per-block descales with 41 sequences: each softmax warp counts the blocks of the sequences before
+    its unit's in chunks of 32 (one per lane), so a batch past 32 sequences takes the chunk loop more
+    than once; lengths include 0, 1, 128 and 129."""
+    g = torch.Generator().manual_seed(404)
+    seqlens = [int(x) for x in torch.randint(0, 300, (37,), generator=g)] + [0, 1, 128, 129]
+    inp = _per_block_inputs(seqlens, True, True, seed=405, H=2)
+    o, lse = _run(fa, inp)
+    _check(inp, o, lse)
