@@ -775,6 +775,34 @@ def run_gpu_fp8(args, world, rank, local, pg):
         raise fa.FAError(st, "timed steps")
     ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in evs])), pg, dev)
     value = world * flops / (ms * 1e-3) / 1e12
+    # the same forward with one descale per (128-token block, head) (fa_fwd_fp8_per_block): the inputs'
+    # per-tensor descales repeated into [num_blocks, H] arrays, so the output is the same computation
+    nb = B * ((N + 127) // 128)
+    blk = {n: torch.full((nb, H), float(ds[n]), dtype=torch.float32, device=dev) for n in ("q", "k", "v")}
+
+    def fwd_block():
+        st = fa.fa_fwd_fp8_per_block(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, N,
+                                     d, scale, causal, None, T, blk["q"].data_ptr(), blk["k"].data_ptr(),
+                                     blk["v"].data_ptr(), nb, sp)
+        if st != fa.FA_OK:
+            raise fa.FAError(st, "fa_fwd_fp8_per_block")
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        fwd_block()
+    evb = []
+    for _ in range(args.steps):
+        flush.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fwd_block()
+        b.record(stream)
+        evb.append((a, b))
+    torch.cuda.synchronize(dev)
+    st = fa.fa_check_device_status(sp)
+    if st != fa.FA_OK:
+        raise fa.FAError(st, "per-block steps")
+    ms_blk = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in evb])), pg, dev)
     # end to end through the public API: e4m3 inputs from pinned host memory, O and LSE back, pipelined
     # across steps over two buffer slots (see pipelined_e2e)
     host_in = [inp_h.q.pin_memory(), inp_h.k.pin_memory(), inp_h.v.pin_memory()]
@@ -823,6 +851,10 @@ def run_gpu_fp8(args, world, rank, local, pg):
                 "d2h_bytes_per_step": T * H * d * 2 + T * H * 4},
         "gpu_launches": args.steps,
         "clocks": clk,
+        "per_block_descales": {"ms": round(ms_blk, 4), "tflops": round(flops / (ms_blk * 1e-3) / 1e12, 1),
+                               "frac": round(flops / (ms_blk * 1e-3) / 1e12 / fp8_peak, 4),
+                               "note": "fa_fwd_fp8_per_block on the same inputs, one descale per (128-token block, "
+                                       "head); timed after the per-tensor steps, outside the headline value"},
     }
     if rank == 0 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(real_inputs(inp_h), budget_s=args.cpu_budget)
