@@ -8,25 +8,25 @@
 //   dS = P ∘ (dP − D),  dQ = scale·dS K,  dK = scale·dSᵀ Q.
 //
 // Three kernels on one stream:
-//   fa_bwd_pre_kernel   D (fp32 [T, H]) and a zeroed fp32 dQ accumulator
-//   fa_bwd_main_kernel  one CTA per (sequence, head, 128-key tile j):
-//                       K_j, V_j stay in shared memory; Q_i, dO_i stream in.
-//                       Per Q tile (BQ rows: 64 at d = 128, 128 at d = 64):
-//                         Sᵀ  = K_j Q_iᵀ        (tensor memory, fp32)
-//                         dPᵀ = V_j dO_iᵀ
-//                         Pᵀ  = 2^(c·Sᵀ − LSE_i·log2 e), masked   (warps 0-3)
-//                         dV += Pᵀ dO_i         (Pᵀ read from tensor memory)
-//                         dSᵀ = Pᵀ ∘ (dPᵀ − D_i)                  (warps 0-3)
-//                         dK += dSᵀ Q_i         (dSᵀ read from tensor memory)
-//                         dQ_i partial = dS K_j (dSᵀ staged in shared memory)
-//                       and warps 4-7 stage the dQ partial in shared memory,
-//                       from where TMA reduce-adds it into the fp32
-//                       accumulator.  dK (× scale) and dV are written once
-//                       at the end.
-//   fa_bwd_post_kernel  dq = scale · accumulator, rounded to the dtype
-// All five MMAs are M = 128 (full tensor-core rate): at d = 128 the dQ
-// product is formed transposed, dQᵀ = K_jᵀ dSᵀ (M = d), at d = 64 directly
-// (M = BQ = 128).
+//   fa_bwd_pre_kernel        D (fp32 [T, H]) and a zeroed fp32 dQ accumulator
+//   fa_bwd_main_q128_kernel  work unit = (sequence, head, 128-key tile j), run by persistent CTAs:
+//                            K_j, V_j stay in shared memory; Q_i, dO_i (128 query rows per
+//                            step) stream in.  Per step:
+//                              Sᵀ  = K_j Q_iᵀ, dPᵀ = V_j dO_iᵀ      (tensor memory, fp32)
+//                              Pᵀ  = 2^(c·Sᵀ − LSE_i·log2 e), masked (two compute warpgroups)
+//                              dV += Pᵀ dO_i                          (Pᵀ read from tensor memory)
+//                              dSᵀ = Pᵀ ∘ (dPᵀ − D_i)
+//                              dK += dSᵀ Q_i                          (dSᵀ read from tensor memory)
+//                              dQ_i partial = dS K_j                  (dSᵀ staged in shared memory)
+//                            and the dQ warpgroup stages the partial in shared memory, from where
+//                            TMA reduce-adds it into the fp32 accumulator.  dK (× scale) and dV
+//                            are written once per unit.  With dropout the keep mask of each
+//                            (query, key) is regenerated from the same Philox stream as the
+//                            forward: dV takes the dropped Pᵀ (its 1/(1 − p) applied at the end)
+//                            and dSᵀ = Pᵀ ∘ (Z ∘ dPᵀ / (1 − p) − D).
+//   fa_bwd_post_kernel       dq = scale · accumulator, rounded to the dtype
+// All five MMAs are 128 × 128 × d or 128 × d × 128 (full tensor-core rate): at d = 128 the dQ product
+// is formed transposed, dQᵀ = K_jᵀ dSᵀ (M = d), at d = 64 directly (M = 128 queries).
 #include "fa_internal.h"
 #include "sm100.cuh"
 
@@ -114,68 +114,7 @@ struct BwdParams {
   Dropout drop;
 };
 
-constexpr int kBwdThreads = 384;  // 3 warpgroups
 constexpr int kBK = 128;  // keys per CTA
-
-template <int D>
-struct BwdCfg {
-  static constexpr int BQ = (D == 128) ? 64 : 128;  // query rows per inner step
-  static constexpr int NCH = D / 64;
-  static constexpr uint32_t KV_TILE = kBK * D * 2;
-  static constexpr uint32_t Q_TILE = BQ * D * 2;
-  static constexpr uint32_t DS_TILE = kBK * BQ * 2;
-  static constexpr int STAGES = 2;
-  // tensor memory columns
-  static constexpr uint32_t T_ST = 0;          // Sᵀ  [128 keys × BQ]
-  static constexpr uint32_t T_DPT = BQ;        // dPᵀ [128 keys × BQ]
-  static constexpr uint32_t T_DQ = 2 * BQ;     // dQᵀ [d × 64] or dQ [128 × 64]: 64 columns
-  static constexpr uint32_t T_DK = (D == 128) ? 256 : 320;
-  static constexpr uint32_t T_DV = T_DK + D;
-  // dSᵀ as packed 16-bit (BQ/2 columns), A of the dK product: two buffers at d = 128 in the free
-  // columns [192, 256), one at d = 64 in [448, 512)
-  static constexpr int NDS = (D == 128) ? 2 : 1;
-  static constexpr uint32_t T_DS = (D == 128) ? 192 : 448;
-  static constexpr uint32_t T_DS_STRIDE = BQ / 2;
-  // barriers
-  static constexpr int B_KV = 0;
-  static constexpr int B_QFULL = 1;
-  static constexpr int B_QEMPTY = B_QFULL + STAGES;
-  static constexpr int B_ROWFULL = B_QEMPTY + STAGES;  // LSE / D of the Q tile in shared memory
-  static constexpr int B_SFULL = B_ROWFULL + STAGES;
-  static constexpr int B_DPFULL = B_SFULL + 1;
-  static constexpr int B_DPFREE = B_DPFULL + 1;   // the compute warpgroup has read dPᵀ out
-  static constexpr int B_PREADY = B_DPFREE + 1;
-  static constexpr int B_DSREADY = B_PREADY + 1;
-  static constexpr int B_DQFULL = B_DSREADY + 1;
-  static constexpr int B_DQFREE = B_DQFULL + 1;
-  static constexpr int B_DSFREE = B_DQFREE + 1;   // [NDS]: dK and dQ have read dSᵀ buffer b
-  static constexpr int B_DQSFREE = B_DSFREE + NDS;  // [2] dQ staging buffer b may be written
-  static constexpr int B_DQSFULL = B_DQSFREE + 2;   // [2] dQ staging buffer b written (128 arrivals)
-  static constexpr int B_DKV = B_DQSFULL + 2;
-  static constexpr int B_DRAIN = B_DKV + 1;
-  static constexpr int NBARS = B_DRAIN + 1;
-  // shared memory
-  static constexpr uint32_t OFF_K = 0;
-  static constexpr uint32_t OFF_V = KV_TILE;
-  static constexpr uint32_t OFF_Q = 2 * KV_TILE;
-  static constexpr uint32_t OFF_DO = OFF_Q + STAGES * Q_TILE;
-  static constexpr uint32_t OFF_DS = OFF_DO + STAGES * Q_TILE;
-  // dQ partial staging for the TMA reduce-add: 2 buffers of D/32 boxes [BQ rows × 32 fp32], 128-byte swizzle
-  static constexpr int NBOX = D / 32;
-  static constexpr uint32_t DQ_BOX = BQ * 128;
-  static constexpr uint32_t DQ_TILE = NBOX * DQ_BOX;
-  static constexpr uint32_t OFF_DQS = OFF_DS + NDS * DS_TILE;
-  static constexpr uint32_t OFF_ROW = OFF_DQS + 2 * DQ_TILE;  // per stage: −lse·log2(e)[BQ], −D[BQ] (fp32)
-  static constexpr uint32_t OFF_BAR = OFF_ROW + STAGES * 2 * BQ * 4;
-  static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
-  static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;
-  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-  // registers per thread after setmaxnreg (block of 384 launched at 168: 3 × 168 = 504 per lane triple)
-  static constexpr uint32_t REGS_CMP = 256;  // Pᵀ / dSᵀ warpgroup
-  static constexpr uint32_t REGS_DQ = 128;   // dQ warpgroup
-  static constexpr uint32_t REGS_IO = 120;   // producer / MMA warpgroup
-  static_assert(REGS_CMP + REGS_DQ + REGS_IO <= 504, "register budget");
-};
 
 __device__ __forceinline__ void drain_wait_b(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
   const uint64_t t0 = globaltimer_ns();
@@ -223,540 +162,12 @@ __device__ __forceinline__ void bwd_issue_acc(uint32_t d_tmem, uint32_t a_tmem, 
   for (int kk = 0; kk < BQ / 16; ++kk) mma_ts(d_tmem, a_tmem + kk * 8, db + ((kk * 2048) >> 4), IDESC, kk > 0 ? 1u : acc);
 }
 
-// dQ partial: K dim = the 128 keys, both operands MN-major (+2 KB per 16 keys).
-template <uint32_t IDESC>
-__device__ __forceinline__ void bwd_issue_dq(uint32_t d_tmem, uint64_t da, uint64_t db) {
-  da = opaque64(da);
-  db = opaque64(db);
-#pragma unroll
-  for (int kk = 0; kk < kBK / 16; ++kk) mma_ss(d_tmem, da + ((kk * 2048) >> 4), db + ((kk * 2048) >> 4), IDESC, kk > 0 ? 1u : 0u);
-}
-
-template <int D, bool BF16, bool DROP>
-__global__ void __launch_bounds__(kBwdThreads, 1)
-    fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                       const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
-  using C = BwdCfg<D>;
-  constexpr int BQ = C::BQ;
-  // Sᵀ = K Qᵀ and dPᵀ = V dOᵀ: M = 128 keys, N = BQ, both operands K-major
-  constexpr uint32_t IDESC_ST = idesc_f16(BF16, kBK, BQ, false, false);
-  // dV += Pᵀ dO and dK += dSᵀ Q: A from tensor memory, B (dO / Q) MN-major, N = d
-  constexpr uint32_t IDESC_DKV = idesc_f16(BF16, kBK, D, false, true);
-  // d = 128: dQᵀ = Kᵀ dSᵀ, M = d, N = 64, A = K MN-major, B = dSᵀ MN-major
-  // d = 64 : dQ  = dS K,   M = 128, N = 64, A = dS MN-major, B = K MN-major
-  constexpr uint32_t IDESC_DQ = idesc_f16(BF16, 128, 64, true, true);
-
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const uint32_t s_base = smem_u32(smem);
-  const uint32_t sK = s_base + C::OFF_K;
-  const uint32_t sV = s_base + C::OFF_V;
-  const uint32_t sQ = s_base + C::OFF_Q;
-  const uint32_t sDO = s_base + C::OFF_DO;
-  const uint32_t sDS = s_base + C::OFF_DS;
-  float* row_buf = reinterpret_cast<float*>(smem + C::OFF_ROW);
-  const uint32_t bar0 = s_base + C::OFF_BAR;
-  auto bar = [&](int i) -> uint32_t { return bar0 + 8u * i; };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
-  int* abort_flag = reinterpret_cast<int*>(smem + C::OFF_MISC + 4);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-
-  // ---- work unit: heads in groups, heaviest key tiles (the first ones when causal) first
-  const int BH = p.B * p.H;
-  const int nkb = p.num_kblocks;
-  const int G = p.heads_group;
-  const int unit = blockIdx.x;
-  const int group = unit / (G * nkb);
-  const int g_heads = min(G, BH - group * G);
-  const int r = unit - group * G * nkb;
-  const int kb = r / g_heads;
-  const int bh = group * G + r % g_heads;
-  const int b = bh / p.H;
-  const int h = bh - b * p.H;
-
-  int tok0, L;
-  if (p.cu_seqlens != nullptr) {
-    tok0 = __ldg(p.cu_seqlens + b);
-    const int end = __ldg(p.cu_seqlens + b + 1);
-    L = end - tok0;
-    if (tok0 < 0 || L < 0 || end > p.T || L > p.N) {
-      if (threadIdx.x == 0) record_status(1);
-      return;
-    }
-  } else {
-    tok0 = b * p.N;
-    L = p.N;
-  }
-  const int k0 = kb * kBK;
-  if (k0 >= L) return;
-  const int nq_all = (L + BQ - 1) / BQ;
-  const int i_begin = p.causal ? k0 / BQ : 0;
-  const int n_it = nq_all - i_begin;  // ≥ 1
-
-  if (warp == 9) {
-    tmem_alloc(smem_u32(tmem_slot), 512);
-    tmem_relinquish();
-  }
-  if (threadIdx.x == 0) {
-    mbar_init(bar(C::B_KV), 1);
-    for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(bar(C::B_QFULL + s), 1);
-      mbar_init(bar(C::B_QEMPTY + s), 1);
-      mbar_init(bar(C::B_ROWFULL + s), 32);
-    }
-    mbar_init(bar(C::B_SFULL), 1);
-    mbar_init(bar(C::B_DPFULL), 1);
-    mbar_init(bar(C::B_DPFREE), 128);
-    mbar_init(bar(C::B_PREADY), 128);
-    mbar_init(bar(C::B_DSREADY), 128);
-    mbar_init(bar(C::B_DQFULL), 1);
-    mbar_init(bar(C::B_DQFREE), 128);
-    for (int b = 0; b < C::NDS; ++b) mbar_init(bar(C::B_DSFREE + b), 1);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bar(C::B_DQSFREE + b), 1);
-      mbar_init(bar(C::B_DQSFULL + b), 128);
-    }
-    mbar_init(bar(C::B_DKV), 1);
-    mbar_init(bar(C::B_DRAIN), 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 8 && lane == 0) {
-    prefetch_tmap(&tm_q);
-    prefetch_tmap(&tm_k);
-    prefetch_tmap(&tm_v);
-    prefetch_tmap(&tm_do);
-    prefetch_tmap(&tm_dq);
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const Watchdog wd{abort_flag, p.timeout_ns};
-
-  if (warp >= 8) {
-    regs_dec<C::REGS_IO>();
-    // The producer and MMA warps run their loops with all 32 lanes (warp-uniform state);
-    // one elected lane (always the lowest) issues each copy, MMA and commit.
-    if (warp == 8) {
-      // ================================================================ TMA producer (+ row terms)
-      const uint64_t pol_kv = l2_policy_evict_first();
-      const uint64_t pol_q = l2_policy_evict_last();
-      if (elect_one()) {
-        mbar_arrive_expect_tx(bar(C::B_KV), 2 * C::KV_TILE);
-        for (int c = 0; c < C::NCH; ++c) {
-          tma_load_3d(sK + c * (kBK * 128), &tm_k, bar(C::B_KV), c * 64, h, tok0 + k0, pol_kv);
-          tma_load_3d(sV + c * (kBK * 128), &tm_v, bar(C::B_KV), c * 64, h, tok0 + k0, pol_kv);
-        }
-      }
-      __syncwarp();
-      int issued = 0;
-      const float LOG2E = 1.4426950408889634f;
-      for (int it = 0; it < n_it; ++it) {
-        const int s = it % C::STAGES;
-        if (it >= C::STAGES && !warp_wait_b(bar(C::B_QEMPTY + s), ((it / C::STAGES) - 1) & 1, wd)) break;
-        const int i0 = (i_begin + it) * BQ;
-        if (elect_one()) {
-          mbar_arrive_expect_tx(bar(C::B_QFULL + s), 2 * C::Q_TILE);
-          for (int c = 0; c < C::NCH; ++c) {
-            tma_load_3d(sQ + s * C::Q_TILE + c * (BQ * 128), &tm_q, bar(C::B_QFULL + s), c * 64, h, tok0 + i0, pol_q);
-            tma_load_3d(sDO + s * C::Q_TILE + c * (BQ * 128), &tm_do, bar(C::B_QFULL + s), c * 64, h, tok0 + i0,
-                        pol_q);
-          }
-        }
-        __syncwarp();
-        // −LSE·log2 e and −D of the tile's query rows; rows past the sequence get 0
-        float* lse_s = row_buf + s * 2 * BQ;
-        float* del_s = lse_s + BQ;
-        for (int q = lane; q < BQ; q += 32) {
-          const int qrow = i0 + q;
-          const bool v = qrow < L;
-          lse_s[q] = v ? -__ldg(p.lse + (size_t)(tok0 + qrow) * p.H + h) * LOG2E : 0.f;
-          del_s[q] = v ? -__ldg(p.delta + (size_t)(tok0 + qrow) * p.H + h) : 0.f;
-        }
-        mbar_arrive(bar(C::B_ROWFULL + s));  // release: the stores above are visible to waiters
-        issued = it + 1;
-      }
-      if (elect_one()) {
-        drain_wait_b(bar(C::B_KV), 0, p.timeout_ns);
-        for (int it = max(0, issued - C::STAGES); it < issued; ++it)
-          drain_wait_b(bar(C::B_QFULL + it % C::STAGES), (it / C::STAGES) & 1, p.timeout_ns);
-      }
-      __syncwarp();
-    } else if (warp == 9) {
-      // ================================================================ MMA issuer
-      // Per Q tile i:  dV += Pᵀ_i dO_i,  Sᵀ_{i+1} = K Qᵀ_{i+1},  dPᵀ_{i+1} = V dOᵀ_{i+1},
-      // dK += dSᵀ_i Q_i,  dQ_i (at d = 64, with one dSᵀ buffer, dPᵀ_{i+1} comes last).  Sᵀ_{i+1} overwrites the columns of Pᵀ_i only after dV_i
-      // (issued before it; tcgen05 MMAs of one thread run in order) has read them, and
-      // dPᵀ_{i+1} overwrites dPᵀ_i once the compute warpgroup has read it out (dPᵀ free).
-      // dSᵀ_i has columns of its own, so dPᵀ_{i+1} need not wait for dK_i.
-      const uint32_t tST = tmem + C::T_ST, tDPT = tmem + C::T_DPT, tDQ = tmem + C::T_DQ;
-      const uint32_t tDK = tmem + C::T_DK, tDV = tmem + C::T_DV, tDS = tmem + C::T_DS;
-      const uint64_t dK_kmaj = sdesc_sw128(sK, 16, 1024), dV_kmaj = sdesc_sw128(sV, 16, 1024);
-      const uint64_t dQ_kmaj = sdesc_sw128(sQ, 16, 1024), dDO_kmaj = sdesc_sw128(sDO, 16, 1024);
-      const uint64_t dQ_mn = sdesc_sw128(sQ, BQ * 128, 1024), dDO_mn = sdesc_sw128(sDO, BQ * 128, 1024);
-      // dQ operands (see IDESC_DQ)
-      const uint64_t dqa = (D == 128) ? sdesc_sw128(sK, kBK * 128, 1024) : sdesc_sw128(sDS, kBK * 128, 1024);
-      const uint64_t dqb = (D == 128) ? sdesc_sw128(sDS, 16, 1024) : sdesc_sw128(sK, 16, 1024);
-      constexpr uint32_t DS16 = C::DS_TILE >> 4;  // dSᵀ buffer stride in descriptor units
-      constexpr uint32_t QT16 = C::Q_TILE >> 4;  // stage stride of Q / dO in descriptor units
-      bool ok = warp_wait_b(bar(C::B_KV), 0, wd) && warp_wait_b(bar(C::B_QFULL + 0), 0, wd);
-      if (ok) {
-        tc_fence_after();
-        if (elect_one()) {
-          bwd_issue_kt<D, BQ, IDESC_ST>(tST, dK_kmaj, dQ_kmaj);
-          tc_commit(bar(C::B_SFULL));
-          bwd_issue_kt<D, BQ, IDESC_ST>(tDPT, dV_kmaj, dDO_kmaj);
-          tc_commit(bar(C::B_DPFULL));
-        }
-        __syncwarp();
-      }
-      for (int it = 0; ok && it < n_it; ++it) {
-        const int s = it % C::STAGES;
-        const int s1 = (it + 1) % C::STAGES;
-        const bool more = it + 1 < n_it;
-        // dV += Pᵀ dO
-        if (!warp_wait_b(bar(C::B_PREADY), it & 1, wd)) { ok = false; break; }
-        tc_fence_after();
-        if (elect_one()) bwd_issue_acc<BQ, IDESC_DKV>(tDV, tST, dDO_mn + s * QT16, it > 0 ? 1u : 0u);
-        __syncwarp();
-        if (more) {
-          // Sᵀ and dPᵀ of the next Q tile, computed while dS of this one is formed
-          if (!warp_wait_b(bar(C::B_QFULL + s1), ((it + 1) / C::STAGES) & 1, wd)) { ok = false; break; }
-          tc_fence_after();
-          if (elect_one()) {
-            bwd_issue_kt<D, BQ, IDESC_ST>(tST, dK_kmaj, dQ_kmaj + s1 * QT16);
-            tc_commit(bar(C::B_SFULL));
-          }
-          __syncwarp();
-          if constexpr (C::NDS == 2) {
-            // with two dSᵀ buffers the next dPᵀ goes ahead of dK_i / dQ_i
-            if (!warp_wait_b(bar(C::B_DPFREE), it & 1, wd)) { ok = false; break; }
-            tc_fence_after();
-            if (elect_one()) {
-              bwd_issue_kt<D, BQ, IDESC_ST>(tDPT, dV_kmaj, dDO_kmaj + s1 * QT16);
-              tc_commit(bar(C::B_DPFULL));
-            }
-            __syncwarp();
-          }
-        }
-        // dK += dSᵀ Q
-        if (!warp_wait_b(bar(C::B_DSREADY), it & 1, wd)) { ok = false; break; }
-        tc_fence_after();
-        const int db = it % C::NDS;  // dSᵀ buffer of this Q tile
-        if (elect_one())
-          bwd_issue_acc<BQ, IDESC_DKV>(tDK, tDS + db * C::T_DS_STRIDE, dQ_mn + s * QT16, it > 0 ? 1u : 0u);
-        __syncwarp();
-        // dQ partial, once the dQ warpgroup has read the previous one out
-        if (it > 0 && !warp_wait_b(bar(C::B_DQFREE), (it - 1) & 1, wd)) { ok = false; break; }
-        tc_fence_after();
-        if (elect_one()) {
-          if constexpr (D == 128) bwd_issue_dq<IDESC_DQ>(tDQ, dqa, dqb + db * DS16);
-          else bwd_issue_dq<IDESC_DQ>(tDQ, dqa + db * DS16, dqb);
-          tc_commit(bar(C::B_DQFULL));
-          tc_commit(bar(C::B_DSFREE + db));  // dK_i and dQ_i have read dSᵀ buffer db
-          tc_commit(bar(C::B_QEMPTY + s));   // Q_i, dO_i and their row terms are no longer read
-        }
-        __syncwarp();
-        if constexpr (C::NDS == 1) {
-          // one dSᵀ buffer: the next dPᵀ follows dK_i / dQ_i, which the next dSᵀ write waits for anyway
-          if (more) {
-            if (!warp_wait_b(bar(C::B_DPFREE), it & 1, wd)) { ok = false; break; }
-            tc_fence_after();
-            if (elect_one()) {
-              bwd_issue_kt<D, BQ, IDESC_ST>(tDPT, dV_kmaj, dDO_kmaj + s1 * QT16);
-              tc_commit(bar(C::B_DPFULL));
-            }
-            __syncwarp();
-          }
-        }
-      }
-      if (elect_one()) {
-        tc_commit(bar(C::B_DKV));
-        tc_commit(bar(C::B_DRAIN));
-        drain_wait_b(bar(C::B_DRAIN), 0, p.timeout_ns);
-      }
-      __syncwarp();
-    }
-  } else if (warp < 4) {
-    // ================================================================ Pᵀ / dSᵀ warpgroup (thread = key row)
-    regs_inc<C::REGS_CMP>();
-    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
-    const uint32_t tST = tmem + lane_off + C::T_ST;
-    const uint32_t tDPT = tmem + lane_off + C::T_DPT;
-    const uint32_t tDS = tmem + lane_off + C::T_DS;
-    const uint32_t tDV = tmem + lane_off + C::T_DV;
-    const int kr = 32 * warp + lane;  // key row within the tile
-    const int key = k0 + kr;          // position in the sequence
-    const float c = p.scale_log2;
-    const uint32_t keep_bias = keep_flag_bias(p.drop.t);     // used by the dropout variant only
-    const uint32_t ks_bits = __float_as_uint(p.drop.keep_scale);
-    bool ok = true;
-    for (int it = 0; it < n_it; ++it) {
-      const int i0 = (i_begin + it) * BQ;
-      const int s = it % C::STAGES;
-      if (!warp_wait_b(bar(C::B_ROWFULL + s), (it / C::STAGES) & 1, wd)) { ok = false; break; }
-      const float* lse_s = row_buf + s * 2 * BQ;
-      const float* del_s = lse_s + BQ;
-      // visible queries for this key: q >= key (causal) and q < L; key < L
-      const int q_lo = p.causal ? key - i0 : 0;  // first visible column
-      const int q_hi = (key < L) ? L - i0 : -1;  // one past the last visible column
-      const bool full = __all_sync(0xffffffffu, q_lo <= 0 && q_hi >= BQ);  // no masking in this tile
-      // dropout: the random bytes of this key for the BQ queries of the step, word g = queries 4g .. 4g+3
-      // (byte = query offset).  One Philox call covers the 4 keys of a lane quad (key mod 4 = lane mod 4)
-      // × 4 queries: each lane of the quad makes BQ/16 of the step's calls, reorders its call's bytes
-      // from (query word, key byte) to (key word, query byte), and the quad exchanges words.
-      uint32_t rw[DROP ? BQ / 4 : 1];
-      if constexpr (DROP) {
-        const uint32_t bh = (uint32_t)(b * p.H + h), kg = (uint32_t)key >> 2;
-        const uint32_t g0 = (uint32_t)i0 / 4u + (uint32_t)(lane & 3);
-#pragma unroll
-        for (int m = 0; m < BQ / 16; ++m) {
-          const uint4 r4 = philox4x32_10(kg, g0 + 4u * m, bh, p.drop.offset, p.drop.seed_lo, p.drop.seed_hi);
-          const uint32_t a0 = prmt(r4.x, r4.y, 0x5140u), a1 = prmt(r4.x, r4.y, 0x7362u);
-          const uint32_t a2 = prmt(r4.z, r4.w, 0x5140u), a3 = prmt(r4.z, r4.w, 0x7362u);
-          uint32_t x[4] = {prmt(a0, a2, 0x5410u), prmt(a0, a2, 0x7632u), prmt(a1, a3, 0x5410u), prmt(a1, a3, 0x7632u)};
-          quad_transpose(x, lane);
-#pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) rw[4 * m + c4] = x[c4];
-        }
-      }
-      // words 4·m0 .. 4·(m0 + nm) − 1 of the step (held in registers: parking them in shared memory at
-      // d = 64, where it fits, removed the spills but measured slower)
-      auto drop_words = [&](int m0, int nm, uint32_t* out) {
-        if constexpr (DROP) {
-#pragma unroll
-          for (int k = 0; k < 4 * nm; ++k) out[k] = rw[4 * m0 + k];
-        }
-      };
-      if (!warp_wait_b(bar(C::B_SFULL), it & 1, wd)) { ok = false; break; }
-      tc_fence_after();
-      const float2 c2 = make_float2(c, c);
-      // dropout factor (0 or 1/(1 − p)) of the query whose random byte is byte c of word w
-      auto mk = [&](uint32_t w, int c) -> float {
-        if constexpr (!DROP) return 1.f;
-        uint32_t e, o;
-        keep_flags(w, keep_bias, e, o);
-        const uint32_t sel = c == 0 ? 0x9999u : c == 1 ? 0xDDDDu : c == 2 ? 0xBBBBu : 0xFFFFu;
-        return __uint_as_float(prmt(e, o, sel) & ks_bits);  // the keep flag's sign fills all 32 bits
-      };
-      float pt[BQ];
-      {
-        uint32_t sr[BQ];
-#pragma unroll
-        for (int q = 0; q < BQ / 32; ++q) tmem_ld32(tST + 32u * q, reinterpret_cast<uint32_t(&)[32]>(sr[32 * q]));
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < BQ; i += 2) {
-          const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), c2,
-                                      make_float2(lse_s[i], lse_s[i + 1]));
-          pt[i] = ex2(x.x);
-          pt[i + 1] = ex2(x.y);
-        }
-        if (!full) {
-#pragma unroll
-          for (int i = 0; i < BQ; ++i) pt[i] = (i >= q_lo && i < q_hi) ? pt[i] : 0.f;
-        }
-      }
-#pragma unroll
-      for (int q = 0; q < BQ / 64; ++q) {
-        uint32_t wq[DROP ? 16 : 1];
-        drop_words(4 * q, 4, wq);  // queries 64q .. 64q + 63
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          pk[i] = pack2<BF16>(pt[64 * q + 2 * i] * mk(wq[DROP ? i >> 1 : 0], (2 * i) & 3),
-                              pt[64 * q + 2 * i + 1] * mk(wq[DROP ? i >> 1 : 0], (2 * i + 1) & 3));
-        tmem_st32(tST + 32u * q, pk);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(C::B_PREADY));
-      if (!warp_wait_b(bar(C::B_DPFULL), it & 1, wd)) { ok = false; break; }
-      tc_fence_after();
-      // dSᵀ buffer db: dK and dQ of the Q tile that used it before must have read it
-      const int db = it % C::NDS;
-      if (it >= C::NDS && !warp_wait_b(bar(C::B_DSFREE + db), ((it / C::NDS) - 1) & 1, wd)) { ok = false; break; }
-      // dSᵀ = Pᵀ ∘ (dPᵀ − D), 32 query columns at a time: into its tensor-memory columns (A of the
-      // dK product) and into shared memory as 128-byte swizzled rows = keys (operand of the dQ product)
-      uint8_t* ds_row = smem + C::OFF_DS + db * C::DS_TILE + kr * 128;
-      const uint32_t tDSb = tDS + db * C::T_DS_STRIDE;
-#pragma unroll
-      for (int q = 0; q < BQ / 32; ++q) {
-        uint32_t dr[32];
-        tmem_ld32(tDPT + 32u * q, dr);
-        tmem_wait_ld();
-        if (q == BQ / 32 - 1) {
-          // dPᵀ fully read out: the next dPᵀ may overwrite it
-          tc_fence_before();
-          mbar_arrive(bar(C::B_DPFREE));
-        }
-        // −D of these 32 queries.  At BQ = 128 they are read here with loads the compiler cannot hoist
-        // (all 128 values would not fit in registers beside Pᵀ); at BQ = 64 the compiler may schedule
-        // them early, which measures faster.
-        float nd[32];
-        if constexpr (BQ == 128) {
-#pragma unroll
-          for (int v = 0; v < 8; ++v) ld_shared_v4f(del_s + 32 * q + 4 * v, nd + 4 * v);
-        } else {
-#pragma unroll
-          for (int v = 0; v < 32; ++v) nd[v] = del_s[32 * q + v];
-        }
-        uint32_t wq[DROP ? 8 : 1];
-        drop_words(2 * q, 2, wq);  // queries 32q .. 32q + 31
-        uint32_t dsk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int col = 32 * q + 2 * i;
-          const float2 dpv = make_float2(__uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1]));
-          const uint32_t w = wq[DROP ? i >> 1 : 0];
-          const float2 dd = DROP ? __ffma2_rn(dpv, make_float2(mk(w, (2 * i) & 3), mk(w, (2 * i + 1) & 3)),
-                                              make_float2(nd[2 * i], nd[2 * i + 1]))
-                                 : __fadd2_rn(dpv, make_float2(nd[2 * i], nd[2 * i + 1]));
-          const float2 ds = __fmul2_rn(make_float2(pt[col], pt[col + 1]), dd);
-          dsk[i] = pack2<BF16>(ds.x, ds.y);
-        }
-        tmem_st16(tDSb + 16u * q, dsk);
-        // 32 query columns = 64 bytes = 4 of the row's eight 16-byte chunks (64-query chunk q / 2)
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          const int chunk = (q & 1) * 4 + ch;
-          const int sw = chunk ^ (kr & 7);
-          *reinterpret_cast<uint4*>(ds_row + (q >> 1) * (kBK * 128) + sw * 16) =
-              make_uint4(dsk[4 * ch], dsk[4 * ch + 1], dsk[4 * ch + 2], dsk[4 * ch + 3]);
-        }
-      }
-      fence_proxy_async_smem();
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(C::B_DSREADY));
-    }
-    // ---- epilogue: dV rows of this tile
-    if (ok && warp_wait_b(bar(C::B_DKV), 0, wd)) {
-      tc_fence_after();
-      const bool valid = key < L;
-      uint8_t* dst = reinterpret_cast<uint8_t*>(p.dv) + (((size_t)(tok0 + (valid ? key : 0)) * p.H + h) * D) * 2;
-#pragma unroll
-      for (int q = 0; q < D / 32; ++q) {
-        uint32_t r32[32];
-        tmem_ld32(tDV + 32u * q, r32);
-        tmem_wait_ld();
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = pack2<BF16>(__uint_as_float(r32[2 * i]), __uint_as_float(r32[2 * i + 1]));
-        if (valid) {
-#pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            st_global_v4(dst + q * 64 + v4 * 16, pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
-        }
-      }
-    }
-    __syncwarp();
-  } else {
-    // ================================================================ dQ warpgroup (warps 4-7)
-    regs_dec<C::REGS_DQ>();
-    const int quarter = warp & 3;
-    const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
-    const uint32_t tDQ = tmem + lane_off + C::T_DQ;
-    const uint32_t tDK = tmem + lane_off + C::T_DK;
-    const int lrow = 32 * quarter + lane;  // tensor-memory lane of this thread
-    const bool issuer = (warp == 4 && lane == 0);
-    const uint32_t sDQS = s_base + C::OFF_DQS;
-    bool ok = true;
-    for (int it = 0; it < n_it; ++it) {
-      const int i0 = (i_begin + it) * BQ;
-      if (!warp_wait_b(bar(C::B_DQFULL), it & 1, wd)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t qr[64];
-      tmem_ld32(tDQ, reinterpret_cast<uint32_t(&)[32]>(qr[0]));
-      tmem_ld32(tDQ + 32u, reinterpret_cast<uint32_t(&)[32]>(qr[32]));
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar(C::B_DQFREE));
-      // The partial goes to the fp32 accumulator by TMA reduce-add from a shared-memory staging buffer
-      // (coalesced, asynchronous).  Buffer b = it & 1 is written once the reduce issued from it two
-      // steps ago has read it; the issuing thread signals that, and issues the next reduce when all
-      // 128 threads have written.  Rows past the end of the sequence hold exact zeros (P is 0 there),
-      // rows past T are clipped by the TMA unit.
-      const int b = it & 1;
-      const uint32_t u = (uint32_t)it >> 1;  // use of buffer b
-      const uint32_t buf = sDQS + b * C::DQ_TILE;
-      if (issuer) {
-        if (it >= 2) bulk_wait_group_read<1>();
-        mbar_arrive(bar(C::B_DQSFREE + b));
-      }
-      if (!warp_wait_b(bar(C::B_DQSFREE + b), u & 1, wd)) { ok = false; break; }
-      if constexpr (D == 128) {
-        // dQᵀ: lane = feature 32·quarter + lane (box `quarter`), columns = 64 queries (box rows)
-        const uint32_t box = buf + quarter * C::DQ_BOX + ((lane & 3) << 2);
-#pragma unroll
-        for (int q = 0; q < 64; ++q) st_shared_f32(box + q * 128 + ((((lane >> 2) ^ (q & 7))) << 4), qr[q]);
-      } else {
-        // dQ: lane = query row (box row), columns = 64 features (boxes 0 and 1)
-#pragma unroll
-        for (int k = 0; k < 2; ++k)
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            st_shared_v4(buf + k * C::DQ_BOX + lrow * 128 + ((j ^ (lrow & 7)) << 4), qr[32 * k + 4 * j],
-                         qr[32 * k + 4 * j + 1], qr[32 * k + 4 * j + 2], qr[32 * k + 4 * j + 3]);
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(bar(C::B_DQSFULL + b));
-      bool fail = false;
-      if (issuer) {
-        if (mbar_wait(bar(C::B_DQSFULL + b), u & 1, wd)) {
-#pragma unroll
-          for (int k = 0; k < C::NBOX; ++k) tma_reduce_add_3d(&tm_dq, buf + k * C::DQ_BOX, 32 * k, h, tok0 + i0);
-          bulk_commit_group();
-        } else {
-          fail = true;
-        }
-      }
-      if (__any_sync(0xffffffffu, fail)) { ok = false; break; }  // the whole warp leaves together
-    }
-    if (issuer) bulk_wait_group_all();  // every reduce performed before the kernel ends
-    // ---- epilogue: dK rows (× scale)
-    if (ok && warp_wait_b(bar(C::B_DKV), 0, wd)) {
-      tc_fence_after();
-      const int key = k0 + lrow;
-      const bool valid = key < L;
-      uint8_t* dst = reinterpret_cast<uint8_t*>(p.dk) + (((size_t)(tok0 + (valid ? key : 0)) * p.H + h) * D) * 2;
-#pragma unroll
-      for (int q = 0; q < D / 32; ++q) {
-        uint32_t r32[32];
-        tmem_ld32(tDK + 32u * q, r32);
-        tmem_wait_ld();
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pk[i] = pack2<BF16>(__uint_as_float(r32[2 * i]) * p.scale, __uint_as_float(r32[2 * i + 1]) * p.scale);
-        if (valid) {
-#pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            st_global_v4(dst + q * 64 + v4 * 16, pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
-        }
-      }
-    }
-    __syncwarp();
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 9) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
-  }
-}
-
-// ============================================================================ main kernel at d = 128, 128-query steps
+// ============================================================================ main kernel, 128-query steps
 //
-// Same work unit and equations as fa_bwd_main_kernel, but every Q step covers 128 query rows, so the
-// score, dP, dV, dK and dQ products are all 128 × 128 × 128 (N = 128: at N = 64 the tensor core is
-// starved by its shared-memory operand reads).  Two compute warpgroups form Pᵀ and dSᵀ concurrently,
-// one per 64-query half of the step (thread = key row, as before).  Tensor memory cannot hold Sᵀ and
+// Every Q step covers 128 query rows, so the score, dP, dV, dK and dQ products are all 128 × 128 × 128
+// at d = 128 (N = 128: at N = 64 the tensor core is starved by its shared-memory operand reads).  Two
+// compute warpgroups form Pᵀ and dSᵀ concurrently, one per 64-query half of the step (thread = key
+// row).  Tensor memory cannot hold Sᵀ and
 // dPᵀ of a step beside dK and dV (128 columns each) plus a dQ partial, so columns are reused:
 //   [0, 128)    Sᵀ(j); once both halves are in registers, dQᵀ(j − 1) = Kᵀ dSᵀ(j − 1) [128 features ×
 //               128 queries]; once that has been read out, Pᵀ(j) packed into [0, 64) (half a in
@@ -775,8 +186,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 // turn) and adds it into the accumulator with a TMA reduce-add (per-thread red.global.add of the same
 // data measured far slower).
 constexpr int kBwd128Threads = 512;  // 4 warpgroups
-// Column pairs i (of 32 per query half) with bit (i % 8) set take the FMA-pipe exp2 in unmasked halves.
-constexpr uint32_t kBwd128PolyMask = 0x00u;
 
 template <int D>
 struct Bq128 {
@@ -850,7 +259,7 @@ __device__ __forceinline__ void bwd_issue_dq128(uint32_t d_tmem, uint64_t da, ui
 // A decoded work unit of the backward: key tile [k0, k0 + 128) of the sequence whose tokens are
 // [tok0, tok0 + L), head h; n_it Q steps from query tile i_begin.
 struct BwdUnit {
-  int tok0, L, k0, h, i_begin, n_it;
+  int tok0, L, k0, b, h, i_begin, n_it;
 };
 
 // Unit order: heads in groups (K, V, Q and dO of a group stay in L2), heaviest key tiles (the first
@@ -880,6 +289,7 @@ __device__ __forceinline__ bool decode_bwd_unit(const BwdParams& p, int unit, Bw
   const int kb = r / g_heads;
   const int bh = group * G + r % g_heads;
   const int b = bh / p.H;
+  u.b = b;
   u.h = bh - b * p.H;
   if (p.cu_seqlens != nullptr) {
     u.tok0 = __ldg(p.cu_seqlens + b);
@@ -900,7 +310,7 @@ __device__ __forceinline__ bool decode_bwd_unit(const BwdParams& p, int unit, Bw
   return true;
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool DROP>
 __global__ void __launch_bounds__(kBwd128Threads, 1)
     fa_bwd_main_q128_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -1271,6 +681,8 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
     const int kr = 32 * quarter + lane;  // key row within the tile
     const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
     uint8_t* ds_row = smem + C::OFF_DS + a * C::CHUNK + kr * 128;
+    const uint32_t keep_bias = keep_flag_bias(p.drop.t);  // used by the dropout variant only
+    const uint32_t ks_bits = __float_as_uint(p.drop.keep_scale);
     uint32_t g = 0;  // steps so far (all units)
     bool ok = true;
     int unit;
@@ -1288,6 +700,27 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
         const int q_lo = p.causal ? key - i0 : 0;    // first visible column of the half
         const int q_hi = (key < U.L) ? U.L - i0 : -1;  // one past the last visible column
         const bool full = __all_sync(0xffffffffu, q_lo <= 0 && q_hi >= 64);
+        // dropout: the random bytes of this key for the half's 64 queries, word w = queries 4w .. 4w+3
+        // (byte = query offset), the same Philox numbering as the forward.  One call covers the 4 keys
+        // of a lane quad (key mod 4 = lane mod 4) × 4 queries: each lane of the quad makes 4 of the
+        // half's 16 calls, reorders its call's bytes from (query word, key byte) to (key word, query
+        // byte), and the quad exchanges words.  Made before Sᵀ is read, while the registers are free.
+        uint32_t rw[DROP ? 16 : 1];
+        if constexpr (DROP) {
+          const uint32_t bh = (uint32_t)(U.b * p.H + U.h), kg = (uint32_t)key >> 2;
+          const uint32_t g0 = (uint32_t)i0 / 4u + (uint32_t)(lane & 3);
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const uint4 r4 = philox4x32_10(kg, g0 + 4u * m, bh, p.drop.offset, p.drop.seed_lo, p.drop.seed_hi);
+            const uint32_t a0 = prmt(r4.x, r4.y, 0x5140u), a1 = prmt(r4.x, r4.y, 0x7362u);
+            const uint32_t a2 = prmt(r4.z, r4.w, 0x5140u), a3 = prmt(r4.z, r4.w, 0x7362u);
+            uint32_t x[4] = {prmt(a0, a2, 0x5410u), prmt(a0, a2, 0x7632u), prmt(a1, a3, 0x5410u),
+                             prmt(a1, a3, 0x7632u)};
+            quad_transpose(x, lane);
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) rw[4 * m + c4] = x[c4];
+          }
+        }
         // ---- Pᵀ = 2^(c·Sᵀ − LSE·log2 e), masked
         if (!warp_wait_b(bar(C::B_SFULL), g & 1, wd)) { ok = false; break; }
         tc_fence_after();
@@ -1324,7 +757,24 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
           break;
         }
         tc_fence_after();
-        tmem_st32(tP, pk);
+        if constexpr (DROP) {
+          // the dV product takes the dropped Pᵀ (its 1/(1 − p) is applied to dV at the end); pk keeps
+          // the undropped values for dSᵀ
+#pragma unroll
+          for (int hq = 0; hq < 2; ++hq) {
+            uint32_t pd[16];
+#pragma unroll
+            for (int w = 0; w < 8; ++w) {  // word w of this 32-query quarter: pairs 2w, 2w + 1
+              uint32_t m01, m23;
+              keep_pair_masks(rw[8 * hq + w], keep_bias, m01, m23);
+              pd[2 * w] = pk[16 * hq + 2 * w] & m01;
+              pd[2 * w + 1] = pk[16 * hq + 2 * w + 1] & m23;
+            }
+            tmem_st16(tP + 16u * hq, pd);
+          }
+        } else {
+          tmem_st32(tP, pk);
+        }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(C::B_PREADY + a));
@@ -1339,7 +789,17 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const float2 dpv = make_float2(__uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1]));
-            const float2 dd = __fadd2_rn(dpv, make_float2(del_h[2 * i], del_h[2 * i + 1]));
+            float2 dd;
+            if constexpr (DROP) {
+              // dSᵀ = Pᵀ ∘ (Z ∘ dPᵀ / (1 − p) − D): the keep flag's sign fills the factor's 32 bits
+              uint32_t e, o;
+              keep_flags(rw[i >> 1], keep_bias, e, o);  // once per word: the compiler shares it across i, i ^ 1
+              const float f0 = __uint_as_float(prmt(e, o, (i & 1) ? 0xBBBBu : 0x9999u) & ks_bits);
+              const float f1 = __uint_as_float(prmt(e, o, (i & 1) ? 0xFFFFu : 0xDDDDu) & ks_bits);
+              dd = __ffma2_rn(dpv, make_float2(f0, f1), make_float2(del_h[2 * i], del_h[2 * i + 1]));
+            } else {
+              dd = __fadd2_rn(dpv, make_float2(del_h[2 * i], del_h[2 * i + 1]));
+            }
             const float2 ds = __fmul2_rn(unpack2<BF16>(pk[i]), dd);
             dsk[i] = pack2<BF16>(ds.x, ds.y);
           }
@@ -1460,7 +920,7 @@ __global__ void __launch_bounds__(kBwd128Threads, 1)
       uint8_t* dv_row = reinterpret_cast<uint8_t*>(p.dv) + (((size_t)(U.tok0 + (valid ? key : 0)) * p.H + U.h) * D) * 2;
 #pragma unroll 1
       for (int t = 0; t < 2; ++t) {  // dK, then dV
-        const float f = t == 0 ? p.scale : 1.f;
+        const float f = t == 0 ? p.scale : (DROP ? p.drop.keep_scale : 1.f);  // dV: the dropout's 1/(1 − p)
         uint8_t* row = t == 0 ? dk_row : dv_row;
 #pragma unroll
         for (int q = 0; q < D / 32; ++q) {
@@ -1546,39 +1006,9 @@ cudaError_t launch_bwd_post(const Problem& pb, const BwdArgs& a, cudaStream_t st
 }
 
 template <int D, bool BF16, bool DROP>
-static cudaError_t launch_main_t(const Problem& pb, const BwdArgs& a, cudaStream_t stream) {
-  using C = BwdCfg<D>;
-  static std::atomic<unsigned long long> configured{0};  // per instantiation, one bit per device
-  auto kern = fa_bwd_main_kernel<D, BF16, DROP>;
-  if (cudaError_t e = set_smem_once(configured, reinterpret_cast<const void*>(kern), C::SMEM_BYTES); e != cudaSuccess)
-    return e;
-  BwdParams p;
-  p.lse = a.lse;
-  p.delta = a.delta;
-  p.dq_acc = a.dq_acc;
-  p.dk = a.dk;
-  p.dv = a.dv;
-  p.cu_seqlens = pb.cu_seqlens;
-  p.B = pb.B;
-  p.H = pb.H;
-  p.N = pb.N;
-  p.T = pb.T;
-  p.causal = pb.causal;
-  p.num_kblocks = (pb.N + kBK - 1) / kBK;
-  p.heads_group = 8;
-  p.scale = pb.scale;
-  p.scale_log2 = pb.scale * 1.4426950408889634f;
-  p.timeout_ns = pb.timeout_ns;
-  p.drop = pb.drop;
-  const long long units = (long long)pb.B * pb.H * p.num_kblocks;
-  kern<<<dim3((unsigned)units), dim3(kBwdThreads), C::SMEM_BYTES, stream>>>(a.tm_q, a.tm_k, a.tm_v, a.tm_do, a.tm_dq, p);
-  return cudaPeekAtLastError();
-}
-
-template <int D, bool BF16>
 static cudaError_t launch_main_q128_t(const Problem& pb, const BwdArgs& a, cudaStream_t stream) {
   static std::atomic<unsigned long long> configured{0};  // per instantiation, one bit per device
-  auto kern = fa_bwd_main_q128_kernel<D, BF16>;
+  auto kern = fa_bwd_main_q128_kernel<D, BF16, DROP>;
   if (cudaError_t e = set_smem_once(configured, reinterpret_cast<const void*>(kern), Bq128<D>::SMEM_BYTES);
       e != cudaSuccess)
     return e;
@@ -1608,20 +1038,16 @@ static cudaError_t launch_main_q128_t(const Problem& pb, const BwdArgs& a, cudaS
 
 template <bool DROP>
 static cudaError_t launch_main_d(const Problem& pb, const BwdArgs& a, cudaStream_t stream) {
-  if constexpr (!DROP) {
-    if (pb.d == 128)
-      return pb.bf16 ? launch_main_q128_t<128, true>(pb, a, stream) : launch_main_q128_t<128, false>(pb, a, stream);
-    return pb.bf16 ? launch_main_q128_t<64, true>(pb, a, stream) : launch_main_q128_t<64, false>(pb, a, stream);
-  }
   if (pb.d == 128)
-    return pb.bf16 ? launch_main_t<128, true, DROP>(pb, a, stream) : launch_main_t<128, false, DROP>(pb, a, stream);
-  return pb.bf16 ? launch_main_t<64, true, DROP>(pb, a, stream) : launch_main_t<64, false, DROP>(pb, a, stream);
+    return pb.bf16 ? launch_main_q128_t<128, true, DROP>(pb, a, stream)
+                   : launch_main_q128_t<128, false, DROP>(pb, a, stream);
+  return pb.bf16 ? launch_main_q128_t<64, true, DROP>(pb, a, stream) : launch_main_q128_t<64, false, DROP>(pb, a, stream);
 }
 
 // Rows per Q / dO tile the main kernel loads, and per box of its dQ reduce-adds (the host encodes the
 // tensor maps with these box heights).
-int bwd_q_tile_rows(int d, bool dropout) { return (d == 128 && dropout) ? 64 : 128; }
-int bwd_dq_box_rows(int d, bool dropout) { return dropout ? (d == 128 ? 64 : 128) : 32; }
+int bwd_q_tile_rows(int, bool) { return 128; }
+int bwd_dq_box_rows(int, bool) { return 32; }
 
 cudaError_t launch_bwd_main(const Problem& pb, const BwdArgs& a, cudaStream_t stream) {
   return pb.drop.t != 0u ? launch_main_d<true>(pb, a, stream) : launch_main_d<false>(pb, a, stream);
