@@ -98,6 +98,43 @@ def ring_block(rank: int, step: int, world: int, causal: bool) -> Tuple[int, Opt
     return src, "full"
 
 
+class _Staged:
+    """Completion of a host-staged exchange: waits for the CPU transfers, then copies what was received
+    into the device tensors (on the current stream)."""
+
+    def __init__(self, reqs, pairs):
+        self.reqs, self.pairs = reqs, pairs
+
+    def wait(self):
+        for r in self.reqs:
+            r.wait()
+        for dst, src in self.pairs:
+            dst.copy_(src)
+
+
+def _exchange(sends, recvs, nxt, prv, group):
+    """Send ``sends`` to rank ``nxt`` and receive ``recvs`` from rank ``prv`` (tensors of this rank's
+    device) → objects with ``wait()``.  NCCL moves device memory directly.  A backend that moves host
+    memory only (gloo) gets host copies: the sends are copied out first (which waits for the kernels
+    that wrote them), the receives land in host buffers and are copied in by ``wait()``."""
+    import torch.distributed as dist
+    on_device = any(t.is_cuda for t in list(sends) + list(recvs))
+    if not on_device or dist.get_backend(group) == "nccl":
+        ops = [dist.P2POp(dist.isend, t, nxt, group) for t in sends] + \
+              [dist.P2POp(dist.irecv, t, prv, group) for t in recvs]
+        return dist.batch_isend_irecv(ops)
+    host_s = [t.cpu() for t in sends]
+    host_r = [_host_like(t) for t in recvs]
+    ops = [dist.P2POp(dist.isend, t, nxt, group) for t in host_s] + \
+          [dist.P2POp(dist.irecv, t, prv, group) for t in host_r]
+    return [_Staged(dist.batch_isend_irecv(ops), list(zip(recvs, host_r)))]
+
+
+def _host_like(t):
+    import torch
+    return torch.empty(t.shape, dtype=t.dtype, device="cpu")
+
+
 def _default_block(q, k, v, causal, scale, out, lse):
     attention_forward(q, k, v, causal=causal, scale=scale, out=out, lse=lse)
 
@@ -181,9 +218,7 @@ def ring_attention_forward(q, k, v, causal: bool = False, scale: Optional[float]
         reqs = []
         if t < world - 1:  # pass the shard in hand on while computing with it
             rk, rv = bufs[t % 2]
-            ops = [dist.P2POp(dist.isend, cur_k, nxt, group), dist.P2POp(dist.isend, cur_v, nxt, group),
-                   dist.P2POp(dist.irecv, rk, prv, group), dist.P2POp(dist.irecv, rv, prv, group)]
-            reqs = dist.batch_isend_irecv(ops)
+            reqs = _exchange([cur_k, cur_v], [rk, rv], nxt, prv, group)
         ra.consume(t, cur_k, cur_v)
         for r in reqs:
             r.wait()
@@ -294,19 +329,13 @@ def ring_attention_backward(q, k, v, o, lse, do, causal: bool = False, scale: Op
         kv_reqs = []
         if t < world - 1:  # the next shard's K and V stream in while this block computes
             rk, rv = kv_bufs[t % 2]
-            kv_reqs = dist.batch_isend_irecv([dist.P2POp(dist.isend, cur_k, nxt, group),
-                                              dist.P2POp(dist.isend, cur_v, nxt, group),
-                                              dist.P2POp(dist.irecv, rk, prv, group),
-                                              dist.P2POp(dist.irecv, rv, prv, group)])
+            kv_reqs = _exchange([cur_k, cur_v], [rk, rv], nxt, prv, group)
         for r in acc_reqs:  # this shard's accumulators have arrived
             r.wait()
         rb.consume(t, cur_k, cur_v, *cur_acc)
         # the accumulators move on once this rank has added to them (after the last step: home)
         nxt_acc = acc_bufs[t % 2]
-        acc_reqs = dist.batch_isend_irecv([dist.P2POp(dist.isend, cur_acc[0], nxt, group),
-                                           dist.P2POp(dist.isend, cur_acc[1], nxt, group),
-                                           dist.P2POp(dist.irecv, nxt_acc[0], prv, group),
-                                           dist.P2POp(dist.irecv, nxt_acc[1], prv, group)])
+        acc_reqs = _exchange([cur_acc[0], cur_acc[1]], [nxt_acc[0], nxt_acc[1]], nxt, prv, group)
         for r in kv_reqs:
             r.wait()
         if t < world - 1:
