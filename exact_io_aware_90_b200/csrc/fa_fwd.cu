@@ -662,7 +662,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             }
             c2 = make_float2(c * kd, c * kd);
             lv = __log2f(vd);
-            inv_vd = 1.f / vd;
+            inv_vd = ex2(-lv);  // 1 / v_descale as P sees it (2^lv), one MUFU operation
           }
         }
         if (!warp_wait(bar(C::B_SFULL + t), step & 1, wd)) { ok = false; break; }
