@@ -61,7 +61,7 @@ def load_peaks():
 # The source files each profiled kernel is built from: its own file and the two shared headers.
 KERNEL_SOURCES = {
     "fa_fwd_kernel": ["fa_fwd.cu", "sm100.cuh", "fa_internal.h"],
-    "fa_bwd_main_kernel": ["fa_bwd.cu", "sm100.cuh", "fa_internal.h"],
+    "fa_bwd_main_q128_kernel": ["fa_bwd.cu", "sm100.cuh", "fa_internal.h"],
     "fa_bwd_dropout": ["fa_bwd.cu", "sm100.cuh", "fa_internal.h"],
     "fa_decode_split_kernel": ["fa_decode.cu", "sm100.cuh", "fa_internal.h"],
     "fa_merge_kernel": ["fa_merge.cu", "sm100.cuh", "fa_internal.h"],
@@ -310,10 +310,10 @@ def run_gpu(args, world, rank, local, pg):
     else:
         stages = [("fa_fwd_kernel", fwd)]
         if backward:
-            stages += [("fa_bwd_pre_kernel", bwd_pre), ("fa_bwd_main_kernel", bwd_main),
+            stages += [("fa_bwd_pre_kernel", bwd_pre), ("fa_bwd_main_q128_kernel", bwd_main),
                        ("fa_bwd_post_kernel", bwd_post)]
         launches = {name: 1 for name, _ in stages}
-        flops_of = {"fa_fwd_kernel": flops_fwd, "fa_bwd_main_kernel": flops_bwd}
+        flops_of = {"fa_fwd_kernel": flops_fwd, "fa_bwd_main_q128_kernel": flops_bwd}
     drop_kw = dict(dropout_p=drop_p, seed=drop_seed, offset=drop_off) if drop_p > 0.0 else {}
 
     def one_step(record):
