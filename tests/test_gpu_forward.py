@@ -256,3 +256,28 @@ def test_concurrent_launches_on_two_streams(fa):
         assert all(torch.equal(x, y) for x, y in zip(got_b, ref_b))
     O_ref, L_ref = oracle_forward(b)
     assert max_abs(f64(ref_b[0]), O_ref) <= O_TOL and max_abs(f64(ref_b[1]), L_ref) <= LSE_TOL
+
+
+def test_repeated_calls_on_other_tensors_and_shapes(fa):
+    """The library keeps the encoded tensor maps of recent calls, keyed by address and sizes: calls that
+    alternate between two sets of tensors of one shape, reuse one allocation for a shorter sequence, and
+    come back to the first set each match the oracle for their own inputs."""
+    dev = torch.device("cuda")
+    a = workloads.random_inputs(2, 128, "bf16", seed=31, B=1, N=384, causal=True, backward=False)
+    b = workloads.random_inputs(2, 128, "bf16", seed=32, B=1, N=384, causal=True, backward=False)
+    ta = [t.to(dev) for t in (a.q, a.k, a.v)]
+    tb = [t.to(dev) for t in (b.q, b.k, b.v)]
+    refs = {id(a): oracle_forward(a), id(b): oracle_forward(b)}
+    for inp, ts in ((a, ta), (b, tb), (a, ta), (b, tb)):
+        o, lse = fa.attention_forward(*ts, causal=True, scale=inp.scale, batch=1)
+        assert fa.fa_check_device_status(torch.cuda.current_stream().cuda_stream) == fa.FA_OK
+        O_ref, L_ref = refs[id(inp)]
+        assert max_abs(f64(o), O_ref) <= O_TOL and max_abs(f64(lse), L_ref) <= LSE_TOL
+    # the same storage viewed as a shorter sequence: a different key (T), so a map of its own
+    short = workloads.random_inputs(2, 128, "bf16", seed=33, B=1, N=200, causal=True, backward=False)
+    for t, src in zip(ta, (short.q, short.k, short.v)):
+        t[:200].copy_(src.to(dev))
+    o, lse = fa.attention_forward(*(t[:200] for t in ta), causal=True, scale=short.scale, batch=1)
+    assert fa.fa_check_device_status(torch.cuda.current_stream().cuda_stream) == fa.FA_OK
+    O_ref, L_ref = oracle_forward(short)
+    assert max_abs(f64(o), O_ref) <= O_TOL and max_abs(f64(lse), L_ref) <= LSE_TOL
