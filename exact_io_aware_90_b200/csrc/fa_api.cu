@@ -3,7 +3,6 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
-#include <mutex>
 
 #include "../../include/fa.h"
 #include "fa_internal.h"
@@ -31,54 +30,7 @@ static EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// Encoded tensor maps of recent calls.  A map depends only on what its key holds (address, sizes,
-// element kind, box rows; the swizzle and the rest are fixed per kind), so a call on the same tensors as
-// an earlier one copies the 128-byte map instead of encoding it again (an encode costs about a
-// microsecond on the host, a visible part of a short call).  A small table with round-robin
-// replacement, under a mutex.
-namespace {
-struct TmapKey {
-  const void* base;
-  int T, H, d, rows, kind;  // kind: 0 fp16, 1 bf16, 2 e4m3, 3 fp32
-  bool operator==(const TmapKey& o) const {
-    return base == o.base && T == o.T && H == o.H && d == o.d && rows == o.rows && kind == o.kind;
-  }
-};
-struct TmapCache {
-  static constexpr int kEntries = 32;
-  std::mutex mu;
-  TmapKey keys[kEntries];
-  CUtensorMap maps[kEntries];
-  int used = 0, next = 0;
-};
-TmapCache& tmap_cache() {
-  static TmapCache c;
-  return c;
-}
-bool tmap_lookup(const TmapKey& k, CUtensorMap* map) {
-  TmapCache& c = tmap_cache();
-  std::lock_guard<std::mutex> lock(c.mu);
-  for (int i = 0; i < c.used; ++i)
-    if (c.keys[i] == k) {
-      std::memcpy(map, &c.maps[i], sizeof(CUtensorMap));
-      return true;
-    }
-  return false;
-}
-void tmap_store(const TmapKey& k, const CUtensorMap* map) {
-  TmapCache& c = tmap_cache();
-  std::lock_guard<std::mutex> lock(c.mu);
-  const int i = c.next;
-  c.keys[i] = k;
-  std::memcpy(&c.maps[i], map, sizeof(CUtensorMap));
-  c.next = (i + 1) % TmapCache::kEntries;
-  if (c.used < TmapCache::kEntries) ++c.used;
-}
-}  // namespace
-
 bool encode_tmap(CUtensorMap* map, const void* base, int T, int H, int d, bool bf16, int rows) {
-  const TmapKey key{base, T, H, d, rows, bf16 ? 1 : 0};
-  if (tmap_lookup(key, map)) return true;
   EncodeTiledFn fn = get_encode_fn();
   if (fn == nullptr) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T};
@@ -88,15 +40,11 @@ bool encode_tmap(CUtensorMap* map, const void* base, int T, int H, int d, bool b
   CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return false;
-  tmap_store(key, map);
-  return true;
+  return r == CUDA_SUCCESS;
 }
 
 // e4m3 [T, H, d] as bytes: one 128-byte box per row (d = 128), 128-byte swizzle.
 bool encode_tmap_e4m3(CUtensorMap* map, const void* base, int T, int H, int d, int rows) {
-  const TmapKey key{base, T, H, d, rows, 2};
-  if (tmap_lookup(key, map)) return true;
   EncodeTiledFn fn = get_encode_fn();
   if (fn == nullptr) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T};
@@ -106,14 +54,10 @@ bool encode_tmap_e4m3(CUtensorMap* map, const void* base, int T, int H, int d, i
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return false;
-  tmap_store(key, map);
-  return true;
+  return r == CUDA_SUCCESS;
 }
 
 bool encode_tmap_f32(CUtensorMap* map, const void* base, int T, int H, int d, int rows) {
-  const TmapKey key{base, T, H, d, rows, 3};
-  if (tmap_lookup(key, map)) return true;
   EncodeTiledFn fn = get_encode_fn();
   if (fn == nullptr) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T};
@@ -123,9 +67,7 @@ bool encode_tmap_f32(CUtensorMap* map, const void* base, int T, int H, int d, in
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return false;
-  tmap_store(key, map);
-  return true;
+  return r == CUDA_SUCCESS;
 }
 
 static bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }

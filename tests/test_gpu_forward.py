@@ -259,9 +259,9 @@ def test_concurrent_launches_on_two_streams(fa):
 
 
 def test_repeated_calls_on_other_tensors_and_shapes(fa):
-    """The library keeps the encoded tensor maps of recent calls, keyed by address and sizes: calls that
-    alternate between two sets of tensors of one shape, reuse one allocation for a shorter sequence, and
-    come back to the first set each match the oracle for their own inputs."""
+    """Calls that alternate between two sets of tensors of one shape, reuse one allocation for a shorter
+    sequence, and come back to the first set each match the oracle for their own inputs (nothing of an
+    earlier call's tensors carries over into a later call)."""
     dev = torch.device("cuda")
     a = workloads.random_inputs(2, 128, "bf16", seed=31, B=1, N=384, causal=True, backward=False)
     b = workloads.random_inputs(2, 128, "bf16", seed=32, B=1, N=384, causal=True, backward=False)
