@@ -1114,7 +1114,8 @@ def config_summary(r):
 
 
 def run_configs(args, world, rank, local, pg, headline):
-    """The other measured workloads (fp16 d = 64, varlen, 128k, the tiny call) and the dropout step, measured after the headline."""
+    """The other measured workloads (fp16 d = 64, varlen, 128k, the tiny call) and the dropout step,
+    measured after the headline."""
     import copy
     out = {}
     for name in CONFIG_WORKLOADS + ["causal_n8k_d128+dropout0.1"]:
