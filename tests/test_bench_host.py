@@ -107,3 +107,18 @@ def test_bench_rejects_dropout_where_it_does_not_apply(extra):
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference"] + extra,
                        capture_output=True, text=True, timeout=120)
     assert r.returncode == 2 and "--dropout" in r.stderr and r.stdout.strip() == ""
+
+
+@pytest.mark.parametrize("name", ["tiny_d64", "mha_n4k_d64", "causal_n8k_d128+dropout0.1"])
+def test_config_cpu_baseline(name):
+    """The oracle baseline of an extra workload: a bounded sample (a fraction of a second of oracle work
+    here), reported with its sample, the cores and BLAS threads, and a positive throughput."""
+    sys.path.insert(0, ROOT)
+    import bench
+    r = bench.config_cpu_baseline(name, budget_s=0.4)
+    assert r["kind"] == "oracle" and r["unit"] == "TFLOP/s" and r["value"] > 0
+    assert r["cores"] >= 1 and r["cores_available"] >= 1 and "sample" in r
+    if "+dropout" in name:
+        assert "dropout oracle" in r["sample"]
+    else:
+        assert "query rows" in r["sample"]
